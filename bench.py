@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the W4 path on B200: prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (``value``): W4A16 GEMV HBM GB/s at M=1 over the 8B decode sweep -- one step is
+one M=1 GEMV through each of the four (K, N) shapes {(4096,4096), (4096,1024),
+(4096,14336), (14336,4096)} (asymmetric INT4, group 128, weights quantized with the
+20-ratio clip search), i.e. 73.6 MB of algorithmic bytes. The weights rotate over R
+prepacked copies whose total size is at least 3x the 126 MB L2, so no step reads weights
+from L2. Every other row of the path is measured in ``rows`` with its own roofline: the W4A8
+prefill GEMM (M=4096, both shapes), the FP8 row quant, the quantizer on the full 8B weight
+set (6.98e9 weights, 20 ratios), the MoE grouped GEMM and the GEMV at M=4 and 16.
+
+Multi-GPU: every rank runs the same per-GPU work on its own weights (weak scaling, no
+collective on the data path); timings are CUDA events, max over ranks.
+``--impl reference`` times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "W4A16 GEMV HBM GB/s (M=1) & W4A8 GEMM TFLOP/s; % of B200 roofline"
+DECODE_SHAPES = [(4096, 4096), (4096, 1024), (4096, 14336), (14336, 4096)]  # (K, N)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained"),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def gemv_bytes(M, N, K, g=128):
+    """Algorithmic bytes of one W4A16 GEMV: packed codes, 2+2 bytes of scale and zero per
+    group, the bf16 activations and the bf16 output."""
+    return N * K // 2 + N * (K // g) * 4 + 2 * M * K + 2 * M * N
+
+
+# ------------------------------------------------------------------ clocks
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, maxmhz, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                maxmhz = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(mhz)) if mhz else None, "sm_max_mhz": maxmhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------ timing helpers
+
+def time_region(fn, iters, stream=None):
+    """Device time (ms) of `iters` calls of fn, CUDA events on the launching stream."""
+    stream = stream or torch.cuda.current_stream()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for i in range(iters):
+        fn(i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e)
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+# ------------------------------------------------------------------ our arm
+
+class Decode:
+    """The decode sweep: quantize (GPU), prepack R copies per shape, M=1 activations."""
+
+    def __init__(self, M, seed, dev, copies=None):
+        from bit_gemm_wise_b200 import synth, w4
+        self.w4 = w4
+        self.M = M
+        g = 128
+        grid = synth.clip_grid_20()
+        self.shapes = DECODE_SHAPES
+        self.bytes_per_step = sum(gemv_bytes(M, N, K) for K, N in self.shapes)
+        packed_per_step = sum(w4.w4_prepack_bytes(N, K, g, w4.W4_LAYOUT_GEMV) for K, N in self.shapes)
+        self.R = copies or max(2, -(-3 * L2_BYTES // packed_per_step))
+        self.packed, self.x, self.y = [], [], []
+        for K, N in self.shapes:
+            W = synth.decode_weight(K, N, seed, device=dev)
+            codes, scales, zeros, _ = w4.alloc_quantized(N, K, g, "asym", device=dev, chosen=False)
+            w4.w4_quantize(W, N, K, g, "asym", grid, codes, scales, zeros, None)
+            nb = w4.w4_prepack_bytes(N, K, g, w4.W4_LAYOUT_GEMV)
+            p = torch.empty(self.R * nb, dtype=torch.uint8, device=dev)
+            w4.w4_prepack(codes, scales, zeros, N, K, g, "asym", w4.W4_LAYOUT_GEMV, p[:nb])
+            for r in range(1, self.R):
+                p[r * nb:(r + 1) * nb].copy_(p[:nb])
+            self.packed.append((p, nb))
+            self.x.append(synth.decode_activation(M, K, seed, device=dev))
+            self.y.append(torch.empty(M, N, dtype=torch.bfloat16, device=dev))
+            del W, codes, scales, zeros
+        self.launches_per_step = len(self.shapes)
+
+    def step(self, i):
+        for (K, N), (p, nb), x, y in zip(self.shapes, self.packed, self.x, self.y):
+            self.w4.w4a16_gemv(x, self.M, p[(i % self.R) * nb:], N, K, 128, "asym", y, 0)
+
+
+def run_ours(args, rank, world, dev):
+    from bit_gemm_wise_b200 import synth, w4
+    pk = peaks()
+    dist = world > 1
+    stream = torch.cuda.current_stream()
+
+    dec = Decode(1, args.seed, dev)
+    for i in range(args.warmup):
+        dec.step(i)
+    torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with Clocks(torch.cuda.current_device()) as clk:
+        ms = time_region(dec.step, args.steps, stream)
+    if dist:
+        torch.distributed.barrier()
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * dec.bytes_per_step / (ms_step * 1e-3) / 1e9
+
+    # per-shape launch times (events around blocks of launches of one shape)
+    per_shape = {}
+    for si, (K, N) in enumerate(dec.shapes):
+        p, nb = dec.packed[si]
+        n_it = max(8, args.steps)
+
+        def one(i, si=si, K=K, N=N, p=p, nb=nb):
+            w4.w4a16_gemv(dec.x[si], 1, p[(i % dec.R) * nb:], N, K, 128, "asym", dec.y[si], 0)
+
+        one(0)
+        t_ms = time_region(one, n_it, stream) / n_it
+        per_shape[f"{K}x{N}"] = {"us": round(t_ms * 1e3, 3),
+                                 "GBps": round(gemv_bytes(1, N, K) / (t_ms * 1e-3) / 1e9, 1)}
+
+    # e2e through the public API with host buffers: h2d x, GEMVs, d2h y per step
+    xh = [x.cpu().pin_memory() for x in dec.x]
+    yh = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in dec.y]
+    h2d = sum(x.numel() * 2 for x in xh)
+    d2h = sum(y.numel() * 2 for y in yh)
+
+    def e2e_step(i):
+        for si, (K, N) in enumerate(dec.shapes):
+            dec.x[si].copy_(xh[si], non_blocking=True)
+        dec.step(i)
+        for si in range(len(dec.shapes)):
+            yh[si].copy_(dec.y[si], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    e2e_ms = time_region(e2e_step, args.steps, stream) / args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = world * dec.bytes_per_step / (e2e_ms * 1e-3) / 1e9
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 x int4 -> fp32 accumulate", "data": "synthetic (seeded; no checkpoint or dataset)",
+        "config": {"workload": "decode GEMV sweep (K,N) in {(4096,4096),(4096,1024),(4096,14336),(14336,4096)}, "
+                               "M=1, INT4 asym group 128, 20-ratio MSE clip",
+                   "bytes_per_step": dec.bytes_per_step, "weight_copies": dec.R,
+                   "l2": f"inputs larger than L2: weights rotate over {dec.R} copies "
+                         f"({dec.R * sum(nb for _, nb in dec.packed) / 1e6:.0f} MB > 3 x L2)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": round(value / world / pk["hbm"], 4), "traffic": None,
+                     "peak_source": f"{pk['src']} copy bandwidth"},
+        "per_shape": per_shape,
+        "gpu_launches": dec.launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+    }
+    if not args.headline_only:
+        out["rows"] = measure_rows(args, dev, pk)
+    del dec
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu:
+        out["cpu_baseline"] = cpu_baseline(args.seed, budget_s=args.cpu_seconds)
+    return out
+
+
+def measure_rows(args, dev, pk):
+    """Every other row of the path, each timed with CUDA events (after warm-up)."""
+    from bit_gemm_wise_b200 import synth, w4
+    rows = {}
+    fp8_peak = 2.0 * pk["bf16"]  # dense FP8 = 2x dense BF16 (nominal ratio), burst
+
+    # GEMV at M = 4 and 16 (ALU-bound on the CUDA cores)
+    for M in (4, 16):
+        d = Decode(M, args.seed, dev)
+        d.step(0)
+        ms = time_region(d.step, 20) / 20
+        rows[f"w4a16_gemv_M{M}"] = {"value": round(d.bytes_per_step / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                                    "us_per_step": round(ms * 1e3, 2),
+                                    "frac_hbm": round(d.bytes_per_step / (ms * 1e-3) / 1e9 / pk["hbm"], 4)}
+        del d
+
+    # W4A8 prefill GEMM (M=4096) and the FP8 row quant feeding it
+    for K, N in synth.PREFILL_SHAPES:
+        M = synth.PREFILL_M
+        W = synth.prefill_weight(K, N, args.seed, device=dev)
+        codes, scales, zeros, _ = w4.alloc_quantized(N, K, 128, "asym", device=dev, chosen=False)
+        w4.w4_quantize(W, N, K, 128, "asym", [1.0], codes, scales, zeros, None)
+        packed = w4.alloc_packed(N, K, 128, w4.W4_LAYOUT_GEMM, device=dev)
+        w4.w4_prepack(codes, scales, zeros, N, K, 128, "asym", w4.W4_LAYOUT_GEMM, packed)
+        X = synth.prefill_activation(M, K, args.seed, device=dev)
+        X8 = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        sa = torch.empty(M, dtype=torch.float32, device=dev)
+        G = torch.empty(M, K // 128, dtype=torch.float32, device=dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+        def rq(i):
+            w4.fp8_row_quant(X, M, K, 128, X8, sa, G)
+
+        def gemm(i):
+            w4.w4a8_gemm(X8, sa, G, M, packed, N, K, 128, "asym", Y, 0)
+
+        rq(0); gemm(0)
+        n = 10
+        t_rq = t_gemm = 0.0
+        for i in range(n):
+            flush_l2(flush)
+            t_rq += time_region(rq, 1)
+            flush_l2(flush)
+            t_gemm += time_region(gemm, 1)
+        t_rq /= n
+        t_gemm /= n
+        flops = 2.0 * M * N * K
+        tf = flops / (t_gemm * 1e-3) / 1e12
+        rq_bytes = M * K * 2 + M * K + M * 4 + M * (K // 128) * 4
+        rows[f"w4a8_gemm_{K}x{N}"] = {
+            "value": round(tf, 1), "unit": "TFLOP/s", "us": round(t_gemm * 1e3, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp8_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4),
+                         "peak_source": f"{pk['src']} bf16 burst x 2 (dense FP8/BF16 nominal ratio)"}}
+        rows[f"fp8_row_quant_{M}x{K}"] = {
+            "value": round(rq_bytes / (t_rq * 1e-3) / 1e9, 1), "unit": "GB/s", "us": round(t_rq * 1e3, 1),
+            "frac_hbm": round(rq_bytes / (t_rq * 1e-3) / 1e9 / pk["hbm"], 4)}
+        rows[f"w4a8_rowquant_plus_gemm_{K}x{N}"] = {
+            "value": round(flops / ((t_gemm + t_rq) * 1e-3) / 1e12, 1), "unit": "TFLOP/s"}
+        del W, codes, scales, zeros, packed, X, X8, sa, G, Y, flush
+        torch.cuda.empty_cache()
+
+    # MoE grouped GEMM (32 experts, top-4 of 4096 tokens, group 32)
+    c = synth.MOE
+    r = synth.moe_routing(args.seed)
+    off = r.expert_row_offsets.to(dev)
+    Mt = int(r.expert_row_offsets[-1])
+    Xm = synth.moe_activation(args.seed, device=dev)[r.token_of_row.to(dev)].contiguous()
+    X8 = torch.empty(Mt, c["K"], dtype=torch.uint8, device=dev)
+    sa = torch.empty(Mt, dtype=torch.float32, device=dev)
+    G = torch.empty(Mt, c["K"] // 32, dtype=torch.float32, device=dev)
+    w4.fp8_row_quant(Xm, Mt, c["K"], 32, X8, sa, G)
+    for kind in ("gate_up", "down"):
+        N = c["N_gate_up"] if kind == "gate_up" else c["N_down"]
+        K = c["K"]
+        nb = w4.w4_prepack_bytes(N, K, 32, w4.W4_LAYOUT_GEMM)
+        packed = torch.empty(c["E"] * nb, dtype=torch.uint8, device=dev)
+        for e in range(c["E"]):
+            W = synth.moe_weight(kind, e, args.seed, device=dev)
+            codes, scales, zeros, _ = w4.alloc_quantized(N, K, 32, "asym", device=dev, chosen=False)
+            w4.w4_quantize(W, N, K, 32, "asym", [1.0], codes, scales, zeros, None)
+            w4.w4_prepack(codes, scales, zeros, N, K, 32, "asym", w4.W4_LAYOUT_GEMM, packed[e * nb:])
+        Y = torch.empty(Mt, N, dtype=torch.bfloat16, device=dev)
+
+        def mg(i):
+            w4.w4a8_grouped_gemm(X8, sa, G, off, c["E"], Mt, packed, N, K, 32, "asym", Y)
+
+        mg(0)
+        ms = time_region(mg, 5) / 5
+        flops = 2.0 * Mt * N * K
+        tf = flops / (ms * 1e-3) / 1e12
+        rows[f"w4a8_grouped_{kind}"] = {
+            "value": round(tf, 1), "unit": "TFLOP/s", "us": round(ms * 1e3, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp8_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4)}}
+        del packed, Y
+    del Xm, X8, sa, G
+    torch.cuda.empty_cache()
+
+    # quantizer throughput on the full 8B weight set (20 ratios, asym g128)
+    rows["w4_quantize_8b_set"] = quantizer_full_set(args, dev)
+    return rows
+
+
+def quantizer_full_set(args, dev):
+    from bit_gemm_wise_b200 import synth, w4
+    grid = synth.clip_grid_20()
+    layer = synth.LLAMA8B_LAYER
+    n_layers = args.quant_layers
+    mats = []
+    for L in range(n_layers):
+        for name, N, K in layer:
+            W = synth.llama8b_weight(L, name, args.seed, device=dev)
+            out = w4.alloc_quantized(N, K, 128, "asym", device=dev, chosen=False)
+            mats.append((W, N, K, out))
+    weights = sum(N * K for _, N, K, _ in mats)
+
+    def q(i):
+        for W, N, K, (codes, scales, zeros, _) in mats:
+            w4.w4_quantize(W, N, K, 128, "asym", grid, codes, scales, zeros, None)
+
+    q(0)
+    ms = time_region(q, 1)
+    res = {"value": round(weights / (ms * 1e-3) / 1e9, 2), "unit": "G weights/s",
+           "input_GBps": round(2 * weights / (ms * 1e-3) / 1e9, 1), "ms": round(ms, 2),
+           "weights": weights, "layers": n_layers, "bound": "alu"}
+    del mats
+    torch.cuda.empty_cache()
+    return res
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_decode_inputs(seed):
+    """Synthetic quantized decode weights for timing the oracle GEMV (values do not affect
+    its speed): random codes, fp16 scales, zeros in 0..15, and bf16 activations."""
+    import oracle  # noqa: F401
+    from bit_gemm_wise_b200 import synth
+    rng = np.random.default_rng(seed)
+    items = []
+    for K, N in DECODE_SHAPES:
+        codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+        scales = np.full((N, K // 128), 0x2100, np.uint16)
+        zeros = rng.integers(0, 16, (N, K // 128)).astype(np.int16)
+        x = synth.bf16_bits(synth.decode_activation(1, K, seed))
+        items.append((K, N, codes, scales, zeros, x))
+    return items
+
+
+def cpu_baseline(seed, budget_s=12.0):
+    import oracle
+    items = oracle_decode_inputs(seed)
+    oracle.gemv_ref(items[1][5], *items[1][2:5], 128, "asym")  # warm (build, page-in)
+    t0 = time.perf_counter()
+    nbytes = 0
+    steps = 0
+    while True:
+        for K, N, codes, scales, zeros, x in items:
+            oracle.gemv_ref(x, codes, scales, zeros, 128, "asym")
+            nbytes += gemv_bytes(1, N, K)
+        steps += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"{steps} full decode steps (4 M=1 GEMVs, fp64 scalar C, OpenMP over rows)",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    import oracle
+    items = oracle_decode_inputs(args.seed)
+    oracle.gemv_ref(items[1][5], *items[1][2:5], 128, "asym")
+    step_bytes = sum(gemv_bytes(1, N, K) for K, N in DECODE_SHAPES)
+    # a bounded sample per step: the first shape set that fits ~2 s
+    def step():
+        for K, N, codes, scales, zeros, x in items:
+            oracle.gemv_ref(x, codes, scales, zeros, 128, "asym")
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    val = step_bytes * args.steps / dt / 1e9
+    cores = os.cpu_count()
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "decode GEMV sweep, M=1 (CPU oracle)"},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": "full decode steps (4 M=1 GEMVs), fp64 scalar C, OpenMP over rows"},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--quant-layers", type=int, default=32)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        from bit_gemm_wise_b200 import w4
+        w4.lib()
+        out = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,125 @@
+// w4_prepack: canonical quantized weight -> kernel layout (lossless move of codes,
+// scales and zeros; see w4_layout.cuh). One thread per output 32-bit word.
+#include "w4_common.cuh"
+#include "w4_layout.cuh"
+
+namespace w4 {
+
+__device__ __forceinline__ uint32_t nib_at(const uint8_t *codes, int64_t N, int64_t K, int64_t n, int64_t k) {
+    if (n >= N || k >= K) return 0;
+    const uint8_t b = codes[n * (K / 2) + (k >> 1)];
+    return (k & 1) ? (b >> 4) : (b & 0xF);
+}
+
+__device__ __forceinline__ uint32_t scale_entry(const uint16_t *scales, const int16_t *zeros, int64_t N, int64_t J,
+                                                int64_t n, int64_t j) {
+    if (n >= N || j >= J) return 0;
+    const uint32_t s = scales[n * J + j];
+    const uint32_t z = zeros ? (uint16_t)zeros[n * J + j] : 8u;
+    return s | (z << 16);
+}
+
+__global__ void prepack_gemv_codes(const uint8_t *__restrict__ codes, int64_t N, int64_t K, int64_t U,
+                                   int64_t nwords, uint32_t *__restrict__ out) {
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nwords;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int w = idx & 3;
+        const int t = (idx >> 2) & 31;
+        const int64_t u = (idx >> 7) % U;
+        const int64_t o = (idx >> 7) / U;
+        const int64_t n = o * 8 + (t >> 2);
+        const int64_t k0 = u * 128 + (t & 3) * 32 + w * 8;
+        uint32_t word = 0;
+        for (int i = 0; i < 4; ++i) {
+            word |= nib_at(codes, N, K, n, k0 + 2 * i) << (4 * i);
+            word |= nib_at(codes, N, K, n, k0 + 2 * i + 1) << (16 + 4 * i);
+        }
+        out[idx] = word;
+    }
+}
+
+__global__ void prepack_gemv_scales(const uint16_t *__restrict__ scales, const int16_t *__restrict__ zeros,
+                                    int64_t N, int64_t K, int g, int64_t U, int64_t nent,
+                                    uint32_t *__restrict__ out) {
+    const int per_unit = 128 / g;
+    const int64_t J = K / g;
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nent;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int gg = idx % per_unit;
+        const int r = (idx / per_unit) % 8;
+        const int64_t u = (idx / per_unit / 8) % U;
+        const int64_t o = idx / per_unit / 8 / U;
+        out[idx] = scale_entry(scales, zeros, N, J, o * 8 + r, u * per_unit + gg);
+    }
+}
+
+__global__ void prepack_gemm_codes(const uint8_t *__restrict__ codes, int64_t N, int64_t K, int64_t Kpad,
+                                   int64_t nwords, uint32_t *__restrict__ out) {
+    const int64_t wpr = Kpad / 8;  // words per row
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nwords;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = idx / wpr;
+        const int64_t k0 = (idx % wpr) * 8;
+        uint32_t word = 0;
+        for (int p = 0; p < 8; ++p) word |= nib_at(codes, N, K, n, k0 + p / 2 + 4 * (p % 2)) << (4 * p);
+        out[idx] = word;
+    }
+}
+
+__global__ void prepack_gemm_scales(const uint16_t *__restrict__ scales, const int16_t *__restrict__ zeros,
+                                    int64_t N, int64_t K, int g, int64_t Npad, int64_t nent,
+                                    uint32_t *__restrict__ out) {
+    const int64_t J = K / g;
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nent;
+         idx += (int64_t)gridDim.x * blockDim.x)
+        out[idx] = scale_entry(scales, zeros, N, J, idx % Npad, idx / Npad);
+}
+
+static int grid_for(int64_t n) {
+    const int64_t b = (n + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 32;
+    return (int)(b < cap ? (b > 0 ? b : 1) : cap);
+}
+
+}  // namespace w4
+
+using namespace w4;
+
+W4_API size_t w4_prepack_bytes(int64_t N, int64_t K, int group, int layout) {
+    if (N < 1 || K < 32 || K % 32 != 0 || !valid_group(group) || K % group != 0) return 0;
+    if (layout == W4_LAYOUT_GEMV) return gemv_layout(N, K, group).total;
+    if (layout == W4_LAYOUT_GEMM) return gemm_layout(N, K, group).total;
+    return 0;
+}
+
+W4_API w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, const int16_t *zeros, int64_t N,
+                            int64_t K, int group, int mode, int layout, void *packed, cudaStream_t stream) {
+    if (!codes || !scales_fp16 || !packed) return W4_ERR_NULL;
+    if (!valid_mode(mode)) return W4_ERR_ARG;
+    if (mode == W4_ASYM && !zeros) return W4_ERR_NULL;
+    if (mode == W4_SYM && zeros) return W4_ERR_ARG;
+    if (N < 1 || K < 32 || K % 32 != 0) return W4_ERR_SHAPE;
+    if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
+    if (layout != W4_LAYOUT_GEMV && layout != W4_LAYOUT_GEMM) return W4_ERR_ARG;
+    if (!aligned16(codes) || !aligned16(scales_fp16) || (zeros && !aligned16(zeros)) || !aligned16(packed))
+        return W4_ERR_ALIGN;
+    uint8_t *base = static_cast<uint8_t *>(packed);
+    if (layout == W4_LAYOUT_GEMV) {
+        const GemvLayout L = gemv_layout(N, K, group);
+        const int64_t nwords = (int64_t)(L.codes_bytes / 4);
+        const int64_t nent = (int64_t)(L.scales_bytes / 4);
+        prepack_gemv_codes<<<grid_for(nwords), 256, 0, stream>>>(codes, N, K, L.U, nwords,
+                                                                 reinterpret_cast<uint32_t *>(base));
+        prepack_gemv_scales<<<grid_for(nent), 256, 0, stream>>>(scales_fp16, zeros, N, K, group, L.U, nent,
+                                                                reinterpret_cast<uint32_t *>(base + L.codes_bytes));
+    } else {
+        const GemmLayout L = gemm_layout(N, K, group);
+        const int64_t nwords = (int64_t)(L.codes_bytes / 4);
+        const int64_t nent = (int64_t)(L.scales_bytes / 4);
+        prepack_gemm_codes<<<grid_for(nwords), 256, 0, stream>>>(codes, N, K, L.Kpad, nwords,
+                                                                 reinterpret_cast<uint32_t *>(base));
+        prepack_gemm_scales<<<grid_for(nent), 256, 0, stream>>>(scales_fp16, zeros, N, K, group, L.Npad, nent,
+                                                                reinterpret_cast<uint32_t *>(base + L.codes_bytes));
+    }
+    return launch_status();
+}

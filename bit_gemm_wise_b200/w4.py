@@ -1,0 +1,175 @@
+"""Thin ctypes binding of ``libw4.so`` (declared in ``include/w4.h``).
+
+Every function here has the name of the C entry point it calls and only marshals
+arguments: torch tensors become device pointers, the current torch CUDA stream becomes the
+``cudaStream_t``. All computation happens in the library's CUDA kernels. There is no CPU
+path: if the library is missing or a call returns an error, these functions raise.
+Tensors must be contiguous CUDA tensors that the caller allocated (helpers at the bottom
+allocate outputs of the right shape with torch).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+W4_OK = 0
+W4_SYM, W4_ASYM = 0, 1
+W4_LAYOUT_GEMV, W4_LAYOUT_GEMM = 0, 1
+
+STATUS = {
+    0: "W4_OK", 1: "W4_ERR_NULL", 2: "W4_ERR_SHAPE", 3: "W4_ERR_GROUP", 4: "W4_ERR_ALIGN",
+    5: "W4_ERR_ARG", 6: "W4_ERR_UNSUPPORTED", 7: "W4_ERR_CUDA", 8: "W4_ERR_TIMEOUT",
+    9: "W4_ERR_DEVICE_CHECK", 10: "W4_ERR_WORKSPACE",
+}
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4.so")
+
+# (name, restype, argtypes) of every exported entry point
+_P, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = [
+    ("w4_status_str", ctypes.c_char_p, [_I]),
+    ("w4_version", _I, []),
+    ("w4_quantize", _I, [_P, _I64, _I64, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
+    ("w4_prepack_bytes", _SZ, [_I64, _I64, _I, _I]),
+    ("w4_prepack", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P]),
+    ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P]),
+    ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
+    ("w4a8_gemm", _I, [_P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
+    ("w4a8_grouped_gemm", _I, [_P, _P, _P, _P, _I, _I64, _P, _I64, _I64, _I, _I, _P, _P]),
+    ("w4_device_status", _I, [_P, ctypes.POINTER(ctypes.c_int)]),
+]
+
+_lib = None
+
+
+class W4Error(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m bit_gemm_wise_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, rc: int):
+    if rc != W4_OK:
+        raise W4Error(fn, rc)
+
+
+def _mode(mode) -> int:
+    if mode in ("sym", W4_SYM):
+        return W4_SYM
+    if mode in ("asym", W4_ASYM):
+        return W4_ASYM
+    return int(mode)
+
+
+# ------------------------------------------------------------------ entry points
+
+def w4_status_str(code: int) -> str:
+    return lib().w4_status_str(code).decode()
+
+
+def w4_version() -> int:
+    return lib().w4_version()
+
+
+def w4_quantize(W, N, K, group, mode, clip_grid, codes, scales, zeros=None, chosen=None, stream=None):
+    grid = (ctypes.c_float * len(clip_grid))(*[float(r) for r in clip_grid])
+    rc = lib().w4_quantize(_ptr(W), N, K, group, _mode(mode), ctypes.cast(grid, _P), len(clip_grid),
+                           _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(chosen), _stream(stream))
+    _check("w4_quantize", rc)
+
+
+def w4_prepack_bytes(N, K, group, layout) -> int:
+    return int(lib().w4_prepack_bytes(N, K, group, layout))
+
+
+def w4_prepack(codes, scales, zeros, N, K, group, mode, layout, packed, stream=None):
+    rc = lib().w4_prepack(_ptr(codes), _ptr(scales), _ptr(zeros), N, K, group, _mode(mode), layout,
+                          _ptr(packed), _stream(stream))
+    _check("w4_prepack", rc)
+
+
+def fp8_row_quant(X, M, K, group, X8, row_scale, group_sums=None, stream=None):
+    rc = lib().fp8_row_quant(_ptr(X), M, K, group, _ptr(X8), _ptr(row_scale), _ptr(group_sums),
+                             _stream(stream))
+    _check("fp8_row_quant", rc)
+
+
+def w4a16_gemv(x, M, packed, N, K, group, mode, y, out_fp32=0, stream=None):
+    rc = lib().w4a16_gemv(_ptr(x), M, _ptr(packed), N, K, group, _mode(mode), _ptr(y), int(out_fp32),
+                          _stream(stream))
+    _check("w4a16_gemv", rc)
+
+
+def w4a8_gemm(X8, row_scale, group_sums, M, packed, N, K, group, mode, Y, out_fp32=0, stream=None):
+    rc = lib().w4a8_gemm(_ptr(X8), _ptr(row_scale), _ptr(group_sums), M, _ptr(packed), N, K, group,
+                         _mode(mode), _ptr(Y), int(out_fp32), _stream(stream))
+    _check("w4a8_gemm", rc)
+
+
+def w4a8_grouped_gemm(X8, row_scale, group_sums, expert_row_offsets, E, M_total, packed, N, K, group,
+                      mode, Y, stream=None):
+    rc = lib().w4a8_grouped_gemm(_ptr(X8), _ptr(row_scale), _ptr(group_sums), _ptr(expert_row_offsets), E,
+                                 M_total, _ptr(packed), N, K, group, _mode(mode), _ptr(Y), _stream(stream))
+    _check("w4a8_grouped_gemm", rc)
+
+
+def w4_device_status(stream=None) -> int:
+    code = ctypes.c_int(-1)
+    rc = lib().w4_device_status(_stream(stream), ctypes.byref(code))
+    _check("w4_device_status", rc)
+    return code.value
+
+
+# ------------------------------------------------------------------ allocation helpers
+
+def alloc_quantized(N, K, group, mode, device="cuda", chosen=True):
+    """Empty canonical outputs of w4_quantize: codes u8 [N,K/2], scales fp16 bits [N,K/g],
+    zeros int16 [N,K/g] (asym only), chosen u8 [N,K/g] (optional)."""
+    J = K // group
+    codes = torch.empty(N, K // 2, dtype=torch.uint8, device=device)
+    scales = torch.empty(N, J, dtype=torch.int16, device=device)
+    zeros = torch.empty(N, J, dtype=torch.int16, device=device) if _mode(mode) == W4_ASYM else None
+    ch = torch.empty(N, J, dtype=torch.uint8, device=device) if chosen else None
+    return codes, scales, zeros, ch
+
+
+def alloc_packed(N, K, group, layout, device="cuda", copies: int = 1):
+    nbytes = w4_prepack_bytes(N, K, group, layout)
+    if nbytes == 0:
+        raise W4Error("w4_prepack_bytes", 2)
+    return torch.empty(copies * nbytes, dtype=torch.uint8, device=device)

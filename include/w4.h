@@ -1,0 +1,198 @@
+/*
+ * w4.h -- C ABI of libw4: blockwise 4-bit weight quantization and the matmuls that consume
+ * it, for NVIDIA B200 (sm_100a).
+ *
+ * Conventions for every entry point
+ *   - All tensors are dense, row-major and contiguous. Device pointers unless the name says
+ *     _host. Every device base pointer must be 16-byte aligned (W4_ERR_ALIGN otherwise).
+ *   - The caller allocates and owns every buffer. No entry point allocates, frees or
+ *     synchronizes device memory, except w4_device_status(), which synchronizes `stream`.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream) and
+ *     runs asynchronously. A return of W4_OK means the launch was enqueued.
+ *   - Arguments are validated on the host before anything is launched; on any error the
+ *     call returns a non-zero w4_status and has no side effect. There is no fallback: an
+ *     unsupported shape is an error, never a silently different computation.
+ *   - Device-side anomalies (a bounded wait that expired) are recorded in a device status
+ *     word that w4_device_status() reads; kernels never trap.
+ *
+ * Formats
+ *   bf16 inputs are raw 16-bit bfloat16 patterns; scales are IEEE binary16 patterns;
+ *   zeros are int16; FP8 values are E4M3 ("fn": no infinities, max 448) bytes.
+ *
+ * Canonical ("portable") quantized weight for W[N, K] and group g (the parity surface):
+ *   codes  uint8 [N, K/2]  byte j of row n = q[n, 2j] | q[n, 2j+1] << 4
+ *   scales uint16 [N, K/g] fp16 bits, one per group of g consecutive weights along K
+ *   zeros  int16 [N, K/g]  integer zero point (asymmetric only)
+ *   Symmetric codes are offset-binary: nibble = c + 8 with c in [-7, 7] (nibble 0 unused);
+ *   dequantized weight = (nibble - 8) * s. Asymmetric: (q - z) * s with q in [0, 15].
+ *
+ * Sources: "Quantizing LLMs Without Guesswork: What 4 Bits Really Cost" (QLWG) and
+ * "Four-bit inference ... Tahoma" (TAHOMA), sections named per entry point.
+ */
+#ifndef W4_H_
+#define W4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4_OK = 0,
+    W4_ERR_NULL = 1,         /* a required pointer is NULL                              */
+    W4_ERR_SHAPE = 2,        /* a size is out of the supported range                   */
+    W4_ERR_GROUP = 3,        /* group not in {32, 64, 128} or K not a multiple of it   */
+    W4_ERR_ALIGN = 4,        /* a device pointer is not 16-byte aligned                */
+    W4_ERR_ARG = 5,          /* any other bad argument (mode, clip grid, layout, ...)  */
+    W4_ERR_UNSUPPORTED = 6,  /* valid request this library does not implement          */
+    W4_ERR_CUDA = 7,         /* a CUDA runtime call failed (launch error)              */
+    W4_ERR_TIMEOUT = 8,      /* device status: a bounded wait in a kernel expired      */
+    W4_ERR_DEVICE_CHECK = 9, /* device status: a kernel's own consistency check failed */
+    W4_ERR_WORKSPACE = 10    /* workspace missing or smaller than the query says       */
+} w4_status;
+
+typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
+
+/* Kernel layouts produced by w4_prepack. */
+typedef enum { W4_LAYOUT_GEMV = 0, W4_LAYOUT_GEMM = 1 } w4_layout;
+
+/* Human-readable name of a status code (static storage). */
+const char *w4_status_str(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int w4_version(void);
+
+/*
+ * w4_quantize -- group-wise INT4 quantizer with the data-free MSE clip search.
+ *   QLWG "Scale and zero point" (symmetric max|x|/7; asymmetric (max-min)/15 with integer
+ *   zero round(-min/s)), "Granularity" (one FP16 scale per g consecutive weights of a row),
+ *   "Quantize, then dequantize" (zero-range guard s = 1, round half to even);
+ *   TAHOMA "The naive symmetric baseline", "Achievement 1: asymmetric W4", "MSE clipping"
+ *   (for each block: every ratio of the grid contracts the range about its midpoint, the
+ *   block is quantized and reconstructed, and a ratio replaces the incumbent only with a
+ *   strictly smaller block error that includes the clipped weights).
+ *
+ *   W_bf16         device, bf16 [N, K]
+ *   group          32, 64 or 128; K % group == 0; K % 32 == 0
+ *   mode           W4_SYM (amax/7, offset-binary codes) or W4_ASYM (scale + zero point)
+ *   clip_grid_host HOST, n_clip fp32 ratios in (0, 1], finite; clip_grid_host[0] == 1.0f
+ *                  (the incumbent is the full range); 1 <= n_clip <= 64. For W4_SYM the
+ *                  ratio scales max|w|; for W4_ASYM it contracts [min, max] about its
+ *                  midpoint.
+ *   codes          device, uint8 [N, K/2], canonical packing (see above)
+ *   scales_fp16    device, uint16 [N, K/group]
+ *   zeros          device, int16 [N, K/group]; required for W4_ASYM, must be NULL for W4_SYM
+ *   chosen_idx     device, uint8 [N, K/group], index of the winning ratio; may be NULL
+ *   Arithmetic: fp32, IEEE division, no FMA contraction, scale rounded to fp16 before the
+ *   codes, zero point and block error are formed; block error = sum of squares reduced in a
+ *   fixed tree (32 contiguous chunks of group/32 weights summed in order, then pairwise at
+ *   distances 16, 8, 4, 2, 1). Results are bit-identical run to run.
+ *   Errors: NULL / SHAPE (N < 1, K < 32) / GROUP / ALIGN / ARG (mode, grid, zeros vs mode).
+ */
+w4_status w4_quantize(const void *W_bf16, int64_t N, int64_t K, int group, int mode,
+                      const float *clip_grid_host, int n_clip, uint8_t *codes,
+                      uint16_t *scales_fp16, int16_t *zeros, uint8_t *chosen_idx,
+                      cudaStream_t stream);
+
+/*
+ * w4_prepack_bytes / w4_prepack -- lossless re-layout of a canonical quantized weight into a
+ *   kernel layout; no value is dequantized or requantized (TAHOMA "MSE clipping": portable
+ *   codes, scales and zero terms are rearranged once into a GPU-specific layout).
+ *   layout W4_LAYOUT_GEMV feeds w4a16_gemv, W4_LAYOUT_GEMM feeds w4a8_gemm and (one slab per
+ *   expert) w4a8_grouped_gemm. The packed buffer is opaque; its size is
+ *   w4_prepack_bytes(N, K, group, layout) (0 for invalid arguments) and includes padding of
+ *   N and K to the kernel tiles. For W4_SYM, zeros must be NULL (z = 8 is implied).
+ *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG.
+ */
+size_t w4_prepack_bytes(int64_t N, int64_t K, int group, int layout);
+w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, const int16_t *zeros,
+                     int64_t N, int64_t K, int group, int mode, int layout, void *packed,
+                     cudaStream_t stream);
+
+/*
+ * fp8_row_quant -- dynamic per-row FP8 E4M3 activation quantization
+ *   (TAHOMA "Achievement 2: 8-bit activations without a calibration set"): for every row m,
+ *   amax = max_k |x[m,k]|, s[m] = max(amax, 1e-8f) / 448.0f, X8[m,k] = e4m3(x[m,k] / s[m])
+ *   with IEEE fp32 division, round-to-nearest-even and saturation to +-448. An all-zero row
+ *   gives all-zero codes.
+ *   X_bf16      device, bf16 [M, K]; M >= 1, K >= 16, K % 16 == 0
+ *   X_e4m3      device, uint8 [M, K]
+ *   row_scale   device, fp32 [M]
+ *   group_sums  device, fp32 [M, K/group] or NULL: sum of the E4M3 VALUES (not scaled by
+ *               s[m]) of each group of `group` consecutive codes, summed exactly and rounded
+ *               once to fp32. w4a8_gemm needs them (it applies the weight zero point
+ *               through them). group must be 32, 64 or 128 when group_sums != NULL.
+ *   Errors: NULL / SHAPE / GROUP / ALIGN.
+ */
+w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uint8_t *X_e4m3,
+                        float *row_scale, float *group_sums, cudaStream_t stream);
+
+/*
+ * w4a16_gemv -- weight-only INT4 decode GEMV with the dequantization fused into the
+ *   product (QLWG "Weight-only methods": 4-bit weights, 16-bit activations, dequantized
+ *   inside the matmul; "The Problem & Context": decode reads every weight once and that
+ *   read sets the pace):
+ *     y[m, n] = sum_j s[n,j] * sum_{k in group j} x[m,k] * (q[n,k] - z[n,j])
+ *   with fp32 accumulation; the output is rounded once (to bf16, or kept fp32).
+ *   x_bf16   device, bf16 [M, K]; 1 <= M <= 16
+ *   packed   device, w4_prepack(..., W4_LAYOUT_GEMV) of W[N, K]
+ *   y        device, bf16 [M, N] (out_fp32 == 0) or fp32 [M, N] (out_fp32 == 1)
+ *   Errors: NULL / SHAPE (M outside 1..16, N < 1, K < 32) / GROUP / ALIGN / ARG.
+ */
+w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
+                     int group, int mode, void *y, int out_fp32, cudaStream_t stream);
+
+/*
+ * w4a8_gemm -- W4A8 GEMM on the FP8 tensor cores (TAHOMA "Achievement 2", the list under
+ *   "the A8 in W4A8": packed 4-bit weights are read from HBM and expanded to E4M3 in the
+ *   kernel, the activation and expanded weight enter an FP8 tensor-core MMA, accumulation
+ *   is FP32, the per-token activation scale is applied in the epilogue, the result is BF16):
+ *     Y[m, n] = s_a[m] * sum_j s[n,j] * sum_{k in group j} a8[m,k] * (q[n,k] - z[n,j])
+ *   with a8 the E4M3 value of X_e4m3[m,k]. The expanded weights are exact small integers
+ *   in E4M3; the group scale multiplies fp32 per-group partial sums and the zero point is
+ *   applied through the activation group sums, so the MMA operands are exactly the
+ *   dequantized operands.
+ *   X_e4m3      device, uint8 [M, K] from fp8_row_quant
+ *   row_scale   device, fp32 [M] from fp8_row_quant
+ *   group_sums  device, fp32 [M, K/group] from fp8_row_quant with the same group
+ *   packed      device, w4_prepack(..., W4_LAYOUT_GEMM) of W[N, K]
+ *   Y           device, bf16 [M, N] (out_fp32 == 0) or fp32 [M, N] (out_fp32 == 1)
+ *   M >= 1; N >= 1; K >= 128, K % 32 == 0.
+ *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG.
+ */
+w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const float *group_sums,
+                    int64_t M, const void *packed, int64_t N, int64_t K, int group, int mode,
+                    void *Y, int out_fp32, cudaStream_t stream);
+
+/*
+ * w4a8_grouped_gemm -- w4a8_gemm for E experts at once (mixture-of-experts layers whose
+ *   expert weights are 4-bit; the blog post "4-bit by default", gpt-oss paragraph). Rows
+ *   [off[e], off[e+1]) of X_e4m3 / row_scale / group_sums / Y belong to expert e and are
+ *   multiplied by expert e's weight.
+ *   expert_row_offsets  device, int32 [E+1], non-decreasing, off[0] == 0, off[E] == M_total
+ *   packed              device, E slabs of w4_prepack_bytes(N, K, group, W4_LAYOUT_GEMM)
+ *                       bytes each, slab e at packed + e * that size
+ *   Y                   device, bf16 [M_total, N]
+ *   1 <= E <= 1024. Errors: NULL / SHAPE / GROUP / ALIGN / ARG.
+ */
+w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale,
+                            const float *group_sums, const int32_t *expert_row_offsets, int E,
+                            int64_t M_total, const void *packed, int64_t N, int64_t K, int group,
+                            int mode, void *Y, cudaStream_t stream);
+
+/*
+ * w4_device_status -- synchronizes `stream`, then reads and clears the device status word
+ *   of the current device. *code_out receives W4_OK or the first W4_ERR_TIMEOUT /
+ *   W4_ERR_DEVICE_CHECK recorded since the last call. Returns W4_ERR_CUDA if the
+ *   synchronization itself fails.
+ */
+w4_status w4_device_status(cudaStream_t stream, int *code_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4_H_ */

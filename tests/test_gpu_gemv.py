@@ -1,0 +1,115 @@
+"""GPU w4a16_gemv vs the CPU oracle's fp64 product of the dequantized weight.
+
+Tolerances (relative Frobenius): bf16 output against the fp64 result rounded to bf16 at
+1e-3 (the benchmark spec's bound); fp32 output against the unrounded fp64 result at 1e-4. The
+kernel forms each 32-wide chunk as sum x*(128+q) - (128+z)*sum x in fp32; the offset of 128
+makes the fp32 partial sums about 30x larger than the result, so its rounding error is
+~2^-24 * 30 * sqrt(32) per chunk, i.e. ~1e-5 relative: 1e-4 leaves a margin of 10."""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_gemm_wise_b200 import synth, w4
+from helpers import bf16_round, cuda, np_of, rel_frob, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@functools.lru_cache(maxsize=None)
+def quantized(kind, K, N, group, mode, grid_name):
+    if kind == "decode":
+        W = synth.decode_weight(K, N)
+    elif kind == "single":
+        W, _ = synth.single_layer()
+    else:
+        W = synth.student_t3_weight(N, K, 3, 700 + N + K)
+    grid = {"one": [1.0], "twenty": synth.clip_grid_20()}[grid_name]
+    codes, scales, zeros, _ = oracle.quantize(synth.bf16_bits(W), group, mode, grid, want_chosen=False)
+    return codes, scales, zeros
+
+
+def gpu_gemv(codes, scales, zeros, N, K, group, mode, x_bits, out_fp32):
+    M = x_bits.shape[0]
+    packed = w4.alloc_packed(N, K, group, w4.W4_LAYOUT_GEMV)
+    c = to_dev(codes)
+    s = to_dev(scales.view(np.int16))
+    z = to_dev(zeros) if zeros is not None else None
+    w4.w4_prepack(c, s, z, N, K, group, mode, w4.W4_LAYOUT_GEMV, packed)
+    x = to_dev(x_bits.view(np.int16)).view(torch.bfloat16)
+    y = torch.empty(M, N, dtype=torch.float32 if out_fp32 else torch.bfloat16, device=cuda())
+    w4.w4a16_gemv(x, M, packed, N, K, group, mode, y, out_fp32)
+    torch.cuda.synchronize()
+    return y.float().cpu().numpy().astype(np.float64)
+
+
+def check(codes, scales, zeros, group, mode, x_bits):
+    N, K = codes.shape[0], codes.shape[1] * 2
+    ref = oracle.gemv_ref(x_bits, codes, scales, zeros, group, mode)
+    y32 = gpu_gemv(codes, scales, zeros, N, K, group, mode, x_bits, 1)
+    e32 = rel_frob(ref, y32)
+    assert e32 <= 1e-4, e32
+    y16 = gpu_gemv(codes, scales, zeros, N, K, group, mode, x_bits, 0)
+    e16 = rel_frob(bf16_round(ref), y16)
+    assert e16 <= 1e-3, e16
+    return e32, e16
+
+
+def test_single_layer_m1():
+    codes, scales, zeros = quantized("single", 576, 1536, 32, "sym", "one")
+    _, x = synth.single_layer()
+    check(codes, scales, None, 32, "sym", synth.bf16_bits(x))
+
+
+@pytest.mark.parametrize("K,N", synth.DECODE_SHAPES)
+@pytest.mark.parametrize("M", synth.DECODE_M)
+def test_decode_sweep_full_size(K, N, M):
+    codes, scales, zeros = quantized("decode", K, N, 128, "asym", "twenty")
+    x = synth.decode_activation(M, K)
+    check(codes, scales, zeros, 128, "asym", synth.bf16_bits(x))
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 9, 16])
+@pytest.mark.parametrize("group,mode", [(32, "sym"), (64, "asym"), (128, "asym"), (128, "sym")])
+def test_ragged(M, group, mode):
+    N = 77                              # not a multiple of 8
+    K = 320 if group < 128 else 384     # 320: not a multiple of the 128-wide unit
+    codes, scales, zeros = quantized("t3", K, N, group, mode, "twenty")
+    x = synth.normal((M, K), 1.0, 4, 31 * M + group)
+    check(codes, scales, zeros, group, mode, synth.bf16_bits(x))
+
+
+def test_tiny():
+    for N, K, g in [(1, 32, 32), (8, 128, 128), (9, 64, 32)]:
+        codes, scales, zeros = quantized("t3", K, N, g, "asym", "one")
+        x = synth.normal((1, K), 1.0, 5, N + K)
+        check(codes, scales, zeros, g, "asym", synth.bf16_bits(x))
+
+
+def test_extreme_zero_points():
+    """Blocks far from zero make |z| large (one-signed blocks); the chunk offset removal
+    must still be exact to fp32 rounding."""
+    rng = np.random.default_rng(3)
+    W = rng.normal(0, 0.02, (64, 256))
+    blocks = W.reshape(64, 8, 32)
+    pick = rng.integers(0, 3, (64, 8))
+    blocks[pick == 1] = 1.0 + rng.uniform(0, 0.02, (int((pick == 1).sum()), 32))     # z far below 0
+    blocks[pick == 2] = -3.0 - rng.uniform(0, 0.05, (int((pick == 2).sum()), 32))    # z far above 15
+    W = blocks.reshape(64, 256)
+    bits = synth.bf16_bits(torch.tensor(W, dtype=torch.float32).to(torch.bfloat16))
+    codes, scales, zeros, _ = oracle.quantize(bits, 32, "asym", synth.clip_grid_20(), want_chosen=False)
+    assert np.abs(zeros).max() > 241
+    x = synth.normal((4, 256), 1.0, 6, 1)
+    check(codes, scales, zeros, 32, "asym", synth.bf16_bits(x))
+
+
+def test_one_hot_column():
+    codes, scales, zeros = quantized("t3", 256, 64, 128, "asym", "one")
+    x = np.zeros((1, 256), np.float32)
+    x[0, 131] = 1.0
+    xb = synth.bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+    y = gpu_gemv(codes, scales, zeros, 64, 256, 128, "asym", xb, 1)
+    Wd = oracle.dequantize(codes, scales, zeros, 128, "asym")
+    assert np.array_equal(y[0], Wd[:, 131])
