@@ -55,56 +55,51 @@ def gemv_bytes(M, N, K, g=128):
 # ------------------------------------------------------------------ clocks
 
 class Clocks:
-    """nvidia-smi sampler running during the timed region."""
+    """Samples SM clock and clock-event reasons with NVML every ~2 ms while the timed
+    region runs (from just before its first launch until after its final synchronize)."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, index: int):
         self.index = index
-        self.lines = []
-        self.proc = None
+        self.mhz, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
 
     def __enter__(self):
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        except Exception:  # no NVML: report no samples
+            self.nv = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.mhz.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __exit__(self, *exc):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self.nv:
+            self.t.join(timeout=2)
 
     def summary(self):
-        mhz, maxmhz, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                mhz.append(float(f[1]))
-                maxmhz = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(mhz)) if mhz else None, "sm_max_mhz": maxmhz,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+        return {"sm_mhz": float(np.median(self.mhz)) if self.mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.mhz)}
 
 
 # ------------------------------------------------------------------ timing helpers
@@ -129,7 +124,9 @@ def flush_l2(buf):
 # ------------------------------------------------------------------ our arm
 
 class Decode:
-    """The decode sweep: quantize (GPU), prepack R copies per shape, M=1 activations."""
+    """The decode sweep: quantize (GPU), prepack R copies per shape, M=1 activations.
+    Step i runs one GEMV per shape on weight copy i % R; each step is captured once in a
+    CUDA graph (the decode loop replays graphs, as serving engines do)."""
 
     def __init__(self, M, seed, dev, copies=None):
         from bit_gemm_wise_b200 import synth, w4
@@ -141,7 +138,7 @@ class Decode:
         self.bytes_per_step = sum(gemv_bytes(M, N, K) for K, N in self.shapes)
         packed_per_step = sum(w4.w4_prepack_bytes(N, K, g, w4.W4_LAYOUT_GEMV) for K, N in self.shapes)
         self.R = copies or max(2, -(-3 * L2_BYTES // packed_per_step))
-        self.packed, self.x, self.y = [], [], []
+        self.packed, self.x, self.y, self.ws = [], [], [], []
         for K, N in self.shapes:
             W = synth.decode_weight(K, N, seed, device=dev)
             codes, scales, zeros, _ = w4.alloc_quantized(N, K, g, "asym", device=dev, chosen=False)
@@ -154,12 +151,46 @@ class Decode:
             self.packed.append((p, nb))
             self.x.append(synth.decode_activation(M, K, seed, device=dev))
             self.y.append(torch.empty(M, N, dtype=torch.bfloat16, device=dev))
+            self.ws.append(w4.alloc_gemv_workspace(N, K, g, device=dev))
             del W, codes, scales, zeros
         self.launches_per_step = len(self.shapes)
+        self.graphs = None
+        # consecutive GEMVs may overlap: each streams its weights while its predecessor
+        # finishes (programmatic dependent launch); activations are read after it completes
+        self.flags = w4.W4_OVERLAP_PREVIOUS
+
+    def gemv(self, si, i):
+        (K, N), (p, nb) = self.shapes[si], self.packed[si]
+        self.w4.w4a16_gemv(self.x[si], self.M, p[(i % self.R) * nb:], N, K, 128, "asym", self.y[si],
+                           self.flags, self.ws[si])
+
+    def step_eager(self, i):
+        for si in range(len(self.shapes)):
+            self.gemv(si, i)
+
+    def capture(self):
+        self.step_eager(0)  # first calls set kernel attributes outside the capture
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        self.graphs = []
+        for r in range(self.R):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                self.step_eager(r)
+            self.graphs.append(g)
+        self.shape_graphs = []
+        for si in range(len(self.shapes)):
+            gs = []
+            for r in range(self.R):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    self.gemv(si, r)
+                gs.append(g)
+            self.shape_graphs.append(gs)
+        torch.cuda.synchronize()
 
     def step(self, i):
-        for (K, N), (p, nb), x, y in zip(self.shapes, self.packed, self.x, self.y):
-            self.w4.w4a16_gemv(x, self.M, p[(i % self.R) * nb:], N, K, 128, "asym", y, 0)
+        self.graphs[i % self.R].replay()
 
 
 def run_ours(args, rank, world, dev):
@@ -169,6 +200,7 @@ def run_ours(args, rank, world, dev):
     stream = torch.cuda.current_stream()
 
     dec = Decode(1, args.seed, dev)
+    dec.capture()
     for i in range(args.warmup):
         dec.step(i)
     torch.cuda.synchronize()
@@ -185,30 +217,26 @@ def run_ours(args, rank, world, dev):
     ms_step = ms / args.steps
     value = world * dec.bytes_per_step / (ms_step * 1e-3) / 1e9
 
-    # per-shape launch times (events around blocks of launches of one shape)
+    # per-shape launch times (graph replays of one shape's GEMV, events around the block)
     per_shape = {}
     for si, (K, N) in enumerate(dec.shapes):
-        p, nb = dec.packed[si]
-        n_it = max(8, args.steps)
+        n_it = max(8 * dec.R, args.steps)
+        gs = dec.shape_graphs[si]
+        t_ms = time_region(lambda i, gs=gs: gs[i % len(gs)].replay(), n_it, stream) / n_it
+        per_shape[f"K{K}xN{N}"] = {"us": round(t_ms * 1e3, 3),
+                                   "GBps": round(gemv_bytes(1, N, K) / (t_ms * 1e-3) / 1e9, 1)}
 
-        def one(i, si=si, K=K, N=N, p=p, nb=nb):
-            w4.w4a16_gemv(dec.x[si], 1, p[(i % dec.R) * nb:], N, K, 128, "asym", dec.y[si], 0)
-
-        one(0)
-        t_ms = time_region(one, n_it, stream) / n_it
-        per_shape[f"{K}x{N}"] = {"us": round(t_ms * 1e3, 3),
-                                 "GBps": round(gemv_bytes(1, N, K) / (t_ms * 1e-3) / 1e9, 1)}
-
-    # e2e through the public API with host buffers: h2d x, GEMVs, d2h y per step
+    # e2e through the public Python API with host buffers, every step: pinned h2d of the
+    # activations, the four w4a16_gemv calls (not graphed), d2h of the outputs
     xh = [x.cpu().pin_memory() for x in dec.x]
     yh = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in dec.y]
     h2d = sum(x.numel() * 2 for x in xh)
     d2h = sum(y.numel() * 2 for y in yh)
 
     def e2e_step(i):
-        for si, (K, N) in enumerate(dec.shapes):
+        for si in range(len(dec.shapes)):
             dec.x[si].copy_(xh[si], non_blocking=True)
-        dec.step(i)
+        dec.step_eager(i)
         for si in range(len(dec.shapes)):
             yh[si].copy_(dec.y[si], non_blocking=True)
 
@@ -258,8 +286,9 @@ def measure_rows(args, dev, pk):
     # GEMV at M = 4 and 16 (ALU-bound on the CUDA cores)
     for M in (4, 16):
         d = Decode(M, args.seed, dev)
+        d.capture()
         d.step(0)
-        ms = time_region(d.step, 20) / 20
+        ms = time_region(d.step, 6 * d.R) / (6 * d.R)
         rows[f"w4a16_gemv_M{M}"] = {"value": round(d.bytes_per_step / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                                     "us_per_step": round(ms * 1e3, 2),
                                     "frac_hbm": round(d.bytes_per_step / (ms * 1e-3) / 1e9 / pk["hbm"], 4)}

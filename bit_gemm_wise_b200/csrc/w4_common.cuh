@@ -115,6 +115,11 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Named barrier over `n` threads (a multiple of 32); id 0 is __syncthreads.
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // Streaming 128-bit global load that does not allocate in L1.
 __device__ __forceinline__ uint4 ldg_stream(const void *p) {
     uint4 v;

@@ -6,24 +6,36 @@
 //
 //   y[m, n] = sum_j s[n,j] * sum_{k in j} x[m,k] * (q[n,k] - z[n,j])
 //
-// HBM-bound streaming kernel on the CUDA cores (W4_LAYOUT_GEMV, see w4_layout.cuh):
-//  * one CTA (8 warps) per octet of 8 weight rows; the warps take the octet's 128-wide
-//    units round-robin, every lane streams one 16-byte word of codes per unit
-//    (ld.global.nc.L1::no_allocate, a warp reads 512 contiguous bytes);
-//  * the octet's scales/zeros and the activation rows are staged into shared memory by
-//    one bulk copy (cp.async.bulk, completion on an mbarrier with a bounded wait);
-//  * nibbles become bf16 pairs with one AND/OR: (w & 0x000F000F) | 0x43004300 is the pair
-//    (128 + q_a, 128 + q_b), exact in bf16;
-//  * fma.rn.f32.bf16 multiplies the bf16 activation by the bf16 (128 + q) exactly and
-//    accumulates in fp32; per 32-wide chunk the offset is removed with the chunk's
-//    activation sum: sum x*(q - z) = sum x*(128 + q) - (128 + z) * sum x;
-//  * the chunk partial is scaled by the group's fp16 scale in fp32 and summed over the
-//    row; the four chunk lanes of a row reduce by shuffles, the 8 warps through shared
-//    memory in a fixed order (deterministic).
+// HBM-bound streaming kernel on the CUDA cores (W4_LAYOUT_GEMV, see w4_layout.cuh).
+//  * Persistent stream-K: the weight is a sequence of T = (N/8) * (Kpad/128) units of
+//    512 bytes (8 rows x 128 k) in octet-major order; CTA c of P (one per SM) owns the
+//    contiguous unit range [t0, t1) with |t1 - t0| differing by at most one between CTAs,
+//    so every SM streams the same number of bytes whatever N and K are.
+//  * Warp w of a CTA takes units t0 + w, t0 + w + W, ... (so the W warps read W
+//    consecutive 512-byte units, i.e. contiguous memory) and keeps a queue of the next
+//    units' codes and scales in registers (128-bit streaming loads that bypass L1), so
+//    each SM keeps ~64 KB of loads in flight. The activations (and the per-32-chunk
+//    activation sums) are staged once per CTA in shared memory with a bulk copy
+//    (cp.async.bulk, bounded mbarrier wait).
+//  * A lane (row r = lane/4, chunk c = lane%4) turns a 16-byte word of codes into bf16
+//    pairs with one AND/OR each
+//    ((w & 0x000F000F) | 0x43004300 is the exact pair 128 + q), multiplies them into fp32
+//    with fma.rn.f32.bf16, and removes the offset per 32-wide chunk with the chunk's
+//    activation sum: sum x*(q - z) = sum x*(128 + q) - (128 + z) * sum x. The chunk
+//    partial times the fp16 group scale is accumulated per octet in registers.
+//  * Octets wholly inside a CTA's range are reduced in shared memory (fixed warp order)
+//    and written. An octet split between CTAs is finished by the last of its CTAs to
+//    arrive on a per-octet counter: it adds the CTAs' partials in CTA order (so results are
+//    deterministic) and resets the counter. Partials and counters live in the caller's
+//    workspace, which every call leaves zero-filled.
 #include "w4_common.cuh"
 #include "w4_layout.cuh"
 
 namespace w4 {
+namespace gemv {
+
+constexpr int SMEM_LIMIT = 100 * 1024;
+constexpr int PF = 4;  // units queued per warp
 
 __device__ __forceinline__ void fma2_bf16(float &a0, float &a1, uint32_t x, uint32_t q) {
     asm("{\n .reg .b16 xl, xh, ql, qh;\n mov.b32 {xl, xh}, %2;\n mov.b32 {ql, qh}, %3;\n"
@@ -34,198 +46,407 @@ __device__ __forceinline__ void fma2_bf16(float &a0, float &a1, uint32_t x, uint
 
 __device__ __forceinline__ uint32_t magic_pair(uint32_t w) { return (w & 0x000F000Fu) | 0x43004300u; }
 
-struct GemvArgs {
-    const uint16_t *x;
-    const uint8_t *packed;
-    void *y;
-    int *status;
-    int64_t N, K, Kpad, U;
-    size_t codes_bytes;
-    int M, g, out_fp32, stage_x;
-    uint32_t slab_bytes;  // scales of one octet
+// Division of 32-bit unsigned values by an invariant divisor d (Granlund & Montgomery,
+// "Division by invariant integers using multiplication", 1994): with l = ceil(log2 d),
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (t + ((n - t) >> min(l,1))) >> max(l-1,0)
+// where t = mulhi(m, n). Exact for every n < 2^32.
+struct FastDiv {
+    uint32_t d, m, s1, s2;
 };
 
-template <int MT>
-__global__ void __launch_bounds__(256) gemv_kernel(const GemvArgs a) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
-    uint32_t *sz = reinterpret_cast<uint32_t *>(smem + 16);                    // scales slab
-    float *sx = reinterpret_cast<float *>(smem + 16 + a.slab_bytes);           // [MT][Kpad/32]
-    const int nck = (int)(a.Kpad / 32);
-    float *red = sx + MT * nck;                                                // [8][8][MT]
-    uint16_t *xs = reinterpret_cast<uint16_t *>(red + 64 * MT);                // [M][K] if staged
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < d) ++l;
+    FastDiv f;
+    f.d = d;
+    f.m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d) + 1);
+    f.s1 = l < 1 ? l : 1;
+    f.s2 = l > 1 ? l - 1 : 0;
+    return f;
+}
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int r = lane >> 2, c = lane & 3;
-    const int64_t o = blockIdx.x;
-    const int M = a.M;
-    const int64_t K = a.K;
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+    const uint32_t t = __umulhi(f.m, n);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
 
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
-        const uint32_t xbytes = a.stage_x ? (uint32_t)(M * K * 2) : 0u;
-        mbar_arrive_expect_tx(bar, a.slab_bytes + xbytes);
-        bulk_g2s(sz, a.packed + a.codes_bytes + (size_t)o * a.slab_bytes, a.slab_bytes, bar);
-        if (a.stage_x) bulk_g2s(xs, a.x, xbytes, bar);
-    }
+struct Args {
+    const uint16_t *x;
+    const uint8_t *codes;      // packed codes
+    const uint8_t *scales;     // packed scales (u32 entries)
+    void *y;
+    float *ws_part;            // [P][2][8][MT] partials of boundary octets
+    int *ws_count;             // [N8] arrival counters (zero between calls)
+    int *status;
+    int64_t N, K;
+    uint32_t U, T;             // U = units per octet, T = total units (< 2^31)
+    FastDiv divU;
+    uint32_t base, rem, step;  // range of CTA c starts at c*base + min(c, rem)*step
+    FastDiv divB1, divB;       // division by base + step and by base
+    int M, g, out_fp32, nol, pdl;
+    uint32_t sub;              // scale bytes per unit
+    uint32_t off_sx, off_slot;
+};
 
-    // first codes of this warp, issued before waiting on the staged data
-    const uint8_t *octet_codes = a.packed + (size_t)o * (size_t)a.U * 512;
-    constexpr int UNR = 4;
-    uint4 q[UNR];
-#pragma unroll
-    for (int i = 0; i < UNR; ++i) {
-        const int64_t u = warp + 8 * i;
-        if (u < a.U) q[i] = ldg_stream(octet_codes + u * 512 + lane * 16);
-    }
+__device__ __forceinline__ uint32_t range_start(const Args &a, uint32_t c) {
+    return c * a.base + (c < a.rem ? c : a.rem) * a.step;
+}
 
-    if (!mbar_wait_bounded(bar, 0, a.status)) {
-        mbar_wait_bounded(bar, 0, a.status);  // let copies in flight land before leaving
-        return;
-    }
+__device__ __forceinline__ uint32_t cta_of_unit(const Args &a, uint32_t t) {
+    const uint32_t big = (a.base + a.step) * a.rem;
+    return t < big ? fdiv(t, a.divB1) : a.rem + fdiv(t - big, a.divB);
+}
 
-    // activation sums of every 32-wide chunk (chunks past K are zero)
-    for (int idx = tid; idx < MT * nck; idx += 256) {
-        const int m = idx / nck, ck = idx - m * nck;
-        float s = 0.0f;
-        if (m < M && (int64_t)ck * 32 < K) {
-            if (a.stage_x) {
-                const uint32_t *xv = reinterpret_cast<const uint32_t *>(xs + (int64_t)m * K + ck * 32);
-#pragma unroll
-                for (int t = 0; t < 16; ++t) s = __fadd_rn(__fadd_rn(s, bf16_lo(xv[t])), bf16_hi(xv[t]));
-            } else {
-                const uint4 *xv = reinterpret_cast<const uint4 *>(a.x + (int64_t)m * K + ck * 32);
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const uint4 v = __ldg(xv + t);
-                    s = __fadd_rn(__fadd_rn(s, bf16_lo(v.x)), bf16_hi(v.x));
-                    s = __fadd_rn(__fadd_rn(s, bf16_lo(v.y)), bf16_hi(v.y));
-                    s = __fadd_rn(__fadd_rn(s, bf16_lo(v.z)), bf16_hi(v.z));
-                    s = __fadd_rn(__fadd_rn(s, bf16_lo(v.w)), bf16_hi(v.w));
-                }
-            }
-        }
-        sx[idx] = s;
-    }
-    __syncthreads();
-
-    float y[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) y[m] = 0.0f;
-    const int per_unit = 128 / a.g;
-
-    for (int64_t u0 = warp; u0 < a.U; u0 += 8 * UNR) {
-#pragma unroll
-        for (int i = 0; i < UNR; ++i) {
-            const int64_t u = u0 + 8 * i;
-            if (u >= a.U) break;
-            const uint4 w4v = q[i];
-            // prefetch the unit UNR rounds ahead into the slot just consumed
-            const int64_t un = u + 8 * UNR;
-            if (un < a.U) q[i] = ldg_stream(octet_codes + un * 512 + lane * 16);
-            const int64_t k0 = u * 128 + c * 32;
-            if (k0 >= K) continue;
-            const uint32_t e = sz[(u * 8 + r) * per_unit + (c * 32) / a.g];
-            const float s = __half2float(__ushort_as_half((unsigned short)(e & 0xFFFF)));
-            const float cz = (float)(128 + (int)(int16_t)(e >> 16));
-            const uint32_t wv[4] = {w4v.x, w4v.y, w4v.z, w4v.w};
-            uint32_t p[4][4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                p[t][0] = magic_pair(wv[t]);
-                p[t][1] = magic_pair(wv[t] >> 4);
-                p[t][2] = magic_pair(wv[t] >> 8);
-                p[t][3] = magic_pair(wv[t] >> 12);
-            }
-            const int ck = (int)(k0 >> 5);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                if (m >= M) break;
-                float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    uint4 xv;
-                    if (a.stage_x)
-                        xv = *reinterpret_cast<const uint4 *>(xs + (int64_t)m * K + k0 + 8 * t);
-                    else
-                        xv = __ldg(reinterpret_cast<const uint4 *>(a.x + (int64_t)m * K + k0 + 8 * t));
-                    fma2_bf16(a0, a1, xv.x, p[t][0]);
-                    fma2_bf16(a0, a1, xv.y, p[t][1]);
-                    fma2_bf16(a0, a1, xv.z, p[t][2]);
-                    fma2_bf16(a0, a1, xv.w, p[t][3]);
-                }
-                const float part = fmaf(-cz, sx[m * nck + ck], a0 + a1);
-                y[m] = fmaf(s, part, y[m]);
-            }
-        }
-    }
-
+template <int MT, int W>
+__device__ __forceinline__ void flush_octet(uint32_t ol, float (&y)[MT], float *slot, int warp, int lane) {
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
         y[m] += __shfl_xor_sync(FULL, y[m], 1);
         y[m] += __shfl_xor_sync(FULL, y[m], 2);
     }
-    if (c == 0) {
+    if ((lane & 3) == 0) {
+        float *d = slot + (ol * W + warp) * 8 * MT + (lane >> 2) * MT;
 #pragma unroll
-        for (int m = 0; m < MT; ++m) red[(warp * 8 + r) * MT + m] = y[m];
+        for (int m = 0; m < MT; ++m) d[m] = y[m];
     }
-    __syncthreads();
-    if (tid < 8 * MT) {
-        const int rr = tid / MT, m = tid % MT;
-        const int64_t n = o * 8 + rr;
-        if (m < M && n < a.N) {
-            float acc = red[rr * MT + m];
 #pragma unroll
-            for (int w = 1; w < 8; ++w) acc += red[(w * 8 + rr) * MT + m];
-            if (a.out_fp32) static_cast<float *>(a.y)[(int64_t)m * a.N + n] = acc;
-            else static_cast<__nv_bfloat16 *>(a.y)[(int64_t)m * a.N + n] = __float2bfloat16_rn(acc);
-        }
-    }
+    for (int m = 0; m < MT; ++m) y[m] = 0.0f;
+}
+
+template <int MT> struct Warps { static constexpr int value = MT == 1 ? 32 : (MT <= 4 ? 16 : 8); };
+
+__device__ __forceinline__ void store_y(const Args &a, int m, int64_t n, float v) {
+    if (a.out_fp32) static_cast<float *>(a.y)[(int64_t)m * a.N + n] = v;
+    else static_cast<__nv_bfloat16 *>(a.y)[(int64_t)m * a.N + n] = __float2bfloat16_rn(v);
 }
 
 template <int MT>
-static w4_status launch_gemv(GemvArgs a, cudaStream_t stream, int64_t N8) {
-    const int nck = (int)(a.Kpad / 32);
-    const size_t base = 16 + a.slab_bytes + (size_t)MT * nck * 4 + (size_t)64 * MT * 4;
-    const size_t xbytes = (size_t)a.M * a.K * 2;
-    a.stage_x = (xbytes <= 48 * 1024) ? 1 : 0;
-    const size_t smem = base + (a.stage_x ? xbytes : 0);
-    if (smem > 200 * 1024) return W4_ERR_SHAPE;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return W4_ERR_CUDA;
-    gemv_kernel<MT><<<(unsigned)N8, 256, smem, stream>>>(a);
+__global__ void __launch_bounds__(Warps<MT>::value * 32, 1) gemv_kernel(const Args a) {
+    constexpr int W = Warps<MT>::value;
+    constexpr int THREADS = W * 32;
+    extern __shared__ __align__(16) uint8_t smem[];
+    int *flags = reinterpret_cast<int *>(smem);   // [1..2] last-arriver flags
+    float *sx = reinterpret_cast<float *>(smem + a.off_sx);
+    float *slot = reinterpret_cast<float *>(smem + a.off_slot);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = lane >> 2, cc = lane & 3;
+    const uint32_t c = blockIdx.x;
+    const uint32_t t0 = range_start(a, c), t1 = range_start(a, c + 1);
+    const uint32_t o_first = fdiv(t0, a.divU), o_last = fdiv(t1 - 1, a.divU);
+    const int M = a.M;
+    const uint32_t Kc = (uint32_t)a.K, Uc = a.U;
+    const int nck = (int)(Uc * 4);  // 32-wide chunks per row (padded)
+
+    // ---- the weight stream does not depend on earlier kernels: start it first
+    const uint32_t tb = t0 + (uint32_t)warp;
+    const int per_unit = 128 / a.g;
+    const uint32_t sc_lane = (uint32_t)(r * per_unit + (cc * 32) / a.g) * 4;
+    const uint8_t *cp = a.codes + (size_t)tb * 512 + lane * 16;
+    const uint8_t *sp = a.scales + (size_t)tb * a.sub + sc_lane;
+    const size_t cstep = (size_t)W * 512, sstep = (size_t)W * a.sub;
+    uint4 qv[PF];
+    uint32_t ev[PF];
+#pragma unroll
+    for (int i = 0; i < PF; ++i) {
+        if (tb + (uint32_t)(i * W) < t1) {
+            qv[i] = ldg_stream(cp + i * cstep);
+            ev[i] = __ldg(reinterpret_cast<const uint32_t *>(sp + i * sstep));
+        }
+    }
+    cp += PF * cstep;
+    sp += PF * sstep;
+
+    for (int i = tid; i < a.nol * W * 8 * MT; i += THREADS) slot[i] = 0.0f;
+    // activations may be written by the previous kernel in the stream
+    if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // activation sums of every 32-wide chunk (chunks past K are zero)
+    for (int idx = tid; idx < MT * nck; idx += THREADS) {
+        const int m = idx / nck, ck = idx - m * nck;
+        float s = 0.0f;
+        if (m < M && (uint32_t)ck * 32 < Kc) {
+            const uint4 *xv = reinterpret_cast<const uint4 *>(a.x + (int64_t)m * a.K + ck * 32);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const uint4 v = __ldg(xv + t);
+                s = __fadd_rn(__fadd_rn(s, bf16_lo(v.x)), bf16_hi(v.x));
+                s = __fadd_rn(__fadd_rn(s, bf16_lo(v.y)), bf16_hi(v.y));
+                s = __fadd_rn(__fadd_rn(s, bf16_lo(v.z)), bf16_hi(v.z));
+                s = __fadd_rn(__fadd_rn(s, bf16_lo(v.w)), bf16_hi(v.w));
+            }
+        }
+        sx[idx] = s;
+    }
+    __syncthreads();
+    if (a.pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    float y[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) y[m] = 0.0f;
+    uint32_t cur_ol = 0xffffffffu;  // octet of the accumulated partial, relative to o_first
+    for (uint32_t tq = tb; tq < t1; tq += (uint32_t)(PF * W)) {
+#pragma unroll
+        for (int i = 0; i < PF; ++i) {
+            const uint32_t t = tq + (uint32_t)(i * W);
+            if (t >= t1) break;
+            const uint4 wq = qv[i];
+            const uint32_t e = ev[i];
+            if (t + (uint32_t)(PF * W) < t1) {
+                qv[i] = ldg_stream(cp);
+                ev[i] = __ldg(reinterpret_cast<const uint32_t *>(sp));
+            }
+            cp += cstep;
+            sp += sstep;
+            const uint32_t o = fdiv(t, a.divU);
+            const uint32_t ol = o - o_first;
+            if (ol != cur_ol) {
+                if (cur_ol != 0xffffffffu) flush_octet<MT, W>(cur_ol, y, slot, warp, lane);
+                cur_ol = ol;
+            }
+            const uint32_t k0 = (t - o * Uc) * 128u + (uint32_t)cc * 32u;
+            if (k0 >= Kc) continue;
+            const float scl = __half2float(__ushort_as_half((unsigned short)(e & 0xFFFF)));
+            const float cz = (float)(int)(int16_t)(e >> 16) + 128.0f;
+            uint32_t p[4][4];
+            const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                p[q][0] = magic_pair(wv[q]);
+                p[q][1] = magic_pair(wv[q] >> 4);
+                p[q][2] = magic_pair(wv[q] >> 8);
+                p[q][3] = magic_pair(wv[q] >> 12);
+            }
+            const uint32_t ck = k0 >> 5;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (m >= M) break;
+                float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+                const uint4 *xp = reinterpret_cast<const uint4 *>(a.x + (int64_t)m * a.K + k0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 xv = __ldg(xp + q);
+                    fma2_bf16(a0, a1, xv.x, p[q][0]);
+                    fma2_bf16(a2, a3, xv.y, p[q][1]);
+                    fma2_bf16(a0, a1, xv.z, p[q][2]);
+                    fma2_bf16(a2, a3, xv.w, p[q][3]);
+                }
+                y[m] = fmaf(scl, fmaf(-cz, sx[m * nck + ck], (a0 + a1) + (a2 + a3)), y[m]);
+            }
+        }
+    }
+    if (cur_ol != 0xffffffffu) flush_octet<MT, W>(cur_ol, y, slot, warp, lane);
+    __syncthreads();
+
+    // ---------------------------------------------------- per-octet reduction
+    const int nol = (int)(o_last - o_first + 1);
+    for (int idx = tid; idx < nol * 8 * MT; idx += THREADS) {
+        const int ol = idx / (8 * MT), rm = idx - ol * 8 * MT;
+        const int rr = rm / MT, m = rm - rr * MT;
+        float acc = 0.0f;
+        for (int w = 0; w < W; ++w) acc += slot[(ol * W + w) * 8 * MT + rm];
+        const uint32_t o = o_first + ol;
+        const bool inside = o * Uc >= t0 && (o + 1) * Uc <= t1;
+        if (inside) {
+            const int64_t n = (int64_t)o * 8 + rr;
+            if (m < M && n < a.N) store_y(a, m, n, acc);
+        } else {
+            const int which = (o == o_first) ? 0 : 1;
+            a.ws_part[(((int64_t)c * 2 + which) * 8 + rr) * MT + m] = acc;
+        }
+    }
+    // boundary octets (stream-K partitions only): the last CTA to arrive adds all partials
+    // in CTA order and resets the counter
+    const bool b0 = !(o_first * Uc >= t0 && (o_first + 1) * Uc <= t1);
+    const bool b1 = (o_last != o_first) && !(o_last * Uc >= t0 && (o_last + 1) * Uc <= t1);
+    if (!b0 && !b1) return;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        flags[1] = 0;
+        flags[2] = 0;
+        for (int which = 0; which < 2; ++which) {
+            if (!(which == 0 ? b0 : b1)) continue;
+            const uint32_t o = which == 0 ? o_first : o_last;
+            const uint32_t cnt = cta_of_unit(a, (o + 1) * Uc - 1) - cta_of_unit(a, o * Uc) + 1;
+            const int prev = atomicAdd(&a.ws_count[o], 1);
+            flags[1 + which] = (prev == (int)cnt - 1) ? 1 : 0;
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    for (int which = 0; which < 2; ++which) {
+        if (!flags[1 + which]) continue;
+        const uint32_t o = which == 0 ? o_first : o_last;
+        const uint32_t cf = cta_of_unit(a, o * Uc), cl = cta_of_unit(a, (o + 1) * Uc - 1);
+        for (int rm = tid; rm < 8 * MT; rm += THREADS) {
+            const int rr = rm / MT, m = rm - rr * MT;
+            float acc = 0.0f;
+            for (uint32_t k = cf; k <= cl; ++k) {
+                const int wk = (fdiv(range_start(a, k), a.divU) == o) ? 0 : 1;
+                acc += __ldcg(a.ws_part + (((int64_t)k * 2 + wk) * 8 + rr) * MT + m);
+            }
+            const int64_t n = (int64_t)o * 8 + rr;
+            if (m < M && n < a.N) store_y(a, m, n, acc);
+        }
+        if (tid == 0) a.ws_count[o] = 0;
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+struct Plan {
+    Args a;
+    int P, smem;
+};
+
+static int sm_count_cached() {
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return num_sms();
+    if (!cache[dev]) cache[dev] = num_sms();
+    return cache[dev];
+}
+
+// Work partition. With N8 octets of U units each and S SMs: if whole octets split evenly
+// enough (fewer octets than SMs, or the busiest SM at most ~8% above the mean), every CTA
+// gets whole octets and no partial sum crosses CTAs; otherwise the unit stream is split
+// evenly (stream-K) and octets cut by a range boundary are finished through the workspace.
+template <int MT>
+static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g) {
+    constexpr int W = Warps<MT>::value;
+    const GemvLayout L = gemv_layout(N, K, g);
+    Args &a = p.a;
+    const int64_t T = L.N8 * L.U;
+    if (T >= (1LL << 31)) return false;
+    a.N = N; a.K = K; a.U = (uint32_t)L.U; a.T = (uint32_t)T;
+    a.divU = make_fastdiv(a.U);
+    a.M = (int)M; a.g = g;
+    a.sub = (uint32_t)(8 * (128 / g) * 4);
+    a.off_sx = 64;
+    a.off_slot = a.off_sx + (uint32_t)(MT * L.U * 4 * 4);
+    a.pdl = 0;
+    const int64_t S = sm_count_cached();
+    int64_t P;
+    bool aligned;
+    if (L.N8 <= S) {
+        P = L.N8;
+        aligned = true;
+    } else {
+        const int64_t per = (L.N8 + S - 1) / S;
+        aligned = (double)per <= 1.08 * (double)L.N8 / (double)S;
+        P = aligned ? (L.N8 + per - 1) / per : (S < T ? S : T);
+    }
+    while (true) {
+        if (aligned) {
+            a.base = (uint32_t)((L.N8 / P) * L.U);
+            a.rem = (uint32_t)(L.N8 % P);
+            a.step = a.U;
+        } else {
+            a.base = (uint32_t)(T / P);
+            a.rem = (uint32_t)(T % P);
+            a.step = 1;
+        }
+        const int64_t maxr = (int64_t)a.base + (a.rem ? a.step : 0);
+        const int64_t nol = (maxr + L.U - 1) / L.U + 1;
+        const size_t smem = a.off_slot + (size_t)nol * W * 8 * MT * 4;
+        if (smem <= (size_t)SMEM_LIMIT) {
+            a.nol = (int)nol;
+            p.P = (int)P;
+            p.smem = (int)smem;
+            break;
+        }
+        if (P >= T) return false;
+        aligned = false;
+        P = P * 2 < T ? P * 2 : T;
+    }
+    a.divB1 = make_fastdiv(a.base + a.step);
+    a.divB = make_fastdiv(a.base);
+    return true;
+}
+
+template <int MT>
+static size_t ws_need(int64_t N, int64_t K, int g) {
+    Plan p;
+    if (!make_plan<MT>(p, MT, N, K, g)) return 0;
+    return (size_t)p.P * 2 * 8 * MT * 4;
+}
+
+template <int MT>
+static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, int64_t K, int g, void *y, int out_fp32,
+                     void *ws, size_t ws_bytes, int pdl, cudaStream_t stream) {
+    constexpr int W = Warps<MT>::value;
+    Plan p;
+    if (!make_plan<MT>(p, M, N, K, g)) return W4_ERR_SHAPE;
+    const GemvLayout L = gemv_layout(N, K, g);
+    const size_t need = (size_t)p.P * 2 * 8 * MT * 4 + (size_t)L.N8 * 4;
+    if (!ws || ws_bytes < need) return W4_ERR_WORKSPACE;
+    Args &a = p.a;
+    a.x = static_cast<const uint16_t *>(x);
+    a.codes = static_cast<const uint8_t *>(packed);
+    a.scales = static_cast<const uint8_t *>(packed) + L.codes_bytes;
+    a.y = y;
+    a.out_fp32 = out_fp32;
+    a.ws_part = static_cast<float *>(ws);
+    a.ws_count = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + (size_t)p.P * 2 * 8 * MT * 4);
+    a.status = device_status_ptr();
+    a.pdl = pdl;
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT) !=
+            cudaSuccess)
+            return W4_ERR_CUDA;
+        attr_done[dev] = 1;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.P);
+    cfg.blockDim = dim3(W * 32);
+    cfg.dynamicSmemBytes = (size_t)p.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemv_kernel<MT>, a) != cudaSuccess) return W4_ERR_CUDA;
     return launch_status();
 }
 
+size_t workspace_bytes(int64_t N, int64_t K, int g) {
+    const GemvLayout L = gemv_layout(N, K, g);
+    size_t worst = 0;
+    const size_t cand[5] = {ws_need<1>(N, K, g), ws_need<2>(N, K, g), ws_need<4>(N, K, g), ws_need<8>(N, K, g),
+                            ws_need<16>(N, K, g)};
+    for (size_t v : cand) worst = v > worst ? v : worst;
+    return (worst + (size_t)L.N8 * 4 + 255) / 256 * 256;
+}
+
+}  // namespace gemv
 }  // namespace w4
 
 using namespace w4;
 
+W4_API size_t w4a16_gemv_workspace_bytes(int64_t N, int64_t K, int group) {
+    if (N < 1 || K < 32 || K % 32 != 0 || !valid_group(group) || K % group != 0) return 0;
+    return gemv::workspace_bytes(N, K, group);
+}
+
 W4_API w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K, int group,
-                            int mode, void *y, int out_fp32, cudaStream_t stream) {
+                            int mode, void *y, int flags, void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
     if (!x_bf16 || !packed || !y) return W4_ERR_NULL;
-    if (!valid_mode(mode) || (out_fp32 != 0 && out_fp32 != 1)) return W4_ERR_ARG;
+    if (!valid_mode(mode) || (flags & ~(W4_OUT_FP32 | W4_OVERLAP_PREVIOUS))) return W4_ERR_ARG;
+    const int out_fp32 = (flags & W4_OUT_FP32) ? 1 : 0;
+    const int pdl = (flags & W4_OVERLAP_PREVIOUS) ? 1 : 0;
     if (M < 1 || M > 16 || N < 1 || N > (int64_t)0x7fffffff * 8 || K < 32 || K % 32 != 0) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
-    if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(y)) return W4_ERR_ALIGN;
-    const GemvLayout L = gemv_layout(N, K, group);
-    GemvArgs a;
-    a.x = static_cast<const uint16_t *>(x_bf16);
-    a.packed = static_cast<const uint8_t *>(packed);
-    a.y = y;
-    a.status = device_status_ptr();
-    a.N = N; a.K = K; a.Kpad = L.Kpad; a.U = L.U;
-    a.codes_bytes = L.codes_bytes;
-    a.M = (int)M; a.g = group; a.out_fp32 = out_fp32; a.stage_x = 0;
-    a.slab_bytes = (uint32_t)(L.scales_bytes / (size_t)L.N8);
-    if (M <= 1) return launch_gemv<1>(a, stream, L.N8);
-    if (M <= 2) return launch_gemv<2>(a, stream, L.N8);
-    if (M <= 4) return launch_gemv<4>(a, stream, L.N8);
-    if (M <= 8) return launch_gemv<8>(a, stream, L.N8);
-    return launch_gemv<16>(a, stream, L.N8);
+    if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(y) || (workspace && !aligned16(workspace)))
+        return W4_ERR_ALIGN;
+    if (M <= 1) return gemv::run<1>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
+    if (M <= 2) return gemv::run<2>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
+    if (M <= 4) return gemv::run<4>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
+    if (M <= 8) return gemv::run<8>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
+    return gemv::run<16>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
 }

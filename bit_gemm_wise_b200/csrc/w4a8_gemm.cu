@@ -131,8 +131,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-
 // Find the (expert, first row, rows) of this CTA's token tile; false if past the last tile.
 __device__ __forceinline__ bool locate_tile(const Args &a, int t, int &e, int64_t &row0, int64_t &rows) {
     if (!a.offsets) {

@@ -17,6 +17,7 @@ import torch
 W4_OK = 0
 W4_SYM, W4_ASYM = 0, 1
 W4_LAYOUT_GEMV, W4_LAYOUT_GEMM = 0, 1
+W4_OUT_FP32, W4_OVERLAP_PREVIOUS = 1, 2  # flags of w4a16_gemv
 
 STATUS = {
     0: "W4_OK", 1: "W4_ERR_NULL", 2: "W4_ERR_SHAPE", 3: "W4_ERR_GROUP", 4: "W4_ERR_ALIGN",
@@ -35,7 +36,8 @@ SIGNATURES = [
     ("w4_prepack_bytes", _SZ, [_I64, _I64, _I, _I]),
     ("w4_prepack", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P]),
     ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P]),
-    ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
+    ("w4a16_gemv_workspace_bytes", _SZ, [_I64, _I64, _I]),
+    ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a8_gemm", _I, [_P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
     ("w4a8_grouped_gemm", _I, [_P, _P, _P, _P, _I, _I64, _P, _I64, _I64, _I, _I, _P, _P]),
     ("w4_device_status", _I, [_P, ctypes.POINTER(ctypes.c_int)]),
@@ -129,8 +131,14 @@ def fp8_row_quant(X, M, K, group, X8, row_scale, group_sums=None, stream=None):
     _check("fp8_row_quant", rc)
 
 
-def w4a16_gemv(x, M, packed, N, K, group, mode, y, out_fp32=0, stream=None):
-    rc = lib().w4a16_gemv(_ptr(x), M, _ptr(packed), N, K, group, _mode(mode), _ptr(y), int(out_fp32),
+def w4a16_gemv_workspace_bytes(N, K, group) -> int:
+    return int(lib().w4a16_gemv_workspace_bytes(N, K, group))
+
+
+def w4a16_gemv(x, M, packed, N, K, group, mode, y, flags, workspace, stream=None):
+    """flags: W4_OUT_FP32 (fp32 y) | W4_OVERLAP_PREVIOUS (programmatic dependent launch)."""
+    rc = lib().w4a16_gemv(_ptr(x), M, _ptr(packed), N, K, group, _mode(mode), _ptr(y), int(flags),
+                          _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _check("w4a16_gemv", rc)
 
@@ -166,6 +174,14 @@ def alloc_quantized(N, K, group, mode, device="cuda", chosen=True):
     zeros = torch.empty(N, J, dtype=torch.int16, device=device) if _mode(mode) == W4_ASYM else None
     ch = torch.empty(N, J, dtype=torch.uint8, device=device) if chosen else None
     return codes, scales, zeros, ch
+
+
+def alloc_gemv_workspace(N, K, group, device="cuda"):
+    """Zero-filled workspace for w4a16_gemv (calls leave it zero-filled)."""
+    nbytes = w4a16_gemv_workspace_bytes(N, K, group)
+    if nbytes == 0:
+        raise W4Error("w4a16_gemv_workspace_bytes", 2)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
 def alloc_packed(N, K, group, layout, device="cuda", copies: int = 1):

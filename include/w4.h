@@ -56,6 +56,14 @@ typedef enum {
 
 typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
 
+/* Flags of w4a16_gemv. */
+enum {
+    W4_OUT_FP32 = 1,        /* write y as fp32 instead of bf16                              */
+    W4_OVERLAP_PREVIOUS = 2 /* programmatic dependent launch: the kernel may start while the
+                               previous kernel on the stream is finishing; it streams its
+                               weights at once and reads x only after that kernel completed */
+};
+
 /* Kernel layouts produced by w4_prepack. */
 typedef enum { W4_LAYOUT_GEMV = 0, W4_LAYOUT_GEMM = 1 } w4_layout;
 
@@ -136,14 +144,26 @@ w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uin
  *   inside the matmul; "The Problem & Context": decode reads every weight once and that
  *   read sets the pace):
  *     y[m, n] = sum_j s[n,j] * sum_{k in group j} x[m,k] * (q[n,k] - z[n,j])
- *   with fp32 accumulation; the output is rounded once (to bf16, or kept fp32).
- *   x_bf16   device, bf16 [M, K]; 1 <= M <= 16
- *   packed   device, w4_prepack(..., W4_LAYOUT_GEMV) of W[N, K]
- *   y        device, bf16 [M, N] (out_fp32 == 0) or fp32 [M, N] (out_fp32 == 1)
- *   Errors: NULL / SHAPE (M outside 1..16, N < 1, K < 32) / GROUP / ALIGN / ARG.
+ *   with fp32 accumulation; the output is rounded once (to bf16, or kept fp32). The weight
+ *   stream is split evenly over one block per SM; rows whose reduction is split between
+ *   two blocks are finished by the last of them in a fixed order, so results are
+ *   bit-identical run to run on a given GPU.
+ *   x_bf16          device, bf16 [M, K]; 1 <= M <= 16
+ *   packed          device, w4_prepack(..., W4_LAYOUT_GEMV) of W[N, K]
+ *   y               device, bf16 [M, N], or fp32 [M, N] with W4_OUT_FP32 in flags
+ *   flags           W4_OUT_FP32 | W4_OVERLAP_PREVIOUS (see the enum); other bits: W4_ERR_ARG
+ *   workspace       device scratch of at least w4a16_gemv_workspace_bytes(N, K, group)
+ *                   bytes. It must be zero-filled before its first use; every call that
+ *                   completes leaves it zero-filled again, so one workspace can serve any
+ *                   sequence of calls on one stream. Calls that may run concurrently on
+ *                   the GPU need separate workspaces.
+ *   Errors: NULL / SHAPE (M outside 1..16, N < 1, K < 32) / GROUP / ALIGN / ARG /
+ *   WORKSPACE (missing or too small).
  */
+size_t w4a16_gemv_workspace_bytes(int64_t N, int64_t K, int group);
 w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
-                     int group, int mode, void *y, int out_fp32, cudaStream_t stream);
+                     int group, int mode, void *y, int flags, void *workspace,
+                     size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * w4a8_gemm -- W4A8 GEMM on the FP8 tensor cores (TAHOMA "Achievement 2", the list under

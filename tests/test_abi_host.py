@@ -90,9 +90,10 @@ def test_host_validation_rejects_before_launch(lib):
     assert rc("fp8_row_quant", FAKE, 4, 72, 32, FAKE, FAKE, None, None) == 2
     assert rc("fp8_row_quant", FAKE, 4, 96, 64, FAKE, FAKE, FAKE, None) == 3
     # gemv: M range, mode, out flag
-    assert rc("w4a16_gemv", FAKE, 17, FAKE, 16, 128, 128, 1, FAKE, 0, None) == 2
-    assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 3, FAKE, 0, None) == 5
-    assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 2, None) == 5
+    assert rc("w4a16_gemv", FAKE, 17, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE, 1 << 20, None) == 2
+    assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 3, FAKE, 0, FAKE, 1 << 20, None) == 5
+    assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 4, FAKE, 1 << 20, None) == 5
+    assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE + 8, 1 << 20, None) == 4
     # gemm: group sums are required, K >= 128
     assert rc("w4a8_gemm", FAKE, FAKE, None, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None) == 1
     assert rc("w4a8_gemm", FAKE, FAKE, FAKE, 4, FAKE, 16, 96, 32, 1, FAKE, 0, None) == 2

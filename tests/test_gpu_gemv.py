@@ -40,7 +40,8 @@ def gpu_gemv(codes, scales, zeros, N, K, group, mode, x_bits, out_fp32):
     w4.w4_prepack(c, s, z, N, K, group, mode, w4.W4_LAYOUT_GEMV, packed)
     x = to_dev(x_bits.view(np.int16)).view(torch.bfloat16)
     y = torch.empty(M, N, dtype=torch.float32 if out_fp32 else torch.bfloat16, device=cuda())
-    w4.w4a16_gemv(x, M, packed, N, K, group, mode, y, out_fp32)
+    ws = w4.alloc_gemv_workspace(N, K, group)
+    w4.w4a16_gemv(x, M, packed, N, K, group, mode, y, out_fp32, ws)
     torch.cuda.synchronize()
     return y.float().cpu().numpy().astype(np.float64)
 
@@ -113,3 +114,39 @@ def test_one_hot_column():
     y = gpu_gemv(codes, scales, zeros, 64, 256, 128, "asym", xb, 1)
     Wd = oracle.dequantize(codes, scales, zeros, 128, "asym")
     assert np.array_equal(y[0], Wd[:, 131])
+
+
+def test_overlapped_chain_reads_predecessor_output():
+    """Three K x K GEMVs back to back with W4_OVERLAP_PREVIOUS, each consuming the previous
+    one's bf16 output: the overlapped kernel must read its activations only after its
+    predecessor finished. Compared with the oracle's own chain (bf16 between layers)."""
+    K, g = 2048, 128
+    layers = [quantized("t3", K, K, g, "asym", "twenty") if i == 0 else None for i in range(1)]
+    qs = []
+    for i in range(3):
+        W = synth.student_t3_weight(K, K, 9, 950 + i)
+        qs.append(oracle.quantize(synth.bf16_bits(W), g, "asym", [1.0], want_chosen=False)[:3])
+    x0 = synth.normal((1, K), 1.0, 9, 999)
+    # oracle chain
+    xb = synth.bf16_bits(x0)
+    for codes, scales, zeros in qs:
+        y = oracle.gemv_ref(xb, codes, scales, zeros, g, "asym")
+        xb = synth.bf16_bits(torch.from_numpy(y).to(torch.float32).to(torch.bfloat16))
+    ref = y
+    # GPU chain, one workspace shared by the three calls
+    ws = w4.alloc_gemv_workspace(K, K, g)
+    packs = []
+    for codes, scales, zeros in qs:
+        p = w4.alloc_packed(K, K, g, w4.W4_LAYOUT_GEMV)
+        w4.w4_prepack(to_dev(codes), to_dev(scales.view(np.int16)), to_dev(zeros), K, K, g, "asym",
+                      w4.W4_LAYOUT_GEMV, p)
+        packs.append(p)
+    bufs = [x0.to(cuda())] + [torch.empty(1, K, dtype=torch.bfloat16, device=cuda()) for _ in range(3)]
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for i, p in enumerate(packs):
+            w4.w4a16_gemv(bufs[i], 1, p, K, K, g, "asym", bufs[i + 1], w4.W4_OVERLAP_PREVIOUS, ws)
+        torch.cuda.synchronize()
+        got = bufs[3].float().cpu().numpy().astype(np.float64)
+        assert rel_frob(bf16_round(ref), got) <= 2e-3
+    assert w4.w4_device_status() == 0
