@@ -40,6 +40,7 @@ W4_API const char *w4_status_str(int status) {
         case W4_ERR_TIMEOUT: return "device wait timed out";
         case W4_ERR_DEVICE_CHECK: return "device check failed";
         case W4_ERR_WORKSPACE: return "workspace missing or too small";
+        case W4_ERR_SCRATCH_LIMIT: return "request exceeds the fixed scratch of the allocation-free entry point";
         default: return "unknown status";
     }
 }

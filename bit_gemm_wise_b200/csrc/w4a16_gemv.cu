@@ -31,6 +31,8 @@
 #include "w4_common.cuh"
 #include "w4_layout.cuh"
 
+#include <mutex>
+
 namespace w4 {
 namespace gemv {
 
@@ -449,4 +451,75 @@ W4_API w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, i
     if (M <= 4) return gemv::run<4>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
     if (M <= 8) return gemv::run<8>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
     return gemv::run<16>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
+}
+
+// ------------------------------------------------------------------ allocation-free variant
+//
+// Callers that must not allocate device memory on the hot path -- a plug-in running inside
+// another runtime that owns all device memory, or a latency-critical decode loop where
+// cudaMalloc's implicit device synchronisation is not acceptable -- can call
+// w4a16_gemv_noalloc. Its scratch (the partial sums and arrival counters of the stream-K
+// fixup) is a fixed array in this library's device memory, reserved when the library loads
+// on a GPU and held until the process exits.
+
+namespace w4 {
+namespace gemv {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mu;
+static void *g_noalloc_ptr[64];
+
+// Device address of the scratch array on the current device. Host code must not use the
+// symbol itself (that is a host-side stand-in, not a device address); the address is looked
+// up once per device, with that device current.
+static void *noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+template <int MT>
+static w4_status run_noalloc(const void *x, int64_t M, const void *packed, int64_t N, int64_t K, int g, void *y,
+                             int out_fp32, int pdl, cudaStream_t stream) {
+    Plan p;
+    if (!make_plan<MT>(p, M, N, K, g)) return W4_ERR_SHAPE;
+    const GemvLayout L = gemv_layout(N, K, g);
+    const size_t part = (size_t)p.P * 2 * 8 * MT * 4;
+    const size_t need = part + (size_t)L.N8 * 4;
+    if (need > kNoAllocScratchBytes) return W4_ERR_SCRATCH_LIMIT;
+    uint8_t *ws = static_cast<uint8_t *>(noalloc_scratch());
+    if (!ws) return W4_ERR_CUDA;
+    // the arrival counters must start at zero; a call normally leaves them at zero, but the
+    // array outlives every call, so clear them on the caller's stream first
+    if (cudaMemsetAsync(ws + part, 0, (size_t)L.N8 * 4, stream) != cudaSuccess) return W4_ERR_CUDA;
+    return run<MT>(x, M, packed, N, K, g, y, out_fp32, ws, kNoAllocScratchBytes, pdl, stream);
+}
+
+}  // namespace gemv
+}  // namespace w4
+
+W4_API size_t w4a16_gemv_noalloc_scratch_limit(void) { return w4::gemv::kNoAllocScratchBytes; }
+
+W4_API w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
+                                    int group, int mode, void *y, int flags, cudaStream_t stream) {
+    if (!x_bf16 || !packed || !y) return W4_ERR_NULL;
+    if (!valid_mode(mode) || (flags & ~(W4_OUT_FP32 | W4_OVERLAP_PREVIOUS))) return W4_ERR_ARG;
+    if (M < 1 || M > 16 || N < 1 || N > (int64_t)0x7fffffff * 8 || K < 32 || K % 32 != 0) return W4_ERR_SHAPE;
+    if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
+    if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(y)) return W4_ERR_ALIGN;
+    const int out_fp32 = (flags & W4_OUT_FP32) ? 1 : 0;
+    const int pdl = (flags & W4_OVERLAP_PREVIOUS) ? 1 : 0;
+    if (M <= 1) return gemv::run_noalloc<1>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
+    if (M <= 2) return gemv::run_noalloc<2>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
+    if (M <= 4) return gemv::run_noalloc<4>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
+    if (M <= 8) return gemv::run_noalloc<8>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
+    return gemv::run_noalloc<16>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
 }

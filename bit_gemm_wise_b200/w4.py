@@ -22,7 +22,7 @@ W4_OUT_FP32, W4_OVERLAP_PREVIOUS = 1, 2  # flags of w4a16_gemv
 STATUS = {
     0: "W4_OK", 1: "W4_ERR_NULL", 2: "W4_ERR_SHAPE", 3: "W4_ERR_GROUP", 4: "W4_ERR_ALIGN",
     5: "W4_ERR_ARG", 6: "W4_ERR_UNSUPPORTED", 7: "W4_ERR_CUDA", 8: "W4_ERR_TIMEOUT",
-    9: "W4_ERR_DEVICE_CHECK", 10: "W4_ERR_WORKSPACE",
+    9: "W4_ERR_DEVICE_CHECK", 10: "W4_ERR_WORKSPACE", 11: "W4_ERR_SCRATCH_LIMIT",
 }
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4.so")
@@ -38,6 +38,8 @@ SIGNATURES = [
     ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P]),
     ("w4a16_gemv_workspace_bytes", _SZ, [_I64, _I64, _I]),
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
+    ("w4a16_gemv_noalloc_scratch_limit", _SZ, []),
+    ("w4a16_gemv_noalloc", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
     ("w4a8_gemm", _I, [_P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
     ("w4a8_grouped_gemm", _I, [_P, _P, _P, _P, _I, _I64, _P, _I64, _I64, _I, _I, _P, _P]),
     ("w4_device_status", _I, [_P, ctypes.POINTER(ctypes.c_int)]),
@@ -141,6 +143,17 @@ def w4a16_gemv(x, M, packed, N, K, group, mode, y, flags, workspace, stream=None
                           _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _check("w4a16_gemv", rc)
+
+
+def w4a16_gemv_noalloc_scratch_limit() -> int:
+    return int(lib().w4a16_gemv_noalloc_scratch_limit())
+
+
+def w4a16_gemv_noalloc(x, M, packed, N, K, group, mode, y, flags, stream=None):
+    """w4a16_gemv with the library's fixed scratch array instead of a caller workspace."""
+    rc = lib().w4a16_gemv_noalloc(_ptr(x), M, _ptr(packed), N, K, group, _mode(mode), _ptr(y), int(flags),
+                                  _stream(stream))
+    _check("w4a16_gemv_noalloc", rc)
 
 
 def w4a8_gemm(X8, row_scale, group_sums, M, packed, N, K, group, mode, Y, out_fp32=0, stream=None):

@@ -51,7 +51,9 @@ typedef enum {
     W4_ERR_CUDA = 7,         /* a CUDA runtime call failed (launch error)              */
     W4_ERR_TIMEOUT = 8,      /* device status: a bounded wait in a kernel expired      */
     W4_ERR_DEVICE_CHECK = 9, /* device status: a kernel's own consistency check failed */
-    W4_ERR_WORKSPACE = 10    /* workspace missing or smaller than the query says       */
+    W4_ERR_WORKSPACE = 10,   /* workspace missing or smaller than the query says       */
+    W4_ERR_SCRATCH_LIMIT = 11 /* request needs more scratch than the allocation-free
+                                entry point holds (w4a16_gemv_noalloc_scratch_limit)  */
 } w4_status;
 
 typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
@@ -164,6 +166,34 @@ size_t w4a16_gemv_workspace_bytes(int64_t N, int64_t K, int group);
 w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
                      int group, int mode, void *y, int flags, void *workspace,
                      size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * w4a16_gemv_noalloc -- w4a16_gemv for callers that cannot allocate device memory.
+ *   (No counterpart in the source pages: this is a calling convention, not part of the
+ *   method.) Some callers must not call cudaMalloc on their hot path: a plug-in running
+ *   inside another runtime that owns all device memory, or a latency-critical decode loop
+ *   in which cudaMalloc's implicit device synchronisation is not acceptable. This entry
+ *   point computes exactly what w4a16_gemv computes (same kernel, same partition, same
+ *   result bits) but keeps its scratch in a fixed array of w4a16_gemv_noalloc_scratch_limit()
+ *   bytes (1 MiB) inside the library's device memory; every GPU that loads the library
+ *   holds that array until the process exits. The caller still passes x, packed and y.
+ *   Behaviour:
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on a device looks up the array's device address; make that first call
+ *     before any stream capture on that device.
+ *   - Each call clears the arrival counters it needs (cudaMemsetAsync on `stream`) before its
+ *     kernel, because the array keeps the previous call's contents.
+ *   - All calls share the one array: calls that may overlap on the GPU (different streams,
+ *     or W4_OVERLAP_PREVIOUS after another noalloc call still running) race on it and give
+ *     wrong results. Serialise them, or use w4a16_gemv with separate workspaces.
+ *   - A request whose scratch would exceed the limit (N above about 1.7 million rows) returns
+ *     W4_ERR_SCRATCH_LIMIT without launching anything.
+ *   Arguments and other errors as w4a16_gemv.
+ */
+size_t w4a16_gemv_noalloc_scratch_limit(void);
+w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, int64_t N,
+                             int64_t K, int group, int mode, void *y, int flags,
+                             cudaStream_t stream);
 
 /*
  * w4a8_gemm -- W4A8 GEMM on the FP8 tensor cores (TAHOMA "Achievement 2", the list under
