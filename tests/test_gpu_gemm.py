@@ -216,3 +216,22 @@ def test_extreme_zero_points():
     ref = oracle.w4a8_ref_dense(X8, s_a, codes, scales, zeros, g, "asym")
     packed = upload_weight(codes, scales, zeros, N, K, g, "asym")
     check_errors(ref, gpu_gemm(X8, s_a, G, packed, N, K, g, "asym", 1), gpu_gemm(X8, s_a, G, packed, N, K, g, "asym", 0))
+
+
+def test_persistent_tiles_with_long_zero_point_tail():
+    """More tiles than SMs, each with K = 11520 (90 groups -> 5 zero-point pseudo-stages, more
+    than the 4-slot ring): every pipeline role must stay in lockstep with the ring across
+    tiles. 32 sampled token rows against every output column."""
+    M, N, K, g = 256, 20480, 11520, 128
+    W = synth.normal((N, K), 0.02, 2, 31)
+    codes, scales, zeros, _ = oracle.quantize(synth.bf16_bits(W), g, "asym", [1.0], want_chosen=False)
+    X = synth.outlier_activation(M, K, 8, 20.0, 2, 32)
+    X8, s_a, G = oracle.row_quant(synth.bf16_bits(X), g)
+    packed = upload_weight(codes, scales, zeros, N, K, g, "asym")
+    y32 = gpu_gemm(X8, s_a, G, packed, N, K, g, "asym", 1)
+    y16 = gpu_gemm(X8, s_a, G, packed, N, K, g, "asym", 0)
+    rows = np.linspace(0, M - 1, 32).astype(int)
+    Wd = oracle.dequantize(codes, scales, zeros, g, "asym")
+    A = oracle.e4m3_decode(X8[rows]).astype(np.float64) * s_a[rows, None].astype(np.float64)
+    check_errors(A @ Wd.T, y32[rows], y16[rows])
+    assert w4.w4_device_status() == 0
