@@ -277,14 +277,18 @@ def run_ours(args, rank, world, dev):
     return out
 
 
+ROW_GROUPS = ("gemv", "prefill", "moe", "quantize")
+
+
 def measure_rows(args, dev, pk):
     """Every other row of the path, each timed with CUDA events (after warm-up)."""
     from bit_gemm_wise_b200 import synth, w4
     rows = {}
     fp8_peak = 2.0 * pk["bf16"]  # dense FP8 = 2x dense BF16 (nominal ratio), burst
+    want = set(args.rows.split(",")) if args.rows else set(ROW_GROUPS)
 
     # GEMV at M = 4 and 16 (ALU-bound on the CUDA cores)
-    for M in (4, 16):
+    for M in ((4, 16) if "gemv" in want else ()):
         d = Decode(M, args.seed, dev)
         d.capture()
         d.step(0)
@@ -295,7 +299,7 @@ def measure_rows(args, dev, pk):
         del d
 
     # W4A8 prefill GEMM (M=4096) and the FP8 row quant feeding it
-    for K, N in synth.PREFILL_SHAPES:
+    for K, N in (synth.PREFILL_SHAPES if "prefill" in want else ()):
         M = synth.PREFILL_M
         W = synth.prefill_weight(K, N, args.seed, device=dev)
         codes, scales, zeros, _ = w4.alloc_quantized(N, K, 128, "asym", device=dev, chosen=False)
@@ -342,6 +346,15 @@ def measure_rows(args, dev, pk):
         torch.cuda.empty_cache()
 
     # MoE grouped GEMM (32 experts, top-4 of 4096 tokens, group 32)
+    if "moe" in want:
+        moe_rows(args, dev, fp8_peak, rows)
+    if "quantize" in want:
+        rows["w4_quantize_8b_set"] = quantizer_full_set(args, dev)
+    return rows
+
+
+def moe_rows(args, dev, fp8_peak, rows):
+    from bit_gemm_wise_b200 import synth, w4
     c = synth.MOE
     r = synth.moe_routing(args.seed)
     off = r.expert_row_offsets.to(dev)
@@ -377,10 +390,6 @@ def measure_rows(args, dev, pk):
         del packed, Y
     del Xm, X8, sa, G
     torch.cuda.empty_cache()
-
-    # quantizer throughput on the full 8B weight set (20 ratios, asym g128)
-    rows["w4_quantize_8b_set"] = quantizer_full_set(args, dev)
-    return rows
 
 
 def quantizer_full_set(args, dev):
@@ -482,6 +491,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--rows", default="", help="comma-separated subset of " + ",".join(ROW_GROUPS))
+    ap.add_argument("--rows-only", action="store_true", help="skip the headline; measure --rows only")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--quant-layers", type=int, default=32)
@@ -504,7 +515,10 @@ def main():
     try:
         from bit_gemm_wise_b200 import w4
         w4.lib()
-        out = run_ours(args, rank, world, dev)
+        if args.rows_only:
+            out = {"rows": measure_rows(args, dev, peaks())}
+        else:
+            out = run_ours(args, rank, world, dev)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -46,10 +46,12 @@ inline GemvLayout gemv_layout(int64_t N, int64_t K, int g) {
 //           (w >> 4) & 0x0F0F0F0F the bytes of k0+4..k0+7.
 //   scales: [Kpad/g][Npad] u32 (group-major: one group's scales for consecutive rows are
 //           contiguous), lo 16 bits fp16 scale, hi 16 bits zero (8 for symmetric).
+//   flags:  one byte per 128-row tile, 1 if some zero point of the tile lies outside
+//           [0, 15] (such tiles need the zero-point correction term), padded to 16 bytes.
 struct GemmLayout {
     int64_t N, K, Npad, Kpad, J;
     int g;
-    size_t codes_bytes, scales_bytes, total;
+    size_t codes_bytes, scales_bytes, flags_bytes, total;
 };
 
 inline GemmLayout gemm_layout(int64_t N, int64_t K, int g) {
@@ -60,7 +62,8 @@ inline GemmLayout gemm_layout(int64_t N, int64_t K, int g) {
     L.J = L.Kpad / g;
     L.codes_bytes = (size_t)L.Npad * (size_t)L.Kpad / 2;
     L.scales_bytes = (size_t)L.J * (size_t)L.Npad * 4;
-    L.total = L.codes_bytes + L.scales_bytes;
+    L.flags_bytes = (size_t)((L.Npad / 128 + 15) / 16 * 16);
+    L.total = L.codes_bytes + L.scales_bytes + L.flags_bytes;
     return L;
 }
 

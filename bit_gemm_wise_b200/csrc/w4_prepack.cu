@@ -75,6 +75,23 @@ __global__ void prepack_gemm_scales(const uint16_t *__restrict__ scales, const i
         out[idx] = scale_entry(scales, zeros, N, J, idx % Npad, idx / Npad);
 }
 
+// one thread per 128-row tile: flag tiles with a zero point outside [0, 15]
+__global__ void prepack_gemm_flags(const int16_t *__restrict__ zeros, int64_t N, int64_t K, int g, int64_t ntiles,
+                                   uint8_t *__restrict__ out, int64_t nbytes) {
+    const int64_t J = K / g;
+    for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < nbytes; t += (int64_t)gridDim.x * blockDim.x) {
+        uint8_t f = 0;
+        if (zeros && t < ntiles) {
+            for (int64_t n = t * 128; n < (t + 1) * 128 && n < N && !f; ++n)
+                for (int64_t j = 0; j < J; ++j) {
+                    const int z = zeros[n * J + j];
+                    if (z < 0 || z > 15) { f = 1; break; }
+                }
+        }
+        out[t] = f;
+    }
+}
+
 static int grid_for(int64_t n) {
     const int64_t b = (n + 255) / 256;
     const int64_t cap = (int64_t)num_sms() * 32;
@@ -120,6 +137,8 @@ W4_API w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, c
                                                                  reinterpret_cast<uint32_t *>(base));
         prepack_gemm_scales<<<grid_for(nent), 256, 0, stream>>>(scales_fp16, zeros, N, K, group, L.Npad, nent,
                                                                 reinterpret_cast<uint32_t *>(base + L.codes_bytes));
+        prepack_gemm_flags<<<grid_for((int64_t)L.flags_bytes), 256, 0, stream>>>(
+            zeros, N, K, group, L.Npad / 128, base + L.codes_bytes + L.scales_bytes, (int64_t)L.flags_bytes);
     }
     return launch_status();
 }

@@ -49,7 +49,8 @@ constexpr int THREADS = 512;
 constexpr int ZK = 64;        // bf16 elements of the zero-point product per pseudo-stage
 constexpr uint32_t C_BYTES = BM * BK / 2;   // packed codes of a stage
 constexpr uint32_t B_BYTES = BN * BK;       // activations of a stage
-constexpr uint32_t RAW_BYTES = C_BYTES + B_BYTES;
+constexpr uint32_t S_BYTES = BM * 4 * 4;    // scale/zero entries of a stage (up to 4 groups)
+constexpr uint32_t RAW_BYTES = C_BYTES + B_BYTES + S_BYTES;
 constexpr uint32_t A_BYTES = BM * BK;       // expanded weights
 constexpr uint32_t SMEM_BYTES = STAGES * RAW_BYTES + EXP * A_BYTES + 4096 /*control*/ + 1024 /*alignment*/;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
@@ -76,6 +77,7 @@ struct Args {
     int *status;
     int64_t M, N, Npad, K, Kpad;
     int E, g, Jr, out_fp32;
+    size_t flags_off;              // per-tile zero-point flags, from the start of a slab
     int NT;                        // weight tiles (Npad / BM)
     int MTU;                       // token tiles (upper bound for grouped problems)
     int KT;                        // raw stages per tile
@@ -152,6 +154,7 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
 __device__ __forceinline__ uint32_t bf16_bits_rn(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 
 struct Tile {
+    int zflag;      // the weight tile has zero points outside [0, 15]
     int e;          // expert
     int64_t row0;   // first token row
     int64_t rows;   // token rows that belong to this tile's problem (may exceed BN)
@@ -162,11 +165,13 @@ struct Tile {
 // the same time share a token tile and walk one expert's weight; false if t names no tile.
 __device__ __forceinline__ bool locate_tile(const Args &a, int64_t t, Tile &T) {
     const int64_t mt = t / a.NT;
-    T.n0 = (t - mt * a.NT) * BM;
+    const int64_t nt = t - mt * a.NT;
+    T.n0 = nt * BM;
     if (!a.offsets) {
         T.e = 0;
         T.row0 = mt * BN;
         T.rows = a.M - T.row0;
+        T.zflag = a.packed[a.flags_off + nt];
         return T.row0 < a.M;
     }
     int64_t cum = 0;
@@ -177,6 +182,7 @@ __device__ __forceinline__ bool locate_tile(const Args &a, int64_t t, Tile &T) {
             T.e = x;
             T.row0 = lo + (mt - cum) * BN;
             T.rows = hi - T.row0;
+            T.zflag = a.packed[(size_t)x * a.slab_bytes + a.flags_off + nt];
             return true;
         }
         cum += tiles;
@@ -184,8 +190,24 @@ __device__ __forceinline__ bool locate_tile(const Args &a, int64_t t, Tile &T) {
     return false;
 }
 
+// The nibble bytes Q (four codes 0..15, one per byte) minus the zero point zc (0..15) as
+// sign-magnitude E4M3 subnormal bytes, value (q - zc) * 2^-9, exact for every pair.
+// C1 = 0x80808080 - zc * 0x01010101 makes each byte 0x80 + q - zc without inter-byte
+// borrows; bit 7 of that byte says q >= zc, where the magnitude is its low 7 bits, otherwise
+// the byte is 0x100 - it = 0x80 | (zc - q). prmt with the sign-replicate selector turns bit 7
+// of every byte into a byte mask.
+__device__ __forceinline__ uint32_t minus_zero_e4m3(uint32_t Q, uint32_t C1) {
+    const uint32_t D1 = Q + C1;
+    uint32_t P;
+    asm("prmt.b32 %0, %1, %1, 0xBA98;" : "=r"(P) : "r"(D1));
+    P &= 0x7F7F7F7Fu;
+    const uint32_t X = 0x01010100u - D1;
+    return (D1 & P) | (X & ~P);
+}
+
 __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant__ CUtensorMap tm_codes,
-                                                          const __grid_constant__ CUtensorMap tm_act, const Args a) {
+                                                          const __grid_constant__ CUtensorMap tm_act,
+                                                          const __grid_constant__ CUtensorMap tm_sc, const Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *raw = base;                                   // STAGES x (codes | activations)
@@ -194,7 +216,6 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t total_tiles = (int64_t)a.MTU * a.NT;
-    const int SPT = a.KT + a.ZT;  // pipeline stages per tile
     const int GPS = BK / a.g;      // groups per raw stage
     const int KPG = a.g / 32;      // f8 MMAs (K = 32 each) per group
     const int J = (int)(a.Kpad / a.g);
@@ -235,6 +256,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 Tile T;
                 if (!locate_tile(a, t, T)) continue;
+                const int SPT = a.KT + (T.zflag ? a.ZT : 0);  // pipeline stages of this tile
                 for (int s = 0; s < SPT; ++s, ++it) {
                     const int slot = (int)(it % STAGES);
                     // wait for the slot's previous use on every use, including the zero-point
@@ -243,9 +265,10 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                     if (!wait_phase(&sm->empty[slot], ((uint32_t)(it / STAGES) & 1) ^ 1, sm, a.status)) { ok = false; break; }
                     if (s >= a.KT) continue;
                     uint8_t *dst = raw + slot * RAW_BYTES;
-                    mbar_arrive_expect_tx(&sm->full[slot], RAW_BYTES);
+                    mbar_arrive_expect_tx(&sm->full[slot], C_BYTES + B_BYTES + (uint32_t)GPS * BM * 4);
                     tma_load_3d(dst, &tm_codes, s * (BK / 2), (int)T.n0, T.e, &sm->full[slot]);
                     tma_load_2d(dst + C_BYTES, &tm_act, s * BK, (int)T.row0, &sm->full[slot]);
+                    tma_load_3d(dst + C_BYTES + B_BYTES, &tm_sc, (int)T.n0, s * GPS, T.e, &sm->full[slot]);
                 }
             }
             // tail: every stage released, so no commit-arrive lands after this CTA exits
@@ -258,6 +281,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 Tile T;
                 if (!locate_tile(a, t, T)) continue;
+                const int SPT = a.KT + (T.zflag ? a.ZT : 0);
                 for (int s = 0; s < SPT && ok; ++s, ++it) {
                     const int slot = (int)(it % STAGES), eb = (int)(it % EXP);
                     if (s < a.KT) {
@@ -325,14 +349,15 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             float acc[128];
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-            uint32_t ent = scales[n];
-            for (int j = 0; j <= J && ok; ++j, ++jg) {
+            const int JG = J + (T.zflag ? 1 : 0);  // groups, plus the zero-point term if any
+            uint32_t ent0 = scales[n], ent1 = (J > 1) ? scales[a.Npad + n] : 0u;
+            for (int j = 0; j < JG && ok; ++j, ++jg) {
                 const int b = (int)(jg % NBUF);
-                float s512 = -1.0f;  // the zero-point "group" is subtracted
-                uint32_t ent_next = 0;
+                float s512 = -1.0f;  // the zero-point term is subtracted
                 if (j < J) {
-                    s512 = __half2float(__ushort_as_half((unsigned short)(ent & 0xFFFF))) * 512.0f;
-                    ent_next = (j + 1 < J) ? scales[(int64_t)(j + 1) * a.Npad + n] : 0u;
+                    s512 = __half2float(__ushort_as_half((unsigned short)(ent0 & 0xFFFF))) * 512.0f;
+                    ent0 = ent1;
+                    ent1 = (j + 2 < J) ? scales[(int64_t)(j + 2) * a.Npad + n] : 0u;
                 }
                 if (!wait_phase(&sm->acc_full[b], (uint32_t)(jg / NBUF) & 1, sm, a.status)) { ok = false; break; }
                 tc_fence_after();
@@ -347,7 +372,6 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                 }
                 tc_fence_before();
                 mbar_arrive(&sm->acc_empty[b]);
-                ent = ent_next;
             }
             if (!ok) break;
             if (n < a.N) {
@@ -376,6 +400,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             if (!locate_tile(a, t, T)) continue;
             const uint32_t *scales =
                 reinterpret_cast<const uint32_t *>(a.packed + (size_t)T.e * a.slab_bytes + a.codes_bytes);
+            const int SPT = a.KT + (T.zflag ? a.ZT : 0);
             for (int s = 0; s < SPT; ++s, ++it) {
                 const int slot = (int)(it % STAGES), eb = (int)(it % EXP);
                 if (!wait_phase(&sm->exp_empty[eb], ((uint32_t)(it / EXP) & 1) ^ 1, sm, a.status)) { ok = false; break; }
@@ -383,16 +408,22 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                 if (s < a.KT) {
                     if (!wait_phase(&sm->full[slot], (uint32_t)(it / STAGES) & 1, sm, a.status)) { ok = false; break; }
                     const uint8_t *src = raw + slot * RAW_BYTES;
+                    const uint32_t *ssc = reinterpret_cast<const uint32_t *>(src + C_BYTES + B_BYTES);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int idx = et + 128 * i;  // 0..511
                         const int r = idx >> 2, p = idx & 3;
                         const uint4 w = *reinterpret_cast<const uint4 *>(src + r * 64 + p * 16);
+                        // zero point of (row r, the group of this 32-wide part), clamped to [0, 15];
+                        // the remainder z - zc of flagged tiles goes through the correction term
+                        const int z = (int)(int16_t)(ssc[((p * 32) / a.g) * BM + r] >> 16);
+                        const uint32_t zc = (uint32_t)min(max(z, 0), 15);
+                        const uint32_t C1 = 0x80808080u - zc * 0x01010101u;
                         uint4 o0, o1;
-                        o0.x = w.x & 0x0F0F0F0Fu; o0.y = (w.x >> 4) & 0x0F0F0F0Fu;
-                        o0.z = w.y & 0x0F0F0F0Fu; o0.w = (w.y >> 4) & 0x0F0F0F0Fu;
-                        o1.x = w.z & 0x0F0F0F0Fu; o1.y = (w.z >> 4) & 0x0F0F0F0Fu;
-                        o1.z = w.w & 0x0F0F0F0Fu; o1.w = (w.w >> 4) & 0x0F0F0F0Fu;
+                        o0.x = minus_zero_e4m3(w.x & 0x0F0F0F0Fu, C1); o0.y = minus_zero_e4m3((w.x >> 4) & 0x0F0F0F0Fu, C1);
+                        o0.z = minus_zero_e4m3(w.y & 0x0F0F0F0Fu, C1); o0.w = minus_zero_e4m3((w.y >> 4) & 0x0F0F0F0Fu, C1);
+                        o1.x = minus_zero_e4m3(w.z & 0x0F0F0F0Fu, C1); o1.y = minus_zero_e4m3((w.z >> 4) & 0x0F0F0F0Fu, C1);
+                        o1.z = minus_zero_e4m3(w.w & 0x0F0F0F0Fu, C1); o1.w = minus_zero_e4m3((w.w >> 4) & 0x0F0F0F0Fu, C1);
                         const int c0 = (2 * p) ^ (r & 7), c1 = (2 * p + 1) ^ (r & 7);
                         *reinterpret_cast<uint4 *>(dstA + r * 128 + c0 * 16) = o0;
                         *reinterpret_cast<uint4 *>(dstA + r * 128 + c1 * 16) = o1;
@@ -421,7 +452,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                                     if (part < 3) {
                                         const uint32_t en = scales[(int64_t)j * a.Npad + n];
                                         const float sc = __half2float(__ushort_as_half((unsigned short)(en & 0xFFFF)));
-                                        const float sz = sc * (float)(int)(int16_t)(en >> 16);
+                                        const int zz = (int)(int16_t)(en >> 16);
+                                        const float sz = sc * (float)(zz - min(max(zz, 0), 15));
                                         const uint32_t hi = bf16_bits_rn(sz);
                                         v = (part < 2) ? hi : bf16_bits_rn(sz - __uint_as_float(hi << 16));
                                     }
@@ -533,9 +565,22 @@ static w4_status launch(const uint8_t *X8, const float *row_scale, const float *
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4_ERR_CUDA;
     }
+    CUtensorMap tm_sc;
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)L.Npad, (cuuint64_t)L.J, (cuuint64_t)E};
+        const cuuint64_t strides[2] = {(cuuint64_t)(L.Npad * 4), (cuuint64_t)L.total};
+        const cuuint32_t box[3] = {BM, (cuuint32_t)(BK / group), 1};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tm_sc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3,
+                const_cast<uint8_t *>(static_cast<const uint8_t *>(packed) + L.codes_bytes), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+    }
     Args a;
     a.packed = static_cast<const uint8_t *>(packed);
     a.slab_bytes = L.total;
+    a.flags_off = L.codes_bytes + L.scales_bytes;
     a.codes_bytes = L.codes_bytes;
     a.row_scale = row_scale;
     a.gsum = gsum;
@@ -561,7 +606,7 @@ static w4_status launch(const uint8_t *X8, const float *row_scale, const float *
     }
     const int64_t tiles = mtu * a.NT;
     const int grid = (int)(tiles < sm_count_cached() ? tiles : sm_count_cached());
-    w4a8_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_codes, tm_act, a);
+    w4a8_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_codes, tm_act, tm_sc, a);
     return launch_status();
 }
 

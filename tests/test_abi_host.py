@@ -48,7 +48,7 @@ def test_prepack_bytes(lib):
     assert w4.w4_prepack_bytes(4096, 4096, 128, w4.W4_LAYOUT_GEMV) == 4096 * 4096 // 2 + 4096 * 32 * 4
     assert w4.w4_prepack_bytes(1536, 576, 32, w4.W4_LAYOUT_GEMV) == 1536 * 640 // 2 + 1536 * 20 * 4
     # GEMM layout: rows padded to 128
-    assert w4.w4_prepack_bytes(2880, 2880, 32, w4.W4_LAYOUT_GEMM) == 2944 * 2944 // 2 + 92 * 2944 * 4
+    assert w4.w4_prepack_bytes(2880, 2880, 32, w4.W4_LAYOUT_GEMM) == 2944 * 2944 // 2 + 92 * 2944 * 4 + 32
     for bad in [(0, 4096, 128), (16, 100, 32), (16, 4096, 48), (16, 96, 64)]:
         assert w4.w4_prepack_bytes(*bad, w4.W4_LAYOUT_GEMV) == 0
     assert w4.w4_prepack_bytes(16, 4096, 128, 7) == 0
