@@ -307,17 +307,15 @@ def measure_rows(args, dev, pk):
         packed = w4.alloc_packed(N, K, 128, w4.W4_LAYOUT_GEMM, device=dev)
         w4.w4_prepack(codes, scales, zeros, N, K, 128, "asym", w4.W4_LAYOUT_GEMM, packed)
         X = synth.prefill_activation(M, K, args.seed, device=dev)
-        X8 = torch.empty(M, K, dtype=torch.uint8, device=dev)
-        sa = torch.empty(M, dtype=torch.float32, device=dev)
-        G = torch.empty(M, K // 128, dtype=torch.float32, device=dev)
+        X8, sa, _, gop = w4.alloc_row_quant(M, K, 128, device=dev, group_sums=False)
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
         def rq(i):
-            w4.fp8_row_quant(X, M, K, 128, X8, sa, G)
+            w4.fp8_row_quant(X, M, K, 128, X8, sa, None, gop)
 
         def gemm(i):
-            w4.w4a8_gemm(X8, sa, G, M, packed, N, K, 128, "asym", Y, 0)
+            w4.w4a8_gemm(X8, sa, gop, M, packed, N, K, 128, "asym", Y, 0)
 
         rq(0); gemm(0)
         n = 10
@@ -331,7 +329,7 @@ def measure_rows(args, dev, pk):
         t_gemm /= n
         flops = 2.0 * M * N * K
         tf = flops / (t_gemm * 1e-3) / 1e12
-        rq_bytes = M * K * 2 + M * K + M * 4 + M * (K // 128) * 4
+        rq_bytes = M * K * 2 + M * K + M * 4 + gop.numel() * 2
         rows[f"w4a8_gemm_{K}x{N}"] = {
             "value": round(tf, 1), "unit": "TFLOP/s", "us": round(t_gemm * 1e3, 1),
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp8_peak, 1),
@@ -342,7 +340,7 @@ def measure_rows(args, dev, pk):
             "frac_hbm": round(rq_bytes / (t_rq * 1e-3) / 1e9 / pk["hbm"], 4)}
         rows[f"w4a8_rowquant_plus_gemm_{K}x{N}"] = {
             "value": round(flops / ((t_gemm + t_rq) * 1e-3) / 1e12, 1), "unit": "TFLOP/s"}
-        del W, codes, scales, zeros, packed, X, X8, sa, G, Y, flush
+        del W, codes, scales, zeros, packed, X, X8, sa, gop, Y, flush
         torch.cuda.empty_cache()
 
     # MoE grouped GEMM (32 experts, top-4 of 4096 tokens, group 32)
@@ -360,10 +358,8 @@ def moe_rows(args, dev, fp8_peak, rows):
     off = r.expert_row_offsets.to(dev)
     Mt = int(r.expert_row_offsets[-1])
     Xm = synth.moe_activation(args.seed, device=dev)[r.token_of_row.to(dev)].contiguous()
-    X8 = torch.empty(Mt, c["K"], dtype=torch.uint8, device=dev)
-    sa = torch.empty(Mt, dtype=torch.float32, device=dev)
-    G = torch.empty(Mt, c["K"] // 32, dtype=torch.float32, device=dev)
-    w4.fp8_row_quant(Xm, Mt, c["K"], 32, X8, sa, G)
+    X8, sa, _, gop = w4.alloc_row_quant(Mt, c["K"], 32, device=dev, group_sums=False)
+    w4.fp8_row_quant(Xm, Mt, c["K"], 32, X8, sa, None, gop)
     for kind in ("gate_up", "down"):
         N = c["N_gate_up"] if kind == "gate_up" else c["N_down"]
         K = c["K"]
@@ -377,7 +373,7 @@ def moe_rows(args, dev, fp8_peak, rows):
         Y = torch.empty(Mt, N, dtype=torch.bfloat16, device=dev)
 
         def mg(i):
-            w4.w4a8_grouped_gemm(X8, sa, G, off, c["E"], Mt, packed, N, K, 32, "asym", Y)
+            w4.w4a8_grouped_gemm(X8, sa, gop, off, c["E"], Mt, packed, N, K, 32, "asym", Y)
 
         mg(0)
         ms = time_region(mg, 5) / 5
@@ -388,7 +384,7 @@ def moe_rows(args, dev, fp8_peak, rows):
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4)}}
         del packed, Y
-    del Xm, X8, sa, G
+    del Xm, X8, sa, gop
     torch.cuda.empty_cache()
 
 

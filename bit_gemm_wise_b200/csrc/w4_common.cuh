@@ -65,7 +65,22 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps until the
+// phase completes or about 0.5 ms have passed, instead of spinning and taking issue slots
+// from the working warps of its SM sub-partition.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(500000u)
+        : "memory");
+    return ok != 0;
+}
+
+// try_wait without a hint (the hardware's own short time limit), for a single latency-critical
+// thread that should resume as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_short(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
@@ -84,12 +99,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Wait for an mbarrier phase, bounded by wall-clock time. If `abort` (shared, may be null)
 // becomes non-zero the wait gives up at once; if the time runs out it sets *abort, records
 // W4_ERR_TIMEOUT in the device status word and returns false.
+template <bool SHORT = false>
 __device__ __forceinline__ bool mbar_wait_abortable(uint64_t *bar, uint32_t parity, int *abort, int *status,
                                                     uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (SHORT ? mbar_try_wait_short(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (SHORT ? mbar_try_wait_short(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if (abort && *(volatile int *)abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             if (abort) *(volatile int *)abort = 1;

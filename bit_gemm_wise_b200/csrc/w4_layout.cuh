@@ -44,15 +44,21 @@ inline GemvLayout gemv_layout(int64_t N, int64_t K, int g) {
 //           32-bit word (8 consecutive k) the nibble slot p (bits [4p, 4p+4)) holds
 //           q[k0 + p/2 + 4*(p%2)], so that w & 0x0F0F0F0F gives the bytes of k0..k0+3 and
 //           (w >> 4) & 0x0F0F0F0F the bytes of k0+4..k0+7.
-//   scales: [Kpad/g][Npad] u32 (group-major: one group's scales for consecutive rows are
+//   scales: [J = Kpad/g][Npad] u32 (group-major: one group's scales for consecutive rows are
 //           contiguous), lo 16 bits fp16 scale, hi 16 bits zero (8 for symmetric).
-//   flags:  one byte per 128-row tile, 1 if some zero point of the tile lies outside
-//           [0, 15] (such tiles need the zero-point correction term), padded to 16 bytes.
+//   zop:    [Npad][KZ] bf16 with Jr = K/g real groups and KZ = 3 Jr rounded up to 32: the
+//           zero-point operand of the GEMM, a function of the scales and zeros above (kept
+//           here so that the GEMM loads it by TMA). With v = s[n,j] * z[n,j] in fp32,
+//           hi = bf16(v), lo = bf16(v - hi), row n holds
+//           [hi(0..Jr-1) | hi(0..Jr-1) | lo(0..Jr-1) | 0 ...]; padding rows are 0.
 struct GemmLayout {
-    int64_t N, K, Npad, Kpad, J;
+    int64_t N, K, Npad, Kpad, J, Jr, KZ;
     int g;
-    size_t codes_bytes, scales_bytes, flags_bytes, total;
+    size_t codes_bytes, scales_bytes, zop_bytes, total;
 };
+
+// bf16 columns of a zero-point (or group-sum) operand row for Jr groups
+inline int64_t zop_cols(int64_t Jr) { return (3 * Jr + 31) / 32 * 32; }
 
 inline GemmLayout gemm_layout(int64_t N, int64_t K, int g) {
     GemmLayout L;
@@ -60,10 +66,12 @@ inline GemmLayout gemm_layout(int64_t N, int64_t K, int g) {
     L.Npad = (N + 127) / 128 * 128;
     L.Kpad = (K + 127) / 128 * 128;
     L.J = L.Kpad / g;
+    L.Jr = K / g;
+    L.KZ = zop_cols(L.Jr);
     L.codes_bytes = (size_t)L.Npad * (size_t)L.Kpad / 2;
     L.scales_bytes = (size_t)L.J * (size_t)L.Npad * 4;
-    L.flags_bytes = (size_t)((L.Npad / 128 + 15) / 16 * 16);
-    L.total = L.codes_bytes + L.scales_bytes + L.flags_bytes;
+    L.zop_bytes = (size_t)L.Npad * (size_t)L.KZ * 2;
+    L.total = L.codes_bytes + L.scales_bytes + L.zop_bytes;
     return L;
 }
 

@@ -75,20 +75,31 @@ __global__ void prepack_gemm_scales(const uint16_t *__restrict__ scales, const i
         out[idx] = scale_entry(scales, zeros, N, J, idx % Npad, idx / Npad);
 }
 
-// one thread per 128-row tile: flag tiles with a zero point outside [0, 15]
-__global__ void prepack_gemm_flags(const int16_t *__restrict__ zeros, int64_t N, int64_t K, int g, int64_t ntiles,
-                                   uint8_t *__restrict__ out, int64_t nbytes) {
-    const int64_t J = K / g;
-    for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < nbytes; t += (int64_t)gridDim.x * blockDim.x) {
-        uint8_t f = 0;
-        if (zeros && t < ntiles) {
-            for (int64_t n = t * 128; n < (t + 1) * 128 && n < N && !f; ++n)
-                for (int64_t j = 0; j < J; ++j) {
-                    const int z = zeros[n * J + j];
-                    if (z < 0 || z > 15) { f = 1; break; }
-                }
+// bf16 round-to-nearest-even bit pattern of a finite fp32 value
+__device__ __forceinline__ uint32_t bf16_rn_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
+// zero-point operand: one thread per 32-bit word (two bf16 columns) of [Npad][KZ]
+__global__ void prepack_gemm_zop(const uint16_t *__restrict__ scales, const int16_t *__restrict__ zeros, int64_t N,
+                                 int64_t Jr, int64_t KZ, int64_t nwords, uint32_t *__restrict__ out) {
+    const int64_t wpr = KZ / 2;
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nwords;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = idx / wpr;
+        uint32_t word = 0;
+        for (int h = 0; h < 2; ++h) {
+            const int64_t c = (idx % wpr) * 2 + h;
+            const int64_t part = c / Jr, j = c - part * Jr;
+            uint32_t v = 0;
+            if (n < N && part < 3) {
+                const float sc = __half2float(__ushort_as_half(scales[n * Jr + j]));
+                const float z = zeros ? (float)zeros[n * Jr + j] : 8.0f;
+                const float sz = __fmul_rn(sc, z);
+                const uint32_t hi = bf16_rn_bits(sz);
+                v = (part < 2) ? hi : bf16_rn_bits(__fsub_rn(sz, __uint_as_float(hi << 16)));
+            }
+            word |= v << (16 * h);
         }
-        out[t] = f;
+        out[idx] = word;
     }
 }
 
@@ -137,8 +148,9 @@ W4_API w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, c
                                                                  reinterpret_cast<uint32_t *>(base));
         prepack_gemm_scales<<<grid_for(nent), 256, 0, stream>>>(scales_fp16, zeros, N, K, group, L.Npad, nent,
                                                                 reinterpret_cast<uint32_t *>(base + L.codes_bytes));
-        prepack_gemm_flags<<<grid_for((int64_t)L.flags_bytes), 256, 0, stream>>>(
-            zeros, N, K, group, L.Npad / 128, base + L.codes_bytes + L.scales_bytes, (int64_t)L.flags_bytes);
+        const int64_t zwords = (int64_t)(L.zop_bytes / 4);
+        prepack_gemm_zop<<<grid_for(zwords), 256, 0, stream>>>(
+            scales_fp16, zeros, N, L.Jr, L.KZ, zwords, reinterpret_cast<uint32_t *>(base + L.codes_bytes + L.scales_bytes));
     }
     return launch_status();
 }

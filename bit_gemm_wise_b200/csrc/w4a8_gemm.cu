@@ -6,8 +6,9 @@
 // accumulation, per-token activation scale in the epilogue, BF16 result) and
 // "4-bit by default" (mixture-of-experts weights are the 4-bit target).
 //
-//   Y[m, n] = s_a[m] * ( sum_j 512 s[n,j] P_j[m,n]  -  sum_j s[n,j] z[n,j] G[m,j] ),
-//   P_j[m,n] = sum_{k in j} a8[m,k] * (q[n,k] * 2^-9),   G[m,j] = sum_{k in j} a8[m,k]
+//   Y[m, n] = s_a[m] * ( sum_j 512 s[n,j] P_j[m,n]  -  Z[m,n] ),
+//   P_j[m,n] = sum_{k in j} a8[m,k] * (q[n,k] * 2^-9),   Z[m,n] = sum_j s[n,j] z[n,j] G[m,j],
+//   G[m,j] = sum_{k in j} a8[m,k]
 //
 // Design (one persistent CTA per SM, tiles of 128 weight rows x 256 tokens):
 //  * swap-AB: the weight tile is the MMA's A operand (M = 128 weight rows, one TMEM lane per
@@ -15,19 +16,23 @@
 //    group scale is a per-thread scalar;
 //  * expansion: a nibble q in [0, 15] zero-extended to a byte IS the E4M3 pattern of q*2^-9
 //    (exponent field 0/1 spans the integer grid m*2^-9, m = 0..15), so the expanded weights
-//    are exact and the expansion is two AND/shift ops per 8 weights, written straight into
-//    the 128-byte-swizzled K-major layout the MMA reads;
+//    are exact and the expansion is one AND (and one shift) per 4 weights, written straight
+//    into the 128-byte-swizzled K-major layout the MMA reads;
 //  * per group j, kind::f8f6f4 MMAs (K = 32 each) accumulate P_j into one of two TMEM
 //    buffers (2 x 256 columns); 8 promotion warps read it back (tcgen05.ld) and add
-//    512 s[n,j] P_j into fp32 registers while the MMA fills the other buffer;
-//  * the zero-point term is a rank-J product Z = (s z) G^T computed on the tensor cores too:
-//    after a tile's last group the expansion warps write bf16 hi/lo splits of s*z (A) and of
-//    G (B) -- [hi|hi|lo] x [hi|lo|hi] along K, error ~2^-16 relative -- into the same
-//    pipeline buffers, the MMA thread accumulates them with kind::f16 into a TMEM buffer,
-//    and the promotion warps subtract it as one more "group";
+//    512 s[n,j] P_j into fp32 registers (packed f32x2 FMAs) while the MMA fills the other;
+//  * the zero-point term Z is a rank-J product computed on the tensor cores as well: after a
+//    tile's last group, pseudo-stages bring bf16 hi/lo splits of s*z (from the prepacked
+//    weight) and of G (from the row quantizer) by TMA -- [hi|hi|lo] x [hi|lo|hi] along K,
+//    error ~2^-16 relative -- and kind::f16 MMAs accumulate Z into a TMEM buffer that the
+//    promotion warps subtract as one more "group";
 //  * warp roles: warp 0 TMA producer, warp 1 TMEM owner + single-thread MMA issuer, warps
 //    4-11 promotion/epilogue (register budget raised with setmaxnreg), warps 12-15
-//    expansion; rings: 4 raw stages (codes + activations) and 2 expanded-weight buffers;
+//    expansion; one ring of 4 stages, each with raw operands (codes + activations, or the
+//    two zero-point operands) and an expanded-weight buffer: TMA -> full -> expansion ->
+//    exp_full -> MMA -> empty -> TMA. Every stage passes the expansion warps, so each wait
+//    on the ring sees its phases in order, and the MMA thread has one wait and one commit
+//    per stage (plus one of each per accumulator group);
 //  * every mbarrier wait is bounded by wall-clock time; on expiry the kernel records
 //    W4_ERR_TIMEOUT, every role sees the abort flag, TMEM is freed and the CTA returns.
 #include "w4_common.cuh"
@@ -41,43 +46,43 @@ namespace gemm {
 constexpr int BM = 128;       // weight rows per tile (MMA M)
 constexpr int BN = 256;       // tokens per tile (MMA N)
 constexpr int BK = 128;       // k per pipeline stage (one 128-byte swizzle row of E4M3)
-constexpr int STAGES = 4;     // raw stages: packed codes + activations
-constexpr int EXP = 2;        // expanded-weight buffers
+constexpr int STAGES = 4;     // pipeline stages (raw operands + one expanded-weight buffer each)
 constexpr int NBUF = 2;       // TMEM accumulator buffers
 constexpr int TMEM_COLS = NBUF * BN;
 constexpr int THREADS = 512;
-constexpr int ZK = 64;        // bf16 elements of the zero-point product per pseudo-stage
+constexpr int ZKC = 32;       // bf16 columns of the zero-point operands per pseudo-stage (64-byte rows)
 constexpr uint32_t C_BYTES = BM * BK / 2;   // packed codes of a stage
 constexpr uint32_t B_BYTES = BN * BK;       // activations of a stage
-constexpr uint32_t S_BYTES = BM * 4 * 4;    // scale/zero entries of a stage (up to 4 groups)
-constexpr uint32_t RAW_BYTES = C_BYTES + B_BYTES + S_BYTES;
+constexpr uint32_t RAW_BYTES = C_BYTES + B_BYTES;
+constexpr uint32_t ZA_BYTES = BM * ZKC * 2;  // s*z operand of a pseudo-stage (in place of the codes)
+constexpr uint32_t ZB_BYTES = BN * ZKC * 2;  // group-sum operand of a pseudo-stage
 constexpr uint32_t A_BYTES = BM * BK;       // expanded weights
-constexpr uint32_t SMEM_BYTES = STAGES * RAW_BYTES + EXP * A_BYTES + 4096 /*control*/ + 1024 /*alignment*/;
+constexpr uint32_t SMEM_BYTES = STAGES * (RAW_BYTES + A_BYTES) + 1024 /*control*/ + 1024 /*alignment*/;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
+static_assert(ZA_BYTES <= C_BYTES && C_BYTES + ZB_BYTES <= RAW_BYTES, "pseudo-stage operands fit a raw stage");
+static_assert(RAW_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay aligned");
 
 struct Smem {
-    uint64_t full[STAGES];     // raw stage ready (TMA bytes, or a pseudo-stage written by threads)
-    uint64_t empty[STAGES];    // raw stage consumed by the MMA
-    uint64_t exp_full[EXP];    // expanded weights / zero-point A operand ready
-    uint64_t exp_empty[EXP];   // expanded buffer consumed by the MMA
+    uint64_t full[STAGES];     // raw operands landed (TMA bytes); waited by the expansion warps
+    uint64_t exp_full[STAGES]; // expansion warps passed the stage (one arrival per warp); waited by the MMA
+    uint64_t empty[STAGES];    // stage consumed by the MMA: raw and expanded buffers free again
     uint64_t acc_full[NBUF];   // a group's accumulator is complete in TMEM
-    uint64_t acc_empty[NBUF];  // promotion finished reading it
+    uint64_t acc_empty[NBUF];  // promotion finished reading it (one arrival per warp)
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(Smem) <= 1024, "control block");
 
 struct Args {
     const uint8_t *packed;         // slab 0
     size_t slab_bytes;             // bytes per expert slab
     size_t codes_bytes;            // codes part of a slab (scales follow)
     const float *row_scale;        // [M_total]
-    const float *gsum;             // [M_total, Jr]
     const int32_t *offsets;        // [E+1] device, or null: one problem of M rows
     void *Y;                       // [M_total, N]
     int *status;
     int64_t M, N, Npad, K, Kpad;
-    int E, g, Jr, out_fp32;
-    size_t flags_off;              // per-tile zero-point flags, from the start of a slab
+    int E, g, out_fp32;
     int NT;                        // weight tiles (Npad / BM)
     int MTU;                       // token tiles (upper bound for grouped problems)
     int KT;                        // raw stages per tile
@@ -88,29 +93,65 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, Smem 
     return mbar_wait_abortable(bar, parity, &sm->abort, status, kWaitNs);
 }
 
-// K-major operand descriptor, 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes
-// apart (stride byte offset), leading byte offset 16 bytes, descriptor version 1.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+// The wait of a single latency-critical thread (MMA issuer, TMA producer): polls without a
+// suspend hint so that it resumes as soon as the phase completes.
+__device__ __forceinline__ bool wait_phase_short(uint64_t *bar, uint32_t parity, Smem *sm, int *status) {
+    return mbar_wait_abortable<true>(bar, parity, &sm->abort, status, kWaitNs);
 }
+
+// Position in a ring of STAGES slots: slot and the parity of the current use of that slot.
+struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next() {
+        if (++slot == STAGES) { slot = 0; phase ^= 1u; }
+    }
+};
+
+// The same wait taken by a whole warp, with one outcome for all its lanes (the warp then runs
+// warp-collective instructions, which need every lane). Only lane 0 polls, so that twelve
+// waiting warps do not flood the barrier unit that the MMA thread also uses; once lane 0 has
+// seen the phase complete, every lane takes one try_wait of its own for the acquire. That try
+// cannot fail: the barrier's next phase needs this warp's own later arrival (or work that
+// waits for it).
+__device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, Smem *sm, int *status) {
+    bool r = true;
+    if ((threadIdx.x & 31) == 0) r = wait_phase(bar, parity, sm, status);
+    r = __shfl_sync(FULL, r ? 1 : 0, 0) != 0;
+    if (r) r = __all_sync(FULL, mbar_try_wait_short(bar, parity));
+    return r;
+}
+
+// Shared-memory operand descriptors (K-major), kept as two 32-bit words so that the MMA
+// thread only does 32-bit adds: the low word holds the start address in 16-byte units
+// (bits 0-13) and the leading byte offset 16 bytes (bits 16-29, unused by swizzled K-major
+// operands whose K extent fits one swizzle row); the high word holds the stride byte offset
+// between 8-row atoms (bits 32-45), descriptor version 1 (bit 46) and the swizzle mode
+// (bits 61-63: 2 = 128-byte, 4 = 64-byte). Advancing K by 32 bytes adds 2 to the low word.
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr) { return ((saddr & 0x3FFFFu) >> 4) | (1u << 16); }
+constexpr uint32_t kDescHiSW128 = 64u | (1u << 14) | (2u << 29);  // rows of 128 bytes, atoms 1024 bytes apart
+constexpr uint32_t kDescHiSW64 = 32u | (1u << 14) | (4u << 29);   // rows of 64 bytes, atoms 512 bytes apart
 
 // instruction descriptors: D fp32, both operands K-major, N = BN, M = BM;
 // A/B E4M3 (kind::f8f6f4) or BF16 (kind::f16)
 constexpr uint32_t kIdescF8 = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 constexpr uint32_t kIdescBF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-__device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+// D[tmem_d] (+)= A * B for one K step; the descriptors are given as (low word, shared high word)
+__device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint32_t a_lo, uint32_t b_lo, uint32_t accumulate) {
     asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(kIdescF8), "r"(accumulate));
+        "{\n .reg .pred p;\n .reg .b64 da, db;\n setp.ne.b32 p, %4, 0;\n"
+        " mov.b64 da, {%1, %5};\n mov.b64 db, {%2, %5};\n"
+        " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %3, p;\n}\n" ::"r"(tmem_d),
+        "r"(a_lo), "r"(b_lo), "r"(kIdescF8), "r"(accumulate), "r"(kDescHiSW128));
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint32_t a_lo, uint32_t b_lo, uint32_t accumulate) {
     asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(kIdescBF16), "r"(accumulate));
+        "{\n .reg .pred p;\n .reg .b64 da, db;\n setp.ne.b32 p, %4, 0;\n"
+        " mov.b64 da, {%1, %5};\n mov.b64 db, {%2, %5};\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n}\n" ::"r"(tmem_d),
+        "r"(a_lo), "r"(b_lo), "r"(kIdescBF16), "r"(accumulate), "r"(kDescHiSW64));
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -121,18 +162,31 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// 32 lanes x 16 columns of 32-bit accumulator (one column per register)
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Wait for this thread's tcgen05.ld. The registers of the load are in/out operands, so the
+// compiler cannot move a use of them above the wait.
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+// acc[i] += s * (p[2i], p[2i+1]) with the packed fp32 FMA of sm_100 (two lanes per instruction)
+__device__ __forceinline__ void promote16(float2 *acc, float2 s, const uint32_t (&p)[16]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        acc[i] = __ffma2_rn(s, make_float2(__uint_as_float(p[2 * i]), __uint_as_float(p[2 * i + 1])), acc[i]);
+}
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
     asm volatile(
@@ -150,11 +204,7 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// bf16 round-to-nearest-even of an fp32 value, as the 16-bit pattern (finite inputs)
-__device__ __forceinline__ uint32_t bf16_bits_rn(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
-
 struct Tile {
-    int zflag;      // the weight tile has zero points outside [0, 15]
     int e;          // expert
     int64_t row0;   // first token row
     int64_t rows;   // token rows that belong to this tile's problem (may exceed BN)
@@ -171,7 +221,6 @@ __device__ __forceinline__ bool locate_tile(const Args &a, int64_t t, Tile &T) {
         T.e = 0;
         T.row0 = mt * BN;
         T.rows = a.M - T.row0;
-        T.zflag = a.packed[a.flags_off + nt];
         return T.row0 < a.M;
     }
     int64_t cum = 0;
@@ -182,7 +231,6 @@ __device__ __forceinline__ bool locate_tile(const Args &a, int64_t t, Tile &T) {
             T.e = x;
             T.row0 = lo + (mt - cum) * BN;
             T.rows = hi - T.row0;
-            T.zflag = a.packed[(size_t)x * a.slab_bytes + a.flags_off + nt];
             return true;
         }
         cum += tiles;
@@ -190,48 +238,33 @@ __device__ __forceinline__ bool locate_tile(const Args &a, int64_t t, Tile &T) {
     return false;
 }
 
-// The nibble bytes Q (four codes 0..15, one per byte) minus the zero point zc (0..15) as
-// sign-magnitude E4M3 subnormal bytes, value (q - zc) * 2^-9, exact for every pair.
-// C1 = 0x80808080 - zc * 0x01010101 makes each byte 0x80 + q - zc without inter-byte
-// borrows; bit 7 of that byte says q >= zc, where the magnitude is its low 7 bits, otherwise
-// the byte is 0x100 - it = 0x80 | (zc - q). prmt with the sign-replicate selector turns bit 7
-// of every byte into a byte mask.
-__device__ __forceinline__ uint32_t minus_zero_e4m3(uint32_t Q, uint32_t C1) {
-    const uint32_t D1 = Q + C1;
-    uint32_t P;
-    asm("prmt.b32 %0, %1, %1, 0xBA98;" : "=r"(P) : "r"(D1));
-    P &= 0x7F7F7F7Fu;
-    const uint32_t X = 0x01010100u - D1;
-    return (D1 & P) | (X & ~P);
-}
-
+template <int G>  // group size: 32, 64 or 128
 __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                           const __grid_constant__ CUtensorMap tm_act,
-                                                          const __grid_constant__ CUtensorMap tm_sc, const Args a) {
+                                                          const __grid_constant__ CUtensorMap tm_zop,
+                                                          const __grid_constant__ CUtensorMap tm_gop, const Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *raw = base;                                   // STAGES x (codes | activations)
-    uint8_t *sA = base + STAGES * RAW_BYTES;               // EXP x expanded weights
-    Smem *sm = reinterpret_cast<Smem *>(base + STAGES * RAW_BYTES + EXP * A_BYTES);
+    uint8_t *sA = base + STAGES * RAW_BYTES;               // STAGES x expanded weights
+    Smem *sm = reinterpret_cast<Smem *>(base + STAGES * (RAW_BYTES + A_BYTES));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t total_tiles = (int64_t)a.MTU * a.NT;
-    const int GPS = BK / a.g;      // groups per raw stage
-    const int KPG = a.g / 32;      // f8 MMAs (K = 32 each) per group
-    const int J = (int)(a.Kpad / a.g);
+    constexpr int GPS = BK / G;    // groups per raw stage
+    constexpr int KPG = G / 32;    // f8 MMAs (K = 32 each) per group
+    const int J = (int)(a.Kpad / G);
+    const int SPT = a.KT + a.ZT;   // pipeline stages per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm->full[s], 1);
+            mbar_init(&sm->exp_full[s], 4);
             mbar_init(&sm->empty[s], 1);
-        }
-        for (int e = 0; e < EXP; ++e) {
-            mbar_init(&sm->exp_full[e], 128);
-            mbar_init(&sm->exp_empty[e], 1);
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&sm->acc_full[b], 1);
-            mbar_init(&sm->acc_empty[b], 256);
+            mbar_init(&sm->acc_empty[b], 8);
         }
         sm->abort = 0;
         fence_mbar_init();
@@ -251,75 +284,76 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
         asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
         if (warp == 0 && lane == 0) {
             // ------------------------------------------------ TMA producer
-            int64_t it = 0;
+            Ring r;
+            int64_t uses = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 Tile T;
                 if (!locate_tile(a, t, T)) continue;
-                const int SPT = a.KT + (T.zflag ? a.ZT : 0);  // pipeline stages of this tile
-                for (int s = 0; s < SPT; ++s, ++it) {
-                    const int slot = (int)(it % STAGES);
-                    // wait for the slot's previous use on every use, including the zero-point
-                    // pseudo-stages the expansion warps fill: a parity wait can only tell phases
-                    // apart one ring cycle back, so skipping uses would let this thread lap the ring
-                    if (!wait_phase(&sm->empty[slot], ((uint32_t)(it / STAGES) & 1) ^ 1, sm, a.status)) { ok = false; break; }
-                    if (s >= a.KT) continue;
+                for (int s = 0; s < SPT; ++s, r.next(), ++uses) {
+                    const int slot = r.slot;
+                    if (!wait_phase_short(&sm->empty[slot], r.phase ^ 1u, sm, a.status)) { ok = false; break; }
                     uint8_t *dst = raw + slot * RAW_BYTES;
-                    mbar_arrive_expect_tx(&sm->full[slot], C_BYTES + B_BYTES + (uint32_t)GPS * BM * 4);
-                    tma_load_3d(dst, &tm_codes, s * (BK / 2), (int)T.n0, T.e, &sm->full[slot]);
-                    tma_load_2d(dst + C_BYTES, &tm_act, s * BK, (int)T.row0, &sm->full[slot]);
-                    tma_load_3d(dst + C_BYTES + B_BYTES, &tm_sc, (int)T.n0, s * GPS, T.e, &sm->full[slot]);
+                    if (s < a.KT) {
+                        mbar_arrive_expect_tx(&sm->full[slot], C_BYTES + B_BYTES);
+                        tma_load_3d(dst, &tm_codes, s * (BK / 2), (int)T.n0, T.e, &sm->full[slot]);
+                        tma_load_2d(dst + C_BYTES, &tm_act, s * BK, (int)T.row0, &sm->full[slot]);
+                    } else {
+                        const int z = s - a.KT;
+                        mbar_arrive_expect_tx(&sm->full[slot], ZA_BYTES + ZB_BYTES);
+                        tma_load_3d(dst, &tm_zop, z * ZKC, (int)T.n0, T.e, &sm->full[slot]);
+                        tma_load_2d(dst + C_BYTES, &tm_gop, z * ZKC, (int)T.row0, &sm->full[slot]);
+                    }
                 }
             }
-            // tail: every stage released, so no commit-arrive lands after this CTA exits
-            for (int64_t u = it > STAGES ? it - STAGES : 0; u < it && ok; ++u)
+            // tail: wait for the completion of the last STAGES uses (use u: slot u % STAGES,
+            // parity (u / STAGES) & 1), so no commit-arrive lands after this CTA exits
+            for (int64_t u = uses > STAGES ? uses - STAGES : 0; u < uses && ok; ++u)
                 if (!wait_phase(&sm->empty[u % STAGES], (uint32_t)(u / STAGES) & 1, sm, a.status)) break;
         } else if (warp == 1 && lane == 0) {
             // ------------------------------------------------ MMA issuer
-            int64_t it = 0, jg = 0;
+            // One wait per stage (exp_full: the expansion warps have seen the TMA bytes land and
+            // written the expanded weights) and one per accumulator group; one commit per stage
+            // (empty: raw and expanded buffers free) and one per group (acc_full). This thread's
+            // instruction stream sets the pace of the tensor core, so everything between MMAs is
+            // kept to 32-bit arithmetic on precomputed descriptor words.
+            Ring r;
+            uint32_t jg = 0;
             bool ok = true;
+            const uint32_t aLo0 = desc_lo(smem_addr(sA)), rLo0 = desc_lo(smem_addr(raw));
             for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 Tile T;
                 if (!locate_tile(a, t, T)) continue;
-                const int SPT = a.KT + (T.zflag ? a.ZT : 0);
-                for (int s = 0; s < SPT && ok; ++s, ++it) {
-                    const int slot = (int)(it % STAGES), eb = (int)(it % EXP);
-                    if (s < a.KT) {
-                        if (!wait_phase(&sm->full[slot], (uint32_t)(it / STAGES) & 1, sm, a.status)) { ok = false; break; }
-                    } else {
-                        // a pseudo-stage is written by the expansion warps (their exp_full arrival
-                        // covers both operands); complete this use of the raw slot's "full" phase
-                        // here so that its phase count stays one per use
-                        mbar_arrive(&sm->full[slot]);
-                    }
-                    if (!wait_phase(&sm->exp_full[eb], (uint32_t)(it / EXP) & 1, sm, a.status)) { ok = false; break; }
+                for (int s = 0; s < SPT && ok; ++s, r.next()) {
+                    const int slot = r.slot;
+                    if (!wait_phase_short(&sm->exp_full[slot], r.phase, sm, a.status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_addr(sA + eb * A_BYTES);
-                    const uint32_t b_addr = smem_addr(raw + slot * RAW_BYTES + C_BYTES);
+                    const uint32_t rLo = rLo0 + (uint32_t)slot * (RAW_BYTES >> 4);
                     if (s < a.KT) {
+                        const uint32_t aLo = aLo0 + (uint32_t)slot * (A_BYTES >> 4), bLo = rLo + (C_BYTES >> 4);
+#pragma unroll
                         for (int gi = 0; gi < GPS; ++gi, ++jg) {
-                            const int b = (int)(jg % NBUF);
-                            if (!wait_phase(&sm->acc_empty[b], ((uint32_t)(jg / NBUF) & 1) ^ 1, sm, a.status)) { ok = false; break; }
+                            const uint32_t b = jg & 1u;
+                            if (!wait_phase_short(&sm->acc_empty[b], ((jg >> 1) & 1u) ^ 1u, sm, a.status)) { ok = false; break; }
                             tc_fence_after();
-                            for (int kk = 0; kk < KPG; ++kk) {
-                                const uint32_t koff = (uint32_t)(gi * KPG + kk) * 32;
-                                mma_f8(tmem + (uint32_t)(b * BN), sw128_desc(a_addr + koff), sw128_desc(b_addr + koff),
-                                       kk > 0 ? 1u : 0u);
-                            }
+                            const uint32_t d = tmem + b * BN;
+#pragma unroll
+                            for (int kk = 0; kk < KPG; ++kk)
+                                mma_f8(d, aLo + (gi * KPG + kk) * 2, bLo + (gi * KPG + kk) * 2, kk > 0 ? 1u : 0u);
                             mma_commit(&sm->acc_full[b]);
                         }
                     } else {
                         // zero-point term: all pseudo-stages of the tile accumulate into one buffer
                         const int z = s - a.KT;
-                        const int b = (int)(jg % NBUF);
-                        if (z == 0 && !wait_phase(&sm->acc_empty[b], ((uint32_t)(jg / NBUF) & 1) ^ 1, sm, a.status)) {
+                        const uint32_t b = jg & 1u;
+                        if (z == 0 && !wait_phase_short(&sm->acc_empty[b], ((jg >> 1) & 1u) ^ 1u, sm, a.status)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        for (int kk = 0; kk < ZK / 16; ++kk)
-                            mma_bf16(tmem + (uint32_t)(b * BN), sw128_desc(a_addr + kk * 32), sw128_desc(b_addr + kk * 32),
-                                     (z > 0 || kk > 0) ? 1u : 0u);
+                        const uint32_t d = tmem + b * BN, zbLo = rLo + (C_BYTES >> 4);
+                        mma_bf16(d, rLo, zbLo, z > 0 ? 1u : 0u);
+                        mma_bf16(d, rLo + 2, zbLo + 2, 1u);
                         if (z == a.ZT - 1) {
                             mma_commit(&sm->acc_full[b]);
                             ++jg;
@@ -327,7 +361,6 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                     }
                     if (!ok) break;
                     mma_commit(&sm->empty[slot]);
-                    mma_commit(&sm->exp_empty[eb]);
                 }
             }
         }
@@ -346,46 +379,59 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             const int64_t n = T.n0 + row;
             const uint32_t *scales =
                 reinterpret_cast<const uint32_t *>(a.packed + (size_t)T.e * a.slab_bytes + a.codes_bytes);
-            float acc[128];
+            // token scales of this warp's 128 columns, column 32c + l held by lane l; read
+            // now, used (through shuffles) only in the epilogue
+            float rsv[4];
 #pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-            const int JG = J + (T.zflag ? 1 : 0);  // groups, plus the zero-point term if any
+            for (int c = 0; c < 4; ++c) {
+                const int col = half * 128 + c * 32 + lane;
+                const int64_t m = T.row0 + col;
+                rsv[c] = (col < T.rows && m < a.M) ? __ldg(a.row_scale + m) : 0.0f;
+            }
+            float2 acc[64];  // columns (2i, 2i+1) of this thread's weight row
+#pragma unroll
+            for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
             uint32_t ent0 = scales[n], ent1 = (J > 1) ? scales[a.Npad + n] : 0u;
-            for (int j = 0; j < JG && ok; ++j, ++jg) {
+            for (int j = 0; j <= J && ok; ++j, ++jg) {
                 const int b = (int)(jg % NBUF);
-                float s512 = -1.0f;  // the zero-point term is subtracted
+                float s512 = -1.0f;  // group J is the zero-point term, subtracted
                 if (j < J) {
                     s512 = __half2float(__ushort_as_half((unsigned short)(ent0 & 0xFFFF))) * 512.0f;
                     ent0 = ent1;
                     ent1 = (j + 2 < J) ? scales[(int64_t)(j + 2) * a.Npad + n] : 0u;
                 }
-                if (!wait_phase(&sm->acc_full[b], (uint32_t)(jg / NBUF) & 1, sm, a.status)) { ok = false; break; }
+                if (!warp_wait_phase(&sm->acc_full[b], (uint32_t)(jg / NBUF) & 1, sm, a.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN + half * 128);
+                // 8 chunks of 16 columns, double-buffered: the load of chunk c+1 is in flight
+                // while chunk c is promoted
+                const float2 s2 = make_float2(s512, s512);
+                uint32_t pa[16], pb[16];
+                tmem_ld16(taddr, pa);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t p[32];
-                    tmem_ld32(taddr + c * 32, p);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(s512, __uint_as_float(p[i]), acc[c * 32 + i]);
+                for (int c = 0; c < 8; c += 2) {
+                    tmem_wait_ld16(pa);
+                    tmem_ld16(taddr + (c + 1) * 16, pb);
+                    promote16(acc + c * 8, s2, pa);
+                    tmem_wait_ld16(pb);
+                    if (c + 2 < 8) tmem_ld16(taddr + (c + 2) * 16, pa);
+                    promote16(acc + (c + 1) * 8, s2, pb);
                 }
                 tc_fence_before();
-                mbar_arrive(&sm->acc_empty[b]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
             }
             if (!ok) break;
-            if (n < a.N) {
+            const bool row_ok = n < a.N;
 #pragma unroll
-                for (int i = 0; i < 128; ++i) {
-                    const int col = half * 128 + i;
-                    if (col < T.rows) {
-                        const int64_t m = T.row0 + col;
-                        if (m < a.M) {
-                            const float v = acc[i] * __ldg(a.row_scale + m);
-                            if (a.out_fp32) static_cast<float *>(a.Y)[m * a.N + n] = v;
-                            else static_cast<__nv_bfloat16 *>(a.Y)[m * a.N + n] = __float2bfloat16_rn(v);
-                        }
-                    }
+            for (int i = 0; i < 128; ++i) {
+                const float rs = __shfl_sync(FULL, rsv[i >> 5], i & 31);
+                const int col = half * 128 + i;
+                const int64_t m = T.row0 + col;
+                if (row_ok && col < T.rows && m < a.M) {
+                    const float v = ((i & 1) ? acc[i >> 1].y : acc[i >> 1].x) * rs;
+                    if (a.out_fp32) static_cast<float *>(a.Y)[m * a.N + n] = v;
+                    else static_cast<__nv_bfloat16 *>(a.Y)[m * a.N + n] = __float2bfloat16_rn(v);
                 }
             }
         }
@@ -393,112 +439,39 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
         asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
         // ------------------------------------------------ expansion warps
         const int et = threadIdx.x - 384;  // 0..127
-        int64_t it = 0;
+        Ring r;
         bool ok = true;
         for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
             Tile T;
             if (!locate_tile(a, t, T)) continue;
-            const uint32_t *scales =
-                reinterpret_cast<const uint32_t *>(a.packed + (size_t)T.e * a.slab_bytes + a.codes_bytes);
-            const int SPT = a.KT + (T.zflag ? a.ZT : 0);
-            for (int s = 0; s < SPT; ++s, ++it) {
-                const int slot = (int)(it % STAGES), eb = (int)(it % EXP);
-                if (!wait_phase(&sm->exp_empty[eb], ((uint32_t)(it / EXP) & 1) ^ 1, sm, a.status)) { ok = false; break; }
-                uint8_t *dstA = sA + eb * A_BYTES;
+            for (int s = 0; s < SPT; ++s, r.next()) {
+                const int slot = r.slot;
+                // the TMA bytes of this use have landed; the producer issued them only after the
+                // MMA released the slot's previous use, so the expanded buffer is free as well.
+                // Every stage is waited for, pseudo-stages included, so that this role sees each
+                // phase of the ring in order.
+                if (!warp_wait_phase(&sm->full[slot], r.phase, sm, a.status)) { ok = false; break; }
                 if (s < a.KT) {
-                    if (!wait_phase(&sm->full[slot], (uint32_t)(it / STAGES) & 1, sm, a.status)) { ok = false; break; }
                     const uint8_t *src = raw + slot * RAW_BYTES;
-                    const uint32_t *ssc = reinterpret_cast<const uint32_t *>(src + C_BYTES + B_BYTES);
+                    uint8_t *dstA = sA + slot * A_BYTES;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int idx = et + 128 * i;  // 0..511
-                        const int r = idx >> 2, p = idx & 3;
-                        const uint4 w = *reinterpret_cast<const uint4 *>(src + r * 64 + p * 16);
-                        // zero point of (row r, the group of this 32-wide part), clamped to [0, 15];
-                        // the remainder z - zc of flagged tiles goes through the correction term
-                        const int z = (int)(int16_t)(ssc[((p * 32) / a.g) * BM + r] >> 16);
-                        const uint32_t zc = (uint32_t)min(max(z, 0), 15);
-                        const uint32_t C1 = 0x80808080u - zc * 0x01010101u;
+                        const int idx = et + 128 * i;  // 0..511: (row r, 32-wide part p)
+                        const int rr = idx >> 2, p = idx & 3;
+                        const uint4 w = *reinterpret_cast<const uint4 *>(src + rr * 64 + p * 16);
                         uint4 o0, o1;
-                        o0.x = minus_zero_e4m3(w.x & 0x0F0F0F0Fu, C1); o0.y = minus_zero_e4m3((w.x >> 4) & 0x0F0F0F0Fu, C1);
-                        o0.z = minus_zero_e4m3(w.y & 0x0F0F0F0Fu, C1); o0.w = minus_zero_e4m3((w.y >> 4) & 0x0F0F0F0Fu, C1);
-                        o1.x = minus_zero_e4m3(w.z & 0x0F0F0F0Fu, C1); o1.y = minus_zero_e4m3((w.z >> 4) & 0x0F0F0F0Fu, C1);
-                        o1.z = minus_zero_e4m3(w.w & 0x0F0F0F0Fu, C1); o1.w = minus_zero_e4m3((w.w >> 4) & 0x0F0F0F0Fu, C1);
-                        const int c0 = (2 * p) ^ (r & 7), c1 = (2 * p + 1) ^ (r & 7);
-                        *reinterpret_cast<uint4 *>(dstA + r * 128 + c0 * 16) = o0;
-                        *reinterpret_cast<uint4 *>(dstA + r * 128 + c1 * 16) = o1;
+                        o0.x = w.x & 0x0F0F0F0Fu; o0.y = (w.x >> 4) & 0x0F0F0F0Fu;
+                        o0.z = w.y & 0x0F0F0F0Fu; o0.w = (w.y >> 4) & 0x0F0F0F0Fu;
+                        o1.x = w.z & 0x0F0F0F0Fu; o1.y = (w.z >> 4) & 0x0F0F0F0Fu;
+                        o1.z = w.w & 0x0F0F0F0Fu; o1.w = (w.w >> 4) & 0x0F0F0F0Fu;
+                        const int c0 = (2 * p) ^ (rr & 7), c1 = (2 * p + 1) ^ (rr & 7);
+                        *reinterpret_cast<uint4 *>(dstA + rr * 128 + c0 * 16) = o0;
+                        *reinterpret_cast<uint4 *>(dstA + rr * 128 + c1 * 16) = o1;
                     }
-                } else {
-                    // zero-point pseudo-stage z: columns kk = 64z .. 64z+63 of [hi|hi|lo](s z) x [hi|lo|hi](G)
-                    // the MMA released this raw slot's previous use
-                    const bool got = wait_phase(&sm->empty[slot], ((uint32_t)(it / STAGES) & 1) ^ 1, sm, a.status);
-                    if (got) {
-                        const int z = s - a.KT;
-                        uint8_t *dstB = raw + slot * RAW_BYTES + C_BYTES;
-                        const int Jr = a.Jr;
-                        // A': weight row n = n0 + et, 64 bf16, written 8 at a time
-                        const int64_t n = T.n0 + et;
-#pragma unroll 1
-                        for (int c = 0; c < 8; ++c) {
-                            uint32_t wv[4];
-#pragma unroll
-                            for (int q2 = 0; q2 < 4; ++q2) {
-                                uint32_t v2[2];
-#pragma unroll
-                                for (int h = 0; h < 2; ++h) {
-                                    const int kk = z * ZK + c * 8 + q2 * 2 + h;
-                                    const int part = kk / Jr, j = kk - part * Jr;
-                                    uint32_t v = 0;
-                                    if (part < 3) {
-                                        const uint32_t en = scales[(int64_t)j * a.Npad + n];
-                                        const float sc = __half2float(__ushort_as_half((unsigned short)(en & 0xFFFF)));
-                                        const int zz = (int)(int16_t)(en >> 16);
-                                        const float sz = sc * (float)(zz - min(max(zz, 0), 15));
-                                        const uint32_t hi = bf16_bits_rn(sz);
-                                        v = (part < 2) ? hi : bf16_bits_rn(sz - __uint_as_float(hi << 16));
-                                    }
-                                    v2[h] = v;
-                                }
-                                wv[q2] = v2[0] | (v2[1] << 16);
-                            }
-                            *reinterpret_cast<uint4 *>(dstA + et * 128 + ((c ^ (et & 7)) * 16)) =
-                                make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                        }
-                        // B': tokens row0 + et and row0 + et + 128, 64 bf16 each
-#pragma unroll 1
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            const int r = et + 128 * h2;
-                            const int64_t m = T.row0 + r;
-                            const bool live = r < T.rows && m < a.M;
-#pragma unroll 1
-                            for (int c = 0; c < 8; ++c) {
-                                uint32_t wv[4];
-#pragma unroll
-                                for (int q2 = 0; q2 < 4; ++q2) {
-                                    uint32_t v2[2];
-#pragma unroll
-                                    for (int h = 0; h < 2; ++h) {
-                                        const int kk = z * ZK + c * 8 + q2 * 2 + h;
-                                        const int part = kk / Jr, j = kk - part * Jr;
-                                        uint32_t v = 0;
-                                        if (live && part < 3) {
-                                            const float gv = __ldg(a.gsum + m * Jr + j);
-                                            const uint32_t hi = bf16_bits_rn(gv);
-                                            v = (part == 1) ? bf16_bits_rn(gv - __uint_as_float(hi << 16)) : hi;
-                                        }
-                                        v2[h] = v;
-                                    }
-                                    wv[q2] = v2[0] | (v2[1] << 16);
-                                }
-                                *reinterpret_cast<uint4 *>(dstB + r * 128 + ((c ^ (r & 7)) * 16)) =
-                                    make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                            }
-                        }
-                    }
-                    if (!got) { ok = false; break; }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_arrive(&sm->exp_full[eb]);
+                __syncwarp();
+                if ((threadIdx.x & 31) == 0) mbar_arrive(&sm->exp_full[slot]);
             }
         }
     }
@@ -538,19 +511,38 @@ static int sm_count_cached() {
     return cache[dev];
 }
 
-static w4_status launch(const uint8_t *X8, const float *row_scale, const float *gsum, const int32_t *offsets, int E,
+// Launch the kernel instantiation for group size G (first call per device sets its shared
+// memory limit).
+template <int G>
+static w4_status start(int grid, const CUtensorMap &tm_codes, const CUtensorMap &tm_act, const CUtensorMap &tm_zop,
+                       const CUtensorMap &tm_gop, const Args &a, cudaStream_t stream) {
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(w4a8_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+            cudaSuccess)
+            return W4_ERR_CUDA;
+        attr_done[dev] = 1;
+    }
+    w4a8_kernel<G><<<grid, THREADS, SMEM_BYTES, stream>>>(tm_codes, tm_act, tm_zop, tm_gop, a);
+    return launch_status();
+}
+
+static w4_status launch(const uint8_t *X8, const float *row_scale, const uint16_t *gop, const int32_t *offsets, int E,
                         int64_t M, const void *packed, int64_t N, int64_t K, int group, void *Y, int out_fp32,
                         cudaStream_t stream) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return W4_ERR_CUDA;
     const GemmLayout L = gemm_layout(N, K, group);
-    CUtensorMap tm_codes, tm_act;
+    const uint8_t *pk = static_cast<const uint8_t *>(packed);
+    CUtensorMap tm_codes, tm_act, tm_zop, tm_gop;
     {
         const cuuint64_t dims[3] = {(cuuint64_t)(L.Kpad / 2), (cuuint64_t)L.Npad, (cuuint64_t)E};
         const cuuint64_t strides[2] = {(cuuint64_t)(L.Kpad / 2), (cuuint64_t)L.total};
         const cuuint32_t box[3] = {BK / 2, BM, 1};
         const cuuint32_t es[3] = {1, 1, 1};
-        if (enc(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(packed), dims, strides, box, es,
+        if (enc(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(pk), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4_ERR_CUDA;
@@ -565,49 +557,50 @@ static w4_status launch(const uint8_t *X8, const float *row_scale, const float *
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4_ERR_CUDA;
     }
-    CUtensorMap tm_sc;
     {
-        const cuuint64_t dims[3] = {(cuuint64_t)L.Npad, (cuuint64_t)L.J, (cuuint64_t)E};
-        const cuuint64_t strides[2] = {(cuuint64_t)(L.Npad * 4), (cuuint64_t)L.total};
-        const cuuint32_t box[3] = {BM, (cuuint32_t)(BK / group), 1};
+        const cuuint64_t dims[3] = {(cuuint64_t)L.KZ, (cuuint64_t)L.Npad, (cuuint64_t)E};
+        const cuuint64_t strides[2] = {(cuuint64_t)(L.KZ * 2), (cuuint64_t)L.total};
+        const cuuint32_t box[3] = {ZKC, BM, 1};
         const cuuint32_t es[3] = {1, 1, 1};
-        if (enc(&tm_sc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3,
-                const_cast<uint8_t *>(static_cast<const uint8_t *>(packed) + L.codes_bytes), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        if (enc(&tm_zop, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                const_cast<uint8_t *>(pk + L.codes_bytes + L.scales_bytes), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)L.KZ, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)(L.KZ * 2)};
+        const cuuint32_t box[2] = {ZKC, BN};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&tm_gop, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(gop), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4_ERR_CUDA;
     }
     Args a;
-    a.packed = static_cast<const uint8_t *>(packed);
+    a.packed = pk;
     a.slab_bytes = L.total;
-    a.flags_off = L.codes_bytes + L.scales_bytes;
     a.codes_bytes = L.codes_bytes;
     a.row_scale = row_scale;
-    a.gsum = gsum;
     a.offsets = offsets;
     a.Y = Y;
     a.status = device_status_ptr();
     a.M = M; a.N = N; a.Npad = L.Npad; a.K = K; a.Kpad = L.Kpad;
-    a.E = E; a.g = group; a.Jr = (int)(K / group); a.out_fp32 = out_fp32;
+    a.E = E; a.g = group; a.out_fp32 = out_fp32;
     a.NT = (int)(L.Npad / BM);
     const int64_t mtu = offsets ? (M + BN - 1) / BN + E : (M + BN - 1) / BN;
     if (mtu > 0x7fffffffLL) return W4_ERR_SHAPE;
     a.MTU = (int)mtu;
     a.KT = (int)(L.Kpad / BK);
-    a.ZT = (int)((3 * a.Jr + ZK - 1) / ZK);
-    static int attr_done[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        if (cudaFuncSetAttribute(w4a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
-            cudaSuccess)
-            return W4_ERR_CUDA;
-        attr_done[dev] = 1;
-    }
+    a.ZT = (int)(L.KZ / ZKC);
     const int64_t tiles = mtu * a.NT;
     const int grid = (int)(tiles < sm_count_cached() ? tiles : sm_count_cached());
-    w4a8_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_codes, tm_act, tm_sc, a);
-    return launch_status();
+    switch (group) {
+        case 32: return start<32>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream);
+        case 64: return start<64>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream);
+        default: return start<128>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream);
+    }
 }
 
 }  // namespace gemm
@@ -615,31 +608,31 @@ static w4_status launch(const uint8_t *X8, const float *row_scale, const float *
 
 using namespace w4;
 
-W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const float *group_sums, int64_t M,
+W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op, int64_t M,
                            const void *packed, int64_t N, int64_t K, int group, int mode, void *Y, int out_fp32,
                            cudaStream_t stream) {
-    if (!X_e4m3 || !row_scale || !group_sums || !packed || !Y) return W4_ERR_NULL;
+    if (!X_e4m3 || !row_scale || !gsum_op || !packed || !Y) return W4_ERR_NULL;
     if (!valid_mode(mode) || (out_fp32 != 0 && out_fp32 != 1)) return W4_ERR_ARG;
     if (M < 1 || M > 0x7fffffffLL || N < 1 || N > 0x7fffffffLL || K < 128 || K % 32 != 0 || K > (1LL << 24))
         return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
-    if (!aligned16(X_e4m3) || !aligned16(row_scale) || !aligned16(group_sums) || !aligned16(packed) || !aligned16(Y))
+    if (!aligned16(X_e4m3) || !aligned16(row_scale) || !aligned16(gsum_op) || !aligned16(packed) || !aligned16(Y))
         return W4_ERR_ALIGN;
-    return gemm::launch(X_e4m3, row_scale, group_sums, nullptr, 1, M, packed, N, K, group, Y, out_fp32, stream);
+    return gemm::launch(X_e4m3, row_scale, gsum_op, nullptr, 1, M, packed, N, K, group, Y, out_fp32, stream);
 }
 
-W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale, const float *group_sums,
+W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op,
                                    const int32_t *expert_row_offsets, int E, int64_t M_total, const void *packed,
                                    int64_t N, int64_t K, int group, int mode, void *Y, cudaStream_t stream) {
-    if (!X_e4m3 || !row_scale || !group_sums || !expert_row_offsets || !packed || !Y) return W4_ERR_NULL;
+    if (!X_e4m3 || !row_scale || !gsum_op || !expert_row_offsets || !packed || !Y) return W4_ERR_NULL;
     if (!valid_mode(mode)) return W4_ERR_ARG;
     if (E < 1 || E > 1024 || M_total < 1 || M_total > 0x7fffffffLL || N < 1 || N > 0x7fffffffLL || K < 128 ||
         K % 32 != 0 || K > (1LL << 24))
         return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
-    if (!aligned16(X_e4m3) || !aligned16(row_scale) || !aligned16(group_sums) || !aligned16(packed) ||
+    if (!aligned16(X_e4m3) || !aligned16(row_scale) || !aligned16(gsum_op) || !aligned16(packed) ||
         !aligned16(Y) || (reinterpret_cast<uintptr_t>(expert_row_offsets) & 3))
         return W4_ERR_ALIGN;
-    return gemm::launch(X_e4m3, row_scale, group_sums, expert_row_offsets, E, M_total, packed, N, K, group, Y, 0,
+    return gemm::launch(X_e4m3, row_scale, gsum_op, expert_row_offsets, E, M_total, packed, N, K, group, Y, 0,
                         stream);
 }

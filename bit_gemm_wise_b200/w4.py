@@ -35,7 +35,8 @@ SIGNATURES = [
     ("w4_quantize", _I, [_P, _I64, _I64, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
     ("w4_prepack_bytes", _SZ, [_I64, _I64, _I, _I]),
     ("w4_prepack", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P]),
-    ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P]),
+    ("w4a8_gsum_op_cols", _I64, [_I64, _I]),
+    ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]),
     ("w4a16_gemv_workspace_bytes", _SZ, [_I64, _I64, _I]),
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a16_gemv_noalloc_scratch_limit", _SZ, []),
@@ -127,8 +128,12 @@ def w4_prepack(codes, scales, zeros, N, K, group, mode, layout, packed, stream=N
     _check("w4_prepack", rc)
 
 
-def fp8_row_quant(X, M, K, group, X8, row_scale, group_sums=None, stream=None):
-    rc = lib().fp8_row_quant(_ptr(X), M, K, group, _ptr(X8), _ptr(row_scale), _ptr(group_sums),
+def w4a8_gsum_op_cols(K, group) -> int:
+    return int(lib().w4a8_gsum_op_cols(K, group))
+
+
+def fp8_row_quant(X, M, K, group, X8, row_scale, group_sums=None, gsum_op=None, stream=None):
+    rc = lib().fp8_row_quant(_ptr(X), M, K, group, _ptr(X8), _ptr(row_scale), _ptr(group_sums), _ptr(gsum_op),
                              _stream(stream))
     _check("fp8_row_quant", rc)
 
@@ -156,15 +161,15 @@ def w4a16_gemv_noalloc(x, M, packed, N, K, group, mode, y, flags, stream=None):
     _check("w4a16_gemv_noalloc", rc)
 
 
-def w4a8_gemm(X8, row_scale, group_sums, M, packed, N, K, group, mode, Y, out_fp32=0, stream=None):
-    rc = lib().w4a8_gemm(_ptr(X8), _ptr(row_scale), _ptr(group_sums), M, _ptr(packed), N, K, group,
+def w4a8_gemm(X8, row_scale, gsum_op, M, packed, N, K, group, mode, Y, out_fp32=0, stream=None):
+    rc = lib().w4a8_gemm(_ptr(X8), _ptr(row_scale), _ptr(gsum_op), M, _ptr(packed), N, K, group,
                          _mode(mode), _ptr(Y), int(out_fp32), _stream(stream))
     _check("w4a8_gemm", rc)
 
 
-def w4a8_grouped_gemm(X8, row_scale, group_sums, expert_row_offsets, E, M_total, packed, N, K, group,
+def w4a8_grouped_gemm(X8, row_scale, gsum_op, expert_row_offsets, E, M_total, packed, N, K, group,
                       mode, Y, stream=None):
-    rc = lib().w4a8_grouped_gemm(_ptr(X8), _ptr(row_scale), _ptr(group_sums), _ptr(expert_row_offsets), E,
+    rc = lib().w4a8_grouped_gemm(_ptr(X8), _ptr(row_scale), _ptr(gsum_op), _ptr(expert_row_offsets), E,
                                  M_total, _ptr(packed), N, K, group, _mode(mode), _ptr(Y), _stream(stream))
     _check("w4a8_grouped_gemm", rc)
 
@@ -202,3 +207,16 @@ def alloc_packed(N, K, group, layout, device="cuda", copies: int = 1):
     if nbytes == 0:
         raise W4Error("w4_prepack_bytes", 2)
     return torch.empty(copies * nbytes, dtype=torch.uint8, device=device)
+
+
+def alloc_row_quant(M, K, group, device="cuda", group_sums=True):
+    """Empty outputs of fp8_row_quant for the W4A8 GEMM: X8 u8 [M,K], row scales fp32 [M],
+    group sums fp32 [M,K/g] (optional) and the GEMM's group-sum operand bf16 [M, cols]."""
+    cols = w4a8_gsum_op_cols(K, group)
+    if cols == 0:
+        raise W4Error("w4a8_gsum_op_cols", 3)
+    X8 = torch.empty(M, K, dtype=torch.uint8, device=device)
+    sa = torch.empty(M, dtype=torch.float32, device=device)
+    G = torch.empty(M, K // group, dtype=torch.float32, device=device) if group_sums else None
+    gop = torch.empty(M, cols, dtype=torch.bfloat16, device=device)
+    return X8, sa, G, gop

@@ -108,9 +108,12 @@ w4_status w4_quantize(const void *W_bf16, int64_t N, int64_t K, int group, int m
                       cudaStream_t stream);
 
 /*
- * w4_prepack_bytes / w4_prepack -- lossless re-layout of a canonical quantized weight into a
- *   kernel layout; no value is dequantized or requantized (TAHOMA "MSE clipping": portable
- *   codes, scales and zero terms are rearranged once into a GPU-specific layout).
+ * w4_prepack_bytes / w4_prepack -- re-layout of a canonical quantized weight into a kernel
+ *   layout; no code, scale or zero is dequantized or requantized (TAHOMA "MSE clipping":
+ *   portable codes, scales and zero terms are rearranged once into a GPU-specific layout).
+ *   W4_LAYOUT_GEMM also stores, after the moved codes and scales, the GEMM's zero-point
+ *   operand: bf16 hi/lo parts of s[n,j] * z[n,j] (a function of the scales and zeros, so
+ *   the canonical weight stays the only source of truth).
  *   layout W4_LAYOUT_GEMV feeds w4a16_gemv, W4_LAYOUT_GEMM feeds w4a8_gemm and (one slab per
  *   expert) w4a8_grouped_gemm. The packed buffer is opaque; its size is
  *   w4_prepack_bytes(N, K, group, layout) (0 for invalid arguments) and includes padding of
@@ -131,14 +134,20 @@ w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, const in
  *   X_bf16      device, bf16 [M, K]; M >= 1, K >= 16, K % 16 == 0
  *   X_e4m3      device, uint8 [M, K]
  *   row_scale   device, fp32 [M]
- *   group_sums  device, fp32 [M, K/group] or NULL: sum of the E4M3 VALUES (not scaled by
- *               s[m]) of each group of `group` consecutive codes, summed exactly and rounded
- *               once to fp32. w4a8_gemm needs them (it applies the weight zero point
- *               through them). group must be 32, 64 or 128 when group_sums != NULL.
+ *   group_sums  device, fp32 [M, K/group] or NULL: G[m,j], the sum of the E4M3 VALUES (not
+ *               scaled by s[m]) of group j of `group` consecutive codes, summed exactly and
+ *               rounded once to fp32.
+ *   gsum_op     device, bf16 [M, C] with C = w4a8_gsum_op_cols(K, group), or NULL: the
+ *               group-sum operand that w4a8_gemm needs (it applies the weight zero point
+ *               through it). With J = K/group, hi = bf16(G[m,j]) and lo = bf16(G[m,j] - hi),
+ *               row m holds [hi(0..J-1) | lo(0..J-1) | hi(0..J-1) | 0 ...].
+ *   group must be 32, 64 or 128 when group_sums or gsum_op is given.
  *   Errors: NULL / SHAPE / GROUP / ALIGN.
  */
+int64_t w4a8_gsum_op_cols(int64_t K, int group); /* 3 K/group rounded up to 32; 0 if invalid */
 w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uint8_t *X_e4m3,
-                        float *row_scale, float *group_sums, cudaStream_t stream);
+                        float *row_scale, float *group_sums, uint16_t *gsum_op,
+                        cudaStream_t stream);
 
 /*
  * w4a16_gemv -- weight-only INT4 decode GEMV with the dequantization fused into the
@@ -201,26 +210,28 @@ w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, 
  *   kernel, the activation and expanded weight enter an FP8 tensor-core MMA, accumulation
  *   is FP32, the per-token activation scale is applied in the epilogue, the result is BF16):
  *     Y[m, n] = s_a[m] * sum_j s[n,j] * sum_{k in group j} a8[m,k] * (q[n,k] - z[n,j])
- *   with a8 the E4M3 value of X_e4m3[m,k]. The expanded weights are exact small integers
- *   in E4M3; the group scale multiplies fp32 per-group partial sums and the zero point is
- *   applied through the activation group sums, so the MMA operands are exactly the
- *   dequantized operands.
+ *   with a8 the E4M3 value of X_e4m3[m,k], computed as
+ *     s_a[m] * ( sum_j s[n,j] * sum_{k in j} a8[m,k] q[n,k]  -  sum_j s[n,j] z[n,j] G[m,j] ).
+ *   The expanded weights q are exact small integers in E4M3 and the FP8 MMA sums exact
+ *   products; the group scale multiplies fp32 per-group partial sums; the zero-point term
+ *   is a bf16 hi/lo product on the tensor cores (relative error about 2^-16 of that term).
  *   X_e4m3      device, uint8 [M, K] from fp8_row_quant
  *   row_scale   device, fp32 [M] from fp8_row_quant
- *   group_sums  device, fp32 [M, K/group] from fp8_row_quant with the same group
+ *   gsum_op     device, bf16 [M, w4a8_gsum_op_cols(K, group)] from fp8_row_quant with the
+ *               same group
  *   packed      device, w4_prepack(..., W4_LAYOUT_GEMM) of W[N, K]
  *   Y           device, bf16 [M, N] (out_fp32 == 0) or fp32 [M, N] (out_fp32 == 1)
  *   M >= 1; N >= 1; K >= 128, K % 32 == 0.
  *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG.
  */
-w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const float *group_sums,
+w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op,
                     int64_t M, const void *packed, int64_t N, int64_t K, int group, int mode,
                     void *Y, int out_fp32, cudaStream_t stream);
 
 /*
  * w4a8_grouped_gemm -- w4a8_gemm for E experts at once (mixture-of-experts layers whose
  *   expert weights are 4-bit; the blog post "4-bit by default", gpt-oss paragraph). Rows
- *   [off[e], off[e+1]) of X_e4m3 / row_scale / group_sums / Y belong to expert e and are
+ *   [off[e], off[e+1]) of X_e4m3 / row_scale / gsum_op / Y belong to expert e and are
  *   multiplied by expert e's weight.
  *   expert_row_offsets  device, int32 [E+1], non-decreasing, off[0] == 0, off[E] == M_total
  *   packed              device, E slabs of w4_prepack_bytes(N, K, group, W4_LAYOUT_GEMM)
@@ -229,7 +240,7 @@ w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const float *
  *   1 <= E <= 1024. Errors: NULL / SHAPE / GROUP / ALIGN / ARG.
  */
 w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale,
-                            const float *group_sums, const int32_t *expert_row_offsets, int E,
+                            const uint16_t *gsum_op, const int32_t *expert_row_offsets, int E,
                             int64_t M_total, const void *packed, int64_t N, int64_t K, int group,
                             int mode, void *Y, cudaStream_t stream);
 

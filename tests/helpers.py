@@ -41,3 +41,21 @@ def bf16_round(a):
 
 
 bf16_bits = synth.bf16_bits
+
+
+def gsum_operand(G, K, group):
+    """The W4A8 GEMM's group-sum operand (the format w4.h documents for fp8_row_quant's
+    gsum_op) built from fp32 group sums G [M, J]: row m = [hi | lo | hi | 0 ...] with
+    hi = bf16(G) and lo = bf16(G - hi), both round-to-nearest-even, padded to a multiple of
+    32 columns. Returned as uint16 bit patterns."""
+    G = np.asarray(G, np.float32)
+    M, J = G.shape
+    assert J == K // group
+    cols = (3 * J + 31) // 32 * 32
+    hi = torch.from_numpy(G).to(torch.bfloat16)
+    lo = (torch.from_numpy(G) - hi.float()).to(torch.bfloat16)
+    h = hi.view(torch.int16).numpy().view(np.uint16)
+    l = lo.view(torch.int16).numpy().view(np.uint16)
+    out = np.zeros((M, cols), np.uint16)
+    out[:, :J], out[:, J:2 * J], out[:, 2 * J:3 * J] = h, l, h
+    return out

@@ -47,11 +47,25 @@ def test_prepack_bytes(lib):
     # GEMV layout: codes of N padded to 8 and K to 128, plus 4 bytes per (row, group)
     assert w4.w4_prepack_bytes(4096, 4096, 128, w4.W4_LAYOUT_GEMV) == 4096 * 4096 // 2 + 4096 * 32 * 4
     assert w4.w4_prepack_bytes(1536, 576, 32, w4.W4_LAYOUT_GEMV) == 1536 * 640 // 2 + 1536 * 20 * 4
-    # GEMM layout: rows padded to 128
-    assert w4.w4_prepack_bytes(2880, 2880, 32, w4.W4_LAYOUT_GEMM) == 2944 * 2944 // 2 + 92 * 2944 * 4 + 32
+    # GEMM layout: rows and K padded to 128; codes, scales of the padded groups, and the
+    # zero-point operand with 3 * 90 real groups rounded up to 288 bf16 columns
+    assert w4.w4_prepack_bytes(2880, 2880, 32, w4.W4_LAYOUT_GEMM) == \
+        2944 * 2944 // 2 + 92 * 2944 * 4 + 2944 * 288 * 2
+    assert w4.w4_prepack_bytes(3840, 15360, 128, w4.W4_LAYOUT_GEMM) == \
+        3840 * 15360 // 2 + 120 * 3840 * 4 + 3840 * 384 * 2
     for bad in [(0, 4096, 128), (16, 100, 32), (16, 4096, 48), (16, 96, 64)]:
         assert w4.w4_prepack_bytes(*bad, w4.W4_LAYOUT_GEMV) == 0
     assert w4.w4_prepack_bytes(16, 4096, 128, 7) == 0
+
+
+def test_gsum_op_cols(lib):
+    assert w4.w4a8_gsum_op_cols(2880, 32) == 288
+    assert w4.w4a8_gsum_op_cols(4096, 128) == 96
+    assert w4.w4a8_gsum_op_cols(15360, 128) == 384
+    assert w4.w4a8_gsum_op_cols(3840, 128) == 96
+    assert w4.w4a8_gsum_op_cols(160, 32) == 32
+    for bad in [(96, 64), (128, 48), (0, 32)]:
+        assert w4.w4a8_gsum_op_cols(*bad) == 0
 
 
 FAKE = 0x1000  # 16-byte aligned non-null address; never dereferenced (calls fail validation)
@@ -86,15 +100,17 @@ def test_host_validation_rejects_before_launch(lib):
     assert rc("w4_quantize", FAKE, 16, 128, 128, 1, gp, 0, FAKE, FAKE, FAKE, None, None) == 5
     assert rc("w4_quantize", FAKE, 16, 128, 128, 1, gp, 65, FAKE, FAKE, FAKE, None, None) == 5
     # row quant
-    assert rc("fp8_row_quant", None, 4, 64, 32, FAKE, FAKE, None, None) == 1
-    assert rc("fp8_row_quant", FAKE, 4, 72, 32, FAKE, FAKE, None, None) == 2
-    assert rc("fp8_row_quant", FAKE, 4, 96, 64, FAKE, FAKE, FAKE, None) == 3
+    assert rc("fp8_row_quant", None, 4, 64, 32, FAKE, FAKE, None, None, None) == 1
+    assert rc("fp8_row_quant", FAKE, 4, 72, 32, FAKE, FAKE, None, None, None) == 2
+    assert rc("fp8_row_quant", FAKE, 4, 96, 64, FAKE, FAKE, FAKE, None, None) == 3
+    assert rc("fp8_row_quant", FAKE, 4, 96, 64, FAKE, FAKE, None, FAKE, None) == 3
+    assert rc("fp8_row_quant", FAKE, 4, 128, 64, FAKE, FAKE, None, FAKE + 4, None) == 4
     # gemv: M range, mode, out flag
     assert rc("w4a16_gemv", FAKE, 17, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE, 1 << 20, None) == 2
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 3, FAKE, 0, FAKE, 1 << 20, None) == 5
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 4, FAKE, 1 << 20, None) == 5
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE + 8, 1 << 20, None) == 4
-    # gemm: group sums are required, K >= 128
+    # gemm: the group-sum operand is required, K >= 128
     assert rc("w4a8_gemm", FAKE, FAKE, None, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None) == 1
     assert rc("w4a8_gemm", FAKE, FAKE, FAKE, 4, FAKE, 16, 96, 32, 1, FAKE, 0, None) == 2
     # grouped gemm: expert count range

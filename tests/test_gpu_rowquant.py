@@ -1,40 +1,49 @@
 """GPU fp8_row_quant vs the CPU oracle: E4M3 bytes, row scales and group sums must be
-bit-identical."""
+bit-identical, and the GEMM's group-sum operand must be the documented bf16 hi/lo split of
+the oracle's group sums, bit for bit."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from bit_gemm_wise_b200 import synth, w4
-from helpers import cuda, np_of
+from helpers import cuda, gsum_operand, np_of
 
 pytestmark = pytest.mark.gpu
 
 
-def gpu_row_quant(X, group):
+def gpu_row_quant(X, group, op_only=False):
     M, K = X.shape
     Xd = X.to(cuda())
-    X8 = torch.empty(M, K, dtype=torch.uint8, device=cuda())
-    s = torch.empty(M, dtype=torch.float32, device=cuda())
-    G = torch.empty(M, K // group, dtype=torch.float32, device=cuda()) if group else None
-    w4.fp8_row_quant(Xd, M, K, group if group else 32, X8, s, G)
+    if group:
+        X8, s, G, gop = w4.alloc_row_quant(M, K, group, device=cuda(), group_sums=not op_only)
+        gop.fill_(7.0)  # the kernel must write every column, padding included
+    else:
+        X8 = torch.empty(M, K, dtype=torch.uint8, device=cuda())
+        s = torch.empty(M, dtype=torch.float32, device=cuda())
+        G = gop = None
+    w4.fp8_row_quant(Xd, M, K, group if group else 32, X8, s, G, gop)
     torch.cuda.synchronize()
-    return np_of(X8), np_of(s), (np_of(G) if G is not None else None)
+    op = gop.view(torch.int16).cpu().numpy().view(np.uint16) if gop is not None else None
+    return np_of(X8), np_of(s), (np_of(G) if G is not None else None), op
 
 
-def check(X, group, rows=None):
-    gX8, gs, gG = gpu_row_quant(X, group)
+def check(X, group, rows=None, op_only=False):
+    gX8, gs, gG, gop = gpu_row_quant(X, group, op_only)
     bits = synth.bf16_bits(X)
     if rows is not None:
         bits = bits[rows]
         gX8, gs = gX8[rows], gs[rows]
         gG = gG[rows] if gG is not None else None
+        gop = gop[rows] if gop is not None else None
     X8, s, G = oracle.row_quant(bits, group)
     assert np.array_equal(gs.view(np.uint32), s.view(np.uint32))
     bad = np.argwhere(gX8 != X8)
     assert bad.size == 0, f"{len(bad)} byte mismatches, first {bad[:3].tolist()}"
     if group:
-        assert np.array_equal(gG.view(np.uint32), G.view(np.uint32))
+        if not op_only:
+            assert np.array_equal(gG.view(np.uint32), G.view(np.uint32))
+        assert np.array_equal(gop, gsum_operand(G, X.shape[1], group))
 
 
 @pytest.mark.parametrize("K", [3840, 15360])
@@ -78,3 +87,4 @@ def test_ragged_and_long_rows(M, K):
     check(X, 0)
     if K % 32 == 0:
         check(X, 32)
+        check(X, 32, op_only=True)
