@@ -88,6 +88,8 @@ struct Args {
     int M, g, out_fp32, nol, pdl;
     uint32_t sub;              // scale bytes per unit
     uint32_t off_sx, off_slot;
+    uint32_t off_xf;           // M = 1 kernel: padded bf16 copy of x
+    uint32_t off_ring, off_bars;  // M = 1 kernel: per-warp stage rings and their mbarriers
 };
 
 __device__ __forceinline__ uint32_t range_start(const Args &a, uint32_t c) {
@@ -120,6 +122,69 @@ template <int MT> struct Warps { static constexpr int value = MT == 1 ? 32 : (MT
 __device__ __forceinline__ void store_y(const Args &a, int m, int64_t n, float v) {
     if (a.out_fp32) static_cast<float *>(a.y)[(int64_t)m * a.N + n] = v;
     else static_cast<__nv_bfloat16 *>(a.y)[(int64_t)m * a.N + n] = __float2bfloat16_rn(v);
+}
+
+// Per-octet reduction of the warps' partials (fixed warp order) and, for octets cut by a
+// range boundary (stream-K partitions only), the cross-CTA fixup: the last CTA to arrive on
+// the octet's counter adds all CTAs' partials in CTA order and resets the counter.
+template <int MT, int W>
+__device__ __forceinline__ void finish(const Args &a, const float *slot, int *flags, uint32_t c, uint32_t t0,
+                                       uint32_t t1, uint32_t o_first, uint32_t o_last, int tid) {
+    constexpr int THREADS = W * 32;
+    const int M = a.M;
+    const uint32_t Uc = a.U;
+    const int nol = (int)(o_last - o_first + 1);
+    for (int idx = tid; idx < nol * 8 * MT; idx += THREADS) {
+        const int ol = idx / (8 * MT), rm = idx - ol * 8 * MT;
+        const int rr = rm / MT, m = rm - rr * MT;
+        float acc = 0.0f;
+        for (int w = 0; w < W; ++w) acc += slot[(ol * W + w) * 8 * MT + rm];
+        const uint32_t o = o_first + ol;
+        const bool inside = o * Uc >= t0 && (o + 1) * Uc <= t1;
+        if (inside) {
+            const int64_t n = (int64_t)o * 8 + rr;
+            if (m < M && n < a.N) store_y(a, m, n, acc);
+        } else {
+            const int which = (o == o_first) ? 0 : 1;
+            a.ws_part[(((int64_t)c * 2 + which) * 8 + rr) * MT + m] = acc;
+        }
+    }
+    // boundary octets (stream-K partitions only): the last CTA to arrive adds all partials
+    // in CTA order and resets the counter
+    const bool b0 = !(o_first * Uc >= t0 && (o_first + 1) * Uc <= t1);
+    const bool b1 = (o_last != o_first) && !(o_last * Uc >= t0 && (o_last + 1) * Uc <= t1);
+    if (!b0 && !b1) return;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        flags[1] = 0;
+        flags[2] = 0;
+        for (int which = 0; which < 2; ++which) {
+            if (!(which == 0 ? b0 : b1)) continue;
+            const uint32_t o = which == 0 ? o_first : o_last;
+            const uint32_t cnt = cta_of_unit(a, (o + 1) * Uc - 1) - cta_of_unit(a, o * Uc) + 1;
+            const int prev = atomicAdd(&a.ws_count[o], 1);
+            flags[1 + which] = (prev == (int)cnt - 1) ? 1 : 0;
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    for (int which = 0; which < 2; ++which) {
+        if (!flags[1 + which]) continue;
+        const uint32_t o = which == 0 ? o_first : o_last;
+        const uint32_t cf = cta_of_unit(a, o * Uc), cl = cta_of_unit(a, (o + 1) * Uc - 1);
+        for (int rm = tid; rm < 8 * MT; rm += THREADS) {
+            const int rr = rm / MT, m = rm - rr * MT;
+            float acc = 0.0f;
+            for (uint32_t k = cf; k <= cl; ++k) {
+                const int wk = (fdiv(range_start(a, k), a.divU) == o) ? 0 : 1;
+                acc += __ldcg(a.ws_part + (((int64_t)k * 2 + wk) * 8 + rr) * MT + m);
+            }
+            const int64_t n = (int64_t)o * 8 + rr;
+            if (m < M && n < a.N) store_y(a, m, n, acc);
+        }
+        if (tid == 0) a.ws_count[o] = 0;
+    }
 }
 
 template <int MT>
@@ -239,59 +304,166 @@ __global__ void __launch_bounds__(Warps<MT>::value * 32, 1) gemv_kernel(const Ar
     if (cur_ol != 0xffffffffu) flush_octet<MT, W>(cur_ol, y, slot, warp, lane);
     __syncthreads();
 
-    // ---------------------------------------------------- per-octet reduction
-    const int nol = (int)(o_last - o_first + 1);
-    for (int idx = tid; idx < nol * 8 * MT; idx += THREADS) {
-        const int ol = idx / (8 * MT), rm = idx - ol * 8 * MT;
-        const int rr = rm / MT, m = rm - rr * MT;
-        float acc = 0.0f;
-        for (int w = 0; w < W; ++w) acc += slot[(ol * W + w) * 8 * MT + rm];
-        const uint32_t o = o_first + ol;
-        const bool inside = o * Uc >= t0 && (o + 1) * Uc <= t1;
-        if (inside) {
-            const int64_t n = (int64_t)o * 8 + rr;
-            if (m < M && n < a.N) store_y(a, m, n, acc);
+    finish<MT, W>(a, slot, flags, c, t0, t1, o_first, o_last, tid);
+}
+
+// ---------------------------------------------------------------- M = 1 kernel
+//
+// Each warp streams a contiguous run of 512-byte units through its own ring of shared-memory
+// stages filled by 1-D bulk copies (one copy of codes and one of scales per stage of SU
+// units, issued by the warp's lane 0, completion on an mbarrier), so loading costs almost no
+// instructions; lanes read their 16 bytes of codes and their scale entry from shared memory.
+// x is staged once per CTA as bf16 with 16 bytes of padding after every 32 values, so the
+// four 32-wide chunks a warp reads at once start in different banks.
+constexpr int W1 = 16;   // warps of the M = 1 kernel
+constexpr int SU = 8;    // units per stage
+constexpr int NS = 2;    // stages per warp
+
+__device__ __forceinline__ uint32_t xb_index(uint32_t k) { return k + (k >> 5) * 8; }
+
+// One unit for one lane: 16 bytes of codes (32 weights of row r, chunk at k0) against the
+// padded bf16 x at xp, offset removed with the chunk sum sxc, times the group scale.
+__device__ __forceinline__ void unit_m1(float &y, const uint4 wq, uint32_t e, const uint4 *xp, float sxc) {
+    const float scl = __half2float(__ushort_as_half((unsigned short)(e & 0xFFFF)));
+    const float cz = (float)(int)(int16_t)(e >> 16) + 128.0f;
+    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+    const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 xv = xp[q];
+        fma2_bf16(a0, a1, xv.x, magic_pair(wv[q]));
+        fma2_bf16(a2, a3, xv.y, magic_pair(wv[q] >> 4));
+        fma2_bf16(a0, a1, xv.z, magic_pair(wv[q] >> 8));
+        fma2_bf16(a2, a3, xv.w, magic_pair(wv[q] >> 12));
+    }
+    y = fmaf(scl, fmaf(-cz, sxc, (a0 + a1) + (a2 + a3)), y);
+}
+
+// shared-memory bytes of the M = 1 kernel's regions
+inline uint32_t xb_bytes(uint32_t U) { return U * 4 * 40 * 2; }              // padded bf16 x
+inline uint32_t ring_bytes(uint32_t sub) { return W1 * NS * SU * (512 + sub); }
+
+__global__ void __launch_bounds__(W1 * 32, 1) gemv1_kernel(const Args a) {
+    constexpr int W = W1, THREADS = W1 * 32;
+    extern __shared__ __align__(16) uint8_t smem[];
+    int *flags = reinterpret_cast<int *>(smem);
+    float *sx = reinterpret_cast<float *>(smem + a.off_sx);
+    uint16_t *xb = reinterpret_cast<uint16_t *>(smem + a.off_xf);
+    float *slot = reinterpret_cast<float *>(smem + a.off_slot);
+    uint8_t *ring = smem + a.off_ring;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + a.off_bars);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = lane >> 2, cc = lane & 3;
+    const uint32_t c = blockIdx.x;
+    const uint32_t t0 = range_start(a, c), t1 = range_start(a, c + 1);
+    const uint32_t o_first = fdiv(t0, a.divU), o_last = fdiv(t1 - 1, a.divU);
+    const uint32_t Kc = (uint32_t)a.K, Uc = a.U;
+    const int nck = (int)(Uc * 4);
+    const uint32_t sub = a.sub, stage_bytes = SU * (512 + sub);
+
+    // this warp's contiguous run [wt0, wt1) of the CTA's units, in stages of SU units
+    const uint32_t n = t1 - t0;
+    const uint32_t wt0 = t0 + (uint32_t)(((uint64_t)n * warp) / W);
+    const uint32_t wt1 = t0 + (uint32_t)(((uint64_t)n * (warp + 1)) / W);
+    const uint32_t nst = (wt1 - wt0 + SU - 1) / SU;
+    uint8_t *wring = ring + (size_t)warp * NS * stage_bytes;
+    uint64_t *wbar = bars + warp * NS;
+
+    // lane 0 fills stage j of this warp's run into ring slot j % NS
+    auto issue = [&](uint32_t j) {
+        const uint32_t u0 = wt0 + j * SU;
+        const uint32_t cnt = (wt1 - u0) < (uint32_t)SU ? (wt1 - u0) : (uint32_t)SU;
+        uint8_t *dst = wring + (j % NS) * stage_bytes;
+        uint64_t *bar = wbar + (j % NS);
+        mbar_arrive_expect_tx(bar, cnt * (512 + sub));
+        bulk_g2s(dst, a.codes + (size_t)u0 * 512, cnt * 512, bar);
+        bulk_g2s(dst + SU * 512, a.scales + (size_t)u0 * sub, cnt * sub, bar);
+    };
+    // ---- the weight stream does not depend on earlier kernels: start it first
+    if (lane == 0) {
+        for (int j = 0; j < NS; ++j) mbar_init(wbar + j, 1);
+        fence_mbar_init();
+        for (uint32_t j = 0; j < (uint32_t)NS && j < nst; ++j) issue(j);
+    }
+    for (int i = tid; i < a.nol * W * 8; i += THREADS) slot[i] = 0.0f;
+    // activations may be written by the previous kernel in the stream
+    if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // x as padded bf16 and the sum of every 32-wide chunk (chunks past K are zero)
+    for (int ck = tid; ck < nck; ck += THREADS) {
+        float s = 0.0f;
+        const bool live = (uint32_t)ck * 32 < Kc;
+        const uint4 *xv = reinterpret_cast<const uint4 *>(a.x + ck * 32);
+        uint4 *dst = reinterpret_cast<uint4 *>(xb + xb_index((uint32_t)ck * 32));
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const uint4 u4 = live ? __ldg(xv + t) : make_uint4(0u, 0u, 0u, 0u);
+            s = __fadd_rn(__fadd_rn(s, bf16_lo(u4.x)), bf16_hi(u4.x));
+            s = __fadd_rn(__fadd_rn(s, bf16_lo(u4.y)), bf16_hi(u4.y));
+            s = __fadd_rn(__fadd_rn(s, bf16_lo(u4.z)), bf16_hi(u4.z));
+            s = __fadd_rn(__fadd_rn(s, bf16_lo(u4.w)), bf16_hi(u4.w));
+            dst[t] = u4;
+        }
+        sx[ck] = s;
+    }
+    __syncthreads();
+    if (a.pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    const int per_unit = 128 / a.g;
+    const uint32_t sc_lane = (uint32_t)(r * per_unit + (cc * 32) / a.g);  // u32 index in a unit's scales
+    float y[1] = {0.0f};
+    uint32_t o = fdiv(wt0, a.divU), u = wt0 - o * Uc;
+    uint32_t cur_ol = 0xffffffffu;  // set by the first (checked) stage
+    const bool kpad = (Kc & 127u) != 0;
+    bool ok = true;
+    for (uint32_t j = 0; j < nst && ok; ++j) {
+        const uint32_t sl = j % NS;
+        // lane 0 polls; every lane then takes the (now immediate) wait for its own acquire
+        bool got = true;
+        if (lane == 0) got = mbar_wait_bounded(wbar + sl, (j / NS) & 1u, a.status);
+        got = __shfl_sync(FULL, got ? 1 : 0, 0) != 0;
+        if (!got) { ok = false; break; }
+        (void)mbar_try_wait(wbar + sl, (j / NS) & 1u);
+        const uint8_t *st = wring + sl * stage_bytes;
+        const uint32_t u0 = wt0 + j * SU;
+        const uint32_t cnt = (wt1 - u0) < (uint32_t)SU ? (wt1 - u0) : (uint32_t)SU;
+        const uint4 *cw = reinterpret_cast<const uint4 *>(st) + lane;
+        const uint32_t *sw = reinterpret_cast<const uint32_t *>(st + SU * 512) + sc_lane;
+        if (cnt == (uint32_t)SU && u + SU <= Uc && o - o_first == cur_ol && !kpad) {
+            // fast path: a full stage inside the current octet, no padding chunks
+            const uint32_t k0 = u * 128u + (uint32_t)cc * 32u;
+            const uint4 *xp = reinterpret_cast<const uint4 *>(xb + xb_index(k0));
+            const float *sxp = sx + (k0 >> 5);
+#pragma unroll
+            for (int i = 0; i < SU; ++i)
+                unit_m1(y[0], cw[i * 32], sw[i * (sub >> 2)], xp + i * 20, sxp[i * 4]);
+            u += SU;
+            if (u == Uc) { u = 0; ++o; }
         } else {
-            const int which = (o == o_first) ? 0 : 1;
-            a.ws_part[(((int64_t)c * 2 + which) * 8 + rr) * MT + m] = acc;
-        }
-    }
-    // boundary octets (stream-K partitions only): the last CTA to arrive adds all partials
-    // in CTA order and resets the counter
-    const bool b0 = !(o_first * Uc >= t0 && (o_first + 1) * Uc <= t1);
-    const bool b1 = (o_last != o_first) && !(o_last * Uc >= t0 && (o_last + 1) * Uc <= t1);
-    if (!b0 && !b1) return;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        flags[1] = 0;
-        flags[2] = 0;
-        for (int which = 0; which < 2; ++which) {
-            if (!(which == 0 ? b0 : b1)) continue;
-            const uint32_t o = which == 0 ? o_first : o_last;
-            const uint32_t cnt = cta_of_unit(a, (o + 1) * Uc - 1) - cta_of_unit(a, o * Uc) + 1;
-            const int prev = atomicAdd(&a.ws_count[o], 1);
-            flags[1 + which] = (prev == (int)cnt - 1) ? 1 : 0;
-        }
-        __threadfence();
-    }
-    __syncthreads();
-    for (int which = 0; which < 2; ++which) {
-        if (!flags[1 + which]) continue;
-        const uint32_t o = which == 0 ? o_first : o_last;
-        const uint32_t cf = cta_of_unit(a, o * Uc), cl = cta_of_unit(a, (o + 1) * Uc - 1);
-        for (int rm = tid; rm < 8 * MT; rm += THREADS) {
-            const int rr = rm / MT, m = rm - rr * MT;
-            float acc = 0.0f;
-            for (uint32_t k = cf; k <= cl; ++k) {
-                const int wk = (fdiv(range_start(a, k), a.divU) == o) ? 0 : 1;
-                acc += __ldcg(a.ws_part + (((int64_t)k * 2 + wk) * 8 + rr) * MT + m);
+            for (uint32_t i = 0; i < cnt; ++i) {
+                const uint32_t ol = o - o_first;
+                if (ol != cur_ol) {
+                    if (cur_ol != 0xffffffffu) flush_octet<1, W>(cur_ol, y, slot, warp, lane);
+                    cur_ol = ol;
+                }
+                const uint32_t k0 = u * 128u + (uint32_t)cc * 32u;
+                if (++u == Uc) { u = 0; ++o; }
+                if (k0 >= Kc) continue;
+                unit_m1(y[0], cw[i * 32], sw[i * (sub >> 2)], reinterpret_cast<const uint4 *>(xb + xb_index(k0)),
+                        sx[k0 >> 5]);
             }
-            const int64_t n = (int64_t)o * 8 + rr;
-            if (m < M && n < a.N) store_y(a, m, n, acc);
         }
-        if (tid == 0) a.ws_count[o] = 0;
+        // every lane has read the slot: lane 0 refills it with stage j + NS
+        __syncwarp();
+        if (lane == 0 && j + NS < nst) issue(j + NS);
     }
+    if (cur_ol != 0xffffffffu) flush_octet<1, W>(cur_ol, y, slot, warp, lane);
+    // no bulk copy may still be in flight when the CTA exits: on a failed wait, wait (bounded)
+    // for the copies this warp issued
+    if (!ok && lane == 0)
+        for (uint32_t j = 0; j < nst && j < (uint32_t)NS; ++j) (void)mbar_wait_bounded(wbar + j, 0, a.status);
+    __syncthreads();
+    finish<1, W>(a, slot, flags, c, t0, t1, o_first, o_last, tid);
 }
 
 // ------------------------------------------------------------------ host side
@@ -314,9 +486,13 @@ static int sm_count_cached() {
 // enough (fewer octets than SMs, or the busiest SM at most ~8% above the mean), every CTA
 // gets whole octets and no partial sum crosses CTAs; otherwise the unit stream is split
 // evenly (stream-K) and octets cut by a range boundary are finished through the workspace.
+constexpr int SMEM_LIMIT_M1 = 227 * 1024;
+
+// xf: plan for the M = 1 kernel (padded bf16 x, per-warp stage rings, W1 warps)
 template <int MT>
-static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g) {
-    constexpr int W = Warps<MT>::value;
+static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool xf = false) {
+    const int W = xf ? W1 : Warps<MT>::value;
+    const size_t limit = xf ? (size_t)SMEM_LIMIT_M1 : (size_t)SMEM_LIMIT;
     const GemvLayout L = gemv_layout(N, K, g);
     Args &a = p.a;
     const int64_t T = L.N8 * L.U;
@@ -327,6 +503,13 @@ static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g) {
     a.sub = (uint32_t)(8 * (128 / g) * 4);
     a.off_sx = 64;
     a.off_slot = a.off_sx + (uint32_t)(MT * L.U * 4 * 4);
+    a.off_xf = a.off_ring = a.off_bars = 0;
+    if (xf) {
+        a.off_xf = a.off_slot;
+        a.off_ring = a.off_xf + xb_bytes((uint32_t)L.U);
+        a.off_bars = a.off_ring + ring_bytes(a.sub);
+        a.off_slot = a.off_bars + W1 * NS * 8;
+    }
     a.pdl = 0;
     const int64_t S = sm_count_cached();
     int64_t P;
@@ -352,7 +535,7 @@ static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g) {
         const int64_t maxr = (int64_t)a.base + (a.rem ? a.step : 0);
         const int64_t nol = (maxr + L.U - 1) / L.U + 1;
         const size_t smem = a.off_slot + (size_t)nol * W * 8 * MT * 4;
-        if (smem <= (size_t)SMEM_LIMIT) {
+        if (smem <= limit) {
             a.nol = (int)nol;
             p.P = (int)P;
             p.smem = (int)smem;
@@ -367,10 +550,21 @@ static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g) {
     return true;
 }
 
+// The plan a call of M rows will use: the M = 1 kernel's when it applies and its shared
+// memory (which grows with K) fits, else the general kernel's.
+template <int MT>
+static bool plan_for(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool &xf) {
+    xf = MT == 1;
+    if (xf && make_plan<MT>(p, M, N, K, g, true)) return true;
+    xf = false;
+    return make_plan<MT>(p, M, N, K, g, false);
+}
+
 template <int MT>
 static size_t ws_need(int64_t N, int64_t K, int g) {
     Plan p;
-    if (!make_plan<MT>(p, MT, N, K, g)) return 0;
+    bool xf;
+    if (!plan_for<MT>(p, MT, N, K, g, xf)) return 0;
     return (size_t)p.P * 2 * 8 * MT * 4;
 }
 
@@ -379,7 +573,8 @@ static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, in
                      void *ws, size_t ws_bytes, int pdl, cudaStream_t stream) {
     constexpr int W = Warps<MT>::value;
     Plan p;
-    if (!make_plan<MT>(p, M, N, K, g)) return W4_ERR_SHAPE;
+    bool xf;
+    if (!plan_for<MT>(p, M, N, K, g, xf)) return W4_ERR_SHAPE;
     const GemvLayout L = gemv_layout(N, K, g);
     const size_t need = (size_t)p.P * 2 * 8 * MT * 4 + (size_t)L.N8 * 4;
     if (!ws || ws_bytes < need) return W4_ERR_WORKSPACE;
@@ -400,11 +595,14 @@ static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, in
         if (cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT) !=
             cudaSuccess)
             return W4_ERR_CUDA;
+        if (MT == 1 && cudaFuncSetAttribute(gemv1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            SMEM_LIMIT_M1) != cudaSuccess)
+            return W4_ERR_CUDA;
         attr_done[dev] = 1;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.P);
-    cfg.blockDim = dim3(W * 32);
+    cfg.blockDim = dim3(xf ? W1 * 32 : W * 32);
     cfg.dynamicSmemBytes = (size_t)p.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -412,7 +610,8 @@ static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, in
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemv_kernel<MT>, a) != cudaSuccess) return W4_ERR_CUDA;
+    const cudaError_t e = xf ? cudaLaunchKernelEx(&cfg, gemv1_kernel, a) : cudaLaunchKernelEx(&cfg, gemv_kernel<MT>, a);
+    if (e != cudaSuccess) return W4_ERR_CUDA;
     return launch_status();
 }
 
@@ -490,7 +689,8 @@ template <int MT>
 static w4_status run_noalloc(const void *x, int64_t M, const void *packed, int64_t N, int64_t K, int g, void *y,
                              int out_fp32, int pdl, cudaStream_t stream) {
     Plan p;
-    if (!make_plan<MT>(p, M, N, K, g)) return W4_ERR_SHAPE;
+    bool xf;
+    if (!plan_for<MT>(p, M, N, K, g, xf)) return W4_ERR_SHAPE;
     const GemvLayout L = gemv_layout(N, K, g);
     const size_t part = (size_t)p.P * 2 * 8 * MT * 4;
     const size_t need = part + (size_t)L.N8 * 4;
