@@ -46,6 +46,29 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
+# DRAM bytes per launch of the roofline kernels, from one ncu capture each
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by kernel and shape, with the SHA-1 of
+# the kernel's source file at capture time: a number is reported only while the source is
+# unchanged (otherwise the counters describe a different kernel and "traffic" is null).
+NCU_TRAFFIC = {
+    # profiles/w4a16_gemv_m1_k4096_n14336_full.md
+    "w4a16_gemv M1 K4096xN14336": {"bytes": 31242496, "sha1": "961edcf2b56045a28adb7b1a1672443968c1c9a7"},
+}
+
+
+def source_sha1(rel):
+    import hashlib
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+def traffic_for(key, rel):
+    t = NCU_TRAFFIC.get(key)
+    if not t or t["sha1"] != source_sha1(rel):
+        return None
+    return t["bytes"]
+
+
 def gemv_bytes(M, N, K, g=128):
     """Algorithmic bytes of one W4A16 GEMV: packed codes, 2+2 bytes of scale and zero per
     group, the bf16 activations and the bf16 output."""
@@ -226,6 +249,19 @@ def run_ours(args, rank, world, dev):
         per_shape[f"K{K}xN{N}"] = {"us": round(t_ms * 1e3, 3),
                                    "GBps": round(gemv_bytes(1, N, K) / (t_ms * 1e-3) / 1e9, 1)}
 
+    # roofline of the dominant kernel: the shape whose GEMV launch takes longest;
+    # algorithmic bytes of one launch over its event-timed duration
+    dom = max(per_shape, key=lambda k: per_shape[k]["us"])
+    dK, dN = (int(v) for v in dom[1:].split("xN"))
+    dbytes = gemv_bytes(1, dN, dK)
+    dach = dbytes / (per_shape[dom]["us"] * 1e-6) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(dach, 1), "peak": pk["hbm"], "unit": "GB/s",
+                "frac": round(dach / pk["hbm"], 4),
+                "traffic": traffic_for(f"w4a16_gemv M1 {dom}", "bit_gemm_wise_b200/csrc/w4a16_gemv.cu"),
+                "kernel": f"w4a16_gemv M=1 {dom}", "bytes_per_launch": dbytes,
+                "peak_source": f"{pk['src']} copy bandwidth (of {pk['src']})",
+                "step_frac": round(value / world / pk["hbm"], 4)}
+
     # e2e through the public Python API with host buffers, every step: pinned h2d of the
     # activations, the four w4a16_gemv calls (not graphed), d2h of the outputs
     xh = [x.cpu().pin_memory() for x in dec.x]
@@ -260,9 +296,7 @@ def run_ours(args, rank, world, dev):
                    "l2": f"inputs larger than L2: weights rotate over {dec.R} copies "
                          f"({dec.R * sum(nb for _, nb in dec.packed) / 1e6:.0f} MB > 3 x L2)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": round(value / world / pk["hbm"], 4), "traffic": None,
-                     "peak_source": f"{pk['src']} copy bandwidth"},
+        "roofline": roofline,
         "per_shape": per_shape,
         "gpu_launches": dec.launches_per_step * args.steps,
         "clocks": clk.summary(),
@@ -297,6 +331,13 @@ def measure_rows(args, dev, pk):
                                     "us_per_step": round(ms * 1e3, 2),
                                     "frac_hbm": round(d.bytes_per_step / (ms * 1e-3) / 1e9 / pk["hbm"], 4)}
         del d
+
+    # context for the FP8 rows: cuBLAS FP8 GEMM (torch._scaled_mm, e4m3, 8192^3, best of 10)
+    fp8_cublas = None
+    if "prefill" in want or "moe" in want:
+        fp8_cublas = measure_fp8_cublas(dev)
+        rows["fp8_dense_cublas_8192"] = {"value": round(fp8_cublas, 1), "unit": "TFLOP/s",
+                                         "note": "context: torch._scaled_mm e4m3 8192^3, best of 10"}
 
     # W4A8 prefill GEMM (M=4096) and the FP8 row quant feeding it
     for K, N in (synth.PREFILL_SHAPES if "prefill" in want else ()):
@@ -334,7 +375,8 @@ def measure_rows(args, dev, pk):
             "value": round(tf, 1), "unit": "TFLOP/s", "us": round(t_gemm * 1e3, 1),
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4),
-                         "peak_source": f"{pk['src']} bf16 burst x 2 (dense FP8/BF16 nominal ratio)"}}
+                         "peak_source": f"{pk['src']} bf16 burst x 2 (dense FP8/BF16 nominal ratio)",
+                         "frac_of_cublas_fp8": round(tf / fp8_cublas, 4) if fp8_cublas else None}}
         rows[f"fp8_row_quant_{M}x{K}"] = {
             "value": round(rq_bytes / (t_rq * 1e-3) / 1e9, 1), "unit": "GB/s", "us": round(t_rq * 1e3, 1),
             "frac_hbm": round(rq_bytes / (t_rq * 1e-3) / 1e9 / pk["hbm"], 4)}
@@ -349,6 +391,21 @@ def measure_rows(args, dev, pk):
     if "quantize" in want:
         rows["w4_quantize_8b_set"] = quantizer_full_set(args, dev)
     return rows
+
+
+def measure_fp8_cublas(dev, n=8192, reps=10):
+    """Dense FP8 GEMM throughput of cuBLAS on this GPU (context for the FP8 rows)."""
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    one = torch.tensor(1.0, device=dev)
+
+    def mm(i):
+        torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+    mm(0)
+    best = min(time_region(mm, 1) for _ in range(reps))
+    del a, b
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
 
 
 def moe_rows(args, dev, fp8_peak, rows):
