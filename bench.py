@@ -127,6 +127,21 @@ class Clocks:
 
 # ------------------------------------------------------------------ timing helpers
 
+def max_over_ranks(vals, dev):
+    """Element-wise maximum of a list of floats over all ranks (the job's time is its
+    slowest rank's); identity without a process group."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return list(vals)
+    t = torch.tensor(vals, dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world, units_per_rank_step, ms_step):
+    """Whole-job throughput: the units all ranks processed per step over the (max) step time."""
+    return world * units_per_rank_step / (ms_step * 1e-3)
+
+
 def time_region(fn, iters, stream=None):
     """Device time (ms) of `iters` calls of fn, CUDA events on the launching stream."""
     stream = stream or torch.cuda.current_stream()
@@ -234,11 +249,9 @@ def run_ours(args, rank, world, dev):
         ms = time_region(dec.step, args.steps, stream)
     if dist:
         torch.distributed.barrier()
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks([ms], dev)[0]
     ms_step = ms / args.steps
-    value = world * dec.bytes_per_step / (ms_step * 1e-3) / 1e9
+    value = job_throughput(world, dec.bytes_per_step, ms_step) / 1e9
 
     # per-shape launch times (graph replays of one shape's GEMV, events around the block)
     per_shape = {}
@@ -279,11 +292,8 @@ def run_ours(args, rank, world, dev):
     for i in range(args.warmup):
         e2e_step(i)
     e2e_ms = time_region(e2e_step, args.steps, stream) / args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = world * dec.bytes_per_step / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks([e2e_ms], dev)[0]
+    e2e_val = job_throughput(world, dec.bytes_per_step, e2e_ms) / 1e9
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -302,7 +312,9 @@ def run_ours(args, rank, world, dev):
         "clocks": clk.summary(),
         "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
     }
-    if not args.headline_only:
+    # the other rows are single-GPU measurements: taken at N = 1 only, so that a scaling run
+    # times the headline alone
+    if not args.headline_only and world == 1:
         out["rows"] = measure_rows(args, dev, pk)
     del dec
     torch.cuda.empty_cache()
