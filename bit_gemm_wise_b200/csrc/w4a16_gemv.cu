@@ -362,29 +362,50 @@ __global__ void __launch_bounds__(W1 * 32, 1) gemv1_kernel(const Args a) {
     const int nck = (int)(Uc * 4);
     const uint32_t sub = a.sub, stage_bytes = SU * (512 + sub);
 
-    // this warp's contiguous run [wt0, wt1) of the CTA's units, in stages of SU units
+    // this warp's contiguous run [wt0, wt1) of the CTA's units, cut into stages of at most SU
+    // units that never cross an octet boundary (so a stage has one octet and one flush)
     const uint32_t n = t1 - t0;
     const uint32_t wt0 = t0 + (uint32_t)(((uint64_t)n * warp) / W);
     const uint32_t wt1 = t0 + (uint32_t)(((uint64_t)n * (warp + 1)) / W);
-    const uint32_t nst = (wt1 - wt0 + SU - 1) / SU;
     uint8_t *wring = ring + (size_t)warp * NS * stage_bytes;
     uint64_t *wbar = bars + warp * NS;
-
-    // lane 0 fills stage j of this warp's run into ring slot j % NS
-    auto issue = [&](uint32_t j) {
-        const uint32_t u0 = wt0 + j * SU;
-        const uint32_t cnt = (wt1 - u0) < (uint32_t)SU ? (wt1 - u0) : (uint32_t)SU;
-        uint8_t *dst = wring + (j % NS) * stage_bytes;
-        uint64_t *bar = wbar + (j % NS);
+    struct Cursor {
+        uint32_t t, o, u;  // next unit, its octet and its position in the octet
+    };
+    auto stage_len = [&](const Cursor &q) {
+        uint32_t cnt = wt1 - q.t;
+        cnt = cnt < (uint32_t)SU ? cnt : (uint32_t)SU;
+        return cnt < Uc - q.u ? cnt : Uc - q.u;
+    };
+    auto advance = [&](Cursor &q, uint32_t cnt) {
+        q.t += cnt;
+        q.u += cnt;
+        if (q.u == Uc) { q.u = 0; ++q.o; }
+    };
+    Cursor cons;
+    cons.t = wt0;
+    cons.o = fdiv(wt0, a.divU);
+    cons.u = wt0 - cons.o * Uc;
+    Cursor prod = cons;
+    uint32_t jp = 0;  // stages issued
+    // lane 0 fills the producer cursor's next stage into ring slot jp % NS
+    auto issue = [&]() {
+        const uint32_t cnt = stage_len(prod);
+        uint8_t *dst = wring + (jp % NS) * stage_bytes;
+        uint64_t *bar = wbar + (jp % NS);
         mbar_arrive_expect_tx(bar, cnt * (512 + sub));
-        bulk_g2s(dst, a.codes + (size_t)u0 * 512, cnt * 512, bar);
-        bulk_g2s(dst + SU * 512, a.scales + (size_t)u0 * sub, cnt * sub, bar);
+        bulk_g2s(dst, a.codes + (size_t)prod.t * 512, cnt * 512, bar);
+        bulk_g2s(dst + SU * 512, a.scales + (size_t)prod.t * sub, cnt * sub, bar);
     };
     // ---- the weight stream does not depend on earlier kernels: start it first
     if (lane == 0) {
         for (int j = 0; j < NS; ++j) mbar_init(wbar + j, 1);
         fence_mbar_init();
-        for (uint32_t j = 0; j < (uint32_t)NS && j < nst; ++j) issue(j);
+    }
+    for (int j = 0; j < NS && prod.t < wt1; ++j) {  // warp-uniform cursor, lane 0 issues
+        if (lane == 0) issue();
+        advance(prod, stage_len(prod));
+        ++jp;
     }
     for (int i = tid; i < a.nol * W * 8; i += THREADS) slot[i] = 0.0f;
     // activations may be written by the previous kernel in the stream
@@ -412,11 +433,11 @@ __global__ void __launch_bounds__(W1 * 32, 1) gemv1_kernel(const Args a) {
     const int per_unit = 128 / a.g;
     const uint32_t sc_lane = (uint32_t)(r * per_unit + (cc * 32) / a.g);  // u32 index in a unit's scales
     float y[1] = {0.0f};
-    uint32_t o = fdiv(wt0, a.divU), u = wt0 - o * Uc;
-    uint32_t cur_ol = 0xffffffffu;  // set by the first (checked) stage
+    uint32_t cur_ol = 0xffffffffu;
     const bool kpad = (Kc & 127u) != 0;
     bool ok = true;
-    for (uint32_t j = 0; j < nst && ok; ++j) {
+    uint32_t j = 0;  // stages consumed
+    for (; cons.t < wt1; ++j) {
         const uint32_t sl = j % NS;
         // lane 0 polls; every lane then takes the (now immediate) wait for its own acquire
         bool got = true;
@@ -424,44 +445,36 @@ __global__ void __launch_bounds__(W1 * 32, 1) gemv1_kernel(const Args a) {
         got = __shfl_sync(FULL, got ? 1 : 0, 0) != 0;
         if (!got) { ok = false; break; }
         (void)mbar_try_wait(wbar + sl, (j / NS) & 1u);
+        const uint32_t cnt = stage_len(cons);
+        const uint32_t ol = cons.o - o_first;
+        if (ol != cur_ol) {
+            if (cur_ol != 0xffffffffu) flush_octet<1, W>(cur_ol, y, slot, warp, lane);
+            cur_ol = ol;
+        }
         const uint8_t *st = wring + sl * stage_bytes;
-        const uint32_t u0 = wt0 + j * SU;
-        const uint32_t cnt = (wt1 - u0) < (uint32_t)SU ? (wt1 - u0) : (uint32_t)SU;
         const uint4 *cw = reinterpret_cast<const uint4 *>(st) + lane;
         const uint32_t *sw = reinterpret_cast<const uint32_t *>(st + SU * 512) + sc_lane;
-        if (cnt == (uint32_t)SU && u + SU <= Uc && o - o_first == cur_ol && !kpad) {
-            // fast path: a full stage inside the current octet, no padding chunks
-            const uint32_t k0 = u * 128u + (uint32_t)cc * 32u;
-            const uint4 *xp = reinterpret_cast<const uint4 *>(xb + xb_index(k0));
-            const float *sxp = sx + (k0 >> 5);
+        const uint32_t k0 = cons.u * 128u + (uint32_t)cc * 32u;
+        const uint4 *xp = reinterpret_cast<const uint4 *>(xb + xb_index(k0));
+        const float *sxp = sx + (k0 >> 5);
 #pragma unroll
-            for (int i = 0; i < SU; ++i)
+        for (int i = 0; i < SU; ++i)
+            if ((uint32_t)i < cnt && (!kpad || k0 + (uint32_t)i * 128u < Kc))
                 unit_m1(y[0], cw[i * 32], sw[i * (sub >> 2)], xp + i * 20, sxp[i * 4]);
-            u += SU;
-            if (u == Uc) { u = 0; ++o; }
-        } else {
-            for (uint32_t i = 0; i < cnt; ++i) {
-                const uint32_t ol = o - o_first;
-                if (ol != cur_ol) {
-                    if (cur_ol != 0xffffffffu) flush_octet<1, W>(cur_ol, y, slot, warp, lane);
-                    cur_ol = ol;
-                }
-                const uint32_t k0 = u * 128u + (uint32_t)cc * 32u;
-                if (++u == Uc) { u = 0; ++o; }
-                if (k0 >= Kc) continue;
-                unit_m1(y[0], cw[i * 32], sw[i * (sub >> 2)], reinterpret_cast<const uint4 *>(xb + xb_index(k0)),
-                        sx[k0 >> 5]);
-            }
-        }
-        // every lane has read the slot: lane 0 refills it with stage j + NS
+        advance(cons, cnt);
+        // every lane has read the slot: lane 0 refills it with the next stage
         __syncwarp();
-        if (lane == 0 && j + NS < nst) issue(j + NS);
+        if (prod.t < wt1) {
+            if (lane == 0) issue();
+            advance(prod, stage_len(prod));
+            ++jp;
+        }
     }
     if (cur_ol != 0xffffffffu) flush_octet<1, W>(cur_ol, y, slot, warp, lane);
-    // no bulk copy may still be in flight when the CTA exits: on a failed wait, wait (bounded)
-    // for the copies this warp issued
+    // no bulk copy may still be in flight when the CTA exits: after a failed wait, wait
+    // (bounded) for every stage this warp issued and did not consume
     if (!ok && lane == 0)
-        for (uint32_t j = 0; j < nst && j < (uint32_t)NS; ++j) (void)mbar_wait_bounded(wbar + j, 0, a.status);
+        for (uint32_t q = j; q < jp; ++q) (void)mbar_wait_bounded(wbar + q % NS, (q / NS) & 1u, a.status);
     __syncthreads();
     finish<1, W>(a, slot, flags, c, t0, t1, o_first, o_last, tid);
 }
