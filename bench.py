@@ -51,8 +51,8 @@ def peaks():
 # the kernel's source file at capture time: a number is reported only while the source is
 # unchanged (otherwise the counters describe a different kernel and "traffic" is null).
 NCU_TRAFFIC = {
-    # profiles/w4a16_gemv_m1_k4096_n14336_full.md
-    "w4a16_gemv M1 K4096xN14336": {"bytes": 31242496, "sha1": "961edcf2b56045a28adb7b1a1672443968c1c9a7"},
+    # profiles/w4a16_gemv_m1_k14336_n4096_full.md
+    "w4a16_gemv M1 K14336xN4096": {"bytes": 31281920, "sha1": "d93d79618f5921b63c0af20b0cd088e89948c139"},
 }
 
 
@@ -273,6 +273,7 @@ def run_ours(args, rank, world, dev):
                 "traffic": traffic_for(f"w4a16_gemv M1 {dom}", "bit_gemm_wise_b200/csrc/w4a16_gemv.cu"),
                 "kernel": f"w4a16_gemv M=1 {dom}", "bytes_per_launch": dbytes,
                 "peak_source": f"{pk['src']} copy bandwidth (of {pk['src']})",
+                "frac_of_spec_8000": round(dach / 8000.0, 4),
                 "step_frac": round(value / world / pk["hbm"], 4)}
 
     # e2e through the public Python API with host buffers, every step: pinned h2d of the
@@ -291,9 +292,23 @@ def run_ours(args, rank, world, dev):
 
     for i in range(args.warmup):
         e2e_step(i)
-    e2e_ms = time_region(e2e_step, args.steps, stream) / args.steps
-    e2e_ms = max_over_ranks([e2e_ms], dev)[0]
+    eager_ms = time_region(e2e_step, args.steps, stream) / args.steps
+    # the same step captured once per weight copy as a CUDA graph (pinned-host copies of x in,
+    # the four API calls, copies of y out), replayed as a serving loop would
+    e2e_graphs = []
+    side = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    for r in range(dec.R):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=side):
+            e2e_step(r)
+        e2e_graphs.append(gr)
+    for i in range(args.warmup):
+        e2e_graphs[i % dec.R].replay()
+    e2e_ms = time_region(lambda i: e2e_graphs[i % dec.R].replay(), args.steps, stream) / args.steps
+    e2e_ms, eager_ms = max_over_ranks([e2e_ms, eager_ms], dev)
     e2e_val = job_throughput(world, dec.bytes_per_step, e2e_ms) / 1e9
+    eager_val = job_throughput(world, dec.bytes_per_step, eager_ms) / 1e9
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -310,10 +325,14 @@ def run_ours(args, rank, world, dev):
         "per_shape": per_shape,
         "gpu_launches": dec.launches_per_step * args.steps,
         "clocks": clk.summary(),
-        "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "per step: pinned-host copies of the activations in, the four w4a16_gemv API calls, "
+                       "copies of the outputs out, replayed from a CUDA graph",
+                "eager_value": round(eager_val, 1)},
     }
     # the other rows are single-GPU measurements: taken at N = 1 only, so that a scaling run
     # times the headline alone
+    del e2e_graphs
     if not args.headline_only and world == 1:
         out["rows"] = measure_rows(args, dev, pk)
     del dec
@@ -333,16 +352,50 @@ def measure_rows(args, dev, pk):
     fp8_peak = 2.0 * pk["bf16"]  # dense FP8 = 2x dense BF16 (nominal ratio), burst
     want = set(args.rows.split(",")) if args.rows else set(ROW_GROUPS)
 
-    # GEMV at M = 4 and 16 (ALU-bound on the CUDA cores)
+    # GEMV at M = 4 and 16 (bound by the CUDA cores' issue rate): GB/s, and the FMA work as a
+    # fraction of the CUDA-core fp32 FMA peak (148 SMs x 128 lanes x 2 flop x 1965 MHz)
+    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
     for M in ((4, 16) if "gemv" in want else ()):
         d = Decode(M, args.seed, dev)
         d.capture()
         d.step(0)
         ms = time_region(d.step, 6 * d.R) / (6 * d.R)
+        flops = sum(2.0 * M * N * K for K, N in d.shapes)
         rows[f"w4a16_gemv_M{M}"] = {"value": round(d.bytes_per_step / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                                     "us_per_step": round(ms * 1e3, 2),
-                                    "frac_hbm": round(d.bytes_per_step / (ms * 1e-3) / 1e9 / pk["hbm"], 4)}
+                                    "frac_hbm": round(d.bytes_per_step / (ms * 1e-3) / 1e9 / pk["hbm"], 4),
+                                    "fp32_fma_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                                    "frac_fp32_fma_peak": round(flops / (ms * 1e-3) / 1e12 / fp32_peak, 4)}
         del d
+
+    # single linear layer (K=576, N=1536, group 32 symmetric, M=1): launch-latency-dominated,
+    # reported in microseconds
+    if "gemv" in want:
+        c = synth.SINGLE_LAYER
+        N, K, g = c["N"], c["K"], c["group"]
+        W, x = synth.single_layer(args.seed, device=dev)
+        codes, scales, _, _ = w4.alloc_quantized(N, K, g, "sym", device=dev, chosen=False)
+        w4.w4_quantize(W, N, K, g, "sym", [1.0], codes, scales, None, None)
+        packed = w4.alloc_packed(N, K, g, w4.W4_LAYOUT_GEMV, device=dev)
+        w4.w4_prepack(codes, scales, None, N, K, g, "sym", w4.W4_LAYOUT_GEMV, packed)
+        y = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+        ws = w4.alloc_gemv_workspace(N, K, g, device=dev)
+
+        def one(i):
+            w4.w4a16_gemv(x, 1, packed, N, K, g, "sym", y, 0, ws)
+
+        one(0)
+        gr = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        with torch.cuda.graph(gr, stream=side):
+            for _ in range(20):
+                one(0)
+        gr.replay()
+        us = time_region(lambda i: gr.replay(), 10) / 200 * 1e3
+        rows["w4a16_gemv_single_layer"] = {"value": round(us, 2), "unit": "us per call",
+                                           "GBps": round(gemv_bytes(1, N, K, g) / (us * 1e-6) / 1e9, 1),
+                                           "note": "0.5 MB problem: launch and latency bound, not a roofline row"}
+        del W, x, codes, scales, packed, y, ws
 
     # context for the FP8 rows: cuBLAS FP8 GEMM (torch._scaled_mm, e4m3, 8192^3, best of 10)
     fp8_cublas = None
@@ -388,7 +441,8 @@ def measure_rows(args, dev, pk):
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4),
                          "peak_source": f"{pk['src']} bf16 burst x 2 (dense FP8/BF16 nominal ratio)",
-                         "frac_of_cublas_fp8": round(tf / fp8_cublas, 4) if fp8_cublas else None}}
+                         "frac_of_cublas_fp8": round(tf / fp8_cublas, 4) if fp8_cublas else None,
+                         "frac_of_spec_4500": round(tf / 4500.0, 4)}}
         rows[f"fp8_row_quant_{M}x{K}"] = {
             "value": round(rq_bytes / (t_rq * 1e-3) / 1e9, 1), "unit": "GB/s", "us": round(t_rq * 1e3, 1),
             "frac_hbm": round(rq_bytes / (t_rq * 1e-3) / 1e9 / pk["hbm"], 4)}
