@@ -181,6 +181,48 @@ __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
                  : "memory");
 }
 
+// 32 lanes x 16 columns of 32-bit values from registers into TMEM (one column per register)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float2 *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "f"(v[0].x), "f"(v[0].y), "f"(v[1].x), "f"(v[1].y), "f"(v[2].x), "f"(v[2].y), "f"(v[3].x), "f"(v[3].y),
+        "f"(v[4].x), "f"(v[4].y), "f"(v[5].x), "f"(v[5].y), "f"(v[6].x), "f"(v[6].y), "f"(v[7].x), "f"(v[7].y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Transpose 8x8 blocks of 16-bit values held by each aligned group of 8 lanes: lane l holds
+// row l as R[k] = (col 2k, col 2k+1); afterwards it holds column l as R[k] = (row 2k, row 2k+1).
+// Butterfly stages over lane distance 4 and 2 swap 32-bit pairs; distance 1 swaps halves.
+__device__ __forceinline__ void transpose8x8_b16(uint32_t (&R)[4], int lane) {
+    const int l = lane & 7;
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {  // distance 4: registers (0, 2) and (1, 3)
+        const bool up = (l & 4) != 0;
+        const uint32_t recv = __shfl_xor_sync(FULL, up ? R[p] : R[p + 2], 4);
+        if (up) R[p] = recv;
+        else R[p + 2] = recv;
+    }
+#pragma unroll
+    for (int p = 0; p < 4; p += 2) {  // distance 2: registers (0, 1) and (2, 3)
+        const bool up = (l & 2) != 0;
+        const uint32_t recv = __shfl_xor_sync(FULL, up ? R[p] : R[p + 1], 2);
+        if (up) R[p] = recv;
+        else R[p + 1] = recv;
+    }
+    const bool odd = (l & 1) != 0;
+#pragma unroll
+    for (int p = 0; p < 4; p += 2) {  // distance 1: 16-bit halves of registers (p, p + 1)
+        const uint32_t recv = __shfl_xor_sync(FULL, __byte_perm(R[p], R[p + 1], odd ? 0x5410 : 0x7632), 1);
+        const uint32_t a = __byte_perm(odd ? recv : R[p], odd ? R[p] : recv, odd ? 0x7610 : 0x5410);
+        const uint32_t b = __byte_perm(odd ? recv : R[p + 1], odd ? R[p + 1] : recv, odd ? 0x7632 : 0x7610);
+        R[p] = a;
+        R[p + 1] = b;
+    }
+}
+
 // acc[i] += s * (p[2i], p[2i+1]) with the packed fp32 FMA of sm_100 (two lanes per instruction)
 __device__ __forceinline__ void promote16(float2 *acc, float2 s, const uint32_t (&p)[16]) {
 #pragma unroll
@@ -392,6 +434,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
             uint32_t ent0 = scales[n], ent1 = (J > 1) ? scales[a.Npad + n] : 0u;
+            int bl = 0;           // TMEM buffer of the tile's last group
+            uint32_t tl_addr = 0;  // this warp's columns in it
             for (int j = 0; j <= J && ok; ++j, ++jg) {
                 const int b = (int)(jg % NBUF);
                 float s512 = -1.0f;  // group J is the zero-point term, subtracted
@@ -417,23 +461,79 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                     if (c + 2 < 8) tmem_ld16(taddr + (c + 2) * 16, pa);
                     promote16(acc + (c + 1) * 8, s2, pb);
                 }
+                if (j == J) {
+                    // the tile's last group: its buffer holds the tile's result for the epilogue
+                    // below and is released after it
+                    bl = b;
+                    tl_addr = taddr;
+                    continue;  // ends the loop (j > J) with jg counted
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
             }
             if (!ok) break;
-            const bool row_ok = n < a.N;
+            // Epilogue. The result goes through the last group's TMEM buffer so that the store
+            // loop can stay rolled (an unrolled 128-column loop runs once per tile and its code
+            // is fetched cold every time): 8 stores of 16 columns, then per 16-column chunk one
+            // load, the row scale (lane-held, broadcast by shuffle) and the global stores.
 #pragma unroll
-            for (int i = 0; i < 128; ++i) {
-                const float rs = __shfl_sync(FULL, rsv[i >> 5], i & 31);
-                const int col = half * 128 + i;
-                const int64_t m = T.row0 + col;
-                if (row_ok && col < T.rows && m < a.M) {
-                    const float v = ((i & 1) ? acc[i >> 1].y : acc[i >> 1].x) * rs;
-                    if (a.out_fp32) static_cast<float *>(a.Y)[m * a.N + n] = v;
-                    else static_cast<__nv_bfloat16 *>(a.Y)[m * a.N + n] = __float2bfloat16_rn(v);
+            for (int c = 0; c < 8; ++c) tmem_st16(tl_addr + c * 16, acc + c * 8);
+            tmem_wait_st();
+            const bool row_ok = n < a.N;
+            const int64_t lim = (T.rows < (int64_t)BN ? T.rows : (int64_t)BN);  // valid columns of the tile
+            const int64_t lim_m = a.M - T.row0;
+            const int64_t ncol = (lim < lim_m ? lim : lim_m) - half * 128;      // valid columns of this half
+            // bf16 output with N a multiple of 8: 8x8 transposes across lanes, so that each lane
+            // stores 8 consecutive outputs of one token row (16-byte stores); otherwise one value
+            // per lane and store
+            const bool vec = !a.out_fp32 && (a.N & 7) == 0;
+            const int64_t nbase = T.n0 + quarter * 32 + 8 * (lane >> 3);  // first row of the lane's group
+            const int li = lane & 7;
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+                uint32_t v[16];
+                tmem_ld16(tl_addr + c * 16, v);
+                tmem_wait_ld16(v);
+                const float rsc = (c >> 1) == 0 ? rsv[0] : (c >> 1) == 1 ? rsv[1] : (c >> 1) == 2 ? rsv[2] : rsv[3];
+                const int64_t m0 = T.row0 + half * 128 + c * 16;
+                const int l0 = (c & 1) * 16;
+                if (vec) {
+                    uint32_t h0[4], h1[4];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float r0 = __shfl_sync(FULL, rsc, l0 + 2 * q), r1 = __shfl_sync(FULL, rsc, l0 + 2 * q + 1);
+                        const __nv_bfloat162 b2 =
+                            __floats2bfloat162_rn(__uint_as_float(v[2 * q]) * r0, __uint_as_float(v[2 * q + 1]) * r1);
+                        const uint32_t w = *reinterpret_cast<const uint32_t *>(&b2);
+                        if (q < 4) h0[q] = w;
+                        else h1[q - 4] = w;
+                    }
+                    transpose8x8_b16(h0, lane);
+                    transpose8x8_b16(h1, lane);
+                    if (nbase < a.N) {
+                        __nv_bfloat16 *yb = static_cast<__nv_bfloat16 *>(a.Y);
+                        if (c * 16 + li < ncol)
+                            *reinterpret_cast<uint4 *>(yb + (m0 + li) * a.N + nbase) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+                        if (c * 16 + 8 + li < ncol)
+                            *reinterpret_cast<uint4 *>(yb + (m0 + 8 + li) * a.N + nbase) =
+                                make_uint4(h1[0], h1[1], h1[2], h1[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float rs = __shfl_sync(FULL, rsc, l0 + k);
+                        if (row_ok && c * 16 + k < ncol) {
+                            const float val = __uint_as_float(v[k]) * rs;
+                            if (a.out_fp32) static_cast<float *>(a.Y)[(m0 + k) * a.N + n] = val;
+                            else static_cast<__nv_bfloat16 *>(a.Y)[(m0 + k) * a.N + n] = __float2bfloat16_rn(val);
+                        }
+                    }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->acc_empty[bl]);
         }
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
