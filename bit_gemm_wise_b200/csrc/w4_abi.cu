@@ -58,3 +58,26 @@ W4_API w4_status w4_device_status(cudaStream_t stream, int *code_out) {
     *code_out = v;
     return W4_OK;
 }
+
+// ------------------------------------------------------------------ bounded-wait self-test
+namespace w4 {
+
+// One thread initializes an mbarrier that expects one arrival and waits for its first phase
+// without ever arriving: the bounded wait must expire, record W4_ERR_TIMEOUT and return.
+__global__ void selftest_wait_kernel(uint64_t limit_ns, int *status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    (void)mbar_wait_bounded(&bar, 0, status, limit_ns);
+}
+
+}  // namespace w4
+
+W4_API w4_status w4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t stream) {
+    if (limit_ns < 1000 || limit_ns > 1000000000LL) return W4_ERR_ARG;
+    int *status = w4::device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    w4::selftest_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_ns, status);
+    return w4::launch_status();
+}

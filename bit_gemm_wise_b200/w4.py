@@ -44,6 +44,7 @@ SIGNATURES = [
     ("w4a8_gemm", _I, [_P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
     ("w4a8_grouped_gemm", _I, [_P, _P, _P, _P, _I, _I64, _P, _I64, _I64, _I, _I, _P, _P]),
     ("w4_device_status", _I, [_P, ctypes.POINTER(ctypes.c_int)]),
+    ("w4_selftest_bounded_wait", _I, [_I64, _P]),
 ]
 
 _lib = None
@@ -179,6 +180,11 @@ def w4_device_status(stream=None) -> int:
     rc = lib().w4_device_status(_stream(stream), ctypes.byref(code))
     _check("w4_device_status", rc)
     return code.value
+
+
+def w4_selftest_bounded_wait(limit_ns, stream=None):
+    """Launch a bounded wait that must expire (diagnostic of the kernels' failure path)."""
+    _check("w4_selftest_bounded_wait", lib().w4_selftest_bounded_wait(int(limit_ns), _stream(stream)))
 
 
 # ------------------------------------------------------------------ allocation helpers

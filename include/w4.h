@@ -252,6 +252,17 @@ w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale,
  */
 w4_status w4_device_status(cudaStream_t stream, int *code_out);
 
+/*
+ * w4_selftest_bounded_wait -- diagnostic (no counterpart in the source pages): launches one
+ *   block whose thread waits, with the same bounded mbarrier wait the W4A8 GEMM and the
+ *   W4A16 GEMV use, for a barrier phase that nothing completes. After limit_ns nanoseconds
+ *   (1e3 .. 1e9) the wait gives up and records W4_ERR_TIMEOUT in the device status word, and
+ *   the kernel returns normally; the context stays usable. It lets a test check the failure
+ *   path of every bounded wait without faulting or hanging a GPU.
+ *   Errors: ARG (limit out of range) / CUDA (launch).
+ */
+w4_status w4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
