@@ -416,12 +416,14 @@ def measure_rows(args, dev, pk):
         X8, sa, _, gop = w4.alloc_row_quant(M, K, 128, device=dev, group_sums=False)
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        ws = w4.alloc_gemm_workspace(M, N, K, 128, device=dev)
+        sched = w4.w4a8_gemm_schedule(M, N, K, 128, torch.cuda.get_device_properties(dev).multi_processor_count)
 
         def rq(i):
             w4.fp8_row_quant(X, M, K, 128, X8, sa, None, gop)
 
         def gemm(i):
-            w4.w4a8_gemm(X8, sa, gop, M, packed, N, K, 128, "asym", Y, 0)
+            w4.w4a8_gemm(X8, sa, gop, M, packed, N, K, 128, "asym", Y, 0, ws)
 
         rq(0); gemm(0)
         n = 10
@@ -438,6 +440,7 @@ def measure_rows(args, dev, pk):
         rq_bytes = M * K * 2 + M * K + M * 4 + gop.numel() * 2
         rows[f"w4a8_gemm_{K}x{N}"] = {
             "value": round(tf, 1), "unit": "TFLOP/s", "us": round(t_gemm * 1e3, 1),
+            "tiles": sched["tiles"], "split_tiles": sched["split_tiles"],
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4),
                          "peak_source": f"{pk['src']} bf16 burst x 2 (dense FP8/BF16 nominal ratio)",
@@ -448,7 +451,7 @@ def measure_rows(args, dev, pk):
             "frac_hbm": round(rq_bytes / (t_rq * 1e-3) / 1e9 / pk["hbm"], 4)}
         rows[f"w4a8_rowquant_plus_gemm_{K}x{N}"] = {
             "value": round(flops / ((t_gemm + t_rq) * 1e-3) / 1e12, 1), "unit": "TFLOP/s"}
-        del W, codes, scales, zeros, packed, X, X8, sa, gop, Y, flush
+        del W, codes, scales, zeros, packed, X, X8, sa, gop, Y, flush, ws
         torch.cuda.empty_cache()
 
     # MoE grouped GEMM (32 experts, top-4 of 4096 tokens, group 32)

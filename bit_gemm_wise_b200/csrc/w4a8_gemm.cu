@@ -87,7 +87,45 @@ struct Args {
     int MTU;                       // token tiles (upper bound for grouped problems)
     int KT;                        // raw stages per tile
     int ZT;                        // zero-point pseudo-stages per tile
+    int64_t DPT;                   // tiles [0, DPT) are whole-tile work, strided over the grid
+    int64_t R;                     // tiles [DPT, DPT + R) are split along K over PS CTAs
+    int64_t PS;
+    float *part;                   // split tiles: 2 PS partial-result slots (PART_FLOATS each)
+    uint32_t *cnt;                 // split tiles: R x 8 arrival counters (zero between calls)
 };
+
+// ------------------------------------------------------------------ split-K schedule
+// The last, partial wave of tiles is spread over the CTAs along K: its R tiles form R*KT
+// k-blocks in tile-major order, and CTA c takes the contiguous range
+// [c*Q/PS, (c+1)*Q/PS) of them (Q = R*KT). With R <= PS a range covers at most two tiles, so
+// a CTA has at most two segments. Each segment's fp32 partial sum goes to the CTA's slot
+// 2c + (0 for the first segment, 1 for the second); the last contributor to arrive (per
+// promotion warp, counted in the workspace) adds the partials of the tile in CTA order and
+// stores the result, so the result does not depend on arrival order.
+constexpr int PART_FLOATS = BM * BN;  // one slot: the 128 x 256 fp32 tile
+
+__host__ __device__ __forceinline__ int64_t split_begin(int64_t Q, int64_t PS, int64_t c) { return c * Q / PS; }
+
+// the CTA whose range holds k-block q: the largest c with split_begin(c) <= q
+__host__ __device__ __forceinline__ int64_t split_cta_of(int64_t Q, int64_t PS, int64_t q) {
+    return ((q + 1) * PS + Q - 1) / Q - 1;
+}
+
+// partial-result slot of contributor c to split tile i
+__host__ __device__ __forceinline__ int64_t split_slot(int64_t Q, int64_t PS, int KT, int64_t c, int64_t i) {
+    return 2 * c + (split_begin(Q, PS, c) / KT == i ? 0 : 1);
+}
+
+// the segment that starts at k-block q of a range ending at q1: split tile i, k-blocks
+// [kb0, kb1) of it; returns the start of the next segment
+__host__ __device__ __forceinline__ int64_t split_segment(int64_t q, int64_t q1, int KT, int64_t &i, int &kb0,
+                                                          int &kb1) {
+    i = q / KT;
+    const int64_t e = (i + 1) * KT < q1 ? (i + 1) * KT : q1;
+    kb0 = (int)(q - i * KT);
+    kb1 = (int)(e - i * KT);
+    return e;
+}
 
 __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, Smem *sm, int *status) {
     return mbar_wait_abortable(bar, parity, &sm->abort, status, kWaitNs);
@@ -280,6 +318,99 @@ __device__ __forceinline__ bool locate_tile(const Args &a, int64_t t, Tile &T) {
     return false;
 }
 
+// One unit of a CTA's work: k-blocks [kb0, kb1) of tile t, followed by the zero-point
+// pseudo-stages when z. seg < 0: a whole tile, stored directly; otherwise the ordinal (0 or 1)
+// of a split-tile segment in this CTA's range.
+struct Item {
+    int64_t t;
+    int kb0, kb1;
+    int seg;
+    bool z;
+};
+
+// The sequence of items of this CTA, identical for every role: its whole tiles, then its
+// split-tile segments.
+struct Work {
+    int64_t t, q, q1;
+    int seg = 0;
+    __device__ __forceinline__ explicit Work(const Args &a) {
+        t = blockIdx.x;
+        const int64_t Q = a.R * a.KT;
+        q = blockIdx.x < a.PS ? split_begin(Q, a.PS, blockIdx.x) : 0;
+        q1 = blockIdx.x < a.PS ? split_begin(Q, a.PS, blockIdx.x + 1) : 0;
+    }
+    __device__ __forceinline__ bool next(const Args &a, Item &it) {
+        if (t < a.DPT) {
+            it.t = t;
+            it.kb0 = 0;
+            it.kb1 = a.KT;
+            it.seg = -1;
+            it.z = true;
+            t += gridDim.x;
+            return true;
+        }
+        if (q < q1) {
+            int64_t i;
+            q = split_segment(q, q1, a.KT, i, it.kb0, it.kb1);
+            it.t = a.DPT + i;
+            it.seg = seg++;
+            it.z = it.kb1 == a.KT;  // the segment that ends the tile also adds its zero-point term
+            return true;
+        }
+        return false;
+    }
+};
+
+// Split tile, promotion warp wq (weight rows 32*(wq&3).., token columns 128*(wq>>2)..): store
+// this warp's partial sum in the CTA's slot and count it. The warp whose arrival completes the
+// count reads every contributor's partial of its part, in CTA order, into acc, resets the
+// counter for the next call and returns true; the others return false.
+// Slot layout: [8 warps][32 column quads][32 lanes] float4, so that each store or load of a
+// warp covers 512 contiguous bytes.
+__device__ __forceinline__ bool split_combine(const Args &a, const Item &it, int wq, int lane, float2 (&acc)[64]) {
+    const int64_t Q = a.R * a.KT;
+    const int64_t i = it.t - a.DPT, me = blockIdx.x;
+    const int64_t c0 = split_cta_of(Q, a.PS, i * a.KT), c1 = split_cta_of(Q, a.PS, i * a.KT + a.KT - 1);
+    const int64_t slot = 2 * me + it.seg;
+    if (i < 0 || i >= a.R || c0 < 0 || me < c0 || me > c1 || c1 >= a.PS || split_slot(Q, a.PS, a.KT, me, i) != slot) {
+        if (lane == 0) record_status(a.status, W4_ERR_DEVICE_CHECK);
+        return false;
+    }
+    float4 *mine = reinterpret_cast<float4 *>(a.part) + (slot * 8 + wq) * 1024 + lane;
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+        __stcg(mine + k * 32, make_float4(acc[2 * k].x, acc[2 * k].y, acc[2 * k + 1].x, acc[2 * k + 1].y));
+    __threadfence();
+    __syncwarp();
+    uint32_t *ctr = a.cnt + i * 8 + wq;
+    uint32_t old = 0;
+    if (lane == 0) old = atomicAdd(ctr, 1u);
+    old = __shfl_sync(FULL, old, 0);
+    if (old != (uint32_t)(c1 - c0)) return false;
+    __threadfence();
+    for (int64_t c = c0; c <= c1; ++c) {
+        const float4 *src =
+            reinterpret_cast<const float4 *>(a.part) + (split_slot(Q, a.PS, a.KT, c, i) * 8 + wq) * 1024 + lane;
+        const bool first = c == c0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // 16 loads in flight per lane, then the adds
+            float4 v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = __ldcg(src + (h * 16 + k) * 32);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float2 &x = acc[2 * (h * 16 + k)], &y = acc[2 * (h * 16 + k) + 1];
+                x.x = (first ? 0.0f : x.x) + v[k].x;
+                x.y = (first ? 0.0f : x.y) + v[k].y;
+                y.x = (first ? 0.0f : y.x) + v[k].z;
+                y.y = (first ? 0.0f : y.y) + v[k].w;
+            }
+        }
+    }
+    if (lane == 0) atomicExch(ctr, 0u);
+    return true;
+}
+
 template <int G>  // group size: 32, 64 or 128
 __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                           const __grid_constant__ CUtensorMap tm_act,
@@ -292,11 +423,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
     Smem *sm = reinterpret_cast<Smem *>(base + STAGES * (RAW_BYTES + A_BYTES));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t total_tiles = (int64_t)a.MTU * a.NT;
     constexpr int GPS = BK / G;    // groups per raw stage
     constexpr int KPG = G / 32;    // f8 MMAs (K = 32 each) per group
-    const int J = (int)(a.Kpad / G);
-    const int SPT = a.KT + a.ZT;   // pipeline stages per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -329,19 +457,22 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             Ring r;
             int64_t uses = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            Work w(a);
+            Item it;
+            while (ok && w.next(a, it)) {
                 Tile T;
-                if (!locate_tile(a, t, T)) continue;
-                for (int s = 0; s < SPT; ++s, r.next(), ++uses) {
+                if (!locate_tile(a, it.t, T)) continue;
+                const int send = it.kb1 + (it.z ? a.ZT : 0);
+                for (int s = it.kb0; s < send; ++s, r.next(), ++uses) {
                     const int slot = r.slot;
                     if (!wait_phase_short(&sm->empty[slot], r.phase ^ 1u, sm, a.status)) { ok = false; break; }
                     uint8_t *dst = raw + slot * RAW_BYTES;
-                    if (s < a.KT) {
+                    if (s < it.kb1) {
                         mbar_arrive_expect_tx(&sm->full[slot], C_BYTES + B_BYTES);
                         tma_load_3d(dst, &tm_codes, s * (BK / 2), (int)T.n0, T.e, &sm->full[slot]);
                         tma_load_2d(dst + C_BYTES, &tm_act, s * BK, (int)T.row0, &sm->full[slot]);
                     } else {
-                        const int z = s - a.KT;
+                        const int z = s - it.kb1;
                         mbar_arrive_expect_tx(&sm->full[slot], ZA_BYTES + ZB_BYTES);
                         tma_load_3d(dst, &tm_zop, z * ZKC, (int)T.n0, T.e, &sm->full[slot]);
                         tma_load_2d(dst + C_BYTES, &tm_gop, z * ZKC, (int)T.row0, &sm->full[slot]);
@@ -363,15 +494,18 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             uint32_t jg = 0;
             bool ok = true;
             const uint32_t aLo0 = desc_lo(smem_addr(sA)), rLo0 = desc_lo(smem_addr(raw));
-            for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            Work w(a);
+            Item it;
+            while (ok && w.next(a, it)) {
                 Tile T;
-                if (!locate_tile(a, t, T)) continue;
-                for (int s = 0; s < SPT && ok; ++s, r.next()) {
+                if (!locate_tile(a, it.t, T)) continue;
+                const int send = it.kb1 + (it.z ? a.ZT : 0);
+                for (int s = it.kb0; s < send && ok; ++s, r.next()) {
                     const int slot = r.slot;
                     if (!wait_phase_short(&sm->exp_full[slot], r.phase, sm, a.status)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t rLo = rLo0 + (uint32_t)slot * (RAW_BYTES >> 4);
-                    if (s < a.KT) {
+                    if (s < it.kb1) {
                         const uint32_t aLo = aLo0 + (uint32_t)slot * (A_BYTES >> 4), bLo = rLo + (C_BYTES >> 4);
 #pragma unroll
                         for (int gi = 0; gi < GPS; ++gi, ++jg) {
@@ -386,7 +520,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                         }
                     } else {
                         // zero-point term: all pseudo-stages of the tile accumulate into one buffer
-                        const int z = s - a.KT;
+                        const int z = s - it.kb1;
                         const uint32_t b = jg & 1u;
                         if (z == 0 && !wait_phase_short(&sm->acc_empty[b], ((jg >> 1) & 1u) ^ 1u, sm, a.status)) {
                             ok = false;
@@ -415,9 +549,11 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
         const int row = quarter * 32 + lane;
         int64_t jg = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        Work w(a);
+        Item it;
+        while (ok && w.next(a, it)) {
             Tile T;
-            if (!locate_tile(a, t, T)) continue;
+            if (!locate_tile(a, it.t, T)) continue;
             const int64_t n = T.n0 + row;
             const uint32_t *scales =
                 reinterpret_cast<const uint32_t *>(a.packed + (size_t)T.e * a.slab_bytes + a.codes_bytes);
@@ -433,16 +569,19 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             float2 acc[64];  // columns (2i, 2i+1) of this thread's weight row
 #pragma unroll
             for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            uint32_t ent0 = scales[n], ent1 = (J > 1) ? scales[a.Npad + n] : 0u;
-            int bl = 0;           // TMEM buffer of the tile's last group
+            // groups [jb, je) of the item, then (when it.z) the zero-point term as group je
+            const int jb = it.kb0 * GPS, je = it.kb1 * GPS, jn = je + (it.z ? 1 : 0);
+            uint32_t ent0 = scales[(int64_t)jb * a.Npad + n];
+            uint32_t ent1 = (jb + 1 < je) ? scales[(int64_t)(jb + 1) * a.Npad + n] : 0u;
+            int bl = 0;           // TMEM buffer of the item's last group
             uint32_t tl_addr = 0;  // this warp's columns in it
-            for (int j = 0; j <= J && ok; ++j, ++jg) {
+            for (int j = jb; j < jn && ok; ++j, ++jg) {
                 const int b = (int)(jg % NBUF);
-                float s512 = -1.0f;  // group J is the zero-point term, subtracted
-                if (j < J) {
+                float s512 = -1.0f;  // the zero-point term is subtracted
+                if (j < je) {
                     s512 = __half2float(__ushort_as_half((unsigned short)(ent0 & 0xFFFF))) * 512.0f;
                     ent0 = ent1;
-                    ent1 = (j + 2 < J) ? scales[(int64_t)(j + 2) * a.Npad + n] : 0u;
+                    ent1 = (j + 2 < je) ? scales[(int64_t)(j + 2) * a.Npad + n] : 0u;
                 }
                 if (!warp_wait_phase(&sm->acc_full[b], (uint32_t)(jg / NBUF) & 1, sm, a.status)) { ok = false; break; }
                 tc_fence_after();
@@ -461,18 +600,25 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                     if (c + 2 < 8) tmem_ld16(taddr + (c + 2) * 16, pa);
                     promote16(acc + (c + 1) * 8, s2, pb);
                 }
-                if (j == J) {
-                    // the tile's last group: its buffer holds the tile's result for the epilogue
-                    // below and is released after it
+                if (j == jn - 1) {
+                    // the item's last group: its buffer holds the result for the epilogue below
+                    // and is released after it
                     bl = b;
                     tl_addr = taddr;
-                    continue;  // ends the loop (j > J) with jg counted
+                    continue;  // ends the loop with jg counted
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
             }
             if (!ok) break;
+            if (it.seg >= 0 && !split_combine(a, it, warp - 4, lane, acc)) {
+                // a split tile's partial sum, stored for the contributor that finishes the tile
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->acc_empty[bl]);
+                continue;
+            }
             // Epilogue. The result goes through the last group's TMEM buffer so that the store
             // loop can stay rolled (an unrolled 128-column loop runs once per tile and its code
             // is fetched cold every time): 8 stores of 16 columns, then per 16-column chunk one
@@ -541,17 +687,20 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
         const int et = threadIdx.x - 384;  // 0..127
         Ring r;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        Work w(a);
+        Item it;
+        while (ok && w.next(a, it)) {
             Tile T;
-            if (!locate_tile(a, t, T)) continue;
-            for (int s = 0; s < SPT; ++s, r.next()) {
+            if (!locate_tile(a, it.t, T)) continue;
+            const int send = it.kb1 + (it.z ? a.ZT : 0);
+            for (int s = it.kb0; s < send; ++s, r.next()) {
                 const int slot = r.slot;
                 // the TMA bytes of this use have landed; the producer issued them only after the
                 // MMA released the slot's previous use, so the expanded buffer is free as well.
                 // Every stage is waited for, pseudo-stages included, so that this role sees each
                 // phase of the ring in order.
                 if (!warp_wait_phase(&sm->full[slot], r.phase, sm, a.status)) { ok = false; break; }
-                if (s < a.KT) {
+                if (s < it.kb1) {
                     const uint8_t *src = raw + slot * RAW_BYTES;
                     uint8_t *dstA = sA + slot * A_BYTES;
 #pragma unroll
@@ -629,9 +778,50 @@ static w4_status start(int grid, const CUtensorMap &tm_codes, const CUtensorMap 
     return launch_status();
 }
 
+// Work split of a dense problem of `tiles` tiles of KT k-blocks over `sms` SMs. Whole tiles go
+// round-robin over the grid; when the last wave would leave a useful share of the SMs idle,
+// its R tiles are split along K instead, over PS CTAs with at least kMinSplitBlocks k-blocks
+// each and at most about kMaxParts contributors per tile.
+constexpr int64_t kMinSplitBlocks = 8;
+constexpr int64_t kMaxParts = 8;
+
+struct Plan {
+    int64_t tiles, dpt, r, ps;
+    int grid;
+    size_t ws_bytes;
+};
+
+static Plan make_plan(int64_t tiles, int64_t KT, int sms, bool splittable) {
+    Plan p;
+    p.tiles = tiles;
+    p.dpt = tiles;
+    p.r = 0;
+    p.ps = 0;
+    p.grid = (int)(tiles < sms ? tiles : sms);
+    p.ws_bytes = 0;
+    if (!splittable || sms < 1 || tiles < 1) return p;
+    const int64_t waves = tiles / sms, r = tiles % sms;
+    if (r == 0 || (waves > 0 && r > sms - sms / 8)) return p;  // the last wave is (nearly) full
+    int64_t ps = r * KT / kMinSplitBlocks;
+    if (ps > r * kMaxParts) ps = r * kMaxParts;
+    if (ps > sms) ps = sms;
+    if (ps < r + r / 4 + 1) return p;  // splitting would shorten the last wave by too little
+    p.dpt = tiles - r;
+    p.r = r;
+    p.ps = ps;
+    p.grid = waves > 0 ? sms : (int)ps;
+    p.ws_bytes = (size_t)(2 * ps) * PART_FLOATS * sizeof(float) + (size_t)(r * 8) * sizeof(uint32_t);
+    return p;
+}
+
+static int64_t dense_tiles(int64_t M, int64_t N, int64_t K, int group) {
+    const GemmLayout L = gemm_layout(N, K, group);
+    return ((M + BN - 1) / BN) * (L.Npad / BM);
+}
+
 static w4_status launch(const uint8_t *X8, const float *row_scale, const uint16_t *gop, const int32_t *offsets, int E,
                         int64_t M, const void *packed, int64_t N, int64_t K, int group, void *Y, int out_fp32,
-                        cudaStream_t stream) {
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return W4_ERR_CUDA;
     const GemmLayout L = gemm_layout(N, K, group);
@@ -694,8 +884,16 @@ static w4_status launch(const uint8_t *X8, const float *row_scale, const uint16_
     a.MTU = (int)mtu;
     a.KT = (int)(L.Kpad / BK);
     a.ZT = (int)(L.KZ / ZKC);
-    const int64_t tiles = mtu * a.NT;
-    const int grid = (int)(tiles < sm_count_cached() ? tiles : sm_count_cached());
+    const Plan P = make_plan(mtu * a.NT, a.KT, sm_count_cached(), !offsets && workspace != nullptr);
+    if (P.ws_bytes > workspace_bytes) return W4_ERR_WORKSPACE;
+    a.DPT = P.dpt;
+    a.R = P.r;
+    a.PS = P.ps;
+    a.part = P.r ? static_cast<float *>(workspace) : nullptr;
+    a.cnt = P.r ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
+                                               (size_t)(2 * P.ps) * PART_FLOATS * sizeof(float))
+                : nullptr;
+    const int grid = P.grid;
     switch (group) {
         case 32: return start<32>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream);
         case 64: return start<64>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream);
@@ -708,17 +906,72 @@ static w4_status launch(const uint8_t *X8, const float *row_scale, const uint16_
 
 using namespace w4;
 
+static bool gemm_shape_ok(int64_t M, int64_t N, int64_t K) {
+    return M >= 1 && M <= 0x7fffffffLL && N >= 1 && N <= 0x7fffffffLL && K >= 128 && K % 32 == 0 && K <= (1LL << 24);
+}
+
+W4_API size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int group) {
+    if (!gemm_shape_ok(M, N, K) || !valid_group(group) || K % group != 0) return 0;
+    const int sms = gemm::sm_count_cached();
+    if (sms < 1) return 0;
+    return gemm::make_plan(gemm::dense_tiles(M, N, K, group), gemm_layout(N, K, group).Kpad / gemm::BK, sms, true)
+        .ws_bytes;
+}
+
+W4_API w4_status w4a8_gemm_schedule(int64_t M, int64_t N, int64_t K, int group, int sms, int64_t *out) {
+    if (!out) return W4_ERR_NULL;
+    if (!gemm_shape_ok(M, N, K) || sms < 1 || sms > 4096) return W4_ERR_SHAPE;
+    if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
+    const int64_t KT = gemm_layout(N, K, group).Kpad / gemm::BK;
+    const gemm::Plan p = gemm::make_plan(gemm::dense_tiles(M, N, K, group), KT, sms, true);
+    out[0] = p.tiles;
+    out[1] = p.dpt;
+    out[2] = p.r;
+    out[3] = p.ps;
+    out[4] = p.grid;
+    out[5] = (int64_t)p.ws_bytes;
+    out[6] = KT;
+    return W4_OK;
+}
+
+W4_API w4_status w4a8_gemm_split_segment(int64_t R, int64_t KT, int64_t PS, int64_t c, int s, int64_t *out) {
+    if (!out) return W4_ERR_NULL;
+    if (R < 1 || KT < 1 || KT > (1LL << 20) || PS < R || PS > 4096 || c < 0 || c >= PS || s < 0) return W4_ERR_ARG;
+    const int64_t Q = R * KT;
+    int64_t q = gemm::split_begin(Q, PS, c);
+    const int64_t q1 = gemm::split_begin(Q, PS, c + 1);
+    for (int k = 0; k < 7; ++k) out[k] = -1;
+    out[0] = 0;
+    for (int k = 0; q < q1; ++k) {
+        int64_t i;
+        int kb0, kb1;
+        q = gemm::split_segment(q, q1, (int)KT, i, kb0, kb1);
+        if (k == s) {
+            out[0] = 1;
+            out[1] = i;
+            out[2] = kb0;
+            out[3] = kb1;
+            out[4] = gemm::split_cta_of(Q, PS, i * KT);
+            out[5] = gemm::split_cta_of(Q, PS, i * KT + KT - 1);
+            out[6] = gemm::split_slot(Q, PS, (int)KT, c, i);
+            break;
+        }
+    }
+    return W4_OK;
+}
+
 W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op, int64_t M,
                            const void *packed, int64_t N, int64_t K, int group, int mode, void *Y, int out_fp32,
-                           cudaStream_t stream) {
+                           void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     if (!X_e4m3 || !row_scale || !gsum_op || !packed || !Y) return W4_ERR_NULL;
     if (!valid_mode(mode) || (out_fp32 != 0 && out_fp32 != 1)) return W4_ERR_ARG;
-    if (M < 1 || M > 0x7fffffffLL || N < 1 || N > 0x7fffffffLL || K < 128 || K % 32 != 0 || K > (1LL << 24))
-        return W4_ERR_SHAPE;
+    if (!gemm_shape_ok(M, N, K)) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
-    if (!aligned16(X_e4m3) || !aligned16(row_scale) || !aligned16(gsum_op) || !aligned16(packed) || !aligned16(Y))
+    if (!aligned16(X_e4m3) || !aligned16(row_scale) || !aligned16(gsum_op) || !aligned16(packed) || !aligned16(Y) ||
+        !aligned16(workspace))
         return W4_ERR_ALIGN;
-    return gemm::launch(X_e4m3, row_scale, gsum_op, nullptr, 1, M, packed, N, K, group, Y, out_fp32, stream);
+    return gemm::launch(X_e4m3, row_scale, gsum_op, nullptr, 1, M, packed, N, K, group, Y, out_fp32, workspace,
+                        workspace_bytes, stream);
 }
 
 W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op,
@@ -734,5 +987,5 @@ W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale
         !aligned16(Y) || (reinterpret_cast<uintptr_t>(expert_row_offsets) & 3))
         return W4_ERR_ALIGN;
     return gemm::launch(X_e4m3, row_scale, gsum_op, expert_row_offsets, E, M_total, packed, N, K, group, Y, 0,
-                        stream);
+                        nullptr, 0, stream);
 }

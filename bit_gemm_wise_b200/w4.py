@@ -41,7 +41,10 @@ SIGNATURES = [
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a16_gemv_noalloc_scratch_limit", _SZ, []),
     ("w4a16_gemv_noalloc", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
-    ("w4a8_gemm", _I, [_P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
+    ("w4a8_gemm", _I, [_P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
+    ("w4a8_gemm_workspace_bytes", _SZ, [_I64, _I64, _I64, _I]),
+    ("w4a8_gemm_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
+    ("w4a8_gemm_split_segment", _I, [_I64, _I64, _I64, _I64, _I, _P]),
     ("w4a8_grouped_gemm", _I, [_P, _P, _P, _P, _I, _I64, _P, _I64, _I64, _I, _I, _P, _P]),
     ("w4_device_status", _I, [_P, ctypes.POINTER(ctypes.c_int)]),
     ("w4_selftest_bounded_wait", _I, [_I64, _P]),
@@ -162,10 +165,34 @@ def w4a16_gemv_noalloc(x, M, packed, N, K, group, mode, y, flags, stream=None):
     _check("w4a16_gemv_noalloc", rc)
 
 
-def w4a8_gemm(X8, row_scale, gsum_op, M, packed, N, K, group, mode, Y, out_fp32=0, stream=None):
+def w4a8_gemm(X8, row_scale, gsum_op, M, packed, N, K, group, mode, Y, out_fp32=0, workspace=None, stream=None):
+    """workspace: None (every tile whole) or alloc_gemm_workspace(M, N, K, group) (the last
+    wave's tiles may be split along K)."""
     rc = lib().w4a8_gemm(_ptr(X8), _ptr(row_scale), _ptr(gsum_op), M, _ptr(packed), N, K, group,
-                         _mode(mode), _ptr(Y), int(out_fp32), _stream(stream))
+                         _mode(mode), _ptr(Y), int(out_fp32), _ptr(workspace),
+                         0 if workspace is None else workspace.numel() * workspace.element_size(),
+                         _stream(stream))
     _check("w4a8_gemm", rc)
+
+
+def w4a8_gemm_workspace_bytes(M, N, K, group) -> int:
+    return int(lib().w4a8_gemm_workspace_bytes(M, N, K, group))
+
+
+def w4a8_gemm_schedule(M, N, K, group, sms) -> dict:
+    """Host-only: how w4a8_gemm with a workspace divides the problem over `sms` SMs."""
+    out = (ctypes.c_int64 * 7)()
+    _check("w4a8_gemm_schedule", lib().w4a8_gemm_schedule(M, N, K, group, sms, out))
+    keys = ("tiles", "whole_tiles", "split_tiles", "split_blocks", "grid", "workspace_bytes", "k_blocks")
+    return dict(zip(keys, (int(v) for v in out)))
+
+
+def w4a8_gemm_split_segment(R, KT, PS, c, s):
+    """Host-only: segment s of block c among PS blocks sharing R split tiles of KT k-blocks:
+    None, or (tile, kb0, kb1, first_block, last_block, slot)."""
+    out = (ctypes.c_int64 * 7)()
+    _check("w4a8_gemm_split_segment", lib().w4a8_gemm_split_segment(R, KT, PS, c, s, out))
+    return None if out[0] == 0 else tuple(int(v) for v in out[1:])
 
 
 def w4a8_grouped_gemm(X8, row_scale, gsum_op, expert_row_offsets, E, M_total, packed, N, K, group,
@@ -206,6 +233,12 @@ def alloc_gemv_workspace(N, K, group, device="cuda"):
     if nbytes == 0:
         raise W4Error("w4a16_gemv_workspace_bytes", 2)
     return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def alloc_gemm_workspace(M, N, K, group, device="cuda"):
+    """Zero-filled workspace for w4a8_gemm, or None when the shape is never split."""
+    nbytes = w4a8_gemm_workspace_bytes(M, N, K, group)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device) if nbytes else None
 
 
 def alloc_packed(N, K, group, layout, device="cuda", copies: int = 1):

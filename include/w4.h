@@ -221,12 +221,43 @@ w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, 
  *               same group
  *   packed      device, w4_prepack(..., W4_LAYOUT_GEMM) of W[N, K]
  *   Y           device, bf16 [M, N] (out_fp32 == 0) or fp32 [M, N] (out_fp32 == 1)
+ *   workspace   NULL, or device scratch of at least w4a8_gemm_workspace_bytes(M, N, K, group)
+ *               bytes, zero-filled before its first use (every call that completes leaves
+ *               its counters zero again; calls that may overlap on the GPU need separate
+ *               workspaces). The output is cut into tiles of 128 weight rows x 256 tokens,
+ *               one persistent block per SM. Without a workspace every tile is one block's
+ *               work. With it, when the last wave of tiles would leave many SMs idle, those
+ *               tiles are split along K over all SMs; each part's fp32 partial sum goes
+ *               through the workspace and the last part to finish adds them in a fixed order
+ *               (bit-identical results run to run; a different fp32 summation order than the
+ *               unsplit schedule, within the same error bounds). A query result of 0 means
+ *               the shape is never split and the workspace is not used.
  *   M >= 1; N >= 1; K >= 128, K % 32 == 0.
- *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG.
+ *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG / WORKSPACE (non-NULL and smaller than the
+ *   query's result).
  */
+size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int group);
 w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op,
                     int64_t M, const void *packed, int64_t N, int64_t K, int group, int mode,
-                    void *Y, int out_fp32, cudaStream_t stream);
+                    void *Y, int out_fp32, void *workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
+/*
+ * w4a8_gemm_schedule -- host-only query (no GPU call): how w4a8_gemm with a workspace divides
+ *   the problem (M, N, K, group) over `sms` SMs (1 .. 4096). out[7] receives: tiles (128
+ *   weight rows x 256 tokens each), whole tiles (the first ones, round-robin over the
+ *   grid), split tiles (the rest), blocks sharing the split tiles, grid size, workspace
+ *   bytes, k-blocks of 128 per tile. Errors: NULL / SHAPE / GROUP.
+ *
+ * w4a8_gemm_split_segment -- host-only query: segment s (0 or 1) of block c (0 <= c < PS) when
+ *   R split tiles of KT k-blocks are shared by PS >= R blocks, computed by the same functions
+ *   the kernel uses. out[7] receives: found (0/1), split tile index, first and one-past-last
+ *   k-block, first and last block contributing to that tile, partial-result slot of
+ *   (c, tile). Errors: NULL / ARG.
+ */
+w4_status w4a8_gemm_schedule(int64_t M, int64_t N, int64_t K, int group, int sms, int64_t *out);
+w4_status w4a8_gemm_split_segment(int64_t R, int64_t KT, int64_t PS, int64_t c, int s,
+                                  int64_t *out);
 
 /*
  * w4a8_grouped_gemm -- w4a8_gemm for E experts at once (mixture-of-experts layers whose

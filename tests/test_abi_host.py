@@ -111,8 +111,9 @@ def test_host_validation_rejects_before_launch(lib):
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 4, FAKE, 1 << 20, None) == 5
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE + 8, 1 << 20, None) == 4
     # gemm: the group-sum operand is required, K >= 128
-    assert rc("w4a8_gemm", FAKE, FAKE, None, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None) == 1
-    assert rc("w4a8_gemm", FAKE, FAKE, FAKE, 4, FAKE, 16, 96, 32, 1, FAKE, 0, None) == 2
+    assert rc("w4a8_gemm", FAKE, FAKE, None, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, None) == 1
+    assert rc("w4a8_gemm", FAKE, FAKE, FAKE, 4, FAKE, 16, 96, 32, 1, FAKE, 0, None, 0, None) == 2
+    assert rc("w4a8_gemm", FAKE, FAKE, FAKE, 4, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE + 8, 1 << 20, None) == 4
     # grouped gemm: expert count range
     assert rc("w4a8_grouped_gemm", FAKE, FAKE, FAKE, FAKE, 0, 16, FAKE, 16, 128, 128, 1, FAKE, None) == 2
     # prepack
@@ -120,3 +121,67 @@ def test_host_validation_rejects_before_launch(lib):
     assert rc("w4_prepack", FAKE, FAKE, None, 16, 128, 128, 0, 9, FAKE, None) == 5
     # device status needs an out pointer
     assert rc("w4_device_status", None, None) == 1
+
+
+# ------------------------------------------------------------------ W4A8 GEMM work split
+
+def test_gemm_schedule_of_the_prefill_shapes(lib):
+    # 4096 tokens x 15360 -> 3840: 16 x 30 = 480 tiles on 148 SMs, three full waves; the last
+    # 36 tiles (120 k-blocks each) are split over all 148 blocks
+    s = w4.w4a8_gemm_schedule(4096, 3840, 15360, 128, 148)
+    assert (s["tiles"], s["whole_tiles"], s["split_tiles"], s["split_blocks"], s["grid"], s["k_blocks"]) == \
+        (480, 444, 36, 148, 148, 120)
+    assert s["workspace_bytes"] == 2 * 148 * 128 * 256 * 4 + 36 * 8 * 4
+    # 3840 -> 15360: 1920 tiles, the last wave has 144 of 148: left whole
+    s = w4.w4a8_gemm_schedule(4096, 15360, 3840, 128, 148)
+    assert (s["whole_tiles"], s["split_tiles"], s["grid"], s["workspace_bytes"]) == (1920, 0, 148, 0)
+    # two long tiles: 8 parts each (at most 8 contributors per tile), 15 k-blocks per part
+    s = w4.w4a8_gemm_schedule(256, 256, 15360, 128, 148)
+    assert (s["whole_tiles"], s["split_tiles"], s["split_blocks"], s["grid"]) == (0, 2, 16, 16)
+    # ragged K (2880 -> 23 k-blocks, the last one partial): 4 tiles over 11 blocks
+    s = w4.w4a8_gemm_schedule(300, 256, 2880, 32, 148)
+    assert (s["tiles"], s["split_tiles"], s["split_blocks"], s["k_blocks"]) == (4, 4, 11, 23)
+    # short K: too few k-blocks per block to split
+    s = w4.w4a8_gemm_schedule(1000, 130, 640, 128, 148)
+    assert (s["split_tiles"], s["grid"], s["workspace_bytes"]) == (0, 8, 0)
+    with pytest.raises(w4.W4Error):
+        w4.w4a8_gemm_schedule(4096, 3840, 15360, 48, 148)
+
+
+@pytest.mark.parametrize("R,KT,PS", [(36, 120, 148), (2, 120, 16), (4, 23, 11), (12, 90, 96), (1, 9, 1),
+                                     (7, 5, 7), (3, 1000, 148), (100, 13, 131), (147, 8, 148)])
+def test_gemm_split_segments_cover_each_k_block_once(lib, R, KT, PS):
+    """Every k-block of every split tile belongs to exactly one block's segment; a block has at
+    most two segments, stored in slots 2c and 2c+1; each tile has one segment that ends it (and
+    adds the zero-point term); every segment names the same contiguous contributor range."""
+    cover = {}
+    contributors = {}
+    slots = set()
+    for c in range(PS):
+        for s in range(3):
+            seg = w4.w4a8_gemm_split_segment(R, KT, PS, c, s)
+            if s == 2:
+                assert seg is None
+            if seg is None:
+                continue
+            i, kb0, kb1, c0, c1, slot = seg
+            assert 0 <= i < R and 0 <= kb0 < kb1 <= KT
+            assert slot == 2 * c + s and slot not in slots
+            slots.add(slot)
+            assert c0 <= c <= c1 < PS
+            assert contributors.setdefault(i, (c0, c1)) == (c0, c1)
+            for kb in range(kb0, kb1):
+                assert (i, kb) not in cover
+                cover[(i, kb)] = c
+    assert len(cover) == R * KT
+    for i in range(R):
+        owners = sorted({cover[(i, kb)] for kb in range(KT)})
+        assert owners == list(range(contributors[i][0], contributors[i][1] + 1))
+        assert cover[(i, 0)] == contributors[i][0] and cover[(i, KT - 1)] == contributors[i][1]
+
+
+def test_gemm_split_segment_arguments(lib):
+    with pytest.raises(w4.W4Error):
+        w4.w4a8_gemm_split_segment(10, 8, 9, 0, 0)  # fewer blocks than tiles
+    with pytest.raises(w4.W4Error):
+        w4.w4a8_gemm_split_segment(2, 8, 16, 16, 0)  # block out of range
