@@ -328,8 +328,9 @@ struct Item {
     bool z;
 };
 
-// The sequence of items of this CTA, identical for every role: its whole tiles, then its
-// split-tile segments.
+// The sequence of items of this CTA, identical for every role: its split-tile segments first
+// (so that the combine step of a split tile, which only the last contributor runs, overlaps
+// the next whole tile's first stages), then its whole tiles.
 struct Work {
     int64_t t, q, q1;
     int seg = 0;
@@ -340,6 +341,14 @@ struct Work {
         q1 = blockIdx.x < a.PS ? split_begin(Q, a.PS, blockIdx.x + 1) : 0;
     }
     __device__ __forceinline__ bool next(const Args &a, Item &it) {
+        if (q < q1) {
+            int64_t i;
+            q = split_segment(q, q1, a.KT, i, it.kb0, it.kb1);
+            it.t = a.DPT + i;
+            it.seg = seg++;
+            it.z = it.kb1 == a.KT;  // the segment that ends the tile also adds its zero-point term
+            return true;
+        }
         if (t < a.DPT) {
             it.t = t;
             it.kb0 = 0;
@@ -347,14 +356,6 @@ struct Work {
             it.seg = -1;
             it.z = true;
             t += gridDim.x;
-            return true;
-        }
-        if (q < q1) {
-            int64_t i;
-            q = split_segment(q, q1, a.KT, i, it.kb0, it.kb1);
-            it.t = a.DPT + i;
-            it.seg = seg++;
-            it.z = it.kb1 == a.KT;  // the segment that ends the tile also adds its zero-point term
             return true;
         }
         return false;
@@ -388,10 +389,19 @@ __device__ __forceinline__ bool split_combine(const Args &a, const Item &it, int
     old = __shfl_sync(FULL, old, 0);
     if (old != (uint32_t)(c1 - c0)) return false;
     __threadfence();
-    for (int64_t c = c0; c <= c1; ++c) {
+    {   // the first contributor's partial straight into acc: 32 loads in flight per lane
+        const float4 *src =
+            reinterpret_cast<const float4 *>(a.part) + (split_slot(Q, a.PS, a.KT, c0, i) * 8 + wq) * 1024 + lane;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float4 v = __ldcg(src + k * 32);
+            acc[2 * k] = make_float2(v.x, v.y);
+            acc[2 * k + 1] = make_float2(v.z, v.w);
+        }
+    }
+    for (int64_t c = c0 + 1; c <= c1; ++c) {
         const float4 *src =
             reinterpret_cast<const float4 *>(a.part) + (split_slot(Q, a.PS, a.KT, c, i) * 8 + wq) * 1024 + lane;
-        const bool first = c == c0;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // 16 loads in flight per lane, then the adds
             float4 v[16];
@@ -400,10 +410,10 @@ __device__ __forceinline__ bool split_combine(const Args &a, const Item &it, int
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 float2 &x = acc[2 * (h * 16 + k)], &y = acc[2 * (h * 16 + k) + 1];
-                x.x = (first ? 0.0f : x.x) + v[k].x;
-                x.y = (first ? 0.0f : x.y) + v[k].y;
-                y.x = (first ? 0.0f : y.x) + v[k].z;
-                y.y = (first ? 0.0f : y.y) + v[k].w;
+                x.x += v[k].x;
+                x.y += v[k].y;
+                y.x += v[k].z;
+                y.y += v[k].w;
             }
         }
     }
@@ -781,7 +791,10 @@ static w4_status start(int grid, const CUtensorMap &tm_codes, const CUtensorMap 
 // Work split of a dense problem of `tiles` tiles of KT k-blocks over `sms` SMs. Whole tiles go
 // round-robin over the grid; when the last wave would leave a useful share of the SMs idle,
 // its R tiles are split along K instead, over PS CTAs with at least kMinSplitBlocks k-blocks
-// each and at most about kMaxParts contributors per tile.
+// each and at most about kMaxParts contributors per tile. With whole waves as well, PS is the
+// whole grid (the least work per CTA; the combine steps overlap the whole tiles that follow).
+// With none, PS is a multiple of R, so that every CTA works on one tile and each tile has the
+// fewest contributors, since there the combine step is the kernel's last.
 constexpr int64_t kMinSplitBlocks = 8;
 constexpr int64_t kMaxParts = 8;
 
@@ -805,6 +818,7 @@ static Plan make_plan(int64_t tiles, int64_t KT, int sms, bool splittable) {
     int64_t ps = r * KT / kMinSplitBlocks;
     if (ps > r * kMaxParts) ps = r * kMaxParts;
     if (ps > sms) ps = sms;
+    if (waves == 0 && ps / r >= 2) ps = r * (ps / r);
     if (ps < r + r / 4 + 1) return p;  // splitting would shorten the last wave by too little
     p.dpt = tiles - r;
     p.r = r;

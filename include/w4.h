@@ -227,7 +227,7 @@ w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, 
  *               workspaces). The output is cut into tiles of 128 weight rows x 256 tokens,
  *               one persistent block per SM. Without a workspace every tile is one block's
  *               work. With it, when the last wave of tiles would leave many SMs idle, those
- *               tiles are split along K over all SMs; each part's fp32 partial sum goes
+ *               tiles are split along K over the SMs; each part's fp32 partial sum goes
  *               through the workspace and the last part to finish adds them in a fixed order
  *               (bit-identical results run to run; a different fp32 summation order than the
  *               unsplit schedule, within the same error bounds). A query result of 0 means

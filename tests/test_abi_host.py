@@ -138,9 +138,9 @@ def test_gemm_schedule_of_the_prefill_shapes(lib):
     # two long tiles: 8 parts each (at most 8 contributors per tile), 15 k-blocks per part
     s = w4.w4a8_gemm_schedule(256, 256, 15360, 128, 148)
     assert (s["whole_tiles"], s["split_tiles"], s["split_blocks"], s["grid"]) == (0, 2, 16, 16)
-    # ragged K (2880 -> 23 k-blocks, the last one partial): 4 tiles over 11 blocks
+    # ragged K (2880 -> 23 k-blocks, the last one partial): 4 tiles over 8 blocks (2 per tile)
     s = w4.w4a8_gemm_schedule(300, 256, 2880, 32, 148)
-    assert (s["tiles"], s["split_tiles"], s["split_blocks"], s["k_blocks"]) == (4, 4, 11, 23)
+    assert (s["tiles"], s["split_tiles"], s["split_blocks"], s["k_blocks"]) == (4, 4, 8, 23)
     # short K: too few k-blocks per block to split
     s = w4.w4a8_gemm_schedule(1000, 130, 640, 128, 148)
     assert (s["split_tiles"], s["grid"], s["workspace_bytes"]) == (0, 8, 0)
