@@ -362,61 +362,74 @@ struct Work {
     }
 };
 
-// Split tile, promotion warp wq (weight rows 32*(wq&3).., token columns 128*(wq>>2)..): store
-// this warp's partial sum in the CTA's slot and count it. The warp whose arrival completes the
-// count reads every contributor's partial of its part, in CTA order, into acc, resets the
-// counter for the next call and returns true; the others return false.
+// Split tile, promotion warp wq (weight rows 32*(wq&3).., token columns 128*(wq>>2)..), whose
+// partial sum is in TMEM at taddr (32 lanes x 128 columns): store it in the CTA's slot and
+// count it. The warp whose arrival completes the count adds every contributor's partial of its
+// part, in CTA order, into TMEM at taddr, resets the counter for the next call and returns
+// true; the others return false. Kept out of line and working through TMEM so that the
+// promotion loop's code and registers are those of a kernel without split tiles.
 // Slot layout: [8 warps][32 column quads][32 lanes] float4, so that each store or load of a
 // warp covers 512 contiguous bytes.
-__device__ __forceinline__ bool split_combine(const Args &a, const Item &it, int wq, int lane, float2 (&acc)[64]) {
-    const int64_t Q = a.R * a.KT;
-    const int64_t i = it.t - a.DPT, me = blockIdx.x;
-    const int64_t c0 = split_cta_of(Q, a.PS, i * a.KT), c1 = split_cta_of(Q, a.PS, i * a.KT + a.KT - 1);
-    const int64_t slot = 2 * me + it.seg;
-    if (i < 0 || i >= a.R || c0 < 0 || me < c0 || me > c1 || c1 >= a.PS || split_slot(Q, a.PS, a.KT, me, i) != slot) {
-        if (lane == 0) record_status(a.status, W4_ERR_DEVICE_CHECK);
+// Arguments are passed as scalars (no reference to the kernel's parameter block, which would
+// need a local copy of it).
+__device__ __noinline__ bool split_combine(float *part_base, uint32_t *cnt, int *status, int64_t R, int KT,
+                                           int64_t PS, int64_t i, int seg, int wq, uint32_t taddr) {
+    const int lane = threadIdx.x & 31;
+    const int64_t Q = R * KT, me = blockIdx.x;
+    const int64_t c0 = split_cta_of(Q, PS, i * KT), c1 = split_cta_of(Q, PS, i * KT + KT - 1);
+    const int64_t slot = 2 * me + seg;
+    if (i < 0 || i >= R || c0 < 0 || me < c0 || me > c1 || c1 >= PS || split_slot(Q, PS, KT, me, i) != slot) {
+        if (lane == 0) record_status(status, W4_ERR_DEVICE_CHECK);
         return false;
     }
-    float4 *mine = reinterpret_cast<float4 *>(a.part) + (slot * 8 + wq) * 1024 + lane;
+    float4 *part = reinterpret_cast<float4 *>(part_base) + wq * 1024 + lane;  // + slot * 8192
+    {
+        float4 *mine = part + slot * 8192;
+        uint32_t v[16];
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {  // 16 columns: float4 quads 4c .. 4c+3
+            tmem_ld16(taddr + c * 16, v);
+            tmem_wait_ld16(v);
 #pragma unroll
-    for (int k = 0; k < 32; ++k)
-        __stcg(mine + k * 32, make_float4(acc[2 * k].x, acc[2 * k].y, acc[2 * k + 1].x, acc[2 * k + 1].y));
+            for (int q = 0; q < 4; ++q)
+                __stcg(mine + (4 * c + q) * 32, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                            __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+        }
+    }
     __threadfence();
     __syncwarp();
-    uint32_t *ctr = a.cnt + i * 8 + wq;
+    uint32_t *ctr = cnt + i * 8 + wq;
     uint32_t old = 0;
     if (lane == 0) old = atomicAdd(ctr, 1u);
     old = __shfl_sync(FULL, old, 0);
     if (old != (uint32_t)(c1 - c0)) return false;
     __threadfence();
-    {   // the first contributor's partial straight into acc: 32 loads in flight per lane
-        const float4 *src =
-            reinterpret_cast<const float4 *>(a.part) + (split_slot(Q, a.PS, a.KT, c0, i) * 8 + wq) * 1024 + lane;
+    // 64 columns (16 quads) at a time: the first contributor's quads, then each later one's
+    // added in CTA order, then the sums into TMEM
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+        float4 sum[16];
+        const float4 *src = part + split_slot(Q, PS, KT, c0, i) * 8192 + h * 16 * 32;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float4 v = __ldcg(src + k * 32);
-            acc[2 * k] = make_float2(v.x, v.y);
-            acc[2 * k + 1] = make_float2(v.z, v.w);
-        }
-    }
-    for (int64_t c = c0 + 1; c <= c1; ++c) {
-        const float4 *src =
-            reinterpret_cast<const float4 *>(a.part) + (split_slot(Q, a.PS, a.KT, c, i) * 8 + wq) * 1024 + lane;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // 16 loads in flight per lane, then the adds
+        for (int k = 0; k < 16; ++k) sum[k] = __ldcg(src + k * 32);
+#pragma unroll 1
+        for (int64_t c = c0 + 1; c <= c1; ++c) {
+            src = part + split_slot(Q, PS, KT, c, i) * 8192 + h * 16 * 32;
             float4 v[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = __ldcg(src + (h * 16 + k) * 32);
+            for (int k = 0; k < 16; ++k) v[k] = __ldcg(src + k * 32);
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                float2 &x = acc[2 * (h * 16 + k)], &y = acc[2 * (h * 16 + k) + 1];
-                x.x += v[k].x;
-                x.y += v[k].y;
-                y.x += v[k].z;
-                y.y += v[k].w;
+                sum[k].x += v[k].x;
+                sum[k].y += v[k].y;
+                sum[k].z += v[k].z;
+                sum[k].w += v[k].w;
             }
         }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(taddr + (4 * h + c) * 16, reinterpret_cast<const float2 *>(sum + 4 * c));
     }
+    tmem_wait_st();
     if (lane == 0) atomicExch(ctr, 0u);
     return true;
 }
@@ -622,13 +635,6 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                 if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
             }
             if (!ok) break;
-            if (it.seg >= 0 && !split_combine(a, it, warp - 4, lane, acc)) {
-                // a split tile's partial sum, stored for the contributor that finishes the tile
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm->acc_empty[bl]);
-                continue;
-            }
             // Epilogue. The result goes through the last group's TMEM buffer so that the store
             // loop can stay rolled (an unrolled 128-column loop runs once per tile and its code
             // is fetched cold every time): 8 stores of 16 columns, then per 16-column chunk one
@@ -636,6 +642,14 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
 #pragma unroll
             for (int c = 0; c < 8; ++c) tmem_st16(tl_addr + c * 16, acc + c * 8);
             tmem_wait_st();
+            if (it.seg >= 0 &&
+                !split_combine(a.part, a.cnt, a.status, a.R, a.KT, a.PS, it.t - a.DPT, it.seg, warp - 4, tl_addr)) {
+                // a split tile's partial sum, stored for the contributor that finishes the tile
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->acc_empty[bl]);
+                continue;
+            }
             const bool row_ok = n < a.N;
             const int64_t lim = (T.rows < (int64_t)BN ? T.rows : (int64_t)BN);  // valid columns of the tile
             const int64_t lim_m = a.M - T.row0;
