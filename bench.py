@@ -53,6 +53,9 @@ def peaks():
 NCU_TRAFFIC = {
     # profiles/w4a16_gemv_m1_k14336_n4096_full.md
     "w4a16_gemv M1 K14336xN4096": {"bytes": 31281920, "sha1": "d93d79618f5921b63c0af20b0cd088e89948c139"},
+    # profiles/w4a8_gemm_prefill_k3840_n15360_full.md, profiles/w4a8_gemm_prefill_k15360_n3840_split_full.md
+    "w4a8_gemm M4096 K3840xN15360": {"bytes": 158025984, "sha1": "38a05305130d46ce6af5529b9b5c0f0080f33155"},
+    "w4a8_gemm M4096 K15360xN3840": {"bytes": 184479232, "sha1": "38a05305130d46ce6af5529b9b5c0f0080f33155"},
 }
 
 
@@ -442,9 +445,14 @@ def measure_rows(args, dev, pk):
         flops = 2.0 * M * N * K
         tf = flops / (t_gemm * 1e-3) / 1e12
         rq_bytes = M * K * 2 + M * K + M * 4 + gop.numel() * 2
+        # algorithmic bytes of one launch: the prepacked weight (codes, scales, zero-point
+        # operand), E4M3 activations, row scales, group-sum operand, bf16 output
+        alg_bytes = packed.numel() + X8.numel() + sa.numel() * 4 + gop.numel() * 2 + Y.numel() * 2
         rows[f"w4a8_gemm_{K}x{N}"] = {
             "value": round(tf, 1), "unit": "TFLOP/s", "us": round(t_gemm * 1e3, 1),
             "tiles": sched["tiles"], "split_tiles": sched["split_tiles"],
+            "bytes_per_launch": alg_bytes,
+            "traffic": traffic_for(f"w4a8_gemm M{M} K{K}xN{N}", "bit_gemm_wise_b200/csrc/w4a8_gemm.cu"),
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(tf / fp8_peak, 4),
                          "peak_source": f"{pk['src']} bf16 burst x 2 (dense FP8/BF16 nominal ratio)",
