@@ -5,24 +5,41 @@
 // with a 1e-8 floor, recomputed on every call; an all-zero row stays zero.
 //
 // One 256-thread CTA per row. The row is held in registers (16-byte chunks, chunk c of the
-// row goes to thread c mod 256), reduced to max|x| by warp shuffles and shared memory,
-// then every element is divided by the scale (IEEE fp32) and converted with
-// cvt.rn.satfinite.e4m3x2.f32. Optional per-group sums of the E4M3 values are formed as
-// exact integer sums in units of 2^-9 (every E4M3 value is an integer multiple of 2^-9)
-// and rounded once to fp32; from them the optional group-sum operand of the W4A8 GEMM is
-// written: per row [hi(G) | lo(G) | hi(G) | 0 ...] in bf16, hi = bf16(G), lo = bf16(G - hi),
-// padded to a multiple of 32 columns. HBM-bound: 2 bytes read and 1 written per element.
-// Compiled with -fmad=false.
+// row goes to thread c mod 256) and reduced to max|x| (a 16-bit SIMD max over the magnitude
+// bits, then a warp reduction and shared memory); every element is then divided by the
+// scale (the IEEE fp32 quotient, formed from the row's reciprocal by one exact correction
+// step, see div_by_scale) and converted with cvt.rn.satfinite.e4m3x2.f32. Optional per-group
+// sums of the E4M3 values are exact integer sums in units of 2^-9 (every E4M3 value is an
+// integer multiple of 2^-9: a 16-byte chunk's values are added exactly in fp32, the chunks'
+// sums as integers), rounded once to fp32; from them the optional group-sum operand of the
+// W4A8 GEMM is written: per row [hi(G) | lo(G) | hi(G) | 0 ...] in bf16, hi = bf16(G),
+// lo = bf16(G - hi), padded to a multiple of 32 columns. HBM-bound: 2 bytes read and 1
+// written per element. Compiled with -fmad=false.
 #include "w4_common.cuh"
 #include "w4_layout.cuh"
 
 namespace w4 {
 
-// e4m3 byte -> its value times 2^9, as an integer (exact; |v| <= 448 * 512).
-__device__ __forceinline__ int e4m3_times512(uint32_t b) {
-    const int E = (b >> 3) & 15, M = b & 7;
-    const int mag = (E == 0) ? M : ((8 + M) << (E - 1));
-    return (b & 0x80) ? -mag : mag;
+// Sum of the 8 E4M3 values in (o0, o1), times 2^9, as an integer. Each pair goes back to
+// f16x2 (exact: E4M3 is a subset of binary16) and then to fp32; the running sum is exact in
+// fp32 because every partial sum is a multiple of 2^-9 below 8 * 448 < 2^12, which needs at
+// most 21 significant bits. The scaled total is an integer below 2^21, converted exactly.
+__device__ __forceinline__ int e4m3x8_sum_times512(uint32_t o0, uint32_t o1) {
+    float acc = 0.0f;
+    const uint32_t w[2] = {o0, o1};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t f16x2;
+            const uint16_t pair = (uint16_t)(w[i] >> (16 * h));
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(pair));
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&f16x2));
+            acc = __fadd_rn(acc, f.x);
+            acc = __fadd_rn(acc, f.y);
+        }
+    }
+    return __float2int_rn(__fmul_rn(acc, 512.0f));
 }
 
 __device__ __forceinline__ uint16_t bf16_rn_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
@@ -35,6 +52,21 @@ __device__ __forceinline__ void write_gop(uint16_t *row, int64_t Jr, int64_t j, 
     row[2 * Jr + j] = hi;
 }
 
+// x / s rounded to nearest, from r = 1/s rounded to nearest, by Markstein's correction
+// step (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Develop. 34(1), 1990): q0 = x*r, e = q0*s - x (exact with one
+// FMA; minus the remainder, so that a zero x keeps its sign), q = q0 - e*r. For this
+// kernel's operands -- s = max(amax, 1e-8)/448 with amax a finite bf16 magnitude, and
+// |x| <= amax -- the result is the IEEE quotient wherever that can decide an E4M3 code: an
+// exhaustive check of all such (amax, x) pairs finds no difference for |x/s| > 2^-11, for
+// zero quotients, or in sign (smaller quotients may differ in the last bit; both round to a
+// zero code). Rows holding an infinity or a NaN take the IEEE division instead.
+__device__ __forceinline__ float div_by_scale(float x, float s, float r) {
+    const float q0 = __fmul_rn(x, r);
+    const float e = __fmaf_rn(q0, s, -x);
+    return __fmaf_rn(-e, r, q0);
+}
+
 // two floats -> two e4m3 bytes (lo = a, hi = b), RNE, saturating
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float a, float b) {
     uint16_t r;
@@ -42,127 +74,154 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float a, float b) {
     return r;
 }
 
+// 8 bf16 values -> 8 e4m3 bytes (o0: values 0-3, o1: values 4-7)
+template <bool EXACT_DIV>
+__device__ __forceinline__ uint2 quantize8(const uint4 &v, float s, float r) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    uint32_t p[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const float lo = bf16_lo(u[t]), hi = bf16_hi(u[t]);
+        p[t] = EXACT_DIV ? cvt_e4m3x2(__fdiv_rn(lo, s), __fdiv_rn(hi, s))
+                         : cvt_e4m3x2(div_by_scale(lo, s, r), div_by_scale(hi, s, r));
+    }
+    return make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+}
+
+// Row maximum of |x| as bf16 bits: a max over the 15 magnitude bits (16-bit SIMD max), which
+// orders finite values, infinity (0x7F80) and NaN (above) the same way as their magnitudes.
+__device__ __forceinline__ uint32_t absmax_bits(uint32_t acc, const uint4 &v) {
+    acc = __vmaxu2(acc, v.x & 0x7FFF7FFFu);
+    acc = __vmaxu2(acc, v.y & 0x7FFF7FFFu);
+    acc = __vmaxu2(acc, v.z & 0x7FFF7FFFu);
+    return __vmaxu2(acc, v.w & 0x7FFF7FFFu);
+}
+
+// max |x| ignoring NaNs (fmaxf semantics), for the rare rows that hold a NaN
+__device__ __forceinline__ float absmax_float(float acc, const uint4 &v) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) acc = fmaxf(acc, fmaxf(fabsf(bf16_lo(u[t])), fabsf(bf16_hi(u[t]))));
+    return acc;
+}
+
+// Block-wide max of a per-thread value (256 threads); every thread gets the result.
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
+    v = __reduce_max_sync(FULL, v);
+    __syncthreads();  // red may still be read from an earlier reduction
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    v = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) v = v > red[w] ? v : red[w];
+    return v;
+}
+
+__device__ __forceinline__ float block_max_f32(float v, uint32_t *red) {
+    // non-negative floats order like their bit patterns
+    return __uint_as_float(block_max_u32(__float_as_uint(v), red));
+}
+
+// The group-sum outputs of one 16-byte chunk of E4M3 codes (8 values at columns 8c..8c+7),
+// reduced over the lanes that share a group.
+__device__ __forceinline__ void group_sums(uint2 o, bool live, int64_t c, int64_t m, int64_t K, int group,
+                                           float *gsum, uint16_t *gop, int64_t KZ) {
+    const int lanes_per_group = group / 8;  // 4, 8 or 16 threads share a group
+    int isum = live ? e4m3x8_sum_times512(o.x, o.y) : 0;
+    // groups never straddle a 256-chunk stride (256 * 8 is a multiple of the group)
+    for (int off = 1; off < lanes_per_group; off <<= 1) isum += __shfl_xor_sync(FULL, isum, off);
+    if (live && (threadIdx.x % lanes_per_group) == 0) {
+        const int64_t j = (c * 8) / group;
+        const float G = __fmul_rn(__int2float_rn(isum), 0.001953125f);
+        if (gsum) gsum[m * (K / group) + j] = G;
+        if (gop) write_gop(gop + m * KZ, K / group, j, G);
+    }
+}
+
+// row scale: max(amax, 1e-8) / 448, IEEE division
+__device__ __forceinline__ float scale_of(float amax) { return __fdiv_rn(fmaxf(amax, 1e-8f), 448.0f); }
+
 template <int NC>  // 16-byte chunks per thread held in registers
 __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restrict__ X, int64_t K, int group,
                                                         uint8_t *__restrict__ X8, float *__restrict__ row_scale,
                                                         float *__restrict__ gsum, uint16_t *__restrict__ gop,
                                                         int64_t KZ) {
-    __shared__ float red[8];
+    __shared__ uint32_t red[8];
     const int64_t m = blockIdx.x;
     const int tid = threadIdx.x;
     const int64_t nchunk = K / 8;
     const uint4 *src = reinterpret_cast<const uint4 *>(X + m * K);
     uint4 v[NC];
-    float amax = 0.0f;
+    uint32_t mb = 0;
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
         const int64_t c = tid + 256 * i;
-        if (c < nchunk) {
-            v[i] = src[c];
-            const uint32_t *u = reinterpret_cast<const uint32_t *>(&v[i]);
-#pragma unroll
-            for (int t = 0; t < 4; ++t) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[t])), fabsf(bf16_hi(u[t]))));
-        }
+        v[i] = c < nchunk ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        mb = absmax_bits(mb, v[i]);
     }
+    mb = block_max_u32(__vmaxu2(mb, mb >> 16) & 0xFFFFu, red);
+    const bool special = mb >= 0x7F80u;  // an infinity or a NaN in the row
+    float amax = __uint_as_float(mb << 16);
+    if (mb > 0x7F80u) {  // NaN: the maximum of the other values
+        float a = 0.0f;
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, off));
-    if ((tid & 31) == 0) red[tid >> 5] = amax;
-    __syncthreads();
-    amax = red[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
-    const float s = __fdiv_rn(fmaxf(amax, 1e-8f), 448.0f);
+        for (int i = 0; i < NC; ++i) a = absmax_float(a, v[i]);
+        amax = block_max_f32(a, red);
+    }
+    const float s = scale_of(amax);
+    const float r = __frcp_rn(s);
     if (tid == 0) row_scale[m] = s;
 
     uint2 *dst = reinterpret_cast<uint2 *>(X8 + m * K);
-    const int lanes_per_group = group / 8;  // 4, 8 or 16 threads share a group
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
         const int64_t c = tid + 256 * i;
         const bool live = c < nchunk;
-        uint32_t o0 = 0, o1 = 0;
-        int isum = 0;
+        uint2 o = make_uint2(0u, 0u);
         if (live) {
-            const uint32_t *u = reinterpret_cast<const uint32_t *>(&v[i]);
-            const uint32_t p0 = cvt_e4m3x2(__fdiv_rn(bf16_lo(u[0]), s), __fdiv_rn(bf16_hi(u[0]), s));
-            const uint32_t p1 = cvt_e4m3x2(__fdiv_rn(bf16_lo(u[1]), s), __fdiv_rn(bf16_hi(u[1]), s));
-            const uint32_t p2 = cvt_e4m3x2(__fdiv_rn(bf16_lo(u[2]), s), __fdiv_rn(bf16_hi(u[2]), s));
-            const uint32_t p3 = cvt_e4m3x2(__fdiv_rn(bf16_lo(u[3]), s), __fdiv_rn(bf16_hi(u[3]), s));
-            o0 = p0 | (p1 << 16);
-            o1 = p2 | (p3 << 16);
-            dst[c] = make_uint2(o0, o1);
-            if (gsum || gop) {
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    isum += e4m3_times512((o0 >> (8 * t)) & 0xFF);
-                    isum += e4m3_times512((o1 >> (8 * t)) & 0xFF);
-                }
-            }
+            o = special ? quantize8<true>(v[i], s, r) : quantize8<false>(v[i], s, r);
+            dst[c] = o;
         }
-        if (gsum || gop) {
-            // groups never straddle a 256-chunk stride (256 * 8 is a multiple of the group)
-            for (int off = 1; off < lanes_per_group; off <<= 1) isum += __shfl_xor_sync(FULL, isum, off);
-            if (live && (tid % lanes_per_group) == 0) {
-                const int64_t j = (c * 8) / group;
-                const float G = __fmul_rn(__int2float_rn(isum), 0.001953125f);
-                if (gsum) gsum[m * (K / group) + j] = G;
-                if (gop) write_gop(gop + m * KZ, K / group, j, G);
-            }
-        }
+        if (gsum || gop) group_sums(o, live, c, m, K, group, gsum, gop, KZ);
     }
     if (gop && tid < KZ - 3 * (K / group)) gop[m * KZ + 3 * (K / group) + tid] = 0;
 }
 
-// Rows longer than the register budget: three passes over global memory.
+// Rows longer than the register budget: two passes over global memory.
 __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__restrict__ X, int64_t K, int group,
                                                              uint8_t *__restrict__ X8, float *__restrict__ row_scale,
                                                              float *__restrict__ gsum, uint16_t *__restrict__ gop,
                                                              int64_t KZ) {
-    __shared__ float red[8];
+    __shared__ uint32_t red[8];
     const int64_t m = blockIdx.x;
     const int tid = threadIdx.x;
     const int64_t nchunk = K / 8;
     const uint4 *src = reinterpret_cast<const uint4 *>(X + m * K);
-    float amax = 0.0f;
-    for (int64_t c = tid; c < nchunk; c += 256) {
-        const uint4 v = src[c];
-        const uint32_t *u = reinterpret_cast<const uint32_t *>(&v);
-        for (int t = 0; t < 4; ++t) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(u[t])), fabsf(bf16_hi(u[t]))));
+    uint32_t mb = 0;
+    for (int64_t c = tid; c < nchunk; c += 256) mb = absmax_bits(mb, src[c]);
+    mb = block_max_u32(__vmaxu2(mb, mb >> 16) & 0xFFFFu, red);
+    const bool special = mb >= 0x7F80u;
+    float amax = __uint_as_float(mb << 16);
+    if (mb > 0x7F80u) {
+        float a = 0.0f;
+        for (int64_t c = tid; c < nchunk; c += 256) a = absmax_float(a, src[c]);
+        amax = block_max_f32(a, red);
     }
-    for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, off));
-    if ((tid & 31) == 0) red[tid >> 5] = amax;
-    __syncthreads();
-    amax = red[0];
-    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
-    const float s = __fdiv_rn(fmaxf(amax, 1e-8f), 448.0f);
+    const float s = scale_of(amax);
+    const float r = __frcp_rn(s);
     if (tid == 0) row_scale[m] = s;
     uint2 *dst = reinterpret_cast<uint2 *>(X8 + m * K);
-    const int lanes_per_group = group / 8;
     const int64_t iters = (nchunk + 255) / 256;
     for (int64_t i = 0; i < iters; ++i) {
         const int64_t c = tid + 256 * i;
         const bool live = c < nchunk;
-        int isum = 0;
+        uint2 o = make_uint2(0u, 0u);
         if (live) {
             const uint4 v = src[c];
-            const uint32_t *u = reinterpret_cast<const uint32_t *>(&v);
-            uint32_t p[4];
-            for (int t = 0; t < 4; ++t) p[t] = cvt_e4m3x2(__fdiv_rn(bf16_lo(u[t]), s), __fdiv_rn(bf16_hi(u[t]), s));
-            const uint32_t o0 = p[0] | (p[1] << 16), o1 = p[2] | (p[3] << 16);
-            dst[c] = make_uint2(o0, o1);
-            if (gsum || gop)
-                for (int t = 0; t < 4; ++t)
-                    isum += e4m3_times512((o0 >> (8 * t)) & 0xFF) + e4m3_times512((o1 >> (8 * t)) & 0xFF);
+            o = special ? quantize8<true>(v, s, r) : quantize8<false>(v, s, r);
+            dst[c] = o;
         }
-        if (gsum || gop) {
-            for (int off = 1; off < lanes_per_group; off <<= 1) isum += __shfl_xor_sync(FULL, isum, off);
-            if (live && (tid % lanes_per_group) == 0) {
-                const int64_t j = (c * 8) / group;
-                const float G = __fmul_rn(__int2float_rn(isum), 0.001953125f);
-                if (gsum) gsum[m * (K / group) + j] = G;
-                if (gop) write_gop(gop + m * KZ, K / group, j, G);
-            }
-        }
+        if (gsum || gop) group_sums(o, live, c, m, K, group, gsum, gop, KZ);
     }
     if (gop && tid < KZ - 3 * (K / group)) gop[m * KZ + 3 * (K / group) + tid] = 0;
 }

@@ -88,3 +88,55 @@ def test_ragged_and_long_rows(M, K):
     if K % 32 == 0:
         check(X, 32)
         check(X, 32, op_only=True)
+
+
+def rows_below_max(amax_bits, K):
+    """Rows of length K that hold every finite bf16 value of magnitude <= the bf16 amax_bits
+    (in the first row, amax itself first so that every row's maximum is amax); the rest of
+    the last row is zero."""
+    pats = np.arange(65536, dtype=np.uint32)
+    keep = (pats & 0x7FFF) <= amax_bits
+    vals = (pats[keep] << 16).view(np.float32)
+    vals = np.concatenate([[np.float32((np.uint32(amax_bits) << 16).view(np.float32))], vals])
+    per = K - 1  # each row also carries amax in its first column
+    rows = []
+    for i in range(0, vals.size, per):
+        chunk = vals[i:i + per]
+        row = np.zeros(K, np.float32)
+        row[0] = vals[0]
+        row[1:1 + chunk.size] = chunk
+        rows.append(row)
+    return rows
+
+
+@pytest.mark.parametrize("K", [16384, 32768])
+def test_every_value_under_many_row_maxima(K):
+    """The kernel divides by the row scale through the row's reciprocal and one exact
+    correction step; the codes must equal those of the oracle's IEEE division for every
+    bf16 value under row maxima spread over the whole exponent range (K = 16384 takes the
+    register-resident kernel, K = 32768 the three-pass one)."""
+    maxima = [0x0001, 0x0080, 0x0A3C, 0x2F11, 0x3300, 0x3C00, 0x3F80, 0x3FFF, 0x4120, 0x43E0,
+              0x447F, 0x4B01, 0x5F7F, 0x7A00, 0x7F7F]
+    rows = []
+    for a in maxima:
+        rows += rows_below_max(a, K)
+    X = torch.from_numpy(np.array(rows, np.float32)).to(torch.bfloat16)
+    check(X, 128)
+
+
+def test_rows_with_infinities():
+    """A row whose maximum is infinite has an infinite scale: finite values give zero codes
+    through the division fallback (the infinite entries themselves are NaN codes and are not
+    compared, since the sign of a NaN quotient is not fixed)."""
+    K = 512
+    row = np.linspace(-3, 3, K).astype(np.float32)
+    row[7] = np.inf
+    row2 = row.copy()
+    row2[7] = -np.inf
+    X = torch.from_numpy(np.array([row, row2])).to(torch.bfloat16)
+    gX8, gs, _, _ = gpu_row_quant(X, 32)
+    X8, s, _ = oracle.row_quant(synth.bf16_bits(X), 32)
+    assert np.array_equal(gs.view(np.uint32), s.view(np.uint32))
+    finite = np.ones(K, bool)
+    finite[7] = False
+    assert np.array_equal(gX8[:, finite], X8[:, finite])
