@@ -21,35 +21,47 @@
 namespace w4 {
 
 // Sum of the 8 E4M3 values in (o0, o1), times 2^9, as an integer. Each pair goes back to
-// f16x2 (exact: E4M3 is a subset of binary16) and then to fp32; the running sum is exact in
-// fp32 because every partial sum is a multiple of 2^-9 below 8 * 448 < 2^12, which needs at
-// most 21 significant bits. The scaled total is an integer below 2^21, converted exactly.
+// f16x2 (exact: E4M3 is a subset of binary16) and each half is added into an fp32 sum by a
+// mixed-precision FMA with 1.0; the sum is exact in fp32 because every partial sum is a
+// multiple of 2^-9 below 8 * 448 < 2^12, which needs at most 21 significant bits. The scaled
+// total is an integer below 2^21, converted exactly.
 __device__ __forceinline__ int e4m3x8_sum_times512(uint32_t o0, uint32_t o1) {
-    float acc = 0.0f;
+    float acc0 = 0.0f, acc1 = 0.0f;  // two chains (low and high halves of each pair)
+    const uint16_t one = 0x3C00;     // binary16 1.0
     const uint32_t w[2] = {o0, o1};
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            uint32_t f16x2;
             const uint16_t pair = (uint16_t)(w[i] >> (16 * h));
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(pair));
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&f16x2));
-            acc = __fadd_rn(acc, f.x);
-            acc = __fadd_rn(acc, f.y);
+            asm("{\n .reg .b32 f;\n .reg .b16 lo, hi;\n cvt.rn.f16x2.e4m3x2 f, %2;\n mov.b32 {lo, hi}, f;\n"
+                " fma.rn.f32.f16 %0, lo, %3, %0;\n fma.rn.f32.f16 %1, hi, %3, %1;\n}\n"
+                : "+f"(acc0), "+f"(acc1)
+                : "h"(pair), "h"(one));
         }
     }
-    return __float2int_rn(__fmul_rn(acc, 512.0f));
+    return __float2int_rn(__fmul_rn(__fadd_rn(acc0, acc1), 512.0f));
 }
 
 __device__ __forceinline__ uint16_t bf16_rn_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 
-// one group sum -> its three entries in the group-sum operand row (hi, lo, hi at j, Jr + j, 2 Jr + j)
-__device__ __forceinline__ void write_gop(uint16_t *row, int64_t Jr, int64_t j, float G) {
-    const uint16_t hi = bf16_rn_bits(G);
-    row[j] = hi;
-    row[Jr + j] = bf16_rn_bits(__fsub_rn(G, __uint_as_float((uint32_t)hi << 16)));
-    row[2 * Jr + j] = hi;
+// Group outputs of groups [j0, j0 + nj) of row m, whose sums are in sh[0 .. nj), written by
+// the whole block with consecutive threads on consecutive entries: the fp32 sums, and the
+// group-sum operand entries hi(G) at column j, lo(G) at J + j and hi(G) at 2J + j
+// (J = K / group; hi = bf16(G), lo = bf16(G - hi)).
+__device__ __forceinline__ void write_group_outputs(const float *sh, int64_t j0, int nj, int64_t J, int64_t m,
+                                                    float *gsum, uint16_t *gop, int64_t KZ) {
+    if (gsum)
+        for (int t = threadIdx.x; t < nj; t += blockDim.x) gsum[m * J + j0 + t] = sh[t];
+    if (gop) {
+        uint16_t *row = gop + m * KZ;
+        for (int t = threadIdx.x; t < 3 * nj; t += blockDim.x) {
+            const int region = t / nj, jj = t - region * nj;
+            const float G = sh[jj];
+            const uint16_t hi = bf16_rn_bits(G);
+            row[region * J + j0 + jj] = region == 1 ? bf16_rn_bits(__fsub_rn(G, __uint_as_float((uint32_t)hi << 16))) : hi;
+        }
+    }
 }
 
 // x / s rounded to nearest, from r = 1/s rounded to nearest, by Markstein's correction
@@ -122,20 +134,16 @@ __device__ __forceinline__ float block_max_f32(float v, uint32_t *red) {
     return __uint_as_float(block_max_u32(__float_as_uint(v), red));
 }
 
-// The group-sum outputs of one 16-byte chunk of E4M3 codes (8 values at columns 8c..8c+7),
-// reduced over the lanes that share a group.
-__device__ __forceinline__ void group_sums(uint2 o, bool live, int64_t c, int64_t m, int64_t K, int group,
-                                           float *gsum, uint16_t *gop, int64_t KZ) {
+// The group sum of the group holding 16-byte chunk c of E4M3 codes (8 values at columns
+// 8c..8c+7), reduced over the lanes that share the group and stored by the first of them at
+// sh[j - j0] (j the group's index).
+__device__ __forceinline__ void group_sum(uint2 o, bool live, int64_t c, int group, int64_t j0, float *sh) {
     const int lanes_per_group = group / 8;  // 4, 8 or 16 threads share a group
     int isum = live ? e4m3x8_sum_times512(o.x, o.y) : 0;
     // groups never straddle a 256-chunk stride (256 * 8 is a multiple of the group)
     for (int off = 1; off < lanes_per_group; off <<= 1) isum += __shfl_xor_sync(FULL, isum, off);
-    if (live && (threadIdx.x % lanes_per_group) == 0) {
-        const int64_t j = (c * 8) / group;
-        const float G = __fmul_rn(__int2float_rn(isum), 0.001953125f);
-        if (gsum) gsum[m * (K / group) + j] = G;
-        if (gop) write_gop(gop + m * KZ, K / group, j, G);
-    }
+    if (live && (threadIdx.x % lanes_per_group) == 0)
+        sh[(c * 8) / group - j0] = __fmul_rn(__int2float_rn(isum), 0.001953125f);
 }
 
 // row scale: max(amax, 1e-8) / 448, IEEE division
@@ -147,6 +155,7 @@ __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restri
                                                         float *__restrict__ gsum, uint16_t *__restrict__ gop,
                                                         int64_t KZ) {
     __shared__ uint32_t red[8];
+    __shared__ float gsh[NC * 256 * 8 / 32];  // the row's group sums (K <= NC * 2048)
     const int64_t m = blockIdx.x;
     const int tid = threadIdx.x;
     const int64_t nchunk = K / 8;
@@ -173,18 +182,38 @@ __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restri
     if (tid == 0) row_scale[m] = s;
 
     uint2 *dst = reinterpret_cast<uint2 *>(X8 + m * K);
+    const bool sums = gsum || gop;
+    int isum[NC];
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
         const int64_t c = tid + 256 * i;
-        const bool live = c < nchunk;
-        uint2 o = make_uint2(0u, 0u);
-        if (live) {
-            o = special ? quantize8<true>(v[i], s, r) : quantize8<false>(v[i], s, r);
+        isum[i] = 0;
+        if (c < nchunk) {
+            const uint2 o = special ? quantize8<true>(v[i], s, r) : quantize8<false>(v[i], s, r);
             dst[c] = o;
+            if (sums) isum[i] = e4m3x8_sum_times512(o.x, o.y);
         }
-        if (gsum || gop) group_sums(o, live, c, m, K, group, gsum, gop, KZ);
     }
-    if (gop && tid < KZ - 3 * (K / group)) gop[m * KZ + 3 * (K / group) + tid] = 0;
+    if (sums) {
+        // every chunk's group sum over the lanes that share its group, all chunks at once
+        // (groups never straddle a 256-chunk stride: 256 * 8 is a multiple of the group)
+        const int lanes_per_group = group / 8;
+        for (int off = 1; off < lanes_per_group; off <<= 1) {
+#pragma unroll
+            for (int i = 0; i < NC; ++i) isum[i] += __shfl_xor_sync(FULL, isum[i], off);
+        }
+        if (tid % lanes_per_group == 0) {
+#pragma unroll
+            for (int i = 0; i < NC; ++i) {
+                const int64_t c = tid + 256 * i;
+                if (c < nchunk) gsh[(c * 8) / group] = __fmul_rn(__int2float_rn(isum[i]), 0.001953125f);
+            }
+        }
+        __syncthreads();
+        write_group_outputs(gsh, 0, (int)(K / group), K / group, m, gsum, gop, KZ);
+        if (gop)
+            for (int64_t t = 3 * (K / group) + tid; t < KZ; t += 256) gop[m * KZ + t] = 0;
+    }
 }
 
 // Rows longer than the register budget: two passes over global memory.
@@ -193,6 +222,7 @@ __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__r
                                                              float *__restrict__ gsum, uint16_t *__restrict__ gop,
                                                              int64_t KZ) {
     __shared__ uint32_t red[8];
+    __shared__ float gsh[256 * 8 / 32];  // group sums of one round of 256 chunks
     const int64_t m = blockIdx.x;
     const int tid = threadIdx.x;
     const int64_t nchunk = K / 8;
@@ -221,9 +251,18 @@ __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__r
             o = special ? quantize8<true>(v, s, r) : quantize8<false>(v, s, r);
             dst[c] = o;
         }
-        if (gsum || gop) group_sums(o, live, c, m, K, group, gsum, gop, KZ);
+        if (gsum || gop) {
+            // this round's groups: [j0, j0 + nj)
+            const int64_t j0 = i * 2048 / group;
+            const int64_t jend = ((i + 1) * 2048 < K ? (i + 1) * 2048 : K) / group;
+            group_sum(o, live, c, group, j0, gsh);
+            __syncthreads();
+            write_group_outputs(gsh, j0, (int)(jend - j0), K / group, m, gsum, gop, KZ);
+            __syncthreads();  // gsh is reused by the next round
+        }
     }
-    if (gop && tid < KZ - 3 * (K / group)) gop[m * KZ + 3 * (K / group) + tid] = 0;
+    if (gop)
+        for (int64_t t = 3 * (K / group) + tid; t < KZ; t += 256) gop[m * KZ + t] = 0;
 }
 
 }  // namespace w4
