@@ -49,13 +49,14 @@ __device__ __forceinline__ uint16_t bf16_rn_bits(float v) { return __bfloat16_as
 // the whole block with consecutive threads on consecutive entries: the fp32 sums, and the
 // group-sum operand entries hi(G) at column j, lo(G) at J + j and hi(G) at 2J + j
 // (J = K / group; hi = bf16(G), lo = bf16(G - hi)).
+// t0 / stride: this thread's first entry and the number of threads sharing the work.
 __device__ __forceinline__ void write_group_outputs(const float *sh, int64_t j0, int nj, int64_t J, int64_t m,
-                                                    float *gsum, uint16_t *gop, int64_t KZ) {
+                                                    float *gsum, uint16_t *gop, int64_t KZ, int t0, int stride) {
     if (gsum)
-        for (int t = threadIdx.x; t < nj; t += blockDim.x) gsum[m * J + j0 + t] = sh[t];
+        for (int t = t0; t < nj; t += stride) gsum[m * J + j0 + t] = sh[t];
     if (gop) {
         uint16_t *row = gop + m * KZ;
-        for (int t = threadIdx.x; t < 3 * nj; t += blockDim.x) {
+        for (int t = t0; t < 3 * nj; t += stride) {
             const int region = t / nj, jj = t - region * nj;
             const float G = sh[jj];
             const uint16_t hi = bf16_rn_bits(G);
@@ -210,9 +211,78 @@ __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restri
             }
         }
         __syncthreads();
-        write_group_outputs(gsh, 0, (int)(K / group), K / group, m, gsum, gop, KZ);
+        write_group_outputs(gsh, 0, (int)(K / group), K / group, m, gsum, gop, KZ, tid, 256);
         if (gop)
             for (int64_t t = 3 * (K / group) + tid; t < KZ; t += 256) gop[m * KZ + t] = 0;
+    }
+}
+
+// Rows of at most 32 * NCW chunks (K <= 4096): one warp per row, 8 rows per block, the row in
+// registers (chunk c of the row goes to lane c mod 32); every reduction is a warp operation.
+template <int NCW>
+__global__ void __launch_bounds__(256) row_quant_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int64_t K,
+                                                             int group, uint8_t *__restrict__ X8,
+                                                             float *__restrict__ row_scale, float *__restrict__ gsum,
+                                                             uint16_t *__restrict__ gop, int64_t KZ) {
+    __shared__ float gsh_all[8][NCW * 8];  // per warp: its row's group sums (K / 32 at most)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m = (int64_t)blockIdx.x * 8 + warp;
+    if (m >= M) return;  // no block-wide barrier below
+    float *gsh = gsh_all[warp];
+    const int64_t nchunk = K / 8;
+    const uint4 *src = reinterpret_cast<const uint4 *>(X + m * K);
+    uint4 v[NCW];
+    uint32_t mb = 0;
+#pragma unroll
+    for (int i = 0; i < NCW; ++i) {
+        const int64_t c = lane + 32 * i;
+        v[i] = c < nchunk ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        mb = absmax_bits(mb, v[i]);
+    }
+    mb = __reduce_max_sync(FULL, __vmaxu2(mb, mb >> 16) & 0xFFFFu);
+    const bool special = mb >= 0x7F80u;  // an infinity or a NaN in the row
+    float amax = __uint_as_float(mb << 16);
+    if (mb > 0x7F80u) {  // NaN: the maximum of the other values (non-negative floats order as bits)
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NCW; ++i) a = absmax_float(a, v[i]);
+        amax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(a)));
+    }
+    const float s = scale_of(amax);
+    const float r = __frcp_rn(s);
+    if (lane == 0) row_scale[m] = s;
+
+    uint2 *dst = reinterpret_cast<uint2 *>(X8 + m * K);
+    const bool sums = gsum || gop;
+    int isum[NCW];
+#pragma unroll
+    for (int i = 0; i < NCW; ++i) {
+        const int64_t c = lane + 32 * i;
+        isum[i] = 0;
+        if (c < nchunk) {
+            const uint2 o = special ? quantize8<true>(v[i], s, r) : quantize8<false>(v[i], s, r);
+            dst[c] = o;
+            if (sums) isum[i] = e4m3x8_sum_times512(o.x, o.y);
+        }
+    }
+    if (sums) {
+        // groups never straddle a 32-chunk stride (32 * 8 is a multiple of the group)
+        const int lanes_per_group = group / 8;
+        for (int off = 1; off < lanes_per_group; off <<= 1) {
+#pragma unroll
+            for (int i = 0; i < NCW; ++i) isum[i] += __shfl_xor_sync(FULL, isum[i], off);
+        }
+        if (lane % lanes_per_group == 0) {
+#pragma unroll
+            for (int i = 0; i < NCW; ++i) {
+                const int64_t c = lane + 32 * i;
+                if (c < nchunk) gsh[(c * 8) / group] = __fmul_rn(__int2float_rn(isum[i]), 0.001953125f);
+            }
+        }
+        __syncwarp();
+        write_group_outputs(gsh, 0, (int)(K / group), K / group, m, gsum, gop, KZ, lane, 32);
+        if (gop)
+            for (int64_t t = 3 * (K / group) + lane; t < KZ; t += 32) gop[m * KZ + t] = 0;
     }
 }
 
@@ -257,7 +327,7 @@ __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__r
             const int64_t jend = ((i + 1) * 2048 < K ? (i + 1) * 2048 : K) / group;
             group_sum(o, live, c, group, j0, gsh);
             __syncthreads();
-            write_group_outputs(gsh, j0, (int)(jend - j0), K / group, m, gsum, gop, KZ);
+            write_group_outputs(gsh, j0, (int)(jend - j0), K / group, m, gsum, gop, KZ, tid, 256);
             __syncthreads();  // gsh is reused by the next round
         }
     }
@@ -287,9 +357,12 @@ W4_API w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int gro
     const int64_t KZ = gsum_op ? zop_cols(K / g) : 0;
     const int64_t nchunk = K / 8;
     const uint16_t *X = static_cast<const uint16_t *>(X_bf16);
-    const dim3 grid((unsigned)M);
-    if (nchunk <= 256) row_quant_kernel<1><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
-    else if (nchunk <= 512) row_quant_kernel<2><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
+    const dim3 grid((unsigned)M), wgrid((unsigned)((M + 7) / 8));
+    if (nchunk <= 64) row_quant_warp_kernel<2><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
+    else if (nchunk <= 128) row_quant_warp_kernel<4><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
+    else if (nchunk <= 256) row_quant_warp_kernel<8><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
+    else if (nchunk <= 384) row_quant_warp_kernel<12><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
+    else if (nchunk <= 512) row_quant_warp_kernel<16><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
     else if (nchunk <= 1024) row_quant_kernel<4><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
     else if (nchunk <= 2048) row_quant_kernel<8><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
     else row_quant_long_kernel<<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);

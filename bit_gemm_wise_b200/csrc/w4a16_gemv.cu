@@ -496,9 +496,10 @@ static int sm_count_cached() {
 }
 
 // Work partition. With N8 octets of U units each and S SMs: if whole octets split evenly
-// enough (fewer octets than SMs, or the busiest SM at most ~8% above the mean), every CTA
-// gets whole octets and no partial sum crosses CTAs; otherwise the unit stream is split
-// evenly (stream-K) and octets cut by a range boundary are finished through the workspace.
+// enough (fewer octets than SMs; the busiest SM at most ~8% above the mean; or its extra
+// units cheaper than the cross-CTA fixup), every CTA gets whole octets and no partial sum
+// crosses CTAs; otherwise the unit stream is split evenly (stream-K) and octets cut by a
+// range boundary are finished through the workspace.
 constexpr int SMEM_LIMIT_M1 = 227 * 1024;
 
 // xf: plan for the M = 1 kernel (padded bf16 x, per-warp stage rings, W1 warps)
@@ -531,8 +532,12 @@ static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool xf =
         P = L.N8;
         aligned = true;
     } else {
+        // whole octets when the busiest CTA's extra units cost less than the cross-CTA
+        // fixup of an even split (measured at about 3 us, the time of ~160 units at M = 1
+        // and proportionally fewer for more rows), or when they are within 8% of the mean
         const int64_t per = (L.N8 + S - 1) / S;
-        aligned = (double)per <= 1.08 * (double)L.N8 / (double)S;
+        aligned = (double)per <= 1.08 * (double)L.N8 / (double)S ||
+                  (double)(per * L.U) <= (double)T / (double)S + 160.0 / MT;
         P = aligned ? (L.N8 + per - 1) / per : (S < T ? S : T);
     }
     while (true) {
