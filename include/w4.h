@@ -156,9 +156,10 @@ w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uin
  *   read sets the pace):
  *     y[m, n] = sum_j s[n,j] * sum_{k in group j} x[m,k] * (q[n,k] - z[n,j])
  *   with fp32 accumulation; the output is rounded once (to bf16, or kept fp32). The weight
- *   stream is split evenly over one block per SM; rows whose reduction is split between
- *   two blocks are finished by the last of them in a fixed order, so results are
- *   bit-identical run to run on a given GPU.
+ *   stream is split into contiguous ranges, one block per SM: whole 8-row groups per block
+ *   when the uneven split costs less than combining partial rows across blocks, otherwise
+ *   equal ranges, and rows whose reduction is split between blocks are finished by the
+ *   last of them in a fixed order. Results are bit-identical run to run on a given GPU.
  *   x_bf16          device, bf16 [M, K]; 1 <= M <= 16
  *   packed          device, w4_prepack(..., W4_LAYOUT_GEMV) of W[N, K]
  *   y               device, bf16 [M, N], or fp32 [M, N] with W4_OUT_FP32 in flags
@@ -167,7 +168,8 @@ w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uin
  *                   bytes. It must be zero-filled before its first use; every call that
  *                   completes leaves it zero-filled again, so one workspace can serve any
  *                   sequence of calls on one stream. Calls that may run concurrently on
- *                   the GPU need separate workspaces.
+ *                   the GPU need separate workspaces. After a call whose kernel recorded
+ *                   an error in the device status, zero-fill it again.
  *   Errors: NULL / SHAPE (M outside 1..16, N < 1, K < 32) / GROUP / ALIGN / ARG /
  *   WORKSPACE (missing or too small).
  */
@@ -224,7 +226,8 @@ w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, 
  *   workspace   NULL, or device scratch of at least w4a8_gemm_workspace_bytes(M, N, K, group)
  *               bytes, zero-filled before its first use (every call that completes leaves
  *               its counters zero again; calls that may overlap on the GPU need separate
- *               workspaces). The output is cut into tiles of 128 weight rows x 256 tokens,
+ *               workspaces; after a call whose kernel recorded an error in the device
+ *               status, zero-fill it again). The output is cut into tiles of 128 weight rows x 256 tokens,
  *               one persistent block per SM. Without a workspace every tile is one block's
  *               work. With it, when the last wave of tiles would leave many SMs idle, those
  *               tiles are split along K over the SMs; each part's fp32 partial sum goes
