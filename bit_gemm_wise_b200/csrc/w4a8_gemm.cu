@@ -160,6 +160,17 @@ __device__ __forceinline__ bool warp_wait_phase(uint64_t *bar, uint32_t parity, 
     return r;
 }
 
+// The same with lane 0 polling without a suspend hint, for the promotion warps' wait on a
+// finished accumulator: it resumes as soon as the MMA's commit lands, which matters most
+// when every MMA ends a group (group size 32).
+__device__ __forceinline__ bool warp_wait_phase_short(uint64_t *bar, uint32_t parity, Smem *sm, int *status) {
+    bool r = true;
+    if ((threadIdx.x & 31) == 0) r = wait_phase_short(bar, parity, sm, status);
+    r = __shfl_sync(FULL, r ? 1 : 0, 0) != 0;
+    if (r) r = __all_sync(FULL, mbar_try_wait_short(bar, parity));
+    return r;
+}
+
 // Shared-memory operand descriptors (K-major), kept as two 32-bit words so that the MMA
 // thread only does 32-bit adds: the low word holds the start address in 16-byte units
 // (bits 0-13) and the leading byte offset 16 bytes (bits 16-29, unused by swizzled K-major
@@ -606,7 +617,10 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
                     ent0 = ent1;
                     ent1 = (j + 2 < je) ? scales[(int64_t)(j + 2) * a.Npad + n] : 0u;
                 }
-                if (!warp_wait_phase(&sm->acc_full[b], (uint32_t)(jg / NBUF) & 1, sm, a.status)) { ok = false; break; }
+                if (!warp_wait_phase_short(&sm->acc_full[b], (uint32_t)(jg / NBUF) & 1, sm, a.status)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN + half * 128);
                 // 8 chunks of 16 columns, double-buffered: the load of chunk c+1 is in flight
