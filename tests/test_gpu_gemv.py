@@ -1,7 +1,7 @@
 """GPU w4a16_gemv vs the CPU oracle's fp64 product of the dequantized weight.
 
 Tolerances (relative Frobenius): bf16 output against the fp64 result rounded to bf16 at
-1e-3 (the benchmark spec's bound); fp32 output against the unrounded fp64 result at 1e-4. The
+1e-3 (the required bound); fp32 output against the unrounded fp64 result at 1e-4. The
 kernel forms each 32-wide chunk as sum x*(128+q) - (128+z)*sum x in fp32; the offset of 128
 makes the fp32 partial sums about 30x larger than the result, so its rounding error is
 ~2^-24 * 30 * sqrt(32) per chunk, i.e. ~1e-5 relative: 1e-4 leaves a margin of 10."""

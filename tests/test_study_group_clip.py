@@ -1,7 +1,7 @@
 """Study of the pages' design axis: group size and clip grid.
 
 TAHOMA "MSE clipping" searches 11 contracted ranges (ratios 1.00 ... 0.50) per block; the
-decode sweep of this build uses 20 ratios over [0.7, 1.0]. QLWG "Granularity" tabulates
+decode sweep workload uses 20 ratios over [0.7, 1.0]. QLWG "Granularity" tabulates
 weight and output error against group size. This test computes that table with the oracle
 on three synthetic layers:
 - the single layer with outlier input columns, in the pages' orientation W[576, 1536];
