@@ -484,6 +484,7 @@ __global__ void __launch_bounds__(W1 * 32, 1) gemv1_kernel(const Args a) {
 struct Plan {
     Args a;
     int P, smem;
+    bool aligned;  // whole octets per block
 };
 
 static int sm_count_cached() {
@@ -504,7 +505,7 @@ constexpr int SMEM_LIMIT_M1 = 227 * 1024;
 
 // xf: plan for the M = 1 kernel (padded bf16 x, per-warp stage rings, W1 warps)
 template <int MT>
-static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool xf = false) {
+static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool xf, int64_t S) {
     const int W = xf ? W1 : Warps<MT>::value;
     const size_t limit = xf ? (size_t)SMEM_LIMIT_M1 : (size_t)SMEM_LIMIT;
     const GemvLayout L = gemv_layout(N, K, g);
@@ -525,7 +526,6 @@ static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool xf =
         a.off_slot = a.off_bars + W1 * NS * 8;
     }
     a.pdl = 0;
-    const int64_t S = sm_count_cached();
     int64_t P;
     bool aligned;
     if (L.N8 <= S) {
@@ -557,6 +557,7 @@ static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool xf =
             a.nol = (int)nol;
             p.P = (int)P;
             p.smem = (int)smem;
+            p.aligned = aligned;
             break;
         }
         if (P >= T) return false;
@@ -571,11 +572,29 @@ static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool xf =
 // The plan a call of M rows will use: the M = 1 kernel's when it applies and its shared
 // memory (which grows with K) fits, else the general kernel's.
 template <int MT>
-static bool plan_for(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool &xf) {
+static bool plan_for(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool &xf, int64_t S = 0) {
+    if (S <= 0) S = sm_count_cached();
     xf = MT == 1;
-    if (xf && make_plan<MT>(p, M, N, K, g, true)) return true;
+    if (xf && make_plan<MT>(p, M, N, K, g, true, S)) return true;
     xf = false;
-    return make_plan<MT>(p, M, N, K, g, false);
+    return make_plan<MT>(p, M, N, K, g, false, S);
+}
+
+// Host-only view of a plan for `sms` SMs: out = {units, octets, blocks, whole octets (0/1),
+// dynamic shared memory bytes per block, M = 1 ring kernel (0/1)}.
+template <int MT>
+static bool describe_plan(int64_t M, int64_t N, int64_t K, int g, int64_t sms, int64_t *out) {
+    Plan p;
+    bool xf;
+    if (!plan_for<MT>(p, M, N, K, g, xf, sms)) return false;
+    const GemvLayout L = gemv_layout(N, K, g);
+    out[0] = (int64_t)p.a.T;
+    out[1] = L.N8;
+    out[2] = p.P;
+    out[3] = p.aligned ? 1 : 0;
+    out[4] = p.smem;
+    out[5] = xf ? 1 : 0;
+    return true;
 }
 
 template <int MT>
@@ -650,6 +669,20 @@ using namespace w4;
 W4_API size_t w4a16_gemv_workspace_bytes(int64_t N, int64_t K, int group) {
     if (N < 1 || K < 32 || K % 32 != 0 || !valid_group(group) || K % group != 0) return 0;
     return gemv::workspace_bytes(N, K, group);
+}
+
+W4_API w4_status w4a16_gemv_schedule(int64_t M, int64_t N, int64_t K, int group, int sms, int64_t *out) {
+    if (!out) return W4_ERR_NULL;
+    if (M < 1 || M > 16 || N < 1 || N > (int64_t)0x7fffffff * 8 || K < 32 || K % 32 != 0 || sms < 1 || sms > 4096)
+        return W4_ERR_SHAPE;
+    if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
+    bool ok;
+    if (M <= 1) ok = gemv::describe_plan<1>(M, N, K, group, sms, out);
+    else if (M <= 2) ok = gemv::describe_plan<2>(M, N, K, group, sms, out);
+    else if (M <= 4) ok = gemv::describe_plan<4>(M, N, K, group, sms, out);
+    else if (M <= 8) ok = gemv::describe_plan<8>(M, N, K, group, sms, out);
+    else ok = gemv::describe_plan<16>(M, N, K, group, sms, out);
+    return ok ? W4_OK : W4_ERR_SHAPE;
 }
 
 W4_API w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K, int group,

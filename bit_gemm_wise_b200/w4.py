@@ -38,6 +38,7 @@ SIGNATURES = [
     ("w4a8_gsum_op_cols", _I64, [_I64, _I]),
     ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]),
     ("w4a16_gemv_workspace_bytes", _SZ, [_I64, _I64, _I]),
+    ("w4a16_gemv_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a16_gemv_noalloc_scratch_limit", _SZ, []),
     ("w4a16_gemv_noalloc", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
@@ -144,6 +145,14 @@ def fp8_row_quant(X, M, K, group, X8, row_scale, group_sums=None, gsum_op=None, 
 
 def w4a16_gemv_workspace_bytes(N, K, group) -> int:
     return int(lib().w4a16_gemv_workspace_bytes(N, K, group))
+
+
+def w4a16_gemv_schedule(M, N, K, group, sms) -> dict:
+    """Host-only: how w4a16_gemv divides the problem over `sms` SMs."""
+    out = (ctypes.c_int64 * 6)()
+    _check("w4a16_gemv_schedule", lib().w4a16_gemv_schedule(M, N, K, group, sms, out))
+    keys = ("units", "octets", "blocks", "whole_octets", "smem_bytes", "ring_kernel")
+    return dict(zip(keys, (int(v) for v in out)))
 
 
 def w4a16_gemv(x, M, packed, N, K, group, mode, y, flags, workspace, stream=None):

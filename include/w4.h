@@ -174,6 +174,17 @@ w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uin
  *   WORKSPACE (missing or too small).
  */
 size_t w4a16_gemv_workspace_bytes(int64_t N, int64_t K, int group);
+
+/*
+ * w4a16_gemv_schedule -- host-only query (no GPU call): how w4a16_gemv divides the problem
+ *   (M rows, N, K, group) over `sms` SMs (1 .. 4096), by the same planner the launch uses.
+ *   out[6] receives: units of 8 rows x 128 k, 8-row octets, blocks, whole octets per block
+ *   (1) or an even split of the units with a cross-block fixup (0), dynamic shared memory
+ *   bytes per block, and 1 when the M = 1 kernel with per-warp bulk-copy rings runs.
+ *   Errors: NULL / SHAPE / GROUP.
+ */
+w4_status w4a16_gemv_schedule(int64_t M, int64_t N, int64_t K, int group, int sms, int64_t *out);
+
 w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
                      int group, int mode, void *y, int flags, void *workspace,
                      size_t workspace_bytes, cudaStream_t stream);

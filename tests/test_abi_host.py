@@ -185,3 +185,29 @@ def test_gemm_split_segment_arguments(lib):
         w4.w4a8_gemm_split_segment(10, 8, 9, 0, 0)  # fewer blocks than tiles
     with pytest.raises(w4.W4Error):
         w4.w4a8_gemm_split_segment(2, 8, 16, 16, 0)  # block out of range
+
+
+# ------------------------------------------------------------------ W4A16 GEMV work split
+
+@pytest.mark.parametrize("K,N,blocks", [(4096, 4096, 128), (4096, 1024, 128), (4096, 14336, 138), (14336, 4096, 128)])
+def test_gemv_decode_shapes_take_whole_octets(lib, K, N, blocks):
+    """M = 1 on 148 SMs: every decode shape gets whole 8-row octets per block (no cross-block
+    fixup). For (14336, 4096) the busiest block carries 4 octets of 112 units against a mean
+    of 387.5 units (+60), cheaper than the fixup of an even split (~160 units)."""
+    s = w4.w4a16_gemv_schedule(1, N, K, 128, 148)
+    assert s["whole_octets"] == 1 and s["blocks"] == blocks and s["ring_kernel"] == 1
+    assert s["units"] == (N // 8) * (K // 128) and s["octets"] == N // 8
+    assert s["smem_bytes"] <= 227 * 1024
+
+
+def test_gemv_even_split_when_whole_octets_cost_more(lib):
+    # M = 16 units cost ~16x more, so the fixup is worth only ~10 units: 448 > 387.5 + 10
+    s = w4.w4a16_gemv_schedule(16, 4096, 14336, 128, 148)
+    assert s["whole_octets"] == 0 and s["blocks"] == 148 and s["ring_kernel"] == 0
+    # M = 1 with 512 octets of 8 units each on 148 SMs: 4 octets (32 units) vs mean 27.7 + 160
+    assert w4.w4a16_gemv_schedule(1, 4096, 1024, 128, 148)["whole_octets"] == 1
+    # fewer octets than SMs: one octet per block
+    s = w4.w4a16_gemv_schedule(1, 512, 65536, 128, 148)
+    assert s["whole_octets"] == 1 and s["blocks"] == 64
+    with pytest.raises(w4.W4Error):
+        w4.w4a16_gemv_schedule(17, 4096, 4096, 128, 148)
