@@ -211,3 +211,48 @@ def test_gemv_even_split_when_whole_octets_cost_more(lib):
     assert s["whole_octets"] == 1 and s["blocks"] == 64
     with pytest.raises(w4.W4Error):
         w4.w4a16_gemv_schedule(17, 4096, 4096, 128, 148)
+
+
+def test_gemm_schedule_invariants_over_many_shapes(lib):
+    """For any shape and SM count: the grid fits the SMs, whole and split tiles add up, a
+    split wave is partial, its blocks number at least the split tiles (so a block's range
+    touches at most two tiles) and at most the SMs, and the workspace holds 2 slots per
+    split block plus 8 counters per split tile."""
+    rng = __import__("random").Random(7)
+    for _ in range(400):
+        M = rng.choice([1, 7, 256, 300, 1000, 4096, 9000])
+        N = rng.choice([128, 200, 1536, 3840, 4096, 15360])
+        K = rng.choice([128, 256, 576, 2880, 3840, 8192, 15360])
+        g = rng.choice([g for g in (32, 64, 128) if K % g == 0])
+        sms = rng.choice([1, 2, 8, 132, 148, 160])
+        s = w4.w4a8_gemm_schedule(M, N, K, g, sms)
+        assert 1 <= s["grid"] <= sms
+        assert s["whole_tiles"] + s["split_tiles"] == s["tiles"] == -(-M // 256) * -(-N // 128)
+        if s["split_tiles"]:
+            assert s["split_tiles"] < sms and s["split_tiles"] <= s["split_blocks"] <= sms
+            assert s["whole_tiles"] % sms == 0
+            assert s["split_tiles"] * s["k_blocks"] >= 8 * s["split_blocks"]  # >= 8 k-blocks per block
+            assert s["workspace_bytes"] == 2 * s["split_blocks"] * 128 * 256 * 4 + s["split_tiles"] * 32
+        else:
+            assert s["workspace_bytes"] == 0 and s["grid"] == min(s["tiles"], sms)
+
+
+def test_gemv_schedule_invariants_over_many_shapes(lib):
+    """For any shape and SM count: shared memory within the per-block limit; at most one
+    block per SM, except when a block's range of octets would not fit shared memory, where
+    the planner doubles the blocks of an even split (blocks never wait on one another, so
+    extra waves are correct); the M = 1 ring kernel serves only M = 1."""
+    rng = __import__("random").Random(11)
+    for _ in range(300):
+        M = rng.choice([1, 2, 3, 4, 8, 16])
+        N = rng.choice([8, 100, 1024, 1536, 4096, 14336, 100000])
+        K = rng.choice([32, 128, 576, 4096, 14336, 65536])
+        g = rng.choice([g for g in (32, 64, 128) if K % g == 0])
+        sms = rng.choice([1, 16, 132, 148])
+        s = w4.w4a16_gemv_schedule(M, N, K, g, sms)
+        assert 1 <= s["blocks"] <= s["units"]
+        assert s["blocks"] <= sms or s["whole_octets"] == 0
+        assert s["smem_bytes"] <= 227 * 1024
+        assert s["octets"] == -(-N // 8) and s["units"] == s["octets"] * -(-K // 128)
+        if M > 1:
+            assert s["ring_kernel"] == 0
