@@ -170,8 +170,9 @@ w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uin
  *                   sequence of calls on one stream. Calls that may run concurrently on
  *                   the GPU need separate workspaces. After a call whose kernel recorded
  *                   an error in the device status, zero-fill it again.
- *   Errors: NULL / SHAPE (M outside 1..16, N < 1, K < 32) / GROUP / ALIGN / ARG /
- *   WORKSPACE (missing or too small).
+ *   Errors: NULL / SHAPE (M outside 1..16, N < 1, K < 32, or M > 1 with the rows' per-chunk
+ *   activation sums, 16 bytes per row per 128 of K, beyond the block's shared memory: about
+ *   K * M > 750,000) / GROUP / ALIGN / ARG / WORKSPACE (missing or too small).
  */
 size_t w4a16_gemv_workspace_bytes(int64_t N, int64_t K, int group);
 

@@ -249,7 +249,13 @@ def test_gemv_schedule_invariants_over_many_shapes(lib):
         K = rng.choice([32, 128, 576, 4096, 14336, 65536])
         g = rng.choice([g for g in (32, 64, 128) if K % g == 0])
         sms = rng.choice([1, 16, 132, 148])
-        s = w4.w4a16_gemv_schedule(M, N, K, g, sms)
+        try:
+            s = w4.w4a16_gemv_schedule(M, N, K, g, sms)
+        except w4.W4Error:
+            # the activations' per-chunk sums of M > 1 rows are staged in shared memory:
+            # 16 bytes per row per 128 of K, which 16 rows at K = 65536 exceed
+            assert M * K * 16 // 128 > 96 * 1024, (M, N, K, g, sms)
+            continue
         assert 1 <= s["blocks"] <= s["units"]
         assert s["blocks"] <= sms or s["whole_octets"] == 0
         assert s["smem_bytes"] <= 227 * 1024
