@@ -98,7 +98,9 @@ struct Args {
 // The last, partial wave of tiles is spread over the CTAs along K: its R tiles form R*KT
 // k-blocks in tile-major order, and CTA c takes the contiguous range
 // [c*Q/PS, (c+1)*Q/PS) of them (Q = R*KT). With R <= PS a range covers at most two tiles, so
-// a CTA has at most two segments. Each segment's fp32 partial sum goes to the CTA's slot
+// a CTA has at most two segments. The plan keeps PS <= Q/8, so no range is empty and the
+// contributors of a tile are exactly the CTAs from the one holding its first k-block to the
+// one holding its last. Each segment's fp32 partial sum goes to the CTA's slot
 // 2c + (0 for the first segment, 1 for the second); the last contributor to arrive (per
 // promotion warp, counted in the workspace) adds the partials of the tile in CTA order and
 // stores the result, so the result does not depend on arrival order.
@@ -848,6 +850,7 @@ static Plan make_plan(int64_t tiles, int64_t KT, int sms, bool splittable) {
     if (ps > sms) ps = sms;
     if (waves == 0 && ps / r >= 2) ps = r * (ps / r);
     if (ps < r + r / 4 + 1) return p;  // splitting would shorten the last wave by too little
+    if (ps * kMinSplitBlocks > r * KT) return p;  // every CTA needs a non-empty range
     p.dpt = tiles - r;
     p.r = r;
     p.ps = ps;
@@ -978,7 +981,8 @@ W4_API w4_status w4a8_gemm_schedule(int64_t M, int64_t N, int64_t K, int group, 
 
 W4_API w4_status w4a8_gemm_split_segment(int64_t R, int64_t KT, int64_t PS, int64_t c, int s, int64_t *out) {
     if (!out) return W4_ERR_NULL;
-    if (R < 1 || KT < 1 || KT > (1LL << 20) || PS < R || PS > 4096 || c < 0 || c >= PS || s < 0) return W4_ERR_ARG;
+    if (R < 1 || KT < 1 || KT > (1LL << 20) || PS < R || PS > 4096 || PS > R * KT || c < 0 || c >= PS || s < 0)
+        return W4_ERR_ARG;
     const int64_t Q = R * KT;
     int64_t q = gemm::split_begin(Q, PS, c);
     const int64_t q1 = gemm::split_begin(Q, PS, c + 1);

@@ -265,8 +265,8 @@ w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_
  *   bytes, k-blocks of 128 per tile. Errors: NULL / SHAPE / GROUP.
  *
  * w4a8_gemm_split_segment -- host-only query: segment s (0 or 1) of block c (0 <= c < PS) when
- *   R split tiles of KT k-blocks are shared by PS >= R blocks, computed by the same functions
- *   the kernel uses. out[7] receives: found (0/1), split tile index, first and one-past-last
+ *   R split tiles of KT k-blocks are shared by PS blocks, R <= PS <= R * KT (every block gets
+ *   at least one k-block), computed by the same functions the kernel uses. out[7] receives: found (0/1), split tile index, first and one-past-last
  *   k-block, first and last block contributing to that tile, partial-result slot of
  *   (c, tile). Errors: NULL / ARG.
  */

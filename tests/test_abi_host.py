@@ -180,11 +180,22 @@ def test_gemm_split_segments_cover_each_k_block_once(lib, R, KT, PS):
         assert cover[(i, 0)] == contributors[i][0] and cover[(i, KT - 1)] == contributors[i][1]
 
 
+def test_gemm_split_segments_random(lib):
+    rng = __import__("random").Random(3)
+    for _ in range(40):
+        PS = rng.randint(1, 300)
+        R = rng.randint(1, PS)
+        KT = rng.randint(-(-PS // R), 200)  # every block gets at least one k-block
+        test_gemm_split_segments_cover_each_k_block_once(lib, R, KT, PS)
+
+
 def test_gemm_split_segment_arguments(lib):
     with pytest.raises(w4.W4Error):
         w4.w4a8_gemm_split_segment(10, 8, 9, 0, 0)  # fewer blocks than tiles
     with pytest.raises(w4.W4Error):
         w4.w4a8_gemm_split_segment(2, 8, 16, 16, 0)  # block out of range
+    with pytest.raises(w4.W4Error):
+        w4.w4a8_gemm_split_segment(1, 9, 12, 0, 0)  # more blocks than k-blocks: empty ranges
 
 
 # ------------------------------------------------------------------ W4A16 GEMV work split
