@@ -379,44 +379,55 @@ EXPORT void o_w4a8_ref_pairs(const uint8_t *X8, const float *s_a, int64_t K, con
 
 /* ------------------------------------------------------------------ generic fake quant */
 
-/* [P2] fake_quant / [P5] quantize_blocked on double data: blocks of `block` consecutive
- * values (block = n for per-tensor), `bits`-bit symmetric or asymmetric, rint half-even,
- * zero-range guard scale = 1. Returns the dequantized values; the scale of each block in
- * scale_out (may be NULL). */
+/* A b-bit uniform quantizer of one block is a lattice: integer codes c in [c_lo, c_hi], a
+ * step (the scale) and an integer offset (the zero point, 0 for symmetric codes). A value v
+ * goes to c = clamp(rint(v / step) + offset, c_lo, c_hi) and comes back as (c - offset) * step.
+ * [P2] "Scale and zero point" fixes the lattice of a block from its extremes:
+ *   symmetric   step = max|v| / (2^(b-1) - 1), codes -(2^(b-1) - 1) .. 2^(b-1) - 1
+ *   asymmetric  step = (max - min) / (2^b - 1), offset = rint(-min / step), codes 0 .. 2^b - 1
+ * and [P2] "Quantize, then dequantize" replaces a zero step (a constant block) by 1 before the
+ * offset is formed; [P5] states the same symmetric lattice and its scale/2 error bound. */
+typedef struct {
+    double step, offset, c_lo, c_hi;
+} lattice;
+
+static lattice block_lattice(const double *v, int64_t len, int bits, int symmetric) {
+    double lo = v[0], hi = v[0];
+    for (int64_t i = 1; i < len; ++i) {
+        lo = v[i] < lo ? v[i] : lo;
+        hi = v[i] > hi ? v[i] : hi;
+    }
+    lattice L;
+    if (symmetric) {
+        L.c_hi = ldexp(1.0, bits - 1) - 1.0;
+        L.c_lo = -L.c_hi;
+        L.step = fmax(fabs(lo), fabs(hi)) / L.c_hi;
+    } else {
+        L.c_lo = 0.0;
+        L.c_hi = ldexp(1.0, bits) - 1.0;
+        L.step = (hi - lo) / L.c_hi;
+    }
+    if (L.step == 0.0) L.step = 1.0;
+    L.offset = symmetric ? 0.0 : rint(-lo / L.step);
+    return L;
+}
+
+static double lattice_round_trip(const lattice *L, double v) {
+    double c = rint(v / L->step) + L->offset;
+    c = c < L->c_lo ? L->c_lo : (c > L->c_hi ? L->c_hi : c);
+    return (c - L->offset) * L->step;
+}
+
+/* Fake quantization of n doubles in blocks of `block` consecutive values (block = n for one
+ * per-tensor scale; the last block may be shorter): every value goes through its block's
+ * lattice. out receives the reconstructed values, scale_out (may be NULL) each block's step. */
 EXPORT void o_fake_quant(const double *x, int64_t n, int64_t block, int bits, int symmetric,
                          double *out, double *scale_out) {
-    for (int64_t b0 = 0; b0 < n; b0 += block) {
-        int64_t len = (b0 + block <= n) ? block : n - b0;
-        double scale;
-        if (symmetric) {
-            double qmax = ldexp(1.0, bits - 1) - 1.0;
-            double a = 0.0;
-            for (int64_t i = 0; i < len; ++i) if (fabs(x[b0 + i]) > a) a = fabs(x[b0 + i]);
-            scale = a / qmax;
-            if (scale == 0.0) scale = 1.0;
-            for (int64_t i = 0; i < len; ++i) {
-                double q = rint(x[b0 + i] / scale);
-                if (q > qmax) q = qmax;
-                if (q < -qmax) q = -qmax;
-                out[b0 + i] = q * scale;
-            }
-        } else {
-            double qmax = ldexp(1.0, bits) - 1.0;
-            double lo = x[b0], hi = x[b0];
-            for (int64_t i = 1; i < len; ++i) {
-                if (x[b0 + i] < lo) lo = x[b0 + i];
-                if (x[b0 + i] > hi) hi = x[b0 + i];
-            }
-            scale = (hi - lo) / qmax;
-            if (scale == 0.0) scale = 1.0;
-            double zp = rint(-lo / scale);
-            for (int64_t i = 0; i < len; ++i) {
-                double q = rint(x[b0 + i] / scale) + zp;
-                if (q > qmax) q = qmax;
-                if (q < 0.0) q = 0.0;
-                out[b0 + i] = (q - zp) * scale;
-            }
-        }
-        if (scale_out) scale_out[b0 / block] = scale;
+    for (int64_t b = 0; b * block < n; ++b) {
+        const double *v = x + b * block;
+        int64_t len = n - b * block < block ? n - b * block : block;
+        lattice L = block_lattice(v, len, bits, symmetric);
+        for (int64_t i = 0; i < len; ++i) out[b * block + i] = lattice_round_trip(&L, v[i]);
+        if (scale_out) scale_out[b] = L.step;
     }
 }
