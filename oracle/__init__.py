@@ -70,6 +70,12 @@ def _load():
         lib.o_w4a8_ref_pairs.argtypes = [P, P, I64, P, P, P, I64, I, I, P, P, P, I64, P]
         lib.o_fake_quant.restype = None
         lib.o_fake_quant.argtypes = [P, I64, I64, I, I, P, P]
+        lib.o_moe_route.restype = None
+        lib.o_moe_route.argtypes = [P, I64, I, I, P, P]
+        lib.o_swiglu_row_quant.restype = None
+        lib.o_swiglu_row_quant.argtypes = [P, I64, I64, P, P, P]
+        lib.o_moe_combine.restype = None
+        lib.o_moe_combine.argtypes = [P, I64, P, P, I64, I, P]
         _lib = lib
     return _lib
 
@@ -238,6 +244,99 @@ def w4a8_ref_dense(X8, s_a, codes, scales, zeros, group: int, mode) -> np.ndarra
     A = e4m3_decode(X8).astype(np.float64) * np.asarray(s_a, np.float64)[:, None]
     W = dequantize(codes, scales, zeros, group, mode)
     return A @ W.T
+
+
+# ------------------------------------------------------------------ mixture-of-experts layer
+
+def moe_route(logits, k: int):
+    """Top-k experts per token (descending logit, equal logits in ascending expert order) and
+    their gate weights, the fp64 softmax of the k selected logits. logits: fp32 [T, E]."""
+    lib = _load()
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    experts = np.empty((T, k), np.int32)
+    gates = np.empty((T, k), np.float64)
+    lib.o_moe_route(_p(lg), T, E, k, _p(experts), _p(gates))
+    return experts, gates
+
+
+def moe_grouping(experts, E: int):
+    """Rows of the expert-grouped layout: for each expert, its tokens in ascending order.
+    Returns (token_of_row int64 [T*k], expert_row_offsets int32 [E+1], row_of int32 [T, k])
+    with row_of[t, i] the grouped row holding token t's i-th expert."""
+    experts = np.asarray(experts, np.int64)
+    T, k = experts.shape
+    off = np.zeros(E + 1, np.int32)
+    token_of_row = []
+    row_of = np.empty((T, k), np.int32)
+    for e in range(E):
+        toks = [t for t in range(T) for i in range(k) if experts[t, i] == e]
+        for t in toks:
+            i = int(np.nonzero(experts[t] == e)[0][0])
+            row_of[t, i] = len(token_of_row)
+            token_of_row.append(t)
+        off[e + 1] = len(token_of_row)
+    return np.asarray(token_of_row, np.int64), off, row_of
+
+
+def swiglu_row_quant(Y_bits, H: int):
+    """SwiGLU of the gate_up output (bf16 [R, 2H]: gate | up) and the per-row E4M3 quant of
+    the result. Returns (X8 u8 [R, H], row_scale f32 [R], h f32 [R, H])."""
+    lib = _load()
+    Y = _c(Y_bits, np.uint16)
+    R = Y.shape[0]
+    assert Y.shape[1] == 2 * H
+    X8 = np.empty((R, H), np.uint8)
+    s = np.empty(R, np.float32)
+    h = np.empty((R, H), np.float32)
+    lib.o_swiglu_row_quant(_p(Y), R, H, _p(X8), _p(s), _p(h))
+    return X8, s, h
+
+
+def moe_combine(rows, row_of, gates) -> np.ndarray:
+    """y[t] = sum_i gates[t, i] * rows[row_of[t, i]] in fp64."""
+    lib = _load()
+    rows = _c(rows, np.float64)
+    row_of = _c(row_of, np.int32)
+    gates = _c(gates, np.float64)
+    T, k = row_of.shape
+    N = rows.shape[1]
+    y = np.empty((T, N), np.float64)
+    lib.o_moe_combine(_p(rows), N, _p(row_of), _p(gates), T, k, _p(y))
+    return y
+
+
+def moe_layer_ref(X_bits, logits, k: int, gu, dn, group: int, mode):
+    """The whole expert layer in the oracle's arithmetic: route; per-row E4M3 quant of every
+    routed token row; fp64 W4A8 gate_up product rounded to bf16 (the GEMM's output type);
+    SwiGLU and the per-row E4M3 quant of its result; fp64 W4A8 down product; weighted
+    combine. gu / dn: (codes, scales, zeros) stacked over experts [E, N, ...]. Small shapes
+    only (dense fp64 matmuls). Returns (y fp64 [T, N_down], intermediates dict)."""
+    import torch
+    experts, gates = moe_route(logits, k)
+    E = gu[0].shape[0]
+    token_of_row, off, row_of = moe_grouping(experts, E)
+    Xr = np.asarray(X_bits, np.uint16)[token_of_row]
+    X8, s_a, _ = row_quant(Xr, 0)
+    A = e4m3_decode(X8).astype(np.float64) * s_a.astype(np.float64)[:, None]
+    H = gu[0].shape[1] // 2
+    Ygu = np.empty((Xr.shape[0], 2 * H), np.float64)
+    for e in range(E):
+        r0, r1 = off[e], off[e + 1]
+        if r1 > r0:
+            Ygu[r0:r1] = A[r0:r1] @ dequantize(gu[0][e], gu[1][e], None if gu[2] is None else gu[2][e], group, mode).T
+    Ygu_bits = torch.from_numpy(Ygu).to(torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    H8, s_h, _ = swiglu_row_quant(Ygu_bits, H)
+    Ah = e4m3_decode(H8).astype(np.float64) * s_h.astype(np.float64)[:, None]
+    Nd = dn[0].shape[1]
+    Yd = np.empty((Xr.shape[0], Nd), np.float64)
+    for e in range(E):
+        r0, r1 = off[e], off[e + 1]
+        if r1 > r0:
+            Yd[r0:r1] = Ah[r0:r1] @ dequantize(dn[0][e], dn[1][e], None if dn[2] is None else dn[2][e], group, mode).T
+    y = moe_combine(Yd, row_of, gates)
+    return y, dict(experts=experts, gates=gates, token_of_row=token_of_row, offsets=off, row_of=row_of,
+                   X8=X8, s_a=s_a, gate_up_bits=Ygu_bits, H8=H8, s_h=s_h, down=Yd)
 
 
 # ------------------------------------------------------------------ page formulas

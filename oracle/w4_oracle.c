@@ -300,30 +300,101 @@ EXPORT void o_dequantize(const uint8_t *codes, const uint16_t *scales, const int
  * values G[m, j] = sum_{k in group j} e4m3val(code[m,k]), summed exactly (every E4M3 value
  * is an integer multiple of 2^-9 and a group of <= 128 of them is below 2^25 * 2^-9) and
  * rounded once to fp32. */
+/* Row quant of one row of K fp32 values: amax, s = max(amax, 1e-8) / 448, codes e4m3(x / s),
+ * and the exact per-group sums of the E4M3 values when g > 0. */
+static void row_quant_one(const float *x, int64_t K, int g, uint8_t *X8, float *row_scale, float *gsum) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf(x[k]);
+        if (a > amax) amax = a;
+    }
+    float floor_amax = amax > 1e-8f ? amax : 1e-8f;
+    float s = floor_amax / 448.0f;
+    *row_scale = s;
+    for (int64_t k = 0; k < K; ++k) X8[k] = o_e4m3_encode(x[k] / s);
+    if (gsum && g > 0) {
+        for (int64_t j = 0; j < K / g; ++j) {
+            int64_t acc = 0; /* exact sum in units of 2^-9 */
+            for (int k = 0; k < g; ++k) {
+                double v = (double)o_e4m3_decode(X8[j * g + k]);
+                acc += (int64_t)llrint(v * 512.0);
+            }
+            gsum[j] = (float)ldexp((double)acc, -9);
+        }
+    }
+}
+
+/* Per-row FP8 E4M3 ([P3] "Achievement 2"): amax = max|x| of the row,
+ * s = max(amax, 1e-8) / 448, codes = e4m3(x / s). Also the per-group sums of the E4M3 values
+ * G[m, j] = sum_{k in group j} e4m3val(code[m,k]), summed exactly (every E4M3 value is an
+ * integer multiple of 2^-9 and a group of <= 128 of them is below 2^25 * 2^-9) and rounded
+ * once to fp32. */
 EXPORT void o_row_quant(const uint16_t *X, int64_t M, int64_t K, int g, uint8_t *X8,
                         float *row_scale, float *gsum) {
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
-        float amax = 0.0f;
-        for (int64_t k = 0; k < K; ++k) {
-            float a = fabsf(bf16_to_f32(X[m * K + k]));
-            if (a > amax) amax = a;
-        }
-        float floor_amax = amax > 1e-8f ? amax : 1e-8f;
-        float s = floor_amax / 448.0f;
-        row_scale[m] = s;
-        for (int64_t k = 0; k < K; ++k) X8[m * K + k] = o_e4m3_encode(bf16_to_f32(X[m * K + k]) / s);
-        if (gsum && g > 0) {
-            for (int64_t j = 0; j < K / g; ++j) {
-                int64_t acc = 0; /* exact sum in units of 2^-9 */
-                for (int k = 0; k < g; ++k) {
-                    double v = (double)o_e4m3_decode(X8[m * K + j * g + k]);
-                    acc += (int64_t)llrint(v * 512.0);
-                }
-                gsum[m * (K / g) + j] = (float)ldexp((double)acc, -9);
-            }
-        }
+        float *x = (float *)malloc((size_t)K * sizeof(float));
+        for (int64_t k = 0; k < K; ++k) x[k] = bf16_to_f32(X[m * K + k]);
+        row_quant_one(x, K, g, X8 + m * K, row_scale + m, gsum ? gsum + m * (K / (g > 0 ? g : 1)) : NULL);
+        free(x);
     }
+}
+
+/* ------------------------------------------------------------------ mixture-of-experts layer */
+
+/* Router ("4-bit by default", the MoE expert weights of gpt-oss; the pages leave the router
+ * open): the k largest logits of each token in descending order, equal logits taken in
+ * ascending expert order; gate weights are the softmax of the k selected logits (fp64). */
+EXPORT void o_moe_route(const float *logits, int64_t T, int E, int k, int32_t *experts, double *gates) {
+    for (int64_t t = 0; t < T; ++t) {
+        const float *l = logits + t * E;
+        unsigned char taken[1024];
+        memset(taken, 0, sizeof(taken));
+        for (int i = 0; i < k; ++i) {
+            int best = -1;
+            for (int e = 0; e < E; ++e)
+                if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+            taken[best] = 1;
+            experts[t * k + i] = best;
+        }
+        double mx = l[experts[t * k]], den = 0.0;
+        for (int i = 0; i < k; ++i) den += exp((double)l[experts[t * k + i]] - mx);
+        for (int i = 0; i < k; ++i) gates[t * k + i] = exp((double)l[experts[t * k + i]] - mx) / den;
+    }
+}
+
+/* SwiGLU between the two expert projections, then the per-row E4M3 quantization of the
+ * down projection's input. A row of the gate_up output holds [gate (H) | up (H)] (bf16);
+ * h = silu(gate) * up = gate * up / (1 + exp(-gate)), evaluated in fp64 and rounded to fp32
+ * (the precision in which the GPU quantizes it), then the row quant above. h_out (may be
+ * NULL) receives the fp32 h. */
+EXPORT void o_swiglu_row_quant(const uint16_t *Y, int64_t R, int64_t H, uint8_t *X8, float *row_scale,
+                               float *h_out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        float *h = (float *)malloc((size_t)H * sizeof(float));
+        for (int64_t j = 0; j < H; ++j) {
+            double gv = (double)bf16_to_f32(Y[r * 2 * H + j]);
+            double uv = (double)bf16_to_f32(Y[r * 2 * H + H + j]);
+            h[j] = (float)(gv * uv / (1.0 + exp(-gv)));
+        }
+        row_quant_one(h, H, 0, X8 + r * H, row_scale + r, NULL);
+        if (h_out) memcpy(h_out + r * H, h, (size_t)H * sizeof(float));
+        free(h);
+    }
+}
+
+/* Weighted combine of the experts' outputs: y[t, n] = sum_i gates[t, i] * rows[row_of[t, i], n]
+ * (fp64), rows being the down projection's outputs in expert-grouped order. */
+EXPORT void o_moe_combine(const double *rows, int64_t N, const int32_t *row_of, const double *gates, int64_t T,
+                          int k, double *y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int i = 0; i < k; ++i) acc += gates[t * k + i] * rows[(int64_t)row_of[t * k + i] * N + n];
+            y[t * N + n] = acc;
+        }
 }
 
 /* ------------------------------------------------------------------ reference products */

@@ -474,3 +474,117 @@ def test_row_quant_floor_below_1e8():
     # amax above the floor: the scale is amax / 448
     a = np.float32(oracle.bf16_to_f32(bf16_bits_of(X[1:2]))[0, 0])
     assert s[1] == np.float32(np.abs(a) / np.float32(448.0))
+
+
+# ------------------------------------------------------------------ mixture-of-experts layer
+
+def test_moe_route_topk_and_softmax_gates():
+    """Top-k against numpy's stable argsort of the negated logits (ties to the lower expert),
+    gates against scipy's softmax of the selected logits; a two-expert closed form."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(21)
+    lg = rng.random((300, 32)).astype(np.float32)
+    lg[7, [3, 9, 12]] = lg[7].max() + 0.5      # a three-way tie at the top
+    ex, g = oracle.moe_route(lg, 4)
+    ref = np.argsort(-lg, axis=1, kind="stable")[:, :4]
+    assert np.array_equal(ex, ref)
+    assert list(ex[7, :3]) == [3, 9, 12]
+    sel = np.take_along_axis(lg.astype(np.float64), ref, axis=1)
+    assert np.allclose(g, softmax(sel, axis=1), rtol=1e-14, atol=0)
+    assert np.allclose(g.sum(1), 1.0, rtol=0, atol=1e-15)
+    # k = 2, logits a > b: gates 1 / (1 + e^(b - a)) and the rest
+    ex2, g2 = oracle.moe_route(np.array([[0.0, 2.0, 0.5]], np.float32), 2)
+    assert list(ex2[0]) == [1, 2]
+    assert abs(g2[0, 0] - 1.0 / (1.0 + np.exp(-1.5))) < 1e-15
+
+
+def test_moe_grouping_covers_every_pair_once():
+    rng = np.random.default_rng(22)
+    lg = rng.random((64, 8)).astype(np.float32)
+    ex, _ = oracle.moe_route(lg, 3)
+    tor, off, row_of = oracle.moe_grouping(ex, 8)
+    assert off[0] == 0 and off[-1] == 64 * 3 and np.all(np.diff(off) >= 0)
+    seen = set()
+    for t in range(64):
+        for i in range(3):
+            r = row_of[t, i]
+            assert tor[r] == t and off[ex[t, i]] <= r < off[ex[t, i] + 1]
+            seen.add(int(r))
+    assert seen == set(range(64 * 3))
+    for e in range(8):  # tokens ascending inside an expert
+        assert np.all(np.diff(tor[off[e]:off[e + 1]]) > 0)
+
+
+def test_swiglu_row_quant_against_library_sigmoid_and_codec():
+    """h = gate * sigmoid(gate) * up against scipy's expit in fp64 (rounded to fp32); the
+    codes against torch's float8_e4m3fn cast of h / s; closed forms silu(0) = 0 and
+    silu(v) - silu(-v) = v."""
+    from scipy.special import expit
+    rng = np.random.default_rng(23)
+    H = 96
+    g = rng.normal(0, 3, (5, H)).astype(np.float32)
+    u = rng.normal(0, 1, (5, H)).astype(np.float32)
+    g[0, :4] = [0.0, -0.0, 40.0, -40.0]
+    Y = torch.from_numpy(np.concatenate([g, u], 1)).to(torch.bfloat16)
+    gb, ub = Y[:, :H].double().numpy(), Y[:, H:].double().numpy()
+    X8, s, h = oracle.swiglu_row_quant(synth.bf16_bits(Y), H)
+    ref = (gb * expit(gb) * ub).astype(np.float32)
+    assert np.array_equal(h, ref)
+    assert h[0, 0] == 0.0 and h[0, 1] == 0.0
+    amax = np.abs(h).max(1)
+    assert np.array_equal(s, (np.maximum(amax, np.float32(1e-8)) / np.float32(448.0)).astype(np.float32))
+    q = (torch.from_numpy(h) / torch.from_numpy(s)[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(X8, q)
+    # silu(v) - silu(-v) = v with up = 1
+    v = np.linspace(-6, 6, H).astype(np.float32)
+    Y2 = torch.from_numpy(np.stack([np.concatenate([v, np.ones(H, np.float32)]),
+                                    np.concatenate([-v, np.ones(H, np.float32)])])).to(torch.bfloat16)
+    vb = Y2[0, :H].double().numpy()
+    _, _, h2 = oracle.swiglu_row_quant(synth.bf16_bits(Y2), H)
+    assert np.allclose(h2[0].astype(np.float64) - h2[1], vb, rtol=0, atol=4e-6 * np.abs(vb).max())
+
+
+def test_moe_combine_against_einsum_and_one_hot():
+    rng = np.random.default_rng(24)
+    rows = rng.normal(0, 1, (40, 17))
+    row_of = rng.permutation(40).reshape(10, 4).astype(np.int32)
+    gates = rng.random((10, 4))
+    y = oracle.moe_combine(rows, row_of, gates)
+    assert np.allclose(y, np.einsum("tk,tkn->tn", gates, rows[row_of]), rtol=1e-14, atol=1e-14)
+    onehot = np.zeros((10, 4))
+    onehot[:, 2] = 1.0
+    assert np.array_equal(oracle.moe_combine(rows, row_of, onehot), rows[row_of[:, 2]])
+
+
+def test_moe_layer_ref_matches_independent_numpy_composition():
+    """The layer reference against a composition written here from numpy / torch library
+    routines only (argsort, softmax, matmul, float8 cast, expit), at a tiny size."""
+    from scipy.special import expit, softmax
+    E, k, T, K, H, g = 4, 2, 12, 64, 32, 32
+    rng = np.random.default_rng(25)
+    X = torch.from_numpy(rng.normal(0, 1, (T, K)).astype(np.float32)).to(torch.bfloat16)
+    lg = rng.random((T, E)).astype(np.float32)
+    gu = [oracle.quantize(synth.bf16_bits(synth.normal((2 * H, K), 0.02, 9, e)), g, "asym", [1.0], False)[:3]
+          for e in range(E)]
+    dn = [oracle.quantize(synth.bf16_bits(synth.normal((K, H), 0.02, 9, 50 + e)), g, "asym", [1.0], False)[:3]
+          for e in range(E)]
+    stack = lambda L: tuple(np.stack([x[i] for x in L]) for i in range(3))
+    y, _ = oracle.moe_layer_ref(synth.bf16_bits(X), lg, k, stack(gu), stack(dn), g, "asym")
+
+    def e4m3_rows(a):  # per-row E4M3 quantization with torch's codec
+        a = torch.from_numpy(np.asarray(a, np.float32))
+        s = torch.clamp(a.abs().amax(1), min=1e-8) / 448.0
+        return (a / s[:, None]).to(torch.float8_e4m3fn).double() * s.double()[:, None]
+
+    ref = np.zeros((T, K))
+    order = np.argsort(-lg, axis=1, kind="stable")[:, :k]
+    for t in range(T):
+        w = softmax(lg[t, order[t]].astype(np.float64))
+        a = e4m3_rows(X[t:t + 1].float().numpy())
+        for i, e in enumerate(order[t]):
+            Wgu = oracle.dequantize(*gu[e], g, "asym")
+            z = torch.from_numpy(a.numpy() @ Wgu.T).float().to(torch.bfloat16).double().numpy()
+            hh = (z[:, :H] * expit(z[:, :H]) * z[:, H:]).astype(np.float32)
+            o = e4m3_rows(hh).numpy() @ oracle.dequantize(*dn[e], g, "asym").T
+            ref[t] += w[i] * o[0]
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
