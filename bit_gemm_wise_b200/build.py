@@ -27,6 +27,7 @@ SOURCES = {
     "w4_prepack.cu": [],
     "w4a16_gemv.cu": [],
     "w4a8_gemm.cu": [],
+    "w4_moe.cu": [],
 }
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -147,6 +147,18 @@ __device__ __forceinline__ void group_sum(uint2 o, bool live, int64_t c, int gro
         sh[(c * 8) / group - j0] = __fmul_rn(__int2float_rn(isum), 0.001953125f);
 }
 
+// The source row of output row m (rows == nullptr: m itself); an index outside [0, msrc)
+// is recorded as W4_ERR_DEVICE_CHECK and gives -1 (the row is then quantized as zeros).
+__device__ __forceinline__ int64_t source_row(const int32_t *rows, int64_t m, int64_t msrc, int *status) {
+    if (!rows) return m;
+    const int64_t r = rows[m];
+    if (r < 0 || r >= msrc) {
+        if ((threadIdx.x & 31) == 0) record_status(status, W4_ERR_DEVICE_CHECK);
+        return -1;
+    }
+    return r;
+}
+
 // row scale: max(amax, 1e-8) / 448, IEEE division
 __device__ __forceinline__ float scale_of(float amax) { return __fdiv_rn(fmaxf(amax, 1e-8f), 448.0f); }
 
@@ -154,19 +166,21 @@ template <int NC>  // 16-byte chunks per thread held in registers
 __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restrict__ X, int64_t K, int group,
                                                         uint8_t *__restrict__ X8, float *__restrict__ row_scale,
                                                         float *__restrict__ gsum, uint16_t *__restrict__ gop,
-                                                        int64_t KZ) {
+                                                        int64_t KZ, const int32_t *__restrict__ rows, int64_t msrc,
+                                                        int *status) {
     __shared__ uint32_t red[8];
     __shared__ float gsh[NC * 256 * 8 / 32];  // the row's group sums (K <= NC * 2048)
     const int64_t m = blockIdx.x;
     const int tid = threadIdx.x;
     const int64_t nchunk = K / 8;
-    const uint4 *src = reinterpret_cast<const uint4 *>(X + m * K);
+    const int64_t srow = source_row(rows, m, msrc, status);
+    const uint4 *src = reinterpret_cast<const uint4 *>(X + (srow < 0 ? 0 : srow) * K);
     uint4 v[NC];
     uint32_t mb = 0;
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
         const int64_t c = tid + 256 * i;
-        v[i] = c < nchunk ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        v[i] = (c < nchunk && srow >= 0) ? src[c] : make_uint4(0u, 0u, 0u, 0u);
         mb = absmax_bits(mb, v[i]);
     }
     mb = block_max_u32(__vmaxu2(mb, mb >> 16) & 0xFFFFu, red);
@@ -223,20 +237,23 @@ template <int NCW>
 __global__ void __launch_bounds__(256) row_quant_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int64_t K,
                                                              int group, uint8_t *__restrict__ X8,
                                                              float *__restrict__ row_scale, float *__restrict__ gsum,
-                                                             uint16_t *__restrict__ gop, int64_t KZ) {
+                                                             uint16_t *__restrict__ gop, int64_t KZ,
+                                                             const int32_t *__restrict__ rows, int64_t msrc,
+                                                             int *status) {
     __shared__ float gsh_all[8][NCW * 8];  // per warp: its row's group sums (K / 32 at most)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t m = (int64_t)blockIdx.x * 8 + warp;
     if (m >= M) return;  // no block-wide barrier below
     float *gsh = gsh_all[warp];
     const int64_t nchunk = K / 8;
-    const uint4 *src = reinterpret_cast<const uint4 *>(X + m * K);
+    const int64_t srow = source_row(rows, m, msrc, status);
+    const uint4 *src = reinterpret_cast<const uint4 *>(X + (srow < 0 ? 0 : srow) * K);
     uint4 v[NCW];
     uint32_t mb = 0;
 #pragma unroll
     for (int i = 0; i < NCW; ++i) {
         const int64_t c = lane + 32 * i;
-        v[i] = c < nchunk ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        v[i] = (c < nchunk && srow >= 0) ? src[c] : make_uint4(0u, 0u, 0u, 0u);
         mb = absmax_bits(mb, v[i]);
     }
     mb = __reduce_max_sync(FULL, __vmaxu2(mb, mb >> 16) & 0xFFFFu);
@@ -290,21 +307,23 @@ __global__ void __launch_bounds__(256) row_quant_warp_kernel(const uint16_t *__r
 __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__restrict__ X, int64_t K, int group,
                                                              uint8_t *__restrict__ X8, float *__restrict__ row_scale,
                                                              float *__restrict__ gsum, uint16_t *__restrict__ gop,
-                                                             int64_t KZ) {
+                                                             int64_t KZ, const int32_t *__restrict__ rows, int64_t msrc,
+                                                        int *status) {
     __shared__ uint32_t red[8];
     __shared__ float gsh[256 * 8 / 32];  // group sums of one round of 256 chunks
     const int64_t m = blockIdx.x;
     const int tid = threadIdx.x;
     const int64_t nchunk = K / 8;
-    const uint4 *src = reinterpret_cast<const uint4 *>(X + m * K);
+    const int64_t srow = source_row(rows, m, msrc, status);
+    const uint4 *src = reinterpret_cast<const uint4 *>(X + (srow < 0 ? 0 : srow) * K);
     uint32_t mb = 0;
-    for (int64_t c = tid; c < nchunk; c += 256) mb = absmax_bits(mb, src[c]);
+    for (int64_t c = tid; c < nchunk && srow >= 0; c += 256) mb = absmax_bits(mb, src[c]);
     mb = block_max_u32(__vmaxu2(mb, mb >> 16) & 0xFFFFu, red);
     const bool special = mb >= 0x7F80u;
     float amax = __uint_as_float(mb << 16);
     if (mb > 0x7F80u) {
         float a = 0.0f;
-        for (int64_t c = tid; c < nchunk; c += 256) a = absmax_float(a, src[c]);
+        for (int64_t c = tid; c < nchunk && srow >= 0; c += 256) a = absmax_float(a, src[c]);
         amax = block_max_f32(a, red);
     }
     const float s = scale_of(amax);
@@ -317,7 +336,7 @@ __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__r
         const bool live = c < nchunk;
         uint2 o = make_uint2(0u, 0u);
         if (live) {
-            const uint4 v = src[c];
+            const uint4 v = srow >= 0 ? src[c] : make_uint4(0u, 0u, 0u, 0u);
             o = special ? quantize8<true>(v, s, r) : quantize8<false>(v, s, r);
             dst[c] = o;
         }
@@ -335,6 +354,76 @@ __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__r
         for (int64_t t = 3 * (K / group) + tid; t < KZ; t += 256) gop[m * KZ + t] = 0;
 }
 
+// SwiGLU between the expert projections, then the row quant of its result: row r of the
+// gate_up output holds [gate (H) | up (H)] in bf16; h = gate * up / (1 + exp(-gate)) in fp32
+// (expf, then a product, a sum and an IEEE division), amax over the row, s = max(amax, 1e-8)
+// / 448 and codes e4m3(h / s) with the IEEE division (h is an fp32 value, so the bf16-domain
+// reciprocal shortcut of the other kernels does not apply). One 256-thread block per row,
+// the row's h held in registers (NC chunks of 8 per thread, H <= NC * 2048).
+template <int NC>
+__global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t *__restrict__ Y, int64_t H, int group,
+                                                           uint8_t *__restrict__ X8, float *__restrict__ row_scale,
+                                                           uint16_t *__restrict__ gop, int64_t KZ) {
+    __shared__ uint32_t red[8];
+    __shared__ float gsh[NC * 256 * 8 / 32];
+    const int64_t r = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int64_t nchunk = H / 8;
+    const uint4 *gsrc = reinterpret_cast<const uint4 *>(Y + r * 2 * H);
+    const uint4 *usrc = reinterpret_cast<const uint4 *>(Y + r * 2 * H + H);
+    float h[NC][8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        const int64_t c = tid + 256 * i;
+        const uint4 gv = c < nchunk ? gsrc[c] : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 uv = c < nchunk ? usrc[c] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t g4[4] = {gv.x, gv.y, gv.z, gv.w}, u4[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float gj = (j & 1) ? bf16_hi(g4[j >> 1]) : bf16_lo(g4[j >> 1]);
+            const float uj = (j & 1) ? bf16_hi(u4[j >> 1]) : bf16_lo(u4[j >> 1]);
+            h[i][j] = __fdiv_rn(__fmul_rn(gj, uj), __fadd_rn(1.0f, expf(-gj)));
+            amax = fmaxf(amax, fabsf(h[i][j]));
+        }
+    }
+    amax = block_max_f32(amax, red);
+    const float s = scale_of(amax);
+    if (tid == 0) row_scale[r] = s;
+    uint2 *dst = reinterpret_cast<uint2 *>(X8 + r * H);
+    int isum[NC];
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        const int64_t c = tid + 256 * i;
+        isum[i] = 0;
+        if (c < nchunk) {
+            uint32_t p[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) p[t] = cvt_e4m3x2(__fdiv_rn(h[i][2 * t], s), __fdiv_rn(h[i][2 * t + 1], s));
+            const uint2 o = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
+            dst[c] = o;
+            if (gop) isum[i] = e4m3x8_sum_times512(o.x, o.y);
+        }
+    }
+    if (gop) {
+        const int lanes_per_group = group / 8;
+        for (int off = 1; off < lanes_per_group; off <<= 1) {
+#pragma unroll
+            for (int i = 0; i < NC; ++i) isum[i] += __shfl_xor_sync(FULL, isum[i], off);
+        }
+        if (tid % lanes_per_group == 0) {
+#pragma unroll
+            for (int i = 0; i < NC; ++i) {
+                const int64_t c = tid + 256 * i;
+                if (c < nchunk) gsh[(c * 8) / group] = __fmul_rn(__int2float_rn(isum[i]), 0.001953125f);
+            }
+        }
+        __syncthreads();
+        write_group_outputs(gsh, 0, (int)(H / group), H / group, r, nullptr, gop, KZ, tid, 256);
+        for (int64_t t = 3 * (H / group) + tid; t < KZ; t += 256) gop[r * KZ + t] = 0;
+    }
+}
+
 }  // namespace w4
 
 using namespace w4;
@@ -342,6 +431,28 @@ using namespace w4;
 W4_API int64_t w4a8_gsum_op_cols(int64_t K, int group) {
     if (K < 1 || !valid_group(group) || K % group != 0) return 0;
     return zop_cols(K / group);
+}
+
+// Output row m is the quantization of source row rows[m] (rows == nullptr: row m).
+static w4_status row_quant_launch(const void *X_bf16, const int32_t *rows, int64_t msrc, int64_t M, int64_t K,
+                                  int group, uint8_t *X_e4m3, float *row_scale, float *group_sums, uint16_t *gsum_op,
+                                  cudaStream_t stream) {
+    int *st = device_status_ptr();
+    const bool sums = group_sums || gsum_op;
+    const int g = sums ? group : 32;
+    const int64_t KZ = gsum_op ? zop_cols(K / g) : 0;
+    const int64_t nchunk = K / 8;
+    const uint16_t *X = static_cast<const uint16_t *>(X_bf16);
+    const dim3 grid((unsigned)M), wgrid((unsigned)((M + 7) / 8));
+    if (nchunk <= 64) row_quant_warp_kernel<2><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 128) row_quant_warp_kernel<4><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 256) row_quant_warp_kernel<8><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 384) row_quant_warp_kernel<12><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 512) row_quant_warp_kernel<16><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 1024) row_quant_kernel<4><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 2048) row_quant_kernel<8><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else row_quant_long_kernel<<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    return launch_status();
 }
 
 W4_API w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uint8_t *X_e4m3,
@@ -353,18 +464,35 @@ W4_API w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int gro
     if (!aligned16(X_bf16) || !aligned16(X_e4m3) || !aligned16(row_scale) || (group_sums && !aligned16(group_sums)) ||
         (gsum_op && !aligned16(gsum_op)))
         return W4_ERR_ALIGN;
-    const int g = sums ? group : 32;
-    const int64_t KZ = gsum_op ? zop_cols(K / g) : 0;
-    const int64_t nchunk = K / 8;
-    const uint16_t *X = static_cast<const uint16_t *>(X_bf16);
-    const dim3 grid((unsigned)M), wgrid((unsigned)((M + 7) / 8));
-    if (nchunk <= 64) row_quant_warp_kernel<2><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
-    else if (nchunk <= 128) row_quant_warp_kernel<4><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
-    else if (nchunk <= 256) row_quant_warp_kernel<8><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
-    else if (nchunk <= 384) row_quant_warp_kernel<12><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
-    else if (nchunk <= 512) row_quant_warp_kernel<16><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
-    else if (nchunk <= 1024) row_quant_kernel<4><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
-    else if (nchunk <= 2048) row_quant_kernel<8><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
-    else row_quant_long_kernel<<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ);
+    return row_quant_launch(X_bf16, nullptr, M, M, K, group, X_e4m3, row_scale, group_sums, gsum_op, stream);
+}
+
+W4_API w4_status fp8_row_quant_gather(const void *X_bf16, int64_t M_src, int64_t K, int group,
+                                      const int32_t *row_index, int64_t M, uint8_t *X_e4m3, float *row_scale,
+                                      float *group_sums, uint16_t *gsum_op, cudaStream_t stream) {
+    if (!X_bf16 || !row_index || !X_e4m3 || !row_scale) return W4_ERR_NULL;
+    if (M < 1 || M > 0x7fffffff || M_src < 1 || M_src > 0x7fffffff || K < 16 || K % 16 != 0) return W4_ERR_SHAPE;
+    const bool sums = group_sums || gsum_op;
+    if (sums && (!valid_group(group) || K % group != 0)) return W4_ERR_GROUP;
+    if (!aligned16(X_bf16) || !aligned16(X_e4m3) || !aligned16(row_scale) || (group_sums && !aligned16(group_sums)) ||
+        (gsum_op && !aligned16(gsum_op)) || (reinterpret_cast<uintptr_t>(row_index) & 3))
+        return W4_ERR_ALIGN;
+    return row_quant_launch(X_bf16, row_index, M_src, M, K, group, X_e4m3, row_scale, group_sums, gsum_op, stream);
+}
+
+W4_API w4_status w4_moe_swiglu_quant(const void *gate_up_bf16, int64_t R, int64_t H, int group, uint8_t *X_e4m3,
+                                     float *row_scale, uint16_t *gsum_op, cudaStream_t stream) {
+    if (!gate_up_bf16 || !X_e4m3 || !row_scale) return W4_ERR_NULL;
+    if (R < 1 || R > 0x7fffffff || H < 16 || H % 16 != 0 || H > 8 * 2048) return W4_ERR_SHAPE;
+    if (gsum_op && (!valid_group(group) || H % group != 0)) return W4_ERR_GROUP;
+    if (!aligned16(gate_up_bf16) || !aligned16(X_e4m3) || !aligned16(row_scale) || (gsum_op && !aligned16(gsum_op)))
+        return W4_ERR_ALIGN;
+    const int g = gsum_op ? group : 32;
+    const int64_t KZ = gsum_op ? zop_cols(H / g) : 0;
+    const int64_t nchunk = H / 8;
+    const uint16_t *Y = static_cast<const uint16_t *>(gate_up_bf16);
+    if (nchunk <= 512) swiglu_quant_kernel<2><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, row_scale, gsum_op, KZ);
+    else if (nchunk <= 1024) swiglu_quant_kernel<4><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, row_scale, gsum_op, KZ);
+    else swiglu_quant_kernel<8><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, row_scale, gsum_op, KZ);
     return launch_status();
 }

@@ -10,31 +10,28 @@
 namespace w4 {
 
 // ---------------------------------------------------------------- W4_LAYOUT_GEMV
-// The weight is cut into units of 8 rows x 128 k ("octet x unit"). N is padded to a
-// multiple of 8 and K to a multiple of 128 with code 0, scale 0.
-//   codes:  [N8 = Npad/8][U = Kpad/128][32 lanes][4 words], 512 bytes per unit. Lane
-//           t = 4r + c owns row r of the octet and the 32-wide chunk c of the unit; word w
-//           holds k = 128u + 32c + 8w + (0..7) with q[k0 + 2i] in bits [4i, 4i+4) and
-//           q[k0 + 2i + 1] in bits [16 + 4i, 20 + 4i), i = 0..3, so that masking the word
-//           (shifted by 4i) with 0x000F000F lines up two codes with one bf16x2 pair of x.
-//   scales: [N8][U][8 rows][128/g] u32, lo 16 bits the fp16 scale, hi 16 bits the zero
-//           (8 for symmetric weights). One octet's scales are contiguous (TMA-staged).
+// One record per weight row, rows in order, so that any run of consecutive rows is one
+// contiguous byte range (the GEMV stages whole rows with one bulk copy):
+//   record n = [codes: K/2 bytes, the canonical bytes of row n (byte j = q[2j] | q[2j+1] << 4)]
+//              [scales: J = K/g u32, lo 16 bits the fp16 scale, hi 16 bits the zero (8 for
+//               symmetric weights), padded with zero words to a multiple of 16 bytes]
+// so that, in every 32-bit code word (8 consecutive k), w & 0x0F0F0F0F holds the codes of
+// the even k and w & 0xF0F0F0F0 sixteen times the codes of the odd k, byte by byte.
 struct GemvLayout {
-    int64_t N, K, Npad, Kpad, N8, U;
+    int64_t N, K, J;
     int g;
-    size_t codes_bytes, scales_bytes, total;
+    size_t code_bytes;   // per row
+    size_t row_bytes;    // record size (multiple of 16)
+    size_t total;
 };
 
 inline GemvLayout gemv_layout(int64_t N, int64_t K, int g) {
     GemvLayout L;
     L.N = N; L.K = K; L.g = g;
-    L.Npad = (N + 7) / 8 * 8;
-    L.Kpad = (K + 127) / 128 * 128;
-    L.N8 = L.Npad / 8;
-    L.U = L.Kpad / 128;
-    L.codes_bytes = (size_t)L.Npad * (size_t)L.Kpad / 2;
-    L.scales_bytes = (size_t)L.Npad * (size_t)(L.Kpad / g) * 4;
-    L.total = L.codes_bytes + L.scales_bytes;
+    L.J = K / g;
+    L.code_bytes = (size_t)K / 2;
+    L.row_bytes = L.code_bytes + ((size_t)L.J * 4 + 15) / 16 * 16;
+    L.total = (size_t)N * L.row_bytes;
     return L;
 }
 

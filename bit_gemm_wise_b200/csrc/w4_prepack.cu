@@ -19,37 +19,18 @@ __device__ __forceinline__ uint32_t scale_entry(const uint16_t *scales, const in
     return s | (z << 16);
 }
 
-__global__ void prepack_gemv_codes(const uint8_t *__restrict__ codes, int64_t N, int64_t K, int64_t U,
-                                   int64_t nwords, uint32_t *__restrict__ out) {
+// W4_LAYOUT_GEMV: one thread per 32-bit word of the row records
+__global__ void prepack_gemv_rows(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ scales,
+                                  const int16_t *__restrict__ zeros, int64_t N, int64_t K, int g,
+                                  int64_t row_words, int64_t nwords, uint32_t *__restrict__ out) {
+    const int64_t J = K / g, cw = K / 8;  // code words per row
     for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nwords;
          idx += (int64_t)gridDim.x * blockDim.x) {
-        const int w = idx & 3;
-        const int t = (idx >> 2) & 31;
-        const int64_t u = (idx >> 7) % U;
-        const int64_t o = (idx >> 7) / U;
-        const int64_t n = o * 8 + (t >> 2);
-        const int64_t k0 = u * 128 + (t & 3) * 32 + w * 8;
-        uint32_t word = 0;
-        for (int i = 0; i < 4; ++i) {
-            word |= nib_at(codes, N, K, n, k0 + 2 * i) << (4 * i);
-            word |= nib_at(codes, N, K, n, k0 + 2 * i + 1) << (16 + 4 * i);
-        }
-        out[idx] = word;
-    }
-}
-
-__global__ void prepack_gemv_scales(const uint16_t *__restrict__ scales, const int16_t *__restrict__ zeros,
-                                    int64_t N, int64_t K, int g, int64_t U, int64_t nent,
-                                    uint32_t *__restrict__ out) {
-    const int per_unit = 128 / g;
-    const int64_t J = K / g;
-    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nent;
-         idx += (int64_t)gridDim.x * blockDim.x) {
-        const int gg = idx % per_unit;
-        const int r = (idx / per_unit) % 8;
-        const int64_t u = (idx / per_unit / 8) % U;
-        const int64_t o = idx / per_unit / 8 / U;
-        out[idx] = scale_entry(scales, zeros, N, J, o * 8 + r, u * per_unit + gg);
+        const int64_t n = idx / row_words, w = idx - n * row_words;
+        uint32_t v;
+        if (w < cw) v = reinterpret_cast<const uint32_t *>(codes + n * (K / 2))[w];
+        else v = scale_entry(scales, zeros, N, J, n, w - cw);
+        out[idx] = v;
     }
 }
 
@@ -134,12 +115,10 @@ W4_API w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, c
     uint8_t *base = static_cast<uint8_t *>(packed);
     if (layout == W4_LAYOUT_GEMV) {
         const GemvLayout L = gemv_layout(N, K, group);
-        const int64_t nwords = (int64_t)(L.codes_bytes / 4);
-        const int64_t nent = (int64_t)(L.scales_bytes / 4);
-        prepack_gemv_codes<<<grid_for(nwords), 256, 0, stream>>>(codes, N, K, L.U, nwords,
-                                                                 reinterpret_cast<uint32_t *>(base));
-        prepack_gemv_scales<<<grid_for(nent), 256, 0, stream>>>(scales_fp16, zeros, N, K, group, L.U, nent,
-                                                                reinterpret_cast<uint32_t *>(base + L.codes_bytes));
+        const int64_t row_words = (int64_t)(L.row_bytes / 4);
+        const int64_t nwords = (int64_t)(L.total / 4);
+        prepack_gemv_rows<<<grid_for(nwords), 256, 0, stream>>>(codes, scales_fp16, zeros, N, K, group, row_words,
+                                                                nwords, reinterpret_cast<uint32_t *>(base));
     } else {
         const GemmLayout L = gemm_layout(N, K, group);
         const int64_t nwords = (int64_t)(L.codes_bytes / 4);

@@ -6,28 +6,38 @@
 //
 //   y[m, n] = sum_j s[n,j] * sum_{k in j} x[m,k] * (q[n,k] - z[n,j])
 //
-// HBM-bound streaming kernel on the CUDA cores (W4_LAYOUT_GEMV, see w4_layout.cuh).
-//  * Persistent stream-K: the weight is a sequence of T = (N/8) * (Kpad/128) units of
-//    512 bytes (8 rows x 128 k) in octet-major order; CTA c of P (one per SM) owns the
-//    contiguous unit range [t0, t1) with |t1 - t0| differing by at most one between CTAs,
-//    so every SM streams the same number of bytes whatever N and K are.
-//  * Warp w of a CTA takes units t0 + w, t0 + w + W, ... (so the W warps read W
-//    consecutive 512-byte units, i.e. contiguous memory) and keeps a queue of the next
-//    units' codes and scales in registers (128-bit streaming loads that bypass L1), so
-//    each SM keeps ~64 KB of loads in flight. The activations (and the per-32-chunk
-//    activation sums) are staged once per CTA in shared memory with a bulk copy
-//    (cp.async.bulk, bounded mbarrier wait).
-//  * A lane (row r = lane/4, chunk c = lane%4) turns a 16-byte word of codes into bf16
-//    pairs with one AND/OR each
-//    ((w & 0x000F000F) | 0x43004300 is the exact pair 128 + q), multiplies them into fp32
-//    with fma.rn.f32.bf16, and removes the offset per 32-wide chunk with the chunk's
-//    activation sum: sum x*(q - z) = sum x*(128 + q) - (128 + z) * sum x. The chunk
-//    partial times the fp16 group scale is accumulated per octet in registers.
-//  * Octets wholly inside a CTA's range are reduced in shared memory (fixed warp order)
-//    and written. An octet split between CTAs is finished by the last of its CTAs to
-//    arrive on a per-octet counter: it adds the CTAs' partials in CTA order (so results are
-//    deterministic) and resets the counter. Partials and counters live in the caller's
-//    workspace, which every call leaves zero-filled.
+// A streaming kernel on the CUDA cores, layout W4_LAYOUT_GEMV (one record of codes and
+// scales per weight row, see w4_layout.cuh).
+//
+// Integer dot products. The codes are 4-bit integers, so the inner product runs on the
+// integer dot-product unit (dp4a: four 8-bit products and a 32-bit sum per instruction, on
+// a different pipe from the bit operations that unpack the codes). Each thread owns a slice
+// of KC = 128/MT consecutive k and keeps the activations of that slice in registers as
+// 24-bit fixed point with one exponent per slice: X[k] = rint(x[k] * 2^S), |X| < 2^19, with
+// S chosen from the slice's largest |x| (exact for every x within 2^11 of that maximum;
+// smaller ones are rounded to 2^-S, i.e. 2^-19 of the maximum). Three byte planes of 16X
+// (even k) and of X (odd k) meet the code bytes w & 0x0F0F0F0F (q of the even k) and
+// w & 0xF0F0F0F0 (16 q of the odd k), so six dp4a per 8 weights give the exact integer
+// D = 16 * sum X q; per group segment the planes' sums are combined in fp32:
+//   sum x (q - z) = 2^-S (D / 16 - z sum X),  partial += s * that.
+// Every integer sum is exact; the fp32 roundings are those of the per-segment combine and
+// of the row sum, so the result is within a few fp32 roundings of the exact product of the
+// fixed-point activations.
+//
+// Data movement. One persistent block per SM owns a contiguous run of rows. A producer warp
+// streams the block's rows through a ring of shared-memory stages with 1-D bulk copies
+// (one copy per stage: consecutive rows are consecutive records), so the whole ring
+// (~150 KB per SM) is in flight from the first instruction. The activations are converted
+// to byte planes once per block (all threads cooperate, each element once) into an area at
+// the end of the ring that the producer fills only after every thread has loaded its planes
+// into registers. A stage holds one row per "slot" of threads; each thread adds its
+// slice's partial for that row and stores it in shared memory; after the last stage the
+// row sums are formed in a fixed order (bit-identical results run to run).
+//
+// Rows longer than a block's threads can cover (K > 448 KC) are split along K over several
+// blocks; their partial sums go through the caller's workspace and the last block of a row
+// range to arrive adds them in a fixed order. M > MT activation rows run as ceil(M/MT)
+// sweeps over the weights (the launch's second grid dimension).
 #include "w4_common.cuh"
 #include "w4_layout.cuh"
 
@@ -36,455 +46,471 @@
 namespace w4 {
 namespace gemv {
 
-constexpr int SMEM_LIMIT = 100 * 1024;
-constexpr int PF = 4;  // units queued per warp
-
-__device__ __forceinline__ void fma2_bf16(float &a0, float &a1, uint32_t x, uint32_t q) {
-    asm("{\n .reg .b16 xl, xh, ql, qh;\n mov.b32 {xl, xh}, %2;\n mov.b32 {ql, qh}, %3;\n"
-        " fma.rn.f32.bf16 %0, xl, ql, %0;\n fma.rn.f32.bf16 %1, xh, qh, %1;\n}\n"
-        : "+f"(a0), "+f"(a1)
-        : "r"(x), "r"(q));
-}
-
-__device__ __forceinline__ uint32_t magic_pair(uint32_t w) { return (w & 0x000F000Fu) | 0x43004300u; }
-
-// Division of 32-bit unsigned values by an invariant divisor d (Granlund & Montgomery,
-// "Division by invariant integers using multiplication", 1994): with l = ceil(log2 d),
-// m = floor(2^32 (2^l - d) / d) + 1, n / d = (t + ((n - t) >> min(l,1))) >> max(l-1,0)
-// where t = mulhi(m, n). Exact for every n < 2^32.
-struct FastDiv {
-    uint32_t d, m, s1, s2;
-};
-
-inline FastDiv make_fastdiv(uint32_t d) {
-    uint32_t l = 0;
-    while (l < 32 && (1ull << l) < d) ++l;
-    FastDiv f;
-    f.d = d;
-    f.m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d) + 1);
-    f.s1 = l < 1 ? l : 1;
-    f.s2 = l > 1 ? l - 1 : 0;
-    return f;
-}
-
-__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
-    const uint32_t t = __umulhi(f.m, n);
-    return (t + ((n - t) >> f.s1)) >> f.s2;
-}
+constexpr int NCW = 14;                 // consumer warps
+constexpr int NCT = NCW * 32;           // consumer threads
+constexpr int THREADS = NCT + 32;       // + one producer warp
+constexpr int SMEM_MAX = 227 * 1024;
+constexpr int RED_BUDGET = 48 * 1024;   // row-partial buffer
+constexpr int MAX_STAGES = 16;
+constexpr uint32_t SLACK = 64;          // bytes after the ring (reads past a short last slice)
 
 struct Args {
-    const uint16_t *x;
-    const uint8_t *codes;      // packed codes
-    const uint8_t *scales;     // packed scales (u32 entries)
-    void *y;
-    float *ws_part;            // [P][2][8][MT] partials of boundary octets
-    int *ws_count;             // [N8] arrival counters (zero between calls)
+    const uint16_t *x;   // [M, K] bf16
+    const uint8_t *w;    // packed row records
+    void *y;             // [M, N]
+    float *ws_part;      // [kparts][M][N] partial sums (K split only)
+    int *ws_count;       // [sweeps][nrb] arrival counters (K split only; zero between calls)
     int *status;
     int64_t N, K;
-    uint32_t U, T;             // U = units per octet, T = total units (< 2^31)
-    FastDiv divU;
-    uint32_t base, rem, step;  // range of CTA c starts at c*base + min(c, rem)*step
-    FastDiv divB1, divB;       // division by base + step and by base
-    int M, g, out_fp32, nol, pdl;
-    uint32_t sub;              // scale bytes per unit
-    uint32_t off_sx, off_slot;
-    uint32_t off_xf;           // M = 1 kernel: padded bf16 copy of x
-    uint32_t off_ring, off_bars;  // M = 1 kernel: per-warp stage rings and their mbarriers
+    int M, J, g;
+    uint32_t RS;         // row record bytes
+    uint32_t RSp;        // bytes of one row in a stage
+    uint32_t KPB;        // code bytes of one row in a stage (the scales follow)
+    int tpr;             // slices of the whole row
+    int spp;             // slices per K part (threads per row)
+    int kparts;
+    int nslot;           // thread slots (each takes rpt rows of a stage)
+    int rpt;             // rows per thread and stage
+    int rpc;             // rows per block (last block may have fewer)
+    int nrb;             // row blocks
+    int NS, NS_early;    // ring stages; stages issued before the planes are loaded
+    uint32_t SB;         // stage bytes
+    uint32_t off_sx, off_pp, off_red, off_ring, off_planes;
+    int warpred;         // MT > 1 with spp a multiple of 32: partials reduced over the warp first
+    int nred;            // partials per (row, m): spp, or spp / 32 with warpred
+    int out_fp32, pdl;
 };
 
-__device__ __forceinline__ uint32_t range_start(const Args &a, uint32_t c) {
-    return c * a.base + (c < a.rem ? c : a.rem) * a.step;
+__device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int32_t dp4a_su(uint32_t a, uint32_t b, int32_t c) {
+    int32_t d;
+    asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
-__device__ __forceinline__ uint32_t cta_of_unit(const Args &a, uint32_t t) {
-    const uint32_t big = (a.base + a.step) * a.rem;
-    return t < big ? fdiv(t, a.divB1) : a.rem + fdiv(t - big, a.divB);
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
 }
 
-template <int MT, int W>
-__device__ __forceinline__ void flush_octet(uint32_t ol, float (&y)[MT], float *slot, int warp, int lane) {
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-        y[m] += __shfl_xor_sync(FULL, y[m], 1);
-        y[m] += __shfl_xor_sync(FULL, y[m], 2);
-    }
-    if ((lane & 3) == 0) {
-        float *d = slot + (ol * W + warp) * 8 * MT + (lane >> 2) * MT;
-#pragma unroll
-        for (int m = 0; m < MT; ++m) d[m] = y[m];
-    }
-#pragma unroll
-    for (int m = 0; m < MT; ++m) y[m] = 0.0f;
+// 2^e as an fp32 (0 below the subnormal range); e <= 127
+__device__ __forceinline__ float exp2i(int e) {
+    if (e >= -126) return __int_as_float((e + 127) << 23);
+    if (e >= -149) return __int_as_float(1 << (e + 149));
+    return 0.0f;
 }
 
-template <int MT> struct Warps { static constexpr int value = MT == 1 ? 32 : (MT <= 4 ? 16 : 8); };
-
-__device__ __forceinline__ void store_y(const Args &a, int m, int64_t n, float v) {
-    if (a.out_fp32) static_cast<float *>(a.y)[(int64_t)m * a.N + n] = v;
-    else static_cast<__nv_bfloat16 *>(a.y)[(int64_t)m * a.N + n] = __float2bfloat16_rn(v);
-}
-
-// Per-octet reduction of the warps' partials (fixed warp order) and, for octets cut by a
-// range boundary (stream-K partitions only), the cross-CTA fixup: the last CTA to arrive on
-// the octet's counter adds all CTAs' partials in CTA order and resets the counter.
-template <int MT, int W>
-__device__ __forceinline__ void finish(const Args &a, const float *slot, int *flags, uint32_t c, uint32_t t0,
-                                       uint32_t t1, uint32_t o_first, uint32_t o_last, int tid) {
-    constexpr int THREADS = W * 32;
-    const int M = a.M;
-    const uint32_t Uc = a.U;
-    const int nol = (int)(o_last - o_first + 1);
-    for (int idx = tid; idx < nol * 8 * MT; idx += THREADS) {
-        const int ol = idx / (8 * MT), rm = idx - ol * 8 * MT;
-        const int rr = rm / MT, m = rm - rr * MT;
-        float acc = 0.0f;
-        for (int w = 0; w < W; ++w) acc += slot[(ol * W + w) * 8 * MT + rm];
-        const uint32_t o = o_first + ol;
-        const bool inside = o * Uc >= t0 && (o + 1) * Uc <= t1;
-        if (inside) {
-            const int64_t n = (int64_t)o * 8 + rr;
-            if (m < M && n < a.N) store_y(a, m, n, acc);
-        } else {
-            const int which = (o == o_first) ? 0 : 1;
-            a.ws_part[(((int64_t)c * 2 + which) * 8 + rr) * MT + m] = acc;
-        }
-    }
-    // boundary octets (stream-K partitions only): the last CTA to arrive adds all partials
-    // in CTA order and resets the counter
-    const bool b0 = !(o_first * Uc >= t0 && (o_first + 1) * Uc <= t1);
-    const bool b1 = (o_last != o_first) && !(o_last * Uc >= t0 && (o_last + 1) * Uc <= t1);
-    if (!b0 && !b1) return;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        flags[1] = 0;
-        flags[2] = 0;
-        for (int which = 0; which < 2; ++which) {
-            if (!(which == 0 ? b0 : b1)) continue;
-            const uint32_t o = which == 0 ? o_first : o_last;
-            const uint32_t cnt = cta_of_unit(a, (o + 1) * Uc - 1) - cta_of_unit(a, o * Uc) + 1;
-            const int prev = atomicAdd(&a.ws_count[o], 1);
-            flags[1 + which] = (prev == (int)cnt - 1) ? 1 : 0;
-        }
-        __threadfence();
-    }
-    __syncthreads();
-    for (int which = 0; which < 2; ++which) {
-        if (!flags[1 + which]) continue;
-        const uint32_t o = which == 0 ? o_first : o_last;
-        const uint32_t cf = cta_of_unit(a, o * Uc), cl = cta_of_unit(a, (o + 1) * Uc - 1);
-        for (int rm = tid; rm < 8 * MT; rm += THREADS) {
-            const int rr = rm / MT, m = rm - rr * MT;
-            float acc = 0.0f;
-            for (uint32_t k = cf; k <= cl; ++k) {
-                const int wk = (fdiv(range_start(a, k), a.divU) == o) ? 0 : 1;
-                acc += __ldcg(a.ws_part + (((int64_t)k * 2 + wk) * 8 + rr) * MT + m);
-            }
-            const int64_t n = (int64_t)o * 8 + rr;
-            if (m < M && n < a.N) store_y(a, m, n, acc);
-        }
-        if (tid == 0) a.ws_count[o] = 0;
-    }
-}
-
+// Sum of v[m] over the warp for MT values at once: after the exchange at distance 16 (MT >= 2)
+// and 8 (MT = 4) each lane keeps the partial sums of one m, then a butterfly over the
+// remaining distances; lane l ends with the sum for m = l / (32 / MT). Fixed order.
 template <int MT>
-__global__ void __launch_bounds__(Warps<MT>::value * 32, 1) gemv_kernel(const Args a) {
-    constexpr int W = Warps<MT>::value;
-    constexpr int THREADS = W * 32;
-    extern __shared__ __align__(16) uint8_t smem[];
-    int *flags = reinterpret_cast<int *>(smem);   // [1..2] last-arriver flags
-    float *sx = reinterpret_cast<float *>(smem + a.off_sx);
-    float *slot = reinterpret_cast<float *>(smem + a.off_slot);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r = lane >> 2, cc = lane & 3;
-    const uint32_t c = blockIdx.x;
-    const uint32_t t0 = range_start(a, c), t1 = range_start(a, c + 1);
-    const uint32_t o_first = fdiv(t0, a.divU), o_last = fdiv(t1 - 1, a.divU);
-    const int M = a.M;
-    const uint32_t Kc = (uint32_t)a.K, Uc = a.U;
-    const int nck = (int)(Uc * 4);  // 32-wide chunks per row (padded)
-
-    // ---- the weight stream does not depend on earlier kernels: start it first
-    const uint32_t tb = t0 + (uint32_t)warp;
-    const int per_unit = 128 / a.g;
-    const uint32_t sc_lane = (uint32_t)(r * per_unit + (cc * 32) / a.g) * 4;
-    const uint8_t *cp = a.codes + (size_t)tb * 512 + lane * 16;
-    const uint8_t *sp = a.scales + (size_t)tb * a.sub + sc_lane;
-    const size_t cstep = (size_t)W * 512, sstep = (size_t)W * a.sub;
-    uint4 qv[PF];
-    uint32_t ev[PF];
-#pragma unroll
-    for (int i = 0; i < PF; ++i) {
-        if (tb + (uint32_t)(i * W) < t1) {
-            qv[i] = ldg_stream(cp + i * cstep);
-            ev[i] = __ldg(reinterpret_cast<const uint32_t *>(sp + i * sstep));
-        }
+__device__ __forceinline__ float warp_transpose_sum(const float (&v)[MT], int lane) {
+    float r;
+    if constexpr (MT == 1) {
+        r = v[0];
+    } else if constexpr (MT == 2) {
+        const bool b4 = lane & 16;
+        r = (b4 ? v[1] : v[0]) + __shfl_xor_sync(FULL, b4 ? v[0] : v[1], 16);
+    } else {
+        const bool b4 = lane & 16, b3 = lane & 8;
+        const float k0 = (b4 ? v[2] : v[0]) + __shfl_xor_sync(FULL, b4 ? v[0] : v[2], 16);
+        const float k1 = (b4 ? v[3] : v[1]) + __shfl_xor_sync(FULL, b4 ? v[1] : v[3], 16);
+        r = (b3 ? k1 : k0) + __shfl_xor_sync(FULL, b3 ? k0 : k1, 8);
     }
-    cp += PF * cstep;
-    sp += PF * sstep;
-
-    for (int i = tid; i < a.nol * W * 8 * MT; i += THREADS) slot[i] = 0.0f;
-    // activations may be written by the previous kernel in the stream
-    if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
-    // activation sums of every 32-wide chunk (chunks past K are zero)
-    for (int idx = tid; idx < MT * nck; idx += THREADS) {
-        const int m = idx / nck, ck = idx - m * nck;
-        float s = 0.0f;
-        if (m < M && (uint32_t)ck * 32 < Kc) {
-            const uint4 *xv = reinterpret_cast<const uint4 *>(a.x + (int64_t)m * a.K + ck * 32);
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const uint4 v = __ldg(xv + t);
-                s = __fadd_rn(__fadd_rn(s, bf16_lo(v.x)), bf16_hi(v.x));
-                s = __fadd_rn(__fadd_rn(s, bf16_lo(v.y)), bf16_hi(v.y));
-                s = __fadd_rn(__fadd_rn(s, bf16_lo(v.z)), bf16_hi(v.z));
-                s = __fadd_rn(__fadd_rn(s, bf16_lo(v.w)), bf16_hi(v.w));
-            }
-        }
-        sx[idx] = s;
-    }
-    __syncthreads();
-    if (a.pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-    float y[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) y[m] = 0.0f;
-    uint32_t cur_ol = 0xffffffffu;  // octet of the accumulated partial, relative to o_first
-    for (uint32_t tq = tb; tq < t1; tq += (uint32_t)(PF * W)) {
-#pragma unroll
-        for (int i = 0; i < PF; ++i) {
-            const uint32_t t = tq + (uint32_t)(i * W);
-            if (t >= t1) break;
-            const uint4 wq = qv[i];
-            const uint32_t e = ev[i];
-            if (t + (uint32_t)(PF * W) < t1) {
-                qv[i] = ldg_stream(cp);
-                ev[i] = __ldg(reinterpret_cast<const uint32_t *>(sp));
-            }
-            cp += cstep;
-            sp += sstep;
-            const uint32_t o = fdiv(t, a.divU);
-            const uint32_t ol = o - o_first;
-            if (ol != cur_ol) {
-                if (cur_ol != 0xffffffffu) flush_octet<MT, W>(cur_ol, y, slot, warp, lane);
-                cur_ol = ol;
-            }
-            const uint32_t k0 = (t - o * Uc) * 128u + (uint32_t)cc * 32u;
-            if (k0 >= Kc) continue;
-            const float scl = __half2float(__ushort_as_half((unsigned short)(e & 0xFFFF)));
-            const float cz = (float)(int)(int16_t)(e >> 16) + 128.0f;
-            uint32_t p[4][4];
-            const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                p[q][0] = magic_pair(wv[q]);
-                p[q][1] = magic_pair(wv[q] >> 4);
-                p[q][2] = magic_pair(wv[q] >> 8);
-                p[q][3] = magic_pair(wv[q] >> 12);
-            }
-            const uint32_t ck = k0 >> 5;
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                if (m >= M) break;
-                float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-                const uint4 *xp = reinterpret_cast<const uint4 *>(a.x + (int64_t)m * a.K + k0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 xv = __ldg(xp + q);
-                    fma2_bf16(a0, a1, xv.x, p[q][0]);
-                    fma2_bf16(a2, a3, xv.y, p[q][1]);
-                    fma2_bf16(a0, a1, xv.z, p[q][2]);
-                    fma2_bf16(a2, a3, xv.w, p[q][3]);
-                }
-                y[m] = fmaf(scl, fmaf(-cz, sx[m * nck + ck], (a0 + a1) + (a2 + a3)), y[m]);
-            }
-        }
-    }
-    if (cur_ol != 0xffffffffu) flush_octet<MT, W>(cur_ol, y, slot, warp, lane);
-    __syncthreads();
-
-    finish<MT, W>(a, slot, flags, c, t0, t1, o_first, o_last, tid);
+    for (int off = 32 / MT / 2; off >= 1; off >>= 1) r += __shfl_xor_sync(FULL, r, off);
+    return r;
 }
 
-// ---------------------------------------------------------------- M = 1 kernel
-//
-// Each warp streams a contiguous run of 512-byte units through its own ring of shared-memory
-// stages filled by 1-D bulk copies (one copy of codes and one of scales per stage of SU
-// units, issued by the warp's lane 0, completion on an mbarrier), so loading costs almost no
-// instructions; lanes read their 16 bytes of codes and their scale entry from shared memory.
-// x is staged once per CTA as bf16 with 16 bytes of padding after every 32 values, so the
-// four 32-wide chunks a warp reads at once start in different banks.
-constexpr int W1 = 16;   // warps of the M = 1 kernel
-constexpr int SU = 8;    // units per stage
-constexpr int NS = 2;    // stages per warp
+// Geometry shared by host and device for a slice width KC.
+template <int MT> struct Geo {
+    static constexpr int KC = 128 / MT;       // k per slice
+    static constexpr int NCH = KC / 32;       // 16-byte code chunks per slice
+    static constexpr int WPS = KC / 8;        // code words per slice
+    static constexpr int PW = 6 * WPS;        // plane words per slice and activation row
+    static constexpr int PSTRIDE = PW + 4;    // padded (conflict-free 16-byte loads)
+    static constexpr int RPT = MT == 1 ? 2 : 1;  // rows per thread and stage (registers allow two at MT = 1)
+};
 
-__device__ __forceinline__ uint32_t xb_index(uint32_t k) { return k + (k >> 5) * 8; }
-
-// One unit for one lane: 16 bytes of codes (32 weights of row r, chunk at k0) against the
-// padded bf16 x at xp, offset removed with the chunk sum sxc, times the group scale.
-__device__ __forceinline__ void unit_m1(float &y, const uint4 wq, uint32_t e, const uint4 *xp, float sxc) {
-    const float scl = __half2float(__ushort_as_half((unsigned short)(e & 0xFFFF)));
-    const float cz = (float)(int)(int16_t)(e >> 16) + 128.0f;
-    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-    const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint4 xv = xp[q];
-        fma2_bf16(a0, a1, xv.x, magic_pair(wv[q]));
-        fma2_bf16(a2, a3, xv.y, magic_pair(wv[q] >> 4));
-        fma2_bf16(a0, a1, xv.z, magic_pair(wv[q] >> 8));
-        fma2_bf16(a2, a3, xv.w, magic_pair(wv[q] >> 12));
-    }
-    y = fmaf(scl, fmaf(-cz, sxc, (a0 + a1) + (a2 + a3)), y);
-}
-
-// shared-memory bytes of the M = 1 kernel's regions
-inline uint32_t xb_bytes(uint32_t U) { return U * 4 * 40 * 2; }              // padded bf16 x
-inline uint32_t ring_bytes(uint32_t sub) { return W1 * NS * SU * (512 + sub); }
-
-__global__ void __launch_bounds__(W1 * 32, 1) gemv1_kernel(const Args a) {
-    constexpr int W = W1, THREADS = W1 * 32;
+template <int MT, int G>
+__global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
+    using GE_ = Geo<MT>;
+    constexpr int KC = GE_::KC, NCH = GE_::NCH, WPS = GE_::WPS, PSTRIDE = GE_::PSTRIDE;
+    constexpr int GS = G < KC ? G : KC;       // k per combine segment
+    constexpr int NSEG = KC / GS;             // segments per slice
+    constexpr int CPS = GS / 32;              // chunks per segment
+    constexpr int RPT = GE_::RPT;             // rows per thread and stage
     extern __shared__ __align__(16) uint8_t smem[];
-    int *flags = reinterpret_cast<int *>(smem);
-    float *sx = reinterpret_cast<float *>(smem + a.off_sx);
-    uint16_t *xb = reinterpret_cast<uint16_t *>(smem + a.off_xf);
-    float *slot = reinterpret_cast<float *>(smem + a.off_slot);
-    uint8_t *ring = smem + a.off_ring;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + a.off_bars);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    uint64_t *empty = full + MAX_STAGES;
+    uint64_t *planes_done = empty + MAX_STAGES;
+    int *abort_flag = reinterpret_cast<int *>(planes_done + 1);
+    int *last_flag = abort_flag + 1;
+    int *sx = reinterpret_cast<int *>(smem + a.off_sx);          // [MT][spp][NCH] sums of X per chunk
+    float *pp = reinterpret_cast<float *>(smem + a.off_pp);      // [MT][spp] 2^-S per slice
+    float *red = reinterpret_cast<float *>(smem + a.off_red);    // [rpc][MT][spp] row partials
+    const uint32_t ring = smem_addr(smem + a.off_ring);
+    uint32_t *planes = reinterpret_cast<uint32_t *>(smem + a.off_planes);  // [spp][PSTRIDE], one row m at a time
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r = lane >> 2, cc = lane & 3;
-    const uint32_t c = blockIdx.x;
-    const uint32_t t0 = range_start(a, c), t1 = range_start(a, c + 1);
-    const uint32_t o_first = fdiv(t0, a.divU), o_last = fdiv(t1 - 1, a.divU);
-    const uint32_t Kc = (uint32_t)a.K, Uc = a.U;
-    const int nck = (int)(Uc * 4);
-    const uint32_t sub = a.sub, stage_bytes = SU * (512 + sub);
+    const int kp = (int)(blockIdx.x % (unsigned)a.kparts);
+    const int rb = (int)(blockIdx.x / (unsigned)a.kparts);
+    const int m0 = (int)blockIdx.y * MT;
+    const int64_t row0 = (int64_t)rb * a.rpc;
+    const int rows = (int)((a.N - row0) < a.rpc ? (a.N - row0) : a.rpc);
+    const int nstages = (rows + a.nslot * a.rpt - 1) / (a.nslot * a.rpt);
+    const int sl0 = kp * a.spp;                                    // first slice of this part
+    const int nsl = (a.tpr - sl0) < a.spp ? (a.tpr - sl0) : a.spp;  // slices of this part
+    const int64_t k0 = (int64_t)sl0 * KC;                          // first k of this part
+    const int J0 = (int)(k0 / a.g);                                // first group of this part
 
-    // this warp's contiguous run [wt0, wt1) of the CTA's units, cut into stages of at most SU
-    // units that never cross an octet boundary (so a stage has one octet and one flush)
-    const uint32_t n = t1 - t0;
-    const uint32_t wt0 = t0 + (uint32_t)(((uint64_t)n * warp) / W);
-    const uint32_t wt1 = t0 + (uint32_t)(((uint64_t)n * (warp + 1)) / W);
-    uint8_t *wring = ring + (size_t)warp * NS * stage_bytes;
-    uint64_t *wbar = bars + warp * NS;
-    struct Cursor {
-        uint32_t t, o, u;  // next unit, its octet and its position in the octet
-    };
-    auto stage_len = [&](const Cursor &q) {
-        uint32_t cnt = wt1 - q.t;
-        cnt = cnt < (uint32_t)SU ? cnt : (uint32_t)SU;
-        return cnt < Uc - q.u ? cnt : Uc - q.u;
-    };
-    auto advance = [&](Cursor &q, uint32_t cnt) {
-        q.t += cnt;
-        q.u += cnt;
-        if (q.u == Uc) { q.u = 0; ++q.o; }
-    };
-    Cursor cons;
-    cons.t = wt0;
-    cons.o = fdiv(wt0, a.divU);
-    cons.u = wt0 - cons.o * Uc;
-    Cursor prod = cons;
-    uint32_t jp = 0;  // stages issued
-    // lane 0 fills the producer cursor's next stage into ring slot jp % NS
-    auto issue = [&]() {
-        const uint32_t cnt = stage_len(prod);
-        uint8_t *dst = wring + (jp % NS) * stage_bytes;
-        uint64_t *bar = wbar + (jp % NS);
-        mbar_arrive_expect_tx(bar, cnt * (512 + sub));
-        bulk_g2s(dst, a.codes + (size_t)prod.t * 512, cnt * 512, bar);
-        bulk_g2s(dst + SU * 512, a.scales + (size_t)prod.t * sub, cnt * sub, bar);
-    };
-    // ---- the weight stream does not depend on earlier kernels: start it first
-    if (lane == 0) {
-        for (int j = 0; j < NS; ++j) mbar_init(wbar + j, 1);
+    if (tid == 0) {
+        for (int i = 0; i < a.NS; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, NCW);
+        }
+        mbar_init(planes_done, NCW);
+        *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int j = 0; j < NS && prod.t < wt1; ++j) {  // warp-uniform cursor, lane 0 issues
-        if (lane == 0) issue();
-        advance(prod, stage_len(prod));
-        ++jp;
-    }
-    for (int i = tid; i < a.nol * W * 8; i += THREADS) slot[i] = 0.0f;
-    // activations may be written by the previous kernel in the stream
-    if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
-    // x as padded bf16 and the sum of every 32-wide chunk (chunks past K are zero)
-    for (int ck = tid; ck < nck; ck += THREADS) {
-        float s = 0.0f;
-        const bool live = (uint32_t)ck * 32 < Kc;
-        const uint4 *xv = reinterpret_cast<const uint4 *>(a.x + ck * 32);
-        uint4 *dst = reinterpret_cast<uint4 *>(xb + xb_index((uint32_t)ck * 32));
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const uint4 u4 = live ? __ldg(xv + t) : make_uint4(0u, 0u, 0u, 0u);
-            s = __fadd_rn(__fadd_rn(s, bf16_lo(u4.x)), bf16_hi(u4.x));
-            s = __fadd_rn(__fadd_rn(s, bf16_lo(u4.y)), bf16_hi(u4.y));
-            s = __fadd_rn(__fadd_rn(s, bf16_lo(u4.z)), bf16_hi(u4.z));
-            s = __fadd_rn(__fadd_rn(s, bf16_lo(u4.w)), bf16_hi(u4.w));
-            dst[t] = u4;
-        }
-        sx[ck] = s;
-    }
     __syncthreads();
-    if (a.pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    const int per_unit = 128 / a.g;
-    const uint32_t sc_lane = (uint32_t)(r * per_unit + (cc * 32) / a.g);  // u32 index in a unit's scales
-    float y[1] = {0.0f};
-    uint32_t cur_ol = 0xffffffffu;
-    const bool kpad = (Kc & 127u) != 0;
-    bool ok = true;
-    uint32_t j = 0;  // stages consumed
-    for (; cons.t < wt1; ++j) {
-        const uint32_t sl = j % NS;
-        // lane 0 polls; every lane then takes the (now immediate) wait for its own acquire
-        bool got = true;
-        if (lane == 0) got = mbar_wait_bounded(wbar + sl, (j / NS) & 1u, a.status);
-        got = __shfl_sync(FULL, got ? 1 : 0, 0) != 0;
-        if (!got) { ok = false; break; }
-        (void)mbar_try_wait(wbar + sl, (j / NS) & 1u);
-        const uint32_t cnt = stage_len(cons);
-        const uint32_t ol = cons.o - o_first;
-        if (ol != cur_ol) {
-            if (cur_ol != 0xffffffffu) flush_octet<1, W>(cur_ol, y, slot, warp, lane);
-            cur_ol = ol;
+    if (warp == NCW) {
+        // ------------------------------------------------ producer: stream the rows
+        if (a.pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        if (lane == 0) {
+            const uint8_t *src0 = a.w + (size_t)row0 * a.RS;
+            int issued = 0;
+            bool ok = true;
+            for (int s = 0; s < nstages && ok; ++s) {
+                const int slot = s % a.NS;
+                if (s >= a.NS) {
+                    ok = mbar_wait_abortable(empty + slot, ((s / a.NS) - 1) & 1, abort_flag, a.status, 2000000000ull);
+                } else if (s == a.NS_early) {
+                    ok = mbar_wait_abortable(planes_done, 0, abort_flag, a.status, 2000000000ull);
+                }
+                if (!ok) break;
+                const int r0 = s * a.nslot * a.rpt;
+                const int nr = (rows - r0) < a.nslot * a.rpt ? (rows - r0) : a.nslot * a.rpt;
+                uint8_t *dst = smem + a.off_ring + (size_t)slot * a.SB;
+                if (a.kparts == 1) {
+                    mbar_arrive_expect_tx(full + slot, (uint32_t)nr * a.RS);
+                    bulk_g2s(dst, src0 + (size_t)r0 * a.RS, (uint32_t)nr * a.RS, full + slot);
+                } else {
+                    // this part's codes and scales of each row
+                    const uint32_t cb = (uint32_t)(((k0 + (int64_t)nsl * KC < a.K ? k0 + (int64_t)nsl * KC : a.K) - k0) / 2);
+                    const uint32_t scb0 = (uint32_t)(a.K / 2) + 4u * (uint32_t)J0;
+                    const uint32_t scb = (kp == a.kparts - 1) ? a.RS - scb0 : 4u * (uint32_t)(nsl * KC / a.g);
+                    mbar_arrive_expect_tx(full + slot, (uint32_t)nr * (cb + scb));
+                    for (int r = 0; r < nr; ++r) {
+                        const uint8_t *rs = src0 + (size_t)(r0 + r) * a.RS;
+                        bulk_g2s(dst + (size_t)r * a.RSp, rs + k0 / 2, cb, full + slot);
+                        bulk_g2s(dst + (size_t)r * a.RSp + a.KPB, rs + scb0, scb, full + slot);
+                    }
+                }
+                ++issued;
+            }
+            // no bulk copy may be in flight when the block exits
+            for (int s = issued - a.NS > 0 ? issued - a.NS : 0; s < issued; ++s)
+                (void)mbar_wait_bounded(full + (s % a.NS), (s / a.NS) & 1, a.status);
         }
-        const uint8_t *st = wring + sl * stage_bytes;
-        const uint4 *cw = reinterpret_cast<const uint4 *>(st) + lane;
-        const uint32_t *sw = reinterpret_cast<const uint32_t *>(st + SU * 512) + sc_lane;
-        const uint32_t k0 = cons.u * 128u + (uint32_t)cc * 32u;
-        const uint4 *xp = reinterpret_cast<const uint4 *>(xb + xb_index(k0));
-        const float *sxp = sx + (k0 >> 5);
-#pragma unroll
-        for (int i = 0; i < SU; ++i)
-            if ((uint32_t)i < cnt && (!kpad || k0 + (uint32_t)i * 128u < Kc))
-                unit_m1(y[0], cw[i * 32], sw[i * (sub >> 2)], xp + i * 20, sxp[i * 4]);
-        advance(cons, cnt);
-        // every lane has read the slot: lane 0 refills it with the next stage
         __syncwarp();
-        if (prod.t < wt1) {
-            if (lane == 0) issue();
-            advance(prod, stage_len(prod));
-            ++jp;
+    } else {
+        // ------------------------------------------------ consumers
+        // activations may be written by the previous kernel in the stream
+        if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+
+        // this thread's slice; its chunks are visited in an order rotated per lane so that
+        // the 16-byte code loads of a warp hit distinct banks (planes are loaded in that order)
+        const int slot = tid / a.spp, sl = tid - slot * a.spp;
+        const bool active = slot < a.nslot && sl < nsl;
+        constexpr int ROT_DIV = 8 / NCH;          // lanes sharing a rotation
+        const int rraw = (lane / ROT_DIV) % NCH;
+        const int rot = NSEG == 1 ? rraw : rraw / CPS * CPS;   // segments keep their chunks together
+        const int srot = NSEG == 1 ? 0 : rot / CPS;          // rotation in segments
+        uint32_t xp[MT][NCH][4][6];
+        float q16[MT], q16x256[MT], q16x65536[MT], sxf[MT][NSEG];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            // (1) byte planes of activation row m0 + m, one task per 8 consecutive k; the loads
+            // of XB rounds of tasks are issued together so that their latencies overlap
+            const int tasks = a.spp * WPS;
+            constexpr int XB = 4;
+            for (int tb = 0; tb < tasks; tb += XB * NCT) {
+                uint4 xv[XB];
+#pragma unroll
+                for (int r = 0; r < XB; ++r) {
+                    const int t = tb + r * NCT + warp * 32 + lane;
+                    const int tsl = t / WPS, wi = t - tsl * WPS;
+                    const int64_t k = k0 + (int64_t)tsl * KC + wi * 8;
+                    const bool live = t < tasks && tsl < nsl && m0 + m < a.M && k < a.K;
+                    xv[r] = live ? __ldg(reinterpret_cast<const uint4 *>(a.x + (int64_t)(m0 + m) * a.K + k))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int r = 0; r < XB; ++r) {
+                    if (tb + r * NCT + warp * 32 >= tasks) break;  // uniform over the warp
+                    const int t = tb + r * NCT + warp * 32 + lane;
+                    const int tsl = t / WPS, wi = t - tsl * WPS;
+                    const uint32_t e[4] = {xv[r].x, xv[r].y, xv[r].z, xv[r].w};
+                    // largest magnitude pattern of the slice (bf16 bits order like magnitudes)
+                    uint32_t mx = 0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) mx = max(mx, max(e[i] & 0x7FFFu, (e[i] >> 16) & 0x7FFFu));
+#pragma unroll
+                    for (int off = WPS / 2; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(FULL, mx, off));
+                    // exponent of the largest |x|: |x| in [2^ex, 2^(ex+1))
+                    int ex;
+                    if (mx >= 0x80u) ex = (int)(mx >> 7) - 127;
+                    else ex = (31 - __clz((int)(mx | 1u))) - 133;
+                    const int S = 18 - ex;
+                    const float f1 = exp2i(S < 127 ? S : 127), f2 = exp2i(S < 127 ? 0 : S - 127);
+                    int X[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t bb = (i & 1) ? (e[i >> 1] >> 16) : (e[i >> 1] & 0xFFFFu);
+                        const float sv = __fmul_rn(__fmul_rn(__uint_as_float(bb << 16), f1), f2);
+                        X[i] = __float_as_int(__fadd_rn(sv, 12582912.0f)) - 0x4B400000;
+                    }
+                    if (mx >= 0x7F80u || mx == 0u) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) X[i] = 0;
+                    }
+                    // planes: even k as 16 X, odd k as X; byte p of each in 4-byte words
+                    uint32_t pw[6];
+#pragma unroll
+                    for (int par = 0; par < 2; ++par) {
+                        const uint32_t sh = par ? 0u : 4u;
+                        const uint32_t V0 = (uint32_t)X[par] << sh, V1 = (uint32_t)X[2 + par] << sh;
+                        const uint32_t V2 = (uint32_t)X[4 + par] << sh, V3 = (uint32_t)X[6 + par] << sh;
+#pragma unroll
+                        for (int pl = 0; pl < 3; ++pl) {
+                            const uint32_t lo = __byte_perm(V0, V1, (uint32_t)(pl | ((4 + pl) << 4)));
+                            const uint32_t hi = __byte_perm(V2, V3, (uint32_t)(pl | ((4 + pl) << 4)));
+                            pw[par * 3 + pl] = __byte_perm(lo, hi, 0x5410u);
+                        }
+                    }
+                    int xs = X[0] + X[1] + X[2] + X[3] + X[4] + X[5] + X[6] + X[7];
+                    xs += __shfl_xor_sync(FULL, xs, 1);
+                    xs += __shfl_xor_sync(FULL, xs, 2);
+                    if (t < tasks) {
+                        uint32_t *dst = planes + tsl * PSTRIDE + wi * 6;
+                        reinterpret_cast<uint2 *>(dst)[0] = make_uint2(pw[0], pw[1]);
+                        reinterpret_cast<uint2 *>(dst)[1] = make_uint2(pw[2], pw[3]);
+                        reinterpret_cast<uint2 *>(dst)[2] = make_uint2(pw[4], pw[5]);
+                        if ((wi & 3) == 0) sx[(m * a.spp + tsl) * NCH + (wi >> 2)] = xs;
+                        if (wi == 0)
+                            pp[m * a.spp + tsl] =
+                                (mx >= 0x7F80u) ? __int_as_float(0x7FC00000) : (mx == 0u ? 0.0f : exp2i(-S));
+                    }
+                }
+            }
+            named_bar_sync(1, NCT);
+            // (2) this thread's planes of row m into registers
+            const uint32_t pb = smem_addr(planes + (active ? sl : 0) * PSTRIDE);
+#pragma unroll
+            for (int j = 0; j < NCH; ++j) {
+                const int c = (j + rot) % NCH;
+#pragma unroll
+                for (int q = 0; q < 6; ++q) {  // 24 words of chunk c: 6 loads of 4
+                    const uint4 v = lds128(pb + (uint32_t)(c * 24 + q * 4) * 4u);
+                    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) xp[m][j][(q * 4 + r) / 6][(q * 4 + r) % 6] = vv[r];
+                }
+            }
+            const float p = active ? pp[m * a.spp + sl] : 0.0f;
+            q16[m] = __fmul_rn(p, 0.0625f);
+            q16x256[m] = __fmul_rn(p, 16.0f);
+            q16x65536[m] = __fmul_rn(p, 4096.0f);
+#pragma unroll
+            for (int js = 0; js < NSEG; ++js) {
+                const int seg = (js + srot) % NSEG;
+                int sum = 0;
+#pragma unroll
+                for (int c = 0; c < CPS; ++c) sum += active ? sx[(m * a.spp + sl) * NCH + seg * CPS + c] : 0;
+                sxf[m][js] = __fmul_rn((float)sum, p);
+            }
+            if (m + 1 < MT) named_bar_sync(1, NCT);  // the next row's tasks overwrite the planes
+        }
+        if (a.pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(planes_done);
+
+        // (3) the rows: RPT per thread and stage (rows slot, slot + nslot, ... of the stage)
+        const uint32_t code_off = (uint32_t)sl * (KC / 2);
+        uint32_t sc_off[NSEG];  // byte offset of each segment's scale word in a row
+        bool seg_live[NSEG];
+#pragma unroll
+        for (int js = 0; js < NSEG; ++js) {
+            const int seg = (js + srot) % NSEG;
+            const int jg = (int)((k0 + (int64_t)sl * KC + seg * GS) / a.g);
+            seg_live[js] = jg < a.J;
+            sc_off[js] = a.KPB + 4u * (uint32_t)(jg - J0);
+        }
+        const int SR = a.nslot * RPT;  // rows per stage
+        bool ok = true;
+        for (int s = 0; s < nstages; ++s) {
+            const int slot_s = s % a.NS;
+            bool got = true;
+            if (lane == 0) got = mbar_wait_abortable(full + slot_s, (s / a.NS) & 1, abort_flag, a.status, 2000000000ull);
+            got = __shfl_sync(FULL, got ? 1 : 0, 0) != 0;
+            if (!got) { ok = false; break; }
+            (void)mbar_try_wait_short(full + slot_s, (s / a.NS) & 1);
+            const uint32_t sbase = ring + (uint32_t)slot_s * a.SB;
+            float yv[RPT][MT];
+            bool live[RPT];
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                live[i] = active && s * SR + slot + i * a.nslot < rows;
+#pragma unroll
+                for (int m = 0; m < MT; ++m) yv[i][m] = 0.0f;
+            }
+            if (live[0]) {
+                uint32_t rbase[RPT];
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) rbase[i] = sbase + (uint32_t)(slot + i * a.nslot) * a.RSp;
+#pragma unroll
+                for (int js = 0; js < NSEG; ++js) {
+                    // independent accumulators per row and plane
+                    uint32_t A0[RPT][MT], A1[RPT][MT];
+                    int32_t A2[RPT][MT];
+#pragma unroll
+                    for (int i = 0; i < RPT; ++i)
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) { A0[i][m] = 0u; A1[i][m] = 0u; A2[i][m] = 0; }
+#pragma unroll
+                    for (int jc = 0; jc < CPS; ++jc) {
+                        const int j = js * CPS + jc;
+                        const uint32_t coff = code_off + (uint32_t)(((j + rot) % NCH) * 16);
+                        uint4 cj[RPT];
+#pragma unroll
+                        for (int i = 0; i < RPT; ++i)
+                            cj[i] = (i == 0 || live[i]) ? lds128(rbase[i] + coff) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+#pragma unroll
+                            for (int i = 0; i < RPT; ++i) {
+                                const uint32_t wv = w == 0 ? cj[i].x : w == 1 ? cj[i].y : w == 2 ? cj[i].z : cj[i].w;
+                                const uint32_t L = wv & 0x0F0F0F0Fu, H = wv & 0xF0F0F0F0u;
+#pragma unroll
+                                for (int m = 0; m < MT; ++m) {
+                                    A0[i][m] = dp4a_uu(xp[m][j][w][0], L, A0[i][m]);
+                                    A1[i][m] = dp4a_uu(xp[m][j][w][1], L, A1[i][m]);
+                                    A2[i][m] = dp4a_su(xp[m][j][w][2], L, A2[i][m]);
+                                    A0[i][m] = dp4a_uu(xp[m][j][w][3], H, A0[i][m]);
+                                    A1[i][m] = dp4a_uu(xp[m][j][w][4], H, A1[i][m]);
+                                    A2[i][m] = dp4a_su(xp[m][j][w][5], H, A2[i][m]);
+                                }
+                            }
+                        }
+                    }
+                    if (seg_live[js]) {
+#pragma unroll
+                        for (int i = 0; i < RPT; ++i) {
+                            if (i > 0 && !live[i]) continue;
+                            const uint32_t e = lds32(rbase[i] + sc_off[js]);
+                            const float scl = __half2float(__ushort_as_half((unsigned short)(e & 0xFFFFu)));
+                            const float zf = (float)(int)(int16_t)(e >> 16);
+#pragma unroll
+                            for (int m = 0; m < MT; ++m) {
+                                // (D / 16) 2^-S with D = A0 + 256 A1 + 65536 A2
+                                float d = __fmul_rn((float)A0[i][m], q16[m]);
+                                d = __fmaf_rn((float)A1[i][m], MT == 1 ? q16x256[m] : __fmul_rn(q16[m], 256.0f), d);
+                                d = __fmaf_rn((float)A2[i][m], MT == 1 ? q16x65536[m] : __fmul_rn(q16[m], 65536.0f), d);
+                                yv[i][m] = __fmaf_rn(scl, __fmaf_rn(-zf, sxf[m][js], d), yv[i][m]);
+                            }
+                        }
+                    }
+                }
+                if (!a.warpred) {
+#pragma unroll
+                    for (int i = 0; i < RPT; ++i) {
+                        if (!live[i]) continue;
+                        const uint32_t rl = (uint32_t)(s * SR + slot + i * a.nslot);
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) red[(rl * MT + m) * (uint32_t)a.nred + sl] = yv[i][m];
+                    }
+                }
+            }
+            if (MT > 1 && a.warpred) {
+                // the warp's 32 slices belong to one row: transpose-reduce its MT partials so
+                // that lane l ends with the warp's sum for m = l / (32 / MT)
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) {
+                    const float r = warp_transpose_sum<MT>(yv[i], lane);
+                    const int rl = s * SR + slot + i * a.nslot;
+                    if (slot < a.nslot && rl < rows && (lane & (32 / MT - 1)) == 0)
+                        red[((uint32_t)rl * MT + lane / (32 / MT)) * (uint32_t)a.nred + sl / 32] = r;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + slot_s);
+        }
+        if (!ok) *(volatile int *)abort_flag = 1;
+
+        // (4) row sums in a fixed order: one warp per (row, m)
+        named_bar_sync(1, NCT);
+        const bool aborted = *(volatile int *)abort_flag != 0;
+        float *outp = nullptr;
+        if (a.kparts > 1) outp = a.ws_part + (size_t)kp * a.M * a.N;
+        for (int o = warp; o < rows * MT; o += NCW) {
+            const int rl = o / MT, m = o - rl * MT;
+            float acc = 0.0f;
+            const int nv = a.warpred ? (nsl + 31) / 32 : nsl;
+            for (int i = lane; i < nv; i += 32) acc += red[(size_t)o * a.nred + i];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(FULL, acc, off);
+            const int64_t n = row0 + rl;
+            if (lane == 0 && m0 + m < a.M && !aborted) {
+                if (outp) outp[(int64_t)(m0 + m) * a.N + n] = acc;
+                else if (a.out_fp32) static_cast<float *>(a.y)[(int64_t)(m0 + m) * a.N + n] = acc;
+                else static_cast<__nv_bfloat16 *>(a.y)[(int64_t)(m0 + m) * a.N + n] = __float2bfloat16_rn(acc);
+            }
+        }
+        if (a.kparts > 1) {
+            // the last block of the row range to arrive adds the parts in order and resets the counter
+            __threadfence();
+            named_bar_sync(1, NCT);
+            int *cnt = a.ws_count + (size_t)blockIdx.y * a.nrb + rb;
+            if (tid == 0) {
+                const int prev = atomicAdd(cnt, 1);
+                *last_flag = (prev == a.kparts - 1) ? 1 : 0;
+                __threadfence();
+            }
+            named_bar_sync(1, NCT);
+            if (*last_flag) {
+                for (int o = tid; o < rows * MT; o += NCT) {
+                    const int rl = o / MT, m = o - rl * MT;
+                    if (m0 + m >= a.M) continue;
+                    const int64_t n = row0 + rl, idx = (int64_t)(m0 + m) * a.N + n;
+                    float acc = 0.0f;
+                    for (int p = 0; p < a.kparts; ++p) acc += __ldcg(a.ws_part + (size_t)p * a.M * a.N + idx);
+                    if (aborted) continue;
+                    if (a.out_fp32) static_cast<float *>(a.y)[idx] = acc;
+                    else static_cast<__nv_bfloat16 *>(a.y)[idx] = __float2bfloat16_rn(acc);
+                }
+                if (tid == 0) *cnt = 0;
+            }
         }
     }
-    if (cur_ol != 0xffffffffu) flush_octet<1, W>(cur_ol, y, slot, warp, lane);
-    // no bulk copy may still be in flight when the CTA exits: after a failed wait, wait
-    // (bounded) for every stage this warp issued and did not consume
-    if (!ok && lane == 0)
-        for (uint32_t q = j; q < jp; ++q) (void)mbar_wait_bounded(wbar + q % NS, (q / NS) & 1u, a.status);
-    __syncthreads();
-    finish<1, W>(a, slot, flags, c, t0, t1, o_first, o_last, tid);
 }
 
 // ------------------------------------------------------------------ host side
 
 struct Plan {
     Args a;
-    int P, smem;
-    bool aligned;  // whole octets per block
+    int MT, sweeps, grid_x, smem;
 };
 
 static int sm_count_cached() {
@@ -496,150 +522,147 @@ static int sm_count_cached() {
     return cache[dev];
 }
 
-// Work partition. With N8 octets of U units each and S SMs: if whole octets split evenly
-// enough (fewer octets than SMs; the busiest SM at most ~8% above the mean; or its extra
-// units cheaper than the cross-CTA fixup), every CTA gets whole octets and no partial sum
-// crosses CTAs; otherwise the unit stream is split evenly (stream-K) and octets cut by a
-// range boundary are finished through the workspace.
-constexpr int SMEM_LIMIT_M1 = 227 * 1024;
-
-// xf: plan for the M = 1 kernel (padded bf16 x, per-warp stage rings, W1 warps)
 template <int MT>
-static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool xf, int64_t S) {
-    const int W = xf ? W1 : Warps<MT>::value;
-    const size_t limit = xf ? (size_t)SMEM_LIMIT_M1 : (size_t)SMEM_LIMIT;
+static bool make_plan_parts(Plan &p, int64_t M, int64_t N, int64_t K, int g, int64_t S, int want_parts) {
+    using GE_ = Geo<MT>;
     const GemvLayout L = gemv_layout(N, K, g);
     Args &a = p.a;
-    const int64_t T = L.N8 * L.U;
-    if (T >= (1LL << 31)) return false;
-    a.N = N; a.K = K; a.U = (uint32_t)L.U; a.T = (uint32_t)T;
-    a.divU = make_fastdiv(a.U);
-    a.M = (int)M; a.g = g;
-    a.sub = (uint32_t)(8 * (128 / g) * 4);
-    a.off_sx = 64;
-    a.off_slot = a.off_sx + (uint32_t)(MT * L.U * 4 * 4);
-    a.off_xf = a.off_ring = a.off_bars = 0;
-    if (xf) {
-        a.off_xf = a.off_slot;
-        a.off_ring = a.off_xf + xb_bytes((uint32_t)L.U);
-        a.off_bars = a.off_ring + ring_bytes(a.sub);
-        a.off_slot = a.off_bars + W1 * NS * 8;
-    }
-    a.pdl = 0;
-    int64_t P;
-    bool aligned;
-    if (L.N8 <= S) {
-        P = L.N8;
-        aligned = true;
+    a = Args{};
+    a.N = N; a.K = K; a.M = (int)M; a.J = (int)(K / g); a.g = g;
+    a.RS = (uint32_t)L.row_bytes;
+    a.tpr = (int)((K + GE_::KC - 1) / GE_::KC);
+    // K parts: whole rows when the slices fit the consumer threads, else parts of a multiple
+    // of 512 k (so that every part's scales start on a 16-byte boundary)
+    const int unit = 512 / GE_::KC;
+    if (want_parts == 1) {
+        if (a.tpr > NCT) return false;
+        a.kparts = 1;
+        a.spp = a.tpr;
     } else {
-        // whole octets when the busiest CTA's extra units cost less than the cross-CTA
-        // fixup of an even split (measured at about 3 us, the time of ~160 units at M = 1
-        // and proportionally fewer for more rows), or when they are within 8% of the mean
-        const int64_t per = (L.N8 + S - 1) / S;
-        aligned = (double)per <= 1.08 * (double)L.N8 / (double)S ||
-                  (double)(per * L.U) <= (double)T / (double)S + 160.0 / MT;
-        P = aligned ? (L.N8 + per - 1) / per : (S < T ? S : T);
+        a.spp = (a.tpr + want_parts - 1) / want_parts;
+        a.spp = (a.spp + unit - 1) / unit * unit;
+        if (a.spp > NCT) return false;
+        a.kparts = (a.tpr + a.spp - 1) / a.spp;
+        if (a.kparts == 1) return false;
     }
-    while (true) {
-        if (aligned) {
-            a.base = (uint32_t)((L.N8 / P) * L.U);
-            a.rem = (uint32_t)(L.N8 % P);
-            a.step = a.U;
-        } else {
-            a.base = (uint32_t)(T / P);
-            a.rem = (uint32_t)(T % P);
-            a.step = 1;
-        }
-        const int64_t maxr = (int64_t)a.base + (a.rem ? a.step : 0);
-        const int64_t nol = (maxr + L.U - 1) / L.U + 1;
-        const size_t smem = a.off_slot + (size_t)nol * W * 8 * MT * 4;
-        if (smem <= limit) {
-            a.nol = (int)nol;
-            p.P = (int)P;
-            p.smem = (int)smem;
-            p.aligned = aligned;
-            break;
-        }
-        if (P >= T) return false;
-        aligned = false;
-        P = P * 2 < T ? P * 2 : T;
+    if (a.kparts == 1) {
+        a.RSp = a.RS;
+        a.KPB = (uint32_t)(K / 2);
+    } else {
+        a.KPB = (uint32_t)a.spp * (GE_::KC / 2);
+        a.RSp = a.KPB + (uint32_t)(4 * a.spp * GE_::KC / g);
+        a.RSp = (a.RSp + 15) / 16 * 16;
     }
-    a.divB1 = make_fastdiv(a.base + a.step);
-    a.divB = make_fastdiv(a.base);
+    a.nslot = NCT / a.spp;
+    a.rpt = GE_::RPT;
+    const uint32_t planes_bytes = (uint32_t)(a.spp * GE_::PSTRIDE * 4);  // one activation row at a time
+    const uint32_t sx_bytes = (uint32_t)(MT * a.spp * GE_::NCH * 4);
+    const uint32_t pp_bytes = (uint32_t)(MT * a.spp * 4);
+    a.SB = (uint32_t)(a.nslot * a.rpt) * a.RSp;
+    a.warpred = (MT > 1 && a.spp % 32 == 0) ? 1 : 0;
+    a.nred = a.warpred ? a.spp / 32 : a.spp;
+    // rows per block: N spread over the SMs, capped by the row-partial buffer
+    int64_t nrb = S < N ? S : N;
+    int64_t rpc = (N + nrb - 1) / nrb;
+    const int64_t rpc_cap = RED_BUDGET / ((int64_t)MT * a.nred * 4);
+    if (rpc_cap < 1) return false;
+    if (rpc > rpc_cap) rpc = rpc_cap;
+    a.rpc = (int)rpc;
+    a.nrb = (int)((N + rpc - 1) / rpc);
+    a.off_sx = 512;
+    a.off_pp = a.off_sx + (sx_bytes + 15) / 16 * 16;
+    a.off_red = a.off_pp + (pp_bytes + 15) / 16 * 16;
+    a.off_ring = a.off_red + (uint32_t)((rpc * MT * a.nred * 4 + 15) / 16 * 16);
+    const int64_t avail = (int64_t)SMEM_MAX - a.off_ring - SLACK;
+    int NS = (int)(avail / a.SB);
+    if (NS > MAX_STAGES) NS = MAX_STAGES;
+    if ((int64_t)NS * a.SB >= (int64_t)planes_bytes + 2 * (int64_t)a.SB) {
+        // the planes sit at the end of the ring; the stages below them are issued at once
+        const int64_t ring_bytes = (int64_t)NS * a.SB;
+        const int64_t p0 = (ring_bytes - planes_bytes) / 16 * 16;
+        a.off_planes = (uint32_t)(a.off_ring + p0);
+        a.NS_early = (int)(p0 / a.SB);
+        p.smem = (int)(a.off_ring + ring_bytes + SLACK);
+    } else {
+        // too little room for that: the planes follow the ring
+        NS = (int)((avail - planes_bytes) / a.SB);
+        if (NS > MAX_STAGES) NS = MAX_STAGES;
+        if (NS < 2) return false;
+        a.off_planes = (uint32_t)(a.off_ring + (int64_t)NS * a.SB);
+        a.NS_early = NS;
+        p.smem = (int)(a.off_planes + planes_bytes + SLACK);
+    }
+    a.NS = NS;
+    p.MT = MT;
+    p.sweeps = (int)((M + MT - 1) / MT);
+    p.grid_x = a.nrb * a.kparts;
     return true;
 }
 
-// The plan a call of M rows will use: the M = 1 kernel's when it applies and its shared
-// memory (which grows with K) fits, else the general kernel's.
+// Whole rows per block when they fit (threads and shared memory), else the fewest K parts
+// that do.
 template <int MT>
-static bool plan_for(Plan &p, int64_t M, int64_t N, int64_t K, int g, bool &xf, int64_t S = 0) {
-    if (S <= 0) S = sm_count_cached();
-    xf = MT == 1;
-    if (xf && make_plan<MT>(p, M, N, K, g, true, S)) return true;
-    xf = false;
-    return make_plan<MT>(p, M, N, K, g, false, S);
+static bool make_plan_mt(Plan &p, int64_t M, int64_t N, int64_t K, int g, int64_t S) {
+    const int tpr = (int)((K + Geo<MT>::KC - 1) / Geo<MT>::KC);
+    for (int parts = 1; parts <= tpr; ++parts)
+        if (make_plan_parts<MT>(p, M, N, K, g, S, parts)) return true;
+    return false;
 }
 
-// Host-only view of a plan for `sms` SMs: out = {units, octets, blocks, whole octets (0/1),
-// dynamic shared memory bytes per block, M = 1 ring kernel (0/1)}.
-template <int MT>
-static bool describe_plan(int64_t M, int64_t N, int64_t K, int g, int64_t sms, int64_t *out) {
-    Plan p;
-    bool xf;
-    if (!plan_for<MT>(p, M, N, K, g, xf, sms)) return false;
-    const GemvLayout L = gemv_layout(N, K, g);
-    out[0] = (int64_t)p.a.T;
-    out[1] = L.N8;
-    out[2] = p.P;
-    out[3] = p.aligned ? 1 : 0;
-    out[4] = p.smem;
-    out[5] = xf ? 1 : 0;
-    return true;
+// MT = activation rows per sweep: as many as the registers hold for this K (4, 2 or 1),
+// with whole rows per block when possible
+static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, int64_t S) {
+    const int want = M >= 3 ? 4 : (int)M;
+    if (want >= 4 && make_plan_parts<4>(p, M, N, K, g, S, 1)) return true;
+    if (want >= 2 && make_plan_parts<2>(p, M, N, K, g, S, 1)) return true;
+    return make_plan_mt<1>(p, M, N, K, g, S);
 }
 
-template <int MT>
-static size_t ws_need(int64_t N, int64_t K, int g) {
-    Plan p;
-    bool xf;
-    if (!plan_for<MT>(p, MT, N, K, g, xf)) return 0;
-    return (size_t)p.P * 2 * 8 * MT * 4;
+template <int MT, int G>
+static void *kernel_ptr() { return reinterpret_cast<void *>(gemv_kernel<MT, G>); }
+
+static void *pick_kernel(int MT, int g) {
+    if (MT == 4) return g == 32 ? kernel_ptr<4, 32>() : (g == 64 ? kernel_ptr<4, 64>() : kernel_ptr<4, 128>());
+    if (MT == 2) return g == 32 ? kernel_ptr<2, 32>() : (g == 64 ? kernel_ptr<2, 64>() : kernel_ptr<2, 128>());
+    return g == 32 ? kernel_ptr<1, 32>() : (g == 64 ? kernel_ptr<1, 64>() : kernel_ptr<1, 128>());
 }
 
-template <int MT>
+static size_t ws_need(const Plan &p) {
+    if (p.a.kparts == 1) return 0;
+    const size_t part = (size_t)p.a.kparts * p.a.M * p.a.N * 4;
+    return (part + 255) / 256 * 256 + (size_t)p.sweeps * p.a.nrb * 4;
+}
+
 static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, int64_t K, int g, void *y, int out_fp32,
                      void *ws, size_t ws_bytes, int pdl, cudaStream_t stream) {
-    constexpr int W = Warps<MT>::value;
     Plan p;
-    bool xf;
-    if (!plan_for<MT>(p, M, N, K, g, xf)) return W4_ERR_SHAPE;
-    const GemvLayout L = gemv_layout(N, K, g);
-    const size_t need = (size_t)p.P * 2 * 8 * MT * 4 + (size_t)L.N8 * 4;
-    if (!ws || ws_bytes < need) return W4_ERR_WORKSPACE;
+    if (!make_plan(p, M, N, K, g, sm_count_cached())) return W4_ERR_SHAPE;
     Args &a = p.a;
+    const size_t need = ws_need(p);
+    if (need) {
+        if (!ws || ws_bytes < need) return W4_ERR_WORKSPACE;
+        a.ws_part = static_cast<float *>(ws);
+        a.ws_count = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + (need - (size_t)p.sweeps * a.nrb * 4));
+    }
     a.x = static_cast<const uint16_t *>(x);
-    a.codes = static_cast<const uint8_t *>(packed);
-    a.scales = static_cast<const uint8_t *>(packed) + L.codes_bytes;
+    a.w = static_cast<const uint8_t *>(packed);
     a.y = y;
     a.out_fp32 = out_fp32;
-    a.ws_part = static_cast<float *>(ws);
-    a.ws_count = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + (size_t)p.P * 2 * 8 * MT * 4);
     a.status = device_status_ptr();
     a.pdl = pdl;
-    static int attr_done[64] = {0};
+    void *fn = pick_kernel(p.MT, g);
+    static int attr_done[64][3][3] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        if (cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_LIMIT) !=
-            cudaSuccess)
+    const int mi = p.MT == 4 ? 2 : p.MT - 1, gi = g == 32 ? 0 : (g == 64 ? 1 : 2);
+    if (dev >= 0 && dev < 64 && !attr_done[dev][mi][gi]) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_MAX) != cudaSuccess)
             return W4_ERR_CUDA;
-        if (MT == 1 && cudaFuncSetAttribute(gemv1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            SMEM_LIMIT_M1) != cudaSuccess)
-            return W4_ERR_CUDA;
-        attr_done[dev] = 1;
+        attr_done[dev][mi][gi] = 1;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.P);
-    cfg.blockDim = dim3(xf ? W1 * 32 : W * 32);
+    cfg.gridDim = dim3((unsigned)p.grid_x, (unsigned)p.sweeps);
+    cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = (size_t)p.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -647,18 +670,39 @@ static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, in
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = xf ? cudaLaunchKernelEx(&cfg, gemv1_kernel, a) : cudaLaunchKernelEx(&cfg, gemv_kernel<MT>, a);
-    if (e != cudaSuccess) return W4_ERR_CUDA;
+    void *args[] = {&a};
+    if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return W4_ERR_CUDA;
     return launch_status();
 }
 
+// Host-only view of a plan: out = {activation rows per sweep, sweeps, K parts, row blocks,
+// rows per block, dynamic shared memory bytes, ring stages, workspace bytes}.
+static bool describe_plan(int64_t M, int64_t N, int64_t K, int g, int64_t sms, int64_t *out) {
+    Plan p;
+    if (!make_plan(p, M, N, K, g, sms)) return false;
+    out[0] = p.MT;
+    out[1] = p.sweeps;
+    out[2] = p.a.kparts;
+    out[3] = p.a.nrb;
+    out[4] = p.a.rpc;
+    out[5] = p.smem;
+    out[6] = p.a.NS;
+    out[7] = (int64_t)ws_need(p);
+    return true;
+}
+
+// The workspace a call may need: the largest over M = 1..16 on this device's SM count.
 size_t workspace_bytes(int64_t N, int64_t K, int g) {
-    const GemvLayout L = gemv_layout(N, K, g);
     size_t worst = 0;
-    const size_t cand[5] = {ws_need<1>(N, K, g), ws_need<2>(N, K, g), ws_need<4>(N, K, g), ws_need<8>(N, K, g),
-                            ws_need<16>(N, K, g)};
-    for (size_t v : cand) worst = v > worst ? v : worst;
-    return (worst + (size_t)L.N8 * 4 + 255) / 256 * 256;
+    const int64_t S = sm_count_cached();
+    for (int64_t M = 1; M <= 16; ++M) {
+        Plan p;
+        if (make_plan(p, M, N, K, g, S)) {
+            const size_t v = ws_need(p);
+            worst = v > worst ? v : worst;
+        }
+    }
+    return worst;
 }
 
 }  // namespace gemv
@@ -666,23 +710,20 @@ size_t workspace_bytes(int64_t N, int64_t K, int g) {
 
 using namespace w4;
 
+static bool gemv_shape_ok(int64_t M, int64_t N, int64_t K) {
+    return M >= 1 && M <= 16 && N >= 1 && N <= ((int64_t)1 << 31) && K >= 32 && K % 32 == 0 && K <= ((int64_t)1 << 24);
+}
+
 W4_API size_t w4a16_gemv_workspace_bytes(int64_t N, int64_t K, int group) {
-    if (N < 1 || K < 32 || K % 32 != 0 || !valid_group(group) || K % group != 0) return 0;
+    if (!gemv_shape_ok(1, N, K) || !valid_group(group) || K % group != 0) return 0;
     return gemv::workspace_bytes(N, K, group);
 }
 
 W4_API w4_status w4a16_gemv_schedule(int64_t M, int64_t N, int64_t K, int group, int sms, int64_t *out) {
     if (!out) return W4_ERR_NULL;
-    if (M < 1 || M > 16 || N < 1 || N > (int64_t)0x7fffffff * 8 || K < 32 || K % 32 != 0 || sms < 1 || sms > 4096)
-        return W4_ERR_SHAPE;
+    if (!gemv_shape_ok(M, N, K) || sms < 1 || sms > 4096) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
-    bool ok;
-    if (M <= 1) ok = gemv::describe_plan<1>(M, N, K, group, sms, out);
-    else if (M <= 2) ok = gemv::describe_plan<2>(M, N, K, group, sms, out);
-    else if (M <= 4) ok = gemv::describe_plan<4>(M, N, K, group, sms, out);
-    else if (M <= 8) ok = gemv::describe_plan<8>(M, N, K, group, sms, out);
-    else ok = gemv::describe_plan<16>(M, N, K, group, sms, out);
-    return ok ? W4_OK : W4_ERR_SHAPE;
+    return gemv::describe_plan(M, N, K, group, sms, out) ? W4_OK : W4_ERR_SHAPE;
 }
 
 W4_API w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K, int group,
@@ -692,15 +733,11 @@ W4_API w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, i
     if (!valid_mode(mode) || (flags & ~(W4_OUT_FP32 | W4_OVERLAP_PREVIOUS))) return W4_ERR_ARG;
     const int out_fp32 = (flags & W4_OUT_FP32) ? 1 : 0;
     const int pdl = (flags & W4_OVERLAP_PREVIOUS) ? 1 : 0;
-    if (M < 1 || M > 16 || N < 1 || N > (int64_t)0x7fffffff * 8 || K < 32 || K % 32 != 0) return W4_ERR_SHAPE;
+    if (!gemv_shape_ok(M, N, K)) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
     if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(y) || (workspace && !aligned16(workspace)))
         return W4_ERR_ALIGN;
-    if (M <= 1) return gemv::run<1>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
-    if (M <= 2) return gemv::run<2>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
-    if (M <= 4) return gemv::run<4>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
-    if (M <= 8) return gemv::run<8>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
-    return gemv::run<16>(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
+    return gemv::run(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
 }
 
 // ------------------------------------------------------------------ allocation-free variant
@@ -708,9 +745,9 @@ W4_API w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, i
 // Callers that must not allocate device memory on the hot path -- a plug-in running inside
 // another runtime that owns all device memory, or a latency-critical decode loop where
 // cudaMalloc's implicit device synchronisation is not acceptable -- can call
-// w4a16_gemv_noalloc. Its scratch (the partial sums and arrival counters of the stream-K
-// fixup) is a fixed array in this library's device memory, reserved when the library loads
-// on a GPU and held until the process exits.
+// w4a16_gemv_noalloc. Its scratch (the partial sums and arrival counters of rows split along
+// K over several blocks) is a fixed array in this library's device memory, reserved when the
+// library loads on a GPU and held until the process exits.
 
 namespace w4 {
 namespace gemv {
@@ -736,22 +773,22 @@ static void *noalloc_scratch() {
     return g_noalloc_ptr[dev];
 }
 
-template <int MT>
 static w4_status run_noalloc(const void *x, int64_t M, const void *packed, int64_t N, int64_t K, int g, void *y,
                              int out_fp32, int pdl, cudaStream_t stream) {
     Plan p;
-    bool xf;
-    if (!plan_for<MT>(p, M, N, K, g, xf)) return W4_ERR_SHAPE;
-    const GemvLayout L = gemv_layout(N, K, g);
-    const size_t part = (size_t)p.P * 2 * 8 * MT * 4;
-    const size_t need = part + (size_t)L.N8 * 4;
+    if (!make_plan(p, M, N, K, g, sm_count_cached())) return W4_ERR_SHAPE;
+    const size_t need = ws_need(p);
     if (need > kNoAllocScratchBytes) return W4_ERR_SCRATCH_LIMIT;
-    uint8_t *ws = static_cast<uint8_t *>(noalloc_scratch());
-    if (!ws) return W4_ERR_CUDA;
-    // the arrival counters must start at zero; a call normally leaves them at zero, but the
-    // array outlives every call, so clear them on the caller's stream first
-    if (cudaMemsetAsync(ws + part, 0, (size_t)L.N8 * 4, stream) != cudaSuccess) return W4_ERR_CUDA;
-    return run<MT>(x, M, packed, N, K, g, y, out_fp32, ws, kNoAllocScratchBytes, pdl, stream);
+    uint8_t *ws = nullptr;
+    if (need) {
+        ws = static_cast<uint8_t *>(noalloc_scratch());
+        if (!ws) return W4_ERR_CUDA;
+        // the arrival counters must start at zero; a call normally leaves them at zero, but
+        // the array outlives every call, so clear them on the caller's stream first
+        const size_t cnt = (size_t)p.sweeps * p.a.nrb * 4;
+        if (cudaMemsetAsync(ws + need - cnt, 0, cnt, stream) != cudaSuccess) return W4_ERR_CUDA;
+    }
+    return run(x, M, packed, N, K, g, y, out_fp32, ws, kNoAllocScratchBytes, pdl, stream);
 }
 
 }  // namespace gemv
@@ -763,14 +800,10 @@ W4_API w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *p
                                     int group, int mode, void *y, int flags, cudaStream_t stream) {
     if (!x_bf16 || !packed || !y) return W4_ERR_NULL;
     if (!valid_mode(mode) || (flags & ~(W4_OUT_FP32 | W4_OVERLAP_PREVIOUS))) return W4_ERR_ARG;
-    if (M < 1 || M > 16 || N < 1 || N > (int64_t)0x7fffffff * 8 || K < 32 || K % 32 != 0) return W4_ERR_SHAPE;
+    if (!gemv_shape_ok(M, N, K)) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
     if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(y)) return W4_ERR_ALIGN;
     const int out_fp32 = (flags & W4_OUT_FP32) ? 1 : 0;
     const int pdl = (flags & W4_OVERLAP_PREVIOUS) ? 1 : 0;
-    if (M <= 1) return gemv::run_noalloc<1>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
-    if (M <= 2) return gemv::run_noalloc<2>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
-    if (M <= 4) return gemv::run_noalloc<4>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
-    if (M <= 8) return gemv::run_noalloc<8>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
-    return gemv::run_noalloc<16>(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
+    return gemv::run_noalloc(x_bf16, M, packed, N, K, group, y, out_fp32, pdl, stream);
 }

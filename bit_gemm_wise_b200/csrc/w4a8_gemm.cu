@@ -773,6 +773,373 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
     }
 }
 
+// ------------------------------------------------------------------ split-weight FP16 path
+//
+// With groups of 32 every FP8 MMA (K = 32) ends a group, and the exact per-group promotion
+// (a TMEM readback and 128 x 256 fp32 FMAs on the CUDA cores per MMA) costs several times
+// the MMA itself. For such groups this kernel keeps the whole K in one TMEM accumulator
+// instead: every weight is dequantized exactly and split into two fp16 parts,
+//   w = (q - z) s,  hi = fp16(w),  lo = fp16(w - hi),  w = hi + lo,
+// and the E4M3 activations become fp16 (exact: every E4M3 value is an fp16 value). kind::f16
+// MMAs accumulate A_hi B + A_lo B in fp32, so the tensor core sees the dequantized operands
+// of the method, as in the promoted path, and nothing is read back until the tile is done.
+// Exactness: q - z is an fp16 integer (1024 + q minus 1024 + z) for |z| < 1024, s is the
+// stored fp16 scale, so w has at most 11 + 11 significant bits; hi keeps the leading 11 and
+// the fp16 FMA forms lo = w - hi exactly (it is a multiple of 2^-24, the smallest fp16
+// subnormal, so it never underflows). A group with |z| >= 1024 forms q - z in fp32 and
+// rounds it to fp16, and one with |(q - z) s| >= 65504 overflows fp16; the first is exact
+// while |q - z| <= 2048, and both lie far outside any trained weight's range. The cost is
+// two fp16 MMAs per K step, a quarter of the FP8 rate, with no per-group readback.
+//
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-7
+// epilogue (one TMEM lane quarter each, all 256 columns), warps 8-15 expansion. Two rings:
+// raw stages (packed codes + E4M3 activations, by TMA) and expanded stages (fp16 A_hi, A_lo
+// and B in the 128-byte-swizzled K-major layout the MMA reads). Two TMEM accumulators
+// alternate between tiles, so the epilogue of one tile overlaps the MMAs of the next.
+namespace f16p {
+
+constexpr int BK = 64;                        // k per stage (one 128-byte swizzle row of fp16)
+constexpr int RAW_STAGES = 4;
+constexpr int EXP_STAGES = 2;
+constexpr int EXW = 8;                        // expansion warps
+constexpr uint32_t RC_BYTES = BM * BK / 2;    // packed codes of a stage (4 KB)
+constexpr uint32_t RA_BYTES = BN * BK;        // E4M3 activations of a stage (16 KB)
+constexpr uint32_t RAW_BYTES = RC_BYTES + RA_BYTES;
+constexpr uint32_t AH_BYTES = BM * BK * 2;    // one fp16 weight part (16 KB)
+constexpr uint32_t B_BYTES = BN * BK * 2;     // fp16 activations (32 KB)
+constexpr uint32_t EXP_BYTES = 2 * AH_BYTES + B_BYTES;
+constexpr uint32_t SMEM_BYTES = RAW_STAGES * RAW_BYTES + EXP_STAGES * EXP_BYTES + 1024 + 1024;
+static_assert(RAW_BYTES % 1024 == 0 && EXP_BYTES % 1024 == 0 && AH_BYTES % 1024 == 0, "swizzle atoms stay aligned");
+
+struct Smem {
+    uint64_t raw_full[RAW_STAGES];   // TMA bytes landed
+    uint64_t raw_empty[RAW_STAGES];  // expansion read the stage (one arrival per expansion warp)
+    uint64_t exp_full[EXP_STAGES];   // expansion wrote the operands (one arrival per expansion warp)
+    uint64_t exp_empty[EXP_STAGES];  // the MMAs reading them completed (tcgen05.commit)
+    uint64_t acc_full[NBUF];         // a tile's accumulator is complete
+    uint64_t acc_empty[NBUF];        // the epilogue has read it (one arrival per epilogue warp)
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(Smem) <= 1024, "control block");
+
+// instruction descriptor: D fp32, A and B fp16, both K-major, N = BN, M = BM
+constexpr uint32_t kIdescF16 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint32_t a_lo, uint32_t b_lo, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n .reg .b64 da, db;\n setp.ne.b32 p, %4, 0;\n"
+        " mov.b64 da, {%1, %5};\n mov.b64 db, {%2, %5};\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n}\n" ::"r"(tmem_d),
+        "r"(a_lo), "r"(b_lo), "r"(kIdescF16), "r"(accumulate), "r"(kDescHiSW128));
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cast<__half2 *>(&v); }
+
+// two E4M3 bytes (low 16 bits of v) -> fp16x2, exact
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
+    uint32_t r;
+    asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n" : "=r"(r) : "r"(v));
+    return r;
+}
+
+__device__ __forceinline__ bool wait_f(uint64_t *bar, uint32_t parity, Smem *sm, int *status) {
+    return mbar_wait_abortable<true>(bar, parity, &sm->abort, status, kWaitNs);
+}
+__device__ __forceinline__ bool warp_wait_f(uint64_t *bar, uint32_t parity, Smem *sm, int *status) {
+    bool r = true;
+    if ((threadIdx.x & 31) == 0) r = mbar_wait_abortable(bar, parity, &sm->abort, status, kWaitNs);
+    r = __shfl_sync(FULL, r ? 1 : 0, 0) != 0;
+    if (r) r = __all_sync(FULL, mbar_try_wait_short(bar, parity));
+    return r;
+}
+
+// position in a ring of N slots
+template <int N> struct RingN {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next() {
+        if (++slot == N) { slot = 0; phase ^= 1u; }
+    }
+};
+
+__global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_constant__ CUtensorMap tm_codes,
+                                                                   const __grid_constant__ CUtensorMap tm_act,
+                                                                   const Args a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *raw = base;                                     // RAW_STAGES x (codes | E4M3 activations)
+    uint8_t *ex = base + RAW_STAGES * RAW_BYTES;             // EXP_STAGES x (A_hi | A_lo | B)
+    Smem *sm = reinterpret_cast<Smem *>(ex + EXP_STAGES * EXP_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KT = (int)(a.Kpad / BK);
+    const int64_t ntiles = (int64_t)a.MTU * a.NT;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < RAW_STAGES; ++s) {
+            mbar_init(&sm->raw_full[s], 1);
+            mbar_init(&sm->raw_empty[s], EXW);
+        }
+        for (int s = 0; s < EXP_STAGES; ++s) {
+            mbar_init(&sm->exp_full[s], EXW);
+            mbar_init(&sm->exp_empty[s], 1);
+        }
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&sm->acc_full[b], 1);
+            mbar_init(&sm->acc_empty[b], 4);
+        }
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sm->tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            RingN<RAW_STAGES> r;
+            int64_t uses = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                Tile T;
+                if (!locate_tile(a, t, T)) continue;
+                for (int s = 0; s < KT; ++s, r.next(), ++uses) {
+                    if (!wait_f(&sm->raw_empty[r.slot], r.phase ^ 1u, sm, a.status)) { ok = false; break; }
+                    uint8_t *dst = raw + r.slot * RAW_BYTES;
+                    mbar_arrive_expect_tx(&sm->raw_full[r.slot], RAW_BYTES);
+                    tma_load_3d(dst, &tm_codes, s * (BK / 2), (int)T.n0, T.e, &sm->raw_full[r.slot]);
+                    tma_load_2d(dst + RC_BYTES, &tm_act, s * BK, (int)T.row0, &sm->raw_full[r.slot]);
+                }
+            }
+            // no copy may land after the CTA exits: wait for the last uses' bytes
+            for (int64_t u = uses > RAW_STAGES ? uses - RAW_STAGES : 0; u < uses; ++u)
+                (void)mbar_wait_bounded(&sm->raw_full[u % RAW_STAGES], (uint32_t)(u / RAW_STAGES) & 1, a.status);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            RingN<EXP_STAGES> r;
+            uint32_t tiles_done = 0;
+            int64_t uses = 0;
+            bool ok = true;
+            const uint32_t exLo0 = desc_lo(smem_addr(ex));
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                Tile T;
+                if (!locate_tile(a, t, T)) continue;
+                const uint32_t b = tiles_done & 1u;
+                if (!wait_f(&sm->acc_empty[b], ((tiles_done >> 1) & 1u) ^ 1u, sm, a.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + b * BN;
+                for (int s = 0; s < KT; ++s, r.next()) {
+                    if (!wait_f(&sm->exp_full[r.slot], r.phase, sm, a.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t hLo = exLo0 + (uint32_t)r.slot * (EXP_BYTES >> 4);
+                    const uint32_t lLo = hLo + (AH_BYTES >> 4), bLo = hLo + (2 * AH_BYTES >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {  // K = 16 per fp16 MMA: 32 bytes
+                        mma_f16(d, hLo + kk * 2, bLo + kk * 2, (s > 0 || kk > 0) ? 1u : 0u);
+                        mma_f16(d, lLo + kk * 2, bLo + kk * 2, 1u);
+                    }
+                    mma_commit(&sm->exp_empty[r.slot]);
+                    ++uses;
+                }
+                if (!ok) break;
+                mma_commit(&sm->acc_full[b]);
+                ++tiles_done;
+            }
+            // no commit may arrive after the CTA exits: wait for the last stages' completions
+            for (int64_t u = uses > EXP_STAGES ? uses - EXP_STAGES : 0; u < uses; ++u)
+                (void)mbar_wait_bounded(&sm->exp_empty[u % EXP_STAGES], (uint32_t)(u / EXP_STAGES) & 1, a.status);
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------ epilogue (4 warps)
+        const int quarter = warp & 3;  // TMEM lanes (weight rows) 32*quarter ...
+        uint32_t tiles_done = 0;
+        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            Tile T;
+            if (!locate_tile(a, t, T)) continue;
+            const uint32_t b = tiles_done & 1u;
+            if (!warp_wait_f(&sm->acc_full[b], (tiles_done >> 1) & 1u, sm, a.status)) break;
+            tc_fence_after();
+            const uint32_t tl_addr = tmem + ((uint32_t)(quarter * 32) << 16) + b * BN;
+            const int64_t n = T.n0 + quarter * 32 + lane;
+            const bool row_ok = n < a.N;
+            const int64_t lim = (T.rows < (int64_t)BN ? T.rows : (int64_t)BN);
+            const int64_t lim_m = a.M - T.row0;
+            const int64_t ncol = lim < lim_m ? lim : lim_m;  // valid token columns of the tile
+            const bool vec = !a.out_fp32 && (a.N & 7) == 0;
+            const int64_t nbase = T.n0 + quarter * 32 + 8 * (lane >> 3);
+            const int li = lane & 7;
+#pragma unroll 1
+            for (int c = 0; c < BN / 16; ++c) {
+                uint32_t v[16];
+                tmem_ld16(tl_addr + c * 16, v);
+                // token scale of column 16c + (lane & 15)
+                const int colr = c * 16 + (lane & 15);
+                const float rsc = colr < ncol ? __ldg(a.row_scale + T.row0 + colr) : 0.0f;
+                tmem_wait_ld16(v);
+                const int64_t m0 = T.row0 + c * 16;
+                if (vec) {
+                    uint32_t h0[4], h1[4];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float r0 = __shfl_sync(FULL, rsc, 2 * q), r1 = __shfl_sync(FULL, rsc, 2 * q + 1);
+                        const __nv_bfloat162 b2 =
+                            __floats2bfloat162_rn(__uint_as_float(v[2 * q]) * r0, __uint_as_float(v[2 * q + 1]) * r1);
+                        const uint32_t w = *reinterpret_cast<const uint32_t *>(&b2);
+                        if (q < 4) h0[q] = w;
+                        else h1[q - 4] = w;
+                    }
+                    transpose8x8_b16(h0, lane);
+                    transpose8x8_b16(h1, lane);
+                    if (nbase < a.N) {
+                        __nv_bfloat16 *yb = static_cast<__nv_bfloat16 *>(a.Y);
+                        if (c * 16 + li < ncol)
+                            *reinterpret_cast<uint4 *>(yb + (m0 + li) * a.N + nbase) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+                        if (c * 16 + 8 + li < ncol)
+                            *reinterpret_cast<uint4 *>(yb + (m0 + 8 + li) * a.N + nbase) =
+                                make_uint4(h1[0], h1[1], h1[2], h1[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float rs = __shfl_sync(FULL, rsc, k);
+                        if (row_ok && c * 16 + k < ncol) {
+                            const float val = __uint_as_float(v[k]) * rs;
+                            if (a.out_fp32) static_cast<float *>(a.Y)[(m0 + k) * a.N + n] = val;
+                            else static_cast<__nv_bfloat16 *>(a.Y)[(m0 + k) * a.N + n] = __float2bfloat16_rn(val);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->acc_empty[b]);
+            ++tiles_done;
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------ expansion (8 warps, 256 threads)
+        const int et = threadIdx.x - 256;        // 0..255
+        const int wr = et >> 1, wh = et & 1;      // weight row, half of the stage's 64 k
+        RingN<RAW_STAGES> rr;
+        RingN<EXP_STAGES> re;
+        bool ok = true;
+        const __half2 h1024 = __float2half2_rn(1024.0f);
+        const uint32_t magic = 0x64646464u;      // high bytes of fp16 1024 + q
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            Tile T;
+            if (!locate_tile(a, t, T)) continue;
+            const int64_t n = T.n0 + wr;
+            const uint32_t *scales =
+                reinterpret_cast<const uint32_t *>(a.packed + (size_t)T.e * a.slab_bytes + a.codes_bytes);
+            // this thread's scale entry for stage s is loaded one stage ahead (it does not
+            // depend on the ring): k = 64 s + 32 wh + 0..31 lies in group (64 s + 32 wh) / g
+            uint32_t ent_next = scales[(int64_t)(wh * 32 / a.g) * a.Npad + n];
+            for (int s = 0; s < KT; ++s, rr.next(), re.next()) {
+                const uint32_t ent = ent_next;
+                if (s + 1 < KT) ent_next = scales[((int64_t)(s + 1) * BK + wh * 32) / a.g * a.Npad + n];
+                if (!warp_wait_f(&sm->raw_full[rr.slot], rr.phase, sm, a.status)) { ok = false; break; }
+                if (!warp_wait_f(&sm->exp_empty[re.slot], re.phase ^ 1u, sm, a.status)) { ok = false; break; }
+                const uint8_t *src = raw + rr.slot * RAW_BYTES;
+                uint8_t *dst = ex + re.slot * EXP_BYTES;
+                {
+                    const int z = (int)(int16_t)(ent >> 16);
+                    const __half2 s2 = __half2half2(__ushort_as_half((unsigned short)(ent & 0xFFFFu)));
+                    const uint4 cw = *reinterpret_cast<const uint4 *>(src + wr * 32 + wh * 16);
+                    const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
+                    uint32_t hi[16], lo[16];
+                    if (z > -1024 && z < 1024) {
+                        const __half2 c0 = __hadd2(h1024, __float2half2_rn((float)z));
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint32_t bl = wv[i] & 0x0F0F0F0Fu, bh = (wv[i] >> 4) & 0x0F0F0F0Fu;
+                            const uint32_t p[4] = {__byte_perm(bl, magic, 0x4140), __byte_perm(bl, magic, 0x4342),
+                                                   __byte_perm(bh, magic, 0x4140), __byte_perm(bh, magic, 0x4342)};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __half2 cc = __hsub2(bits_h2(p[e]), c0);
+                                const __half2 h = __hmul2(cc, s2);
+                                hi[4 * i + e] = h2_bits(h);
+                                lo[4 * i + e] = h2_bits(__hfma2(cc, s2, __hneg2(h)));
+                            }
+                        }
+                    } else {
+                        // zero point beyond fp16's exact integers around 1024: q - z in fp32
+                        const float sf = __half2float(__ushort_as_half((unsigned short)(ent & 0xFFFFu)));
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                // nibble slots: k0 + p/2 + 4 (p % 2) holds slot p
+                                const int k0 = 2 * e;  // weights k0 and k0 + 1 of this word
+                                const int p0 = (k0 & 3) * 2 + (k0 >> 2), p1 = ((k0 + 1) & 3) * 2 + ((k0 + 1) >> 2);
+                                const float q0 = (float)((wv[i] >> (4 * p0)) & 0xFu), q1 = (float)((wv[i] >> (4 * p1)) & 0xFu);
+                                const __half2 cc = __floats2half2_rn(q0 - (float)z, q1 - (float)z);
+                                const __half2 h = __hmul2(cc, __float2half2_rn(sf));
+                                hi[4 * i + e] = h2_bits(h);
+                                lo[4 * i + e] = h2_bits(__hfma2(cc, __float2half2_rn(sf), __hneg2(h)));
+                            }
+                        }
+                    }
+                    // 16-byte chunks 4 wh .. 4 wh + 3 of row wr (8 k each), 128-byte swizzle
+                    uint8_t *ah = dst + wr * 128, *al = dst + AH_BYTES + wr * 128;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int pc = (4 * wh + c) ^ (wr & 7);
+                        *reinterpret_cast<uint4 *>(ah + pc * 16) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                        *reinterpret_cast<uint4 *>(al + pc * 16) = make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+                    }
+                }
+                // activations: token row et, 64 E4M3 bytes (64-byte swizzle: 16-byte chunk c of
+                // row r at r*64 + 16*(c ^ ((r >> 1) & 3))) -> 64 fp16 (128-byte swizzle)
+                {
+                    const uint8_t *ar = src + RC_BYTES + et * 64;
+                    uint8_t *br = dst + 2 * AH_BYTES + et * 128;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(ar + 16 * (c ^ ((et >> 1) & 3)));
+                        const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+                        uint32_t o[8];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            o[2 * i] = e4m3x2_to_f16x2(vv[i]);
+                            o[2 * i + 1] = e4m3x2_to_f16x2(vv[i] >> 16);
+                        }
+                        *reinterpret_cast<uint4 *>(br + ((2 * c) ^ (et & 7)) * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4 *>(br + ((2 * c + 1) ^ (et & 7)) * 16) = make_uint4(o[4], o[5], o[6], o[7]);
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&sm->raw_empty[rr.slot]);
+                    mbar_arrive(&sm->exp_full[re.slot]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+}  // namespace f16p
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -864,9 +1231,69 @@ static int64_t dense_tiles(int64_t M, int64_t N, int64_t K, int group) {
     return ((M + BN - 1) / BN) * (L.Npad / BM);
 }
 
+// Groups of 32: the split-weight fp16 kernel (no per-group promotion, no zero-point operand).
+static w4_status launch_f16(const uint8_t *X8, const float *row_scale, const int32_t *offsets, int E, int64_t M,
+                            const void *packed, int64_t N, int64_t K, int group, void *Y, int out_fp32,
+                            cudaStream_t stream) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return W4_ERR_CUDA;
+    const GemmLayout L = gemm_layout(N, K, group);
+    const uint8_t *pk = static_cast<const uint8_t *>(packed);
+    CUtensorMap tm_codes, tm_act;
+    {
+        const cuuint64_t dims[3] = {(cuuint64_t)(L.Kpad / 2), (cuuint64_t)L.Npad, (cuuint64_t)E};
+        const cuuint64_t strides[2] = {(cuuint64_t)(L.Kpad / 2), (cuuint64_t)L.total};
+        const cuuint32_t box[3] = {f16p::BK / 2, BM, 1};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(pk), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K};
+        const cuuint32_t box[2] = {f16p::BK, BN};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&tm_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(X8), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+    }
+    Args a{};
+    a.packed = pk;
+    a.slab_bytes = L.total;
+    a.codes_bytes = L.codes_bytes;
+    a.row_scale = row_scale;
+    a.offsets = offsets;
+    a.Y = Y;
+    a.status = device_status_ptr();
+    a.M = M; a.N = N; a.Npad = L.Npad; a.K = K; a.Kpad = L.Kpad;
+    a.E = E; a.g = group; a.out_fp32 = out_fp32;
+    a.NT = (int)(L.Npad / BM);
+    const int64_t mtu = offsets ? (M + BN - 1) / BN + E : (M + BN - 1) / BN;
+    if (mtu > 0x7fffffffLL || mtu * a.NT > 0x7fffffffLL) return W4_ERR_SHAPE;
+    a.MTU = (int)mtu;
+    const int64_t tiles = mtu * a.NT;
+    const int sms = sm_count_cached();
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        if (cudaFuncSetAttribute(f16p::w4a8_f16split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)f16p::SMEM_BYTES) !=
+            cudaSuccess)
+            return W4_ERR_CUDA;
+        attr_done[dev] = 1;
+    }
+    f16p::w4a8_f16split_kernel<<<grid, THREADS, f16p::SMEM_BYTES, stream>>>(tm_codes, tm_act, a);
+    return launch_status();
+}
+
 static w4_status launch(const uint8_t *X8, const float *row_scale, const uint16_t *gop, const int32_t *offsets, int E,
                         int64_t M, const void *packed, int64_t N, int64_t K, int group, void *Y, int out_fp32,
                         void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (group == 32) return launch_f16(X8, row_scale, offsets, E, M, packed, N, K, group, Y, out_fp32, stream);
     EncodeTiledFn enc = encode_fn();
     if (!enc) return W4_ERR_CUDA;
     const GemmLayout L = gemm_layout(N, K, group);
@@ -959,7 +1386,8 @@ W4_API size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int gro
     if (!gemm_shape_ok(M, N, K) || !valid_group(group) || K % group != 0) return 0;
     const int sms = gemm::sm_count_cached();
     if (sms < 1) return 0;
-    return gemm::make_plan(gemm::dense_tiles(M, N, K, group), gemm_layout(N, K, group).Kpad / gemm::BK, sms, true)
+    return gemm::make_plan(gemm::dense_tiles(M, N, K, group), gemm_layout(N, K, group).Kpad / gemm::BK, sms,
+                           group != 32)
         .ws_bytes;
 }
 
@@ -968,7 +1396,7 @@ W4_API w4_status w4a8_gemm_schedule(int64_t M, int64_t N, int64_t K, int group, 
     if (!gemm_shape_ok(M, N, K) || sms < 1 || sms > 4096) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
     const int64_t KT = gemm_layout(N, K, group).Kpad / gemm::BK;
-    const gemm::Plan p = gemm::make_plan(gemm::dense_tiles(M, N, K, group), KT, sms, true);
+    const gemm::Plan p = gemm::make_plan(gemm::dense_tiles(M, N, K, group), KT, sms, group != 32);
     out[0] = p.tiles;
     out[1] = p.dpt;
     out[2] = p.r;
@@ -1009,7 +1437,7 @@ W4_API w4_status w4a8_gemm_split_segment(int64_t R, int64_t KT, int64_t PS, int6
 W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op, int64_t M,
                            const void *packed, int64_t N, int64_t K, int group, int mode, void *Y, int out_fp32,
                            void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    if (!X_e4m3 || !row_scale || !gsum_op || !packed || !Y) return W4_ERR_NULL;
+    if (!X_e4m3 || !row_scale || !packed || !Y || (!gsum_op && group != 32)) return W4_ERR_NULL;
     if (!valid_mode(mode) || (out_fp32 != 0 && out_fp32 != 1)) return W4_ERR_ARG;
     if (!gemm_shape_ok(M, N, K)) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
@@ -1023,7 +1451,8 @@ W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const 
 W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op,
                                    const int32_t *expert_row_offsets, int E, int64_t M_total, const void *packed,
                                    int64_t N, int64_t K, int group, int mode, void *Y, cudaStream_t stream) {
-    if (!X_e4m3 || !row_scale || !gsum_op || !expert_row_offsets || !packed || !Y) return W4_ERR_NULL;
+    if (!X_e4m3 || !row_scale || !expert_row_offsets || !packed || !Y || (!gsum_op && group != 32))
+        return W4_ERR_NULL;
     if (!valid_mode(mode)) return W4_ERR_ARG;
     if (E < 1 || E > 1024 || M_total < 1 || M_total > 0x7fffffffLL || N < 1 || N > 0x7fffffffLL || K < 128 ||
         K % 32 != 0 || K > (1LL << 24))

@@ -37,6 +37,10 @@ SIGNATURES = [
     ("w4_prepack", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P]),
     ("w4a8_gsum_op_cols", _I64, [_I64, _I]),
     ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]),
+    ("fp8_row_quant_gather", _I, [_P, _I64, _I64, _I, _P, _I64, _P, _P, _P, _P, _P]),
+    ("w4_moe_route", _I, [_P, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
+    ("w4_moe_swiglu_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P]),
+    ("w4_moe_combine", _I, [_P, _I64, _I64, _P, _P, _I64, _I, _P, _P]),
     ("w4a16_gemv_workspace_bytes", _SZ, [_I64, _I64, _I]),
     ("w4a16_gemv_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
@@ -143,15 +147,40 @@ def fp8_row_quant(X, M, K, group, X8, row_scale, group_sums=None, gsum_op=None, 
     _check("fp8_row_quant", rc)
 
 
+def fp8_row_quant_gather(X, M_src, K, group, row_index, M, X8, row_scale, group_sums=None, gsum_op=None,
+                         stream=None):
+    rc = lib().fp8_row_quant_gather(_ptr(X), M_src, K, group, _ptr(row_index), M, _ptr(X8), _ptr(row_scale),
+                                    _ptr(group_sums), _ptr(gsum_op), _stream(stream))
+    _check("fp8_row_quant_gather", rc)
+
+
+def w4_moe_route(logits, T, E, k, experts, gates, expert_row_offsets, token_of_row, row_of, stream=None):
+    rc = lib().w4_moe_route(_ptr(logits), T, E, k, _ptr(experts), _ptr(gates), _ptr(expert_row_offsets),
+                            _ptr(token_of_row), _ptr(row_of), _stream(stream))
+    _check("w4_moe_route", rc)
+
+
+def w4_moe_swiglu_quant(gate_up, R, H, group, X8, row_scale, gsum_op=None, stream=None):
+    rc = lib().w4_moe_swiglu_quant(_ptr(gate_up), R, H, group, _ptr(X8), _ptr(row_scale), _ptr(gsum_op),
+                                   _stream(stream))
+    _check("w4_moe_swiglu_quant", rc)
+
+
+def w4_moe_combine(rows, N, R, row_of, gates, T, k, y, stream=None):
+    rc = lib().w4_moe_combine(_ptr(rows), N, R, _ptr(row_of), _ptr(gates), T, k, _ptr(y), _stream(stream))
+    _check("w4_moe_combine", rc)
+
+
 def w4a16_gemv_workspace_bytes(N, K, group) -> int:
     return int(lib().w4a16_gemv_workspace_bytes(N, K, group))
 
 
 def w4a16_gemv_schedule(M, N, K, group, sms) -> dict:
     """Host-only: how w4a16_gemv divides the problem over `sms` SMs."""
-    out = (ctypes.c_int64 * 6)()
+    out = (ctypes.c_int64 * 8)()
     _check("w4a16_gemv_schedule", lib().w4a16_gemv_schedule(M, N, K, group, sms, out))
-    keys = ("units", "octets", "blocks", "whole_octets", "smem_bytes", "ring_kernel")
+    keys = ("rows_per_sweep", "sweeps", "k_parts", "row_blocks", "rows_per_block", "smem_bytes", "stages",
+            "workspace_bytes")
     return dict(zip(keys, (int(v) for v in out)))
 
 
@@ -237,11 +266,10 @@ def alloc_quantized(N, K, group, mode, device="cuda", chosen=True):
 
 
 def alloc_gemv_workspace(N, K, group, device="cuda"):
-    """Zero-filled workspace for w4a16_gemv (calls leave it zero-filled)."""
+    """Zero-filled workspace for w4a16_gemv (calls leave it zero-filled), or None when no
+    call of this shape needs one (rows short enough for one block)."""
     nbytes = w4a16_gemv_workspace_bytes(N, K, group)
-    if nbytes == 0:
-        raise W4Error("w4a16_gemv_workspace_bytes", 2)
-    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device) if nbytes else None
 
 
 def alloc_gemm_workspace(M, N, K, group, device="cuda"):

@@ -150,38 +150,59 @@ w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uin
                         cudaStream_t stream);
 
 /*
+ * fp8_row_quant_gather -- fp8_row_quant of gathered rows: output row m is the quantization of
+ *   source row row_index[m] of X (M_src rows). Used to lay out the routed tokens of a
+ *   mixture-of-experts layer by expert before the grouped GEMM (each token appears once per
+ *   expert that takes it; its codes and scale are those of fp8_row_quant of that token).
+ *   row_index   device, int32 [M], values in [0, M_src); an index outside that range is
+ *               recorded as W4_ERR_DEVICE_CHECK in the device status and its row is
+ *               quantized as zeros.
+ *   Other arguments as fp8_row_quant (outputs have M rows). Errors as fp8_row_quant.
+ */
+w4_status fp8_row_quant_gather(const void *X_bf16, int64_t M_src, int64_t K, int group,
+                               const int32_t *row_index, int64_t M, uint8_t *X_e4m3,
+                               float *row_scale, float *group_sums, uint16_t *gsum_op,
+                               cudaStream_t stream);
+
+/*
  * w4a16_gemv -- weight-only INT4 decode GEMV with the dequantization fused into the
  *   product (QLWG "Weight-only methods": 4-bit weights, 16-bit activations, dequantized
  *   inside the matmul; "The Problem & Context": decode reads every weight once and that
  *   read sets the pace):
  *     y[m, n] = sum_j s[n,j] * sum_{k in group j} x[m,k] * (q[n,k] - z[n,j])
- *   with fp32 accumulation; the output is rounded once (to bf16, or kept fp32). The weight
- *   stream is split into contiguous ranges, one block per SM: whole 8-row groups per block
- *   when the uneven split costs less than combining partial rows across blocks, otherwise
- *   equal ranges, and rows whose reduction is split between blocks are finished by the
- *   last of them in a fixed order. Results are bit-identical run to run on a given GPU.
+ *   The products of the codes with the activations are exact integer sums: each slice of
+ *   128 / MT activations (MT = 1, 2 or 4 rows per sweep) is held as 24-bit fixed point with
+ *   one exponent per slice, exact for every value within 2^11 of the slice's largest
+ *   magnitude and otherwise rounded to 2^-20 of it; fp32 rounding enters only where a group's
+ *   integer sum is scaled and where a row is summed. The output is rounded once (to bf16, or
+ *   kept fp32). One block per SM takes a contiguous run of rows; rows too long for one block
+ *   are split along K and their parts are added, in a fixed order, by the last block to
+ *   finish. Results are bit-identical run to run on a given GPU. A slice containing an
+ *   infinity or a NaN makes its rows' outputs NaN; slices whose largest magnitude is a bf16
+ *   subnormal contribute 0.
  *   x_bf16          device, bf16 [M, K]; 1 <= M <= 16
  *   packed          device, w4_prepack(..., W4_LAYOUT_GEMV) of W[N, K]
  *   y               device, bf16 [M, N], or fp32 [M, N] with W4_OUT_FP32 in flags
  *   flags           W4_OUT_FP32 | W4_OVERLAP_PREVIOUS (see the enum); other bits: W4_ERR_ARG
- *   workspace       device scratch of at least w4a16_gemv_workspace_bytes(N, K, group)
- *                   bytes. It must be zero-filled before its first use; every call that
- *                   completes leaves it zero-filled again, so one workspace can serve any
- *                   sequence of calls on one stream. Calls that may run concurrently on
- *                   the GPU need separate workspaces. After a call whose kernel recorded
- *                   an error in the device status, zero-fill it again.
- *   Errors: NULL / SHAPE (M outside 1..16, N < 1, K < 32, or M > 1 with the rows' per-chunk
- *   activation sums, 16 bytes per row per 128 of K, beyond the block's shared memory: about
- *   K * M > 750,000) / GROUP / ALIGN / ARG / WORKSPACE (missing or too small).
+ *   workspace       device scratch of at least w4a16_gemv_workspace_bytes(N, K, group) bytes;
+ *                   that query returns 0 for shapes whose rows fit one block (K up to about
+ *                   40,000 at M = 1), and then workspace may be NULL. It must be zero-filled
+ *                   before its first use; every call that completes leaves it zero-filled
+ *                   again, so one workspace can serve any sequence of calls on one stream.
+ *                   Calls that may run concurrently on the GPU need separate workspaces.
+ *                   After a call whose kernel recorded an error in the device status,
+ *                   zero-fill it again.
+ *   Errors: NULL / SHAPE (M outside 1..16, N < 1 or N > 2^31, K < 32, K > 2^24, K % 32) /
+ *   GROUP / ALIGN / ARG / WORKSPACE (needed and missing or too small).
  */
 size_t w4a16_gemv_workspace_bytes(int64_t N, int64_t K, int group);
 
 /*
  * w4a16_gemv_schedule -- host-only query (no GPU call): how w4a16_gemv divides the problem
  *   (M rows, N, K, group) over `sms` SMs (1 .. 4096), by the same planner the launch uses.
- *   out[6] receives: units of 8 rows x 128 k, 8-row octets, blocks, whole octets per block
- *   (1) or an even split of the units with a cross-block fixup (0), dynamic shared memory
- *   bytes per block, and 1 when the M = 1 kernel with per-warp bulk-copy rings runs.
+ *   out[8] receives: activation rows per sweep over the weights (1, 2 or 4), sweeps, K parts
+ *   per row (1 = whole rows per block), row blocks, rows per block, dynamic shared memory
+ *   bytes per block, shared-memory ring stages, workspace bytes this call needs.
  *   Errors: NULL / SHAPE / GROUP.
  */
 w4_status w4a16_gemv_schedule(int64_t M, int64_t N, int64_t K, int group, int sms, int64_t *out);
@@ -197,9 +218,10 @@ w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t 
  *   inside another runtime that owns all device memory, or a latency-critical decode loop
  *   in which cudaMalloc's implicit device synchronisation is not acceptable. This entry
  *   point computes exactly what w4a16_gemv computes (same kernel, same partition, same
- *   result bits) but keeps its scratch in a fixed array of w4a16_gemv_noalloc_scratch_limit()
- *   bytes (1 MiB) inside the library's device memory; every GPU that loads the library
- *   holds that array until the process exits. The caller still passes x, packed and y.
+ *   result bits) but keeps its scratch (the partial sums of rows split along K) in a fixed
+ *   array of w4a16_gemv_noalloc_scratch_limit() bytes (1 MiB) inside the library's device
+ *   memory; every GPU that loads the library holds that array until the process exits. The
+ *   caller still passes x, packed and y.
  *   Behaviour:
  *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *   - The first call on a device looks up the array's device address; make that first call
@@ -209,7 +231,9 @@ w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t 
  *   - All calls share the one array: calls that may overlap on the GPU (different streams,
  *     or W4_OVERLAP_PREVIOUS after another noalloc call still running) race on it and give
  *     wrong results. Serialise them, or use w4a16_gemv with separate workspaces.
- *   - A request whose scratch would exceed the limit (N above about 1.7 million rows) returns
+ *   - Only rows split along K (K beyond about 40,000 at M = 1) use the scratch: such a call
+ *     needs K_parts * M * N * 4 bytes of partial sums plus 4 bytes per row block and sweep,
+ *     the workspace_bytes that w4a16_gemv_schedule reports. A request above the limit returns
  *     W4_ERR_SCRATCH_LIMIT without launching anything.
  *   Arguments and other errors as w4a16_gemv.
  */
@@ -232,7 +256,7 @@ w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, 
  *   X_e4m3      device, uint8 [M, K] from fp8_row_quant
  *   row_scale   device, fp32 [M] from fp8_row_quant
  *   gsum_op     device, bf16 [M, w4a8_gsum_op_cols(K, group)] from fp8_row_quant with the
- *               same group
+ *               same group; may be NULL for group 32 (see below)
  *   packed      device, w4_prepack(..., W4_LAYOUT_GEMM) of W[N, K]
  *   Y           device, bf16 [M, N] (out_fp32 == 0) or fp32 [M, N] (out_fp32 == 1)
  *   workspace   NULL, or device scratch of at least w4a8_gemm_workspace_bytes(M, N, K, group)
@@ -248,6 +272,14 @@ w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, 
  *               unsplit schedule, within the same error bounds). A query result of 0 means
  *               the shape is never split and the workspace is not used.
  *   M >= 1; N >= 1; K >= 128, K % 32 == 0.
+ *   Groups of 32: every FP8 MMA of K = 32 would end a group, and the per-group promotion
+ *   (a TMEM readback and one fp32 FMA per output per group on the CUDA cores) would cost
+ *   several times the MMA. For group 32 the kernel instead dequantizes each weight exactly
+ *   into two fp16 parts, w = (q - z) s = hi + lo (exact for |z| < 1024 and |w| < 65504),
+ *   converts the E4M3 activations to fp16 (exact), and accumulates hi x a + lo x a on the
+ *   fp16 tensor cores over the whole K in TMEM: the same dequantized operands, no zero-point
+ *   operand (gsum_op is not read and may be NULL), no split of the last wave (the workspace
+ *   query returns 0).
  *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG / WORKSPACE (non-NULL and smaller than the
  *   query's result).
  */
@@ -289,6 +321,51 @@ w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale,
                             const uint16_t *gsum_op, const int32_t *expert_row_offsets, int E,
                             int64_t M_total, const void *packed, int64_t N, int64_t K, int group,
                             int mode, void *Y, cudaStream_t stream);
+
+/*
+ * Mixture-of-experts layer around w4a8_grouped_gemm ("4-bit by default", opening section:
+ * MoE expert weights as the 4-bit target, gpt-oss). The pages leave the router, the
+ * activation between the two expert projections and the combine open; this library takes
+ * top-k routing with softmax gates over the selected logits, SwiGLU on [gate | up] halves,
+ * and the gate-weighted sum. A layer is: w4_moe_route; fp8_row_quant_gather of the tokens
+ * in expert order; w4a8_grouped_gemm (gate_up); w4_moe_swiglu_quant; w4a8_grouped_gemm
+ * (down); w4_moe_combine.
+ *
+ * w4_moe_route -- logits fp32 [T, E] (device). For each token the k largest logits in
+ *   descending order (equal logits in ascending expert order) -> experts int32 [T, k];
+ *   gates fp32 [T, k] = softmax over those k logits (fp32, expf); expert_row_offsets int32
+ *   [E+1], rows of expert e being [off[e], off[e+1]) of the grouped layout; token_of_row
+ *   int32 [T*k], the token of every grouped row (tokens ascending inside an expert); row_of
+ *   int32 [T, k], the grouped row of token t's i-th expert. Deterministic (no dependence on
+ *   thread timing). One block; 1 <= E <= 1024, 1 <= k <= min(8, E), T * ceil(E/32) * 4 bytes
+ *   <= 96 KiB (T <= 24576 at E = 32). Errors: NULL / SHAPE / ALIGN (4-byte) / CUDA.
+ */
+w4_status w4_moe_route(const float *logits, int64_t T, int E, int k, int32_t *experts,
+                       float *gates, int32_t *expert_row_offsets, int32_t *token_of_row,
+                       int32_t *row_of, cudaStream_t stream);
+
+/*
+ * w4_moe_swiglu_quant -- SwiGLU between the expert projections, then the per-row E4M3
+ *   quantization of its result for the down projection (TAHOMA "Achievement 2" row scale):
+ *   gate_up_bf16 [R, 2H] holds [gate | up] per row; h = gate * up / (1 + exp(-gate)) in fp32;
+ *   row_scale[r] = max(max|h|, 1e-8) / 448; X_e4m3 [R, H] = e4m3(h / row_scale) with IEEE
+ *   division, RNE, saturation. gsum_op (optional, bf16 [R, w4a8_gsum_op_cols(H, group)]) as
+ *   fp8_row_quant writes it, for down projections with group 64 or 128.
+ *   16 <= H <= 16384, H % 16 == 0. Errors: NULL / SHAPE / GROUP / ALIGN.
+ */
+w4_status w4_moe_swiglu_quant(const void *gate_up_bf16, int64_t R, int64_t H, int group,
+                              uint8_t *X_e4m3, float *row_scale, uint16_t *gsum_op,
+                              cudaStream_t stream);
+
+/*
+ * w4_moe_combine -- y[t, :] = sum_{i < k} gates[t, i] * rows[row_of[t, i], :], fp32 products
+ *   and sums in i order, rounded once to bf16. rows_bf16 [R, N] (the down projection's
+ *   output in grouped order), row_of int32 [T, k], gates fp32 [T, k], y_bf16 [T, N].
+ *   A row index outside [0, R) is recorded as W4_ERR_DEVICE_CHECK and skipped.
+ *   N % 8 == 0, 1 <= k <= 8. Errors: NULL / SHAPE / ALIGN.
+ */
+w4_status w4_moe_combine(const void *rows_bf16, int64_t N, int64_t R, const int32_t *row_of,
+                         const float *gates, int64_t T, int k, void *y_bf16, cudaStream_t stream);
 
 /*
  * w4_device_status -- synchronizes `stream`, then reads and clears the device status word

@@ -306,34 +306,37 @@ def moe_combine(rows, row_of, gates) -> np.ndarray:
     return y
 
 
-def moe_layer_ref(X_bits, logits, k: int, gu, dn, group: int, mode):
+def moe_layer_ref(X_bits, logits, k: int, gu, dn, group: int, mode, tokens=None):
     """The whole expert layer in the oracle's arithmetic: route; per-row E4M3 quant of every
     routed token row; fp64 W4A8 gate_up product rounded to bf16 (the GEMM's output type);
     SwiGLU and the per-row E4M3 quant of its result; fp64 W4A8 down product; weighted
-    combine. gu / dn: (codes, scales, zeros) stacked over experts [E, N, ...]. Small shapes
-    only (dense fp64 matmuls). Returns (y fp64 [T, N_down], intermediates dict)."""
+    combine. gu / dn: (codes, scales, zeros) stacked over experts [E, N, ...]. tokens (optional):
+    evaluate only these tokens (the routing is still computed for all of them; rows of other
+    tokens are left zero and their outputs are not meaningful). Dense fp64 matmuls over an
+    expert's rows. Returns (y fp64 [T, N_down], intermediates dict)."""
     import torch
     experts, gates = moe_route(logits, k)
     E = gu[0].shape[0]
     token_of_row, off, row_of = moe_grouping(experts, E)
     Xr = np.asarray(X_bits, np.uint16)[token_of_row]
+    keep = np.ones(token_of_row.size, bool) if tokens is None else np.isin(token_of_row, np.asarray(tokens))
     X8, s_a, _ = row_quant(Xr, 0)
     A = e4m3_decode(X8).astype(np.float64) * s_a.astype(np.float64)[:, None]
     H = gu[0].shape[1] // 2
-    Ygu = np.empty((Xr.shape[0], 2 * H), np.float64)
+    Ygu = np.zeros((Xr.shape[0], 2 * H), np.float64)
     for e in range(E):
-        r0, r1 = off[e], off[e + 1]
-        if r1 > r0:
-            Ygu[r0:r1] = A[r0:r1] @ dequantize(gu[0][e], gu[1][e], None if gu[2] is None else gu[2][e], group, mode).T
+        sel = np.arange(off[e], off[e + 1])[keep[off[e]:off[e + 1]]]
+        if sel.size:
+            Ygu[sel] = A[sel] @ dequantize(gu[0][e], gu[1][e], None if gu[2] is None else gu[2][e], group, mode).T
     Ygu_bits = torch.from_numpy(Ygu).to(torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     H8, s_h, _ = swiglu_row_quant(Ygu_bits, H)
     Ah = e4m3_decode(H8).astype(np.float64) * s_h.astype(np.float64)[:, None]
     Nd = dn[0].shape[1]
-    Yd = np.empty((Xr.shape[0], Nd), np.float64)
+    Yd = np.zeros((Xr.shape[0], Nd), np.float64)
     for e in range(E):
-        r0, r1 = off[e], off[e + 1]
-        if r1 > r0:
-            Yd[r0:r1] = Ah[r0:r1] @ dequantize(dn[0][e], dn[1][e], None if dn[2] is None else dn[2][e], group, mode).T
+        sel = np.arange(off[e], off[e + 1])[keep[off[e]:off[e + 1]]]
+        if sel.size:
+            Yd[sel] = Ah[sel] @ dequantize(dn[0][e], dn[1][e], None if dn[2] is None else dn[2][e], group, mode).T
     y = moe_combine(Yd, row_of, gates)
     return y, dict(experts=experts, gates=gates, token_of_row=token_of_row, offsets=off, row_of=row_of,
                    X8=X8, s_a=s_a, gate_up_bits=Ygu_bits, H8=H8, s_h=s_h, down=Yd)

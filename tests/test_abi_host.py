@@ -45,8 +45,9 @@ def test_status_strings_and_version(lib):
 
 def test_prepack_bytes(lib):
     # GEMV layout: codes of N padded to 8 and K to 128, plus 4 bytes per (row, group)
-    assert w4.w4_prepack_bytes(4096, 4096, 128, w4.W4_LAYOUT_GEMV) == 4096 * 4096 // 2 + 4096 * 32 * 4
-    assert w4.w4_prepack_bytes(1536, 576, 32, w4.W4_LAYOUT_GEMV) == 1536 * 640 // 2 + 1536 * 20 * 4
+    # one record per row: K/2 code bytes, then K/g scale words padded to 16 bytes
+    assert w4.w4_prepack_bytes(4096, 4096, 128, w4.W4_LAYOUT_GEMV) == 4096 * (4096 // 2 + 32 * 4)
+    assert w4.w4_prepack_bytes(1536, 576, 32, w4.W4_LAYOUT_GEMV) == 1536 * (576 // 2 + 80)
     # GEMM layout: rows and K padded to 128; codes, scales of the padded groups, and the
     # zero-point operand with 3 * 90 real groups rounded up to 288 bf16 columns
     assert w4.w4_prepack_bytes(2880, 2880, 32, w4.W4_LAYOUT_GEMM) == \
@@ -139,8 +140,12 @@ def test_gemm_schedule_of_the_prefill_shapes(lib):
     s = w4.w4a8_gemm_schedule(256, 256, 15360, 128, 148)
     assert (s["whole_tiles"], s["split_tiles"], s["split_blocks"], s["grid"]) == (0, 2, 16, 16)
     # ragged K (2880 -> 23 k-blocks, the last one partial): 4 tiles over 8 blocks (2 per tile)
-    s = w4.w4a8_gemm_schedule(300, 256, 2880, 32, 148)
+    s = w4.w4a8_gemm_schedule(300, 256, 2880, 64, 148)
     assert (s["tiles"], s["split_tiles"], s["split_blocks"], s["k_blocks"]) == (4, 4, 8, 23)
+    # groups of 32 take the split-weight fp16 kernel, which keeps every tile whole
+    s = w4.w4a8_gemm_schedule(300, 256, 2880, 32, 148)
+    assert (s["split_tiles"], s["workspace_bytes"], s["grid"]) == (0, 0, 4)
+    assert w4.w4a8_gemm_workspace_bytes(300, 256, 2880, 32) == 0
     # short K: too few k-blocks per block to split
     s = w4.w4a8_gemm_schedule(1000, 130, 640, 128, 148)
     assert (s["split_tiles"], s["grid"], s["workspace_bytes"]) == (0, 8, 0)
@@ -200,28 +205,41 @@ def test_gemm_split_segment_arguments(lib):
 
 # ------------------------------------------------------------------ W4A16 GEMV work split
 
-@pytest.mark.parametrize("K,N,blocks", [(4096, 4096, 128), (4096, 1024, 128), (4096, 14336, 138), (14336, 4096, 128)])
-def test_gemv_decode_shapes_take_whole_octets(lib, K, N, blocks):
-    """M = 1 on 148 SMs: every decode shape gets whole 8-row octets per block (no cross-block
-    fixup). For (14336, 4096) the busiest block carries 4 octets of 112 units against a mean
-    of 387.5 units (+60), cheaper than the fixup of an even split (~160 units)."""
+@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 1024), (4096, 14336), (14336, 4096)])
+def test_gemv_decode_shapes_one_block_per_sm(lib, K, N):
+    """M = 1 on 148 SMs: whole rows per block (no K split, no workspace), N spread over at
+    most 148 blocks in contiguous runs that differ by at most one row's share."""
     s = w4.w4a16_gemv_schedule(1, N, K, 128, 148)
-    assert s["whole_octets"] == 1 and s["blocks"] == blocks and s["ring_kernel"] == 1
-    assert s["units"] == (N // 8) * (K // 128) and s["octets"] == N // 8
-    assert s["smem_bytes"] <= 227 * 1024
+    assert s["rows_per_sweep"] == 1 and s["sweeps"] == 1 and s["k_parts"] == 1
+    assert s["workspace_bytes"] == 0
+    assert s["rows_per_block"] == -(-N // 148)
+    assert s["row_blocks"] == -(-N // s["rows_per_block"]) <= 148
+    assert s["stages"] >= 3 and s["smem_bytes"] <= 227 * 1024
 
 
-def test_gemv_even_split_when_whole_octets_cost_more(lib):
-    # M = 16 units cost ~16x more, so the fixup is worth only ~10 units: 448 > 387.5 + 10
+def test_gemv_activation_rows_per_sweep(lib):
+    # up to 4 activation rows ride along in registers while K/32 slices fit the block
     s = w4.w4a16_gemv_schedule(16, 4096, 14336, 128, 148)
-    assert s["whole_octets"] == 0 and s["blocks"] == 148 and s["ring_kernel"] == 0
-    # M = 1 with 512 octets of 8 units each on 148 SMs: 4 octets (32 units) vs mean 27.7 + 160
-    assert w4.w4a16_gemv_schedule(1, 4096, 1024, 128, 148)["whole_octets"] == 1
-    # fewer octets than SMs: one octet per block
-    s = w4.w4a16_gemv_schedule(1, 512, 65536, 128, 148)
-    assert s["whole_octets"] == 1 and s["blocks"] == 64
+    assert s["rows_per_sweep"] == 4 and s["sweeps"] == 4 and s["k_parts"] == 1
+    s = w4.w4a16_gemv_schedule(3, 4096, 4096, 128, 148)
+    assert s["rows_per_sweep"] == 4 and s["sweeps"] == 1
+    assert w4.w4a16_gemv_schedule(2, 4096, 4096, 128, 148)["rows_per_sweep"] == 2
+    # longer rows hold fewer activation rows per sweep
+    s = w4.w4a16_gemv_schedule(4, 8192, 28672, 128, 148)
+    assert s["rows_per_sweep"] == 2 and s["sweeps"] == 2 and s["k_parts"] == 1
     with pytest.raises(w4.W4Error):
         w4.w4a16_gemv_schedule(17, 4096, 4096, 128, 148)
+
+
+def test_gemv_long_rows_split_along_k(lib):
+    """A row whose slices (128 k each at M = 1) exceed one block's 448 threads, or whose
+    activation planes (3 bytes per k) and two ring stages exceed its shared memory, is split
+    into parts of a multiple of 512 k; the parts' sums go through the workspace."""
+    s = w4.w4a16_gemv_schedule(1, 512, 65536, 128, 148)
+    assert s["k_parts"] == 2 and s["workspace_bytes"] > 0
+    assert w4.w4a16_gemv_workspace_bytes(512, 65536, 128) >= s["workspace_bytes"]
+    assert w4.w4a16_gemv_schedule(1, 512, 32768, 128, 148)["k_parts"] == 1
+    assert w4.w4a16_gemv_workspace_bytes(4096, 14336, 128) == 0
 
 
 def test_gemm_schedule_invariants_over_many_shapes(lib):
@@ -249,27 +267,23 @@ def test_gemm_schedule_invariants_over_many_shapes(lib):
 
 
 def test_gemv_schedule_invariants_over_many_shapes(lib):
-    """For any shape and SM count: shared memory within the per-block limit; at most one
-    block per SM, except when a block's range of octets would not fit shared memory, where
-    the planner doubles the blocks of an even split (blocks never wait on one another, so
-    extra waves are correct); the M = 1 ring kernel serves only M = 1."""
+    """For any shape and SM count: shared memory within the per-block limit, at least two
+    ring stages, row blocks that cover N exactly, sweeps that cover M, and a workspace
+    exactly when rows are split along K."""
     rng = __import__("random").Random(11)
-    for _ in range(300):
-        M = rng.choice([1, 2, 3, 4, 8, 16])
-        N = rng.choice([8, 100, 1024, 1536, 4096, 14336, 100000])
-        K = rng.choice([32, 128, 576, 4096, 14336, 65536])
+    for _ in range(400):
+        M = rng.choice([1, 2, 3, 4, 5, 8, 16])
+        N = rng.choice([1, 8, 100, 1024, 1536, 4096, 14336, 100000])
+        K = rng.choice([32, 96, 128, 576, 2880, 4096, 14336, 28672, 65536, 131072])
         g = rng.choice([g for g in (32, 64, 128) if K % g == 0])
         sms = rng.choice([1, 16, 132, 148])
-        try:
-            s = w4.w4a16_gemv_schedule(M, N, K, g, sms)
-        except w4.W4Error:
-            # the activations' per-chunk sums of M > 1 rows are staged in shared memory:
-            # 16 bytes per row per 128 of K, which 16 rows at K = 65536 exceed
-            assert M * K * 16 // 128 > 96 * 1024, (M, N, K, g, sms)
-            continue
-        assert 1 <= s["blocks"] <= s["units"]
-        assert s["blocks"] <= sms or s["whole_octets"] == 0
-        assert s["smem_bytes"] <= 227 * 1024
-        assert s["octets"] == -(-N // 8) and s["units"] == s["octets"] * -(-K // 128)
-        if M > 1:
-            assert s["ring_kernel"] == 0
+        s = w4.w4a16_gemv_schedule(M, N, K, g, sms)
+        assert s["rows_per_sweep"] in (1, 2, 4) and s["rows_per_sweep"] <= max(M, 4)
+        assert s["sweeps"] == -(-M // s["rows_per_sweep"])
+        assert (s["row_blocks"] - 1) * s["rows_per_block"] < N <= s["row_blocks"] * s["rows_per_block"]
+        assert s["smem_bytes"] <= 227 * 1024 and 2 <= s["stages"] <= 16
+        assert (s["workspace_bytes"] > 0) == (s["k_parts"] > 1)
+        kc = 128 // s["rows_per_sweep"]
+        slices = -(-K // kc)
+        assert s["k_parts"] >= -(-slices // 448)            # one thread per slice of a part
+        assert s["k_parts"] == 1 or s["rows_per_sweep"] == 1  # several activation rows only for whole rows

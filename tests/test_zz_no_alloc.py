@@ -5,9 +5,11 @@ runtime that owns all device memory, or a decode loop that cannot afford cudaMal
 implicit device synchronisation -- so w4a16_gemv_noalloc keeps its scratch in a fixed array
 inside the library instead of a caller-provided workspace. It must give the same outputs as
 w4a16_gemv with a workspace, call after call (the shared array keeps the previous call's
-contents, so a second call in a row is part of the check). This file is collected last so
-that a failure here never hides the other tests' results; it builds its own inputs and runs
-alone in a fresh process as well.
+contents, so a second call in a row is part of the check). The scratch holds the partial sums
+of rows split along K over several blocks (rows too long for one block), so the cases with
+K = 65536 are the ones that use it; the others check that the entry point is also right when
+no scratch is needed. This file is collected last so that a failure here never hides the
+other tests' results, and it builds its own inputs.
 """
 import numpy as np
 import pytest
@@ -37,9 +39,9 @@ def packed_weight(N, K, g, seed):
     return p
 
 
-# (N, K, M): an octet-aligned partition, a stream-K partition with split octets, a long K,
-# a ragged shape and the largest supported M
-CASES = [(1024, 4096, 1), (4096, 4096, 1), (4096, 14336, 1), (77, 320, 3), (4096, 4096, 16)]
+# (N, K, M): decode shapes (whole rows per block, no scratch), rows split along K (the scratch
+# holds their partial sums) at one and three activation rows, a ragged shape and the largest M
+CASES = [(1024, 4096, 1), (4096, 14336, 1), (300, 65536, 1), (100, 65536, 3), (77, 320, 3), (4096, 4096, 16)]
 
 
 @pytest.mark.parametrize("N,K,M", CASES)
@@ -63,14 +65,41 @@ def test_noalloc_matches_workspace_entry_point(N, K, M, flags):
     assert w4.w4_device_status() == 0
 
 
+def test_noalloc_chain_on_one_stream_with_overlap():
+    """Two calls in a row on one stream with W4_OVERLAP_PREVIOUS, both splitting their rows
+    along K: each call clears its counters with a memset on the stream, which orders it
+    after the previous call; the results must equal the workspace entry point's."""
+    dev = torch.device("cuda:0")
+    N, K, g = 300, 65536, 128
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert w4.w4a16_gemv_schedule(1, N, K, g, sms)["k_parts"] >= 2
+    p = packed_weight(N, K, g, 5)
+    xs = [synth.normal((1, K), 1.0, 3, 40 + i).to(dev) for i in range(2)]
+    ws = w4.alloc_gemv_workspace(N, K, g, device=dev)
+    refs = []
+    for x in xs:
+        r = torch.empty(1, N, dtype=torch.float32, device=dev)
+        w4.w4a16_gemv(x, 1, p, N, K, g, "asym", r, w4.W4_OUT_FP32, ws)
+        refs.append(r)
+    outs = [torch.full((1, N), float("nan"), dtype=torch.float32, device=dev) for _ in xs]
+    for x, o in zip(xs, outs):
+        w4.w4a16_gemv_noalloc(x, 1, p, N, K, g, "asym", o, w4.W4_OUT_FP32 | w4.W4_OVERLAP_PREVIOUS)
+    torch.cuda.synchronize()
+    for o, r in zip(outs, refs):
+        assert torch.isfinite(o).all()
+        assert rel(o, r) <= TOL_F32
+    assert w4.w4_device_status() == 0
+
+
 def test_noalloc_rejects_requests_beyond_its_scratch():
     dev = torch.device("cuda:0")
     limit = w4.w4a16_gemv_noalloc_scratch_limit()
     assert limit == 1 << 20
-    N = 8 * (limit // 4)  # the arrival counters alone exceed the scratch
-    x = torch.zeros(1, 32, dtype=torch.bfloat16, device=dev)
+    # rows split along K need kparts * M * N * 4 bytes of partial sums: 2 parts of 200000 rows
+    N = 200000
     dummy = torch.zeros(256, dtype=torch.uint8, device=dev)
+    x = torch.zeros(1, 65536, dtype=torch.bfloat16, device=dev)
     with pytest.raises(w4.W4Error) as e:
-        w4.w4a16_gemv_noalloc(x, 1, dummy, N, 32, 32, "asym", dummy, 0)
+        w4.w4a16_gemv_noalloc(x, 1, dummy, N, 65536, 128, "asym", dummy, 0)
     assert e.value.code == 11
     torch.cuda.synchronize()
