@@ -70,6 +70,12 @@ def _load():
         lib.o_w4a8_ref_pairs.argtypes = [P, P, I64, P, P, P, I64, I, I, P, P, P, I64, P]
         lib.o_fake_quant.restype = None
         lib.o_fake_quant.argtypes = [P, I64, I64, I, I, P, P]
+        lib.o_nf4_levels.restype = None
+        lib.o_nf4_levels.argtypes = [P]
+        lib.o_nf4_quantize.restype = I
+        lib.o_nf4_quantize.argtypes = [P, I64, I64, P, P]
+        lib.o_nf4_gemv_ref.restype = None
+        lib.o_nf4_gemv_ref.argtypes = [P, I64, P, P, I64, I64, P]
         lib.o_moe_route.restype = None
         lib.o_moe_route.argtypes = [P, I64, I, I, P, P]
         lib.o_swiglu_row_quant.restype = None
@@ -244,6 +250,39 @@ def w4a8_ref_dense(X8, s_a, codes, scales, zeros, group: int, mode) -> np.ndarra
     A = e4m3_decode(X8).astype(np.float64) * np.asarray(s_a, np.float64)[:, None]
     W = dequantize(codes, scales, zeros, group, mode)
     return A @ W.T
+
+
+# ------------------------------------------------------------------ NF4 comparator
+
+def nf4_levels() -> np.ndarray:
+    """The 16 NF4 levels (fp32, ascending)."""
+    lib = _load()
+    out = np.empty(16, np.float32)
+    lib.o_nf4_levels(_p(out))
+    return out
+
+
+def nf4_quantize(W_bits):
+    """NF4 in blocks of 64: (codes u8 [N, K/2] packed as the INT4 codes, absmax f32 [N, K/64])."""
+    lib = _load()
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    codes = np.empty((N, K // 2), np.uint8)
+    absmax = np.empty((N, K // 64), np.float32)
+    if lib.o_nf4_quantize(_p(W), N, K, _p(codes), _p(absmax)):
+        raise ValueError("oracle nf4_quantize: K must be a multiple of 64")
+    return codes, absmax
+
+
+def nf4_gemv_ref(x_bits, codes, absmax) -> np.ndarray:
+    lib = _load()
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    codes = _c(codes, np.uint8)
+    N = codes.shape[0]
+    y = np.empty((M, N), np.float64)
+    lib.o_nf4_gemv_ref(_p(x), M, _p(codes), _p(_c(absmax, np.float32)), N, K, _p(y))
+    return y
 
 
 # ------------------------------------------------------------------ mixture-of-experts layer

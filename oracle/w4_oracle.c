@@ -213,8 +213,8 @@ static void quantize_block(const float *w, int g, int asym, const float *grid, i
         if (w[k] > hi) hi = w[k];
         if (fabsf(w[k]) > amax) amax = fabsf(w[k]);
     }
-    uint8_t nib[128];
-    float e2[128];
+    uint8_t nib[256];
+    float e2[256];
     float best = 0.0f;
     for (int i = 0; i < ngrid; ++i) {
         uint16_t sb;
@@ -236,13 +236,13 @@ static void quantize_block(const float *w, int g, int asym, const float *grid, i
 EXPORT int o_quantize(const uint16_t *W, int64_t N, int64_t K, int g, int asym,
                       const float *grid, int ngrid, uint8_t *codes, uint16_t *scales,
                       int16_t *zeros, uint8_t *chosen) {
-    if (g != 32 && g != 64 && g != 128) return 1;
+    if (g != 32 && g != 64 && g != 128 && g != 256) return 1;
     if (K % g != 0 || K % 2 != 0 || ngrid < 1) return 1;
     int64_t J = K / g;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
-        float w[128];
-        uint8_t nib[128];
+        float w[256];
+        uint8_t nib[256];
         for (int64_t j = 0; j < J; ++j) {
             for (int k = 0; k < g; ++k) w[k] = bf16_to_f32(W[n * K + j * g + k]);
             uint16_t s;
@@ -261,8 +261,8 @@ EXPORT int o_quantize(const uint16_t *W, int64_t N, int64_t K, int g, int asym,
 
 /* Candidate error of one block for one ratio, exposed for the brute-force tests. */
 EXPORT float o_block_sse(const uint16_t *wb, int g, int asym, float r) {
-    float w[128], e2[128];
-    uint8_t nib[128];
+    float w[256], e2[256];
+    uint8_t nib[256];
     float lo, hi, amax;
     for (int k = 0; k < g; ++k) w[k] = bf16_to_f32(wb[k]);
     lo = hi = w[0];
@@ -501,4 +501,97 @@ EXPORT void o_fake_quant(const double *x, int64_t n, int64_t block, int bits, in
         for (int64_t i = 0; i < len; ++i) out[b * block + i] = lattice_round_trip(&L, v[i]);
         if (scale_out) scale_out[b] = L.step;
     }
+}
+
+/* ------------------------------------------------------------------ NF4 comparator */
+
+/* Inverse of the standard normal CDF, Phi(x) = erfc(-x / sqrt(2)) / 2: bisection to a
+ * bracketing interval, then Newton steps on Phi(x) - p (Phi' is the normal density). */
+static double inv_phi(double p) {
+    double lo = -40.0, hi = 40.0;
+    for (int i = 0; i < 200; ++i) {
+        double mid = 0.5 * (lo + hi);
+        if (0.5 * erfc(-mid / sqrt(2.0)) < p) lo = mid; else hi = mid;
+    }
+    double x = 0.5 * (lo + hi);
+    for (int i = 0; i < 3; ++i) {
+        double f = 0.5 * erfc(-x / sqrt(2.0)) - p;
+        double d = exp(-0.5 * x * x) / sqrt(2.0 * 3.14159265358979323846);
+        if (d > 0.0) x -= f / d;
+    }
+    return x;
+}
+
+/* NF4 levels ([P2] "Quantizing LLMs Without Guesswork", NF4 paragraph: 16 levels that are
+ * quantiles of a normal distribution, blocks of 64). The pages leave the construction open;
+ * this is the QLoRA one: with delta = (1/32 + 1/30) / 2, eight positive levels
+ * Phi^-1(p) at p = 1 - delta + i (delta - 1/2) / 8, i = 0..7, seven negative levels
+ * -Phi^-1(p) at p = 1 - delta + i (delta - 1/2) / 7, i = 0..6, and an exact zero, all divided
+ * by Phi^-1(1 - delta) so that the extremes are -1 and 1; sorted ascending, rounded to fp32. */
+EXPORT void o_nf4_levels(float *out) {
+    const double delta = 0.5 * (1.0 / 32.0 + 1.0 / 30.0);
+    const double top = inv_phi(1.0 - delta);
+    double v[16];
+    int n = 0;
+    for (int i = 0; i < 7; ++i) v[n++] = -inv_phi(1.0 - delta + i * (delta - 0.5) / 7.0) / top;
+    v[n++] = 0.0;
+    for (int i = 7; i >= 0; --i) v[n++] = inv_phi(1.0 - delta + i * (delta - 0.5) / 8.0) / top;
+    /* ascending: the negatives were built from -1 upwards, the positives from the smallest */
+    for (int i = 0; i < 16; ++i) out[i] = (float)v[i];
+}
+
+/* NF4 quantization of W[N, K] (bf16) in blocks of 64 along K: a = max|w| (fp32), stored as
+ * the block's fp32 scale; each weight's code is the level nearest to w / a (fp32 IEEE
+ * division, distances |w/a - level| in fp32, ties to the lower level); an all-zero block
+ * has a = 0 and every code at the zero level. Codes packed as the INT4 ones: byte j of a
+ * row = q[2j] | q[2j+1] << 4. */
+EXPORT int o_nf4_quantize(const uint16_t *W, int64_t N, int64_t K, uint8_t *codes, float *absmax) {
+    if (K % 64 != 0) return 1;
+    float lv[16];
+    o_nf4_levels(lv);
+    int zero_code = 7;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < K / 64; ++b) {
+            float w[64], a = 0.0f;
+            for (int i = 0; i < 64; ++i) {
+                w[i] = bf16_to_f32(W[n * K + b * 64 + i]);
+                if (fabsf(w[i]) > a) a = fabsf(w[i]);
+            }
+            absmax[n * (K / 64) + b] = a;
+            uint8_t q[64];
+            for (int i = 0; i < 64; ++i) {
+                if (a == 0.0f) { q[i] = (uint8_t)zero_code; continue; }
+                float t = w[i] / a;
+                int best = 0;
+                float bd = fabsf(t - lv[0]);
+                for (int c = 1; c < 16; ++c) {
+                    float d = fabsf(t - lv[c]);
+                    if (d < bd) { bd = d; best = c; }
+                }
+                q[i] = (uint8_t)best;
+            }
+            for (int i = 0; i < 64; i += 2)
+                codes[n * (K / 2) + (b * 64 + i) / 2] = (uint8_t)(q[i] | (q[i + 1] << 4));
+        }
+    }
+    return 0;
+}
+
+/* NF4 W4A16 GEMV reference: y[m, n] = sum_k x[m,k] * level[q[n,k]] * a[n, k/64] in fp64. */
+EXPORT void o_nf4_gemv_ref(const uint16_t *x, int64_t M, const uint8_t *codes, const float *absmax, int64_t N,
+                           int64_t K, double *y) {
+    float lv[16];
+    o_nf4_levels(lv);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                uint8_t byte = codes[n * (K / 2) + k / 2];
+                int q = (k & 1) ? (byte >> 4) : (byte & 0xF);
+                acc += (double)bf16_to_f32(x[m * K + k]) * (double)lv[q] * (double)absmax[n * (K / 64) + k / 64];
+            }
+            y[m * N + n] = acc;
+        }
 }

@@ -195,7 +195,7 @@ def _rand_weights(N, K, seed, outliers=0):
     return synth.bf16_bits(w), w.float().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("g", [32, 64, 128])
+@pytest.mark.parametrize("g", [32, 64, 128, 256])
 def test_sym_never_emits_minus8_and_error_bound(g):
     bits, w = _rand_weights(64, 1024, 3, outliers=3)
     codes, scales, _, _ = oracle.quantize(bits, g, "sym", [1.0])
@@ -308,7 +308,7 @@ def _candidate_fp64(w32, mode, r):
 
 
 @pytest.mark.parametrize("mode", ["sym", "asym"])
-@pytest.mark.parametrize("g", [32, 128])
+@pytest.mark.parametrize("g", [32, 128, 256])
 def test_clip_search_is_brute_force_argmin(mode, g):
     rng = np.random.default_rng(11)
     grid = synth.clip_grid_20()
@@ -588,3 +588,52 @@ def test_moe_layer_ref_matches_independent_numpy_composition():
             o = e4m3_rows(hh).numpy() @ oracle.dequantize(*dn[e], g, "asym").T
             ref[t] += w[i] * o[0]
     assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ NF4 comparator
+
+def test_nf4_levels_are_normal_quantiles():
+    """The levels against scipy's normal quantile function (an independent inverse CDF):
+    eight positive and seven negative quantiles at equal probability steps from 1 - delta
+    towards 1/2, delta = (1/32 + 1/30) / 2, an exact zero, scaled to [-1, 1]."""
+    from scipy.stats import norm
+    v = oracle.nf4_levels().astype(np.float64)
+    d = 0.5 * (1 / 32 + 1 / 30)
+    top = norm.ppf(1 - d)
+    pos = norm.ppf(np.linspace(1 - d, 0.5, 9)[:-1]) / top
+    neg = -norm.ppf(np.linspace(1 - d, 0.5, 8)[:-1]) / top
+    ref = np.sort(np.concatenate([pos, [0.0], neg])).astype(np.float32)
+    assert np.allclose(v, ref, rtol=0, atol=2e-7)
+    assert v[7] == 0.0 and v[0] == -1.0 and v[15] == 1.0 and np.all(np.diff(v) > 0)
+    # equal probability steps: Phi(level * top) on the positive side
+    p = norm.cdf(v[8:] * top)
+    assert np.allclose(np.diff(p), (1 - d - 0.5) / 8, rtol=0, atol=1e-6)
+
+
+def test_nf4_quantize_is_nearest_level_per_block():
+    rng = np.random.default_rng(31)
+    W = torch.from_numpy(rng.normal(0, 0.02, (40, 256)).astype(np.float32))
+    W[3, 64:128] = 0.0
+    W[5, :64] = torch.linspace(-1, 1, 64)
+    Wb = W.to(torch.bfloat16)
+    codes, a = oracle.nf4_quantize(synth.bf16_bits(Wb))
+    w = Wb.float().numpy()
+    lv = oracle.nf4_levels()
+    blocks = w.reshape(40, 4, 64)
+    amax = np.abs(blocks).max(2)
+    assert np.array_equal(a, amax.astype(np.float32))
+    t = np.divide(blocks, amax[:, :, None], out=np.zeros_like(blocks), where=amax[:, :, None] > 0).astype(np.float32)
+    q = np.argmin(np.abs(t[..., None] - lv).astype(np.float32), axis=-1)
+    q[amax == 0] = 7
+    q = q.reshape(40, 256)
+    assert np.array_equal(oracle.unpack_codes(codes), q)
+
+
+def test_nf4_gemv_ref_matches_numpy():
+    rng = np.random.default_rng(32)
+    Wb = torch.from_numpy(rng.normal(0, 0.02, (24, 192)).astype(np.float32)).to(torch.bfloat16)
+    codes, a = oracle.nf4_quantize(synth.bf16_bits(Wb))
+    x = torch.from_numpy(rng.normal(0, 1, (3, 192)).astype(np.float32)).to(torch.bfloat16)
+    Wd = oracle.nf4_levels().astype(np.float64)[oracle.unpack_codes(codes)] * np.repeat(a.astype(np.float64), 64, 1)
+    ref = x.double().numpy() @ Wd.T
+    assert np.allclose(oracle.nf4_gemv_ref(synth.bf16_bits(x), codes, a), ref, rtol=1e-13, atol=1e-13)

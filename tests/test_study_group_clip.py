@@ -7,8 +7,10 @@ on three synthetic layers:
 - the single layer with outlier input columns, in the pages' orientation W[576, 1536];
 - an 8B-shaped decode layer with 0.1% outlier columns;
 - a Student-t(3) layer.
-For g in {32, 64, 128}, the GPU quantizer gives the same codes, scales and zero points bit
-for bit (tests/test_gpu_quantize.py), so the table holds for the kernels too.
+For g in {32, 64, 128, 256}, the GPU quantizer gives the same codes, scales and zero points
+bit for bit (tests/test_gpu_quantize.py), and tests/test_gpu_study.py recomputes the output
+errors with the GPU quantizer and GEMV. TAHOMA "What the WMT26 paper finds" weighs block 256
+against 128 (smaller, faster, worse), which is why 256 is in the table.
 
 Asserted is only what the method guarantees or what these layers show by a wide margin:
 - a grid that starts with 1.0 never raises a block's error, so the layer's weight error with
@@ -24,6 +26,7 @@ import oracle
 from bit_gemm_wise_b200 import synth
 
 GRIDS = {"none": [1.0], "page 11": synth.clip_grid_page(), "20 in [0.7,1]": synth.clip_grid_20()}
+GROUPS = (32, 64, 128, 256)
 
 
 def layers():
@@ -48,7 +51,7 @@ def table():
         x = X.float().numpy().astype(np.float64)
         y = x @ w.T
         for mode in ("sym", "asym"):
-            for g in (32, 64, 128):
+            for g in GROUPS:
                 for gname, grid in GRIDS.items():
                     codes, scales, zeros, _ = oracle.quantize(bits, g, mode, grid, want_chosen=False)
                     wd = oracle.dequantize(codes, scales, zeros, g, mode)
@@ -80,8 +83,8 @@ def test_smaller_groups_and_asymmetric_codes_lower_the_error(table):
     for name in {r["layer"] for r in table}:
         for gname in GRIDS:
             for mode in ("sym", "asym"):
-                e = [pick(table, layer=name, mode=mode, g=g, grid=gname)["werr"] for g in (32, 64, 128)]
-                assert e[0] < e[1] < e[2], (name, mode, gname, e)
-            for g in (32, 64, 128):
+                e = [pick(table, layer=name, mode=mode, g=g, grid=gname)["werr"] for g in GROUPS]
+                assert all(a < b for a, b in zip(e, e[1:])), (name, mode, gname, e)
+            for g in GROUPS:
                 assert pick(table, layer=name, mode="asym", g=g, grid=gname)["werr"] < \
                     pick(table, layer=name, mode="sym", g=g, grid=gname)["werr"]
