@@ -391,6 +391,40 @@ def measure_rows(args, dev, pk):
                                     "frac_fp32_fma_peak": round(flops / (ms * 1e-3) / 1e12 / fp32_peak, 4)}
         del d
 
+    # NF4 comparator at M = 1 over the same decode shapes: normal-quantile levels, blocks of 64
+    # with an fp32 absmax, a table lookup per code byte (the format the pages compare with)
+    if "gemv" in want:
+        nf = []
+        per_copy = sum(N * K // 2 + N * (K // 64) * 4 for K, N in DECODE_SHAPES)
+        R = max(2, -(-3 * L2_BYTES // per_copy))  # weight copies: more than 3x L2 in all
+        for K, N in DECODE_SHAPES:
+            W = synth.decode_weight(K, N, args.seed, device=dev)
+            codes = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+            am = torch.empty(N, K // 64, dtype=torch.float32, device=dev)
+            w4.w4_nf4_quantize(W, N, K, codes, am)
+            nf.append((K, N, [codes] + [codes.clone() for _ in range(R - 1)], [am] + [am.clone() for _ in range(R - 1)],
+                       synth.decode_activation(1, K, args.seed, device=dev), torch.empty(1, N, dtype=torch.bfloat16, device=dev)))
+            del W
+        nbytes = sum(N * K // 2 + N * (K // 64) * 4 + 2 * K + 2 * N for K, N, *_ in nf)
+
+        def nf_step(i):
+            for K, N, cs, ams, x, y in nf:
+                w4.w4_nf4_gemv(x, 1, cs[i % R], ams[i % R], N, K, y, w4.W4_OVERLAP_PREVIOUS)
+
+        nf_step(0)
+        side = torch.cuda.Stream()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=side):
+            for i in range(4 * R):
+                nf_step(i)
+        gr.replay()
+        ms = float(np.median([time_region(lambda i: gr.replay(), 1) for _ in range(9)])) / (4 * R)
+        rows["nf4_gemv_M1"] = {"value": round(nbytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                               "us_per_step": round(ms * 1e3, 2), "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm"], 4),
+                               "note": "NF4 comparator (normal-quantile levels, blocks of 64, fp32 absmax), same four "
+                                       "decode shapes, one graph of launches"}
+        del nf, gr
+
     # single linear layer (K=576, N=1536, group 32 symmetric, M=1): launch-latency-dominated,
     # reported in microseconds
     if "gemv" in want:

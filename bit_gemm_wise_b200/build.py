@@ -28,6 +28,7 @@ SOURCES = {
     "w4a16_gemv.cu": [],
     "w4a8_gemm.cu": [],
     "w4_moe.cu": [],
+    "w4_nf4.cu": [],
 }
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

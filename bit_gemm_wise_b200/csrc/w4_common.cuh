@@ -17,7 +17,7 @@ constexpr unsigned FULL = 0xffffffffu;
 // ------------------------------------------------------------------ host-side checks
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-inline bool valid_group(int g) { return g == 32 || g == 64 || g == 128; }
+inline bool valid_group(int g) { return g == 32 || g == 64 || g == 128 || g == 256; }
 inline bool valid_mode(int m) { return m == W4_SYM || m == W4_ASYM; }
 
 // Address of this device's status word (kernels record timeouts / failed checks there).

@@ -4,7 +4,7 @@
 // dequantize; "Four-bit inference ... Tahoma", The naive symmetric baseline, Achievement 1,
 // MSE clipping.
 //
-// Eight lanes own one group of G weights (G = 32, 64, 128), four groups per warp. The group
+// Eight lanes own one group of G weights (G = 32, 64, 128, 256), four groups per warp. The group
 // is cut into 32 chunks of G/32 consecutive weights; lane j (0..7) of the group holds chunks
 // j, j+8, j+16 and j+24. The group's min / max / max|w| come from shuffles (exact). Every
 // clip ratio is evaluated in registers: scale rounded to fp16, zero point, codes,
@@ -104,7 +104,13 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restric
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
             const uint16_t *cs = src + (j + 8 * ch) * C;
-            if constexpr (C == 4) {
+            if constexpr (C == 8) {
+                const uint4 v = live ? *reinterpret_cast<const uint4 *>(cs) : make_uint4(0u, 0u, 0u, 0u);
+                w[ch * 8 + 0] = bf16_lo(v.x); w[ch * 8 + 1] = bf16_hi(v.x);
+                w[ch * 8 + 2] = bf16_lo(v.y); w[ch * 8 + 3] = bf16_hi(v.y);
+                w[ch * 8 + 4] = bf16_lo(v.z); w[ch * 8 + 5] = bf16_hi(v.z);
+                w[ch * 8 + 6] = bf16_lo(v.w); w[ch * 8 + 7] = bf16_hi(v.w);
+            } else if constexpr (C == 4) {
                 const uint2 v = live ? *reinterpret_cast<const uint2 *>(cs) : make_uint2(0u, 0u);
                 w[ch * 4 + 0] = bf16_lo(v.x); w[ch * 4 + 1] = bf16_hi(v.x);
                 w[ch * 4 + 2] = bf16_lo(v.y); w[ch * 4 + 3] = bf16_hi(v.y);
@@ -189,7 +195,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t *__restric
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
                 const int c0 = (j + 8 * ch) * C;  // first weight of the chunk
-                if constexpr (C == 4) reinterpret_cast<uint16_t *>(dst)[c0 / 4] = (uint16_t)qv[ch];
+                if constexpr (C == 8) reinterpret_cast<uint32_t *>(dst)[c0 / 8] = qv[ch];
+                else if constexpr (C == 4) reinterpret_cast<uint16_t *>(dst)[c0 / 4] = (uint16_t)qv[ch];
                 else if constexpr (C == 2) dst[c0 / 2] = (uint8_t)qv[ch];
                 else if ((j & 1) == 0) dst[c0 / 2] = (uint8_t)qv[ch];
             }
@@ -239,7 +246,8 @@ W4_API w4_status w4_quantize(const void *W_bf16, int64_t N, int64_t K, int group
     const bool asym = mode == W4_ASYM;
     if (group == 32) { if (asym) W4_Q(32, true); else W4_Q(32, false); }
     else if (group == 64) { if (asym) W4_Q(64, true); else W4_Q(64, false); }
-    else { if (asym) W4_Q(128, true); else W4_Q(128, false); }
+    else if (group == 128) { if (asym) W4_Q(128, true); else W4_Q(128, false); }
+    else { if (asym) W4_Q(256, true); else W4_Q(256, false); }
 #undef W4_Q
     return launch_status();
 }

@@ -622,6 +622,7 @@ template <int MT, int G>
 static void *kernel_ptr() { return reinterpret_cast<void *>(gemv_kernel<MT, G>); }
 
 static void *pick_kernel(int MT, int g) {
+    // groups of 128 or more: every slice (at most 128 k) lies in one group, one kernel serves
     if (MT == 4) return g == 32 ? kernel_ptr<4, 32>() : (g == 64 ? kernel_ptr<4, 64>() : kernel_ptr<4, 128>());
     if (MT == 2) return g == 32 ? kernel_ptr<2, 32>() : (g == 64 ? kernel_ptr<2, 64>() : kernel_ptr<2, 128>());
     return g == 32 ? kernel_ptr<1, 32>() : (g == 64 ? kernel_ptr<1, 64>() : kernel_ptr<1, 128>());

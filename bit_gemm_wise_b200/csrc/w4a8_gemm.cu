@@ -1293,7 +1293,8 @@ static w4_status launch_f16(const uint8_t *X8, const float *row_scale, const int
 static w4_status launch(const uint8_t *X8, const float *row_scale, const uint16_t *gop, const int32_t *offsets, int E,
                         int64_t M, const void *packed, int64_t N, int64_t K, int group, void *Y, int out_fp32,
                         void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    if (group == 32) return launch_f16(X8, row_scale, offsets, E, M, packed, N, K, group, Y, out_fp32, stream);
+    if (group == 32 || group == 256)
+        return launch_f16(X8, row_scale, offsets, E, M, packed, N, K, group, Y, out_fp32, stream);
     EncodeTiledFn enc = encode_fn();
     if (!enc) return W4_ERR_CUDA;
     const GemmLayout L = gemm_layout(N, K, group);
@@ -1387,7 +1388,7 @@ W4_API size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int gro
     const int sms = gemm::sm_count_cached();
     if (sms < 1) return 0;
     return gemm::make_plan(gemm::dense_tiles(M, N, K, group), gemm_layout(N, K, group).Kpad / gemm::BK, sms,
-                           group != 32)
+                           group == 64 || group == 128)
         .ws_bytes;
 }
 
@@ -1396,7 +1397,7 @@ W4_API w4_status w4a8_gemm_schedule(int64_t M, int64_t N, int64_t K, int group, 
     if (!gemm_shape_ok(M, N, K) || sms < 1 || sms > 4096) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
     const int64_t KT = gemm_layout(N, K, group).Kpad / gemm::BK;
-    const gemm::Plan p = gemm::make_plan(gemm::dense_tiles(M, N, K, group), KT, sms, group != 32);
+    const gemm::Plan p = gemm::make_plan(gemm::dense_tiles(M, N, K, group), KT, sms, group == 64 || group == 128);
     out[0] = p.tiles;
     out[1] = p.dpt;
     out[2] = p.r;
@@ -1437,7 +1438,7 @@ W4_API w4_status w4a8_gemm_split_segment(int64_t R, int64_t KT, int64_t PS, int6
 W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op, int64_t M,
                            const void *packed, int64_t N, int64_t K, int group, int mode, void *Y, int out_fp32,
                            void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    if (!X_e4m3 || !row_scale || !packed || !Y || (!gsum_op && group != 32)) return W4_ERR_NULL;
+    if (!X_e4m3 || !row_scale || !packed || !Y || (!gsum_op && (group == 64 || group == 128))) return W4_ERR_NULL;
     if (!valid_mode(mode) || (out_fp32 != 0 && out_fp32 != 1)) return W4_ERR_ARG;
     if (!gemm_shape_ok(M, N, K)) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
@@ -1451,7 +1452,7 @@ W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const 
 W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op,
                                    const int32_t *expert_row_offsets, int E, int64_t M_total, const void *packed,
                                    int64_t N, int64_t K, int group, int mode, void *Y, cudaStream_t stream) {
-    if (!X_e4m3 || !row_scale || !expert_row_offsets || !packed || !Y || (!gsum_op && group != 32))
+    if (!X_e4m3 || !row_scale || !expert_row_offsets || !packed || !Y || (!gsum_op && (group == 64 || group == 128)))
         return W4_ERR_NULL;
     if (!valid_mode(mode)) return W4_ERR_ARG;
     if (E < 1 || E > 1024 || M_total < 1 || M_total > 0x7fffffffLL || N < 1 || N > 0x7fffffffLL || K < 128 ||

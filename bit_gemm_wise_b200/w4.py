@@ -41,6 +41,9 @@ SIGNATURES = [
     ("w4_moe_route", _I, [_P, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
     ("w4_moe_swiglu_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P]),
     ("w4_moe_combine", _I, [_P, _I64, _I64, _P, _P, _I64, _I, _P, _P]),
+    ("w4_nf4_levels", _I, [_P]),
+    ("w4_nf4_quantize", _I, [_P, _I64, _I64, _P, _P, _P]),
+    ("w4_nf4_gemv", _I, [_P, _I64, _P, _P, _I64, _I64, _P, _I, _P]),
     ("w4a16_gemv_workspace_bytes", _SZ, [_I64, _I64, _I]),
     ("w4a16_gemv_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
@@ -169,6 +172,21 @@ def w4_moe_swiglu_quant(gate_up, R, H, group, X8, row_scale, gsum_op=None, strea
 def w4_moe_combine(rows, N, R, row_of, gates, T, k, y, stream=None):
     rc = lib().w4_moe_combine(_ptr(rows), N, R, _ptr(row_of), _ptr(gates), T, k, _ptr(y), _stream(stream))
     _check("w4_moe_combine", rc)
+
+
+def w4_nf4_levels():
+    out = (ctypes.c_float * 16)()
+    _check("w4_nf4_levels", lib().w4_nf4_levels(ctypes.cast(out, _P)))
+    return [float(v) for v in out]
+
+
+def w4_nf4_quantize(W, N, K, codes, absmax, stream=None):
+    _check("w4_nf4_quantize", lib().w4_nf4_quantize(_ptr(W), N, K, _ptr(codes), _ptr(absmax), _stream(stream)))
+
+
+def w4_nf4_gemv(x, M, codes, absmax, N, K, y, flags=0, stream=None):
+    rc = lib().w4_nf4_gemv(_ptr(x), M, _ptr(codes), _ptr(absmax), N, K, _ptr(y), int(flags), _stream(stream))
+    _check("w4_nf4_gemv", rc)
 
 
 def w4a16_gemv_workspace_bytes(N, K, group) -> int:

@@ -368,6 +368,32 @@ w4_status w4_moe_combine(const void *rows_bf16, int64_t N, int64_t R, const int3
                          const float *gates, int64_t T, int k, void *y_bf16, cudaStream_t stream);
 
 /*
+ * NF4 comparator (QLWG, NF4 paragraph: 16 levels that are quantiles of a normal distribution,
+ * blocks of 64; TAHOMA: the NF4 operating point its W4A8 path is measured against). The
+ * levels follow the QLoRA construction (the pages leave it open): with delta = (1/32 + 1/30)/2,
+ * the normal quantiles at eight equal probability steps from 1 - delta down to 1/2 (exclusive),
+ * the negatives of seven such steps, and an exact zero, divided by the largest, in fp32,
+ * ascending. Each block of 64 consecutive weights of a row keeps its max|w| as an fp32 scale
+ * (single-level scales: the pages' double quantization of the scales is not built).
+ *
+ * w4_nf4_levels -- the 16 levels (host array).
+ * w4_nf4_quantize -- W_bf16 [N, K] -> codes uint8 [N, K/2] (packed like the INT4 codes: byte
+ *   j = q[2j] | q[2j+1] << 4) and absmax fp32 [N, K/64]. The code of w is the level nearest to
+ *   w / a (IEEE fp32 division and fp32 distances; ties to the lower level); an all-zero block
+ *   gets a = 0 and the zero level. K % 64 == 0. Errors: NULL / SHAPE / ALIGN.
+ * w4_nf4_gemv -- y[m, n] = sum_k x[m, k] * level[q[n, k]] * a[n, k / 64] with fp32
+ *   accumulation, output bf16 (or fp32 with W4_OUT_FP32); W4_OVERLAP_PREVIOUS as for
+ *   w4a16_gemv. Reads the quantizer's codes and absmax directly (no prepack). 1 <= M <= 4,
+ *   M * K * 4 bytes of activations staged in shared memory (K <= 57,000 at M = 1).
+ *   Errors: NULL / SHAPE / ALIGN / ARG.
+ */
+w4_status w4_nf4_levels(float *levels_host);
+w4_status w4_nf4_quantize(const void *W_bf16, int64_t N, int64_t K, uint8_t *codes, float *absmax,
+                          cudaStream_t stream);
+w4_status w4_nf4_gemv(const void *x_bf16, int64_t M, const uint8_t *codes, const float *absmax,
+                      int64_t N, int64_t K, void *y, int flags, cudaStream_t stream);
+
+/*
  * w4_device_status -- synchronizes `stream`, then reads and clears the device status word
  *   of the current device. *code_out receives W4_OK or the first W4_ERR_TIMEOUT /
  *   W4_ERR_DEVICE_CHECK recorded since the last call. Returns W4_ERR_CUDA if the

@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from bit_gemm_wise_b200 import w4
@@ -252,7 +253,7 @@ def test_gemm_schedule_invariants_over_many_shapes(lib):
         M = rng.choice([1, 7, 256, 300, 1000, 4096, 9000])
         N = rng.choice([128, 200, 1536, 3840, 4096, 15360])
         K = rng.choice([128, 256, 576, 2880, 3840, 8192, 15360])
-        g = rng.choice([g for g in (32, 64, 128) if K % g == 0])
+        g = rng.choice([g for g in (32, 64, 128, 256) if K % g == 0])
         sms = rng.choice([1, 2, 8, 132, 148, 160])
         s = w4.w4a8_gemm_schedule(M, N, K, g, sms)
         assert 1 <= s["grid"] <= sms
@@ -275,7 +276,7 @@ def test_gemv_schedule_invariants_over_many_shapes(lib):
         M = rng.choice([1, 2, 3, 4, 5, 8, 16])
         N = rng.choice([1, 8, 100, 1024, 1536, 4096, 14336, 100000])
         K = rng.choice([32, 96, 128, 576, 2880, 4096, 14336, 28672, 65536, 131072])
-        g = rng.choice([g for g in (32, 64, 128) if K % g == 0])
+        g = rng.choice([g for g in (32, 64, 128, 256) if K % g == 0])
         sms = rng.choice([1, 16, 132, 148])
         s = w4.w4a16_gemv_schedule(M, N, K, g, sms)
         assert s["rows_per_sweep"] in (1, 2, 4) and s["rows_per_sweep"] <= max(M, 4)
@@ -287,3 +288,10 @@ def test_gemv_schedule_invariants_over_many_shapes(lib):
         slices = -(-K // kc)
         assert s["k_parts"] >= -(-slices // 448)            # one thread per slice of a part
         assert s["k_parts"] == 1 or s["rows_per_sweep"] == 1  # several activation rows only for whole rows
+
+
+def test_nf4_levels_of_the_library_equal_the_oracle(lib):
+    """The library computes the NF4 levels on the host with its own normal-quantile routine;
+    they must equal the oracle's bit for bit (both round the same double values to fp32)."""
+    import oracle
+    assert np.array_equal(np.array(w4.w4_nf4_levels(), np.float32), oracle.nf4_levels())

@@ -93,7 +93,7 @@ def run_dense(M, N, K, group, mode, seed=0, grid=(1.0,), outlier_cols=8):
     return errs
 
 
-@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("group", [32, 64, 128, 256])
 @pytest.mark.parametrize("mode", ["asym", "sym"])
 def test_one_tile(group, mode):
     run_dense(128, 128, 256, group, mode)

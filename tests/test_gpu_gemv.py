@@ -75,10 +75,10 @@ def test_decode_sweep_full_size(K, N, M):
 
 
 @pytest.mark.parametrize("M", [1, 2, 3, 5, 9, 16])
-@pytest.mark.parametrize("group,mode", [(32, "sym"), (64, "asym"), (128, "asym"), (128, "sym")])
+@pytest.mark.parametrize("group,mode", [(32, "sym"), (64, "asym"), (128, "asym"), (128, "sym"), (256, "asym")])
 def test_ragged(M, group, mode):
     N = 77                              # not a multiple of 8
-    K = 320 if group < 128 else 384     # 320: not a multiple of the 128-wide unit
+    K = 320 if group < 128 else (384 if group == 128 else 768)  # 320, 384: not multiples of 256
     codes, scales, zeros = quantized("t3", K, N, group, mode, "twenty")
     x = synth.normal((M, K), 1.0, 4, 31 * M + group)
     check(codes, scales, zeros, group, mode, synth.bf16_bits(x))

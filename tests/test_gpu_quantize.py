@@ -66,12 +66,13 @@ def test_decode_small_full_compare():
     check(W, 128, "asym", synth.clip_grid_20())
 
 
-@pytest.mark.parametrize("group", [32, 64, 128])
+@pytest.mark.parametrize("group", [32, 64, 128, 256])
 @pytest.mark.parametrize("mode", ["sym", "asym"])
 @pytest.mark.parametrize("grid", ["one", "page", "twenty"])
 def test_groups_modes_grids(group, mode, grid):
     g = {"one": [1.0], "page": synth.clip_grid_page(), "twenty": synth.clip_grid_20()}[grid]
-    W = synth.student_t3_weight(77, 384, 0, 900 + group)   # ragged N, heavy tails
+    K = 384 if group < 256 else 768                         # 3 groups of 128, 3 of 256
+    W = synth.student_t3_weight(77, K, 0, 900 + group)     # ragged N, heavy tails
     check(W, group, mode, g)
 
 
@@ -88,9 +89,8 @@ def test_moe_expert_weights_g32():
     check(W, 32, "asym", [1.0], rows)
 
 
-def _edge_matrix():
+def _edge_matrix(K=128):
     rng = np.random.default_rng(5)
-    K = 128
     rows = []
     rows.append(np.zeros(K))                                   # all zero -> s = 1 guard
     rows.append(np.full(K, 0.37))                              # constant positive
@@ -108,9 +108,9 @@ def _edge_matrix():
 
 
 @pytest.mark.parametrize("mode", ["sym", "asym"])
-@pytest.mark.parametrize("group", [32, 128])
+@pytest.mark.parametrize("group", [32, 128, 256])
 def test_edge_blocks(mode, group):
-    check(_edge_matrix(), group, mode, synth.clip_grid_20())
+    check(_edge_matrix(max(128, group)), group, mode, synth.clip_grid_20())
 
 
 def test_tiny_shapes():

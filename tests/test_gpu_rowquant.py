@@ -75,7 +75,7 @@ def test_edge_rows():
     rows = [np.zeros(K), np.full(K, 3e-9), np.full(K, -5e-7), np.full(K, 448.0), np.full(K, 1e30),
             np.linspace(-1, 1, K), np.r_[np.ones(K - 1) * 1e-3, 2.0]]
     X = torch.tensor(np.array(rows), dtype=torch.float32).to(torch.bfloat16)
-    for g in (32, 64, 128):
+    for g in (32, 64, 128, 256):
         check(X, g)
     check(X, 0)
 
