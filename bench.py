@@ -59,6 +59,11 @@ NCU_TRAFFIC = {
 }
 
 
+# Warp instructions issued per weight by the quantizer (smsp__inst_executed.sum of one launch
+# over the weights it quantized), from one ncu capture, with the SHA-1 of its source file.
+QUANT_ISSUE = {}
+
+
 def source_sha1(rel):
     import hashlib
     with open(os.path.join(ROOT, rel), "rb") as f:
@@ -555,10 +560,13 @@ def moe_rows(args, dev, fp8_peak, rows):
     off = torch.empty(E + 1, dtype=torch.int32, device=dev)
     tor = torch.empty(R, dtype=torch.int32, device=dev)
     row_of = torch.empty(T, k, dtype=torch.int32, device=dev)
-    X8 = torch.empty(R, K, dtype=torch.uint8, device=dev)
+    route_ws = w4.alloc_moe_route_workspace(T, E, device=dev)
+    # group 32: the grouped GEMMs take the fp16 copy of the E4M3 activations (exact), which
+    # the two row quants write instead of the codes
+    X16 = torch.empty(R, K, dtype=torch.float16, device=dev)
     sa = torch.empty(R, dtype=torch.float32, device=dev)
     Ygu = torch.empty(R, 2 * H, dtype=torch.bfloat16, device=dev)
-    H8 = torch.empty(R, H, dtype=torch.uint8, device=dev)
+    H16 = torch.empty(R, H, dtype=torch.float16, device=dev)
     sh = torch.empty(R, dtype=torch.float32, device=dev)
     Yd = torch.empty(R, K, dtype=torch.bfloat16, device=dev)
     y = torch.empty(T, K, dtype=torch.bfloat16, device=dev)
@@ -574,19 +582,19 @@ def moe_rows(args, dev, fp8_peak, rows):
         packs[kind] = packed
 
     def route(i):
-        w4.w4_moe_route(logits, T, E, k, ex, gt, off, tor, row_of)
+        w4.w4_moe_route(logits, T, E, k, ex, gt, off, tor, row_of, route_ws)
 
     def dispatch(i):
-        w4.fp8_row_quant_gather(X, T, K, g, tor, R, X8, sa)
+        w4.fp8_row_quant_gather(X, T, K, g, tor, R, None, sa, x16=X16)
 
     def gate_up(i):
-        w4.w4a8_grouped_gemm(X8, sa, None, off, E, R, packs["gate_up"], 2 * H, K, g, "asym", Ygu)
+        w4.w4a8_grouped_gemm(None, sa, None, off, E, R, packs["gate_up"], 2 * H, K, g, "asym", Ygu, X16=X16)
 
     def swiglu(i):
-        w4.w4_moe_swiglu_quant(Ygu, R, H, g, H8, sh)
+        w4.w4_moe_swiglu_quant(Ygu, R, H, g, None, sh, x16=H16)
 
     def down(i):
-        w4.w4a8_grouped_gemm(H8, sh, None, off, E, R, packs["down"], K, H, g, "asym", Yd)
+        w4.w4a8_grouped_gemm(None, sh, None, off, E, R, packs["down"], K, H, g, "asym", Yd, X16=H16)
 
     def combine(i):
         w4.w4_moe_combine(Yd, K, R, row_of, gt, T, k, y)
@@ -638,10 +646,24 @@ def quantizer_full_set(args, dev):
             w4.w4_quantize(W, N, K, 128, "asym", grid, codes, scales, zeros, None)
 
     q(0)
-    ms = time_region(q, 1)
-    res = {"value": round(weights / (ms * 1e-3) / 1e9, 2), "unit": "G weights/s",
+    with Clocks(torch.cuda.current_device()) as clk:
+        ms = time_region(q, 1)
+    ck = clk.summary()
+    wps = weights / (ms * 1e-3)
+    res = {"value": round(wps / 1e9, 2), "unit": "G weights/s",
            "input_GBps": round(2 * weights / (ms * 1e-3) / 1e9, 1), "ms": round(ms, 2),
-           "weights": weights, "layers": n_layers, "bound": "alu"}
+           "weights": weights, "layers": n_layers, "bound": "alu", "clocks": ck}
+    # issue-rate roofline: warp instructions per weight (ncu) x weights/s against one warp
+    # instruction per clock on each of the 148 x 4 sub-partitions at the clock seen
+    rec = QUANT_ISSUE.get("w4_quantize g128 asym 20 ratios")
+    mhz = ck.get("sm_mhz") or ck.get("sm_max_mhz")
+    if rec and rec["sha1"] == source_sha1("bit_gemm_wise_b200/csrc/w4_quantize.cu") and mhz:
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        peak = sms * 4 * mhz * 1e6 / 1e12
+        ach = rec["inst_per_weight"] * wps / 1e12
+        res["roofline"] = {"bound": "alu", "achieved": round(ach, 3), "peak": round(peak, 3),
+                           "unit": "T warp-instructions/s", "frac": round(ach / peak, 4),
+                           "inst_per_weight": rec["inst_per_weight"]}
     del mats
     torch.cuda.empty_cache()
     return res

@@ -13,8 +13,10 @@
 // integer multiple of 2^-9: a 16-byte chunk's values are added exactly in fp32, the chunks'
 // sums as integers), rounded once to fp32; from them the optional group-sum operand of the
 // W4A8 GEMM is written: per row [hi(G) | lo(G) | hi(G) | 0 ...] in bf16, hi = bf16(G),
-// lo = bf16(G - hi), padded to a multiple of 32 columns. HBM-bound: 2 bytes read and 1
-// written per element. Compiled with -fmad=false.
+// lo = bf16(G - hi), padded to a multiple of 32 columns. Optionally the E4M3 values are also
+// (or only) written as binary16 -- the exact same values, in the operand type of the W4A8
+// GEMM's split-weight path (groups of 32 and 256). HBM-bound: 2 bytes read and 1 written
+// per element (+2 for the binary16 copy). Compiled with -fmad=false.
 #include "w4_common.cuh"
 #include "w4_layout.cuh"
 
@@ -44,6 +46,25 @@ __device__ __forceinline__ int e4m3x8_sum_times512(uint32_t o0, uint32_t o1) {
 }
 
 __device__ __forceinline__ uint16_t bf16_rn_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+
+// The 8 E4M3 values of (o.x: values 0-3, o.y: values 4-7) as binary16 (exact: E4M3 is a
+// subset of binary16), in order.
+__device__ __forceinline__ uint4 e4m3x8_to_f16x8(uint2 o) {
+    const uint32_t w[2] = {o.x, o.y};
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint16_t pair = (uint16_t)(w[i >> 1] >> (16 * (i & 1)));
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r[i]) : "h"(pair));
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// Store chunk c (8 values) of a row's outputs: the E4M3 codes and/or their binary16 values.
+__device__ __forceinline__ void store_chunk(uint8_t *X8, uint16_t *x16, int64_t m, int64_t K, int64_t c, uint2 o) {
+    if (X8) reinterpret_cast<uint2 *>(X8 + m * K)[c] = o;
+    if (x16) reinterpret_cast<uint4 *>(x16 + m * K)[c] = e4m3x8_to_f16x8(o);
+}
 
 // Group outputs of groups [j0, j0 + nj) of row m, whose sums are in sh[0 .. nj), written by
 // the whole block with consecutive threads on consecutive entries: the fp32 sums, and the
@@ -164,7 +185,8 @@ __device__ __forceinline__ float scale_of(float amax) { return __fdiv_rn(fmaxf(a
 
 template <int NC>  // 16-byte chunks per thread held in registers
 __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restrict__ X, int64_t K, int group,
-                                                        uint8_t *__restrict__ X8, float *__restrict__ row_scale,
+                                                        uint8_t *__restrict__ X8, uint16_t *__restrict__ x16,
+                                                        float *__restrict__ row_scale,
                                                         float *__restrict__ gsum, uint16_t *__restrict__ gop,
                                                         int64_t KZ, const int32_t *__restrict__ rows, int64_t msrc,
                                                         int *status) {
@@ -196,7 +218,6 @@ __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restri
     const float r = __frcp_rn(s);
     if (tid == 0) row_scale[m] = s;
 
-    uint2 *dst = reinterpret_cast<uint2 *>(X8 + m * K);
     const bool sums = gsum || gop;
     int isum[NC];
 #pragma unroll
@@ -205,7 +226,7 @@ __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restri
         isum[i] = 0;
         if (c < nchunk) {
             const uint2 o = special ? quantize8<true>(v[i], s, r) : quantize8<false>(v[i], s, r);
-            dst[c] = o;
+            store_chunk(X8, x16, m, K, c, o);
             if (sums) isum[i] = e4m3x8_sum_times512(o.x, o.y);
         }
     }
@@ -235,7 +256,7 @@ __global__ void __launch_bounds__(256) row_quant_kernel(const uint16_t *__restri
 // registers (chunk c of the row goes to lane c mod 32); every reduction is a warp operation.
 template <int NCW>
 __global__ void __launch_bounds__(256) row_quant_warp_kernel(const uint16_t *__restrict__ X, int64_t M, int64_t K,
-                                                             int group, uint8_t *__restrict__ X8,
+                                                             int group, uint8_t *__restrict__ X8, uint16_t *__restrict__ x16,
                                                              float *__restrict__ row_scale, float *__restrict__ gsum,
                                                              uint16_t *__restrict__ gop, int64_t KZ,
                                                              const int32_t *__restrict__ rows, int64_t msrc,
@@ -269,7 +290,6 @@ __global__ void __launch_bounds__(256) row_quant_warp_kernel(const uint16_t *__r
     const float r = __frcp_rn(s);
     if (lane == 0) row_scale[m] = s;
 
-    uint2 *dst = reinterpret_cast<uint2 *>(X8 + m * K);
     const bool sums = gsum || gop;
     int isum[NCW];
 #pragma unroll
@@ -278,7 +298,7 @@ __global__ void __launch_bounds__(256) row_quant_warp_kernel(const uint16_t *__r
         isum[i] = 0;
         if (c < nchunk) {
             const uint2 o = special ? quantize8<true>(v[i], s, r) : quantize8<false>(v[i], s, r);
-            dst[c] = o;
+            store_chunk(X8, x16, m, K, c, o);
             if (sums) isum[i] = e4m3x8_sum_times512(o.x, o.y);
         }
     }
@@ -305,7 +325,8 @@ __global__ void __launch_bounds__(256) row_quant_warp_kernel(const uint16_t *__r
 
 // Rows longer than the register budget: two passes over global memory.
 __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__restrict__ X, int64_t K, int group,
-                                                             uint8_t *__restrict__ X8, float *__restrict__ row_scale,
+                                                             uint8_t *__restrict__ X8, uint16_t *__restrict__ x16,
+                                                             float *__restrict__ row_scale,
                                                              float *__restrict__ gsum, uint16_t *__restrict__ gop,
                                                              int64_t KZ, const int32_t *__restrict__ rows, int64_t msrc,
                                                         int *status) {
@@ -329,7 +350,6 @@ __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__r
     const float s = scale_of(amax);
     const float r = __frcp_rn(s);
     if (tid == 0) row_scale[m] = s;
-    uint2 *dst = reinterpret_cast<uint2 *>(X8 + m * K);
     const int64_t iters = (nchunk + 255) / 256;
     for (int64_t i = 0; i < iters; ++i) {
         const int64_t c = tid + 256 * i;
@@ -338,7 +358,7 @@ __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__r
         if (live) {
             const uint4 v = srow >= 0 ? src[c] : make_uint4(0u, 0u, 0u, 0u);
             o = special ? quantize8<true>(v, s, r) : quantize8<false>(v, s, r);
-            dst[c] = o;
+            store_chunk(X8, x16, m, K, c, o);
         }
         if (gsum || gop) {
             // this round's groups: [j0, j0 + nj)
@@ -362,7 +382,8 @@ __global__ void __launch_bounds__(256) row_quant_long_kernel(const uint16_t *__r
 // the row's h held in registers (NC chunks of 8 per thread, H <= NC * 2048).
 template <int NC>
 __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t *__restrict__ Y, int64_t H, int group,
-                                                           uint8_t *__restrict__ X8, float *__restrict__ row_scale,
+                                                           uint8_t *__restrict__ X8, uint16_t *__restrict__ x16,
+                                                           float *__restrict__ row_scale,
                                                            uint16_t *__restrict__ gop, int64_t KZ) {
     __shared__ uint32_t red[8];
     __shared__ float gsh[NC * 256 * 8 / 32];
@@ -390,7 +411,6 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t *__res
     amax = block_max_f32(amax, red);
     const float s = scale_of(amax);
     if (tid == 0) row_scale[r] = s;
-    uint2 *dst = reinterpret_cast<uint2 *>(X8 + r * H);
     int isum[NC];
 #pragma unroll
     for (int i = 0; i < NC; ++i) {
@@ -401,7 +421,7 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t *__res
 #pragma unroll
             for (int t = 0; t < 4; ++t) p[t] = cvt_e4m3x2(__fdiv_rn(h[i][2 * t], s), __fdiv_rn(h[i][2 * t + 1], s));
             const uint2 o = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
-            dst[c] = o;
+            store_chunk(X8, x16, r, H, c, o);
             if (gop) isum[i] = e4m3x8_sum_times512(o.x, o.y);
         }
     }
@@ -435,8 +455,8 @@ W4_API int64_t w4a8_gsum_op_cols(int64_t K, int group) {
 
 // Output row m is the quantization of source row rows[m] (rows == nullptr: row m).
 static w4_status row_quant_launch(const void *X_bf16, const int32_t *rows, int64_t msrc, int64_t M, int64_t K,
-                                  int group, uint8_t *X_e4m3, float *row_scale, float *group_sums, uint16_t *gsum_op,
-                                  cudaStream_t stream) {
+                                  int group, uint8_t *X_e4m3, uint16_t *X_f16, float *row_scale, float *group_sums,
+                                  uint16_t *gsum_op, cudaStream_t stream) {
     int *st = device_status_ptr();
     const bool sums = group_sums || gsum_op;
     const int g = sums ? group : 32;
@@ -444,55 +464,59 @@ static w4_status row_quant_launch(const void *X_bf16, const int32_t *rows, int64
     const int64_t nchunk = K / 8;
     const uint16_t *X = static_cast<const uint16_t *>(X_bf16);
     const dim3 grid((unsigned)M), wgrid((unsigned)((M + 7) / 8));
-    if (nchunk <= 64) row_quant_warp_kernel<2><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
-    else if (nchunk <= 128) row_quant_warp_kernel<4><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
-    else if (nchunk <= 256) row_quant_warp_kernel<8><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
-    else if (nchunk <= 384) row_quant_warp_kernel<12><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
-    else if (nchunk <= 512) row_quant_warp_kernel<16><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
-    else if (nchunk <= 1024) row_quant_kernel<4><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
-    else if (nchunk <= 2048) row_quant_kernel<8><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
-    else row_quant_long_kernel<<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    if (nchunk <= 64) row_quant_warp_kernel<2><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, X_f16, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 128) row_quant_warp_kernel<4><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, X_f16, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 256) row_quant_warp_kernel<8><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, X_f16, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 384) row_quant_warp_kernel<12><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, X_f16, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 512) row_quant_warp_kernel<16><<<wgrid, 256, 0, stream>>>(X, M, K, g, X_e4m3, X_f16, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 1024) row_quant_kernel<4><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, X_f16, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else if (nchunk <= 2048) row_quant_kernel<8><<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, X_f16, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
+    else row_quant_long_kernel<<<grid, 256, 0, stream>>>(X, K, g, X_e4m3, X_f16, row_scale, group_sums, gsum_op, KZ, rows, msrc, st);
     return launch_status();
 }
 
 W4_API w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uint8_t *X_e4m3,
-                               float *row_scale, float *group_sums, uint16_t *gsum_op, cudaStream_t stream) {
-    if (!X_bf16 || !X_e4m3 || !row_scale) return W4_ERR_NULL;
+                               float *row_scale, float *group_sums, uint16_t *gsum_op, uint16_t *X_f16,
+                               cudaStream_t stream) {
+    if (!X_bf16 || !(X_e4m3 || X_f16) || !row_scale) return W4_ERR_NULL;
     if (M < 1 || M > 0x7fffffff || K < 16 || K % 16 != 0) return W4_ERR_SHAPE;
     const bool sums = group_sums || gsum_op;
     if (sums && (!valid_group(group) || K % group != 0)) return W4_ERR_GROUP;
-    if (!aligned16(X_bf16) || !aligned16(X_e4m3) || !aligned16(row_scale) || (group_sums && !aligned16(group_sums)) ||
-        (gsum_op && !aligned16(gsum_op)))
+    if (!aligned16(X_bf16) || !aligned16(X_e4m3) || !aligned16(X_f16) || !aligned16(row_scale) ||
+        (group_sums && !aligned16(group_sums)) || (gsum_op && !aligned16(gsum_op)))
         return W4_ERR_ALIGN;
-    return row_quant_launch(X_bf16, nullptr, M, M, K, group, X_e4m3, row_scale, group_sums, gsum_op, stream);
+    return row_quant_launch(X_bf16, nullptr, M, M, K, group, X_e4m3, X_f16, row_scale, group_sums, gsum_op, stream);
 }
 
 W4_API w4_status fp8_row_quant_gather(const void *X_bf16, int64_t M_src, int64_t K, int group,
                                       const int32_t *row_index, int64_t M, uint8_t *X_e4m3, float *row_scale,
-                                      float *group_sums, uint16_t *gsum_op, cudaStream_t stream) {
-    if (!X_bf16 || !row_index || !X_e4m3 || !row_scale) return W4_ERR_NULL;
+                                      float *group_sums, uint16_t *gsum_op, uint16_t *X_f16, cudaStream_t stream) {
+    if (!X_bf16 || !row_index || !(X_e4m3 || X_f16) || !row_scale) return W4_ERR_NULL;
     if (M < 1 || M > 0x7fffffff || M_src < 1 || M_src > 0x7fffffff || K < 16 || K % 16 != 0) return W4_ERR_SHAPE;
     const bool sums = group_sums || gsum_op;
     if (sums && (!valid_group(group) || K % group != 0)) return W4_ERR_GROUP;
-    if (!aligned16(X_bf16) || !aligned16(X_e4m3) || !aligned16(row_scale) || (group_sums && !aligned16(group_sums)) ||
-        (gsum_op && !aligned16(gsum_op)) || (reinterpret_cast<uintptr_t>(row_index) & 3))
+    if (!aligned16(X_bf16) || !aligned16(X_e4m3) || !aligned16(X_f16) || !aligned16(row_scale) ||
+        (group_sums && !aligned16(group_sums)) || (gsum_op && !aligned16(gsum_op)) ||
+        (reinterpret_cast<uintptr_t>(row_index) & 3))
         return W4_ERR_ALIGN;
-    return row_quant_launch(X_bf16, row_index, M_src, M, K, group, X_e4m3, row_scale, group_sums, gsum_op, stream);
+    return row_quant_launch(X_bf16, row_index, M_src, M, K, group, X_e4m3, X_f16, row_scale, group_sums, gsum_op,
+                            stream);
 }
 
 W4_API w4_status w4_moe_swiglu_quant(const void *gate_up_bf16, int64_t R, int64_t H, int group, uint8_t *X_e4m3,
-                                     float *row_scale, uint16_t *gsum_op, cudaStream_t stream) {
-    if (!gate_up_bf16 || !X_e4m3 || !row_scale) return W4_ERR_NULL;
+                                     float *row_scale, uint16_t *gsum_op, uint16_t *X_f16, cudaStream_t stream) {
+    if (!gate_up_bf16 || !(X_e4m3 || X_f16) || !row_scale) return W4_ERR_NULL;
     if (R < 1 || R > 0x7fffffff || H < 16 || H % 16 != 0 || H > 8 * 2048) return W4_ERR_SHAPE;
     if (gsum_op && (!valid_group(group) || H % group != 0)) return W4_ERR_GROUP;
-    if (!aligned16(gate_up_bf16) || !aligned16(X_e4m3) || !aligned16(row_scale) || (gsum_op && !aligned16(gsum_op)))
+    if (!aligned16(gate_up_bf16) || !aligned16(X_e4m3) || !aligned16(X_f16) || !aligned16(row_scale) ||
+        (gsum_op && !aligned16(gsum_op)))
         return W4_ERR_ALIGN;
     const int g = gsum_op ? group : 32;
     const int64_t KZ = gsum_op ? zop_cols(H / g) : 0;
     const int64_t nchunk = H / 8;
     const uint16_t *Y = static_cast<const uint16_t *>(gate_up_bf16);
-    if (nchunk <= 512) swiglu_quant_kernel<2><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, row_scale, gsum_op, KZ);
-    else if (nchunk <= 1024) swiglu_quant_kernel<4><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, row_scale, gsum_op, KZ);
-    else swiglu_quant_kernel<8><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, row_scale, gsum_op, KZ);
+    if (nchunk <= 512) swiglu_quant_kernel<2><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, X_f16, row_scale, gsum_op, KZ);
+    else if (nchunk <= 1024) swiglu_quant_kernel<4><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, X_f16, row_scale, gsum_op, KZ);
+    else swiglu_quant_kernel<8><<<(unsigned)R, 256, 0, stream>>>(Y, H, g, X_e4m3, X_f16, row_scale, gsum_op, KZ);
     return launch_status();
 }

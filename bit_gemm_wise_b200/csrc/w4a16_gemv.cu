@@ -78,6 +78,8 @@ struct Args {
     uint32_t off_sx, off_pp, off_red, off_ring, off_planes;
     int warpred;         // MT > 1 with spp a multiple of 32: partials reduced over the warp first
     int nred;            // partials per (row, m): spp, or spp / 32 with warpred
+    int rstr;            // words between the partials of consecutive (row, m) (nred, padded)
+    int lpr;             // lanes that add one (row, m)'s partials in the final reduction
     int out_fp32, pdl;
 };
 
@@ -138,7 +140,12 @@ template <int MT> struct Geo {
     static constexpr int NCH = KC / 32;       // 16-byte code chunks per slice
     static constexpr int WPS = KC / 8;        // code words per slice
     static constexpr int PW = 6 * WPS;        // plane words per slice and activation row
-    static constexpr int PSTRIDE = PW + 4;    // padded (conflict-free 16-byte loads)
+    // A slice's planes are stored load-major: the 16-byte load q (q = 0..5) of chunk c sits at
+    // word 4 (q NCH + c), so the loads a thread issues for its chunks in rotated order, with
+    // slices PSTRIDE words apart, fall in distinct banks for every 8 lanes when PSTRIDE / 4 is
+    // congruent to NCH modulo 8 (lanes 2r, 2r+1 share the rotation r when NCH = 4, lanes
+    // 4r..4r+3 when NCH = 2). With one chunk any odd PSTRIDE / 4 does.
+    static constexpr int PSTRIDE = NCH == 1 ? PW + 4 : PW + ((4 * NCH - PW % 32) % 32 + 32) % 32;
     static constexpr int RPT = MT == 1 ? 2 : 1;  // rows per thread and stage (registers allow two at MT = 1)
 };
 
@@ -304,10 +311,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
                     xs += __shfl_xor_sync(FULL, xs, 1);
                     xs += __shfl_xor_sync(FULL, xs, 2);
                     if (t < tasks) {
-                        uint32_t *dst = planes + tsl * PSTRIDE + wi * 6;
-                        reinterpret_cast<uint2 *>(dst)[0] = make_uint2(pw[0], pw[1]);
-                        reinterpret_cast<uint2 *>(dst)[1] = make_uint2(pw[2], pw[3]);
-                        reinterpret_cast<uint2 *>(dst)[2] = make_uint2(pw[4], pw[5]);
+                        // word u = 6 (wi % 4) + i of chunk wi / 4 goes to load u / 4, lane u % 4
+                        uint32_t *dst = planes + tsl * PSTRIDE + (wi >> 2) * 4;
+#pragma unroll
+                        for (int h = 0; h < 3; ++h) {
+                            const int u = (wi & 3) * 6 + 2 * h;
+                            *reinterpret_cast<uint2 *>(dst + (u >> 2) * 4 * NCH + (u & 3)) = make_uint2(pw[2 * h], pw[2 * h + 1]);
+                        }
                         if ((wi & 3) == 0) sx[(m * a.spp + tsl) * NCH + (wi >> 2)] = xs;
                         if (wi == 0)
                             pp[m * a.spp + tsl] =
@@ -323,7 +333,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
                 const int c = (j + rot) % NCH;
 #pragma unroll
                 for (int q = 0; q < 6; ++q) {  // 24 words of chunk c: 6 loads of 4
-                    const uint4 v = lds128(pb + (uint32_t)(c * 24 + q * 4) * 4u);
+                    const uint4 v = lds128(pb + (uint32_t)(q * 4 * NCH + c * 4) * 4u);
                     const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int r = 0; r < 4; ++r) xp[m][j][(q * 4 + r) / 6][(q * 4 + r) % 6] = vv[r];
@@ -439,7 +449,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
                         if (!live[i]) continue;
                         const uint32_t rl = (uint32_t)(s * SR + slot + i * a.nslot);
 #pragma unroll
-                        for (int m = 0; m < MT; ++m) red[(rl * MT + m) * (uint32_t)a.nred + sl] = yv[i][m];
+                        for (int m = 0; m < MT; ++m) red[(rl * MT + m) * (uint32_t)a.rstr + sl] = yv[i][m];
                     }
                 }
             }
@@ -451,7 +461,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
                     const float r = warp_transpose_sum<MT>(yv[i], lane);
                     const int rl = s * SR + slot + i * a.nslot;
                     if (slot < a.nslot && rl < rows && (lane & (32 / MT - 1)) == 0)
-                        red[((uint32_t)rl * MT + lane / (32 / MT)) * (uint32_t)a.nred + sl / 32] = r;
+                        red[((uint32_t)rl * MT + lane / (32 / MT)) * (uint32_t)a.rstr + sl / 32] = r;
                 }
             }
             __syncwarp();
@@ -459,23 +469,29 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
         }
         if (!ok) *(volatile int *)abort_flag = 1;
 
-        // (4) row sums in a fixed order: one warp per (row, m)
+        // (4) row sums in a fixed order: lpr lanes per (row, m), each adding every lpr-th
+        // partial in turn, then a butterfly over the lpr lanes
         named_bar_sync(1, NCT);
         const bool aborted = *(volatile int *)abort_flag != 0;
         float *outp = nullptr;
         if (a.kparts > 1) outp = a.ws_part + (size_t)kp * a.M * a.N;
-        for (int o = warp; o < rows * MT; o += NCW) {
-            const int rl = o / MT, m = o - rl * MT;
-            float acc = 0.0f;
+        {
+            const int lpr = a.lpr, opw = 32 / lpr;  // outputs per warp
             const int nv = a.warpred ? (nsl + 31) / 32 : nsl;
-            for (int i = lane; i < nv; i += 32) acc += red[(size_t)o * a.nred + i];
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(FULL, acc, off);
-            const int64_t n = row0 + rl;
-            if (lane == 0 && m0 + m < a.M && !aborted) {
-                if (outp) outp[(int64_t)(m0 + m) * a.N + n] = acc;
-                else if (a.out_fp32) static_cast<float *>(a.y)[(int64_t)(m0 + m) * a.N + n] = acc;
-                else static_cast<__nv_bfloat16 *>(a.y)[(int64_t)(m0 + m) * a.N + n] = __float2bfloat16_rn(acc);
+            const int j = lane & (lpr - 1);
+            for (int ob = warp * opw; ob < rows * MT; ob += NCW * opw) {
+                const int o = ob + lane / lpr;
+                float acc = 0.0f;
+                if (o < rows * MT)
+                    for (int i = j; i < nv; i += lpr) acc += red[(size_t)o * a.rstr + i];
+                for (int off = lpr >> 1; off >= 1; off >>= 1) acc += __shfl_xor_sync(FULL, acc, off);
+                const int rl = o / MT, m = o - rl * MT;
+                const int64_t n = row0 + rl;
+                if (j == 0 && o < rows * MT && m0 + m < a.M && !aborted) {
+                    if (outp) outp[(int64_t)(m0 + m) * a.N + n] = acc;
+                    else if (a.out_fp32) static_cast<float *>(a.y)[(int64_t)(m0 + m) * a.N + n] = acc;
+                    else static_cast<__nv_bfloat16 *>(a.y)[(int64_t)(m0 + m) * a.N + n] = __float2bfloat16_rn(acc);
+                }
             }
         }
         if (a.kparts > 1) {
@@ -561,18 +577,25 @@ static bool make_plan_parts(Plan &p, int64_t M, int64_t N, int64_t K, int g, int
     a.SB = (uint32_t)(a.nslot * a.rpt) * a.RSp;
     a.warpred = (MT > 1 && a.spp % 32 == 0) ? 1 : 0;
     a.nred = a.warpred ? a.spp / 32 : a.spp;
-    // rows per block: N spread over the SMs, capped by the row-partial buffer
+    // rows per block: N spread over the SMs, capped by the row-partial buffer (sized for the
+    // widest padding of a (row, m)'s partials, nred + 31 words)
     int64_t nrb = S < N ? S : N;
     int64_t rpc = (N + nrb - 1) / nrb;
-    const int64_t rpc_cap = RED_BUDGET / ((int64_t)MT * a.nred * 4);
+    const int64_t rpc_cap = RED_BUDGET / ((int64_t)MT * (a.nred + 31) * 4);
     if (rpc_cap < 1) return false;
     if (rpc > rpc_cap) rpc = rpc_cap;
     a.rpc = (int)rpc;
+    // final reduction: as many lanes per (row, m) as the consumer threads allow (a power of
+    // two up to 32); partials of consecutive (row, m) are rstr = lpr (mod 32) words apart, so
+    // a warp's loads hit distinct banks
+    a.lpr = 32;
+    while (a.lpr > 1 && (int64_t)rpc * MT * a.lpr > NCT) a.lpr >>= 1;
+    a.rstr = a.lpr == 32 ? a.nred : a.nred + ((a.lpr - a.nred % 32) % 32 + 32) % 32;
     a.nrb = (int)((N + rpc - 1) / rpc);
     a.off_sx = 512;
     a.off_pp = a.off_sx + (sx_bytes + 15) / 16 * 16;
     a.off_red = a.off_pp + (pp_bytes + 15) / 16 * 16;
-    a.off_ring = a.off_red + (uint32_t)((rpc * MT * a.nred * 4 + 15) / 16 * 16);
+    a.off_ring = a.off_red + (uint32_t)((rpc * MT * a.rstr * 4 + 15) / 16 * 16);
     const int64_t avail = (int64_t)SMEM_MAX - a.off_ring - SLACK;
     int NS = (int)(avail / a.SB);
     if (NS > MAX_STAGES) NS = MAX_STAGES;

@@ -780,9 +780,11 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
 // the MMA itself. For such groups this kernel keeps the whole K in one TMEM accumulator
 // instead: every weight is dequantized exactly and split into two fp16 parts,
 //   w = (q - z) s,  hi = fp16(w),  lo = fp16(w - hi),  w = hi + lo,
-// and the E4M3 activations become fp16 (exact: every E4M3 value is an fp16 value). kind::f16
-// MMAs accumulate A_hi B + A_lo B in fp32, so the tensor core sees the dequantized operands
-// of the method, as in the promoted path, and nothing is read back until the tile is done.
+// and the E4M3 activations arrive as fp16 (exact: every E4M3 value is an fp16 value; the row
+// quant writes that copy, so no tile of activations is converted again for every weight
+// tile). kind::f16 MMAs accumulate A_hi B + A_lo B in fp32, so the tensor core sees the
+// dequantized operands of the method, as in the promoted path, and nothing is read back
+// until the tile is done.
 // Exactness: q - z is an fp16 integer (1024 + q minus 1024 + z) for |z| < 1024, s is the
 // stored fp16 scale, so w has at most 11 + 11 significant bits; hi keeps the leading 11 and
 // the fp16 FMA forms lo = w - hi exactly (it is a multiple of 2^-24, the smallest fp16
@@ -792,32 +794,31 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
 // two fp16 MMAs per K step, a quarter of the FP8 rate, with no per-group readback.
 //
 // Warp roles (512 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps 4-7
-// epilogue (one TMEM lane quarter each, all 256 columns), warps 8-15 expansion. Two rings:
-// raw stages (packed codes + E4M3 activations, by TMA) and expanded stages (fp16 A_hi, A_lo
-// and B in the 128-byte-swizzled K-major layout the MMA reads). Two TMEM accumulators
-// alternate between tiles, so the epilogue of one tile overlaps the MMAs of the next.
+// epilogue (one TMEM lane quarter each, all 256 columns), warps 8-15 expansion. One ring of
+// stages, each holding the packed codes and the fp16 activations (B, 128-byte swizzle,
+// K-major) loaded by TMA, and the expanded A_hi and A_lo the expansion warps write in the
+// layout the MMA reads: TMA -> full -> expansion -> exp_full -> MMA -> empty -> TMA. Two
+// TMEM accumulators alternate between tiles, so the epilogue of one tile overlaps the MMAs
+// of the next.
 namespace f16p {
 
 constexpr int BK = 64;                        // k per stage (one 128-byte swizzle row of fp16)
-constexpr int RAW_STAGES = 4;
-constexpr int EXP_STAGES = 2;
+constexpr int STAGES = 3;
 constexpr int EXW = 8;                        // expansion warps
 constexpr uint32_t RC_BYTES = BM * BK / 2;    // packed codes of a stage (4 KB)
-constexpr uint32_t RA_BYTES = BN * BK;        // E4M3 activations of a stage (16 KB)
-constexpr uint32_t RAW_BYTES = RC_BYTES + RA_BYTES;
-constexpr uint32_t AH_BYTES = BM * BK * 2;    // one fp16 weight part (16 KB)
 constexpr uint32_t B_BYTES = BN * BK * 2;     // fp16 activations (32 KB)
-constexpr uint32_t EXP_BYTES = 2 * AH_BYTES + B_BYTES;
-constexpr uint32_t SMEM_BYTES = RAW_STAGES * RAW_BYTES + EXP_STAGES * EXP_BYTES + 1024 + 1024;
-static_assert(RAW_BYTES % 1024 == 0 && EXP_BYTES % 1024 == 0 && AH_BYTES % 1024 == 0, "swizzle atoms stay aligned");
+constexpr uint32_t AH_BYTES = BM * BK * 2;    // one fp16 weight part (16 KB)
+constexpr uint32_t OFF_B = RC_BYTES, OFF_AH = OFF_B + B_BYTES, OFF_AL = OFF_AH + AH_BYTES;
+constexpr uint32_t STAGE_BYTES = OFF_AL + AH_BYTES;
+constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
+static_assert(RC_BYTES % 1024 == 0 && B_BYTES % 1024 == 0 && AH_BYTES % 1024 == 0, "swizzle atoms stay aligned");
 
 struct Smem {
-    uint64_t raw_full[RAW_STAGES];   // TMA bytes landed
-    uint64_t raw_empty[RAW_STAGES];  // expansion read the stage (one arrival per expansion warp)
-    uint64_t exp_full[EXP_STAGES];   // expansion wrote the operands (one arrival per expansion warp)
-    uint64_t exp_empty[EXP_STAGES];  // the MMAs reading them completed (tcgen05.commit)
-    uint64_t acc_full[NBUF];         // a tile's accumulator is complete
-    uint64_t acc_empty[NBUF];        // the epilogue has read it (one arrival per epilogue warp)
+    uint64_t full[STAGES];       // TMA bytes (codes + activations) landed
+    uint64_t exp_full[STAGES];   // expansion wrote A_hi, A_lo (one arrival per expansion warp)
+    uint64_t empty[STAGES];      // the MMAs reading the stage completed (tcgen05.commit)
+    uint64_t acc_full[NBUF];     // a tile's accumulator is complete
+    uint64_t acc_empty[NBUF];    // the epilogue has read it (one arrival per epilogue warp)
     uint32_t tmem_base;
     int abort;
 };
@@ -836,13 +837,6 @@ __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint32_t a_lo, uint32_t
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cast<__half2 *>(&v); }
-
-// two E4M3 bytes (low 16 bits of v) -> fp16x2, exact
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
-    uint32_t r;
-    asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n" : "=r"(r) : "r"(v));
-    return r;
-}
 
 __device__ __forceinline__ bool wait_f(uint64_t *bar, uint32_t parity, Smem *sm, int *status) {
     return mbar_wait_abortable<true>(bar, parity, &sm->abort, status, kWaitNs);
@@ -869,21 +863,16 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
                                                                    const Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *raw = base;                                     // RAW_STAGES x (codes | E4M3 activations)
-    uint8_t *ex = base + RAW_STAGES * RAW_BYTES;             // EXP_STAGES x (A_hi | A_lo | B)
-    Smem *sm = reinterpret_cast<Smem *>(ex + EXP_STAGES * EXP_BYTES);
+    Smem *sm = reinterpret_cast<Smem *>(base + STAGES * STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = (int)(a.Kpad / BK);
     const int64_t ntiles = (int64_t)a.MTU * a.NT;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < RAW_STAGES; ++s) {
-            mbar_init(&sm->raw_full[s], 1);
-            mbar_init(&sm->raw_empty[s], EXW);
-        }
-        for (int s = 0; s < EXP_STAGES; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm->full[s], 1);
             mbar_init(&sm->exp_full[s], EXW);
-            mbar_init(&sm->exp_empty[s], 1);
+            mbar_init(&sm->empty[s], 1);
         }
         for (int b = 0; b < NBUF; ++b) {
             mbar_init(&sm->acc_full[b], 1);
@@ -906,33 +895,33 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
-            RingN<RAW_STAGES> r;
+            RingN<STAGES> r;
             int64_t uses = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 Tile T;
                 if (!locate_tile(a, t, T)) continue;
                 for (int s = 0; s < KT; ++s, r.next(), ++uses) {
-                    if (!wait_f(&sm->raw_empty[r.slot], r.phase ^ 1u, sm, a.status)) { ok = false; break; }
-                    uint8_t *dst = raw + r.slot * RAW_BYTES;
-                    mbar_arrive_expect_tx(&sm->raw_full[r.slot], RAW_BYTES);
-                    tma_load_3d(dst, &tm_codes, s * (BK / 2), (int)T.n0, T.e, &sm->raw_full[r.slot]);
-                    tma_load_2d(dst + RC_BYTES, &tm_act, s * BK, (int)T.row0, &sm->raw_full[r.slot]);
+                    if (!wait_f(&sm->empty[r.slot], r.phase ^ 1u, sm, a.status)) { ok = false; break; }
+                    uint8_t *dst = base + r.slot * STAGE_BYTES;
+                    mbar_arrive_expect_tx(&sm->full[r.slot], RC_BYTES + B_BYTES);
+                    tma_load_3d(dst, &tm_codes, s * (BK / 2), (int)T.n0, T.e, &sm->full[r.slot]);
+                    tma_load_2d(dst + OFF_B, &tm_act, s * BK, (int)T.row0, &sm->full[r.slot]);
                 }
             }
             // no copy may land after the CTA exits: wait for the last uses' bytes
-            for (int64_t u = uses > RAW_STAGES ? uses - RAW_STAGES : 0; u < uses; ++u)
-                (void)mbar_wait_bounded(&sm->raw_full[u % RAW_STAGES], (uint32_t)(u / RAW_STAGES) & 1, a.status);
+            for (int64_t u = uses > STAGES ? uses - STAGES : 0; u < uses; ++u)
+                (void)mbar_wait_bounded(&sm->full[u % STAGES], (uint32_t)(u / STAGES) & 1, a.status);
         }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
-            RingN<EXP_STAGES> r;
+            RingN<STAGES> r;
             uint32_t tiles_done = 0;
             int64_t uses = 0;
             bool ok = true;
-            const uint32_t exLo0 = desc_lo(smem_addr(ex));
+            const uint32_t lo0 = desc_lo(smem_addr(base));
             for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
                 Tile T;
                 if (!locate_tile(a, t, T)) continue;
@@ -943,14 +932,14 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
                 for (int s = 0; s < KT; ++s, r.next()) {
                     if (!wait_f(&sm->exp_full[r.slot], r.phase, sm, a.status)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t hLo = exLo0 + (uint32_t)r.slot * (EXP_BYTES >> 4);
-                    const uint32_t lLo = hLo + (AH_BYTES >> 4), bLo = hLo + (2 * AH_BYTES >> 4);
+                    const uint32_t st = lo0 + (uint32_t)r.slot * (STAGE_BYTES >> 4);
+                    const uint32_t bLo = st + (OFF_B >> 4), hLo = st + (OFF_AH >> 4), lLo = st + (OFF_AL >> 4);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {  // K = 16 per fp16 MMA: 32 bytes
                         mma_f16(d, hLo + kk * 2, bLo + kk * 2, (s > 0 || kk > 0) ? 1u : 0u);
                         mma_f16(d, lLo + kk * 2, bLo + kk * 2, 1u);
                     }
-                    mma_commit(&sm->exp_empty[r.slot]);
+                    mma_commit(&sm->empty[r.slot]);
                     ++uses;
                 }
                 if (!ok) break;
@@ -958,8 +947,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
                 ++tiles_done;
             }
             // no commit may arrive after the CTA exits: wait for the last stages' completions
-            for (int64_t u = uses > EXP_STAGES ? uses - EXP_STAGES : 0; u < uses; ++u)
-                (void)mbar_wait_bounded(&sm->exp_empty[u % EXP_STAGES], (uint32_t)(u / EXP_STAGES) & 1, a.status);
+            for (int64_t u = uses > STAGES ? uses - STAGES : 0; u < uses; ++u)
+                (void)mbar_wait_bounded(&sm->empty[u % STAGES], (uint32_t)(u / STAGES) & 1, a.status);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 8) {
@@ -1032,8 +1021,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
         // ------------------------------------------------ expansion (8 warps, 256 threads)
         const int et = threadIdx.x - 256;        // 0..255
         const int wr = et >> 1, wh = et & 1;      // weight row, half of the stage's 64 k
-        RingN<RAW_STAGES> rr;
-        RingN<EXP_STAGES> re;
+        RingN<STAGES> r;
         bool ok = true;
         const __half2 h1024 = __float2half2_rn(1024.0f);
         const uint32_t magic = 0x64646464u;      // high bytes of fp16 1024 + q
@@ -1046,86 +1034,62 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
             // this thread's scale entry for stage s is loaded one stage ahead (it does not
             // depend on the ring): k = 64 s + 32 wh + 0..31 lies in group (64 s + 32 wh) / g
             uint32_t ent_next = scales[(int64_t)(wh * 32 / a.g) * a.Npad + n];
-            for (int s = 0; s < KT; ++s, rr.next(), re.next()) {
+            for (int s = 0; s < KT; ++s, r.next()) {
                 const uint32_t ent = ent_next;
                 if (s + 1 < KT) ent_next = scales[((int64_t)(s + 1) * BK + wh * 32) / a.g * a.Npad + n];
-                if (!warp_wait_f(&sm->raw_full[rr.slot], rr.phase, sm, a.status)) { ok = false; break; }
-                if (!warp_wait_f(&sm->exp_empty[re.slot], re.phase ^ 1u, sm, a.status)) { ok = false; break; }
-                const uint8_t *src = raw + rr.slot * RAW_BYTES;
-                uint8_t *dst = ex + re.slot * EXP_BYTES;
-                {
-                    const int z = (int)(int16_t)(ent >> 16);
-                    const __half2 s2 = __half2half2(__ushort_as_half((unsigned short)(ent & 0xFFFFu)));
-                    const uint4 cw = *reinterpret_cast<const uint4 *>(src + wr * 32 + wh * 16);
-                    const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
-                    uint32_t hi[16], lo[16];
-                    if (z > -1024 && z < 1024) {
-                        const __half2 c0 = __hadd2(h1024, __float2half2_rn((float)z));
+                // the stage was refilled only after the MMAs that read its previous A_hi and
+                // A_lo completed, so once its TMA bytes landed both buffers are free
+                if (!warp_wait_f(&sm->full[r.slot], r.phase, sm, a.status)) { ok = false; break; }
+                uint8_t *stg = base + r.slot * STAGE_BYTES;
+                const int z = (int)(int16_t)(ent >> 16);
+                const __half2 s2 = __half2half2(__ushort_as_half((unsigned short)(ent & 0xFFFFu)));
+                const uint4 cw = *reinterpret_cast<const uint4 *>(stg + wr * 32 + wh * 16);
+                const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
+                uint32_t hi[16], lo[16];
+                if (z > -1024 && z < 1024) {
+                    const __half2 c0 = __hadd2(h1024, __float2half2_rn((float)z));
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t bl = wv[i] & 0x0F0F0F0Fu, bh = (wv[i] >> 4) & 0x0F0F0F0Fu;
-                            const uint32_t p[4] = {__byte_perm(bl, magic, 0x4140), __byte_perm(bl, magic, 0x4342),
-                                                   __byte_perm(bh, magic, 0x4140), __byte_perm(bh, magic, 0x4342)};
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t bl = wv[i] & 0x0F0F0F0Fu, bh = (wv[i] >> 4) & 0x0F0F0F0Fu;
+                        const uint32_t p[4] = {__byte_perm(bl, magic, 0x4140), __byte_perm(bl, magic, 0x4342),
+                                               __byte_perm(bh, magic, 0x4140), __byte_perm(bh, magic, 0x4342)};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const __half2 cc = __hsub2(bits_h2(p[e]), c0);
-                                const __half2 h = __hmul2(cc, s2);
-                                hi[4 * i + e] = h2_bits(h);
-                                lo[4 * i + e] = h2_bits(__hfma2(cc, s2, __hneg2(h)));
-                            }
-                        }
-                    } else {
-                        // zero point beyond fp16's exact integers around 1024: q - z in fp32
-                        const float sf = __half2float(__ushort_as_half((unsigned short)(ent & 0xFFFFu)));
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                // nibble slots: k0 + p/2 + 4 (p % 2) holds slot p
-                                const int k0 = 2 * e;  // weights k0 and k0 + 1 of this word
-                                const int p0 = (k0 & 3) * 2 + (k0 >> 2), p1 = ((k0 + 1) & 3) * 2 + ((k0 + 1) >> 2);
-                                const float q0 = (float)((wv[i] >> (4 * p0)) & 0xFu), q1 = (float)((wv[i] >> (4 * p1)) & 0xFu);
-                                const __half2 cc = __floats2half2_rn(q0 - (float)z, q1 - (float)z);
-                                const __half2 h = __hmul2(cc, __float2half2_rn(sf));
-                                hi[4 * i + e] = h2_bits(h);
-                                lo[4 * i + e] = h2_bits(__hfma2(cc, __float2half2_rn(sf), __hneg2(h)));
-                            }
+                        for (int e = 0; e < 4; ++e) {
+                            const __half2 cc = __hsub2(bits_h2(p[e]), c0);
+                            const __half2 h = __hmul2(cc, s2);
+                            hi[4 * i + e] = h2_bits(h);
+                            lo[4 * i + e] = h2_bits(__hfma2(cc, s2, __hneg2(h)));
                         }
                     }
-                    // 16-byte chunks 4 wh .. 4 wh + 3 of row wr (8 k each), 128-byte swizzle
-                    uint8_t *ah = dst + wr * 128, *al = dst + AH_BYTES + wr * 128;
+                } else {
+                    // zero point beyond fp16's exact integers around 1024: q - z in fp32
+                    const float sf = __half2float(__ushort_as_half((unsigned short)(ent & 0xFFFFu)));
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int pc = (4 * wh + c) ^ (wr & 7);
-                        *reinterpret_cast<uint4 *>(ah + pc * 16) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
-                        *reinterpret_cast<uint4 *>(al + pc * 16) = make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+                    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            // nibble slots: k0 + p/2 + 4 (p % 2) holds slot p
+                            const int k0 = 2 * e;  // weights k0 and k0 + 1 of this word
+                            const int p0 = (k0 & 3) * 2 + (k0 >> 2), p1 = ((k0 + 1) & 3) * 2 + ((k0 + 1) >> 2);
+                            const float q0 = (float)((wv[i] >> (4 * p0)) & 0xFu), q1 = (float)((wv[i] >> (4 * p1)) & 0xFu);
+                            const __half2 cc = __floats2half2_rn(q0 - (float)z, q1 - (float)z);
+                            const __half2 h = __hmul2(cc, __float2half2_rn(sf));
+                            hi[4 * i + e] = h2_bits(h);
+                            lo[4 * i + e] = h2_bits(__hfma2(cc, __float2half2_rn(sf), __hneg2(h)));
+                        }
                     }
                 }
-                // activations: token row et, 64 E4M3 bytes (64-byte swizzle: 16-byte chunk c of
-                // row r at r*64 + 16*(c ^ ((r >> 1) & 3))) -> 64 fp16 (128-byte swizzle)
-                {
-                    const uint8_t *ar = src + RC_BYTES + et * 64;
-                    uint8_t *br = dst + 2 * AH_BYTES + et * 128;
+                // 16-byte chunks 4 wh .. 4 wh + 3 of row wr (8 k each), 128-byte swizzle
+                uint8_t *ah = stg + OFF_AH + wr * 128, *al = stg + OFF_AL + wr * 128;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(ar + 16 * (c ^ ((et >> 1) & 3)));
-                        const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-                        uint32_t o[8];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            o[2 * i] = e4m3x2_to_f16x2(vv[i]);
-                            o[2 * i + 1] = e4m3x2_to_f16x2(vv[i] >> 16);
-                        }
-                        *reinterpret_cast<uint4 *>(br + ((2 * c) ^ (et & 7)) * 16) = make_uint4(o[0], o[1], o[2], o[3]);
-                        *reinterpret_cast<uint4 *>(br + ((2 * c + 1) ^ (et & 7)) * 16) = make_uint4(o[4], o[5], o[6], o[7]);
-                    }
+                for (int c = 0; c < 4; ++c) {
+                    const int pc = (4 * wh + c) ^ (wr & 7);
+                    *reinterpret_cast<uint4 *>(ah + pc * 16) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                    *reinterpret_cast<uint4 *>(al + pc * 16) = make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&sm->raw_empty[rr.slot]);
-                    mbar_arrive(&sm->exp_full[re.slot]);
-                }
+                if (lane == 0) mbar_arrive(&sm->exp_full[r.slot]);
             }
         }
     }
@@ -1231,8 +1195,9 @@ static int64_t dense_tiles(int64_t M, int64_t N, int64_t K, int group) {
     return ((M + BN - 1) / BN) * (L.Npad / BM);
 }
 
-// Groups of 32: the split-weight fp16 kernel (no per-group promotion, no zero-point operand).
-static w4_status launch_f16(const uint8_t *X8, const float *row_scale, const int32_t *offsets, int E, int64_t M,
+// Groups of 32 and 256: the split-weight fp16 kernel (no per-group promotion, no zero-point
+// operand); the activations are the fp16 copy of the E4M3 values.
+static w4_status launch_f16(const uint16_t *X16, const float *row_scale, const int32_t *offsets, int E, int64_t M,
                             const void *packed, int64_t N, int64_t K, int group, void *Y, int out_fp32,
                             cudaStream_t stream) {
     EncodeTiledFn enc = encode_fn();
@@ -1251,12 +1216,14 @@ static w4_status launch_f16(const uint8_t *X8, const float *row_scale, const int
             return W4_ERR_CUDA;
     }
     {
+        // fp16 [M][K]: 64 k (128 bytes) x 256 rows per stage, 128-byte swizzle (the MMA's
+        // K-major layout); rows past M and k past K read as zero
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-        const cuuint64_t strides[1] = {(cuuint64_t)K};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
         const cuuint32_t box[2] = {f16p::BK, BN};
         const cuuint32_t es[2] = {1, 1};
-        if (enc(&tm_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(X8), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        if (enc(&tm_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t *>(X16), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4_ERR_CUDA;
     }
@@ -1290,11 +1257,11 @@ static w4_status launch_f16(const uint8_t *X8, const float *row_scale, const int
     return launch_status();
 }
 
-static w4_status launch(const uint8_t *X8, const float *row_scale, const uint16_t *gop, const int32_t *offsets, int E,
-                        int64_t M, const void *packed, int64_t N, int64_t K, int group, void *Y, int out_fp32,
-                        void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+static w4_status launch(const uint8_t *X8, const uint16_t *X16, const float *row_scale, const uint16_t *gop,
+                        const int32_t *offsets, int E, int64_t M, const void *packed, int64_t N, int64_t K, int group,
+                        void *Y, int out_fp32, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     if (group == 32 || group == 256)
-        return launch_f16(X8, row_scale, offsets, E, M, packed, N, K, group, Y, out_fp32, stream);
+        return launch_f16(X16, row_scale, offsets, E, M, packed, N, K, group, Y, out_fp32, stream);
     EncodeTiledFn enc = encode_fn();
     if (!enc) return W4_ERR_CUDA;
     const GemmLayout L = gemm_layout(N, K, group);
@@ -1435,33 +1402,42 @@ W4_API w4_status w4a8_gemm_split_segment(int64_t R, int64_t KT, int64_t PS, int6
     return W4_OK;
 }
 
-W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op, int64_t M,
-                           const void *packed, int64_t N, int64_t K, int group, int mode, void *Y, int out_fp32,
-                           void *workspace, size_t workspace_bytes, cudaStream_t stream) {
-    if (!X_e4m3 || !row_scale || !packed || !Y || (!gsum_op && (group == 64 || group == 128))) return W4_ERR_NULL;
+// The activation operands a group size needs: E4M3 codes and the group-sum operand for the
+// promoted path (64, 128), the binary16 copy for the split-weight path (32, 256).
+static bool operands_given(int group, const uint8_t *X8, const uint16_t *X16, const uint16_t *gop) {
+    if (group == 32 || group == 256) return X16 != nullptr;
+    return X8 && gop;
+}
+
+W4_API w4_status w4a8_gemm(const uint8_t *X_e4m3, const uint16_t *X_f16, const float *row_scale,
+                           const uint16_t *gsum_op, int64_t M, const void *packed, int64_t N, int64_t K, int group,
+                           int mode, void *Y, int out_fp32, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    if (!row_scale || !packed || !Y || !operands_given(group, X_e4m3, X_f16, gsum_op)) return W4_ERR_NULL;
     if (!valid_mode(mode) || (out_fp32 != 0 && out_fp32 != 1)) return W4_ERR_ARG;
     if (!gemm_shape_ok(M, N, K)) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
-    if (!aligned16(X_e4m3) || !aligned16(row_scale) || !aligned16(gsum_op) || !aligned16(packed) || !aligned16(Y) ||
-        !aligned16(workspace))
+    if (!aligned16(X_e4m3) || !aligned16(X_f16) || !aligned16(row_scale) || !aligned16(gsum_op) ||
+        !aligned16(packed) || !aligned16(Y) || !aligned16(workspace))
         return W4_ERR_ALIGN;
-    return gemm::launch(X_e4m3, row_scale, gsum_op, nullptr, 1, M, packed, N, K, group, Y, out_fp32, workspace,
-                        workspace_bytes, stream);
+    return gemm::launch(X_e4m3, X_f16, row_scale, gsum_op, nullptr, 1, M, packed, N, K, group, Y, out_fp32,
+                        workspace, workspace_bytes, stream);
 }
 
-W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op,
-                                   const int32_t *expert_row_offsets, int E, int64_t M_total, const void *packed,
-                                   int64_t N, int64_t K, int group, int mode, void *Y, cudaStream_t stream) {
-    if (!X_e4m3 || !row_scale || !expert_row_offsets || !packed || !Y || (!gsum_op && (group == 64 || group == 128)))
+W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const uint16_t *X_f16, const float *row_scale,
+                                   const uint16_t *gsum_op, const int32_t *expert_row_offsets, int E,
+                                   int64_t M_total, const void *packed, int64_t N, int64_t K, int group, int mode,
+                                   void *Y, cudaStream_t stream) {
+    if (!row_scale || !expert_row_offsets || !packed || !Y || !operands_given(group, X_e4m3, X_f16, gsum_op))
         return W4_ERR_NULL;
     if (!valid_mode(mode)) return W4_ERR_ARG;
     if (E < 1 || E > 1024 || M_total < 1 || M_total > 0x7fffffffLL || N < 1 || N > 0x7fffffffLL || K < 128 ||
         K % 32 != 0 || K > (1LL << 24))
         return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
-    if (!aligned16(X_e4m3) || !aligned16(row_scale) || !aligned16(gsum_op) || !aligned16(packed) ||
-        !aligned16(Y) || (reinterpret_cast<uintptr_t>(expert_row_offsets) & 3))
+    if (!aligned16(X_e4m3) || !aligned16(X_f16) || !aligned16(row_scale) || !aligned16(gsum_op) ||
+        !aligned16(packed) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(expert_row_offsets) & 3))
         return W4_ERR_ALIGN;
-    return gemm::launch(X_e4m3, row_scale, gsum_op, expert_row_offsets, E, M_total, packed, N, K, group, Y, 0,
+    return gemm::launch(X_e4m3, X_f16, row_scale, gsum_op, expert_row_offsets, E, M_total, packed, N, K, group, Y, 0,
                         nullptr, 0, stream);
 }

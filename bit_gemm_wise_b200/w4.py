@@ -36,10 +36,11 @@ SIGNATURES = [
     ("w4_prepack_bytes", _SZ, [_I64, _I64, _I, _I]),
     ("w4_prepack", _I, [_P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P]),
     ("w4a8_gsum_op_cols", _I64, [_I64, _I]),
-    ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]),
-    ("fp8_row_quant_gather", _I, [_P, _I64, _I64, _I, _P, _I64, _P, _P, _P, _P, _P]),
-    ("w4_moe_route", _I, [_P, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
-    ("w4_moe_swiglu_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P]),
+    ("fp8_row_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P, _P, _P]),
+    ("fp8_row_quant_gather", _I, [_P, _I64, _I64, _I, _P, _I64, _P, _P, _P, _P, _P, _P]),
+    ("w4_moe_route_workspace_bytes", _I64, [_I64, _I]),
+    ("w4_moe_route", _I, [_P, _I64, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    ("w4_moe_swiglu_quant", _I, [_P, _I64, _I64, _I, _P, _P, _P, _P, _P]),
     ("w4_moe_combine", _I, [_P, _I64, _I64, _P, _P, _I64, _I, _P, _P]),
     ("w4_nf4_levels", _I, [_P]),
     ("w4_nf4_quantize", _I, [_P, _I64, _I64, _P, _P, _P]),
@@ -49,11 +50,11 @@ SIGNATURES = [
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a16_gemv_noalloc_scratch_limit", _SZ, []),
     ("w4a16_gemv_noalloc", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
-    ("w4a8_gemm", _I, [_P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
+    ("w4a8_gemm", _I, [_P, _P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a8_gemm_workspace_bytes", _SZ, [_I64, _I64, _I64, _I]),
     ("w4a8_gemm_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
     ("w4a8_gemm_split_segment", _I, [_I64, _I64, _I64, _I64, _I, _P]),
-    ("w4a8_grouped_gemm", _I, [_P, _P, _P, _P, _I, _I64, _P, _I64, _I64, _I, _I, _P, _P]),
+    ("w4a8_grouped_gemm", _I, [_P, _P, _P, _P, _P, _I, _I64, _P, _I64, _I64, _I, _I, _P, _P]),
     ("w4_device_status", _I, [_P, ctypes.POINTER(ctypes.c_int)]),
     ("w4_selftest_bounded_wait", _I, [_I64, _P]),
 ]
@@ -144,27 +145,40 @@ def w4a8_gsum_op_cols(K, group) -> int:
     return int(lib().w4a8_gsum_op_cols(K, group))
 
 
-def fp8_row_quant(X, M, K, group, X8, row_scale, group_sums=None, gsum_op=None, stream=None):
+def fp8_row_quant(X, M, K, group, X8, row_scale, group_sums=None, gsum_op=None, stream=None, *, x16=None):
+    """x16: optional fp16 [M, K] copy of the E4M3 values (the operand of w4a8_gemm at groups
+    32 and 256); X8 may then be None."""
     rc = lib().fp8_row_quant(_ptr(X), M, K, group, _ptr(X8), _ptr(row_scale), _ptr(group_sums), _ptr(gsum_op),
-                             _stream(stream))
+                             _ptr(x16), _stream(stream))
     _check("fp8_row_quant", rc)
 
 
 def fp8_row_quant_gather(X, M_src, K, group, row_index, M, X8, row_scale, group_sums=None, gsum_op=None,
-                         stream=None):
+                         stream=None, *, x16=None):
     rc = lib().fp8_row_quant_gather(_ptr(X), M_src, K, group, _ptr(row_index), M, _ptr(X8), _ptr(row_scale),
-                                    _ptr(group_sums), _ptr(gsum_op), _stream(stream))
+                                    _ptr(group_sums), _ptr(gsum_op), _ptr(x16), _stream(stream))
     _check("fp8_row_quant_gather", rc)
 
 
-def w4_moe_route(logits, T, E, k, experts, gates, expert_row_offsets, token_of_row, row_of, stream=None):
+def w4_moe_route_workspace_bytes(T, E):
+    return int(lib().w4_moe_route_workspace_bytes(T, E))
+
+
+def alloc_moe_route_workspace(T, E, device=None):
+    n = w4_moe_route_workspace_bytes(T, E)
+    return torch.empty(max(n, 4), dtype=torch.uint8, device=device)
+
+
+def w4_moe_route(logits, T, E, k, experts, gates, expert_row_offsets, token_of_row, row_of, workspace,
+                 stream=None):
     rc = lib().w4_moe_route(_ptr(logits), T, E, k, _ptr(experts), _ptr(gates), _ptr(expert_row_offsets),
-                            _ptr(token_of_row), _ptr(row_of), _stream(stream))
+                            _ptr(token_of_row), _ptr(row_of), _ptr(workspace), workspace.numel(),
+                            _stream(stream))
     _check("w4_moe_route", rc)
 
 
-def w4_moe_swiglu_quant(gate_up, R, H, group, X8, row_scale, gsum_op=None, stream=None):
-    rc = lib().w4_moe_swiglu_quant(_ptr(gate_up), R, H, group, _ptr(X8), _ptr(row_scale), _ptr(gsum_op),
+def w4_moe_swiglu_quant(gate_up, R, H, group, X8, row_scale, gsum_op=None, stream=None, *, x16=None):
+    rc = lib().w4_moe_swiglu_quant(_ptr(gate_up), R, H, group, _ptr(X8), _ptr(row_scale), _ptr(gsum_op), _ptr(x16),
                                    _stream(stream))
     _check("w4_moe_swiglu_quant", rc)
 
@@ -221,10 +235,12 @@ def w4a16_gemv_noalloc(x, M, packed, N, K, group, mode, y, flags, stream=None):
     _check("w4a16_gemv_noalloc", rc)
 
 
-def w4a8_gemm(X8, row_scale, gsum_op, M, packed, N, K, group, mode, Y, out_fp32=0, workspace=None, stream=None):
+def w4a8_gemm(X8, row_scale, gsum_op, M, packed, N, K, group, mode, Y, out_fp32=0, workspace=None, stream=None,
+              *, X16=None):
     """workspace: None (every tile whole) or alloc_gemm_workspace(M, N, K, group) (the last
-    wave's tiles may be split along K)."""
-    rc = lib().w4a8_gemm(_ptr(X8), _ptr(row_scale), _ptr(gsum_op), M, _ptr(packed), N, K, group,
+    wave's tiles may be split along K). Groups 64 and 128 take X8 and gsum_op, groups 32 and
+    256 take X16 (fp8_row_quant's fp16 copy of the E4M3 values)."""
+    rc = lib().w4a8_gemm(_ptr(X8), _ptr(X16), _ptr(row_scale), _ptr(gsum_op), M, _ptr(packed), N, K, group,
                          _mode(mode), _ptr(Y), int(out_fp32), _ptr(workspace),
                          0 if workspace is None else workspace.numel() * workspace.element_size(),
                          _stream(stream))
@@ -252,8 +268,8 @@ def w4a8_gemm_split_segment(R, KT, PS, c, s):
 
 
 def w4a8_grouped_gemm(X8, row_scale, gsum_op, expert_row_offsets, E, M_total, packed, N, K, group,
-                      mode, Y, stream=None):
-    rc = lib().w4a8_grouped_gemm(_ptr(X8), _ptr(row_scale), _ptr(gsum_op), _ptr(expert_row_offsets), E,
+                      mode, Y, stream=None, *, X16=None):
+    rc = lib().w4a8_grouped_gemm(_ptr(X8), _ptr(X16), _ptr(row_scale), _ptr(gsum_op), _ptr(expert_row_offsets), E,
                                  M_total, _ptr(packed), N, K, group, _mode(mode), _ptr(Y), _stream(stream))
     _check("w4a8_grouped_gemm", rc)
 

@@ -44,7 +44,7 @@ typedef enum {
     W4_OK = 0,
     W4_ERR_NULL = 1,         /* a required pointer is NULL                              */
     W4_ERR_SHAPE = 2,        /* a size is out of the supported range                   */
-    W4_ERR_GROUP = 3,        /* group not in {32, 64, 128} or K not a multiple of it   */
+    W4_ERR_GROUP = 3,        /* group not in {32,64,128,256} or K not a multiple of it */
     W4_ERR_ALIGN = 4,        /* a device pointer is not 16-byte aligned                */
     W4_ERR_ARG = 5,          /* any other bad argument (mode, clip grid, layout, ...)  */
     W4_ERR_UNSUPPORTED = 6,  /* valid request this library does not implement          */
@@ -132,7 +132,7 @@ w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, const in
  *   with IEEE fp32 division, round-to-nearest-even and saturation to +-448. An all-zero row
  *   gives all-zero codes.
  *   X_bf16      device, bf16 [M, K]; M >= 1, K >= 16, K % 16 == 0
- *   X_e4m3      device, uint8 [M, K]
+ *   X_e4m3      device, uint8 [M, K], or NULL when X_f16 is given
  *   row_scale   device, fp32 [M]
  *   group_sums  device, fp32 [M, K/group] or NULL: G[m,j], the sum of the E4M3 VALUES (not
  *               scaled by s[m]) of group j of `group` consecutive codes, summed exactly and
@@ -141,12 +141,15 @@ w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, const in
  *               group-sum operand that w4a8_gemm needs (it applies the weight zero point
  *               through it). With J = K/group, hi = bf16(G[m,j]) and lo = bf16(G[m,j] - hi),
  *               row m holds [hi(0..J-1) | lo(0..J-1) | hi(0..J-1) | 0 ...].
- *   group must be 32, 64 or 128 when group_sums or gsum_op is given.
+ *   X_f16       device, fp16 [M, K], or NULL: the same E4M3 values as binary16 (exact), the
+ *               activation operand w4a8_gemm takes for groups 32 and 256. At least one of
+ *               X_e4m3 and X_f16 must be given.
+ *   group must be 32, 64, 128 or 256 when group_sums or gsum_op is given.
  *   Errors: NULL / SHAPE / GROUP / ALIGN.
  */
 int64_t w4a8_gsum_op_cols(int64_t K, int group); /* 3 K/group rounded up to 32; 0 if invalid */
 w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uint8_t *X_e4m3,
-                        float *row_scale, float *group_sums, uint16_t *gsum_op,
+                        float *row_scale, float *group_sums, uint16_t *gsum_op, uint16_t *X_f16,
                         cudaStream_t stream);
 
 /*
@@ -162,7 +165,7 @@ w4_status fp8_row_quant(const void *X_bf16, int64_t M, int64_t K, int group, uin
 w4_status fp8_row_quant_gather(const void *X_bf16, int64_t M_src, int64_t K, int group,
                                const int32_t *row_index, int64_t M, uint8_t *X_e4m3,
                                float *row_scale, float *group_sums, uint16_t *gsum_op,
-                               cudaStream_t stream);
+                               uint16_t *X_f16, cudaStream_t stream);
 
 /*
  * w4a16_gemv -- weight-only INT4 decode GEMV with the dequantization fused into the
@@ -253,10 +256,13 @@ w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, 
  *   The expanded weights q are exact small integers in E4M3 and the FP8 MMA sums exact
  *   products; the group scale multiplies fp32 per-group partial sums; the zero-point term
  *   is a bf16 hi/lo product on the tensor cores (relative error about 2^-16 of that term).
- *   X_e4m3      device, uint8 [M, K] from fp8_row_quant
+ *   X_e4m3      device, uint8 [M, K] from fp8_row_quant (groups 64 and 128; may be NULL for
+ *               groups 32 and 256)
+ *   X_f16       device, fp16 [M, K] from fp8_row_quant's X_f16 output (groups 32 and 256;
+ *               may be NULL for groups 64 and 128)
  *   row_scale   device, fp32 [M] from fp8_row_quant
  *   gsum_op     device, bf16 [M, w4a8_gsum_op_cols(K, group)] from fp8_row_quant with the
- *               same group; may be NULL for group 32 (see below)
+ *               same group (groups 64 and 128; may be NULL for groups 32 and 256)
  *   packed      device, w4_prepack(..., W4_LAYOUT_GEMM) of W[N, K]
  *   Y           device, bf16 [M, N] (out_fp32 == 0) or fp32 [M, N] (out_fp32 == 1)
  *   workspace   NULL, or device scratch of at least w4a8_gemm_workspace_bytes(M, N, K, group)
@@ -272,20 +278,21 @@ w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, 
  *               unsplit schedule, within the same error bounds). A query result of 0 means
  *               the shape is never split and the workspace is not used.
  *   M >= 1; N >= 1; K >= 128, K % 32 == 0.
- *   Groups of 32: every FP8 MMA of K = 32 would end a group, and the per-group promotion
- *   (a TMEM readback and one fp32 FMA per output per group on the CUDA cores) would cost
- *   several times the MMA. For group 32 the kernel instead dequantizes each weight exactly
+ *   Groups of 32 and 256: at 32 every FP8 MMA of K = 32 would end a group, and the
+ *   per-group promotion (a TMEM readback and one fp32 FMA per output per group on the CUDA
+ *   cores) would cost several times the MMA; at 256 the group spans two k-blocks of the
+ *   promoted schedule. For these groups the kernel instead dequantizes each weight exactly
  *   into two fp16 parts, w = (q - z) s = hi + lo (exact for |z| < 1024 and |w| < 65504),
- *   converts the E4M3 activations to fp16 (exact), and accumulates hi x a + lo x a on the
- *   fp16 tensor cores over the whole K in TMEM: the same dequantized operands, no zero-point
- *   operand (gsum_op is not read and may be NULL), no split of the last wave (the workspace
+ *   and accumulates hi x a + lo x a on the fp16 tensor cores over the whole K in TMEM, a
+ *   being the E4M3 activation values, which it reads as fp16 (X_f16, exact): the same
+ *   dequantized operands, no zero-point operand, no split of the last wave (the workspace
  *   query returns 0).
  *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG / WORKSPACE (non-NULL and smaller than the
  *   query's result).
  */
 size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int group);
-w4_status w4a8_gemm(const uint8_t *X_e4m3, const float *row_scale, const uint16_t *gsum_op,
-                    int64_t M, const void *packed, int64_t N, int64_t K, int group, int mode,
+w4_status w4a8_gemm(const uint8_t *X_e4m3, const uint16_t *X_f16, const float *row_scale,
+                    const uint16_t *gsum_op, int64_t M, const void *packed, int64_t N, int64_t K, int group, int mode,
                     void *Y, int out_fp32, void *workspace, size_t workspace_bytes,
                     cudaStream_t stream);
 
@@ -309,7 +316,7 @@ w4_status w4a8_gemm_split_segment(int64_t R, int64_t KT, int64_t PS, int64_t c, 
 /*
  * w4a8_grouped_gemm -- w4a8_gemm for E experts at once (mixture-of-experts layers whose
  *   expert weights are 4-bit; the blog post "4-bit by default", gpt-oss paragraph). Rows
- *   [off[e], off[e+1]) of X_e4m3 / row_scale / gsum_op / Y belong to expert e and are
+ *   [off[e], off[e+1]) of X_e4m3 / X_f16 / row_scale / gsum_op / Y belong to expert e and are
  *   multiplied by expert e's weight.
  *   expert_row_offsets  device, int32 [E+1], non-decreasing, off[0] == 0, off[E] == M_total
  *   packed              device, E slabs of w4_prepack_bytes(N, K, group, W4_LAYOUT_GEMM)
@@ -317,7 +324,7 @@ w4_status w4a8_gemm_split_segment(int64_t R, int64_t KT, int64_t PS, int64_t c, 
  *   Y                   device, bf16 [M_total, N]
  *   1 <= E <= 1024. Errors: NULL / SHAPE / GROUP / ALIGN / ARG.
  */
-w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale,
+w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const uint16_t *X_f16, const float *row_scale,
                             const uint16_t *gsum_op, const int32_t *expert_row_offsets, int E,
                             int64_t M_total, const void *packed, int64_t N, int64_t K, int group,
                             int mode, void *Y, cudaStream_t stream);
@@ -332,17 +339,23 @@ w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const float *row_scale,
  * (down); w4_moe_combine.
  *
  * w4_moe_route -- logits fp32 [T, E] (device). For each token the k largest logits in
- *   descending order (equal logits in ascending expert order) -> experts int32 [T, k];
- *   gates fp32 [T, k] = softmax over those k logits (fp32, expf); expert_row_offsets int32
- *   [E+1], rows of expert e being [off[e], off[e+1]) of the grouped layout; token_of_row
- *   int32 [T*k], the token of every grouped row (tokens ascending inside an expert); row_of
- *   int32 [T, k], the grouped row of token t's i-th expert. Deterministic (no dependence on
- *   thread timing). One block; 1 <= E <= 1024, 1 <= k <= min(8, E), T * ceil(E/32) * 4 bytes
- *   <= 96 KiB (T <= 24576 at E = 32). Errors: NULL / SHAPE / ALIGN (4-byte) / CUDA.
+ *   descending order (equal logits in ascending expert order; a NaN logit is taken only where
+ *   a scan in expert order that replaces its choice by a strictly larger logit would take it)
+ *   -> experts int32 [T, k]; gates fp32 [T, k] = softmax over those k logits (fp32, expf);
+ *   expert_row_offsets int32 [E+1], rows of expert e being [off[e], off[e+1]) of the grouped
+ *   layout; token_of_row int32 [T*k], the token of every grouped row (tokens ascending inside
+ *   an expert); row_of int32 [T, k], the grouped row of token t's i-th expert. Deterministic
+ *   (no dependence on thread timing). workspace: device scratch of at least
+ *   w4_moe_route_workspace_bytes(T, E) bytes (ceil(T/32) * E int32 expert counts), owned by
+ *   the caller, contents irrelevant between calls. Two launches on `stream`.
+ *   1 <= E <= 1024, 1 <= k <= min(8, E), T * k < 2^31. Errors: NULL / SHAPE / WORKSPACE /
+ *   ALIGN (4-byte) / CUDA.
  */
+int64_t w4_moe_route_workspace_bytes(int64_t T, int E);
 w4_status w4_moe_route(const float *logits, int64_t T, int E, int k, int32_t *experts,
                        float *gates, int32_t *expert_row_offsets, int32_t *token_of_row,
-                       int32_t *row_of, cudaStream_t stream);
+                       int32_t *row_of, void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
 
 /*
  * w4_moe_swiglu_quant -- SwiGLU between the expert projections, then the per-row E4M3
@@ -350,12 +363,13 @@ w4_status w4_moe_route(const float *logits, int64_t T, int E, int k, int32_t *ex
  *   gate_up_bf16 [R, 2H] holds [gate | up] per row; h = gate * up / (1 + exp(-gate)) in fp32;
  *   row_scale[r] = max(max|h|, 1e-8) / 448; X_e4m3 [R, H] = e4m3(h / row_scale) with IEEE
  *   division, RNE, saturation. gsum_op (optional, bf16 [R, w4a8_gsum_op_cols(H, group)]) as
- *   fp8_row_quant writes it, for down projections with group 64 or 128.
- *   16 <= H <= 16384, H % 16 == 0. Errors: NULL / SHAPE / GROUP / ALIGN.
+ *   fp8_row_quant writes it, for down projections with group 64 or 128; X_f16 (optional,
+ *   fp16 [R, H]) the same E4M3 values as binary16, for groups 32 and 256 (X_e4m3 may then
+ *   be NULL). 16 <= H <= 16384, H % 16 == 0. Errors: NULL / SHAPE / GROUP / ALIGN.
  */
 w4_status w4_moe_swiglu_quant(const void *gate_up_bf16, int64_t R, int64_t H, int group,
                               uint8_t *X_e4m3, float *row_scale, uint16_t *gsum_op,
-                              cudaStream_t stream);
+                              uint16_t *X_f16, cudaStream_t stream);
 
 /*
  * w4_moe_combine -- y[t, :] = sum_{i < k} gates[t, i] * rows[row_of[t, i], :], fp32 products

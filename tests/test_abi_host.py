@@ -101,26 +101,42 @@ def test_host_validation_rejects_before_launch(lib):
               None, None) == 5
     assert rc("w4_quantize", FAKE, 16, 128, 128, 1, gp, 0, FAKE, FAKE, FAKE, None, None) == 5
     assert rc("w4_quantize", FAKE, 16, 128, 128, 1, gp, 65, FAKE, FAKE, FAKE, None, None) == 5
-    # row quant
-    assert rc("fp8_row_quant", None, 4, 64, 32, FAKE, FAKE, None, None, None) == 1
-    assert rc("fp8_row_quant", FAKE, 4, 72, 32, FAKE, FAKE, None, None, None) == 2
-    assert rc("fp8_row_quant", FAKE, 4, 96, 64, FAKE, FAKE, FAKE, None, None) == 3
-    assert rc("fp8_row_quant", FAKE, 4, 96, 64, FAKE, FAKE, None, FAKE, None) == 3
-    assert rc("fp8_row_quant", FAKE, 4, 128, 64, FAKE, FAKE, None, FAKE + 4, None) == 4
+    # row quant: codes or their fp16 copy (or both) required
+    assert rc("fp8_row_quant", None, 4, 64, 32, FAKE, FAKE, None, None, None, None) == 1
+    assert rc("fp8_row_quant", FAKE, 4, 64, 32, None, FAKE, None, None, None, None) == 1
+    assert rc("fp8_row_quant", FAKE, 4, 72, 32, FAKE, FAKE, None, None, None, None) == 2
+    assert rc("fp8_row_quant", FAKE, 4, 96, 64, FAKE, FAKE, FAKE, None, None, None) == 3
+    assert rc("fp8_row_quant", FAKE, 4, 96, 64, FAKE, FAKE, None, FAKE, None, None) == 3
+    assert rc("fp8_row_quant", FAKE, 4, 128, 64, FAKE, FAKE, None, FAKE + 4, None, None) == 4
+    assert rc("fp8_row_quant", FAKE, 4, 128, 64, None, FAKE, None, None, FAKE + 8, None) == 4
     # gemv: M range, mode, out flag
     assert rc("w4a16_gemv", FAKE, 17, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE, 1 << 20, None) == 2
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 3, FAKE, 0, FAKE, 1 << 20, None) == 5
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 4, FAKE, 1 << 20, None) == 5
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE + 8, 1 << 20, None) == 4
-    # gemm: the group-sum operand is required, K >= 128
-    assert rc("w4a8_gemm", FAKE, FAKE, None, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, None) == 1
-    assert rc("w4a8_gemm", FAKE, FAKE, FAKE, 4, FAKE, 16, 96, 32, 1, FAKE, 0, None, 0, None) == 2
-    assert rc("w4a8_gemm", FAKE, FAKE, FAKE, 4, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE + 8, 1 << 20, None) == 4
+    # gemm: groups 64/128 need the codes and the group-sum operand, groups 32/256 the fp16
+    # copy of the activations; K >= 128
+    assert rc("w4a8_gemm", FAKE, None, FAKE, None, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, None) == 1
+    assert rc("w4a8_gemm", None, FAKE, FAKE, FAKE, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, None) == 1
+    assert rc("w4a8_gemm", FAKE, None, FAKE, FAKE, 4, FAKE, 16, 128, 32, 1, FAKE, 0, None, 0, None) == 1
+    assert rc("w4a8_gemm", FAKE, FAKE, FAKE, FAKE, 4, FAKE, 16, 96, 32, 1, FAKE, 0, None, 0, None) == 2
+    assert rc("w4a8_gemm", FAKE, None, FAKE, FAKE, 4, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE + 8, 1 << 20, None) == 4
+    assert rc("w4a8_gemm", None, FAKE + 4, FAKE, None, 4, FAKE, 16, 256, 256, 1, FAKE, 0, None, 0, None) == 4
     # grouped gemm: expert count range
-    assert rc("w4a8_grouped_gemm", FAKE, FAKE, FAKE, FAKE, 0, 16, FAKE, 16, 128, 128, 1, FAKE, None) == 2
+    assert rc("w4a8_grouped_gemm", FAKE, None, FAKE, FAKE, FAKE, 0, 16, FAKE, 16, 128, 128, 1, FAKE, None) == 2
     # prepack
     assert rc("w4_prepack", FAKE, FAKE, None, 16, 128, 128, 1, 0, FAKE, None) == 1
     assert rc("w4_prepack", FAKE, FAKE, None, 16, 128, 128, 0, 9, FAKE, None) == 5
+    # moe route: expert and top-k ranges, workspace size
+    ws = lib.w4_moe_route_workspace_bytes(100, 32)
+    assert ws == 4 * 32 * 4  # ceil(100 / 32) blocks of 32 expert counts
+    assert lib.w4_moe_route_workspace_bytes(0, 32) == 0
+    assert rc("w4_moe_route", FAKE, 100, 32, 4, FAKE, FAKE, FAKE, FAKE, FAKE, None, ws, None) == 1
+    assert rc("w4_moe_route", FAKE, 100, 1025, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 2
+    assert rc("w4_moe_route", FAKE, 100, 32, 9, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == 2
+    assert rc("w4_moe_route", FAKE, 100, 4, 5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == 2
+    assert rc("w4_moe_route", FAKE, 100, 32, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 4, None) == 10
+    assert rc("w4_moe_route", FAKE + 2, 100, 32, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == 4
     # device status needs an out pointer
     assert rc("w4_device_status", None, None) == 1
 

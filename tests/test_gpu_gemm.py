@@ -37,11 +37,28 @@ def upload_weight(codes, scales, zeros, N, K, group, mode, copies=1):
     return packed
 
 
+def split_path(group):
+    """Groups 32 and 256 run the split-weight fp16 path, which takes the fp16 copy of the E4M3
+    activations (and neither the codes nor the group-sum operand)."""
+    return group in (32, 256)
+
+
+def x16_of(X8):
+    """The fp16 copy of E4M3 codes (exact), as fp8_row_quant writes it."""
+    return to_dev(X8).view(torch.float8_e4m3fn).to(torch.float16)
+
+
+def gemm_operands(X8, G, K, group):
+    if split_path(group):
+        return None, None, x16_of(X8)
+    return to_dev(X8), to_dev(gsum_operand(G, K, group)), None
+
+
 def gpu_gemm(X8, s_a, G, packed, N, K, group, mode, out_fp32, ws=None):
     M = X8.shape[0]
     Y = torch.empty(M, N, dtype=torch.float32 if out_fp32 else torch.bfloat16, device=cuda())
-    gop = to_dev(gsum_operand(G, K, group))
-    w4.w4a8_gemm(to_dev(X8), to_dev(s_a), gop, M, packed, N, K, group, mode, Y, out_fp32, ws)
+    x8, gop, x16 = gemm_operands(X8, G, K, group)
+    w4.w4a8_gemm(x8, to_dev(s_a), gop, M, packed, N, K, group, mode, Y, out_fp32, ws, X16=x16)
     torch.cuda.synchronize()
     return Y.float().cpu().numpy().astype(np.float64)
 
@@ -189,8 +206,8 @@ def gpu_grouped(codes, scales, zeros, off, X8, s_a, G, N, K, g):
     M = X8.shape[0]
     packed = upload_weight(codes, scales, zeros, N, K, g, "asym", copies=E)
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=cuda())
-    gop = to_dev(gsum_operand(G, K, g))
-    w4.w4a8_grouped_gemm(to_dev(X8), to_dev(s_a), gop, to_dev(off), E, M, packed, N, K, g, "asym", Y)
+    x8, gop, x16 = gemm_operands(X8, G, K, g)
+    w4.w4a8_grouped_gemm(x8, to_dev(s_a), gop, to_dev(off), E, M, packed, N, K, g, "asym", Y, X16=x16)
     torch.cuda.synchronize()
     return Y.float().cpu().numpy().astype(np.float64)
 

@@ -32,11 +32,13 @@ def gpu_route(lg, k):
     off = torch.empty(E + 1, dtype=torch.int32, device=dev)
     tor = torch.empty(T * k, dtype=torch.int32, device=dev)
     row_of = torch.empty(T, k, dtype=torch.int32, device=dev)
-    w4.w4_moe_route(to_dev(lg), T, E, k, ex, gt, off, tor, row_of)
+    ws = w4.alloc_moe_route_workspace(T, E, device=dev)
+    w4.w4_moe_route(to_dev(lg), T, E, k, ex, gt, off, tor, row_of, ws)
     return ex, gt, off, tor, row_of
 
 
-@pytest.mark.parametrize("T,E,k", [(4096, 32, 4), (100, 8, 2), (33, 5, 5), (1, 1, 1)])
+@pytest.mark.parametrize("T,E,k", [(4096, 32, 4), (100, 8, 2), (33, 5, 5), (1, 1, 1), (65, 1024, 8),
+                                   (300, 100, 3)])
 def test_route(T, E, k):
     lg = logits_of(T, E, T + E)
     ex, gt, off, tor, row_of = gpu_route(lg, k)
@@ -48,6 +50,42 @@ def test_route(T, E, k):
     assert np.array_equal(tor.cpu().numpy(), rtor)
     assert np.array_equal(row_of.cpu().numpy(), rrow)
     assert np.allclose(gt.cpu().numpy(), rg, rtol=2e-6, atol=1e-7)
+
+
+def test_route_with_nan_and_infinite_logits():
+    """Non-finite logits follow the oracle's scan in expert order: a NaN is taken only when it
+    is the first expert still untaken; -inf and +inf order like any value."""
+    T, E, k = 40, 37, 4
+    lg = logits_of(T, E, 9)
+    lg[0, 0] = np.nan                  # first expert NaN: chosen first
+    lg[1, 5] = np.nan                  # NaN elsewhere: never chosen while finite ones remain
+    lg[2, :] = np.nan                  # all NaN: experts 0, 1, 2, 3
+    lg[7, 3] = np.nan                  # a NaN after finite ones: skipped
+    lg[3, 7] = np.inf
+    lg[4, :] = -np.inf                 # all equal: ascending experts
+    lg[5, :E - 3] = np.nan             # the first untaken expert is NaN in every round: 0, 1, 2, 3
+    lg[6, 1::2] = 0.5                  # many ties
+    ex, gt, off, tor, row_of = gpu_route(lg, k)
+    rex, rg = oracle.moe_route(lg, k)
+    rtor, roff, rrow = oracle.moe_grouping(rex, E)
+    torch.cuda.synchronize()
+    assert np.array_equal(ex.cpu().numpy(), rex)
+    assert np.array_equal(tor.cpu().numpy(), rtor)
+    assert np.array_equal(row_of.cpu().numpy(), rrow)
+    fin = np.isfinite(rg).all(axis=1)
+    assert np.allclose(gt.cpu().numpy()[fin], rg[fin], rtol=2e-6, atol=1e-7)
+    assert np.array_equal(np.isnan(gt.cpu().numpy()), np.isnan(rg))
+
+
+def test_route_rejects_a_short_workspace():
+    dev = cuda()
+    T, E, k = 64, 32, 2
+    lg = torch.zeros(T, E, dtype=torch.float32, device=dev)
+    outs = [torch.empty(n, dtype=torch.int32, device=dev) for n in (T * k, T * k, E + 1, T * k, T * k)]
+    ws = torch.empty(w4.w4_moe_route_workspace_bytes(T, E) - 4, dtype=torch.uint8, device=dev)
+    with pytest.raises(w4.W4Error) as e:
+        w4.w4_moe_route(lg, T, E, k, *outs, ws)
+    assert e.value.code == 10
 
 
 def test_gather_row_quant_is_row_quant_of_the_gathered_rows():
@@ -134,16 +172,19 @@ def moe_layer_gpu(X, lg, k, pgu, pdn, H, K, g):
     dev = cuda()
     ex, gt, off, tor, row_of = gpu_route(lg, k)
     R = T * k
-    X8 = torch.empty(R, K, dtype=torch.uint8, device=dev)
+    # group 32: the GEMMs take the fp16 copy of the E4M3 activations, so the dispatch writes
+    # only that copy; the SwiGLU quant writes both (the codes are checked below)
+    X16 = torch.empty(R, K, dtype=torch.float16, device=dev)
     sa = torch.empty(R, dtype=torch.float32, device=dev)
-    w4.fp8_row_quant_gather(X, T, K, g, tor, R, X8, sa)
+    w4.fp8_row_quant_gather(X, T, K, g, tor, R, None, sa, x16=X16)
     Ygu = torch.empty(R, 2 * H, dtype=torch.bfloat16, device=dev)
-    w4.w4a8_grouped_gemm(X8, sa, None, off, E, R, pgu, 2 * H, K, g, "asym", Ygu)
+    w4.w4a8_grouped_gemm(None, sa, None, off, E, R, pgu, 2 * H, K, g, "asym", Ygu, X16=X16)
     H8 = torch.empty(R, H, dtype=torch.uint8, device=dev)
+    H16 = torch.empty(R, H, dtype=torch.float16, device=dev)
     sh = torch.empty(R, dtype=torch.float32, device=dev)
-    w4.w4_moe_swiglu_quant(Ygu, R, H, g, H8, sh)
+    w4.w4_moe_swiglu_quant(Ygu, R, H, g, H8, sh, x16=H16)
     Yd = torch.empty(R, K, dtype=torch.bfloat16, device=dev)
-    w4.w4a8_grouped_gemm(H8, sh, None, off, E, R, pdn, K, H, g, "asym", Yd)
+    w4.w4a8_grouped_gemm(None, sh, None, off, E, R, pdn, K, H, g, "asym", Yd, X16=H16)
     y = torch.empty(T, K, dtype=torch.bfloat16, device=dev)
     w4.w4_moe_combine(Yd, K, R, row_of, gt, T, k, y)
     return y, dict(Ygu=Ygu, H8=H8, sh=sh, Yd=Yd)

@@ -1,6 +1,7 @@
 """GPU fp8_row_quant vs the CPU oracle: E4M3 bytes, row scales and group sums must be
-bit-identical, and the GEMM's group-sum operand must be the documented bf16 hi/lo split of
-the oracle's group sums, bit for bit."""
+bit-identical, the GEMM's group-sum operand must be the documented bf16 hi/lo split of
+the oracle's group sums, bit for bit, and the optional fp16 copy must hold exactly the E4M3
+values (binary16 bits of the oracle's decoded codes)."""
 import numpy as np
 import pytest
 import torch
@@ -22,24 +23,30 @@ def gpu_row_quant(X, group, op_only=False):
         X8 = torch.empty(M, K, dtype=torch.uint8, device=cuda())
         s = torch.empty(M, dtype=torch.float32, device=cuda())
         G = gop = None
-    w4.fp8_row_quant(Xd, M, K, group if group else 32, X8, s, G, gop)
+    x16 = torch.full((M, K), float("nan"), dtype=torch.float16, device=cuda())
+    w4.fp8_row_quant(Xd, M, K, group if group else 32, X8, s, G, gop, x16=x16)
     torch.cuda.synchronize()
     op = gop.view(torch.int16).cpu().numpy().view(np.uint16) if gop is not None else None
-    return np_of(X8), np_of(s), (np_of(G) if G is not None else None), op
+    return np_of(X8), np_of(s), (np_of(G) if G is not None else None), op, x16.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def f16_bits_of_codes(X8):
+    return oracle.e4m3_decode(X8).astype(np.float16).view(np.uint16)
 
 
 def check(X, group, rows=None, op_only=False):
-    gX8, gs, gG, gop = gpu_row_quant(X, group, op_only)
+    gX8, gs, gG, gop, gx16 = gpu_row_quant(X, group, op_only)
     bits = synth.bf16_bits(X)
     if rows is not None:
         bits = bits[rows]
-        gX8, gs = gX8[rows], gs[rows]
+        gX8, gs, gx16 = gX8[rows], gs[rows], gx16[rows]
         gG = gG[rows] if gG is not None else None
         gop = gop[rows] if gop is not None else None
     X8, s, G = oracle.row_quant(bits, group)
     assert np.array_equal(gs.view(np.uint32), s.view(np.uint32))
     bad = np.argwhere(gX8 != X8)
     assert bad.size == 0, f"{len(bad)} byte mismatches, first {bad[:3].tolist()}"
+    assert np.array_equal(gx16, f16_bits_of_codes(X8))
     if group:
         if not op_only:
             assert np.array_equal(gG.view(np.uint32), G.view(np.uint32))
@@ -134,9 +141,22 @@ def test_rows_with_infinities():
     row2 = row.copy()
     row2[7] = -np.inf
     X = torch.from_numpy(np.array([row, row2])).to(torch.bfloat16)
-    gX8, gs, _, _ = gpu_row_quant(X, 32)
+    gX8, gs, _, _, _ = gpu_row_quant(X, 32)
     X8, s, _ = oracle.row_quant(synth.bf16_bits(X), 32)
     assert np.array_equal(gs.view(np.uint32), s.view(np.uint32))
     finite = np.ones(K, bool)
     finite[7] = False
     assert np.array_equal(gX8[:, finite], X8[:, finite])
+
+
+def test_fp16_copy_without_codes():
+    """Only the fp16 copy (the operand of the groups-32/256 GEMM path): the same values."""
+    M, K = 77, 2880
+    X = synth.outlier_activation(M, K, 4, 20.0, 2, 11)
+    s = torch.empty(M, dtype=torch.float32, device=cuda())
+    x16 = torch.full((M, K), float("nan"), dtype=torch.float16, device=cuda())
+    w4.fp8_row_quant(X.to(cuda()), M, K, 32, None, s, x16=x16)
+    X8, rs, _ = oracle.row_quant(synth.bf16_bits(X), 0)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_of(s).view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(x16.view(torch.int16).cpu().numpy().view(np.uint16), f16_bits_of_codes(X8))

@@ -53,8 +53,10 @@ def test_noalloc_matches_workspace_entry_point(N, K, M, flags):
     x = synth.normal((M, K), 1.0, 3, M).to(dev)
     dt = torch.float32 if flags & w4.W4_OUT_FP32 else torch.bfloat16
     ws = w4.alloc_gemv_workspace(N, K, g, device=dev)
-    ref = torch.empty(M, N, dtype=dt, device=dev)
+    ref = torch.full((M, N), float("nan"), dtype=dt, device=dev)
     w4.w4a16_gemv(x, M, p, N, K, g, "asym", ref, flags, ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(ref).all() and w4.w4_device_status() == 0
     tol = TOL_F32 if dt == torch.float32 else TOL_BF16
     for _ in range(2):  # two calls in a row on the shared scratch
         got = torch.full((M, N), float("nan"), dtype=dt, device=dev)
