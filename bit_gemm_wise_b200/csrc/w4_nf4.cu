@@ -182,6 +182,109 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) gemv_kernel(const uint16_t *_
     }
 }
 
+
+// M = 1 with K a multiple of 1024 up to 16384: one block per SM owns a contiguous run of rows;
+// thread (slot, sl) takes the 16-byte code chunk sl (32 weights, half an NF4 block) of the rows
+// slot, slot + nslot, ... and holds its 32 activations in registers. The code chunks and block
+// scales of the next PF rows are loaded ahead in registers (issued before the dependency wait
+// under programmatic launch). Each code is looked up in a 16-entry fp32 table in shared
+// memory (one entry per bank, so any lookup pattern is conflict-free) and multiplied into one
+// of four fp32 sums; the chunk's sum times the block scale is reduced over the warp, then over
+// the row's warps in order.
+constexpr int RT = 512;
+constexpr int PF = 4;
+constexpr int MAX_RPB = 256;
+
+__device__ __forceinline__ float lut_at(const float *lut, uint32_t byte_off) {
+    return *reinterpret_cast<const float *>(reinterpret_cast<const char *>(lut) + byte_off);
+}
+
+__global__ void __launch_bounds__(RT, 1) gemv_rows_kernel(const uint16_t *__restrict__ x,
+                                                          const uint8_t *__restrict__ codes,
+                                                          const float *__restrict__ absmax, int64_t N, int64_t K,
+                                                          Levels L, void *y, int out_fp32, int pdl, int rpb) {
+    __shared__ float lut[16];
+    __shared__ float red[MAX_RPB * 16];  // [row][warp of the row]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wpr = (int)(K / 1024);          // warps per row
+    const int nslot = (RT / 32) / wpr;        // rows in flight
+    const int slot = warp / wpr, ws = warp - slot * wpr;
+    const int sl = ws * 32 + lane;            // 16-byte chunk of the row
+    const bool active = slot < nslot;
+    const int64_t row0 = (int64_t)blockIdx.x * rpb;
+    const int rows = (int)((N - row0) < rpb ? (N - row0) : rpb);
+    const int nr = active && slot < rows ? (rows - slot + nslot - 1) / nslot : 0;  // rows of this slot
+    const int64_t rb = K / 2, ab = K / 64;    // code bytes and block scales per row
+    if (tid < 16) lut[tid] = L.v[tid];
+    uint4 cq[PF];
+    float aq[PF];
+#pragma unroll
+    for (int p = 0; p < PF; ++p) {
+        const int64_t n = row0 + slot + (int64_t)p * nslot;
+        const bool ok = p < nr;
+        cq[p] = ok ? __ldg(reinterpret_cast<const uint4 *>(codes + n * rb) + sl) : make_uint4(0u, 0u, 0u, 0u);
+        aq[p] = ok ? __ldg(absmax + n * ab + (sl >> 1)) : 0.0f;
+    }
+    __syncthreads();
+    if (pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+    float xr[32];
+    {
+        const uint4 *xs = reinterpret_cast<const uint4 *>(x) + (int64_t)sl * 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = active ? __ldg(xs + q) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                xr[8 * q + 2 * i] = bf16_lo(u[i]);
+                xr[8 * q + 2 * i + 1] = bf16_hi(u[i]);
+            }
+        }
+    }
+    if (pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int i = 0; i < nr; ++i) {
+        const uint4 c = cq[0];
+        const float am = aq[0];
+#pragma unroll
+        for (int p = 0; p + 1 < PF; ++p) {
+            cq[p] = cq[p + 1];
+            aq[p] = aq[p + 1];
+        }
+        {
+            const int64_t n = row0 + slot + (int64_t)(i + PF) * nslot;
+            const bool ok = i + PF < nr;
+            cq[PF - 1] = ok ? __ldg(reinterpret_cast<const uint4 *>(codes + n * rb) + sl) : make_uint4(0u, 0u, 0u, 0u);
+            aq[PF - 1] = ok ? __ldg(absmax + n * ab + (sl >> 1)) : 0.0f;
+        }
+        const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const uint32_t lo = (wv[w] & 0x0F0F0F0Fu) << 2;  // byte b: 4 q[8w + 2b]
+            const uint32_t hi = (wv[w] >> 2) & 0x3C3C3C3Cu;  // byte b: 4 q[8w + 2b + 1]
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t sel = 0x4440u | (uint32_t)b;
+                acc[(2 * b) & 3] = __fmaf_rn(lut_at(lut, __byte_perm(lo, 0u, sel)), xr[8 * w + 2 * b], acc[(2 * b) & 3]);
+                acc[(2 * b + 1) & 3] =
+                    __fmaf_rn(lut_at(lut, __byte_perm(hi, 0u, sel)), xr[8 * w + 2 * b + 1], acc[(2 * b + 1) & 3]);
+            }
+        }
+        float r = __fmul_rn(__fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3])), am);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) r += __shfl_xor_sync(FULL, r, off);
+        if (lane == 0) red[(slot + i * nslot) * 16 + ws] = r;
+    }
+    __syncthreads();
+    for (int rl = tid; rl < rows; rl += RT) {
+        float acc = 0.0f;
+        for (int w = 0; w < wpr; ++w) acc += red[rl * 16 + w];
+        const int64_t n = row0 + rl;
+        if (out_fp32) static_cast<float *>(y)[n] = acc;
+        else static_cast<__nv_bfloat16 *>(y)[n] = __float2bfloat16_rn(acc);
+    }
+}
+
 }  // namespace nf4
 }  // namespace w4
 
@@ -215,6 +318,32 @@ W4_API w4_status w4_nf4_gemv(const void *x_bf16, int64_t M, const uint8_t *codes
     if (smem > 227 * 1024) return W4_ERR_SHAPE;
     if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(absmax) || !aligned16(y)) return W4_ERR_ALIGN;
     const int out_fp32 = (flags & W4_OUT_FP32) ? 1 : 0, pdl = (flags & W4_OVERLAP_PREVIOUS) ? 1 : 0;
+    if (M == 1 && K % 1024 == 0 && K <= 16384) {
+        // one block per SM, contiguous row runs of at most MAX_RPB rows
+        const int64_t sms = num_sms();
+        int64_t grid = sms < N ? sms : N;
+        if ((N + grid - 1) / grid > nf4::MAX_RPB) grid = (N + nf4::MAX_RPB - 1) / nf4::MAX_RPB;
+        const int rpb = (int)((N + grid - 1) / grid);
+        grid = (N + rpb - 1) / rpb;
+        if (grid > 0x7fffffffLL) return W4_ERR_SHAPE;
+        const nf4::Levels L = nf4::levels();
+        const uint16_t *xp = static_cast<const uint16_t *>(x_bf16);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(nf4::RT);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = pdl;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        void *args[] = {(void *)&xp, (void *)&codes, (void *)&absmax, (void *)&N, (void *)&K, (void *)&L, &y,
+                        (void *)&out_fp32, (void *)&pdl, (void *)&rpb};
+        if (cudaLaunchKernelExC(&cfg, reinterpret_cast<void *>(nf4::gemv_rows_kernel), args) != cudaSuccess)
+            return W4_ERR_CUDA;
+        return launch_status();
+    }
     const int64_t want = (N + 7) / 8;  // a warp per row, 8 warps per block
     const int grid = (int)(want < (int64_t)num_sms() * 2 ? want : (int64_t)num_sms() * 2);
     void *fn = M == 1 ? reinterpret_cast<void *>(nf4::gemv_kernel<1>)

@@ -149,6 +149,111 @@ template <int MT> struct Geo {
     static constexpr int RPT = MT == 1 ? 2 : 1;  // rows per thread and stage (registers allow two at MT = 1)
 };
 
+// Byte planes of activation row m0 + m for the tasks t0 + r NCT (r < XBN) of this thread (one
+// task = 8 consecutive k of a slice; a slice's WPS tasks are consecutive lanes). X = rint(x 2^S)
+// with S from the slice's largest |x| (|X| < 2^19); planes: even k as 16 X, odd k as X, byte p
+// of each in 4-byte words, stored load-major (see Geo); per chunk the sum of X, per slice 2^-S.
+template <int MT, int XBN>
+__device__ __forceinline__ void xprep_rounds(const Args &a, uint32_t *planes, int *sx, float *pp, int m, int m0,
+                                             int64_t k0, int nsl, int t0) {
+    using GE_ = Geo<MT>;
+    constexpr int KC = GE_::KC, NCH = GE_::NCH, WPS = GE_::WPS, PSTRIDE = GE_::PSTRIDE;
+    const int tasks = a.spp * WPS;
+    uint4 xv[XBN];
+#pragma unroll
+    for (int r = 0; r < XBN; ++r) {
+        const int t = t0 + r * NCT;
+        const int tsl = t / WPS, wi = t - tsl * WPS;
+        const int64_t k = k0 + (int64_t)tsl * KC + wi * 8;
+        const bool live = t < tasks && tsl < nsl && m0 + m < a.M && k < a.K;
+        xv[r] = live ? __ldg(reinterpret_cast<const uint4 *>(a.x + (int64_t)(m0 + m) * a.K + k))
+                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // largest magnitude pattern of each slice (bf16 bits order like magnitudes)
+    uint32_t mx[XBN];
+#pragma unroll
+    for (int r = 0; r < XBN; ++r) {
+        const uint32_t e[4] = {xv[r].x, xv[r].y, xv[r].z, xv[r].w};
+        mx[r] = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx[r] = max(mx[r], max(e[i] & 0x7FFFu, (e[i] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+    for (int off = WPS / 2; off >= 1; off >>= 1)
+#pragma unroll
+        for (int r = 0; r < XBN; ++r) mx[r] = max(mx[r], __shfl_xor_sync(FULL, mx[r], off));
+    int xs[XBN];
+#pragma unroll
+    for (int r = 0; r < XBN; ++r) {
+        const uint32_t e[4] = {xv[r].x, xv[r].y, xv[r].z, xv[r].w};
+        // exponent of the largest |x|: |x| in [2^ex, 2^(ex+1))
+        int ex;
+        if (mx[r] >= 0x80u) ex = (int)(mx[r] >> 7) - 127;
+        else ex = (31 - __clz((int)(mx[r] | 1u))) - 133;
+        const int S = 18 - ex;
+        const float f1 = exp2i(S < 127 ? S : 127), f2 = exp2i(S < 127 ? 0 : S - 127);
+        int X[8];
+        // x 2^S is exact (a power of two; |x 2^S| < 2^19); only slices whose largest |x| is
+        // below 2^-109 need the second factor (a warp-uniform branch)
+        if (__any_sync(FULL, S > 127)) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t bb = (i & 1) ? (e[i >> 1] >> 16) : (e[i >> 1] & 0xFFFFu);
+                const float sv = __fmul_rn(__fmul_rn(__uint_as_float(bb << 16), f1), f2);
+                X[i] = __float_as_int(__fadd_rn(sv, 12582912.0f)) - 0x4B400000;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t bb = (i & 1) ? (e[i >> 1] & 0xFFFF0000u) : (e[i >> 1] << 16);
+                X[i] = __float_as_int(__fmaf_rn(__uint_as_float(bb), f1, 12582912.0f)) - 0x4B400000;
+            }
+        }
+        if (mx[r] >= 0x7F80u || mx[r] == 0u) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) X[i] = 0;
+        }
+        uint32_t pw[6];
+#pragma unroll
+        for (int par = 0; par < 2; ++par) {
+            const uint32_t sh = par ? 0u : 4u;
+            const uint32_t V0 = (uint32_t)X[par] << sh, V1 = (uint32_t)X[2 + par] << sh;
+            const uint32_t V2 = (uint32_t)X[4 + par] << sh, V3 = (uint32_t)X[6 + par] << sh;
+#pragma unroll
+            for (int pl = 0; pl < 3; ++pl) {
+                const uint32_t lo = __byte_perm(V0, V1, (uint32_t)(pl | ((4 + pl) << 4)));
+                const uint32_t hi = __byte_perm(V2, V3, (uint32_t)(pl | ((4 + pl) << 4)));
+                pw[par * 3 + pl] = __byte_perm(lo, hi, 0x5410u);
+            }
+        }
+        xs[r] = X[0] + X[1] + X[2] + X[3] + X[4] + X[5] + X[6] + X[7];
+        const int t = t0 + r * NCT;
+        const int tsl = t / WPS, wi = t - tsl * WPS;
+        if (t < tasks) {
+            // word u = 6 (wi % 4) + i of chunk wi / 4 goes to load u / 4, lane u % 4
+            uint32_t *dst = planes + tsl * PSTRIDE + (wi >> 2) * 4;
+#pragma unroll
+            for (int h = 0; h < 3; ++h) {
+                const int u = (wi & 3) * 6 + 2 * h;
+                *reinterpret_cast<uint2 *>(dst + (u >> 2) * 4 * NCH + (u & 3)) = make_uint2(pw[2 * h], pw[2 * h + 1]);
+            }
+            if (wi == 0)
+                pp[m * a.spp + tsl] = (mx[r] >= 0x7F80u) ? __int_as_float(0x7FC00000) : (mx[r] == 0u ? 0.0f : exp2i(-S));
+        }
+    }
+    // sums of X per chunk of 32 k (4 tasks)
+#pragma unroll
+    for (int r = 0; r < XBN; ++r) xs[r] += __shfl_xor_sync(FULL, xs[r], 1);
+#pragma unroll
+    for (int r = 0; r < XBN; ++r) xs[r] += __shfl_xor_sync(FULL, xs[r], 2);
+#pragma unroll
+    for (int r = 0; r < XBN; ++r) {
+        const int t = t0 + r * NCT;
+        const int tsl = t / WPS, wi = t - tsl * WPS;
+        if (t < tasks && (wi & 3) == 0) sx[(m * a.spp + tsl) * NCH + (wi >> 2)] = xs[r];
+    }
+}
+
 template <int MT, int G>
 __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
     using GE_ = Geo<MT>;
@@ -212,7 +317,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
                 uint8_t *dst = smem + a.off_ring + (size_t)slot * a.SB;
                 if (a.kparts == 1) {
                     mbar_arrive_expect_tx(full + slot, (uint32_t)nr * a.RS);
-                    bulk_g2s(dst, src0 + (size_t)r0 * a.RS, (uint32_t)nr * a.RS, full + slot);
+                    bulk_g2s_stream(dst, src0 + (size_t)r0 * a.RS, (uint32_t)nr * a.RS, full + slot);
                 } else {
                     // this part's codes and scales of each row
                     const uint32_t cb = (uint32_t)(((k0 + (int64_t)nsl * KC < a.K ? k0 + (int64_t)nsl * KC : a.K) - k0) / 2);
@@ -221,8 +326,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
                     mbar_arrive_expect_tx(full + slot, (uint32_t)nr * (cb + scb));
                     for (int r = 0; r < nr; ++r) {
                         const uint8_t *rs = src0 + (size_t)(r0 + r) * a.RS;
-                        bulk_g2s(dst + (size_t)r * a.RSp, rs + k0 / 2, cb, full + slot);
-                        bulk_g2s(dst + (size_t)r * a.RSp + a.KPB, rs + scb0, scb, full + slot);
+                        bulk_g2s_stream(dst + (size_t)r * a.RSp, rs + k0 / 2, cb, full + slot);
+                        bulk_g2s_stream(dst + (size_t)r * a.RSp + a.KPB, rs + scb0, scb, full + slot);
                     }
                 }
                 ++issued;
@@ -249,81 +354,16 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
         float q16[MT], q16x256[MT], q16x65536[MT], sxf[MT][NSEG];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-            // (1) byte planes of activation row m0 + m, one task per 8 consecutive k; the loads
-            // of XB rounds of tasks are issued together so that their latencies overlap
+            // (1) byte planes of activation row m0 + m, one task per 8 consecutive k; a thread
+            // takes up to 4 rounds of tasks at once, every step done for all its rounds together
+            // so that the rounds' latencies (loads, shuffle chains) overlap
             const int tasks = a.spp * WPS;
-            constexpr int XB = 4;
-            for (int tb = 0; tb < tasks; tb += XB * NCT) {
-                uint4 xv[XB];
-#pragma unroll
-                for (int r = 0; r < XB; ++r) {
-                    const int t = tb + r * NCT + warp * 32 + lane;
-                    const int tsl = t / WPS, wi = t - tsl * WPS;
-                    const int64_t k = k0 + (int64_t)tsl * KC + wi * 8;
-                    const bool live = t < tasks && tsl < nsl && m0 + m < a.M && k < a.K;
-                    xv[r] = live ? __ldg(reinterpret_cast<const uint4 *>(a.x + (int64_t)(m0 + m) * a.K + k))
-                                 : make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int r = 0; r < XB; ++r) {
-                    if (tb + r * NCT + warp * 32 >= tasks) break;  // uniform over the warp
-                    const int t = tb + r * NCT + warp * 32 + lane;
-                    const int tsl = t / WPS, wi = t - tsl * WPS;
-                    const uint32_t e[4] = {xv[r].x, xv[r].y, xv[r].z, xv[r].w};
-                    // largest magnitude pattern of the slice (bf16 bits order like magnitudes)
-                    uint32_t mx = 0;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) mx = max(mx, max(e[i] & 0x7FFFu, (e[i] >> 16) & 0x7FFFu));
-#pragma unroll
-                    for (int off = WPS / 2; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(FULL, mx, off));
-                    // exponent of the largest |x|: |x| in [2^ex, 2^(ex+1))
-                    int ex;
-                    if (mx >= 0x80u) ex = (int)(mx >> 7) - 127;
-                    else ex = (31 - __clz((int)(mx | 1u))) - 133;
-                    const int S = 18 - ex;
-                    const float f1 = exp2i(S < 127 ? S : 127), f2 = exp2i(S < 127 ? 0 : S - 127);
-                    int X[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t bb = (i & 1) ? (e[i >> 1] >> 16) : (e[i >> 1] & 0xFFFFu);
-                        const float sv = __fmul_rn(__fmul_rn(__uint_as_float(bb << 16), f1), f2);
-                        X[i] = __float_as_int(__fadd_rn(sv, 12582912.0f)) - 0x4B400000;
-                    }
-                    if (mx >= 0x7F80u || mx == 0u) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) X[i] = 0;
-                    }
-                    // planes: even k as 16 X, odd k as X; byte p of each in 4-byte words
-                    uint32_t pw[6];
-#pragma unroll
-                    for (int par = 0; par < 2; ++par) {
-                        const uint32_t sh = par ? 0u : 4u;
-                        const uint32_t V0 = (uint32_t)X[par] << sh, V1 = (uint32_t)X[2 + par] << sh;
-                        const uint32_t V2 = (uint32_t)X[4 + par] << sh, V3 = (uint32_t)X[6 + par] << sh;
-#pragma unroll
-                        for (int pl = 0; pl < 3; ++pl) {
-                            const uint32_t lo = __byte_perm(V0, V1, (uint32_t)(pl | ((4 + pl) << 4)));
-                            const uint32_t hi = __byte_perm(V2, V3, (uint32_t)(pl | ((4 + pl) << 4)));
-                            pw[par * 3 + pl] = __byte_perm(lo, hi, 0x5410u);
-                        }
-                    }
-                    int xs = X[0] + X[1] + X[2] + X[3] + X[4] + X[5] + X[6] + X[7];
-                    xs += __shfl_xor_sync(FULL, xs, 1);
-                    xs += __shfl_xor_sync(FULL, xs, 2);
-                    if (t < tasks) {
-                        // word u = 6 (wi % 4) + i of chunk wi / 4 goes to load u / 4, lane u % 4
-                        uint32_t *dst = planes + tsl * PSTRIDE + (wi >> 2) * 4;
-#pragma unroll
-                        for (int h = 0; h < 3; ++h) {
-                            const int u = (wi & 3) * 6 + 2 * h;
-                            *reinterpret_cast<uint2 *>(dst + (u >> 2) * 4 * NCH + (u & 3)) = make_uint2(pw[2 * h], pw[2 * h + 1]);
-                        }
-                        if ((wi & 3) == 0) sx[(m * a.spp + tsl) * NCH + (wi >> 2)] = xs;
-                        if (wi == 0)
-                            pp[m * a.spp + tsl] =
-                                (mx >= 0x7F80u) ? __int_as_float(0x7FC00000) : (mx == 0u ? 0.0f : exp2i(-S));
-                    }
-                }
+            for (int tb = 0; tb < tasks; tb += 4 * NCT) {
+                const int nr = (tasks - tb + NCT - 1) / NCT;
+                if (nr >= 4) xprep_rounds<MT, 4>(a, planes, sx, pp, m, m0, k0, nsl, tb + warp * 32 + lane);
+                else if (nr == 3) xprep_rounds<MT, 3>(a, planes, sx, pp, m, m0, k0, nsl, tb + warp * 32 + lane);
+                else if (nr == 2) xprep_rounds<MT, 2>(a, planes, sx, pp, m, m0, k0, nsl, tb + warp * 32 + lane);
+                else xprep_rounds<MT, 1>(a, planes, sx, pp, m, m0, k0, nsl, tb + warp * 32 + lane);
             }
             named_bar_sync(1, NCT);
             // (2) this thread's planes of row m into registers

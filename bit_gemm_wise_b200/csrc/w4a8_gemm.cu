@@ -824,15 +824,27 @@ struct Smem {
 };
 static_assert(sizeof(Smem) <= 1024, "control block");
 
-// instruction descriptor: D fp32, A and B fp16, both K-major, N = BN, M = BM
-constexpr uint32_t kIdescF16 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// instruction descriptor: D fp32, A and B fp16, both K-major, M = BM, N = n (a multiple of 16
+// up to BN: a tile's last token columns past its rows are not computed)
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t n) {
+    return (1u << 4) | ((n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
 
-__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint32_t a_lo, uint32_t b_lo, uint32_t accumulate) {
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                        uint32_t accumulate) {
     asm volatile(
         "{\n .reg .pred p;\n .reg .b64 da, db;\n setp.ne.b32 p, %4, 0;\n"
         " mov.b64 da, {%1, %5};\n mov.b64 db, {%2, %5};\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n}\n" ::"r"(tmem_d),
-        "r"(a_lo), "r"(b_lo), "r"(kIdescF16), "r"(accumulate), "r"(kDescHiSW128));
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kDescHiSW128));
+}
+
+// token columns of tile T that hold rows of its problem, rounded up to the MMA's N granule
+__device__ __forceinline__ uint32_t tile_cols16(const Args &a, const Tile &T) {
+    int64_t c = T.rows < (int64_t)BN ? T.rows : (int64_t)BN;
+    const int64_t lim_m = a.M - T.row0;
+    if (c > lim_m) c = lim_m;
+    return (uint32_t)((c + 15) / 16 * 16);
 }
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
@@ -929,6 +941,7 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
                 if (!wait_f(&sm->acc_empty[b], ((tiles_done >> 1) & 1u) ^ 1u, sm, a.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + b * BN;
+                const uint32_t idesc = idesc_f16(tile_cols16(a, T));
                 for (int s = 0; s < KT; ++s, r.next()) {
                     if (!wait_f(&sm->exp_full[r.slot], r.phase, sm, a.status)) { ok = false; break; }
                     tc_fence_after();
@@ -936,8 +949,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
                     const uint32_t bLo = st + (OFF_B >> 4), hLo = st + (OFF_AH >> 4), lLo = st + (OFF_AL >> 4);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {  // K = 16 per fp16 MMA: 32 bytes
-                        mma_f16(d, hLo + kk * 2, bLo + kk * 2, (s > 0 || kk > 0) ? 1u : 0u);
-                        mma_f16(d, lLo + kk * 2, bLo + kk * 2, 1u);
+                        mma_f16(d, hLo + kk * 2, bLo + kk * 2, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                        mma_f16(d, lLo + kk * 2, bLo + kk * 2, idesc, 1u);
                     }
                     mma_commit(&sm->empty[r.slot]);
                     ++uses;
@@ -970,8 +983,9 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
             const bool vec = !a.out_fp32 && (a.N & 7) == 0;
             const int64_t nbase = T.n0 + quarter * 32 + 8 * (lane >> 3);
             const int li = lane & 7;
+            const int nchunks = (int)((ncol + 15) / 16);  // TMEM columns the MMAs wrote
 #pragma unroll 1
-            for (int c = 0; c < BN / 16; ++c) {
+            for (int c = 0; c < nchunks; ++c) {
                 uint32_t v[16];
                 tmem_ld16(tl_addr + c * 16, v);
                 // token scale of column 16c + (lane & 15)
@@ -1031,12 +1045,19 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_f16split_kernel(const __grid_
             const int64_t n = T.n0 + wr;
             const uint32_t *scales =
                 reinterpret_cast<const uint32_t *>(a.packed + (size_t)T.e * a.slab_bytes + a.codes_bytes);
-            // this thread's scale entry for stage s is loaded one stage ahead (it does not
-            // depend on the ring): k = 64 s + 32 wh + 0..31 lies in group (64 s + 32 wh) / g
-            uint32_t ent_next = scales[(int64_t)(wh * 32 / a.g) * a.Npad + n];
+            // this thread's scale entry for stage s (k = 64 s + 32 wh + 0..31 lies in group
+            // (64 s + 32 wh) / g) is loaded four stages ahead, in a queue of registers: it does not
+            // depend on the ring, and an L2 load under the weight stream takes about a stage
+            auto ent_at = [&](int st) -> uint32_t {
+                return st < KT ? __ldg(scales + ((int64_t)st * BK + wh * 32) / a.g * a.Npad + n) : 0u;
+            };
+            uint32_t q0 = ent_at(0), q1 = ent_at(1), q2 = ent_at(2), q3 = ent_at(3);
             for (int s = 0; s < KT; ++s, r.next()) {
-                const uint32_t ent = ent_next;
-                if (s + 1 < KT) ent_next = scales[((int64_t)(s + 1) * BK + wh * 32) / a.g * a.Npad + n];
+                const uint32_t ent = q0;
+                q0 = q1;
+                q1 = q2;
+                q2 = q3;
+                q3 = ent_at(s + 4);
                 // the stage was refilled only after the MMAs that read its previous A_hi and
                 // A_lo completed, so once its TMA bytes landed both buffers are free
                 if (!warp_wait_f(&sm->full[r.slot], r.phase, sm, a.status)) { ok = false; break; }

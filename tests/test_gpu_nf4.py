@@ -55,12 +55,15 @@ def test_quantize_edge_blocks():
 
 
 def test_ragged_rows_and_long_k():
-    for N, K in [(1, 64), (37, 576), (5, 28672)]:
+    # the first three take the general kernel; the rest the one-block-per-SM kernel for M = 1
+    # and K a multiple of 1024 up to 16384 (single rows, ragged row runs, the longest rows,
+    # more rows than 148 blocks of 256 hold)
+    for N, K in [(1, 64), (37, 576), (5, 28672), (1, 1024), (149, 2048), (300, 16384), (40000, 1024)]:
         W = synth.student_t3_weight(N, K, 3, N + K)
         codes, a = gpu_nf4(W)
         rc, ra = oracle.nf4_quantize(synth.bf16_bits(W))
         x = synth.normal((1, K), 1.0, 3, K)
-        y = torch.empty(1, N, dtype=torch.float32, device=cuda())
+        y = torch.full((1, N), float("nan"), dtype=torch.float32, device=cuda())
         w4.w4_nf4_gemv(x.to(cuda()), 1, codes, a, N, K, y, w4.W4_OUT_FP32)
         ref = oracle.nf4_gemv_ref(synth.bf16_bits(x), rc, ra)
         torch.cuda.synchronize()
