@@ -187,13 +187,18 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) gemv_kernel(const uint16_t *_
 // thread (slot, sl) takes the 16-byte code chunk sl (32 weights, half an NF4 block) of the rows
 // slot, slot + nslot, ... and holds its 32 activations in registers. The code chunks and block
 // scales of the next PF rows are loaded ahead in registers (issued before the dependency wait
-// under programmatic launch). Each code is looked up in a 16-entry fp32 table in shared
+// under programmatic launch), and the chunks PF rows beyond those are prefetched into L2, so
+// that the register loads find them there. Each code is looked up in a 16-entry fp32 table in shared
 // memory (one entry per bank, so any lookup pattern is conflict-free) and multiplied into one
 // of four fp32 sums; the chunk's sum times the block scale is reduced over the warp, then over
 // the row's warps in order.
 constexpr int RT = 512;
 constexpr int PF = 4;
 constexpr int MAX_RPB = 256;
+
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 
 __device__ __forceinline__ float lut_at(const float *lut, uint32_t byte_off) {
     return *reinterpret_cast<const float *>(reinterpret_cast<const char *>(lut) + byte_off);
@@ -224,6 +229,7 @@ __global__ void __launch_bounds__(RT, 1) gemv_rows_kernel(const uint16_t *__rest
         const bool ok = p < nr;
         cq[p] = ok ? __ldg(reinterpret_cast<const uint4 *>(codes + n * rb) + sl) : make_uint4(0u, 0u, 0u, 0u);
         aq[p] = ok ? __ldg(absmax + n * ab + (sl >> 1)) : 0.0f;
+        if (p + PF < nr) prefetch_l2(reinterpret_cast<const uint4 *>(codes + (n + (int64_t)PF * nslot) * rb) + sl);
     }
     __syncthreads();
     if (pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -255,6 +261,7 @@ __global__ void __launch_bounds__(RT, 1) gemv_rows_kernel(const uint16_t *__rest
             const bool ok = i + PF < nr;
             cq[PF - 1] = ok ? __ldg(reinterpret_cast<const uint4 *>(codes + n * rb) + sl) : make_uint4(0u, 0u, 0u, 0u);
             aq[PF - 1] = ok ? __ldg(absmax + n * ab + (sl >> 1)) : 0.0f;
+            if (i + 2 * PF < nr) prefetch_l2(reinterpret_cast<const uint4 *>(codes + (n + (int64_t)PF * nslot) * rb) + sl);
         }
         const uint32_t wv[4] = {c.x, c.y, c.z, c.w};
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
