@@ -234,6 +234,12 @@ class Decode:
         for si in range(len(self.shapes)):
             self.gemv(si, i)
 
+    def step_grouped(self, i):
+        """The step's four GEMVs as one grouped launch (w4a16_gemv_grouped)."""
+        self.w4.w4a16_gemv_grouped(self.x, self.M, [p[(i % self.R) * nb:] for p, nb in self.packed],
+                                   [N for K, N in self.shapes], [K for K, N in self.shapes], 128, "asym", self.y,
+                                   self.flags)
+
     def graph_of(self, n_steps, first=0):
         """One CUDA graph holding n_steps consecutive decode steps (weights rotate over the
         copies), the GEMVs chained with programmatic dependent launches, as a decode graph
@@ -396,6 +402,27 @@ def measure_rows(args, dev, pk):
     # GEMV at M = 4 and 16 (bound by the CUDA cores' issue rate): GB/s, and the FMA work as a
     # fraction of the CUDA-core fp32 FMA peak (148 SMs x 128 lanes x 2 flop x 1965 MHz)
     fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    if "gemv" in want:
+        # the same M = 1 decode step as one grouped launch of its four independent GEMVs (the
+        # per-launch phases paid once per step instead of once per GEMV), graph-replayed
+        d = Decode(1, args.seed, dev)
+        d.step_grouped(0)
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        n = 8 * d.R
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=side):
+            for i in range(n):
+                d.step_grouped(i)
+        gr.replay()
+        ms = float(np.median([time_region(lambda i: gr.replay(), 1) for _ in range(9)])) / n
+        gbps = d.bytes_per_step / (ms * 1e-3) / 1e9
+        rows["w4a16_gemv_grouped_step_M1"] = {
+            "value": round(gbps, 1), "unit": "GB/s", "us_per_step": round(ms * 1e3, 2),
+            "roofline": {"bound": "hbm", "achieved": round(gbps, 1), "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": round(gbps / pk["hbm"], 4)},
+            "note": "the headline's four decode GEMVs (same bytes) as one w4a16_gemv_grouped launch per step"}
+        del d, gr
     for M in ((4, 16) if "gemv" in want else ()):
         d = Decode(M, args.seed, dev)
         d.capture(6 * d.R, 3)

@@ -254,8 +254,10 @@ __device__ __forceinline__ void xprep_rounds(const Args &a, uint32_t *planes, in
     }
 }
 
+// The work of one block: row block bx (and K part), activation rows by * MT ... of the
+// problem a.
 template <int MT, int G>
-__global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
+__device__ __forceinline__ void gemv_block(const Args &a, const int bx, const int by) {
     using GE_ = Geo<MT>;
     constexpr int KC = GE_::KC, NCH = GE_::NCH, WPS = GE_::WPS, PSTRIDE = GE_::PSTRIDE;
     constexpr int GS = G < KC ? G : KC;       // k per combine segment
@@ -275,9 +277,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
     uint32_t *planes = reinterpret_cast<uint32_t *>(smem + a.off_planes);  // [spp][PSTRIDE], one row m at a time
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int kp = (int)(blockIdx.x % (unsigned)a.kparts);
-    const int rb = (int)(blockIdx.x / (unsigned)a.kparts);
-    const int m0 = (int)blockIdx.y * MT;
+    const int kp = (int)((unsigned)bx % (unsigned)a.kparts);
+    const int rb = (int)((unsigned)bx / (unsigned)a.kparts);
+    const int m0 = by * MT;
     const int64_t row0 = (int64_t)rb * a.rpc;
     const int rows = (int)((a.N - row0) < a.rpc ? (a.N - row0) : a.rpc);
     const int nstages = (rows + a.nslot * a.rpt - 1) / (a.nslot * a.rpt);
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
             // the last block of the row range to arrive adds the parts in order and resets the counter
             __threadfence();
             named_bar_sync(1, NCT);
-            int *cnt = a.ws_count + (size_t)blockIdx.y * a.nrb + rb;
+            int *cnt = a.ws_count + (size_t)by * a.nrb + rb;
             if (tid == 0) {
                 const int prev = atomicAdd(cnt, 1);
                 *last_flag = (prev == a.kparts - 1) ? 1 : 0;
@@ -562,6 +564,28 @@ __global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const Args a) {
     }
 }
 
+template <int MT, int G>
+__global__ void __launch_bounds__(THREADS, 1) gemv_kernel(const __grid_constant__ Args a) {
+    gemv_block<MT, G>(a, (int)blockIdx.x, (int)blockIdx.y);
+}
+
+// Several independent problems in one launch: blocks [first[j], first[j+1]) work on problem j
+// (whole rows, one K part each), so the per-launch phases (activation conversion, first
+// stage, row sums) are paid once for the group.
+constexpr int MAX_GROUP = 8;
+struct GroupArgs {
+    Args m[MAX_GROUP];
+    int first[MAX_GROUP + 1];
+    int count;
+};
+
+template <int MT, int G>
+__global__ void __launch_bounds__(THREADS, 1) gemv_grouped_kernel(const __grid_constant__ GroupArgs ga) {
+    int j = 0;
+    while (j + 1 < ga.count && (int)blockIdx.x >= ga.first[j + 1]) ++j;
+    gemv_block<MT, G>(ga.m[j], (int)blockIdx.x - ga.first[j], (int)blockIdx.y);
+}
+
 // ------------------------------------------------------------------ host side
 
 struct Plan {
@@ -579,7 +603,8 @@ static int sm_count_cached() {
 }
 
 template <int MT>
-static bool make_plan_parts(Plan &p, int64_t M, int64_t N, int64_t K, int g, int64_t S, int want_parts) {
+static bool make_plan_parts(Plan &p, int64_t M, int64_t N, int64_t K, int g, int64_t S, int want_parts,
+                            int64_t red_budget = RED_BUDGET) {
     using GE_ = Geo<MT>;
     const GemvLayout L = gemv_layout(N, K, g);
     Args &a = p.a;
@@ -621,7 +646,7 @@ static bool make_plan_parts(Plan &p, int64_t M, int64_t N, int64_t K, int g, int
     // widest padding of a (row, m)'s partials, nred + 31 words)
     int64_t nrb = S < N ? S : N;
     int64_t rpc = (N + nrb - 1) / nrb;
-    const int64_t rpc_cap = RED_BUDGET / ((int64_t)MT * (a.nred + 31) * 4);
+    const int64_t rpc_cap = red_budget / ((int64_t)MT * (a.nred + 31) * 4);
     if (rpc_cap < 1) return false;
     if (rpc > rpc_cap) rpc = rpc_cap;
     a.rpc = (int)rpc;
@@ -739,6 +764,84 @@ static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, in
     return launch_status();
 }
 
+// Plans of a group of problems launched together: problem j gets a share of the SMs in
+// proportion to its bytes, whole rows per block and one K part; blocks may hold more rows than
+// in a single launch (a larger row-partial buffer, at least two ring stages), so that the group
+// fits one wave. All problems must take the same activation rows per sweep.
+static bool make_group_plan(int count, int64_t M, const int64_t *N, const int64_t *K, int g, int64_t sms, Plan *pl,
+                            int *first) {
+    double total = 0.0;
+    for (int j = 0; j < count; ++j) total += (double)N[j] * (double)K[j] * (0.5 + 4.0 / g);
+    first[0] = 0;
+    for (int j = 0; j < count; ++j) {
+        const double share = (double)N[j] * (double)K[j] * (0.5 + 4.0 / g) / total;
+        int64_t S = (int64_t)(share * (double)sms);
+        if (S < 1) S = 1;
+        bool ok = false;
+        const int want = M >= 3 ? 4 : (int)M;
+        for (int64_t rb = 3 * RED_BUDGET; rb >= RED_BUDGET && !ok; rb -= RED_BUDGET / 2) {
+            if (want >= 4) ok = make_plan_parts<4>(pl[j], M, N[j], K[j], g, S, 1, rb);
+            else if (want == 2) ok = make_plan_parts<2>(pl[j], M, N[j], K[j], g, S, 1, rb);
+            else ok = make_plan_parts<1>(pl[j], M, N[j], K[j], g, S, 1, rb);
+        }
+        if (!ok || pl[j].a.kparts != 1 || pl[j].MT != pl[0].MT || pl[j].sweeps != pl[0].sweeps)
+            return false;
+        first[j + 1] = first[j] + pl[j].grid_x;
+    }
+    return true;
+}
+
+template <int MT>
+static void *grouped_kernel_ptr(int g) {
+    return g == 32 ? reinterpret_cast<void *>(gemv_grouped_kernel<MT, 32>)
+         : g == 64 ? reinterpret_cast<void *>(gemv_grouped_kernel<MT, 64>)
+                   : reinterpret_cast<void *>(gemv_grouped_kernel<MT, 128>);
+}
+
+static w4_status run_grouped(int count, const void *const *x, int64_t M, const void *const *packed, const int64_t *N,
+                             const int64_t *K, int g, void *const *y, int out_fp32, int pdl, cudaStream_t stream) {
+    Plan pl[MAX_GROUP];
+    GroupArgs ga{};
+    if (!make_group_plan(count, M, N, K, g, sm_count_cached(), pl, ga.first)) return W4_ERR_UNSUPPORTED;
+    int smem = 0;
+    for (int j = 0; j < count; ++j) {
+        Args &a = pl[j].a;
+        a.x = static_cast<const uint16_t *>(x[j]);
+        a.w = static_cast<const uint8_t *>(packed[j]);
+        a.y = y[j];
+        a.out_fp32 = out_fp32;
+        a.status = device_status_ptr();
+        a.pdl = pdl;
+        ga.m[j] = a;
+        if (pl[j].smem > smem) smem = pl[j].smem;
+    }
+    ga.count = count;
+    const int MT = pl[0].MT;
+    void *fn = MT == 4 ? grouped_kernel_ptr<4>(g) : MT == 2 ? grouped_kernel_ptr<2>(g) : grouped_kernel_ptr<1>(g);
+    static int attr_done[64][3][3] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int mi = MT == 4 ? 2 : MT - 1, gi = g == 32 ? 0 : (g == 64 ? 1 : 2);
+    if (dev >= 0 && dev < 64 && !attr_done[dev][mi][gi]) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_MAX) != cudaSuccess)
+            return W4_ERR_CUDA;
+        attr_done[dev][mi][gi] = 1;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ga.first[count], (unsigned)pl[0].sweeps);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *args[] = {&ga};
+    if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return W4_ERR_CUDA;
+    return launch_status();
+}
+
 // Host-only view of a plan: out = {activation rows per sweep, sweeps, K parts, row blocks,
 // rows per block, dynamic shared memory bytes, ring stages, workspace bytes}.
 static bool describe_plan(int64_t M, int64_t N, int64_t K, int g, int64_t sms, int64_t *out) {
@@ -802,6 +905,39 @@ W4_API w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, i
     if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(y) || (workspace && !aligned16(workspace)))
         return W4_ERR_ALIGN;
     return gemv::run(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
+}
+
+W4_API w4_status w4a16_gemv_grouped(int count, const void *const *x_bf16, int64_t M, const void *const *packed,
+                                    const int64_t *N, const int64_t *K, int group, int mode, void *const *y,
+                                    int flags, cudaStream_t stream) {
+    if (!x_bf16 || !packed || !N || !K || !y) return W4_ERR_NULL;
+    if (count < 1 || count > gemv::MAX_GROUP) return W4_ERR_SHAPE;
+    if (!valid_mode(mode) || (flags & ~(W4_OUT_FP32 | W4_OVERLAP_PREVIOUS))) return W4_ERR_ARG;
+    if (!valid_group(group)) return W4_ERR_GROUP;
+    for (int j = 0; j < count; ++j) {
+        if (!x_bf16[j] || !packed[j] || !y[j]) return W4_ERR_NULL;
+        if (!gemv_shape_ok(M, N[j], K[j])) return W4_ERR_SHAPE;
+        if (K[j] % group != 0) return W4_ERR_GROUP;
+        if (!aligned16(x_bf16[j]) || !aligned16(packed[j]) || !aligned16(y[j])) return W4_ERR_ALIGN;
+    }
+    return gemv::run_grouped(count, x_bf16, M, packed, N, K, group, y, (flags & W4_OUT_FP32) ? 1 : 0,
+                             (flags & W4_OVERLAP_PREVIOUS) ? 1 : 0, stream);
+}
+
+// Host-only: the blocks of each problem of a grouped launch on `sms` SMs (0 if the group is not
+// supported).
+W4_API w4_status w4a16_gemv_grouped_schedule(int count, int64_t M, const int64_t *N, const int64_t *K, int group,
+                                             int sms, int64_t *blocks) {
+    if (!N || !K || !blocks) return W4_ERR_NULL;
+    if (count < 1 || count > gemv::MAX_GROUP || sms < 1 || sms > 4096) return W4_ERR_SHAPE;
+    if (!valid_group(group)) return W4_ERR_GROUP;
+    for (int j = 0; j < count; ++j)
+        if (!gemv_shape_ok(M, N[j], K[j]) || K[j] % group != 0) return W4_ERR_SHAPE;
+    gemv::Plan pl[gemv::MAX_GROUP];
+    int first[gemv::MAX_GROUP + 1];
+    if (!gemv::make_group_plan(count, M, N, K, group, sms, pl, first)) return W4_ERR_UNSUPPORTED;
+    for (int j = 0; j < count; ++j) blocks[j] = first[j + 1] - first[j];
+    return W4_OK;
 }
 
 // ------------------------------------------------------------------ allocation-free variant

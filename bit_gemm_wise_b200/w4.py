@@ -49,6 +49,8 @@ SIGNATURES = [
     ("w4a16_gemv_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a16_gemv_noalloc_scratch_limit", _SZ, []),
+    ("w4a16_gemv_grouped", _I, [_I, _P, _I64, _P, _P, _P, _I, _I, _P, _I, _P]),
+    ("w4a16_gemv_grouped_schedule", _I, [_I, _I64, _P, _P, _I, _I, _P]),
     ("w4a16_gemv_noalloc", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P]),
     ("w4a8_gemm", _I, [_P, _P, _P, _P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a8_gemm_workspace_bytes", _SZ, [_I64, _I64, _I64, _I]),
@@ -222,6 +224,27 @@ def w4a16_gemv(x, M, packed, N, K, group, mode, y, flags, workspace, stream=None
                           _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _check("w4a16_gemv", rc)
+
+
+def w4a16_gemv_grouped(xs, M, packeds, Ns, Ks, group, mode, ys, flags, stream=None):
+    """Independent GEMVs (same M, group, mode) in one launch; lists of tensors and sizes."""
+    n = len(xs)
+    P = ctypes.c_void_p * n
+    L = ctypes.c_int64 * n
+    rc = lib().w4a16_gemv_grouped(n, P(*[_ptr(t) for t in xs]), M, P(*[_ptr(t) for t in packeds]),
+                                  L(*Ns), L(*Ks), group, _mode(mode), P(*[_ptr(t) for t in ys]), int(flags),
+                                  _stream(stream))
+    _check("w4a16_gemv_grouped", rc)
+
+
+def w4a16_gemv_grouped_schedule(M, Ns, Ks, group, sms):
+    """Host-only: blocks per problem of a grouped launch on `sms` SMs."""
+    n = len(Ns)
+    out = (ctypes.c_int64 * n)()
+    L = ctypes.c_int64 * n
+    _check("w4a16_gemv_grouped_schedule",
+           lib().w4a16_gemv_grouped_schedule(n, M, L(*Ns), L(*Ks), group, sms, ctypes.cast(out, _P)))
+    return [int(v) for v in out]
 
 
 def w4a16_gemv_noalloc_scratch_limit() -> int:

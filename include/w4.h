@@ -215,6 +215,29 @@ w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t 
                      size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * w4a16_gemv_grouped -- `count` independent w4a16_gemv problems in one launch (for example the
+ *   q, k and v projections of a layer, or its gate and up projections, which read the same
+ *   activations): problem j computes y[j] = x[j] W_j^T exactly as w4a16_gemv does, with the
+ *   same M, group and mode for all. Each problem gets a share of the SMs in proportion to its
+ *   weight bytes and whole weight rows per block, so the launch's fixed phases (activation
+ *   conversion, first stage, row sums) are paid once for the group.
+ *   x_bf16, packed, y   HOST arrays of `count` device pointers (layouts as w4a16_gemv)
+ *   N, K                HOST arrays of `count` sizes
+ *   1 <= count <= 8; flags as w4a16_gemv. No workspace: every problem's rows must fit one
+ *   block's K range (K <= 57344 at M = 1, as for w4a16_gemv without a workspace), and all
+ *   problems must take the same activation rows per sweep. Errors: NULL / SHAPE / GROUP / ARG /
+ *   ALIGN / UNSUPPORTED (a group the planner cannot place) / CUDA.
+ *
+ * w4a16_gemv_grouped_schedule -- host-only query: blocks[j] receives the blocks of problem j in
+ *   such a launch on `sms` SMs. Errors: NULL / SHAPE / GROUP / UNSUPPORTED.
+ */
+w4_status w4a16_gemv_grouped(int count, const void *const *x_bf16, int64_t M,
+                             const void *const *packed, const int64_t *N, const int64_t *K,
+                             int group, int mode, void *const *y, int flags, cudaStream_t stream);
+w4_status w4a16_gemv_grouped_schedule(int count, int64_t M, const int64_t *N, const int64_t *K,
+                                      int group, int sms, int64_t *blocks);
+
+/*
  * w4a16_gemv_noalloc -- w4a16_gemv for callers that cannot allocate device memory.
  *   (No counterpart in the source pages: this is a calling convention, not part of the
  *   method.) Some callers must not call cudaMalloc on their hot path: a plug-in running

@@ -311,3 +311,28 @@ def test_nf4_levels_of_the_library_equal_the_oracle(lib):
     they must equal the oracle's bit for bit (both round the same double values to fp32)."""
     import oracle
     assert np.array_equal(np.array(w4.w4_nf4_levels(), np.float32), oracle.nf4_levels())
+
+
+def test_gemv_grouped_schedule_fits_one_wave_and_validates(lib):
+    """The decode sweep's four GEMVs as one grouped launch: one block per SM at most, each
+    problem a share in proportion to its bytes; invalid groups are rejected before any launch."""
+    Ks, Ns = [4096, 4096, 4096, 14336], [4096, 1024, 14336, 4096]
+    for sms in (148, 132):
+        b = w4.w4a16_gemv_grouped_schedule(1, Ns, Ks, 128, sms)
+        assert sum(b) <= sms and min(b) >= 1
+        assert b[2] > b[0] > b[1]  # more bytes, more blocks
+    small = w4.w4a16_gemv_grouped_schedule(1, [77, 5], [320, 4096], 64, 148)
+    assert small == [77, 5]  # tiny problems: one row per block within the share
+    P = ctypes.c_void_p * 2
+    L = ctypes.c_int64 * 2
+    ptrs = P(FAKE, FAKE)
+    assert rc("w4a16_gemv_grouped", 0, ptrs, 1, ptrs, L(16, 16), L(128, 128), 128, 1, ptrs, 0, None) == 2
+    assert rc("w4a16_gemv_grouped", 9, ptrs, 1, ptrs, L(16, 16), L(128, 128), 128, 1, ptrs, 0, None) == 2
+    assert rc("w4a16_gemv_grouped", 2, None, 1, ptrs, L(16, 16), L(128, 128), 128, 1, ptrs, 0, None) == 1
+    assert rc("w4a16_gemv_grouped", 2, P(FAKE, None), 1, ptrs, L(16, 16), L(128, 128), 128, 1, ptrs, 0, None) == 1
+    assert rc("w4a16_gemv_grouped", 2, ptrs, 1, ptrs, L(16, 16), L(128, 96), 64, 1, ptrs, 0, None) == 3
+    assert rc("w4a16_gemv_grouped", 2, P(FAKE, FAKE + 8), 1, ptrs, L(16, 16), L(128, 128), 128, 1, ptrs, 0,
+              None) == 4
+    assert rc("w4a16_gemv_grouped", 2, ptrs, 1, ptrs, L(16, 16), L(128, 128), 128, 3, ptrs, 0, None) == 5
+    # rows too long for one block (a K split would need a workspace): unsupported in a group
+    assert rc("w4a16_gemv_grouped", 2, ptrs, 1, ptrs, L(16, 16), L(128, 65536), 128, 1, ptrs, 0, None) == 6

@@ -205,3 +205,56 @@ def test_overlapped_chain_reads_predecessor_output():
         got = bufs[3].float().cpu().numpy().astype(np.float64)
         assert rel_frob(bf16_round(ref), got) <= 2e-3
     assert w4.w4_device_status() == 0
+
+
+def upload_gemv(codes, scales, zeros, N, K, group, mode):
+    packed = w4.alloc_packed(N, K, group, w4.W4_LAYOUT_GEMV)
+    w4.w4_prepack(to_dev(codes), to_dev(scales.view(np.int16)), to_dev(zeros) if zeros is not None else None,
+                  N, K, group, mode, w4.W4_LAYOUT_GEMV, packed)
+    return packed
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_grouped_decode_shapes(M):
+    """The four decode GEMVs as one grouped launch: every problem against the oracle, both
+    output types."""
+    probs = []
+    for K, N in synth.DECODE_SHAPES:
+        codes, scales, zeros = quantized("decode", K, N, 128, "asym", "twenty")
+        x_bits = synth.bf16_bits(synth.decode_activation(M, K, 0))
+        probs.append((K, N, upload_gemv(codes, scales, zeros, N, K, 128, "asym"), x_bits,
+                      oracle.gemv_ref(x_bits, codes, scales, zeros, 128, "asym")))
+    xs = [to_dev(p[3].view(np.int16)).view(torch.bfloat16) for p in probs]
+    for out_fp32 in (1, 0):
+        dt = torch.float32 if out_fp32 else torch.bfloat16
+        ys = [torch.full((M, N), float("nan"), dtype=dt, device=cuda()) for K, N, *_ in probs]
+        w4.w4a16_gemv_grouped(xs, M, [p[2] for p in probs], [p[1] for p in probs], [p[0] for p in probs], 128,
+                              "asym", ys, w4.W4_OUT_FP32 if out_fp32 else 0)
+        torch.cuda.synchronize()
+        assert w4.w4_device_status() == 0
+        for (K, N, _, _, ref), y in zip(probs, ys):
+            got = y.double().cpu().numpy()
+            assert np.isfinite(got).all()
+            if out_fp32:
+                assert rel_frob(ref, got) <= 1e-4, (K, N)
+            else:
+                assert rel_frob(bf16_round(ref), got) <= 1e-3, (K, N)
+
+
+def test_grouped_ragged_shapes_group_64():
+    """Unequal, ragged problems in one group: one row per block for the small ones."""
+    M, g = 1, 64
+    probs = []
+    for N, K in [(77, 320), (5, 4096), (1000, 2048)]:
+        codes, scales, zeros = quantized("t3", K, N, g, "asym", "one")
+        x_bits = synth.bf16_bits(synth.normal((M, K), 1.0, 3, K + N))
+        probs.append((K, N, upload_gemv(codes, scales, zeros, N, K, g, "asym"), x_bits,
+                      oracle.gemv_ref(x_bits, codes, scales, zeros, g, "asym")))
+    xs = [to_dev(p[3].view(np.int16)).view(torch.bfloat16) for p in probs]
+    ys = [torch.full((M, N), float("nan"), dtype=torch.float32, device=cuda()) for K, N, *_ in probs]
+    w4.w4a16_gemv_grouped(xs, M, [p[2] for p in probs], [p[1] for p in probs], [p[0] for p in probs], g, "asym",
+                          ys, w4.W4_OUT_FP32)
+    torch.cuda.synchronize()
+    assert w4.w4_device_status() == 0
+    for (K, N, _, _, ref), y in zip(probs, ys):
+        assert rel_frob(ref, y.double().cpu().numpy()) <= 1e-4, (K, N)
