@@ -186,32 +186,22 @@ __device__ __forceinline__ void xprep_rounds(const Args &a, uint32_t *planes, in
 #pragma unroll
     for (int r = 0; r < XBN; ++r) {
         const uint32_t e[4] = {xv[r].x, xv[r].y, xv[r].z, xv[r].w};
-        // exponent of the largest |x|: |x| in [2^ex, 2^(ex+1))
-        int ex;
-        if (mx[r] >= 0x80u) ex = (int)(mx[r] >> 7) - 127;
-        else ex = (31 - __clz((int)(mx[r] | 1u))) - 133;
-        const int S = 18 - ex;
-        const float f1 = exp2i(S < 127 ? S : 127), f2 = exp2i(S < 127 ? 0 : S - 127);
+        // exponent of the largest |x|: |x| in [2^ex, 2^(ex+1)); every step below is a select,
+        // not a branch, so that the rounds of a thread interleave
+        const int ex = mx[r] >= 0x80u ? (int)(mx[r] >> 7) - 127 : (31 - __clz((int)(mx[r] | 1u))) - 133;
+        const int S = 18 - ex;  // -109 <= S <= 151
+        // x 2^S as two exact power-of-two products (2^S alone leaves the fp32 range when the
+        // slice's largest |x| is below 2^-109): 2^min(S, 127), then 2^max(S - 127, 0)
+        const float f1 = __int_as_float(((S < 127 ? S : 127) + 127) << 23);
+        const float f2 = __int_as_float(((S > 127 ? S - 127 : 0) + 127) << 23);
+        const bool zero = mx[r] >= 0x7F80u || mx[r] == 0u;  // infinity / NaN, or all zero
         int X[8];
-        // x 2^S is exact (a power of two; |x 2^S| < 2^19); only slices whose largest |x| is
-        // below 2^-109 need the second factor (a warp-uniform branch)
-        if (__any_sync(FULL, S > 127)) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t bb = (i & 1) ? (e[i >> 1] >> 16) : (e[i >> 1] & 0xFFFFu);
-                const float sv = __fmul_rn(__fmul_rn(__uint_as_float(bb << 16), f1), f2);
-                X[i] = __float_as_int(__fadd_rn(sv, 12582912.0f)) - 0x4B400000;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t bb = (i & 1) ? (e[i >> 1] & 0xFFFF0000u) : (e[i >> 1] << 16);
-                X[i] = __float_as_int(__fmaf_rn(__uint_as_float(bb), f1, 12582912.0f)) - 0x4B400000;
-            }
-        }
-        if (mx[r] >= 0x7F80u || mx[r] == 0u) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) X[i] = 0;
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t bb = (i & 1) ? (e[i >> 1] & 0xFFFF0000u) : (e[i >> 1] << 16);
+            const float sv = __fmul_rn(__fmul_rn(__uint_as_float(bb), f1), f2);
+            const int v = __float_as_int(__fadd_rn(sv, 12582912.0f)) - 0x4B400000;
+            X[i] = zero ? 0 : v;
         }
         uint32_t pw[6];
 #pragma unroll
@@ -237,8 +227,10 @@ __device__ __forceinline__ void xprep_rounds(const Args &a, uint32_t *planes, in
                 const int u = (wi & 3) * 6 + 2 * h;
                 *reinterpret_cast<uint2 *>(dst + (u >> 2) * 4 * NCH + (u & 3)) = make_uint2(pw[2 * h], pw[2 * h + 1]);
             }
+            // 2^-S: normal for S <= 126, subnormal up to S = 149 (0 beyond)
+            const float p2 = S <= 126 ? __int_as_float((127 - S) << 23) : (S <= 149 ? __int_as_float(1 << (149 - S)) : 0.0f);
             if (wi == 0)
-                pp[m * a.spp + tsl] = (mx[r] >= 0x7F80u) ? __int_as_float(0x7FC00000) : (mx[r] == 0u ? 0.0f : exp2i(-S));
+                pp[m * a.spp + tsl] = (mx[r] >= 0x7F80u) ? __int_as_float(0x7FC00000) : (mx[r] == 0u ? 0.0f : p2);
         }
     }
     // sums of X per chunk of 32 k (4 tasks)
