@@ -52,10 +52,10 @@ def peaks():
 # unchanged (otherwise the counters describe a different kernel and "traffic" is null).
 NCU_TRAFFIC = {
     # profiles/w4a16_gemv_m1_k14336_n4096_full.md
-    "w4a16_gemv M1 K14336xN4096": {"bytes": 31291392, "sha1": "b9df13a9adb45b242564e48ea1f1fe0f076ba785"},
-    # profiles/w4a8_gemm_prefill_k3840_n15360_full.md, profiles/w4a8_gemm_prefill_k15360_n3840_split_full.md
-    "w4a8_gemm M4096 K3840xN15360": {"bytes": 158694400, "sha1": "76f8ca5ba6de39985105f48ae8820d0cae4e1f55"},
-    "w4a8_gemm M4096 K15360xN3840": {"bytes": 182854400, "sha1": "76f8ca5ba6de39985105f48ae8820d0cae4e1f55"},
+    "w4a16_gemv M1 K14336xN4096": {"bytes": 31290112, "sha1": "ffaef4ba9295beadb8afbf68546c90969324894b"},
+    # profiles/w4a8_gemm_prefill_traffic.md (median of 11 launches per shape)
+    "w4a8_gemm M4096 K3840xN15360": {"bytes": 153379840, "sha1": "2fc13ed112d7918580956d35db9107959347192d"},
+    "w4a8_gemm M4096 K15360xN3840": {"bytes": 179415552, "sha1": "2fc13ed112d7918580956d35db9107959347192d"},
 }
 
 

@@ -278,7 +278,8 @@ __device__ __forceinline__ void gemv_block(const Args &a, const int bx, const in
     const int sl0 = kp * a.spp;                                    // first slice of this part
     const int nsl = (a.tpr - sl0) < a.spp ? (a.tpr - sl0) : a.spp;  // slices of this part
     const int64_t k0 = (int64_t)sl0 * KC;                          // first k of this part
-    const int J0 = (int)(k0 / a.g);                                // first group of this part
+    const int gsh = __ffs(a.g) - 1;                                // log2 of the group (a power of two)
+    const int J0 = (int)(k0 >> gsh);                               // first group of this part
 
     if (tid == 0) {
         for (int i = 0; i < a.NS; ++i) {
@@ -398,7 +399,7 @@ __device__ __forceinline__ void gemv_block(const Args &a, const int bx, const in
 #pragma unroll
         for (int js = 0; js < NSEG; ++js) {
             const int seg = (js + srot) % NSEG;
-            const int jg = (int)((k0 + (int64_t)sl * KC + seg * GS) / a.g);
+            const int jg = (int)((k0 + (int64_t)sl * KC + seg * GS) >> gsh);
             seg_live[js] = jg < a.J;
             sc_off[js] = a.KPB + 4u * (uint32_t)(jg - J0);
         }

@@ -370,7 +370,9 @@ w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const uint16_t *X_f16, const 
  *   an expert); row_of int32 [T, k], the grouped row of token t's i-th expert. Deterministic
  *   (no dependence on thread timing). workspace: device scratch of at least
  *   w4_moe_route_workspace_bytes(T, E) bytes (ceil(T/32) * E int32 expert counts), owned by
- *   the caller, contents irrelevant between calls. Two launches on `stream`.
+ *   the caller, contents irrelevant between calls. Two launches on `stream`; the second reads
+ *   every earlier block's counts, so its work grows as (T/32)^2 * E (0.5 M reads at T = 4096,
+ *   E = 32).
  *   1 <= E <= 1024, 1 <= k <= min(8, E), T * k < 2^31. Errors: NULL / SHAPE / WORKSPACE /
  *   ALIGN (4-byte) / CUDA.
  */
