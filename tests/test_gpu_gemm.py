@@ -298,3 +298,24 @@ def test_persistent_tiles_with_long_zero_point_tail():
     # 160 tiles on 148 SMs: one whole wave, then 12 tiles split over 96 blocks, 9 zero-point
     # pseudo-stages on the segment that ends each split tile
     assert check_split_run(X8, s_a, G, packed, N, K, g, "asym", A @ Wd.T, rows)
+
+
+@pytest.mark.parametrize("group", [32, 256])
+def test_split_path_persistent_odd_weight_tiles(group):
+    """Split-weight path with more tiles than SMs: 4001 tokens (16 token tiles of 256, the last
+    holding 161 rows) x 1400 outputs (11 weight tiles of 128, the last holding 120 rows) is 176
+    tiles, so some CTAs run two and both TMEM accumulators are used. K = 512. 64 sampled token
+    rows (the tile edges among them) against every output column."""
+    M, N, K = 4001, 1400, 512
+    W = synth.student_t3_weight(N, K, 3, 41)
+    codes, scales, zeros, _ = oracle.quantize(synth.bf16_bits(W), group, "asym", [1.0], want_chosen=False)
+    X = synth.outlier_activation(M, K, 8, 20.0, 3, 42)
+    X8, s_a, G = oracle.row_quant(synth.bf16_bits(X), group)
+    packed = upload_weight(codes, scales, zeros, N, K, group, "asym")
+    y32 = gpu_gemm(X8, s_a, G, packed, N, K, group, "asym", 1)
+    y16 = gpu_gemm(X8, s_a, G, packed, N, K, group, "asym", 0)
+    rows = np.unique(np.concatenate([np.linspace(0, M - 1, 60).astype(int), [255, 256, 3839, 3840, 4000]]))
+    Wd = oracle.dequantize(codes, scales, zeros, group, "asym")
+    A = oracle.e4m3_decode(X8[rows]).astype(np.float64) * s_a[rows, None].astype(np.float64)
+    check_errors(A @ Wd.T, y32[rows], y16[rows])
+    assert w4.w4_device_status() == 0
