@@ -143,6 +143,12 @@ __device__ __forceinline__ void bulk_g2s_stream(void *dst, const void *src, uint
         : "memory");
 }
 
+// Hint to bring `bytes` (a multiple of 16) at src (16-byte aligned) into L2; nothing waits for
+// it and nothing lands in shared memory.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Named barrier over `n` threads (a multiple of 32); id 0 is __syncthreads.
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");

@@ -53,6 +53,7 @@ constexpr int SMEM_MAX = 227 * 1024;
 constexpr int RED_BUDGET = 48 * 1024;   // row-partial buffer
 constexpr int MAX_STAGES = 16;
 constexpr uint32_t SLACK = 64;          // bytes after the ring (reads past a short last slice)
+constexpr uint64_t PF_PIECE = 32 * 1024; // bytes per L2 prefetch instruction
 
 struct Args {
     const uint16_t *x;   // [M, K] bf16
@@ -81,6 +82,9 @@ struct Args {
     int rstr;            // words between the partials of consecutive (row, m) (nred, padded)
     int lpr;             // lanes that add one (row, m)'s partials in the final reduction
     int out_fp32, pdl;
+    const uint8_t *pf;   // bytes to bring into L2 once the block's own stream is issued (or null)
+    uint64_t pf_bytes;   // their count (a multiple of 16)
+    uint64_t pf_chunk;   // per block (a multiple of 16)
 };
 
 __device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
@@ -326,6 +330,18 @@ __device__ __forceinline__ void gemv_block(const Args &a, const int bx, const in
                     }
                 }
                 ++issued;
+            }
+            // the next GEMV's weights: once this block's rows are all requested, its share of
+            // them goes into L2, so that HBM reads them while this launch converts, sums and
+            // exits and the next launch finds them there
+            if (a.pf && ok) {
+                const uint64_t lb = (uint64_t)by * gridDim.x + (uint64_t)bx;
+                const uint64_t b0 = lb * a.pf_chunk;
+                const uint64_t b1 = b0 + a.pf_chunk < a.pf_bytes ? b0 + a.pf_chunk : a.pf_bytes;
+                for (uint64_t o = b0; o < b1; o += PF_PIECE) {
+                    const uint64_t n = b1 - o < PF_PIECE ? b1 - o : PF_PIECE;
+                    bulk_prefetch_l2(a.pf + o, (uint32_t)n);
+                }
             }
             // no bulk copy may be in flight when the block exits
             for (int s = issued - a.NS > 0 ? issued - a.NS : 0; s < issued; ++s)
@@ -716,7 +732,8 @@ static size_t ws_need(const Plan &p) {
 }
 
 static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, int64_t K, int g, void *y, int out_fp32,
-                     void *ws, size_t ws_bytes, int pdl, cudaStream_t stream) {
+                     void *ws, size_t ws_bytes, int pdl, cudaStream_t stream, const void *next = nullptr,
+                     size_t next_bytes = 0) {
     Plan p;
     if (!make_plan(p, M, N, K, g, sm_count_cached())) return W4_ERR_SHAPE;
     Args &a = p.a;
@@ -732,6 +749,13 @@ static w4_status run(const void *x, int64_t M, const void *packed, int64_t N, in
     a.out_fp32 = out_fp32;
     a.status = device_status_ptr();
     a.pdl = pdl;
+    if (next && next_bytes >= 16) {
+        const uint64_t nblk = (uint64_t)p.grid_x * (uint64_t)p.sweeps;
+        a.pf = static_cast<const uint8_t *>(next);
+        a.pf_bytes = (uint64_t)next_bytes / 16 * 16;
+        a.pf_chunk = (a.pf_bytes + nblk - 1) / nblk;
+        a.pf_chunk = (a.pf_chunk + 15) / 16 * 16;
+    }
     void *fn = pick_kernel(p.MT, g);
     static int attr_done[64][3][3] = {};
     int dev = 0;
@@ -898,6 +922,23 @@ W4_API w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, i
     if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(y) || (workspace && !aligned16(workspace)))
         return W4_ERR_ALIGN;
     return gemv::run(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream);
+}
+
+W4_API w4_status w4a16_gemv_prefetch_next(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
+                                          int group, int mode, void *y, int flags, void *workspace,
+                                          size_t workspace_bytes, const void *next, size_t next_bytes,
+                                          cudaStream_t stream) {
+    if (!x_bf16 || !packed || !y || (!next && next_bytes)) return W4_ERR_NULL;
+    if (!valid_mode(mode) || (flags & ~(W4_OUT_FP32 | W4_OVERLAP_PREVIOUS))) return W4_ERR_ARG;
+    const int out_fp32 = (flags & W4_OUT_FP32) ? 1 : 0;
+    const int pdl = (flags & W4_OVERLAP_PREVIOUS) ? 1 : 0;
+    if (!gemv_shape_ok(M, N, K)) return W4_ERR_SHAPE;
+    if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
+    if (!aligned16(x_bf16) || !aligned16(packed) || !aligned16(y) || (workspace && !aligned16(workspace)) ||
+        (next && !aligned16(next)))
+        return W4_ERR_ALIGN;
+    return gemv::run(x_bf16, M, packed, N, K, group, y, out_fp32, workspace, workspace_bytes, pdl, stream, next,
+                     next_bytes);
 }
 
 W4_API w4_status w4a16_gemv_grouped(int count, const void *const *x_bf16, int64_t M, const void *const *packed,

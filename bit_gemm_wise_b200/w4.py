@@ -48,6 +48,7 @@ SIGNATURES = [
     ("w4a16_gemv_workspace_bytes", _SZ, [_I64, _I64, _I]),
     ("w4a16_gemv_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
+    ("w4a16_gemv_prefetch_next", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P, _SZ, _P]),
     ("w4a16_gemv_noalloc_scratch_limit", _SZ, []),
     ("w4a16_gemv_grouped", _I, [_I, _P, _I64, _P, _P, _P, _I, _I, _P, _I, _P]),
     ("w4a16_gemv_grouped_schedule", _I, [_I, _I64, _P, _P, _I, _I, _P]),
@@ -224,6 +225,19 @@ def w4a16_gemv(x, M, packed, N, K, group, mode, y, flags, workspace, stream=None
                           _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _check("w4a16_gemv", rc)
+
+
+def w4a16_gemv_prefetch_next(x, M, packed, N, K, group, mode, y, flags, workspace, next_packed, next_bytes=None,
+                             stream=None):
+    """w4a16_gemv that also brings next_bytes bytes at next_packed (the weights of the GEMV that
+    follows on the stream) into L2 once each block's own rows are requested."""
+    if next_bytes is None:
+        next_bytes = 0 if next_packed is None else next_packed.numel() * next_packed.element_size()
+    rc = lib().w4a16_gemv_prefetch_next(_ptr(x), M, _ptr(packed), N, K, group, _mode(mode), _ptr(y), int(flags),
+                                        _ptr(workspace),
+                                        0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                        _ptr(next_packed), int(next_bytes), _stream(stream))
+    _check("w4a16_gemv_prefetch_next", rc)
 
 
 def w4a16_gemv_grouped(xs, M, packeds, Ns, Ks, group, mode, ys, flags, stream=None):

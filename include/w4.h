@@ -215,6 +215,24 @@ w4_status w4a16_gemv(const void *x_bf16, int64_t M, const void *packed, int64_t 
                      size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * w4a16_gemv_prefetch_next -- w4a16_gemv (same arguments, same results, bit for bit) that also
+ *   names the weights the next GEMV on the stream will read: `next_bytes` bytes at `next`
+ *   (device memory, 16-byte aligned; a trailing partial 16 bytes is not touched). Each block,
+ *   once all of its own weight rows have been requested, issues L2 prefetches of its share of
+ *   that range (no copy into shared memory, no wait), so that HBM reads them while this launch
+ *   converts its activations, adds its row sums and exits; the next launch then streams them
+ *   from L2. A decode step whose GEMVs each name their successor's weights keeps HBM busy
+ *   across the launch boundaries ("The Problem & Context": decode reads every weight once per
+ *   token). Every weight byte is still read from HBM once. next may be NULL with next_bytes 0
+ *   (then this is w4a16_gemv). Errors: as w4a16_gemv, and NULL (next NULL with next_bytes > 0)
+ *   and ALIGN (next not 16-byte aligned).
+ */
+w4_status w4a16_gemv_prefetch_next(const void *x_bf16, int64_t M, const void *packed, int64_t N,
+                                   int64_t K, int group, int mode, void *y, int flags,
+                                   void *workspace, size_t workspace_bytes, const void *next,
+                                   size_t next_bytes, cudaStream_t stream);
+
+/*
  * w4a16_gemv_grouped -- `count` independent w4a16_gemv problems in one launch (for example the
  *   q, k and v projections of a layer, or its gate and up projections, which read the same
  *   activations): problem j computes y[j] = x[j] W_j^T exactly as w4a16_gemv does, with the

@@ -114,6 +114,13 @@ def test_host_validation_rejects_before_launch(lib):
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 3, FAKE, 0, FAKE, 1 << 20, None) == 5
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 4, FAKE, 1 << 20, None) == 5
     assert rc("w4a16_gemv", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 0, FAKE + 8, 1 << 20, None) == 4
+    # gemv naming the next GEMV's weights: a byte count needs a pointer, the pointer 16-byte
+    # alignment; the other checks are w4a16_gemv's
+    assert rc("w4a16_gemv_prefetch_next", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, None, 4096, None) == 1
+    assert rc("w4a16_gemv_prefetch_next", FAKE, 1, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, FAKE + 8, 4096,
+              None) == 4
+    assert rc("w4a16_gemv_prefetch_next", FAKE, 17, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, FAKE, 4096, None) == 2
+    assert rc("w4a16_gemv_prefetch_next", FAKE, 1, FAKE, 16, 128, 128, 3, FAKE, 0, None, 0, FAKE, 4096, None) == 5
     # gemm: groups 64/128 need the codes and the group-sum operand, groups 32/256 the fp16
     # copy of the activations; K >= 128
     assert rc("w4a8_gemm", FAKE, None, FAKE, None, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, None) == 1

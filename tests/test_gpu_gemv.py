@@ -258,3 +258,63 @@ def test_grouped_ragged_shapes_group_64():
     assert w4.w4_device_status() == 0
     for (K, N, _, _, ref), y in zip(probs, ys):
         assert rel_frob(ref, y.double().cpu().numpy()) <= 1e-4, (K, N)
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_prefetch_next_decode_chain(M):
+    """The four decode GEMVs chained with W4_OVERLAP_PREVIOUS, each naming the next one's
+    weights (the last names the first's) for the L2 prefetch: every output against the oracle,
+    and bit-identical to the same calls through w4a16_gemv."""
+    probs = []
+    for K, N in synth.DECODE_SHAPES:
+        codes, scales, zeros = quantized("decode", K, N, 128, "asym", "twenty")
+        x_bits = synth.bf16_bits(synth.decode_activation(M, K, 0))
+        probs.append((K, N, upload_gemv(codes, scales, zeros, N, K, 128, "asym"),
+                      to_dev(x_bits.view(np.int16)).view(torch.bfloat16),
+                      oracle.gemv_ref(x_bits, codes, scales, zeros, 128, "asym")))
+    for out_fp32 in (1, 0):
+        dt = torch.float32 if out_fp32 else torch.bfloat16
+        flags = w4.W4_OVERLAP_PREVIOUS | (w4.W4_OUT_FP32 if out_fp32 else 0)
+        ys = [torch.full((M, N), float("nan"), dtype=dt, device=cuda()) for K, N, *_ in probs]
+        plain = [torch.full((M, N), float("nan"), dtype=dt, device=cuda()) for K, N, *_ in probs]
+        for rep in range(2):
+            for j, (K, N, p, x, _) in enumerate(probs):
+                nxt = probs[(j + 1) % len(probs)][2]
+                w4.w4a16_gemv_prefetch_next(x, M, p, N, K, 128, "asym", ys[j], flags, None, nxt)
+        for j, (K, N, p, x, _) in enumerate(probs):
+            w4.w4a16_gemv(x, M, p, N, K, 128, "asym", plain[j], flags, None)
+        torch.cuda.synchronize()
+        assert w4.w4_device_status() == 0
+        for (K, N, _, _, ref), y, yp in zip(probs, ys, plain):
+            got = y.double().cpu().numpy()
+            assert np.isfinite(got).all()
+            assert torch.equal(y, yp), (K, N)
+            if out_fp32:
+                assert rel_frob(ref, got) <= 1e-4, (K, N)
+            else:
+                assert rel_frob(bf16_round(ref), got) <= 1e-3, (K, N)
+
+
+@pytest.mark.parametrize("next_bytes", [0, 8, 16, 4000, 40965, None])
+def test_prefetch_next_ranges(next_bytes):
+    """Prefetch ranges of every kind (none, below 16 bytes, one 16-byte unit, fewer units than
+    blocks, a count that is not a multiple of 16, a whole buffer) on a shape whose rows are
+    split along K over several blocks: the result equals w4a16_gemv's bit for bit."""
+    N, K, g, M = 100, 65536, 128, 1
+    codes, scales, zeros = quantized("t3", K, N, g, "asym", "one")
+    p = upload_gemv(codes, scales, zeros, N, K, g, "asym")
+    x_bits = synth.bf16_bits(synth.normal((M, K), 1.0, 7, 71))
+    x = to_dev(x_bits.view(np.int16)).view(torch.bfloat16)
+    other = torch.zeros(1 << 20, dtype=torch.uint8, device=cuda())
+    nb = other.numel() if next_bytes is None else next_bytes
+    ws = w4.alloc_gemv_workspace(N, K, g)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device=cuda())
+    yp = torch.full((M, N), float("nan"), dtype=torch.float32, device=cuda())
+    w4.w4a16_gemv_prefetch_next(x, M, p, N, K, g, "asym", y, w4.W4_OUT_FP32, ws,
+                                other if nb else None, nb)
+    w4.w4a16_gemv(x, M, p, N, K, g, "asym", yp, w4.W4_OUT_FP32, ws)
+    torch.cuda.synchronize()
+    assert w4.w4_device_status() == 0
+    assert torch.equal(y, yp)
+    ref = oracle.gemv_ref(x_bits, codes, scales, zeros, g, "asym")
+    assert rel_frob(ref, y.double().cpu().numpy()) <= 1e-4
