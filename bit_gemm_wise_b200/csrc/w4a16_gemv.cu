@@ -78,6 +78,8 @@ struct Args {
     uint32_t SB;         // stage bytes
     uint32_t off_sx, off_pp, off_red, off_ring, off_planes;
     int warpred;         // MT > 1 with spp a multiple of 32: partials reduced over the warp first
+    int direct;          // MT = 1, one warp per row (spp = 32, whole rows, one stage per block):
+                         // the warp adds the row's partials and its lane 0 stores y
     int nred;            // partials per (row, m): spp, or spp / 32 with warpred
     int rstr;            // words between the partials of consecutive (row, m) (nred, padded)
     int lpr;             // lanes that add one (row, m)'s partials in the final reduction
@@ -494,7 +496,21 @@ __device__ __forceinline__ void gemv_block(const Args &a, const int bx, const in
                         }
                     }
                 }
-                if (!a.warpred) {
+                if (a.direct) {
+                    // the warp holds the row's 32 slices: a butterfly over the warp, in a
+                    // fixed order, and lane 0 stores the sum
+#pragma unroll
+                    for (int i = 0; i < RPT; ++i) {
+                        float r = yv[i][0];
+#pragma unroll
+                        for (int off = 16; off >= 1; off >>= 1) r += __shfl_xor_sync(FULL, r, off);
+                        if (lane == 0 && live[i]) {
+                            const int64_t n = row0 + s * SR + slot + i * a.nslot;
+                            if (a.out_fp32) static_cast<float *>(a.y)[(int64_t)m0 * a.N + n] = r;
+                            else static_cast<__nv_bfloat16 *>(a.y)[(int64_t)m0 * a.N + n] = __float2bfloat16_rn(r);
+                        }
+                    }
+                } else if (!a.warpred) {
 #pragma unroll
                     for (int i = 0; i < RPT; ++i) {
                         if (!live[i]) continue;
@@ -519,6 +535,7 @@ __device__ __forceinline__ void gemv_block(const Args &a, const int bx, const in
             if (lane == 0) mbar_arrive(empty + slot_s);
         }
         if (!ok) *(volatile int *)abort_flag = 1;
+        if (a.direct) return;  // every row was stored in the stage loop
 
         // (4) row sums in a fixed order: lpr lanes per (row, m), each adding every lpr-th
         // partial in turn, then a butterfly over the lpr lanes
@@ -659,6 +676,9 @@ static bool make_plan_parts(Plan &p, int64_t M, int64_t N, int64_t K, int g, int
     if (rpc_cap < 1) return false;
     if (rpc > rpc_cap) rpc = rpc_cap;
     a.rpc = (int)rpc;
+    // (only for blocks whose rows fit one stage: in a longer stream the butterfly of every row
+    // lengthens the dot-product-bound loop more than the final pass costs)
+    a.direct = (MT == 1 && a.kparts == 1 && a.spp == 32 && rpc <= (int64_t)a.nslot * a.rpt) ? 1 : 0;
     // final reduction: as many lanes per (row, m) as the consumer threads allow (a power of
     // two up to 32); partials of consecutive (row, m) are rstr = lpr (mod 32) words apart, so
     // a warp's loads hit distinct banks
