@@ -229,11 +229,15 @@ class Decode:
         p, nb = self.packed[si]
         return p[(i % self.R) * nb:(i % self.R + 1) * nb]
 
-    def gemv(self, si, i, next_si=None):
+    def gemv(self, si, i, next_si=None, prefetch=True):
         """GEMV si of step i. It names the weights of the GEMV that follows it on the stream
         (the step's next shape, or the first shape of step i + 1; with next_si given, that
         shape's copy for step i + 1), which it brings into L2 once its own are requested."""
         (K, N) = self.shapes[si]
+        if not prefetch:
+            self.w4.w4a16_gemv(self.x[si], self.M, self.weights(si, i), N, K, 128, "asym", self.y[si], self.flags,
+                               self.ws[si])
+            return
         if next_si is None:
             nsi, ni = (si + 1, i) if si + 1 < len(self.shapes) else (0, i + 1)
         else:
@@ -800,6 +804,12 @@ def main():
     ap.add_argument("--quant-layers", type=int, default=32)
     ap.add_argument("--min-repeats", type=int, default=25, help="repeats of the timed region (median reported)")
     ap.add_argument("--min-seconds", type=float, default=0.3, help="keep repeating the timed region this long")
+    ap.add_argument("--profile-chain", default="", metavar="K,N",
+                    help="only run --launches chained M=1 GEMVs of decode shape (K, N), each naming the next "
+                         "weight copy (a short, bounded run for a profiler); prints one line")
+    ap.add_argument("--launches", type=int, default=8)
+    ap.add_argument("--no-prefetch", action="store_true",
+                    help="with --profile-chain: plain w4a16_gemv calls (the kernel's own DRAM traffic)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -819,7 +829,18 @@ def main():
     try:
         from bit_gemm_wise_b200 import w4
         w4.lib()
-        if args.rows_only:
+        if args.profile_chain:
+            K, N = (int(v) for v in args.profile_chain.split(","))
+            dec = Decode(1, args.seed, dev)
+            si = dec.shapes.index((K, N))
+            for i in range(args.launches):
+                dec.gemv(si, i, next_si=si, prefetch=not args.no_prefetch)
+            torch.cuda.synchronize()
+            from bit_gemm_wise_b200 import w4 as w4_
+            assert w4_.w4_device_status() == 0
+            out = {"profile_chain": f"K{K}xN{N}", "launches": args.launches, "prefetch": not args.no_prefetch,
+                   "bytes_per_launch": gemv_bytes(1, N, K)}
+        elif args.rows_only:
             out = {"rows": measure_rows(args, dev, peaks())}
         else:
             out = run_ours(args, rank, world, dev)

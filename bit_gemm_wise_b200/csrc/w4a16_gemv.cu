@@ -111,6 +111,19 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     return v;
 }
 
+// two fp32 lanes per instruction (sm_100): lane 0 in the low word
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t pair(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
+
 // 2^e as an fp32 (0 below the subnormal range); e <= 127
 __device__ __forceinline__ float exp2i(int e) {
     if (e >= -126) return __int_as_float((e + 127) << 23);
@@ -175,14 +188,14 @@ __device__ __forceinline__ void xprep_rounds(const Args &a, uint32_t *planes, in
         xv[r] = live ? __ldg(reinterpret_cast<const uint4 *>(a.x + (int64_t)(m0 + m) * a.K + k))
                      : make_uint4(0u, 0u, 0u, 0u);
     }
-    // largest magnitude pattern of each slice (bf16 bits order like magnitudes)
+    // largest magnitude pattern of each slice (bf16 bits order like magnitudes): a 16-bit
+    // SIMD max over the magnitude bits of both halves, then the larger half
     uint32_t mx[XBN];
 #pragma unroll
     for (int r = 0; r < XBN; ++r) {
-        const uint32_t e[4] = {xv[r].x, xv[r].y, xv[r].z, xv[r].w};
-        mx[r] = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) mx[r] = max(mx[r], max(e[i] & 0x7FFFu, (e[i] >> 16) & 0x7FFFu));
+        const uint32_t m2 = __vmaxu2(__vmaxu2(xv[r].x & 0x7FFF7FFFu, xv[r].y & 0x7FFF7FFFu),
+                                     __vmaxu2(xv[r].z & 0x7FFF7FFFu, xv[r].w & 0x7FFF7FFFu));
+        mx[r] = max(m2 & 0xFFFFu, m2 >> 16);
     }
 #pragma unroll
     for (int off = WPS / 2; off >= 1; off >>= 1)
@@ -198,16 +211,18 @@ __device__ __forceinline__ void xprep_rounds(const Args &a, uint32_t *planes, in
         const int S = 18 - ex;  // -109 <= S <= 151
         // x 2^S as two exact power-of-two products (2^S alone leaves the fp32 range when the
         // slice's largest |x| is below 2^-109): 2^min(S, 127), then 2^max(S - 127, 0)
-        const float f1 = __int_as_float(((S < 127 ? S : 127) + 127) << 23);
-        const float f2 = __int_as_float(((S > 127 ? S - 127 : 0) + 127) << 23);
-        const bool zero = mx[r] >= 0x7F80u || mx[r] == 0u;  // infinity / NaN, or all zero
+        const uint32_t f1 = (uint32_t)((S < 127 ? S : 127) + 127) << 23;
+        const uint32_t f2 = (uint32_t)((S > 127 ? S - 127 : 0) + 127) << 23;
+        // rint by the 1.5 * 2^23 shift, two elements per instruction. A slice of zeros gives
+        // X = 0; in a slice holding an infinity or a NaN the values are meaningless, and its
+        // 2^-S below is a NaN, which makes the rows' sums NaN
+        const uint64_t F1 = pair(f1, f1), F2 = pair(f2, f2), RND = pair(0x4B400000u, 0x4B400000u);
         int X[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t bb = (i & 1) ? (e[i >> 1] & 0xFFFF0000u) : (e[i >> 1] << 16);
-            const float sv = __fmul_rn(__fmul_rn(__uint_as_float(bb), f1), f2);
-            const int v = __float_as_int(__fadd_rn(sv, 12582912.0f)) - 0x4B400000;
-            X[i] = zero ? 0 : v;
+        for (int h = 0; h < 4; ++h) {
+            const uint64_t v = add_f32x2(mul_f32x2(mul_f32x2(pair(e[h] << 16, e[h] & 0xFFFF0000u), F1), F2), RND);
+            X[2 * h] = (int)(uint32_t)v - 0x4B400000;
+            X[2 * h + 1] = (int)(uint32_t)(v >> 32) - 0x4B400000;
         }
         uint32_t pw[6];
 #pragma unroll
@@ -215,12 +230,12 @@ __device__ __forceinline__ void xprep_rounds(const Args &a, uint32_t *planes, in
             const uint32_t sh = par ? 0u : 4u;
             const uint32_t V0 = (uint32_t)X[par] << sh, V1 = (uint32_t)X[2 + par] << sh;
             const uint32_t V2 = (uint32_t)X[4 + par] << sh, V3 = (uint32_t)X[6 + par] << sh;
-#pragma unroll
-            for (int pl = 0; pl < 3; ++pl) {
-                const uint32_t lo = __byte_perm(V0, V1, (uint32_t)(pl | ((4 + pl) << 4)));
-                const uint32_t hi = __byte_perm(V2, V3, (uint32_t)(pl | ((4 + pl) << 4)));
-                pw[par * 3 + pl] = __byte_perm(lo, hi, 0x5410u);
-            }
+            // plane pl = byte pl of V0..V3: pairs of bytes first, then the planes
+            const uint32_t t01l = __byte_perm(V0, V1, 0x5140u), t01h = __byte_perm(V0, V1, 0x0062u);
+            const uint32_t t23l = __byte_perm(V2, V3, 0x5140u), t23h = __byte_perm(V2, V3, 0x0062u);
+            pw[par * 3 + 0] = __byte_perm(t01l, t23l, 0x5410u);
+            pw[par * 3 + 1] = __byte_perm(t01l, t23l, 0x7632u);
+            pw[par * 3 + 2] = __byte_perm(t01h, t23h, 0x5410u);
         }
         xs[r] = X[0] + X[1] + X[2] + X[3] + X[4] + X[5] + X[6] + X[7];
         const int t = t0 + r * NCT;
