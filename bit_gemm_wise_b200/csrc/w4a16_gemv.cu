@@ -387,7 +387,9 @@ __device__ __forceinline__ void gemv_block(const Args &a, const int bx, const in
             // so that the rounds' latencies (loads, shuffle chains) overlap
             const int tasks = a.spp * WPS;
             for (int tb = 0; tb < tasks; tb += 4 * NCT) {
-                const int nr = (tasks - tb + NCT - 1) / NCT;
+                // rounds in which this warp has a task (warp-uniform; a warp with none skips)
+                const int nr = (tasks - tb - warp * 32 + NCT - 1) / NCT;
+                if (nr <= 0) continue;
                 if (nr >= 4) xprep_rounds<MT, 4>(a, planes, sx, pp, m, m0, k0, nsl, tb + warp * 32 + lane);
                 else if (nr == 3) xprep_rounds<MT, 3>(a, planes, sx, pp, m, m0, k0, nsl, tb + warp * 32 + lane);
                 else if (nr == 2) xprep_rounds<MT, 2>(a, planes, sx, pp, m, m0, k0, nsl, tb + warp * 32 + lane);
