@@ -26,8 +26,8 @@
 //
 // Data movement. One persistent block per SM owns a contiguous run of rows. A producer warp
 // streams the block's rows through a ring of shared-memory stages with 1-D bulk copies
-// (one copy per stage: consecutive rows are consecutive records), so the whole ring
-// (~150 KB per SM) is in flight from the first instruction. The activations are converted
+// (consecutive rows are consecutive records: a stage is one range, copied in 4 KB pieces), so
+// the whole ring (~150 KB per SM) is in flight from the first instruction. The activations are converted
 // to byte planes once per block (all threads cooperate, each element once) into an area at
 // the end of the ring that the producer fills only after every thread has loaded its planes
 // into registers. A stage holds one row per "slot" of threads; each thread adds its
@@ -54,6 +54,7 @@ constexpr int RED_BUDGET = 48 * 1024;   // row-partial buffer
 constexpr int MAX_STAGES = 16;
 constexpr uint32_t SLACK = 64;          // bytes after the ring (reads past a short last slice)
 constexpr uint64_t PF_PIECE = 32 * 1024; // bytes per L2 prefetch instruction
+constexpr uint32_t STREAM_PIECE = 4096;  // bytes per bulk copy of the weight stream (a multiple of 16)
 
 struct Args {
     const uint16_t *x;   // [M, K] bf16
@@ -332,8 +333,15 @@ __device__ __forceinline__ void gemv_block(const Args &a, const int bx, const in
                 const int nr = (rows - r0) < a.nslot * a.rpt ? (rows - r0) : a.nslot * a.rpt;
                 uint8_t *dst = smem + a.off_ring + (size_t)slot * a.SB;
                 if (a.kparts == 1) {
-                    mbar_arrive_expect_tx(full + slot, (uint32_t)nr * a.RS);
-                    bulk_g2s_stream(dst, src0 + (size_t)r0 * a.RS, (uint32_t)nr * a.RS, full + slot);
+                    // the stage's rows are consecutive records: copied in pieces of STREAM_PIECE
+                    // bytes, so that the activation loads the consumers issue meanwhile are not
+                    // queued behind one long copy in the SM's inbound traffic
+                    const uint32_t tot = (uint32_t)nr * a.RS;
+                    mbar_arrive_expect_tx(full + slot, tot);
+                    for (uint32_t o = 0; o < tot; o += STREAM_PIECE) {
+                        const uint32_t n = tot - o < STREAM_PIECE ? tot - o : STREAM_PIECE;
+                        bulk_g2s_stream(dst + o, src0 + (size_t)r0 * a.RS + o, n, full + slot);
+                    }
                 } else {
                     // this part's codes and scales of each row
                     const uint32_t cb = (uint32_t)(((k0 + (int64_t)nsl * KC < a.K ? k0 + (int64_t)nsl * KC : a.K) - k0) / 2);
