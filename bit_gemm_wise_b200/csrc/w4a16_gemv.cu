@@ -753,10 +753,23 @@ static bool make_plan_mt(Plan &p, int64_t M, int64_t N, int64_t K, int g, int64_
 
 // MT = activation rows per sweep: as many as the registers hold for this K (4, 2 or 1),
 // with whole rows per block when possible
+// Whole rows per block with MT rows per sweep. When the row-partial buffer of the default size
+// caps a block's rows so low that the blocks outnumber the SMs (a second, mostly empty wave),
+// a larger buffer (up to four times) is taken if shared memory still holds the ring.
+template <int MT>
+static bool make_plan_whole(Plan &p, int64_t M, int64_t N, int64_t K, int g, int64_t S) {
+    if (!make_plan_parts<MT>(p, M, N, K, g, S, 1)) return false;
+    for (int64_t rb = 2 * RED_BUDGET; rb <= 4 * RED_BUDGET && p.grid_x > S; rb += RED_BUDGET) {
+        Plan q;
+        if (make_plan_parts<MT>(q, M, N, K, g, S, 1, rb) && q.grid_x < p.grid_x) p = q;
+    }
+    return true;
+}
+
 static bool make_plan(Plan &p, int64_t M, int64_t N, int64_t K, int g, int64_t S) {
     const int want = M >= 3 ? 4 : (int)M;
-    if (want >= 4 && make_plan_parts<4>(p, M, N, K, g, S, 1)) return true;
-    if (want >= 2 && make_plan_parts<2>(p, M, N, K, g, S, 1)) return true;
+    if (want >= 4 && make_plan_whole<4>(p, M, N, K, g, S)) return true;
+    if (want >= 2 && make_plan_whole<2>(p, M, N, K, g, S)) return true;
     return make_plan_mt<1>(p, M, N, K, g, S);
 }
 
