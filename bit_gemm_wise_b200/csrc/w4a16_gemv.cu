@@ -454,7 +454,10 @@ __device__ __forceinline__ void gemv_block(const Args &a, const int bx, const in
             if (lane == 0) got = mbar_wait_abortable(full + slot_s, (s / a.NS) & 1, abort_flag, a.status, 2000000000ull);
             got = __shfl_sync(FULL, got ? 1 : 0, 0) != 0;
             if (!got) { ok = false; break; }
-            (void)mbar_try_wait_short(full + slot_s, (s / a.NS) & 1);
+            // lane 0's wait acquired the stage's bytes; the warp barrier orders the other lanes'
+            // reads after it (a try_wait by every lane of every warp costs the barrier unit
+            // hundreds of cycles a stage)
+            __syncwarp();
             const uint32_t sbase = ring + (uint32_t)slot_s * a.SB;
             float yv[RPT][MT];
             bool live[RPT];
