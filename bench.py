@@ -184,15 +184,18 @@ class Decode:
     Step i runs one GEMV per shape on weight copy i % R; each step is captured once in a
     CUDA graph (the decode loop replays graphs, as serving engines do)."""
 
-    def __init__(self, M, seed, dev, copies=None):
+    def __init__(self, M, seed, dev, copies=None, tc=False):
+        """tc: the tensor-core W4A16 (w4a16_gemm_tc, layout W4_LAYOUT_TC) instead of the GEMV."""
         from bit_gemm_wise_b200 import synth, w4
         self.w4 = w4
         self.M = M
+        self.tc = tc
+        layout = w4.W4_LAYOUT_TC if tc else w4.W4_LAYOUT_GEMV
         g = 128
         grid = synth.clip_grid_20()
         self.shapes = DECODE_SHAPES
         self.bytes_per_step = sum(gemv_bytes(M, N, K) for K, N in self.shapes)
-        packed_per_step = sum(w4.w4_prepack_bytes(N, K, g, w4.W4_LAYOUT_GEMV) for K, N in self.shapes)
+        packed_per_step = sum(w4.w4_prepack_bytes(N, K, g, layout) for K, N in self.shapes)
         self.R = copies or max(2, -(-3 * L2_BYTES // packed_per_step))
         self.packed, self.x, self.y, self.ws = [], [], [], []
         # all shapes' activations and outputs live in one buffer each (16-byte aligned views),
@@ -212,9 +215,9 @@ class Decode:
             W = synth.decode_weight(K, N, seed, device=dev)
             codes, scales, zeros, _ = w4.alloc_quantized(N, K, g, "asym", device=dev, chosen=False)
             w4.w4_quantize(W, N, K, g, "asym", grid, codes, scales, zeros, None)
-            nb = w4.w4_prepack_bytes(N, K, g, w4.W4_LAYOUT_GEMV)
+            nb = w4.w4_prepack_bytes(N, K, g, layout)
             p = torch.empty(self.R * nb, dtype=torch.uint8, device=dev)
-            w4.w4_prepack(codes, scales, zeros, N, K, g, "asym", w4.W4_LAYOUT_GEMV, p[:nb])
+            w4.w4_prepack(codes, scales, zeros, N, K, g, "asym", layout, p[:nb])
             for r in range(1, self.R):
                 p[r * nb:(r + 1) * nb].copy_(p[:nb])
             self.packed.append((p, nb))
@@ -225,7 +228,8 @@ class Decode:
                 self.ys[b].append(self.ybufs[b][yo[si]:yo[si] + M * N].view(M, N))
             self.x.append(self.xs[0][si])
             self.y.append(self.ys[0][si])
-            self.ws.append(w4.alloc_gemv_workspace(N, K, g, device=dev))
+            self.ws.append(w4.alloc_tc_workspace(N, K, g, device=dev) if tc else
+                           w4.alloc_gemv_workspace(N, K, g, device=dev))
             del W, codes, scales, zeros
         # each weight copy as a tensor view, made once (a call of the decode loop only looks it up)
         self.wviews = [[p[r * nb:(r + 1) * nb] for r in range(self.R)] for p, nb in self.packed]
@@ -244,6 +248,9 @@ class Decode:
         shape's copy for step i + 1), which it brings into L2 once its own are requested."""
         (K, N) = self.shapes[si]
         x, y = self.xs[buf][si], self.ys[buf][si]
+        if self.tc:
+            self.w4.w4a16_gemm_tc(x, self.M, self.weights(si, i), N, K, 128, "asym", y, self.flags, self.ws[si])
+            return
         if not prefetch:
             self.w4.w4a16_gemv(x, self.M, self.weights(si, i), N, K, 128, "asym", y, self.flags, self.ws[si])
             return
@@ -506,6 +513,29 @@ def measure_rows(args, dev, pk):
                                     "frac_hbm": round(d.bytes_per_step / (ms * 1e-3) / 1e9 / pk["hbm"], 4),
                                     "fp32_fma_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
                                     "frac_fp32_fma_peak": round(flops / (ms * 1e-3) / 1e12 / fp32_peak, 4)}
+        del d
+
+    # the same decode sweep through the tensor-core W4A16 (w4a16_gemm_tc): one expansion per
+    # weight for all M activation rows; bound by HBM like the M = 1 GEMV
+    for M in ((1, 4, 16) if "gemv" in want else ()):
+        d = Decode(M, args.seed, dev, tc=True)
+        d.capture(6 * d.R, 3)
+        d.g_warm.replay()
+        ms = float(np.median([time_region(lambda i: d.g_steps.replay(), 1) for _ in range(5)])) / (6 * d.R)
+        gbps = d.bytes_per_step / (ms * 1e-3) / 1e9
+        shapes_us = {}
+        for si, (K, N) in enumerate(d.shapes):
+            n_l = 8 * d.R
+            gs = d.shape_graph(si, n_l)
+            gs.replay()
+            t_ms = float(np.median([time_region(lambda i: gs.replay(), 1) for _ in range(5)])) / n_l
+            shapes_us[f"K{K}xN{N}"] = round(t_ms * 1e3, 3)
+            del gs
+        rows[f"w4a16_tc_M{M}"] = {
+            "value": round(gbps, 1), "unit": "GB/s", "us_per_step": round(ms * 1e3, 2), "per_shape_us": shapes_us,
+            "roofline": {"bound": "hbm", "achieved": round(gbps, 1), "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": round(gbps / pk["hbm"], 4)},
+            "note": "w4a16_gemm_tc (tcgen05, W4_LAYOUT_TC), same four decode shapes and bytes as w4a16_gemv_M*"}
         del d
 
     # NF4 comparator at M = 1 over the same decode shapes: normal-quantile levels, blocks of 64

@@ -26,6 +26,7 @@ SOURCES = {
     "fp8_row_quant.cu": ["-fmad=false"],
     "w4_prepack.cu": [],
     "w4a16_gemv.cu": [],
+    "w4a16_tc.cu": [],
     "w4a8_gemm.cu": [],
     "w4_moe.cu": [],
     "w4_nf4.cu": [],

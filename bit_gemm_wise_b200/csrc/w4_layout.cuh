@@ -7,6 +7,12 @@
 #include <stdint.h>
 #include <stddef.h>
 
+#ifdef __CUDACC__
+#define W4_HD __host__ __device__
+#else
+#define W4_HD
+#endif
+
 namespace w4 {
 
 // ---------------------------------------------------------------- W4_LAYOUT_GEMV
@@ -69,6 +75,39 @@ inline GemmLayout gemm_layout(int64_t N, int64_t K, int g) {
     L.scales_bytes = (size_t)L.J * (size_t)L.Npad * 4;
     L.zop_bytes = (size_t)L.Npad * (size_t)L.KZ * 2;
     L.total = L.codes_bytes + L.scales_bytes + L.zop_bytes;
+    return L;
+}
+
+// ---------------------------------------------------------------- W4_LAYOUT_TC
+// Units of 128 weight rows x KS k (KS = max(128, g)): tiles of 128 rows in order, inside a
+// tile its k-blocks in order, so that any run of consecutive units is one contiguous byte
+// range. Rows are padded to a multiple of 128 and K to a multiple of KS with zero codes and
+// zero scales. One unit is one record:
+//   [codes: KS/32 chunks x 128 rows x 16 bytes, chunk c of row r at byte (c * 128 + r) * 16;
+//    inside every 32-bit word (8 consecutive k from k0) nibble p holds q[k0 + 2p] for p < 4
+//    and q[k0 + 2(p - 4) + 1] for p >= 4, so that (w >> 4s) & 0x000F000F holds the codes of
+//    k0 + 2s and k0 + 2s + 1 in its two 16-bit halves]
+//   [scales: KS/g groups x 128 rows of u32 (group-major), lo 16 bits fp16 scale, hi 16 bits
+//    zero (8 for symmetric weights)]
+struct TcLayoutGeo {
+    W4_HD static constexpr int ks(int g) { return g > 128 ? g : 128; }
+    W4_HD static constexpr uint32_t code_bytes(int g) { return 128u * (uint32_t)ks(g) / 2u; }
+    W4_HD static constexpr uint32_t record_bytes(int g) { return code_bytes(g) + (uint32_t)(ks(g) / g) * 128u * 4u; }
+};
+
+struct TcLayout {
+    int64_t N, K, T, NKB;
+    int g;
+    size_t rec, total;
+};
+
+inline TcLayout tc_layout(int64_t N, int64_t K, int g) {
+    TcLayout L;
+    L.N = N; L.K = K; L.g = g;
+    L.T = (N + 127) / 128;
+    L.NKB = (K + TcLayoutGeo::ks(g) - 1) / TcLayoutGeo::ks(g);
+    L.rec = TcLayoutGeo::record_bytes(g);
+    L.total = (size_t)L.T * (size_t)L.NKB * L.rec;
     return L;
 }
 

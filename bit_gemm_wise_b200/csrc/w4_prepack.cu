@@ -84,6 +84,30 @@ __global__ void prepack_gemm_zop(const uint16_t *__restrict__ scales, const int1
     }
 }
 
+// W4_LAYOUT_TC: one thread per 32-bit word of the unit records
+__global__ void prepack_tc(const uint8_t *__restrict__ codes, const uint16_t *__restrict__ scales,
+                           const int16_t *__restrict__ zeros, int64_t N, int64_t K, int g, int64_t NKB,
+                           int64_t nwords, uint32_t *__restrict__ out) {
+    const int ks = TcLayoutGeo::ks(g);
+    const int64_t rec_words = TcLayoutGeo::record_bytes(g) / 4, code_words = TcLayoutGeo::code_bytes(g) / 4;
+    const int64_t J = K / g;
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < nwords;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t u = idx / rec_words, wr = idx - u * rec_words;
+        const int64_t t = u / NKB, kb = u - t * NKB;
+        uint32_t v = 0;
+        if (wr < code_words) {
+            const int64_t c = wr / (128 * 4), r = (wr / 4) % 128, i = wr % 4;
+            const int64_t n = t * 128 + r, k0 = kb * ks + c * 32 + i * 8;
+            for (int p = 0; p < 8; ++p) v |= nib_at(codes, N, K, n, k0 + (p < 4 ? 2 * p : 2 * (p - 4) + 1)) << (4 * p);
+        } else {
+            const int64_t e = wr - code_words, gg = e / 128, r = e % 128;
+            v = scale_entry(scales, zeros, N, J, t * 128 + r, kb * (ks / g) + gg);
+        }
+        out[idx] = v;
+    }
+}
+
 static int grid_for(int64_t n) {
     const int64_t b = (n + 255) / 256;
     const int64_t cap = (int64_t)num_sms() * 32;
@@ -98,6 +122,7 @@ W4_API size_t w4_prepack_bytes(int64_t N, int64_t K, int group, int layout) {
     if (N < 1 || K < 32 || K % 32 != 0 || !valid_group(group) || K % group != 0) return 0;
     if (layout == W4_LAYOUT_GEMV) return gemv_layout(N, K, group).total;
     if (layout == W4_LAYOUT_GEMM) return gemm_layout(N, K, group).total;
+    if (layout == W4_LAYOUT_TC) return tc_layout(N, K, group).total;
     return 0;
 }
 
@@ -109,7 +134,7 @@ W4_API w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, c
     if (mode == W4_SYM && zeros) return W4_ERR_ARG;
     if (N < 1 || K < 32 || K % 32 != 0) return W4_ERR_SHAPE;
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
-    if (layout != W4_LAYOUT_GEMV && layout != W4_LAYOUT_GEMM) return W4_ERR_ARG;
+    if (layout != W4_LAYOUT_GEMV && layout != W4_LAYOUT_GEMM && layout != W4_LAYOUT_TC) return W4_ERR_ARG;
     if (!aligned16(codes) || !aligned16(scales_fp16) || (zeros && !aligned16(zeros)) || !aligned16(packed))
         return W4_ERR_ALIGN;
     uint8_t *base = static_cast<uint8_t *>(packed);
@@ -119,6 +144,11 @@ W4_API w4_status w4_prepack(const uint8_t *codes, const uint16_t *scales_fp16, c
         const int64_t nwords = (int64_t)(L.total / 4);
         prepack_gemv_rows<<<grid_for(nwords), 256, 0, stream>>>(codes, scales_fp16, zeros, N, K, group, row_words,
                                                                 nwords, reinterpret_cast<uint32_t *>(base));
+    } else if (layout == W4_LAYOUT_TC) {
+        const TcLayout L = tc_layout(N, K, group);
+        const int64_t nwords = (int64_t)(L.total / 4);
+        prepack_tc<<<grid_for(nwords), 256, 0, stream>>>(codes, scales_fp16, zeros, N, K, group, L.NKB, nwords,
+                                                         reinterpret_cast<uint32_t *>(base));
     } else {
         const GemmLayout L = gemm_layout(N, K, group);
         const int64_t nwords = (int64_t)(L.codes_bytes / 4);

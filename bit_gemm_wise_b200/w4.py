@@ -16,7 +16,7 @@ import torch
 
 W4_OK = 0
 W4_SYM, W4_ASYM = 0, 1
-W4_LAYOUT_GEMV, W4_LAYOUT_GEMM = 0, 1
+W4_LAYOUT_GEMV, W4_LAYOUT_GEMM, W4_LAYOUT_TC = 0, 1, 2
 W4_OUT_FP32, W4_OVERLAP_PREVIOUS = 1, 2  # flags of w4a16_gemv
 
 STATUS = {
@@ -48,6 +48,9 @@ SIGNATURES = [
     ("w4a16_gemv_workspace_bytes", _SZ, [_I64, _I64, _I]),
     ("w4a16_gemv_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
     ("w4a16_gemv", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
+    ("w4a16_gemm_tc_workspace_bytes", _SZ, [_I64, _I64, _I]),
+    ("w4a16_gemm_tc_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
+    ("w4a16_gemm_tc", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a16_gemv_prefetch_next", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P, _SZ, _P]),
     ("w4a16_gemv_noalloc_scratch_limit", _SZ, []),
     ("w4a16_gemv_grouped", _I, [_I, _P, _I64, _P, _P, _P, _I, _I, _P, _I, _P]),
@@ -227,6 +230,26 @@ def w4a16_gemv(x, M, packed, N, K, group, mode, y, flags, workspace, stream=None
     _check("w4a16_gemv", rc)
 
 
+def w4a16_gemm_tc_workspace_bytes(N, K, group) -> int:
+    return int(lib().w4a16_gemm_tc_workspace_bytes(N, K, group))
+
+
+def w4a16_gemm_tc_schedule(M, N, K, group, sms) -> dict:
+    """Host-only: how w4a16_gemm_tc divides the problem over `sms` SMs."""
+    out = (ctypes.c_int64 * 6)()
+    _check("w4a16_gemm_tc_schedule", lib().w4a16_gemm_tc_schedule(M, N, K, group, sms, out))
+    keys = ("tiles", "k_blocks", "units", "ctas", "k_per_block", "record_bytes")
+    return dict(zip(keys, (int(v) for v in out)))
+
+
+def w4a16_gemm_tc(x, M, packed, N, K, group, mode, y, flags, workspace, stream=None):
+    """Tensor-core W4A16 for 1 <= M <= 16 (packed: W4_LAYOUT_TC); flags as w4a16_gemv."""
+    rc = lib().w4a16_gemm_tc(_ptr(x), M, _ptr(packed), N, K, group, _mode(mode), _ptr(y), int(flags),
+                             _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+                             _stream(stream))
+    _check("w4a16_gemm_tc", rc)
+
+
 def w4a16_gemv_prefetch_next(x, M, packed, N, K, group, mode, y, flags, workspace, next_packed, next_bytes=None,
                              stream=None):
     """w4a16_gemv that also brings next_bytes bytes at next_packed (the weights of the GEMV that
@@ -341,6 +364,14 @@ def alloc_gemv_workspace(N, K, group, device="cuda"):
     call of this shape needs one (rows short enough for one block)."""
     nbytes = w4a16_gemv_workspace_bytes(N, K, group)
     return torch.zeros(nbytes, dtype=torch.uint8, device=device) if nbytes else None
+
+
+def alloc_tc_workspace(N, K, group, device="cuda"):
+    """Zero-filled workspace for w4a16_gemm_tc (calls leave its counters zero)."""
+    nbytes = w4a16_gemm_tc_workspace_bytes(N, K, group)
+    if nbytes == 0:
+        raise W4Error("w4a16_gemm_tc_workspace_bytes", 2)
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
 def alloc_gemm_workspace(M, N, K, group, device="cuda"):

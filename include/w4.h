@@ -67,7 +67,7 @@ enum {
 };
 
 /* Kernel layouts produced by w4_prepack. */
-typedef enum { W4_LAYOUT_GEMV = 0, W4_LAYOUT_GEMM = 1 } w4_layout;
+typedef enum { W4_LAYOUT_GEMV = 0, W4_LAYOUT_GEMM = 1, W4_LAYOUT_TC = 2 } w4_layout;
 
 /* Human-readable name of a status code (static storage). */
 const char *w4_status_str(int status);
@@ -115,7 +115,7 @@ w4_status w4_quantize(const void *W_bf16, int64_t N, int64_t K, int group, int m
  *   operand: bf16 hi/lo parts of s[n,j] * z[n,j] (a function of the scales and zeros, so
  *   the canonical weight stays the only source of truth).
  *   layout W4_LAYOUT_GEMV feeds w4a16_gemv, W4_LAYOUT_GEMM feeds w4a8_gemm and (one slab per
- *   expert) w4a8_grouped_gemm. The packed buffer is opaque; its size is
+ *   expert) w4a8_grouped_gemm, W4_LAYOUT_TC feeds w4a16_gemm_tc. The packed buffer is opaque; its size is
  *   w4_prepack_bytes(N, K, group, layout) (0 for invalid arguments) and includes padding of
  *   N and K to the kernel tiles. For W4_SYM, zeros must be NULL (z = 8 is implied).
  *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG.
@@ -285,6 +285,45 @@ size_t w4a16_gemv_noalloc_scratch_limit(void);
 w4_status w4a16_gemv_noalloc(const void *x_bf16, int64_t M, const void *packed, int64_t N,
                              int64_t K, int group, int mode, void *y, int flags,
                              cudaStream_t stream);
+
+/*
+ * w4a16_gemm_tc -- the W4A16 product of w4a16_gemv for a few activation rows, on the tensor
+ *   cores (TAHOMA "Four-bit inference", the W4A16 path: 4-bit weights expanded inside the
+ *   kernel against bf16 activations with fp32 accumulation; "4-bit by default": decode at small
+ *   batch is bound by the weight bytes, so the per-weight work must not grow with the batch):
+ *     y[m, n] = sum_j s[n,j] * sum_{k in group j} (q[n,k] - z[n,j]) * x[m,k]
+ *   computed as sum_j s[n,j] (P_j - (z[n,j] - 8) X_j), P_j = sum_{k in j} (q - 8) x and
+ *   X_j = sum_{k in j} x, both on the tensor cores: the weights are expanded to the exact bf16
+ *   integers q - 8 (one expansion per weight serves all M rows), each product with a bf16
+ *   activation is exact in fp32, P_j and X_j are fp32 sums of the tensor cores, and the
+ *   group scale and zero point are applied to them in fp32. The output is rounded once (to
+ *   bf16, or kept fp32). Agreement with the exact product: about 1e-6 relative in fp32.
+ *   The (128-row tile, k-block) units of the problem are divided evenly over one CTA per SM;
+ *   CTAs sharing a tile leave partial sums in the workspace and the last of them adds them in
+ *   a fixed order, so results are bit-identical run to run on a given GPU.
+ *   x_bf16          device, bf16 [M, K]; 1 <= M <= 16
+ *   packed          device, w4_prepack(..., W4_LAYOUT_TC) of W[N, K]
+ *   y               device, bf16 [M, N], or fp32 [M, N] with W4_OUT_FP32 in flags
+ *   flags           W4_OUT_FP32 | W4_OVERLAP_PREVIOUS (as w4a16_gemv); other bits: W4_ERR_ARG
+ *   workspace       device scratch of at least w4a16_gemm_tc_workspace_bytes(N, K, group) bytes
+ *                   (partial sums for one CTA per SM of the current device, and arrival
+ *                   counters); required. Zero-fill it before its first use; every call that
+ *                   completes leaves its counters zero again. Calls that may run concurrently
+ *                   need separate workspaces. After a call whose kernel recorded an error in
+ *                   the device status, zero-fill it again.
+ *   Errors: NULL / SHAPE (M outside 1..16, N < 1 or N > 2^31, K < 32, K > 2^24, K % 32) /
+ *   GROUP / ALIGN / ARG / WORKSPACE / CUDA.
+ *
+ * w4a16_gemm_tc_schedule -- host-only query (no GPU call) of how w4a16_gemm_tc divides the
+ *   problem over `sms` SMs: out[6] receives tiles of 128 rows, k-blocks per tile, units
+ *   (tiles x k-blocks), CTAs, k per k-block (max(128, group)) and bytes per unit record.
+ *   Errors: NULL / SHAPE / GROUP.
+ */
+size_t w4a16_gemm_tc_workspace_bytes(int64_t N, int64_t K, int group);
+w4_status w4a16_gemm_tc_schedule(int64_t M, int64_t N, int64_t K, int group, int sms, int64_t *out);
+w4_status w4a16_gemm_tc(const void *x_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
+                        int group, int mode, void *y, int flags, void *workspace,
+                        size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * w4a8_gemm -- W4A8 GEMM on the FP8 tensor cores (TAHOMA "Achievement 2", the list under

@@ -58,6 +58,11 @@ def test_prepack_bytes(lib):
     for bad in [(0, 4096, 128), (16, 100, 32), (16, 4096, 48), (16, 96, 64)]:
         assert w4.w4_prepack_bytes(*bad, w4.W4_LAYOUT_GEMV) == 0
     assert w4.w4_prepack_bytes(16, 4096, 128, 7) == 0
+    # tensor-core W4A16 layout: units of 128 rows x max(128, g) k, each KS/2 code bytes per row
+    # and 4 bytes per (row, group); rows padded to 128, K to the unit's k
+    assert w4.w4_prepack_bytes(4096, 4096, 128, w4.W4_LAYOUT_TC) == 32 * 32 * (128 * 64 + 512)
+    assert w4.w4_prepack_bytes(77, 320, 32, w4.W4_LAYOUT_TC) == 1 * 3 * (128 * 64 + 4 * 512)
+    assert w4.w4_prepack_bytes(200, 768, 256, w4.W4_LAYOUT_TC) == 2 * 3 * (128 * 128 + 512)
 
 
 def test_gsum_op_cols(lib):
@@ -121,6 +126,19 @@ def test_host_validation_rejects_before_launch(lib):
               None) == 4
     assert rc("w4a16_gemv_prefetch_next", FAKE, 17, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, FAKE, 4096, None) == 2
     assert rc("w4a16_gemv_prefetch_next", FAKE, 1, FAKE, 16, 128, 128, 3, FAKE, 0, None, 0, FAKE, 4096, None) == 5
+    # tensor-core w4a16: M in 1..16, a workspace of the queried size, flags as the GEMV's
+    tws = lib.w4a16_gemm_tc_workspace_bytes(4096, 4096, 128)
+    assert tws > 0 and tws % 16 == 0
+    assert lib.w4a16_gemm_tc_workspace_bytes(4096, 100, 128) == 0
+    assert rc("w4a16_gemm_tc", None, 4, FAKE, 4096, 4096, 128, 1, FAKE, 0, FAKE, tws, None) == 1
+    assert rc("w4a16_gemm_tc", FAKE, 17, FAKE, 4096, 4096, 128, 1, FAKE, 0, FAKE, tws, None) == 2
+    assert rc("w4a16_gemm_tc", FAKE, 0, FAKE, 4096, 4096, 128, 1, FAKE, 0, FAKE, tws, None) == 2
+    assert rc("w4a16_gemm_tc", FAKE, 4, FAKE, 4096, 4096, 48, 1, FAKE, 0, FAKE, tws, None) == 3
+    assert rc("w4a16_gemm_tc", FAKE, 4, FAKE, 4096, 4096, 128, 3, FAKE, 0, FAKE, tws, None) == 5
+    assert rc("w4a16_gemm_tc", FAKE, 4, FAKE, 4096, 4096, 128, 1, FAKE, 8, FAKE, tws, None) == 5
+    assert rc("w4a16_gemm_tc", FAKE, 4, FAKE, 4096, 4096, 128, 1, FAKE + 2, 0, FAKE, tws, None) == 4
+    assert rc("w4a16_gemm_tc", FAKE, 4, FAKE, 4096, 4096, 128, 1, FAKE, 0, None, 0, None) == 10
+    assert rc("w4a16_gemm_tc", FAKE, 4, FAKE, 4096, 4096, 128, 1, FAKE, 0, FAKE, tws - 16, None) == 10
     # gemm: groups 64/128 need the codes and the group-sum operand, groups 32/256 the fp16
     # copy of the activations; K >= 128
     assert rc("w4a8_gemm", FAKE, None, FAKE, None, 4, FAKE, 16, 128, 128, 1, FAKE, 0, None, 0, None) == 1
@@ -343,3 +361,18 @@ def test_gemv_grouped_schedule_fits_one_wave_and_validates(lib):
     assert rc("w4a16_gemv_grouped", 2, ptrs, 1, ptrs, L(16, 16), L(128, 128), 128, 3, ptrs, 0, None) == 5
     # rows too long for one block (a K split would need a workspace): unsupported in a group
     assert rc("w4a16_gemv_grouped", 2, ptrs, 1, ptrs, L(16, 16), L(128, 65536), 128, 1, ptrs, 0, None) == 6
+
+
+@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 1024), (4096, 14336), (14336, 4096)])
+def test_tc_schedule_of_the_decode_shapes(lib, K, N):
+    """The tensor-core W4A16 splits tiles x k-blocks evenly over one CTA per SM."""
+    s = w4.w4a16_gemm_tc_schedule(4, N, K, 128, 148)
+    assert s["tiles"] == N // 128 and s["k_blocks"] == K // 128 and s["k_per_block"] == 128
+    assert s["units"] == s["tiles"] * s["k_blocks"] and s["ctas"] == 148
+    assert s["record_bytes"] == 128 * 64 + 512
+    small = w4.w4a16_gemm_tc_schedule(1, 77, 320, 32, 148)
+    assert small == {"tiles": 1, "k_blocks": 3, "units": 3, "ctas": 3, "k_per_block": 128,
+                     "record_bytes": 128 * 64 + 4 * 512}
+    assert rc("w4a16_gemm_tc_schedule", 17, 64, 128, 128, 148, FAKE) == 2
+    assert rc("w4a16_gemm_tc_schedule", 1, 64, 128, 96, 148, FAKE) == 3
+    assert rc("w4a16_gemm_tc_schedule", 1, 64, 128, 128, 148, None) == 1
