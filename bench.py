@@ -54,6 +54,8 @@ NCU_TRAFFIC = {
     # profiles/w4a16_gemv_m1_k14336_n4096_full.md: the kernel's own bytes (a chain of launches
     # without the L2 prefetch of the next launch's weights, caches flushed between launches)
     "w4a16_gemv M1 K14336xN4096": {"bytes": 31290624, "sha1": "b089e61bdc768133cc203b6be361c562219a81f8"},
+    # profiles/w4a16_tc_m4_k14336_n4096_full.md: w4a16_gemm_tc at M = 4 (one launch)
+    "w4a16_tc M4 K14336xN4096": {"bytes": 32818432, "sha1": "9fc6804e09b9a30d55bf9586da1ef1ca258aba9e"},
     # profiles/w4a8_gemm_prefill_traffic.md (median of 11 launches per shape)
     "w4a8_gemm M4096 K3840xN15360": {"bytes": 153379840, "sha1": "2fc13ed112d7918580956d35db9107959347192d"},
     "w4a8_gemm M4096 K15360xN3840": {"bytes": 179415552, "sha1": "2fc13ed112d7918580956d35db9107959347192d"},
@@ -531,10 +533,15 @@ def measure_rows(args, dev, pk):
             t_ms = float(np.median([time_region(lambda i: gs.replay(), 1) for _ in range(5)])) / n_l
             shapes_us[f"K{K}xN{N}"] = round(t_ms * 1e3, 3)
             del gs
+        dom_us = shapes_us["K14336xN4096"]
         rows[f"w4a16_tc_M{M}"] = {
             "value": round(gbps, 1), "unit": "GB/s", "us_per_step": round(ms * 1e3, 2), "per_shape_us": shapes_us,
             "roofline": {"bound": "hbm", "achieved": round(gbps, 1), "peak": pk["hbm"], "unit": "GB/s",
-                         "frac": round(gbps / pk["hbm"], 4)},
+                         "frac": round(gbps / pk["hbm"], 4),
+                         "launch_K14336xN4096": {
+                             "achieved": round(gemv_bytes(M, 4096, 14336) / (dom_us * 1e-6) / 1e9, 1),
+                             "traffic": traffic_for(f"w4a16_tc M{M} K14336xN4096",
+                                                    "bit_gemm_wise_b200/csrc/w4a16_tc.cu")}},
             "note": "w4a16_gemm_tc (tcgen05, W4_LAYOUT_TC), same four decode shapes and bytes as w4a16_gemv_M*"}
         del d
 
@@ -893,6 +900,10 @@ def main():
     ap.add_argument("--profile-chain", default="", metavar="K,N",
                     help="only run --launches chained M=1 GEMVs of decode shape (K, N), each naming the next "
                          "weight copy (a short, bounded run for a profiler); prints one line")
+    ap.add_argument("--profile-tc", default="", metavar="K,N",
+                    help="only run --launches w4a16_gemm_tc calls of decode shape (K, N) at M = --tc-m "
+                         "(rotating weight copies, chained like the decode step)")
+    ap.add_argument("--tc-m", type=int, default=4)
     ap.add_argument("--launches", type=int, default=8)
     ap.add_argument("--no-prefetch", action="store_true",
                     help="with --profile-chain: plain w4a16_gemv calls (the kernel's own DRAM traffic)")
@@ -915,7 +926,18 @@ def main():
     try:
         from bit_gemm_wise_b200 import w4
         w4.lib()
-        if args.profile_chain:
+        if args.profile_tc:
+            K, N = (int(v) for v in args.profile_tc.split(","))
+            dec = Decode(args.tc_m, args.seed, dev, tc=True)
+            si = dec.shapes.index((K, N))
+            for i in range(args.launches):
+                dec.gemv(si, i)
+            torch.cuda.synchronize()
+            from bit_gemm_wise_b200 import w4 as w4_
+            assert w4_.w4_device_status() == 0
+            out = {"profile_tc": f"K{K}xN{N}", "M": args.tc_m, "launches": args.launches,
+                   "bytes_per_launch": gemv_bytes(args.tc_m, N, K)}
+        elif args.profile_chain:
             K, N = (int(v) for v in args.profile_chain.split(","))
             dec = Decode(1, args.seed, dev)
             si = dec.shapes.index((K, N))

@@ -20,18 +20,20 @@
 //    into TMEM (tcgen05.st), where the MMA reads its A operand;
 //  * per group j, kind::f16 MMAs (K = 16 each) accumulate P_j into one of several 16-column
 //    TMEM buffers; promotion warps read it back and add s (P - (z - 8) X) to fp32 registers.
-//    For asymmetric weights they form X_j themselves from the activation tile in shared memory
-//    (each half-warp sums half of a stage's k for 16 rows, the halves meet by a shuffle). The
-//    product of an expanded weight and a bf16 activation is exact in fp32; rounding enters in
-//    the accumulation;
+//    For asymmetric weights a group-sum warp forms X_j from the activation tile in shared
+//    memory (each half-warp sums half of a stage's k for 16 rows, the halves meet by a
+//    shuffle) and hands it over next to the accumulator (its barrier counts the MMA commit and
+//    this warp). The product of an expanded weight and a bf16 activation is exact in fp32;
+//    rounding enters in the accumulation;
 //  * stream-K: the (tile, k-block) units of the problem, in order, are split evenly over the
 //    CTAs; when several CTAs share a tile, each warp of the last one to finish adds the
 //    others' partial sums for its 32 rows in CTA order, so results do not depend on timing;
 //  * weights (W4_LAYOUT_TC) are stored unit by unit, each unit one contiguous record, so a
 //    CTA's share is one contiguous byte range streamed by bulk copies;
-//  * warp roles: warps 0-3 expansion, 4-7 promotion (a warp touches the TMEM lane quarter
-//    warp % 4), warp 8 the producer (bulk copies of records, TMA of activation tiles), warp 9
-//    TMEM owner and single-thread MMA issuer;
+//  * warp roles: warps 0-3 and 11-14 expansion (each set half of a stage's k), 4-7 promotion
+//    (a warp touches the TMEM lane quarter warp % 4), warp 8 the producer (one bulk copy per
+//    record, TMA of activation tiles), warp 9 TMEM owner and single-thread MMA issuer, warp 10
+//    group sums;
 //  * every mbarrier wait is bounded by wall-clock time; on expiry the kernel records
 //    W4_ERR_TIMEOUT, every role sees the abort flag, TMEM is freed and the CTA returns.
 #include "w4_common.cuh"
@@ -42,12 +44,11 @@
 namespace w4 {
 namespace tc16 {
 
-constexpr int THREADS = 320;
+constexpr int THREADS = 480;
 constexpr int TM = 128;                       // weight rows per tile (MMA M)
 constexpr int TN = 16;                        // activation rows per tile (MMA N)
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per wait
 constexpr uint32_t SMEM_RING = 200 * 1024;    // shared memory for the stage ring
-constexpr uint32_t STREAM_PIECE = 4096;       // bulk copies of a record in pieces of this size
 
 // Geometry for group size G.
 template <int G> struct Geo {
@@ -75,11 +76,13 @@ template <int G> struct Geo {
 
 struct Smem {
     uint64_t full[16];      // record and activation tile landed (TMA / bulk-copy bytes)
-    uint64_t empty[16];     // the stage is free: MMA commit + 4 expansion + 4 promotion warps
+    uint64_t empty[16];     // the stage is free: MMA commit + 8 expansion + 4 promotion warps
+                            // + the group-sum warp
     uint64_t afull[4];      // an expanded stage is in TMEM (one arrival per expansion warp)
     uint64_t afree[4];      // the MMAs that read an expanded stage completed (commit)
-    uint64_t accf[8];       // a group's accumulators are complete (commit)
+    uint64_t accf[8];       // a group's accumulator (commit) and its sums X_j (group-sum warp)
     uint64_t acce[8];       // the promotion warps read them (one arrival per warp)
+    float xs[8][16];        // X_j per accumulator buffer and activation row
     uint32_t tmem_base;
     int abort;
 };
@@ -95,6 +98,8 @@ struct Args {
     int64_t L;              // units = T * NKB
     int NKB;                // k-blocks (units) per tile
     int M;
+    int mw;                 // float4 per row of a partial sum: ceil(M / 4)
+    int x3d;                // activation tiles by one 3-D TMA (K % 64 == 0), else 2-D per 64 k
     int out_fp32;
     int asym;
     int pdl;
@@ -161,6 +166,14 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
             smem_addr(dst)),
         "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_addr(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
         : "memory");
 }
 
@@ -232,6 +245,37 @@ __device__ __forceinline__ void store_row(const Args &a, int64_t n, const float 
     }
 }
 
+// Sum of the partial sums of weight row r (within its tile) over the CTAs cf..cl, in CTA order:
+// MW float4 (activation rows 4q .. 4q+3) per CTA, 16 loads in flight at a time. CTA cf's part
+// is in its slot w_first, every later CTA's in its slot 0.
+template <int MW>
+__device__ __forceinline__ void reduce_parts(const Args &a, int r, int64_t cf, int64_t cl, int w_first,
+                                             float (&sum)[TN]) {
+    constexpr int CPR = 16 / MW;  // CTAs per round
+    for (int64_t c0 = cf; c0 <= cl; c0 += CPR) {
+        float4 pv[CPR][MW];
+#pragma unroll
+        for (int j = 0; j < CPR; ++j) {
+            const int64_t c = c0 + j <= cl ? c0 + j : cl;
+            const int wc = c == cf ? w_first : 0;
+            const float4 *src = reinterpret_cast<const float4 *>(a.part + (((size_t)c * 2 + wc) * TM + r) * TN);
+#pragma unroll
+            for (int q = 0; q < MW; ++q) pv[j][q] = __ldcg(src + q);
+        }
+#pragma unroll
+        for (int j = 0; j < CPR; ++j) {
+            if (c0 + j > cl) break;
+#pragma unroll
+            for (int q = 0; q < MW; ++q) {
+                sum[4 * q] += pv[j][q].x;
+                sum[4 * q + 1] += pv[j][q].y;
+                sum[4 * q + 2] += pv[j][q].z;
+                sum[4 * q + 3] += pv[j][q].w;
+            }
+        }
+    }
+}
+
 template <int G>
 __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const Args a) {
     using GE = Geo<G>;
@@ -248,14 +292,14 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
     if (threadIdx.x == 0) {
         for (int s = 0; s < GE::NS; ++s) {
             mbar_init(&sm->full[s], 1);
-            mbar_init(&sm->empty[s], 9);
+            mbar_init(&sm->empty[s], 14);
         }
         for (int s = 0; s < GE::NA; ++s) {
-            mbar_init(&sm->afull[s], 4);
+            mbar_init(&sm->afull[s], 8);
             mbar_init(&sm->afree[s], 1);
         }
         for (int b = 0; b < GE::NACC; ++b) {
-            mbar_init(&sm->accf[b], 1);
+            mbar_init(&sm->accf[b], 2);
             mbar_init(&sm->acce[b], 4);
         }
         sm->abort = 0;
@@ -285,13 +329,14 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
                 if (!wait1(&sm->empty[rs.slot], rs.phase ^ 1u, sm, a.status)) break;
                 uint8_t *st = base + (size_t)rs.slot * GE::STAGE;
                 mbar_arrive_expect_tx(&sm->full[rs.slot], GE::XB + GE::REC);
-                for (uint32_t o = 0; o < GE::REC; o += STREAM_PIECE) {
-                    const uint32_t nb = GE::REC - o < STREAM_PIECE ? GE::REC - o : STREAM_PIECE;
-                    bulk_g2s_stream(st + GE::XB + o, src + o, nb, &sm->full[rs.slot]);
-                }
+                bulk_g2s_stream(st + GE::XB, src, GE::REC, &sm->full[rs.slot]);
+                if (a.x3d) {
+                    tma_load_3d(st, &tm_x, 0, 0, kb * (GE::KS / 64), &sm->full[rs.slot]);
+                } else {
 #pragma unroll
-                for (int h = 0; h < GE::KS / 64; ++h)
-                    tma_load_2d(st + h * (TN * 128), &tm_x, kb * GE::KS + 64 * h, 0, &sm->full[rs.slot]);
+                    for (int h = 0; h < GE::KS / 64; ++h)
+                        tma_load_2d(st + h * (TN * 128), &tm_x, kb * GE::KS + 64 * h, 0, &sm->full[rs.slot]);
+                }
                 kb = kb + 1 == a.NKB ? 0 : kb + 1;
                 ++issued;
             }
@@ -338,10 +383,12 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
                 (void)mbar_wait_bounded(&sm->afree[i % GE::NA], (uint32_t)(i / GE::NA) & 1u, a.status);
         }
         __syncwarp();
-    } else if (warp < 4) {
-        // ------------------------------------------------ expansion (row 32 warp + lane)
-        const int r = warp * 32 + lane;
-        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    } else if (warp < 4 || warp >= 11) {
+        // ------------------------------------------------ expansion (row 32 (warp % 4) + lane;
+        // warps 0-3 take the first half of a stage's code chunks, warps 11-14 the second)
+        const int q4 = warp & 3, r = q4 * 32 + lane;
+        const int c0 = warp < 4 ? 0 : GE::CHUNKS / 2;
+        const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
         Ring<GE::NS> rs;
         Ring<GE::NA> ra;
         for (int i = 0; i < n_units; ++i, rs.next(), ra.next()) {
@@ -349,17 +396,17 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
             if (!warp_wait(&sm->afree[ra.slot], ra.phase ^ 1u, sm, a.status)) break;
             tc_fence_after();
             const uint32_t rec = smem_addr(base + (size_t)rs.slot * GE::STAGE + GE::XB);
-            uint4 cw[GE::CHUNKS];
+            uint4 cw[GE::CHUNKS / 2];
 #pragma unroll
-            for (int c = 0; c < GE::CHUNKS; ++c) cw[c] = lds128(rec + (uint32_t)(c * TM + r) * 16u);
+            for (int c = 0; c < GE::CHUNKS / 2; ++c) cw[c] = lds128(rec + (uint32_t)((c0 + c) * TM + r) * 16u);
 #pragma unroll
-            for (int c = 0; c < GE::CHUNKS; ++c) {
+            for (int c = 0; c < GE::CHUNKS / 2; ++c) {
                 uint32_t o[16];
                 expand_word(cw[c].x, o);
                 expand_word(cw[c].y, o + 4);
                 expand_word(cw[c].z, o + 8);
                 expand_word(cw[c].w, o + 12);
-                tmem_st16(tl + (uint32_t)(ra.slot * GE::ACOLS + c * 16), o);
+                tmem_st16(tl + (uint32_t)(ra.slot * GE::ACOLS + (c0 + c) * 16), o);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -389,27 +436,6 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
             uint32_t sc[GE::GPS];
 #pragma unroll
             for (int gg = 0; gg < GE::GPS; ++gg) sc[gg] = lds32(scb + (uint32_t)(gg * TM + r) * 4u);
-            // X_j of activation row (lane & 15): this half-warp's half of the stage's k, read from
-            // the 128-byte-swizzled tile (16-byte chunk c of row t of a 64-k atom sits at chunk
-            // c ^ (t & 7)), summed in k order per group; a group wider than half a stage is
-            // completed with the other half's sum
-            float xsum[GE::XPL];
-#pragma unroll
-            for (int j = 0; j < GE::XPL; ++j) xsum[j] = 0.0f;
-            if (a.asym) {
-                const int tr = lane & 15, h = lane >> 4;
-                const uint32_t xb = smem_addr(base + (size_t)rs.slot * GE::STAGE);
-#pragma unroll
-                for (int c = 0; c < GE::HALF / 8; ++c) {   // 8 k per chunk
-                    const int kin = h * GE::HALF + 8 * c;   // k of the chunk within the stage
-                    const uint4 v = lds128(xb + (uint32_t)((kin >> 6) * (TN * 128) + tr * 128 + ((((kin >> 3) & 7) ^ (tr & 7)) << 4)));
-                    const int j = GE::XPL > 1 ? (8 * c) / G : 0;
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) xsum[j] += __uint_as_float(w[q] << 16) + __uint_as_float(w[q] & 0xFFFF0000u);
-                }
-                if (G > GE::HALF) xsum[0] += __shfl_xor_sync(FULL, xsum[0], 16);
-            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm->empty[rs.slot]);
 #pragma unroll
@@ -418,20 +444,24 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
                 tc_fence_after();
                 uint32_t v[16];
                 tmem_ld16(tl + (uint32_t)(GE::COL_ACC + rb.slot * TN), v);
+                float X[TN];
+                const float4 *xq = reinterpret_cast<const float4 *>(sm->xs[rb.slot]);
+#pragma unroll
+                for (int q = 0; q < TN / 4; ++q) {
+                    const float4 f = xq[q];
+                    X[4 * q] = f.x;
+                    X[4 * q + 1] = f.y;
+                    X[4 * q + 2] = f.z;
+                    X[4 * q + 3] = f.w;
+                }
                 tmem_wait_ld(v);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->acce[rb.slot]);
                 const float s = __half2float(__ushort_as_half((unsigned short)(sc[gg] & 0xFFFFu)));
                 const float zf = (float)((int)(int16_t)(sc[gg] >> 16) - 8);
-                // group gg's sums sit in the half-warp that covers its k (register gg % XPL)
-                const int hsrc = G <= GE::HALF ? 16 * (gg / GE::XPL) : 0;
-                const float xg = xsum[G <= GE::HALF ? gg % GE::XPL : 0];
 #pragma unroll
-                for (int m = 0; m < TN; ++m) {
-                    const float X = __shfl_sync(FULL, xg, hsrc + m);
-                    acc[m] = fmaf(s, fmaf(-zf, X, __uint_as_float(v[m])), acc[m]);
-                }
+                for (int m = 0; m < TN; ++m) acc[m] = fmaf(s, fmaf(-zf, X[m], __uint_as_float(v[m])), acc[m]);
             }
             if (!ok) break;
             if (i + 1 < n_units && kb + 1 < a.NKB) {
@@ -446,7 +476,8 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
                 const int which = t == t0 ? 0 : 1;  // a CTA's first segment, or its last
                 float4 *dst = reinterpret_cast<float4 *>(a.part + (((size_t)blockIdx.x * 2 + which) * TM + r) * TN);
 #pragma unroll
-                for (int q = 0; q < TN / 4; ++q) dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+                for (int q = 0; q < TN / 4; ++q)
+                    if (q < a.mw) dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
                 __threadfence();
                 __syncwarp();
                 const int64_t cf = unit_owner(t * a.NKB, a.L, P), cl = unit_owner(t * a.NKB + a.NKB - 1, a.L, P);
@@ -462,28 +493,11 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
                     float sum[TN];
 #pragma unroll
                     for (int m = 0; m < TN; ++m) sum[m] = 0.0f;
-                    // four CTAs' parts in flight at a time, added in CTA order
-                    for (int64_t c0 = cf; c0 <= cl; c0 += 4) {
-                        float4 pv[4][TN / 4];
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int64_t c = c0 + j <= cl ? c0 + j : cl;
-                            const int wc = c == cf ? w_first : 0;
-                            const float4 *src = reinterpret_cast<const float4 *>(a.part + (((size_t)c * 2 + wc) * TM + r) * TN);
-#pragma unroll
-                            for (int q = 0; q < TN / 4; ++q) pv[j][q] = __ldcg(src + q);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            if (c0 + j > cl) break;
-#pragma unroll
-                            for (int q = 0; q < TN / 4; ++q) {
-                                sum[4 * q] += pv[j][q].x;
-                                sum[4 * q + 1] += pv[j][q].y;
-                                sum[4 * q + 2] += pv[j][q].z;
-                                sum[4 * q + 3] += pv[j][q].w;
-                            }
-                        }
+                    switch (a.mw) {
+                        case 1: reduce_parts<1>(a, r, cf, cl, w_first, sum); break;
+                        case 2: reduce_parts<2>(a, r, cf, cl, w_first, sum); break;
+                        case 3: reduce_parts<3>(a, r, cf, cl, w_first, sum); break;
+                        default: reduce_parts<4>(a, r, cf, cl, w_first, sum); break;
                     }
                     store_row(a, n, sum);
                     if (lane == 0) a.cnt[t * 4 + q4] = 0u;  // ready for the next call
@@ -494,6 +508,47 @@ __global__ void __launch_bounds__(THREADS, 1) w4a16_tc_kernel(const __grid_const
             ++t;
             kb = 0;
             seg_kb = 0;
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------ group sums X_j of the activation rows
+        Ring<GE::NS> rs;
+        Ring<GE::NACC> rb;
+        const int tr = lane & 15, h = lane >> 4;
+        for (int i = 0; i < n_units; ++i, rs.next()) {
+            if (!warp_wait(&sm->full[rs.slot], rs.phase, sm, a.status)) break;
+            // row tr: this half-warp's half of the stage's k, read from the 128-byte-swizzled
+            // tile (16-byte chunk c of row t of a 64-k atom sits at chunk c ^ (t & 7)), summed
+            // in k order per group; a group wider than half a stage is completed with the other
+            // half's sum
+            float xsum[GE::XPL];
+#pragma unroll
+            for (int j = 0; j < GE::XPL; ++j) xsum[j] = 0.0f;
+            if (a.asym) {
+                const uint32_t xb = smem_addr(base + (size_t)rs.slot * GE::STAGE);
+#pragma unroll
+                for (int c = 0; c < GE::HALF / 8; ++c) {   // 8 k per chunk
+                    const int kin = h * GE::HALF + 8 * c;   // k of the chunk within the stage
+                    const uint4 v = lds128(xb + (uint32_t)((kin >> 6) * (TN * 128) + tr * 128 + ((((kin >> 3) & 7) ^ (tr & 7)) << 4)));
+                    const int j = GE::XPL > 1 ? (8 * c) / G : 0;
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) xsum[j] += __uint_as_float(w[q] << 16) + __uint_as_float(w[q] & 0xFFFF0000u);
+                }
+                if (G > GE::HALF) xsum[0] += __shfl_xor_sync(FULL, xsum[0], 16);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->empty[rs.slot]);
+            bool ok = true;
+#pragma unroll
+            for (int gg = 0; gg < GE::GPS; ++gg, rb.next()) {
+                if (!warp_wait(&sm->acce[rb.slot], rb.phase ^ 1u, sm, a.status)) { ok = false; break; }
+                // group gg lies in half gg / XPL (register gg % XPL) when a group fits in a half
+                const int hg = G <= GE::HALF ? gg / GE::XPL : 0;
+                if (h == hg) sm->xs[rb.slot][tr] = xsum[G <= GE::HALF ? gg % GE::XPL : 0];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->accf[rb.slot]);
+            }
+            if (!ok) break;
         }
     }
 
@@ -534,6 +589,10 @@ bool tc_shape_ok(int64_t M, int64_t N, int64_t K) {
 }
 
 int64_t tc_tiles(int64_t N) { return (N + tc16::TM - 1) / tc16::TM; }
+
+// CTAs per 128-row tile at most: a tile shared by more CTAs finishes with a longer ordered
+// reduction of their partial sums than the extra units per CTA cost.
+constexpr int64_t kMaxPerTile = 8;
 
 template <int G>
 w4_status tc_start(const CUtensorMap &tm, const tc16::Args &a, int grid, cudaStream_t stream) {
@@ -576,7 +635,8 @@ W4_API w4_status w4a16_gemm_tc_schedule(int64_t M, int64_t N, int64_t K, int gro
     if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
     const int ks = TcLayoutGeo::ks(group);
     const int64_t nkb = (K + ks - 1) / ks, T = tc_tiles(N), L = T * nkb;
-    const int64_t grid = L < sms ? L : sms;
+    const int64_t gmax = T * kMaxPerTile < (int64_t)sms ? T * kMaxPerTile : (int64_t)sms;
+    const int64_t grid = L < gmax ? L : gmax;
     out[0] = T;
     out[1] = nkb;
     out[2] = L;
@@ -603,19 +663,33 @@ W4_API w4_status w4a16_gemm_tc(const void *x_bf16, int64_t M, const void *packed
     const int ks = TcLayoutGeo::ks(group);
     const int64_t nkb = (K + ks - 1) / ks, T = tc_tiles(N), L = T * nkb;
     const int sms = num_sms();
-    const int grid = (int)(L < sms ? L : sms);
+    const int64_t gmax = T * kMaxPerTile < (int64_t)sms ? T * kMaxPerTile : (int64_t)sms;
+    const int grid = (int)(L < gmax ? L : gmax);
 
     // bf16 [M][K]: boxes of 64 k (128 bytes) x 16 rows with the 128-byte swizzle (the MMA's
     // K-major layout); rows past M and k past K read as zero
     CUtensorMap tm;
-    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)tc16::TN};
-    const cuuint32_t es[2] = {1, 1};
-    if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x_bf16), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return W4_ERR_CUDA;
+    const bool x3d = K % 64 == 0;
+    if (x3d) {
+        // [K/64 atoms][M rows][64 k]: one box holds a whole stage (KS/64 atoms of 16 rows)
+        const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
+        const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+        const cuuint32_t box[3] = {64, (cuuint32_t)tc16::TN, (cuuint32_t)(ks / 64)};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(x_bf16), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+    } else {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {64, (cuuint32_t)tc16::TN};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x_bf16), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W4_ERR_CUDA;
+    }
 
     tc16::Args a;
     a.w = static_cast<const uint8_t *>(packed);
@@ -628,6 +702,8 @@ W4_API w4_status w4a16_gemm_tc(const void *x_bf16, int64_t M, const void *packed
     a.L = L;
     a.NKB = (int)nkb;
     a.M = (int)M;
+    a.mw = (int)((M + 3) / 4);
+    a.x3d = x3d ? 1 : 0;
     a.out_fp32 = (flags & W4_OUT_FP32) ? 1 : 0;
     a.asym = mode == W4_ASYM ? 1 : 0;
     a.pdl = (flags & W4_OVERLAP_PREVIOUS) ? 1 : 0;

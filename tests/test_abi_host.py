@@ -365,10 +365,12 @@ def test_gemv_grouped_schedule_fits_one_wave_and_validates(lib):
 
 @pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 1024), (4096, 14336), (14336, 4096)])
 def test_tc_schedule_of_the_decode_shapes(lib, K, N):
-    """The tensor-core W4A16 splits tiles x k-blocks evenly over one CTA per SM."""
+    """The tensor-core W4A16 splits tiles x k-blocks evenly over at most one CTA per SM and
+    eight per 128-row tile."""
     s = w4.w4a16_gemm_tc_schedule(4, N, K, 128, 148)
     assert s["tiles"] == N // 128 and s["k_blocks"] == K // 128 and s["k_per_block"] == 128
-    assert s["units"] == s["tiles"] * s["k_blocks"] and s["ctas"] == 148
+    # at most 8 CTAs per tile, at most one per SM
+    assert s["units"] == s["tiles"] * s["k_blocks"] and s["ctas"] == min(148, 8 * s["tiles"])
     assert s["record_bytes"] == 128 * 64 + 512
     small = w4.w4a16_gemm_tc_schedule(1, 77, 320, 32, 148)
     assert small == {"tiles": 1, "k_blocks": 3, "units": 3, "ctas": 3, "k_per_block": 128,
