@@ -37,6 +37,7 @@
 //    W4_ERR_TIMEOUT, every role sees the abort flag, TMEM is freed and the CTA returns.
 #include "w4_common.cuh"
 #include "w4_layout.cuh"
+#include "w4_rowquant.cuh"
 
 #include <cuda.h>
 
@@ -70,8 +71,17 @@ struct Smem {
     uint64_t acc_empty[NBUF];  // promotion finished reading it (one arrival per warp)
     uint32_t tmem_base;
     int abort;
+    // the row quant of the kernel variant that quantizes its own activation rows, before the
+    // ring is in use: two halves of row slots in the ring, each completed by one barrier, and
+    // the scale, its reciprocal and the special-row mark of each row of the current batch
+    uint64_t rq_full[2];
+    float rq_s[16], rq_r[16];
+    uint32_t rq_sp[16];
+    uint32_t rq_mb[16];  // the batch's row maxima (magnitude bits), combined by atomicMax
 };
 static_assert(sizeof(Smem) <= 1024, "control block");
+constexpr uint32_t RING_BYTES = STAGES * (RAW_BYTES + A_BYTES);  // ring data bytes (row slots before the GEMM)
+constexpr int RQ_MAX_SLOTS = 32;
 
 struct Args {
     const uint8_t *packed;         // slab 0
@@ -92,6 +102,15 @@ struct Args {
     int64_t PS;
     float *part;                   // split tiles: 2 PS partial-result slots (PART_FLOATS each)
     uint32_t *cnt;                 // split tiles: R x 8 arrival counters (zero between calls)
+    // kernels that quantize their own activation rows (FUSE):
+    const uint16_t *xq;            // bf16 activations [M, K]
+    uint8_t *q8;                   // their E4M3 codes [M, K] (row_scale points at their scales)
+    float *qscale;                 // row scales [M]
+    uint16_t *qgop;                // group-sum operand [M, KZ]
+    uint32_t *qcnt;                // per token tile: rows quantized so far (zero at launch)
+    int64_t KZ;                    // columns of the group-sum operand
+    int64_t qa1, qa2;              // rows [0, qa1) and [qa2, M) first, by every warp; the rest by warps 2-3
+    int qstaged;                   // rows staged through the ring by bulk copies (rows of <= half the ring)
 };
 
 // ------------------------------------------------------------------ split-K schedule
@@ -447,7 +466,286 @@ __device__ __noinline__ bool split_combine(float *part_base, uint32_t *cnt, int 
     return true;
 }
 
-template <int G>  // group size: 32, 64 or 128
+// ------------------------------------------------------------------ row quant inside the GEMM
+// The kernel variant that takes bf16 activations quantizes every activation row itself
+// ("Four-bit inference ... Tahoma", Achievement 2: the per-token scale is recomputed on every
+// forward pass) into the workspace -- E4M3 codes, row scale, group-sum operand, the same
+// values as fp8_row_quant bit for bit -- and the tiles then read those rows like the
+// operands of the two-launch path. One warp quantizes one row: the max over the row's
+// magnitude bits, the row scale and its reciprocal, then a second pass over the row (from
+// L2) that converts, stores the codes and adds each group's codes exactly as integers in
+// units of 2^-9. A finished row is counted in its token tile's counter by a release add
+// after a proxy fence, so that the TMA (async proxy) loads issued after an acquire load of a
+// full count see it. The readers use acquire loads, not fences: a gpu-scope fence would wait
+// for the reader's own earlier stores (the previous tile's outputs) to drain.
+__device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded wait until the counter at p reaches n (acquire); on expiry records W4_ERR_TIMEOUT
+// and raises the CTA's abort flag.
+__device__ __forceinline__ bool count_reached(const uint32_t *p, uint32_t n, Smem *sm, int *status) {
+    if (ld_acquire(p) >= n) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire(p) < n) {
+        if (*(volatile int *)&sm->abort) return false;
+        if (globaltimer_ns() - t0 > kWaitNs) {
+            *(volatile int *)&sm->abort = 1;
+            record_status(status, W4_ERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(128);
+    }
+    return true;
+}
+
+template <int G>
+__device__ __forceinline__ void quant_row_warp(const uint16_t *__restrict__ xq, int64_t K, int64_t KZ, int64_t m,
+                                               int64_t next, int64_t next2, uint8_t *q8, float *qscale,
+                                               uint16_t *qgop, uint32_t *qcnt) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nchunk = K / 8, J = K / G;
+    const uint4 *src = reinterpret_cast<const uint4 *>(xq + m * K);
+    // the warp's next rows into L2 while this one is worked on (a warp holds few loads in flight)
+    if (lane == 0 && next >= 0) bulk_prefetch_l2(xq + next * K, (uint32_t)(K * 2));
+    if (lane == 0 && next2 >= 0) bulk_prefetch_l2(xq + next2 * K, (uint32_t)(K * 2));
+    // pass 1: max over the magnitude bits, eight 16-byte loads per lane in flight
+    // (every loop below runs the same trip count on every lane: the group sums are warp
+    // shuffles over all 32 lanes)
+    uint32_t mb = 0;
+    for (int64_t b = 0; b < nchunk; b += 32 * 8) {
+        const int64_t c0 = b + lane;
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = c0 + 32 * u < nchunk ? __ldg(src + c0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mb = absmax_bits(mb, v[u]);
+    }
+    mb = __reduce_max_sync(FULL, __vmaxu2(mb, mb >> 16) & 0xFFFFu);
+    const bool special = mb >= 0x7F80u;  // an infinity or a NaN in the row
+    float amax = __uint_as_float(mb << 16);
+    if (mb > 0x7F80u) {  // NaN: the maximum of the other values (non-negative floats order as bits)
+        float x = 0.0f;
+        for (int64_t c = lane; c < nchunk; c += 32) x = absmax_float(x, __ldg(src + c));
+        amax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(x)));
+    }
+    const float s = scale_of(amax);
+    const float r = __frcp_rn(s);
+    if (lane == 0) qscale[m] = s;
+    uint2 *dst = reinterpret_cast<uint2 *>(q8 + m * K);
+    uint16_t *gop = qgop + m * KZ;
+    // pass 2 (from L2), four rounds of 32 chunks per iteration with their loads issued first;
+    // a group's G / 8 chunks sit on consecutive lanes of one round (32 * 8 is a multiple of G),
+    // so its sum is a butterfly over those lanes
+    for (int64_t b = 0; b < nchunk; b += 32 * 4) {
+        const int64_t c0 = b + lane;
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = c0 + 32 * u < nchunk ? __ldg(src + c0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t c = c0 + 32 * u;
+            const bool live = c < nchunk;
+            int isum = 0;
+            if (live) {
+                const uint2 o = special ? quantize8<true>(v[u], s, r) : quantize8<false>(v[u], s, r);
+                dst[c] = o;
+                isum = e4m3x8_sum_times512(o.x, o.y);
+            }
+#pragma unroll
+            for (int off = 1; off < G / 8; off <<= 1) isum += __shfl_xor_sync(FULL, isum, off);
+            if (live && (lane & (G / 8 - 1)) == 0) {
+                const float gs = __fmul_rn(__int2float_rn(isum), 0.001953125f);
+                const uint16_t hi = bf16_rn_bits(gs);
+                const int64_t j = (c * 8) / G;
+                gop[j] = hi;
+                gop[J + j] = bf16_rn_bits(__fsub_rn(gs, __uint_as_float((uint32_t)hi << 16)));
+                gop[2 * J + j] = hi;
+            }
+        }
+    }
+    for (int64_t t = 3 * J + lane; t < KZ; t += 32) gop[t] = 0;
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) red_release_add(qcnt + m / BN, 1u);
+}
+
+// The rows [0, qa1) and [qa2, M) quantized by the CTAs before the GEMM's roles start, staged
+// through the (still unused) ring: the CTA's rows (index i = blockIdx.x + k * gridDim.x of that
+// row set) go by batches of h rows into one half of the ring's row slots by bulk copies, while
+// the other half's batch is worked on, so HBM streams the rows at full rate instead of one
+// warp's loads in flight at a time.
+// Per batch: all 16 warps take the rows' maxima by rounds of 32 chunks (combined per row in
+// shared memory), one warp per row forms the row's scale; then all 16 warps convert the batch
+// by rounds of 32 chunks (a round holds whole groups, whose sums are warp butterflies) and
+// store codes and group-sum operand; at the batch's end every thread
+// fences its stores for the async proxy, and after the block barrier one gpu-scope fence
+// (cumulative over the block's stores) precedes the release adds that count each row in its
+// token tile. Returns false (every thread alike) if a bulk copy did not land in time.
+template <int G>
+__device__ __forceinline__ bool quant_rows_staged(const Args &a, uint8_t *ring, Smem *sm) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t K = a.K, nchunk = K / 8, J = K / G;
+    const uint32_t row_bytes = (uint32_t)(K * 2);
+    int nslots = (int)(RING_BYTES / row_bytes);
+    if (nslots > RQ_MAX_SLOTS) nslots = RQ_MAX_SLOTS;
+    const int h = nslots / 2;  // rows per batch (>= 1: the host stages only rows of <= half the ring)
+    const int64_t nA1 = a.qa1, nA = a.qa1 + (a.M - a.qa2);  // the row set: [0, qa1) then [qa2, M)
+    const int64_t nr = blockIdx.x < nA ? (nA - 1 - blockIdx.x) / gridDim.x + 1 : 0;  // rows of this CTA
+    const int64_t nb = (nr + h - 1) / h;
+    auto row_of = [&](int64_t k) {  // the CTA's k-th row
+        const int64_t i = blockIdx.x + k * (int64_t)gridDim.x;
+        return i < nA1 ? i : a.qa2 + (i - nA1);
+    };
+    auto batch_rows = [&](int64_t b) { return (int)(nr - b * h < h ? nr - b * h : h); };
+    auto issue = [&](int64_t b) {  // thread 0: batch b into half b & 1
+        const int half = (int)(b & 1), n = batch_rows(b);
+        mbar_arrive_expect_tx(&sm->rq_full[half], (uint32_t)n * row_bytes);
+        for (int i = 0; i < n; ++i) {
+            const int64_t m = row_of(b * h + i);
+            bulk_g2s(ring + (size_t)(half * h + i) * row_bytes, a.xq + m * K, row_bytes, &sm->rq_full[half]);
+        }
+    };
+    if (threadIdx.x == 0) {
+        mbar_init(&sm->rq_full[0], 1);
+        mbar_init(&sm->rq_full[1], 1);
+        fence_mbar_init();
+    }
+    if (threadIdx.x < 16) sm->rq_mb[threadIdx.x] = 0u;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (nb > 0) issue(0);
+        if (nb > 1) issue(1);
+    }
+    bool ok = true;
+    for (int64_t b = 0; b < nb; ++b) {
+        const int half = (int)(b & 1), n = batch_rows(b);
+        const uint8_t *slots = ring + (size_t)half * h * row_bytes;
+        bool got = true;
+        if (lane == 0) got = wait_phase(&sm->rq_full[half], (uint32_t)(b >> 1) & 1u, sm, a.status);
+        got = __shfl_sync(FULL, got ? 1 : 0, 0) != 0;
+        if (got) got = __all_sync(FULL, mbar_try_wait_short(&sm->rq_full[half], (uint32_t)(b >> 1) & 1u));
+        ok = __syncthreads_and(got ? 1 : 0) != 0;
+        if (!ok) break;
+        // max over each row's magnitude bits: each row's rounds of 32 chunks spread over the 16
+        // warps (row outer, round inner: warp-uniform trip counts, no division)
+        for (int i = 0; i < n; ++i) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(slots + (size_t)i * row_bytes);
+            uint32_t mb = 0;
+            for (int64_t c0 = (int64_t)warp * 32; c0 < nchunk; c0 += THREADS)
+                if (c0 + lane < nchunk) mb = absmax_bits(mb, src[c0 + lane]);
+            mb = __reduce_max_sync(FULL, __vmaxu2(mb, mb >> 16) & 0xFFFFu);
+            if (lane == 0 && mb) atomicMax(&sm->rq_mb[i], mb);
+        }
+        __syncthreads();
+        // scale of row i (warp i), the NaN rows' max over the other values, the group-sum
+        // operand's zero padding
+        if (warp < n) {
+            const int64_t m = row_of(b * h + warp);
+            const uint32_t mb = sm->rq_mb[warp];
+            float amax = __uint_as_float(mb << 16);
+            if (mb > 0x7F80u) {  // NaN: the maximum of the other values
+                const uint4 *src = reinterpret_cast<const uint4 *>(slots + (size_t)warp * row_bytes);
+                float x = 0.0f;
+                for (int64_t c = lane; c < nchunk; c += 32) x = absmax_float(x, src[c]);
+                amax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(x)));
+            }
+            const float sc = scale_of(amax);
+            __syncwarp();  // every lane has read rq_mb[warp] before lane 0 clears it
+            if (lane == 0) {
+                a.qscale[m] = sc;
+                sm->rq_s[warp] = sc;
+                sm->rq_r[warp] = __frcp_rn(sc);
+                sm->rq_sp[warp] = mb >= 0x7F80u ? 1u : 0u;  // an infinity or a NaN in the row
+                sm->rq_mb[warp] = 0u;                        // for the next batch
+            }
+            uint16_t *gop = a.qgop + m * a.KZ;
+            for (int64_t t = 3 * J + lane; t < a.KZ; t += 32) gop[t] = 0;
+        }
+        __syncthreads();
+        // codes and group sums: each row's rounds of 32 chunks spread over the 16 warps (a round
+        // holds whole groups)
+        for (int i = 0; i < n; ++i) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(slots + (size_t)i * row_bytes);
+            const int64_t m = row_of(b * h + i);
+            const float sc = sm->rq_s[i], rc = sm->rq_r[i];
+            const bool sp = sm->rq_sp[i] != 0u;
+            uint2 *dst = reinterpret_cast<uint2 *>(a.q8 + m * K);
+            uint16_t *gop = a.qgop + m * a.KZ;
+            for (int64_t c0 = (int64_t)warp * 32; c0 < nchunk; c0 += THREADS) {
+                const int64_t c = c0 + lane;
+                const bool live = c < nchunk;
+                int isum = 0;
+                if (live) {
+                    const uint2 o = sp ? quantize8<true>(src[c], sc, rc) : quantize8<false>(src[c], sc, rc);
+                    dst[c] = o;
+                    isum = e4m3x8_sum_times512(o.x, o.y);
+                }
+#pragma unroll
+                for (int off = 1; off < G / 8; off <<= 1) isum += __shfl_xor_sync(FULL, isum, off);
+                if (live && (lane & (G / 8 - 1)) == 0) {
+                    const float gs = __fmul_rn(__int2float_rn(isum), 0.001953125f);
+                    const uint16_t hi = bf16_rn_bits(gs);
+                    const int64_t j = (c * 8) / G;
+                    gop[j] = hi;
+                    gop[J + j] = bf16_rn_bits(__fsub_rn(gs, __uint_as_float((uint32_t)hi << 16)));
+                    gop[2 * J + j] = hi;
+                }
+            }
+        }
+        // the batch's stores visible to the gpu and to the async proxy; this CTA's reads of the
+        // slots ordered before the bulk copies (async proxy) that refill them
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (warp == 0) {
+            if (lane == 0) __threadfence();
+            __syncwarp();
+            if (lane < n) red_release_add(a.qcnt + row_of(b * h + lane) / BN, 1u);
+        }
+        if (threadIdx.x == 0 && b + 2 < nb) issue(b + 2);
+    }
+    return ok;
+}
+
+// The producer's wait for the rows of the token tile at row0 (n rows): then the async proxy's
+// loads of them are ordered after the acquire.
+__device__ __forceinline__ bool rows_ready(const uint32_t *qcnt, int64_t row0, int64_t n, Smem *sm, int *status) {
+    if (!count_reached(qcnt + row0 / BN, (uint32_t)n, sm, status)) return false;
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
+}
+
+// A promotion lane's four row scales (token columns half * 128 + 32 c + lane of the tile at
+// row0), written by this kernel: the tile's count acquired first (one acquire load per lane),
+// the scales read through L2; columns past the tile's rows give 0. NaN in x when the wait ran
+// out (kept out of line so that the promotion loop's registers are those of the two-launch
+// kernel).
+__device__ __noinline__ float4 fused_row_scales(const uint32_t *qcnt, const float *row_scale, int64_t row0,
+                                                int64_t rows, int64_t M, int half, Smem *sm, int *status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t n = M - row0 < (int64_t)BN ? M - row0 : (int64_t)BN;
+    if (!count_reached(qcnt + row0 / BN, (uint32_t)n, sm, status))
+        return make_float4(__int_as_float(0x7fffffff), 0.0f, 0.0f, 0.0f);
+    float v[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int col = half * 128 + c * 32 + lane;
+        const int64_t m = row0 + col;
+        v[c] = (col < rows && m < M) ? __ldcg(row_scale + m) : 0.0f;
+    }
+    return make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// group size: 32, 64 or 128; FUSE: the activation rows are quantized by this kernel
+template <int G, bool FUSE>
 __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                           const __grid_constant__ CUtensorMap tm_act,
                                                           const __grid_constant__ CUtensorMap tm_zop,
@@ -486,18 +784,52 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
 
+    if (FUSE && a.qstaged) {
+        // the first tiles' rows (or every row), staged through the ring before it holds any stage
+        quant_rows_staged<G>(a, base, sm);
+        __syncthreads();
+    } else if (FUSE) {
+        // the rows the first tiles of every CTA read, by every warp of the grid: [0, qa1)
+        // (token tiles of the first wave of whole tiles) and [qa2, M) (token tiles of the
+        // split tiles, which CTAs take first)
+        // (CTA index fastest, so that the rows spread over every SM)
+        const int64_t nA1 = a.qa1, nA = a.qa1 + (a.M - a.qa2), step = (int64_t)gridDim.x * (THREADS / 32);
+        for (int64_t i = (int64_t)warp * gridDim.x + blockIdx.x; i < nA; i += step) {
+            const int64_t in = i + step;
+            quant_row_warp<G>(a.xq, a.K, a.KZ, i < nA1 ? i : a.qa2 + (i - nA1),
+                              in < nA ? (in < nA1 ? in : a.qa2 + (in - nA1)) : -1, -1, a.q8, a.qscale, a.qgop,
+                              a.qcnt);
+        }
+    }
+
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
-        if (warp == 0 && lane == 0) {
+        if (FUSE && warp >= 2) {
+            // ------------------------------------------------ row quant of the later token tiles
+            // (warps 2 and 3 of every CTA, in row order, while the tiles of the first rows run;
+            // these warps wait on nothing, so the rows always come out)
+            const int64_t step = (int64_t)gridDim.x * 2;
+            const int64_t m0 = a.qa1 + (int64_t)(warp - 2) * gridDim.x + blockIdx.x;
+            if (lane == 0 && m0 < a.qa2) bulk_prefetch_l2(a.xq + m0 * a.K, (uint32_t)(a.K * 2));
+            for (int64_t m = m0; m < a.qa2; m += step)
+                quant_row_warp<G>(a.xq, a.K, a.KZ, m, m + step < a.qa2 ? m + step : -1,
+                                  m + 2 * step < a.qa2 ? m + 2 * step : -1, a.q8, a.qscale, a.qgop, a.qcnt);
+        } else if (warp == 0 && lane == 0) {
             // ------------------------------------------------ TMA producer
             Ring r;
             int64_t uses = 0;
             bool ok = true;
+            int64_t ready_row0 = -1;  // FUSE: the token tile whose rows are known to be out
             Work w(a);
             Item it;
             while (ok && w.next(a, it)) {
                 Tile T;
                 if (!locate_tile(a, it.t, T)) continue;
+                if (FUSE && T.row0 != ready_row0) {
+                    const int64_t n = a.M - T.row0 < (int64_t)BN ? a.M - T.row0 : (int64_t)BN;
+                    if (!rows_ready(a.qcnt, T.row0, n, sm, a.status)) { ok = false; continue; }
+                    ready_row0 = T.row0;
+                }
                 const int send = it.kb1 + (it.z ? a.ZT : 0);
                 for (int s = it.kb0; s < send; ++s, r.next(), ++uses) {
                     const int slot = r.slot;
@@ -596,11 +928,20 @@ __global__ void __launch_bounds__(THREADS, 1) w4a8_kernel(const __grid_constant_
             // token scales of this warp's 128 columns, column 32c + l held by lane l; read
             // now, used (through shuffles) only in the epilogue
             float rsv[4];
+            if (FUSE) {
+                const float4 v = fused_row_scales(a.qcnt, a.row_scale, T.row0, T.rows, a.M, half, sm, a.status);
+                if (!__all_sync(FULL, v.x == v.x)) {  // NaN: a wait ran out or the CTA aborts
+                    ok = false;
+                    break;
+                }
+                rsv[0] = v.x; rsv[1] = v.y; rsv[2] = v.z; rsv[3] = v.w;
+            } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int col = half * 128 + c * 32 + lane;
-                const int64_t m = T.row0 + col;
-                rsv[c] = (col < T.rows && m < a.M) ? __ldg(a.row_scale + m) : 0.0f;
+                for (int c = 0; c < 4; ++c) {
+                    const int col = half * 128 + c * 32 + lane;
+                    const int64_t m = T.row0 + col;
+                    rsv[c] = (col < T.rows && m < a.M) ? __ldg(a.row_scale + m) : 0.0f;
+                }
             }
             float2 acc[64];  // columns (2i, 2i+1) of this thread's weight row
 #pragma unroll
@@ -1154,19 +1495,19 @@ static int sm_count_cached() {
 
 // Launch the kernel instantiation for group size G (first call per device sets its shared
 // memory limit).
-template <int G>
+template <int G, bool FUSE = false>
 static w4_status start(int grid, const CUtensorMap &tm_codes, const CUtensorMap &tm_act, const CUtensorMap &tm_zop,
                        const CUtensorMap &tm_gop, const Args &a, cudaStream_t stream) {
     static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        if (cudaFuncSetAttribute(w4a8_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(w4a8_kernel<G, FUSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SMEM_BYTES) != cudaSuccess)
             return W4_ERR_CUDA;
         attr_done[dev] = 1;
     }
-    w4a8_kernel<G><<<grid, THREADS, SMEM_BYTES, stream>>>(tm_codes, tm_act, tm_zop, tm_gop, a);
+    w4a8_kernel<G, FUSE><<<grid, THREADS, SMEM_BYTES, stream>>>(tm_codes, tm_act, tm_zop, tm_gop, a);
     return launch_status();
 }
 
@@ -1278,15 +1619,68 @@ static w4_status launch_f16(const uint16_t *X16, const float *row_scale, const i
     return launch_status();
 }
 
+// The workspace of the kernel variant that quantizes its own activation rows: the split-tile
+// partials and counters of the plan, one row counter per token tile (both cleared before
+// every launch by one memset), then the E4M3 rows, the row scales and the group-sum operand.
+struct FusedLayout {
+    size_t cnt, rowcnt, q8, scale, gop, end;  // byte offsets; end = total size
+};
+
+static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static FusedLayout fused_layout(const Plan &P, int64_t M, int64_t K, int64_t KZ) {
+    FusedLayout f;
+    f.cnt = (size_t)(2 * P.ps) * PART_FLOATS * sizeof(float);
+    f.rowcnt = round256(f.cnt + (size_t)(P.r * 8) * sizeof(uint32_t));
+    f.q8 = round256(f.rowcnt + (size_t)((M + BN - 1) / BN) * sizeof(uint32_t));
+    f.scale = round256(f.q8 + (size_t)M * (size_t)K);
+    f.gop = round256(f.scale + (size_t)M * sizeof(float));
+    f.end = round256(f.gop + (size_t)M * (size_t)KZ * 2);
+    return f;
+}
+
+// Row ranges quantized before the roles start: the token tiles of the first `waves` waves of
+// whole tiles, [0, a1), and those of the split tiles, [a2, M), which the CTAs holding split
+// segments take first. Warps 2-3 quantize [a1, a2) while the GEMM runs.
+static void fused_first_rows(const Plan &P, int64_t M, int64_t NT, int waves, int64_t &a1, int64_t &a2) {
+    const int64_t w = (int64_t)P.grid * waves;
+    const int64_t first_whole = P.dpt < w ? P.dpt : w;
+    a1 = first_whole > 0 ? ((first_whole - 1) / NT + 1) * BN : 0;
+    a2 = P.r > 0 ? (P.dpt / NT) * BN : M;
+    if (a2 > M) a2 = M;
+    if (a1 > a2) a1 = a2;
+}
+
+constexpr int64_t kBackgroundMaxK = 8192;
+
+struct FusedIn {
+    const uint16_t *X;  // bf16 activations [M, K]
+};
+
 static w4_status launch(const uint8_t *X8, const uint16_t *X16, const float *row_scale, const uint16_t *gop,
                         const int32_t *offsets, int E, int64_t M, const void *packed, int64_t N, int64_t K, int group,
-                        void *Y, int out_fp32, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+                        void *Y, int out_fp32, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                        const FusedIn *fz = nullptr) {
+    if (fz && (group != 64 && group != 128)) return W4_ERR_UNSUPPORTED;
     if (group == 32 || group == 256)
         return launch_f16(X16, row_scale, offsets, E, M, packed, N, K, group, Y, out_fp32, stream);
     EncodeTiledFn enc = encode_fn();
     if (!enc) return W4_ERR_CUDA;
     const GemmLayout L = gemm_layout(N, K, group);
     const uint8_t *pk = static_cast<const uint8_t *>(packed);
+    const int64_t NT = L.Npad / BM;
+    const int64_t mtu = offsets ? (M + BN - 1) / BN + E : (M + BN - 1) / BN;
+    if (mtu > 0x7fffffffLL) return W4_ERR_SHAPE;
+    const Plan P = make_plan(mtu * NT, L.Kpad / BK, sm_count_cached(), !offsets && workspace != nullptr);
+    FusedLayout FL{};
+    if (fz) {
+        FL = fused_layout(P, M, K, L.KZ);
+        if (!workspace || FL.end > workspace_bytes) return W4_ERR_WORKSPACE;
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        X8 = ws + FL.q8;
+        row_scale = reinterpret_cast<const float *>(ws + FL.scale);
+        gop = reinterpret_cast<const uint16_t *>(ws + FL.gop);
+    }
     CUtensorMap tm_codes, tm_act, tm_zop, tm_gop;
     {
         const cuuint64_t dims[3] = {(cuuint64_t)(L.Kpad / 2), (cuuint64_t)L.Npad, (cuuint64_t)E};
@@ -1329,7 +1723,7 @@ static w4_status launch(const uint8_t *X8, const uint16_t *X16, const float *row
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return W4_ERR_CUDA;
     }
-    Args a;
+    Args a{};
     a.packed = pk;
     a.slab_bytes = L.total;
     a.codes_bytes = L.codes_bytes;
@@ -1339,13 +1733,10 @@ static w4_status launch(const uint8_t *X8, const uint16_t *X16, const float *row
     a.status = device_status_ptr();
     a.M = M; a.N = N; a.Npad = L.Npad; a.K = K; a.Kpad = L.Kpad;
     a.E = E; a.g = group; a.out_fp32 = out_fp32;
-    a.NT = (int)(L.Npad / BM);
-    const int64_t mtu = offsets ? (M + BN - 1) / BN + E : (M + BN - 1) / BN;
-    if (mtu > 0x7fffffffLL) return W4_ERR_SHAPE;
+    a.NT = (int)NT;
     a.MTU = (int)mtu;
     a.KT = (int)(L.Kpad / BK);
     a.ZT = (int)(L.KZ / ZKC);
-    const Plan P = make_plan(mtu * a.NT, a.KT, sm_count_cached(), !offsets && workspace != nullptr);
     if (P.ws_bytes > workspace_bytes) return W4_ERR_WORKSPACE;
     a.DPT = P.dpt;
     a.R = P.r;
@@ -1355,6 +1746,28 @@ static w4_status launch(const uint8_t *X8, const uint16_t *X16, const float *row
                                                (size_t)(2 * P.ps) * PART_FLOATS * sizeof(float))
                 : nullptr;
     const int grid = P.grid;
+    if (fz) {
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        a.xq = fz->X;
+        a.q8 = ws + FL.q8;
+        a.qscale = reinterpret_cast<float *>(ws + FL.scale);
+        a.qgop = reinterpret_cast<uint16_t *>(ws + FL.gop);
+        a.qcnt = reinterpret_cast<uint32_t *>(ws + FL.rowcnt);
+        a.KZ = L.KZ;
+        a.qstaged = (size_t)K * 2 * 2 <= RING_BYTES ? 1 : 0;
+        // staged: the token tiles of the first two waves of whole tiles before the GEMM starts
+        // (room for the background warps to get ahead); streamed: those of the first wave
+        fused_first_rows(P, M, NT, a.qstaged ? 2 : 1, a.qa1, a.qa2);
+        // Rows of at most half the ring are staged through it before the GEMM starts: those of
+        // the token tiles the first tiles read, and the rest while the GEMM runs (by two warps
+        // per block, whose loads in flight keep up with the tiles' demand only for short rows);
+        // rows above kBackgroundMaxK all before the GEMM. Longer rows are streamed by warps.
+        if (a.qstaged && K > kBackgroundMaxK) a.qa1 = a.qa2 = M;
+        // split-tile counters and token-tile row counters start at zero on every call
+        if (cudaMemsetAsync(ws + FL.cnt, 0, FL.q8 - FL.cnt, stream) != cudaSuccess) return W4_ERR_CUDA;
+        return group == 64 ? start<64, true>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream)
+                           : start<128, true>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream);
+    }
     switch (group) {
         case 32: return start<32>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream);
         case 64: return start<64>(grid, tm_codes, tm_act, tm_zop, tm_gop, a, stream);
@@ -1461,4 +1874,49 @@ W4_API w4_status w4a8_grouped_gemm(const uint8_t *X_e4m3, const uint16_t *X_f16,
         return W4_ERR_ALIGN;
     return gemm::launch(X_e4m3, X_f16, row_scale, gsum_op, expert_row_offsets, E, M_total, packed, N, K, group, Y, 0,
                         nullptr, 0, stream);
+}
+
+// ------------------------------------------------------------------ row quant + GEMM in one launch
+
+static bool rowquant_layout(int64_t M, int64_t N, int64_t K, int group, gemm::FusedLayout &F) {
+    if (!gemm_shape_ok(M, N, K) || (group != 64 && group != 128) || K % group != 0) return false;
+    const int sms = gemm::sm_count_cached();
+    if (sms < 1) return false;
+    const GemmLayout L = gemm_layout(N, K, group);
+    const gemm::Plan P = gemm::make_plan(gemm::dense_tiles(M, N, K, group), L.Kpad / gemm::BK, sms, true);
+    F = gemm::fused_layout(P, M, K, L.KZ);
+    return true;
+}
+
+W4_API size_t w4a8_gemm_rowquant_workspace_bytes(int64_t M, int64_t N, int64_t K, int group) {
+    gemm::FusedLayout F;
+    return rowquant_layout(M, N, K, group, F) ? F.end : 0;
+}
+
+W4_API w4_status w4a8_gemm_rowquant_layout(int64_t M, int64_t N, int64_t K, int group, int64_t *out) {
+    if (!out) return W4_ERR_NULL;
+    if (!gemm_shape_ok(M, N, K)) return W4_ERR_SHAPE;
+    if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
+    gemm::FusedLayout F;
+    if (!rowquant_layout(M, N, K, group, F)) return W4_ERR_UNSUPPORTED;
+    out[0] = (int64_t)F.q8;
+    out[1] = (int64_t)F.scale;
+    out[2] = (int64_t)F.gop;
+    out[3] = (int64_t)F.end;
+    return W4_OK;
+}
+
+W4_API w4_status w4a8_gemm_rowquant(const void *X_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
+                                    int group, int mode, void *Y, int out_fp32, void *workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+    if (!X_bf16 || !packed || !Y || !workspace) return W4_ERR_NULL;
+    if (!valid_mode(mode) || (out_fp32 != 0 && out_fp32 != 1)) return W4_ERR_ARG;
+    if (!gemm_shape_ok(M, N, K)) return W4_ERR_SHAPE;
+    if (!valid_group(group) || K % group != 0) return W4_ERR_GROUP;
+    if (group != 64 && group != 128) return W4_ERR_UNSUPPORTED;
+    if (!aligned16(X_bf16) || !aligned16(packed) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return W4_ERR_ALIGN;
+    const gemm::FusedIn fz{static_cast<const uint16_t *>(X_bf16)};
+    return gemm::launch(nullptr, nullptr, nullptr, nullptr, nullptr, 1, M, packed, N, K, group, Y, out_fp32, workspace,
+                        workspace_bytes, stream, &fz);
 }

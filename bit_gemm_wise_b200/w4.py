@@ -60,6 +60,9 @@ SIGNATURES = [
     ("w4a8_gemm_workspace_bytes", _SZ, [_I64, _I64, _I64, _I]),
     ("w4a8_gemm_schedule", _I, [_I64, _I64, _I64, _I, _I, _P]),
     ("w4a8_gemm_split_segment", _I, [_I64, _I64, _I64, _I64, _I, _P]),
+    ("w4a8_gemm_rowquant_workspace_bytes", _SZ, [_I64, _I64, _I64, _I]),
+    ("w4a8_gemm_rowquant_layout", _I, [_I64, _I64, _I64, _I, _P]),
+    ("w4a8_gemm_rowquant", _I, [_P, _I64, _P, _I64, _I64, _I, _I, _P, _I, _P, _SZ, _P]),
     ("w4a8_grouped_gemm", _I, [_P, _P, _P, _P, _P, _I, _I64, _P, _I64, _I64, _I, _I, _P, _P]),
     ("w4_device_status", _I, [_P, ctypes.POINTER(ctypes.c_int)]),
     ("w4_selftest_bounded_wait", _I, [_I64, _P]),
@@ -307,6 +310,26 @@ def w4a8_gemm(X8, row_scale, gsum_op, M, packed, N, K, group, mode, Y, out_fp32=
     _check("w4a8_gemm", rc)
 
 
+def w4a8_gemm_rowquant(X, M, packed, N, K, group, mode, Y, out_fp32, workspace, stream=None):
+    """Row quant and W4A8 GEMM in one launch from bf16 activations X [M, K]; workspace:
+    alloc_gemm_rowquant_workspace(M, N, K, group) (groups 64 and 128)."""
+    rc = lib().w4a8_gemm_rowquant(_ptr(X), M, _ptr(packed), N, K, group, _mode(mode), _ptr(Y), int(out_fp32),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("w4a8_gemm_rowquant", rc)
+
+
+def w4a8_gemm_rowquant_workspace_bytes(M, N, K, group) -> int:
+    return int(lib().w4a8_gemm_rowquant_workspace_bytes(M, N, K, group))
+
+
+def w4a8_gemm_rowquant_layout(M, N, K, group) -> dict:
+    """Host-only: byte offsets of the E4M3 rows, row scales and group-sum operand that
+    w4a8_gemm_rowquant leaves in its workspace, and the workspace size."""
+    out = (ctypes.c_int64 * 4)()
+    _check("w4a8_gemm_rowquant_layout", lib().w4a8_gemm_rowquant_layout(M, N, K, group, out))
+    return dict(zip(("X_e4m3", "row_scale", "gsum_op", "bytes"), (int(v) for v in out)))
+
+
 def w4a8_gemm_workspace_bytes(M, N, K, group) -> int:
     return int(lib().w4a8_gemm_workspace_bytes(M, N, K, group))
 
@@ -378,6 +401,14 @@ def alloc_gemm_workspace(M, N, K, group, device="cuda"):
     """Zero-filled workspace for w4a8_gemm, or None when the shape is never split."""
     nbytes = w4a8_gemm_workspace_bytes(M, N, K, group)
     return torch.zeros(nbytes, dtype=torch.uint8, device=device) if nbytes else None
+
+
+def alloc_gemm_rowquant_workspace(M, N, K, group, device="cuda"):
+    """Workspace for w4a8_gemm_rowquant (uninitialised: every call clears what it needs)."""
+    nbytes = w4a8_gemm_rowquant_workspace_bytes(M, N, K, group)
+    if nbytes == 0:
+        raise W4Error("w4a8_gemm_rowquant_workspace_bytes", 6)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
 def alloc_packed(N, K, group, layout, device="cuda", copies: int = 1):

@@ -377,6 +377,48 @@ w4_status w4a8_gemm(const uint8_t *X_e4m3, const uint16_t *X_f16, const float *r
                     cudaStream_t stream);
 
 /*
+ * w4a8_gemm_rowquant -- fp8_row_quant and w4a8_gemm in ONE launch, from bf16 activations.
+ *   "Four-bit inference ... Tahoma", Achievement 2: the per-token activation scale is
+ *   recomputed on every forward pass, so its cost is paid on every call; here the GEMM's
+ *   persistent blocks quantize the rows themselves instead of a separate launch.
+ *   Computes exactly what fp8_row_quant(X, M, K, group, ...) followed by
+ *   w4a8_gemm(..., workspace) computes -- the same E4M3 codes, row scales and group-sum
+ *   operand bit for bit, then the same Y bit for bit:
+ *     Y[m, n] = s_a[m] * sum_j s[n,j] * sum_{k in group j} e4m3(X[m,k] / s_a[m]) * (q[n,k] - z[n,j]),
+ *     s_a[m] = max(max_k |X[m,k]|, 1e-8) / 448.
+ *   How: one warp quantizes one row (max over the row, scale, codes, exact integer group sums)
+ *   into the workspace and then counts it in its 256-row token tile's counter with a release
+ *   add. Before the roles of the GEMM start, every warp of the grid quantizes the rows of the
+ *   token tiles that the first tiles read; afterwards two otherwise idle warps of every block
+ *   quantize the remaining rows in order. The TMA producer waits (acquire) for a token tile's
+ *   full count before it loads that tile, and the epilogue warps before they read its row
+ *   scales. No block waits on another block's tile work, so the rows always come out; every
+ *   wait is bounded (W4_ERR_TIMEOUT in the device status).
+ *   X_bf16      device, bf16 [M, K], row-major (read only)
+ *   packed      device, w4_prepack(..., W4_LAYOUT_GEMM) of W[N, K] with this group
+ *   Y           device, bf16 [M, N] (out_fp32 == 0) or fp32 [M, N] (out_fp32 == 1)
+ *   workspace   device scratch of at least w4a8_gemm_rowquant_workspace_bytes(M, N, K, group)
+ *               bytes, 256-byte aligned, owned by the caller; no initial contents are needed
+ *               (each call clears its counters with one memset on `stream` before the
+ *               kernel). After the call it holds the E4M3 rows, row scales and group-sum
+ *               operand at the offsets w4a8_gemm_rowquant_layout reports. Calls that may
+ *               overlap on the GPU need separate workspaces.
+ *   group       64 or 128 (the promoted path); 32 and 256 return W4_ERR_UNSUPPORTED.
+ *   M >= 1; N >= 1; K >= 128, K % 32 == 0.
+ *   Errors: NULL / SHAPE / GROUP / ALIGN / ARG / UNSUPPORTED / WORKSPACE (smaller than the
+ *   query's result) / CUDA.
+ * w4a8_gemm_rowquant_layout -- host-only: out[0..3] = byte offsets inside the workspace of
+ *   the E4M3 rows [M, K], the row scales fp32 [M], the group-sum operand bf16
+ *   [M, w4a8_gsum_op_cols(K, group)], and the workspace size. Errors: NULL / SHAPE / GROUP /
+ *   UNSUPPORTED.
+ */
+size_t w4a8_gemm_rowquant_workspace_bytes(int64_t M, int64_t N, int64_t K, int group);
+w4_status w4a8_gemm_rowquant_layout(int64_t M, int64_t N, int64_t K, int group, int64_t *out);
+w4_status w4a8_gemm_rowquant(const void *X_bf16, int64_t M, const void *packed, int64_t N, int64_t K,
+                             int group, int mode, void *Y, int out_fp32, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * w4a8_gemm_schedule -- host-only query (no GPU call): how w4a8_gemm with a workspace divides
  *   the problem (M, N, K, group) over `sms` SMs (1 .. 4096). out[7] receives: tiles (128
  *   weight rows x 256 tokens each), whole tiles (the first ones, round-robin over the

@@ -166,6 +166,38 @@ def test_host_validation_rejects_before_launch(lib):
     assert rc("w4_device_status", None, None) == 1
 
 
+def test_gemm_rowquant_layout_and_validation(lib):
+    """The one-launch row quant + GEMM: workspace regions 256-byte aligned, in order, sized
+    for M x K codes, M scales and the group-sum operand; host checks before any launch."""
+    for M, N, K, g in [(4096, 15360, 3840, 128), (4096, 3840, 15360, 128), (7, 77, 192, 64), (1, 128, 128, 128)]:
+        lay = w4.w4a8_gemm_rowquant_layout(M, N, K, g)
+        cols = w4.w4a8_gsum_op_cols(K, g)
+        assert all(lay[k] % 256 == 0 for k in lay)
+        assert lay["X_e4m3"] + M * K <= lay["row_scale"]
+        assert lay["row_scale"] + 4 * M <= lay["gsum_op"]
+        assert lay["gsum_op"] + 2 * M * cols <= lay["bytes"]
+        assert lay["bytes"] == w4.w4a8_gemm_rowquant_workspace_bytes(M, N, K, g)
+        # the split tiles' partials and counters come first, then one row counter per token tile
+        sched = w4.w4a8_gemm_schedule(M, N, K, g, 148)
+        assert lay["X_e4m3"] >= sched["workspace_bytes"] + 4 * ((M + 255) // 256)
+    # groups of 32 and 256 (the split-weight path) are not offered
+    assert lib.w4a8_gemm_rowquant_workspace_bytes(4096, 4096, 4096, 32) == 0
+    assert lib.w4a8_gemm_rowquant_workspace_bytes(4096, 4096, 4096, 256) == 0
+    ws = w4.w4a8_gemm_rowquant_workspace_bytes(64, 256, 512, 128)
+    assert rc("w4a8_gemm_rowquant", None, 64, FAKE, 256, 512, 128, 1, FAKE, 0, FAKE, ws, None) == 1
+    assert rc("w4a8_gemm_rowquant", FAKE, 64, FAKE, 256, 512, 128, 1, FAKE, 0, None, ws, None) == 1
+    assert rc("w4a8_gemm_rowquant", FAKE, 0, FAKE, 256, 512, 128, 1, FAKE, 0, FAKE, ws, None) == 2
+    assert rc("w4a8_gemm_rowquant", FAKE, 64, FAKE, 256, 96, 32, 1, FAKE, 0, FAKE, ws, None) == 2
+    assert rc("w4a8_gemm_rowquant", FAKE, 64, FAKE, 256, 512, 48, 1, FAKE, 0, FAKE, ws, None) == 3
+    assert rc("w4a8_gemm_rowquant", FAKE, 64, FAKE, 256, 512, 32, 1, FAKE, 0, FAKE, ws, None) == 6
+    assert rc("w4a8_gemm_rowquant", FAKE, 64, FAKE, 256, 512, 128, 3, FAKE, 0, FAKE, ws, None) == 5
+    assert rc("w4a8_gemm_rowquant", FAKE, 64, FAKE, 256, 512, 128, 1, FAKE, 2, FAKE, ws, None) == 5
+    assert rc("w4a8_gemm_rowquant", FAKE + 8, 64, FAKE, 256, 512, 128, 1, FAKE, 0, FAKE, ws, None) == 4
+    assert rc("w4a8_gemm_rowquant", FAKE, 64, FAKE, 256, 512, 128, 1, FAKE, 0, FAKE + 16, ws, None) == 4
+    with pytest.raises(w4.W4Error):
+        w4.w4a8_gemm_rowquant_layout(64, 256, 512, 32)
+
+
 # ------------------------------------------------------------------ W4A8 GEMM work split
 
 def test_gemm_schedule_of_the_prefill_shapes(lib):
