@@ -34,7 +34,11 @@
 //    on the ring sees its phases in order, and the MMA thread has one wait and one commit
 //    per stage (plus one of each per accumulator group);
 //  * every mbarrier wait is bounded by wall-clock time; on expiry the kernel records
-//    W4_ERR_TIMEOUT, every role sees the abort flag, TMEM is freed and the CTA returns.
+//    W4_ERR_TIMEOUT, every role sees the abort flag, TMEM is freed and the CTA returns;
+//  * w4a8_gemm_rowquant runs the same kernel from bf16 activations (FUSE): its blocks
+//    quantize the rows into the workspace first (staged through the ring) and, for short
+//    rows, partly while the tiles run (warps 2-3); the producer and the epilogue read a
+//    token tile's rows only after its row count is complete.
 #include "w4_common.cuh"
 #include "w4_layout.cuh"
 #include "w4_rowquant.cuh"
@@ -471,10 +475,12 @@ __device__ __noinline__ bool split_combine(float *part_base, uint32_t *cnt, int 
 // ("Four-bit inference ... Tahoma", Achievement 2: the per-token scale is recomputed on every
 // forward pass) into the workspace -- E4M3 codes, row scale, group-sum operand, the same
 // values as fp8_row_quant bit for bit -- and the tiles then read those rows like the
-// operands of the two-launch path. One warp quantizes one row: the max over the row's
-// magnitude bits, the row scale and its reciprocal, then a second pass over the row (from
-// L2) that converts, stores the codes and adds each group's codes exactly as integers in
-// units of 2^-9. A finished row is counted in its token tile's counter by a release add
+// operands of the two-launch path. Rows are either staged through the still-empty ring by
+// bulk copies (quant_rows_staged, before the GEMM's roles start) or streamed by one warp per
+// row (quant_row_warp: the max over the row's magnitude bits, the row scale and its
+// reciprocal, then a second pass over the row from L2 that converts, stores the codes and
+// adds each group's codes exactly as integers in units of 2^-9; used while the GEMM runs and
+// for rows too long for the ring). A finished row is counted in its token tile's counter by a release add
 // after a proxy fence, so that the TMA (async proxy) loads issued after an acquire load of a
 // full count see it. The readers use acquire loads, not fences: a gpu-scope fence would wait
 // for the reader's own earlier stores (the previous tile's outputs) to drain.
