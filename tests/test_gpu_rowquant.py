@@ -116,12 +116,13 @@ def rows_below_max(amax_bits, K):
     return rows
 
 
-@pytest.mark.parametrize("K", [16384, 32768])
+@pytest.mark.parametrize("K", [4096, 16384, 32768])
 def test_every_value_under_many_row_maxima(K):
     """The kernel divides by the row scale through the row's reciprocal and one exact
     correction step; the codes must equal those of the oracle's IEEE division for every
-    bf16 value under row maxima spread over the whole exponent range (K = 16384 takes the
-    register-resident kernel, K = 32768 the three-pass one)."""
+    bf16 value under row maxima spread over the whole exponent range (K = 4096 takes the
+    register-resident warp kernel, K = 16384 the register-resident block kernel, K = 32768
+    the three-pass one)."""
     maxima = [0x0001, 0x0080, 0x0A3C, 0x2F11, 0x3300, 0x3C00, 0x3F80, 0x3FFF, 0x4120, 0x43E0,
               0x447F, 0x4B01, 0x5F7F, 0x7A00, 0x7F7F]
     rows = []
@@ -131,11 +132,12 @@ def test_every_value_under_many_row_maxima(K):
     check(X, 128)
 
 
-def test_rows_with_infinities():
+@pytest.mark.parametrize("K", [512, 3840])
+def test_rows_with_infinities(K):
     """A row whose maximum is infinite has an infinite scale: finite values give zero codes
     through the division fallback (the infinite entries themselves are NaN codes and are not
-    compared, since the sign of a NaN quotient is not fixed)."""
-    K = 512
+    compared, since the sign of a NaN quotient is not fixed). K = 512 and 3840 take the
+    warp-per-row kernel with 4 and 16 chunks per lane."""
     row = np.linspace(-3, 3, K).astype(np.float32)
     row[7] = np.inf
     row2 = row.copy()
