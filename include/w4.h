@@ -272,9 +272,11 @@ w4_status w4a16_gemv_grouped_schedule(int count, int64_t M, const int64_t *N, co
  *     before any stream capture on that device.
  *   - Each call clears the arrival counters it needs (cudaMemsetAsync on `stream`) before its
  *     kernel, because the array keeps the previous call's contents.
- *   - All calls share the one array: calls that may overlap on the GPU (different streams,
- *     or W4_OVERLAP_PREVIOUS after another noalloc call still running) race on it and give
- *     wrong results. Serialise them, or use w4a16_gemv with separate workspaces.
+ *   - All calls share the one array: calls on different streams that may run at the same
+ *     time race on it and give wrong results. Serialise them, or use w4a16_gemv with
+ *     separate workspaces. On one stream, a call that uses the array starts with its memset,
+ *     which waits for the stream's previous kernel, so W4_OVERLAP_PREVIOUS never overlaps
+ *     such a call with the call before it.
  *   - Only rows split along K (K beyond about 40,000 at M = 1) use the scratch: such a call
  *     needs K_parts * M * N * 4 bytes of partial sums plus 4 bytes per row block and sweep,
  *     the workspace_bytes that w4a16_gemv_schedule reports. A request above the limit returns
