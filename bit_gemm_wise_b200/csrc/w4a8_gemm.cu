@@ -1657,7 +1657,7 @@ static void fused_first_rows(const Plan &P, int64_t M, int64_t NT, int waves, in
     if (a1 > a2) a1 = a2;
 }
 
-constexpr int64_t kBackgroundMaxK = 8192;
+constexpr int64_t kBackgroundMaxK = 16384;
 
 struct FusedIn {
     const uint16_t *X;  // bf16 activations [M, K]
@@ -1765,9 +1765,10 @@ static w4_status launch(const uint8_t *X8, const uint16_t *X16, const float *row
         // (room for the background warps to get ahead); streamed: those of the first wave
         fused_first_rows(P, M, NT, a.qstaged ? 2 : 1, a.qa1, a.qa2);
         // Rows of at most half the ring are staged through it before the GEMM starts: those of
-        // the token tiles the first tiles read, and the rest while the GEMM runs (by two warps
-        // per block, whose loads in flight keep up with the tiles' demand only for short rows);
-        // rows above kBackgroundMaxK all before the GEMM. Longer rows are streamed by warps.
+        // the token tiles the first two waves and the split tiles read; the rest are quantized
+        // while the GEMM runs, by two warps per block, whose loads in flight keep up with the
+        // third wave's demand up to rows of kBackgroundMaxK elements; longer staged rows all go
+        // before the GEMM. Rows too long for the ring are streamed by warps.
         if (a.qstaged && K > kBackgroundMaxK) a.qa1 = a.qa2 = M;
         // split-tile counters and token-tile row counters start at zero on every call
         if (cudaMemsetAsync(ws + FL.cnt, 0, FL.q8 - FL.cnt, stream) != cudaSuccess) return W4_ERR_CUDA;
