@@ -77,11 +77,9 @@ struct Smem {
     int abort;
     // the row quant of the kernel variant that quantizes its own activation rows, before the
     // ring is in use: two halves of row slots in the ring, each completed by one barrier, and
-    // the scale, its reciprocal and the special-row mark of each row of the current batch
+    // the row maxima (magnitude bits, by atomicMax) of the batches of each parity
     uint64_t rq_full[2];
-    float rq_s[16], rq_r[16];
-    uint32_t rq_sp[16];
-    uint32_t rq_mb[16];  // the batch's row maxima (magnitude bits), combined by atomicMax
+    uint32_t rq_mb[2][16];
 };
 static_assert(sizeof(Smem) <= 1024, "control block");
 constexpr uint32_t RING_BYTES = STAGES * (RAW_BYTES + A_BYTES);  // ring data bytes (row slots before the GEMM)
@@ -587,14 +585,17 @@ __device__ __forceinline__ void quant_row_warp(const uint16_t *__restrict__ xq, 
 // through the (still unused) ring: the CTA's rows (index i = blockIdx.x + k * gridDim.x of that
 // row set) go by batches of h rows into one half of the ring's row slots by bulk copies, while
 // the other half's batch is worked on, so HBM streams the rows at full rate instead of one
-// warp's loads in flight at a time.
-// Per batch: all 16 warps take the rows' maxima by rounds of 32 chunks (combined per row in
-// shared memory), one warp per row forms the row's scale; then all 16 warps convert the batch
-// by rounds of 32 chunks (a round holds whole groups, whose sums are warp butterflies) and
-// store codes and group-sum operand; at the batch's end every thread
-// fences its stores for the async proxy, and after the block barrier one gpu-scope fence
-// (cumulative over the block's stores) precedes the release adds that count each row in its
-// token tile. Returns false (every thread alike) if a bulk copy did not land in time.
+// warp's loads in flight at a time. Two block barriers per batch:
+//  1. after the batch's rows landed -- it also ends the previous batch: that batch's rows are
+//     counted in their token tiles (one gpu-scope fence, cumulative over the block's stores,
+//     then release adds), its half of the slots is refilled with the next batch, and the row
+//     maxima of the next parity are cleared;
+//  2. after all 16 warps took the rows' maxima by rounds of 32 chunks (combined per row in
+//     shared memory).
+// Then every warp forms each row's scale from its maximum and converts rounds of 32 chunks
+// (a round holds whole groups, whose sums are warp butterflies), storing codes and group-sum
+// operand, and fences its stores for the async proxy. Returns false (every thread alike) if a
+// bulk copy did not land in time.
 template <int G>
 __device__ __forceinline__ bool quant_rows_staged(const Args &a, uint8_t *ring, Smem *sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -624,22 +625,39 @@ __device__ __forceinline__ bool quant_rows_staged(const Args &a, uint8_t *ring, 
         mbar_init(&sm->rq_full[1], 1);
         fence_mbar_init();
     }
-    if (threadIdx.x < 16) sm->rq_mb[threadIdx.x] = 0u;
+    if (threadIdx.x < 32) sm->rq_mb[threadIdx.x >> 4][threadIdx.x & 15] = 0u;
     __syncthreads();
     if (threadIdx.x == 0) {
         if (nb > 0) issue(0);
         if (nb > 1) issue(1);
     }
     bool ok = true;
-    for (int64_t b = 0; b < nb; ++b) {
-        const int half = (int)(b & 1), n = batch_rows(b);
-        const uint8_t *slots = ring + (size_t)half * h * row_bytes;
+    for (int64_t b = 0; b <= nb; ++b) {  // the pass with b == nb only ends batch nb - 1
+        const int half = (int)(b & 1);
         bool got = true;
-        if (lane == 0) got = wait_phase(&sm->rq_full[half], (uint32_t)(b >> 1) & 1u, sm, a.status);
-        got = __shfl_sync(FULL, got ? 1 : 0, 0) != 0;
-        if (got) got = __all_sync(FULL, mbar_try_wait_short(&sm->rq_full[half], (uint32_t)(b >> 1) & 1u));
-        ok = __syncthreads_and(got ? 1 : 0) != 0;
+        if (b < nb) {
+            if (lane == 0) got = wait_phase(&sm->rq_full[half], (uint32_t)(b >> 1) & 1u, sm, a.status);
+            got = __shfl_sync(FULL, got ? 1 : 0, 0) != 0;
+            if (got) got = __all_sync(FULL, mbar_try_wait_short(&sm->rq_full[half], (uint32_t)(b >> 1) & 1u));
+        }
+        ok = __syncthreads_and(got ? 1 : 0) != 0;  // barrier 1
         if (!ok) break;
+        if (b > 0) {
+            // batch b - 1 is done by every warp: count its rows, refill its half
+            const int np = batch_rows(b - 1);
+            if (warp == 0) {
+                if (lane == 0) __threadfence();
+                __syncwarp();
+                if (lane < np) red_release_add(a.qcnt + row_of((b - 1) * h + lane) / BN, 1u);
+            }
+            if (threadIdx.x == 0 && b + 1 < nb) issue(b + 1);
+        }
+        if (b == nb) break;
+        // the maxima of the next batch (last read by batch b - 1, before barrier 1)
+        if (threadIdx.x < 16) sm->rq_mb[half ^ 1][threadIdx.x] = 0u;
+        const int n = batch_rows(b);
+        const uint8_t *slots = ring + (size_t)half * h * row_bytes;
+        uint32_t *mbs = sm->rq_mb[half];
         // max over each row's magnitude bits: each row's rounds of 32 chunks spread over the 16
         // warps (row outer, round inner: warp-uniform trip counts, no division)
         for (int i = 0; i < n; ++i) {
@@ -648,43 +666,29 @@ __device__ __forceinline__ bool quant_rows_staged(const Args &a, uint8_t *ring, 
             for (int64_t c0 = (int64_t)warp * 32; c0 < nchunk; c0 += THREADS)
                 if (c0 + lane < nchunk) mb = absmax_bits(mb, src[c0 + lane]);
             mb = __reduce_max_sync(FULL, __vmaxu2(mb, mb >> 16) & 0xFFFFu);
-            if (lane == 0 && mb) atomicMax(&sm->rq_mb[i], mb);
+            if (lane == 0 && mb) atomicMax(&mbs[i], mb);
         }
-        __syncthreads();
-        // scale of row i (warp i), the NaN rows' max over the other values, the group-sum
-        // operand's zero padding
-        if (warp < n) {
-            const int64_t m = row_of(b * h + warp);
-            const uint32_t mb = sm->rq_mb[warp];
+        __syncthreads();  // barrier 2
+        // scale, codes and group sums: each warp forms every row's scale from its maximum,
+        // then converts its share of the row's rounds (a round holds whole groups)
+        for (int i = 0; i < n; ++i) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(slots + (size_t)i * row_bytes);
+            const int64_t m = row_of(b * h + i);
+            const uint32_t mb = mbs[i];
             float amax = __uint_as_float(mb << 16);
             if (mb > 0x7F80u) {  // NaN: the maximum of the other values
-                const uint4 *src = reinterpret_cast<const uint4 *>(slots + (size_t)warp * row_bytes);
                 float x = 0.0f;
                 for (int64_t c = lane; c < nchunk; c += 32) x = absmax_float(x, src[c]);
                 amax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(x)));
             }
-            const float sc = scale_of(amax);
-            __syncwarp();  // every lane has read rq_mb[warp] before lane 0 clears it
-            if (lane == 0) {
-                a.qscale[m] = sc;
-                sm->rq_s[warp] = sc;
-                sm->rq_r[warp] = __frcp_rn(sc);
-                sm->rq_sp[warp] = mb >= 0x7F80u ? 1u : 0u;  // an infinity or a NaN in the row
-                sm->rq_mb[warp] = 0u;                        // for the next batch
+            const float sc = scale_of(amax), rc = __frcp_rn(sc);
+            const bool sp = mb >= 0x7F80u;  // an infinity or a NaN in the row
+            uint16_t *gop = a.qgop + m * a.KZ;
+            if (warp == (i & 15)) {  // the row's scale and the group-sum operand's zero padding
+                if (lane == 0) a.qscale[m] = sc;
+                for (int64_t t = 3 * J + lane; t < a.KZ; t += 32) gop[t] = 0;
             }
-            uint16_t *gop = a.qgop + m * a.KZ;
-            for (int64_t t = 3 * J + lane; t < a.KZ; t += 32) gop[t] = 0;
-        }
-        __syncthreads();
-        // codes and group sums: each row's rounds of 32 chunks spread over the 16 warps (a round
-        // holds whole groups)
-        for (int i = 0; i < n; ++i) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(slots + (size_t)i * row_bytes);
-            const int64_t m = row_of(b * h + i);
-            const float sc = sm->rq_s[i], rc = sm->rq_r[i];
-            const bool sp = sm->rq_sp[i] != 0u;
             uint2 *dst = reinterpret_cast<uint2 *>(a.q8 + m * K);
-            uint16_t *gop = a.qgop + m * a.KZ;
             for (int64_t c0 = (int64_t)warp * 32; c0 < nchunk; c0 += THREADS) {
                 const int64_t c = c0 + lane;
                 const bool live = c < nchunk;
@@ -706,17 +710,10 @@ __device__ __forceinline__ bool quant_rows_staged(const Args &a, uint8_t *ring, 
                 }
             }
         }
-        // the batch's stores visible to the gpu and to the async proxy; this CTA's reads of the
-        // slots ordered before the bulk copies (async proxy) that refill them
+        // the batch's stores visible to the async proxy; this thread's reads of the slots
+        // ordered before the bulk copies (async proxy) that refill them after barrier 1
         asm volatile("fence.proxy.async.global;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
-        if (warp == 0) {
-            if (lane == 0) __threadfence();
-            __syncwarp();
-            if (lane < n) red_release_add(a.qcnt + row_of(b * h + lane) / BN, 1u);
-        }
-        if (threadIdx.x == 0 && b + 2 < nb) issue(b + 2);
     }
     return ok;
 }
