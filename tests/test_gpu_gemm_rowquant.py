@@ -173,3 +173,42 @@ def test_prefill_full_size(K, N):
     assert np.array_equal(np_of(asa)[rows].view(np.uint32), np.asarray(s_ao, np.float32).view(np.uint32))
     assert np.array_equal(np_of(agop)[rows].view(np.uint16), gsum_operand(Go, K, group))
     assert w4.w4_device_status() == 0
+
+
+def packed_weight_gpu(N, K, group, seed):
+    """A prepacked weight quantized on the GPU (its quantizer is bit-exact against the oracle
+    in the quantizer tests); the comparison below is between two paths on the same weight."""
+    dev = cuda()
+    W = synth.normal((N, K), 0.02, seed, 960).to(dev)
+    codes, scales, zeros, _ = w4.alloc_quantized(N, K, group, "asym", device=dev, chosen=False)
+    w4.w4_quantize(W, N, K, group, "asym", [1.0], codes, scales, zeros, None)
+    p = w4.alloc_packed(N, K, group, w4.W4_LAYOUT_GEMM, device=dev)
+    w4.w4_prepack(codes, scales, zeros, N, K, group, "asym", w4.W4_LAYOUT_GEMM, p)
+    return p
+
+
+@pytest.mark.parametrize("M,N,K", [(2048, 8192, 1024), (2048, 6144, 65536)])
+def test_rows_quantized_while_the_gemm_runs(M, N, K):
+    """Shapes with more waves of tiles than the rows quantized before the GEMM starts cover:
+    the rest of the rows come from two warps per block while the tiles run. At K = 1024 the
+    first rows are staged through the shared-memory ring (2048 x 8192: 512 whole tiles, rows
+    from 1280 on in the background); at K = 65536 they are streamed by warps and the last wave
+    is split along K (2048 x 6144: 384 tiles, rows 1024 to 1535 in the background). Y, codes,
+    scales and group-sum operand equal the two-launch path's bit for bit; sampled rows of the
+    workspace equal the oracle's row quant."""
+    group = 128
+    packed = packed_weight_gpu(N, K, group, 6)
+    X = synth.outlier_activation(M, K, 8, 20.0, 6, 940)
+    Xd = X.to(cuda())
+    ws = w4.alloc_gemm_rowquant_workspace(M, N, K, group, device=cuda())
+    Yr, X8, sa, gop = two_launch(Xd, M, packed, N, K, group, "asym", 0)
+    Y = one_launch(Xd, M, packed, N, K, group, "asym", 0, ws)
+    assert torch.equal(Y, Yr)
+    check_same_rows(ws, M, N, K, group, X8, sa, gop)
+    rows = np.unique(np.r_[0, 255, 256, np.linspace(0, M - 1, 12).astype(int), M - 1])
+    X8o, s_ao, Go = oracle.row_quant(synth.bf16_bits(X[torch.from_numpy(rows)]), group)
+    a8, asa, agop = workspace_rows(ws, M, N, K, group)
+    assert np.array_equal(np_of(a8)[rows], X8o)
+    assert np.array_equal(np_of(asa)[rows].view(np.uint32), np.asarray(s_ao, np.float32).view(np.uint32))
+    assert np.array_equal(np_of(agop)[rows].view(np.uint16), gsum_operand(Go, K, group))
+    assert w4.w4_device_status() == 0
